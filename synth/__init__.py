@@ -1,0 +1,232 @@
+"""Seeded synthetic inputs for the DeepSeek Sparse Attention (DSA) hot path.
+
+This module only draws and encodes inputs (random numbers, FP8/BF16 encoding,
+packing of decode caches). It holds none of the method's arithmetic, and it is
+the only code shared by the CUDA path's tests/bench and the CPU oracle.
+
+Workload recipes (DeepSeek-V3.2 breakdown page, section 2 "Architecture: DSA";
+the research summary page, "Key points": 2048 selected tokens, few FP8 indexer
+heads, MLA in MQA mode, 128K context):
+
+* ``tiny``        L=256, H_I=4, d_I=32, k=32, Hq=4, d_qk=80 (64 latent + 16
+                  rope), d_v=64. Indexer q/k integers uniform in [-4, 4] (exact
+                  in e4m3), w integers in [-2, 2]; main q/kv ~ N(0,1) -> bf16;
+                  scale 1/sqrt(80).
+* ``prefill4k``   L=4096, H_I=8, d_I=128, k=2048, Hq=128, d_qk=576 (512 + 64),
+                  d_v=512. Indexer q/k = e4m3(clip(N(0,1), +-448)),
+                  w ~ N(0,1)/sqrt(8); q/kv ~ N(0,1) -> bf16; scale 1/sqrt(576).
+* ``prefill32k``  as prefill4k with L=32768.
+* ``prefill32k_int`` as prefill32k with integer indexer inputs (as ``tiny``).
+* ``prefill128k`` as prefill4k with L=131072.
+* ``decode``      64 sequences, one query each, context lengths uniform in
+                  [8192, 131072]; packed FP8 key cache (d_I=128) and bf16
+                  latent cache (576); H_I=8, Hq=128, k=2048, d_v=512.
+
+Every tensor has its own seed, derived from (base seed, config, tensor name,
+chunk), so a tensor can be regenerated independently of the others and of the
+chunking used on the device.
+"""
+from __future__ import annotations
+
+import math
+import zlib
+from dataclasses import dataclass, field
+from typing import Optional
+
+import torch
+
+E4M3_MAX = 448.0
+
+CONFIGS = {
+    "tiny": dict(kind="prefill", L=256, H_I=4, d_I=32, k=32, Hq=4, d_qk=80, d_v=64,
+                 indexer="int"),
+    "prefill4k": dict(kind="prefill", L=4096, H_I=8, d_I=128, k=2048, Hq=128, d_qk=576,
+                      d_v=512, indexer="normal"),
+    "prefill32k": dict(kind="prefill", L=32768, H_I=8, d_I=128, k=2048, Hq=128, d_qk=576,
+                       d_v=512, indexer="normal"),
+    "prefill32k_int": dict(kind="prefill", L=32768, H_I=8, d_I=128, k=2048, Hq=128,
+                           d_qk=576, d_v=512, indexer="int"),
+    "prefill128k": dict(kind="prefill", L=131072, H_I=8, d_I=128, k=2048, Hq=128,
+                        d_qk=576, d_v=512, indexer="normal"),
+    "decode": dict(kind="decode", B=64, ctx_lo=8192, ctx_hi=131072, H_I=8, d_I=128, k=2048,
+                   Hq=128, d_qk=576, d_v=512, indexer="normal"),
+}
+
+# rows of a large tensor drawn per seed; keeps device temporaries bounded
+_CHUNK_ELEMS = 1 << 27
+
+
+def tensor_seed(base: int, config: str, name: str, chunk: int = 0) -> int:
+    return zlib.crc32(f"{base}:{config}:{name}:{chunk}".encode()) & 0x7FFFFFFF
+
+
+def _gen(device, seed: int) -> torch.Generator:
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    return g
+
+
+def _rows_per_chunk(row_elems: int) -> int:
+    return max(1, _CHUNK_ELEMS // max(1, row_elems))
+
+
+def normal(shape, base, config, name, device, dtype=torch.float32, scale=1.0):
+    """N(0, scale^2) samples, drawn in fp32 chunk by chunk along dim 0, cast to dtype."""
+    shape = tuple(int(s) for s in shape)
+    out = torch.empty(shape, dtype=dtype, device=device)
+    if out.numel() == 0:
+        return out
+    row = int(math.prod(shape[1:])) if len(shape) > 1 else 1
+    step = _rows_per_chunk(row)
+    for c, r0 in enumerate(range(0, shape[0], step)):
+        r1 = min(shape[0], r0 + step)
+        g = _gen(device, tensor_seed(base, config, name, c))
+        x = torch.randn((r1 - r0,) + shape[1:], generator=g, device=device, dtype=torch.float32)
+        if scale != 1.0:
+            x.mul_(scale)
+        out[r0:r1] = x.to(dtype)
+    return out
+
+
+def integers(shape, lo, hi, base, config, name, device):
+    """Integers uniform in [lo, hi] (inclusive), returned as fp32."""
+    shape = tuple(int(s) for s in shape)
+    out = torch.empty(shape, dtype=torch.float32, device=device)
+    if out.numel() == 0:
+        return out
+    row = int(math.prod(shape[1:])) if len(shape) > 1 else 1
+    step = _rows_per_chunk(row)
+    for c, r0 in enumerate(range(0, shape[0], step)):
+        r1 = min(shape[0], r0 + step)
+        g = _gen(device, tensor_seed(base, config, name, c))
+        out[r0:r1] = torch.randint(lo, hi + 1, (r1 - r0,) + shape[1:], generator=g,
+                                   device=device, dtype=torch.int32).float()
+    return out
+
+
+def to_e4m3_bytes(x: torch.Tensor) -> torch.Tensor:
+    """Encode fp32 as OCP FP8 E4M3 (round to nearest even, saturated to +-448) -> uint8."""
+    return x.clamp(-E4M3_MAX, E4M3_MAX).to(torch.float8_e4m3fn).view(torch.uint8)
+
+
+@dataclass
+class DSAInputs:
+    """One batch of DSA inputs. FP8 tensors hold raw e4m3 bytes (uint8)."""
+    config: str
+    q_idx: torch.Tensor      # uint8 (e4m3) [T, H_I, d_I]
+    w: torch.Tensor          # fp32 [T, H_I]
+    k_idx: torch.Tensor      # uint8 (e4m3) [S, d_I]
+    q: torch.Tensor          # bf16 [T, Hq, d_qk]
+    kv: torch.Tensor         # bf16 [S, d_qk]
+    pos: Optional[torch.Tensor]     # int32 [T] or None (suffix-aligned causal)
+    k_base: Optional[torch.Tensor]  # int32 [T] or None (single sequence)
+    k: int
+    scale: float
+    d_v: int
+    meta: dict = field(default_factory=dict)
+
+    @property
+    def T(self):
+        return self.q_idx.shape[0]
+
+    @property
+    def S(self):
+        return self.k_idx.shape[0]
+
+    def positions(self) -> torch.Tensor:
+        """Explicit pos[t] (last visible key of row t, relative to k_base[t])."""
+        if self.pos is not None:
+            return self.pos
+        return torch.arange(self.T, dtype=torch.int32, device=self.q_idx.device) + (self.S - self.T)
+
+    def bases(self) -> torch.Tensor:
+        if self.k_base is not None:
+            return self.k_base
+        return torch.zeros(self.T, dtype=torch.int32, device=self.q_idx.device)
+
+    def to(self, device) -> "DSAInputs":
+        mv = lambda t: None if t is None else t.to(device)
+        return DSAInputs(self.config, mv(self.q_idx), mv(self.w), mv(self.k_idx), mv(self.q),
+                         mv(self.kv), mv(self.pos), mv(self.k_base), self.k, self.scale,
+                         self.d_v, dict(self.meta))
+
+
+def _indexer_tensors(cfg, name, T, S, base, device, with_main=True):
+    H_I, d_I = cfg["H_I"], cfg["d_I"]
+    if cfg["indexer"] == "int":
+        q_idx = to_e4m3_bytes(integers((T, H_I, d_I), -4, 4, base, name, "q_idx", device))
+        k_idx = to_e4m3_bytes(integers((S, d_I), -4, 4, base, name, "k_idx", device))
+        w = integers((T, H_I), -2, 2, base, name, "w", device)
+    else:
+        q_idx = to_e4m3_bytes(normal((T, H_I, d_I), base, name, "q_idx", device))
+        k_idx = to_e4m3_bytes(normal((S, d_I), base, name, "k_idx", device))
+        w = normal((T, H_I), base, name, "w", device, scale=1.0 / math.sqrt(H_I))
+    return q_idx, w, k_idx
+
+
+def prefill_inputs(name: str = "prefill4k", device="cpu", seed: int = 0, L: int = None,
+                   overrides: dict = None) -> DSAInputs:
+    """One causal prefill sequence: T = S = L, pos[t] = t, k_base = 0."""
+    cfg = dict(CONFIGS[name])
+    if overrides:
+        cfg.update(overrides)
+    if L is not None:
+        cfg["L"] = L
+    L = cfg["L"]
+    q_idx, w, k_idx = _indexer_tensors(cfg, name, L, L, seed, device)
+    q = normal((L, cfg["Hq"], cfg["d_qk"]), seed, name, "q", device, dtype=torch.bfloat16)
+    kv = normal((L, cfg["d_qk"]), seed, name, "kv", device, dtype=torch.bfloat16)
+    return DSAInputs(name, q_idx, w, k_idx, q, kv, None, None, cfg["k"],
+                     1.0 / math.sqrt(cfg["d_qk"]), cfg["d_v"], meta=cfg)
+
+
+def decode_inputs(name: str = "decode", device="cpu", seed: int = 0, B: int = None,
+                  ctx: list = None, overrides: dict = None) -> DSAInputs:
+    """B sequences with one query each, keys packed per sequence in one cache.
+
+    Sequence b owns cache rows [k_base[b], k_base[b] + ctx[b]); its query sees
+    all of them: pos[b] = ctx[b] - 1.
+    """
+    cfg = dict(CONFIGS[name])
+    if overrides:
+        cfg.update(overrides)
+    if B is not None:
+        cfg["B"] = B
+    B = cfg["B"]
+    if ctx is None:
+        g = _gen("cpu", tensor_seed(seed, name, "ctx"))
+        ctx = torch.randint(cfg["ctx_lo"], cfg["ctx_hi"] + 1, (B,), generator=g).tolist()
+    ctx = [int(c) for c in ctx]
+    base = [0]
+    for c in ctx[:-1]:
+        base.append(base[-1] + c)
+    S = sum(ctx)
+    q_idx, w, k_idx = _indexer_tensors(cfg, name, B, S, seed, device)
+    q = normal((B, cfg["Hq"], cfg["d_qk"]), seed, name, "q", device, dtype=torch.bfloat16)
+    kv = normal((S, cfg["d_qk"]), seed, name, "kv", device, dtype=torch.bfloat16)
+    pos = torch.tensor([c - 1 for c in ctx], dtype=torch.int32, device=device)
+    k_base = torch.tensor(base, dtype=torch.int32, device=device)
+    meta = dict(cfg)
+    meta["ctx"] = ctx
+    return DSAInputs(name, q_idx, w, k_idx, q, kv, pos, k_base, cfg["k"],
+                     1.0 / math.sqrt(cfg["d_qk"]), cfg["d_v"], meta=meta)
+
+
+def make_inputs(name: str, device="cpu", seed: int = 0, **kw) -> DSAInputs:
+    if CONFIGS[name]["kind"] == "decode":
+        return decode_inputs(name, device, seed, **kw)
+    return prefill_inputs(name, device, seed, **kw)
+
+
+def sample_rows(T: int, k: int, n: int, seed: int = 0) -> list:
+    """Query rows checked at large L: 0, k-1, k, T-1 plus a seeded random set."""
+    fixed = [r for r in (0, k - 1, k, T - 1) if 0 <= r < T]
+    g = _gen("cpu", tensor_seed(seed, "rows", str(T)))
+    rest = torch.randperm(T, generator=g)[: max(0, n)].tolist()
+    out = []
+    for r in fixed + rest:
+        if r not in out:
+            out.append(r)
+        if len(out) >= max(n, len(fixed)):
+            break
+    return sorted(out)
