@@ -1,0 +1,449 @@
+"""Benchmark of the DSA hot path on B200: one JSON line on stdout (rank 0).
+
+A step is one pass of the whole hot path over one batch of synthetic inputs:
+the 128K-token causal prefill (lightning indexer + Top-k selector + sparse MQA
+attention over 2048 selected latent rows per token) followed by one decode
+step of 64 sequences (contexts uniform in [8K, 128K]). `value` is prefill
+tokens/s over the whole job (all ranks); decode seqs/s is reported beside it.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU (torchrun): every rank runs the same independent workload (weak
+scaling, no collective on the data path); the step time is the max over ranks.
+Inputs (19 GB of queries) are far larger than L2, so no flush is needed
+between steps. `--impl reference` times the CPU oracle on bounded samples of
+the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "DSA prefill tokens/s & decode seqs/s at 128K ctx; % of FP8/BF16 TC / HBM roofline"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--prefill", default="prefill128k")
+    ap.add_argument("--decode", default="decode")
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--seed", type=int, default=0)
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------- distributed
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(world, x: float) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, local_rank):
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+        ids = [v for v in vis.split(",") if v.strip()]
+        self.index = ids[local_rank] if local_rank < len(ids) else str(local_rank)
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.index, f"--query-gpu={self.FIELDS}", "--format=csv",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.3)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9 or not parts[1].split()[0].isdigit():
+                    continue
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [int(r[1].split()[0]) for r in rows]
+        mx = max(int(r[2].split()[0]) for r in rows)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v == "Active"})
+        loaded = [s for s in sm if s > 0.5 * mx] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": reasons,
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------- workloads
+
+def algorithmic_work(x):
+    """Per-launch algorithmic work of one forward over batch x (units in the docstrings)."""
+    pos = x.positions().cpu().long()
+    n = pos + 1
+    H_I, d_I = x.q_idx.shape[1], x.q_idx.shape[2]
+    Hq, d_qk = x.q.shape[1], x.q.shape[2]
+    d_v, k = x.d_v, x.k
+    sel = torch.clamp(n, max=k)
+    # indexer: FP8 flops of q.k over the causal pairs of rows that need scoring (n > k)
+    scored = n[n > k]
+    idx_flops = float(scored.sum().item()) * 2 * H_I * d_I
+    # attention: bf16 flops of q.c (d_qk) and p.v (d_v) per (row, selected entry, head)
+    attn_flops = float(sel.sum().item()) * Hq * 2 * (d_qk + d_v)
+    # bytes a perfect implementation moves: every key of every row's range read once
+    # (decode), the selected latent rows gathered once per row, q read, out/lse written
+    idx_bytes = float(n.sum().item()) * d_I + x.T * (H_I * d_I + 4 * H_I + 4 * k)
+    attn_bytes = (float(sel.sum().item()) * d_qk * 2 + x.T * Hq * (d_qk * 2 + d_v * 2 + 4)
+                  + x.T * k * 4)
+    return dict(idx_flops=idx_flops, attn_flops=attn_flops, idx_bytes=idx_bytes,
+                attn_bytes=attn_bytes)
+
+
+class Batch:
+    def __init__(self, x, dsa):
+        self.x = x
+        self.T, self.S = x.T, x.S
+        self.H_I, self.d_I = x.q_idx.shape[1], x.q_idx.shape[2]
+        self.Hq, self.d_qk = x.q.shape[1], x.q.shape[2]
+        dev = x.q.device
+        self.idx = torch.empty((self.T, x.k), dtype=torch.int32, device=dev)
+        self.out = torch.empty((self.T, self.Hq, x.d_v), dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty((self.T, self.Hq), dtype=torch.float32, device=dev)
+        self.ws = dsa.alloc_workspace(self.T, self.S, self.H_I, self.d_I, x.k, self.Hq,
+                                      self.d_qk, x.d_v, dev)
+        self.work = algorithmic_work(x)
+
+
+def run_indexer(dsa, b, stream):
+    x = b.x
+    dsa.indexer_topk(x.q_idx, x.w, x.k_idx, x.k, pos=x.pos, k_base=x.k_base, idx=b.idx,
+                     workspace=b.ws, stream=stream)
+
+
+def run_attn(dsa, b, stream):
+    x = b.x
+    dsa.sparse_mla_attn(x.q, x.kv, b.idx, x.scale, x.d_v, pos=x.pos, k_base=x.k_base, out=b.out,
+                        lse=b.lse, workspace=b.ws, stream=stream)
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm=p["hbm_gbs"], bf16=p["bf16_tflops"],
+                    bf16_sustained=p.get("bf16_tflops_sustained", p["bf16_tflops"]),
+                    source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+# --------------------------------------------------------- CPU baseline
+
+def time_oracle_sample(x, rows):
+    import numpy as np
+    import oracle
+    r = torch.tensor(rows, device=x.q.device)
+    q_idx = x.q_idx[r].cpu().numpy()
+    w = x.w[r].cpu().numpy()
+    k_idx = x.k_idx.cpu().numpy()
+    q = x.q[r].cpu()
+    kv = x.kv.cpu()
+    pos = x.positions()[r].cpu().numpy()
+    base = x.bases()[r].cpu().numpy()
+    t0 = time.perf_counter()
+    idx = oracle.indexer_topk(q_idx, w, k_idx, pos, base, x.k)
+    oracle.sparse_attn(q, kv, None, pos, base, x.scale, x.d_v, idx_rows=idx)
+    return time.perf_counter() - t0, oracle.num_threads()
+
+
+def cpu_baseline(x, seed=0, target_s=15.0):
+    """The oracle as it stands on a bounded sample of query rows of workload x."""
+    import oracle
+    threads = oracle.num_threads()
+    g = torch.Generator().manual_seed(seed)
+    n = max(4, threads)
+    rows = sorted(torch.randperm(x.T, generator=g)[:n].tolist())
+    dt, cores = time_oracle_sample(x, rows)
+    # grow once towards the target duration if the first sample was short
+    if dt < target_s / 4:
+        n2 = min(x.T, int(n * min(8.0, target_s / max(dt, 1e-3))))
+        rows = sorted(torch.randperm(x.T, generator=g)[:n2].tolist())
+        dt, cores = time_oracle_sample(x, rows)
+    return dict(value=len(rows) / dt, unit="tokens/s", cores=cores, kind="oracle",
+                sample=f"{len(rows)} uniformly drawn query rows of the {x.config} workload "
+                       f"(L={x.T}); indexer scores of all causal keys, full sort, fp64 "
+                       f"attention over the selected rows; {dt:.1f} s")
+
+
+# ----------------------------------------------------------- ours
+
+def bench_ours(args, world, rank, local):
+    import sparse_attention_20_b200 as dsa
+    from sparse_attention_20_b200 import build as dsa_build
+    if rank == 0:
+        dsa_build.build()
+    barrier(world)
+    dsa.load_library()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    xp = synth.make_inputs(args.prefill, device=dev, seed=args.seed + rank)
+    xd = synth.make_inputs(args.decode, device=dev, seed=args.seed + rank)
+    bp, bd = Batch(xp, dsa), Batch(xd, dsa)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev is not None: ev[0].record(stream)
+        run_indexer(dsa, bp, stream)
+        if ev is not None: ev[1].record(stream)
+        run_attn(dsa, bp, stream)
+        if ev is not None: ev[2].record(stream)
+        run_indexer(dsa, bd, stream)
+        if ev is not None: ev[3].record(stream)
+        run_attn(dsa, bd, stream)
+        if ev is not None: ev[4].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert dsa.device_status() == 0, dsa.last_error()
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    n0 = dsa.launch_count()
+    start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    end.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    launches = dsa.launch_count() - n0
+    clk = clocks.stop()
+    total_ms = max_over_ranks(world, start.elapsed_time(end))
+    parts = [[e[j].elapsed_time(e[j + 1]) for e in evs] for j in range(4)]
+    p_idx, p_attn, d_idx, d_attn = (max_over_ranks(world, statistics.mean(p)) for p in parts)
+    assert dsa.device_status() == 0, dsa.last_error()
+
+    ms_step = total_ms / args.steps
+    prefill_ms = p_idx + p_attn
+    decode_ms = d_idx + d_attn
+    tokens = world * xp.T
+    peaks = measured_peaks()
+    wp, wd = bp.work, bd.work
+    attn_tflops = wp["attn_flops"] / (p_attn * 1e-3) / 1e12
+    fp8_peak = 2.0 * peaks["bf16_sustained"]
+    result = {
+        "metric": METRIC,
+        "value": tokens / (ms_step * 1e-3),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded; shapes and distributions of the pages' 128K workloads)",
+        "config": {"workload": f"{args.prefill} causal prefill (L={xp.T}, H_I={bp.H_I}, "
+                               f"d_I={bp.d_I}, k={xp.k}, Hq={bp.Hq}, d_qk={bp.d_qk}, "
+                               f"d_v={xp.d_v}) + {args.decode} step ({xd.T} seqs, "
+                               f"ctx U[8192,131072])",
+                   "global_batch": world, "seq_len": xp.T, "parallelism": f"replicas{world}",
+                   "l2": "inputs larger than L2 (19 GB of queries, 151 MB latent cache)"},
+        "prefill_tokens_per_s": tokens / (prefill_ms * 1e-3),
+        "decode": {"value": world * xd.T / (decode_ms * 1e-3), "unit": "seqs/s",
+                   "ms_per_step": decode_ms,
+                   "hbm_gbs": (wd["idx_bytes"] + wd["attn_bytes"]) / (decode_ms * 1e-3) / 1e9,
+                   "hbm_frac": (wd["idx_bytes"] + wd["attn_bytes"]) / (decode_ms * 1e-3) / 1e9
+                   / peaks["hbm"]},
+        "kernels_ms": {"prefill_indexer_topk": p_idx, "prefill_sparse_attn": p_attn,
+                       "decode_indexer_topk": d_idx, "decode_sparse_attn": d_attn},
+        "roofline": {"bound": "tensor", "kernel": "prefill sparse MLA attention",
+                     "achieved": attn_tflops, "peak": peaks["bf16_sustained"],
+                     "unit": "TFLOP/s", "frac": attn_tflops / peaks["bf16_sustained"],
+                     "traffic": None,
+                     "peak_source": f"{peaks['source']} bf16 sustained"},
+        "rooflines": {
+            "prefill_indexer_topk": {"bound": "tensor", "unit": "TFLOP/s",
+                                     "achieved": wp["idx_flops"] / (p_idx * 1e-3) / 1e12,
+                                     "peak": fp8_peak,
+                                     "frac": wp["idx_flops"] / (p_idx * 1e-3) / 1e12 / fp8_peak,
+                                     "peak_source": "2 x measured bf16 sustained (fp8 ratio)"},
+            "decode_step": {"bound": "hbm", "unit": "GB/s",
+                            "achieved": (wd["idx_bytes"] + wd["attn_bytes"]) / (decode_ms * 1e-3)
+                            / 1e9, "peak": peaks["hbm"]},
+        },
+        "gpu_launches": launches,
+        "clocks": clk,
+    }
+    if not args.no_e2e:
+        result["e2e"] = bench_e2e(args, world, dsa, bp, bd, stream)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(xp, seed=args.seed)
+    return result
+
+
+def bench_e2e(args, world, dsa, bp, bd, stream):
+    """Same step through the C ABI with inputs in pinned host memory: every step
+    copies its inputs host->device and reads idx/out/lse back."""
+    def host(t):
+        try:
+            h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+        except RuntimeError:
+            h = torch.empty(t.shape, dtype=t.dtype)
+        h.copy_(t)
+        return h
+
+    pairs_in, pairs_out = [], []
+    for b in (bp, bd):
+        x = b.x
+        for t in (x.q_idx, x.w, x.k_idx, x.q, x.kv, x.pos, x.k_base):
+            if t is not None:
+                pairs_in.append((host(t), t))
+        for t in (b.idx, b.out, b.lse):
+            pairs_out.append((host(t), t))
+    h2d = sum(h.numel() * h.element_size() for h, _ in pairs_in)
+    d2h = sum(h.numel() * h.element_size() for h, _ in pairs_out)
+
+    def step():
+        for h, d in pairs_in:
+            d.copy_(h, non_blocking=True)
+        for b in (bp, bd):
+            run_indexer(dsa, b, stream)
+            run_attn(dsa, b, stream)
+        for h, d in pairs_out:
+            h.copy_(d, non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    start.record(stream)
+    for _ in range(args.e2e_steps):
+        step()
+    end.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(world, start.elapsed_time(end)) / args.e2e_steps
+    return {"value": world * bp.T / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "pinned": all(h.is_pinned() for h, _ in pairs_in + pairs_out)}
+
+
+# ------------------------------------------------------ reference arm
+
+def bench_reference(args, world, rank):
+    """The CPU oracle as the reference arm, on bounded samples of the same workload."""
+    import oracle
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    x = synth.make_inputs(args.prefill, device=dev, seed=args.seed)
+    threads = oracle.num_threads()
+    g = torch.Generator().manual_seed(args.seed)
+    per_step = max(2, threads)
+    samples = []
+    for i in range(args.warmup + args.steps):
+        rows = sorted(torch.randperm(x.T, generator=g)[:per_step].tolist())
+        dt, cores = time_oracle_sample(x, rows)
+        if i >= args.warmup:
+            samples.append((len(rows), dt))
+    rows_total = sum(n for n, _ in samples)
+    secs = sum(d for _, d in samples)
+    value = rows_total / secs
+    sample = (f"{per_step} uniformly drawn query rows of the {x.config} workload per step "
+              f"(L={x.T}); oracle indexer + full sort + fp64 attention")
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": f"{args.prefill} causal prefill (sampled rows)", "seq_len": x.T},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        # rank 0 alone times the oracle; other ranks exit without work
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        if int(os.environ.get("RANK", "0")) == 0:
+            print(json.dumps(bench_reference(args, world, 0)), flush=True)
+        return
+    world, rank, local = dist_setup(args)
+    res = bench_ours(args, world, rank, local)
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

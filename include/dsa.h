@@ -1,0 +1,138 @@
+/*
+ * dsa.h -- C ABI of the DeepSeek Sparse Attention (DSA) hot path, B200 (sm_100a).
+ *
+ * The operations (page "Paper Breakdown: DeepSeek-V3.2", section 2
+ * "Architecture: DSA (2.1)"):
+ *
+ *   index score   I_{t,s} = sum_{j<H_I} w_{t,j} * ReLU(q^I_{t,j} . k^I_s)
+ *   selector      the k candidates s <= pos[t] with the largest I_{t,s}
+ *                 ("Top-k selector on I_{t,s}"; past tokens only, per the
+ *                 summary page "DeepSeek V3.2: Sparse Attention and
+ *                 Reinforcement Learning Updates"; k = 2048 per the research
+ *                 summary's "Key points")
+ *   attention     u_t = Attn(h_t, {c_s : s selected}), MLA in MQA mode: every
+ *                 query head attends to the same latent row c_s
+ *                 ("DSA under MLA (MQA Mode)").
+ *
+ * Conventions shared by every entry point
+ *  - Pointers are DEVICE pointers owned by the caller. The library keeps no
+ *    pointer after a call returns and allocates no device memory: scratch
+ *    comes from the caller's `workspace`. `stream` is a cudaStream_t (NULL =
+ *    legacy default stream); every call is asynchronous on it.
+ *  - Tensors are dense and row-major. FP8 tensors hold OCP E4M3 bytes; BF16
+ *    tensors hold bfloat16 values. Every pointer must be 16-byte aligned.
+ *  - Query row t sees the candidates s = 0..pos[t] of its own sequence, whose
+ *    key/latent rows sit at k_base[t] + s in the caches. pos == NULL means
+ *    pos[t] = t + S - T (one causal sequence whose last T rows are the
+ *    queries); k_base == NULL means k_base[t] = 0. k_base[t] + pos[t] < S.
+ *  - Return value: DSA_OK, or a negative dsa_status. Arguments are checked
+ *    before any launch; nothing is launched when a check fails. The message of
+ *    the last failure on the calling thread is dsa_last_error().
+ *  - Kernels that wait on on-chip barriers bound every wait; a wait that runs
+ *    out records DSA_ERR_TIMEOUT in a device status word read (and cleared)
+ *    by dsa_device_status().
+ */
+#ifndef DSA_H
+#define DSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    DSA_OK = 0,
+    DSA_ERR_ARG = -1,         /* NULL pointer, size <= 0, misaligned pointer, bad pos/k_base */
+    DSA_ERR_UNSUPPORTED = -2, /* a dimension outside the supported set (below) */
+    DSA_ERR_CUDA = -3,        /* a CUDA runtime error at launch (or an earlier asynchronous one) */
+    DSA_ERR_TIMEOUT = -4,     /* a kernel gave up a bounded wait (see dsa_device_status) */
+    DSA_ERR_WORKSPACE = -5    /* workspace NULL or smaller than dsa_workspace_size() */
+} dsa_status;
+
+/*
+ * Bytes of device workspace that dsa_indexer_topk, dsa_sparse_mla_attn and
+ * dsa_forward need for these sizes (the maximum over the three). 0 is a valid
+ * answer; a NULL workspace is then accepted. The workspace is scratch: its
+ * contents on entry do not matter and are undefined on return. Two calls in
+ * flight at the same time need two workspaces.
+ */
+size_t dsa_workspace_size(int T, int S, int H_I, int d_I, int k, int Hq, int d_qk, int d_v);
+
+/*
+ * Lightning indexer + Top-k selector ("Index score" and "Top-k selector",
+ * section 2 of "Paper Breakdown: DeepSeek-V3.2").
+ *
+ *   q_idx   e4m3 [T, H_I, d_I]   indexer query heads
+ *   w       fp32 [T, H_I]        head weights
+ *   k_idx   e4m3 [S, d_I]        indexer keys
+ *   pos     int32 [T] or NULL    last candidate of each row (see above)
+ *   k_base  int32 [T] or NULL    first cache row of each row's sequence
+ *   k       number of selected entries per row
+ *   idx     int32 [T, k] (out)   row t: the min(k, pos[t]+1) selected s values
+ *                                (relative to k_base[t]), distinct, in
+ *                                unspecified order, followed by -1 padding.
+ *
+ * Scores are formed in fp32 (FP8 products are exact in fp32). Among equal
+ * scores the lower s is selected first, so the result is unique.
+ * Supported: H_I <= 16, d_I in {32, 64, 128, 256}, 1 <= k <= 4096.
+ */
+int dsa_indexer_topk(const void* q_idx, const float* w, const void* k_idx, const int32_t* pos,
+                     const int32_t* k_base, int T, int S, int H_I, int d_I, int k, int32_t* idx,
+                     void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Sparse MQA attention over the selected latent rows ("Attention" and "DSA
+ * under MLA (MQA Mode)", section 2 of "Paper Breakdown: DeepSeek-V3.2").
+ *
+ *   q      bf16 [T, Hq, d_qk]   query heads (latent + rope parts)
+ *   kv     bf16 [S, d_qk]       latent rows c_s; the value is c_s[0:d_v]
+ *   idx    int32 [T, k]         selected s per row (relative to k_base[t]).
+ *                               Entries < 0 or > pos[t] are ignored. Valid
+ *                               entries come first: the call reads only the
+ *                               first min(k, pos[t]+1) entries of a row.
+ *   scale  softmax scale (e.g. 1/sqrt(d_qk))
+ *   out    bf16 [T, Hq, d_v] (out)   sum_s softmax_s(scale q.c_s) c_s[0:d_v]
+ *   lse    fp32 [T, Hq] (out)        log sum_s exp(scale q.c_s) (natural log);
+ *                                    -inf and out = 0 for a row with no entry
+ * Supported: Hq <= 1024, d_v <= d_qk <= 1024, d_v even, d_qk % 8 == 0,
+ * 1 <= k <= 4096.
+ */
+int dsa_sparse_mla_attn(const void* q, const void* kv, const int32_t* idx, const int32_t* pos,
+                        const int32_t* k_base, int T, int S, int Hq, int d_qk, int d_v, int k,
+                        float scale, void* out, float* lse, void* workspace, size_t ws_bytes,
+                        void* stream);
+
+/*
+ * The whole hot path: dsa_indexer_topk followed by dsa_sparse_mla_attn on the
+ * same stream. `idx` is an output the caller keeps (it is also the input of
+ * the attention step). Argument meanings and limits as above.
+ */
+int dsa_forward(const void* q_idx, const float* w, const void* k_idx, const void* q,
+                const void* kv, const int32_t* pos, const int32_t* k_base, int T, int S, int H_I,
+                int d_I, int Hq, int d_qk, int d_v, int k, float scale, int32_t* idx, void* out,
+                float* lse, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Waits for `stream`, then returns and clears the device status word:
+ * DSA_OK, DSA_ERR_TIMEOUT (a kernel gave up a bounded wait) or DSA_ERR_CUDA
+ * (an asynchronous CUDA error; its text is in dsa_last_error()).
+ */
+int dsa_device_status(void* stream);
+
+/* Text of the last error on the calling thread ("" when none). */
+const char* dsa_last_error(void);
+
+/* ABI version: bumped on any change of a signature or a convention. */
+int dsa_abi_version(void);
+
+/* Number of kernels this process has launched through the library so far
+ * (all threads, all devices): a diagnostic for launch accounting. */
+uint64_t dsa_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_H */

@@ -1,0 +1,207 @@
+"""DeepSeek Sparse Attention (DSA) hot path on B200 (sm_100a): Python binding.
+
+A thin ctypes layer over ``libdsa.so`` (C ABI in ``include/dsa.h``): it checks
+tensor dtypes/devices, passes raw device pointers and the current CUDA stream,
+and raises on a non-zero status. Every step of the computation runs in the
+library's CUDA kernels; PyTorch only provides device memory and streams. There
+is no CPU fallback: without the built library (or without a GPU) every call
+raises.
+
+Entry points mirror the C ABI:
+  * ``indexer_topk``     lightning indexer + Top-k selector -> idx [T, k]
+  * ``sparse_mla_attn``  sparse MQA attention over idx -> out [T, Hq, d_v], lse [T, Hq]
+  * ``forward``          both, on one stream
+  * ``workspace_size``, ``device_status``, ``last_error``
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libdsa.so")
+
+DSA_OK = 0
+STATUS_NAMES = {0: "DSA_OK", -1: "DSA_ERR_ARG", -2: "DSA_ERR_UNSUPPORTED", -3: "DSA_ERR_CUDA",
+                -4: "DSA_ERR_TIMEOUT", -5: "DSA_ERR_WORKSPACE"}
+
+# Every symbol include/dsa.h declares.
+EXPORTS = ("dsa_workspace_size", "dsa_indexer_topk", "dsa_sparse_mla_attn", "dsa_forward",
+           "dsa_device_status", "dsa_last_error", "dsa_abi_version", "dsa_launch_count")
+
+
+class DSAError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"{STATUS_NAMES.get(code, code)}: {msg}")
+        self.code = code
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libdsa.so (raises OSError if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(path):
+            raise OSError(f"{path} is missing: build it with "
+                          "`python -m sparse_attention_20_b200.build`")
+        lib = ctypes.CDLL(path)
+        P, I, Z, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float
+        lib.dsa_workspace_size.argtypes = [I] * 8
+        lib.dsa_workspace_size.restype = Z
+        lib.dsa_indexer_topk.argtypes = [P, P, P, P, P, I, I, I, I, I, P, P, Z, P]
+        lib.dsa_indexer_topk.restype = I
+        lib.dsa_sparse_mla_attn.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, P, P, P, Z, P]
+        lib.dsa_sparse_mla_attn.restype = I
+        lib.dsa_forward.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, F, P, P, P, P, Z,
+                                    P]
+        lib.dsa_forward.restype = I
+        lib.dsa_device_status.argtypes = [P]
+        lib.dsa_device_status.restype = I
+        lib.dsa_last_error.restype = ctypes.c_char_p
+        lib.dsa_abi_version.restype = I
+        lib.dsa_launch_count.restype = ctypes.c_uint64
+        _lib = lib
+    return _lib
+
+
+def last_error() -> str:
+    return load_library().dsa_last_error().decode()
+
+
+def _check(rc: int):
+    if rc != DSA_OK:
+        raise DSAError(rc, last_error())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _fp8(t: torch.Tensor, name: str) -> torch.Tensor:
+    if t.dtype == torch.float8_e4m3fn:
+        t = t.view(torch.uint8)
+    if t.dtype != torch.uint8:
+        raise TypeError(f"{name} must hold e4m3 bytes (uint8 or float8_e4m3fn), got {t.dtype}")
+    return _dev(t, name)
+
+
+def _dev(t: torch.Tensor, name: str) -> torch.Tensor:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def _i32(t: Optional[torch.Tensor], name: str):
+    if t is None:
+        return None
+    if t.dtype != torch.int32:
+        raise TypeError(f"{name} must be int32")
+    return _dev(t, name)
+
+
+def workspace_size(T, S, H_I, d_I, k, Hq, d_qk, d_v) -> int:
+    return int(load_library().dsa_workspace_size(T, S, H_I, d_I, k, Hq, d_qk, d_v))
+
+
+def alloc_workspace(T, S, H_I, d_I, k, Hq, d_qk, d_v, device=None) -> torch.Tensor:
+    n = workspace_size(T, S, H_I, d_I, k, Hq, d_qk, d_v)
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=device or "cuda")
+
+
+def indexer_topk(q_idx, w, k_idx, k: int, pos=None, k_base=None, idx=None, workspace=None,
+                 stream=None) -> torch.Tensor:
+    """idx [T, k] int32: the Top-k s per query row (a set, -1 padded)."""
+    q_idx = _fp8(q_idx, "q_idx")
+    k_idx = _fp8(k_idx, "k_idx")
+    w = _dev(w, "w")
+    if w.dtype != torch.float32:
+        raise TypeError("w must be float32")
+    T, H_I, d_I = q_idx.shape
+    S = k_idx.shape[0]
+    pos, k_base = _i32(pos, "pos"), _i32(k_base, "k_base")
+    if idx is None:
+        idx = torch.empty((T, k), dtype=torch.int32, device=q_idx.device)
+    if workspace is None:
+        workspace = alloc_workspace(T, S, H_I, d_I, k, 1, 8, 2, q_idx.device)
+    lib = load_library()
+    _check(lib.dsa_indexer_topk(_ptr(q_idx), _ptr(w), _ptr(k_idx), _ptr(pos), _ptr(k_base), T, S,
+                                H_I, d_I, k, _ptr(idx), _ptr(workspace), workspace.numel(),
+                                _stream(stream)))
+    return idx
+
+
+def sparse_mla_attn(q, kv, idx, scale: float, d_v: int, pos=None, k_base=None, out=None,
+                    lse=None, workspace=None, stream=None):
+    """(out bf16 [T, Hq, d_v], lse fp32 [T, Hq]) of sparse MQA attention over idx."""
+    q, kv = _dev(q, "q"), _dev(kv, "kv")
+    if q.dtype != torch.bfloat16 or kv.dtype != torch.bfloat16:
+        raise TypeError("q and kv must be bfloat16")
+    idx = _i32(idx, "idx")
+    T, Hq, d_qk = q.shape
+    S = kv.shape[0]
+    k = idx.shape[1]
+    pos, k_base = _i32(pos, "pos"), _i32(k_base, "k_base")
+    if out is None:
+        out = torch.empty((T, Hq, d_v), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((T, Hq), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = alloc_workspace(T, S, 1, 32, k, Hq, d_qk, d_v, q.device)
+    lib = load_library()
+    _check(lib.dsa_sparse_mla_attn(_ptr(q), _ptr(kv), _ptr(idx), _ptr(pos), _ptr(k_base), T, S, Hq,
+                                   d_qk, d_v, k, float(scale), _ptr(out), _ptr(lse),
+                                   _ptr(workspace), workspace.numel(), _stream(stream)))
+    return out, lse
+
+
+def forward(q_idx, w, k_idx, q, kv, k: int, scale: float, d_v: int, pos=None, k_base=None,
+            idx=None, out=None, lse=None, workspace=None, stream=None):
+    """The whole hot path: (idx, out, lse)."""
+    q_idx, k_idx = _fp8(q_idx, "q_idx"), _fp8(k_idx, "k_idx")
+    q, kv, w = _dev(q, "q"), _dev(kv, "kv"), _dev(w, "w")
+    T, H_I, d_I = q_idx.shape
+    _, Hq, d_qk = q.shape
+    S = k_idx.shape[0]
+    pos, k_base = _i32(pos, "pos"), _i32(k_base, "k_base")
+    dev = q.device
+    if idx is None:
+        idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+    if out is None:
+        out = torch.empty((T, Hq, d_v), dtype=torch.bfloat16, device=dev)
+    if lse is None:
+        lse = torch.empty((T, Hq), dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = alloc_workspace(T, S, H_I, d_I, k, Hq, d_qk, d_v, dev)
+    lib = load_library()
+    _check(lib.dsa_forward(_ptr(q_idx), _ptr(w), _ptr(k_idx), _ptr(q), _ptr(kv), _ptr(pos),
+                           _ptr(k_base), T, S, H_I, d_I, Hq, d_qk, d_v, k, float(scale), _ptr(idx),
+                           _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(),
+                           _stream(stream)))
+    return idx, out, lse
+
+
+def device_status(stream=None) -> int:
+    """Wait for the stream and return (and clear) the device status word."""
+    return int(load_library().dsa_device_status(_stream(stream)))
+
+
+def abi_version() -> int:
+    return int(load_library().dsa_abi_version())
+
+
+def launch_count() -> int:
+    """Kernels launched through the library by this process so far."""
+    return int(load_library().dsa_launch_count())

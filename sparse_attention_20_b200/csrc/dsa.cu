@@ -1,0 +1,305 @@
+// C ABI of the DSA hot path (declared in include/dsa.h): argument checks,
+// workspace layout and kernel dispatch. All kernels live in the headers
+// included below and are compiled here as one translation unit for sm_100a.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+
+#include "dsa.h"
+#include "attn_simple.cuh"
+#include "common.cuh"
+#include "indexer_scores.cuh"
+#include "topk_select.cuh"
+
+namespace {
+
+thread_local char g_err[512] = {0};
+std::atomic<unsigned long long> g_launches{0};
+
+int fail(int code, const char* fmt, ...)
+{
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof g_err, fmt, ap);
+    va_end(ap);
+    return code;
+}
+
+bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int cuda_fail(cudaError_t e, const char* where)
+{
+    return fail(DSA_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+#define DSA_LAUNCH_CHECK(where)                                      \
+    do {                                                             \
+        g_launches.fetch_add(1, std::memory_order_relaxed);          \
+        cudaError_t e_ = cudaGetLastError();                         \
+        if (e_ != cudaSuccess) return cuda_fail(e_, where);          \
+    } while (0)
+
+// ------------------------------------------------------------ workspace plan
+
+constexpr size_t kAlign = 256;
+constexpr size_t kScoreBlockBytes = size_t(1) << 30;  // score rows kept per block of queries
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+// Query rows whose full score rows fit in one block of the score buffer.
+int index_rows_per_block(int T, int S)
+{
+    const size_t per_row = (size_t)S * sizeof(float);
+    const size_t rows = std::max<size_t>(1, kScoreBlockBytes / per_row);
+    return (int)std::min<size_t>((size_t)T, rows);
+}
+
+size_t indexer_workspace(int T, int S)
+{
+    return align_up((size_t)index_rows_per_block(T, S) * (size_t)S * sizeof(float));
+}
+
+int num_sms()
+{
+    static int sms = 0;
+    if (!sms) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (sms <= 0) sms = 148;
+    }
+    return sms;
+}
+
+// Splits of each row's selected set so that few rows still fill the GPU.
+int attn_splits(int T, int Hq, int k)
+{
+    if (const char* e = getenv("DSA_ATTN_SPLITS")) {
+        const int v = atoi(e);
+        if (v >= 1) return std::min(v, std::max(1, k));
+    }
+    const long long ctas = (long long)T * dsa::ceil_div(Hq, dsa::kAttnHeads);
+    const long long want = 2LL * num_sms();
+    if (ctas >= want) return 1;
+    const int s = (int)((want + ctas - 1) / ctas);
+    return std::max(1, std::min({s, 16, std::max(1, k / 64)}));
+}
+
+size_t attn_workspace(int T, int Hq, int d_v, int k)
+{
+    const int splits = attn_splits(T, Hq, k);
+    if (splits == 1) return 0;
+    return align_up((size_t)T * splits * Hq * d_v * sizeof(float)) +
+           align_up((size_t)T * splits * Hq * sizeof(float));
+}
+
+// ---------------------------------------------------------- argument checks
+
+int check_rows(const int32_t* pos, const int32_t* k_base, int T, int S)
+{
+    if (T <= 0 || S <= 0) return fail(DSA_ERR_ARG, "T=%d and S=%d must be positive", T, S);
+    if (!pos && T > S) return fail(DSA_ERR_ARG, "pos == NULL needs T <= S (T=%d, S=%d)", T, S);
+    if ((pos && !al16(pos)) || (k_base && !al16(k_base)))
+        return fail(DSA_ERR_ARG, "pos / k_base must be 16-byte aligned");
+    return DSA_OK;
+}
+
+int check_indexer(const void* q_idx, const float* w, const void* k_idx, const int32_t* pos,
+                  const int32_t* k_base, int T, int S, int H_I, int d_I, int k, const int32_t* idx)
+{
+    if (!q_idx || !w || !k_idx || !idx) return fail(DSA_ERR_ARG, "NULL q_idx, w, k_idx or idx");
+    if (!al16(q_idx) || !al16(w) || !al16(k_idx) || !al16(idx))
+        return fail(DSA_ERR_ARG, "q_idx, w, k_idx and idx must be 16-byte aligned");
+    if (int rc = check_rows(pos, k_base, T, S)) return rc;
+    if (H_I <= 0 || H_I > 16) return fail(DSA_ERR_UNSUPPORTED, "H_I=%d (supported: 1..16)", H_I);
+    if (d_I != 32 && d_I != 64 && d_I != 128 && d_I != 256)
+        return fail(DSA_ERR_UNSUPPORTED, "d_I=%d (supported: 32, 64, 128, 256)", d_I);
+    if (k <= 0 || k > 4096) return fail(DSA_ERR_UNSUPPORTED, "k=%d (supported: 1..4096)", k);
+    return DSA_OK;
+}
+
+int check_attn(const void* q, const void* kv, const int32_t* idx, const int32_t* pos,
+               const int32_t* k_base, int T, int S, int Hq, int d_qk, int d_v, int k,
+               const void* out, const float* lse)
+{
+    if (!q || !kv || !idx || !out || !lse) return fail(DSA_ERR_ARG, "NULL q, kv, idx, out or lse");
+    if (!al16(q) || !al16(kv) || !al16(idx) || !al16(out) || !al16(lse))
+        return fail(DSA_ERR_ARG, "q, kv, idx, out and lse must be 16-byte aligned");
+    if (int rc = check_rows(pos, k_base, T, S)) return rc;
+    if (Hq <= 0 || Hq > 1024) return fail(DSA_ERR_UNSUPPORTED, "Hq=%d (supported: 1..1024)", Hq);
+    if (d_qk <= 0 || d_qk > 1024 || d_qk % 8)
+        return fail(DSA_ERR_UNSUPPORTED, "d_qk=%d (supported: multiples of 8 up to 1024)", d_qk);
+    if (d_v <= 0 || d_v > d_qk || d_v % 2)
+        return fail(DSA_ERR_UNSUPPORTED, "d_v=%d (supported: even, <= d_qk)", d_v);
+    if (k <= 0 || k > 4096) return fail(DSA_ERR_UNSUPPORTED, "k=%d (supported: 1..4096)", k);
+    return DSA_OK;
+}
+
+// ----------------------------------------------------------------- indexer
+
+template <int NT, int DI>
+void launch_scores(dim3 grid, cudaStream_t st, const uint8_t* q_idx, const float* w,
+                   const uint8_t* k_idx, const int* pos, const int* k_base, int T, int S, int H_I,
+                   int row0, float* scores, long long ld, int keys_per_cta)
+{
+    dsa::indexer_scores_kernel<NT, DI><<<grid, dsa::kScoreThreads, 0, st>>>(
+        q_idx, w, k_idx, pos, k_base, T, S, H_I, row0, scores, ld, keys_per_cta);
+}
+
+using ScoresFn = void (*)(dim3, cudaStream_t, const uint8_t*, const float*, const uint8_t*,
+                          const int*, const int*, int, int, int, int, float*, long long, int);
+
+ScoresFn pick_scores(int H_I, int d_I)
+{
+    const bool two = H_I > 8;
+    switch (d_I) {
+        case 32: return two ? launch_scores<2, 32> : launch_scores<1, 32>;
+        case 64: return two ? launch_scores<2, 64> : launch_scores<1, 64>;
+        case 128: return two ? launch_scores<2, 128> : launch_scores<1, 128>;
+        default: return two ? launch_scores<2, 256> : launch_scores<1, 256>;
+    }
+}
+
+int indexer_scan_select(const uint8_t* q_idx, const float* w, const uint8_t* k_idx,
+                        const int32_t* pos, const int32_t* k_base, int T, int S, int H_I, int d_I,
+                        int k, int32_t* idx, void* workspace, cudaStream_t st)
+{
+    const int RB = index_rows_per_block(T, S);
+    float* scores = reinterpret_cast<float*>(workspace);
+    const long long ld = S;
+    constexpr int kKeysPerCta = 2048;
+    ScoresFn scores_fn = pick_scores(H_I, d_I);
+    for (int row0 = 0; row0 < T; row0 += RB) {
+        const int rb = std::min(RB, T - row0);
+        // longest candidate range in this block of rows
+        const int n_max = pos ? S : std::min(S, row0 + rb + S - T);
+        dim3 grid(dsa::ceil_div(n_max, kKeysPerCta), rb);
+        scores_fn(grid, st, q_idx, w, k_idx, pos, k_base, T, S, H_I, row0, scores, ld, kKeysPerCta);
+        DSA_LAUNCH_CHECK("indexer_scores_kernel");
+        dsa::topk_dense_rows_kernel<dsa::kSelectThreads>
+            <<<rb, dsa::kSelectThreads, 0, st>>>(scores, ld, pos, T, S, row0, k, idx);
+        DSA_LAUNCH_CHECK("topk_dense_rows_kernel");
+    }
+    return DSA_OK;
+}
+
+// --------------------------------------------------------------- attention
+
+int attn_simple(const __nv_bfloat16* q, const __nv_bfloat16* kv, const int32_t* idx,
+                const int32_t* pos, const int32_t* k_base, int T, int S, int Hq, int d_qk,
+                int d_v, int k, float scale, __nv_bfloat16* out, float* lse, void* workspace,
+                cudaStream_t st)
+{
+    const int splits = attn_splits(T, Hq, k);
+    const int kcap = dsa::ceil_div(k, splits);
+    const size_t smem = dsa::attn_simple_smem(d_qk, kcap);
+    cudaError_t e = cudaFuncSetAttribute(dsa::sparse_attn_simple_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(sparse_attn_simple_kernel)");
+    float* part_o = nullptr;
+    float* part_lse = nullptr;
+    if (splits > 1) {
+        part_o = reinterpret_cast<float*>(workspace);
+        part_lse = reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) +
+                                            align_up((size_t)T * splits * Hq * d_v * sizeof(float)));
+    }
+    dim3 grid(T, dsa::ceil_div(Hq, dsa::kAttnHeads), splits);
+    dsa::sparse_attn_simple_kernel<<<grid, dsa::kAttnThreads, smem, st>>>(
+        q, kv, idx, pos, k_base, T, S, Hq, d_qk, d_v, k, kcap, scale, out, lse, part_o, part_lse);
+    DSA_LAUNCH_CHECK("sparse_attn_simple_kernel");
+    if (splits > 1) {
+        dsa::lse_combine_kernel<<<dim3(T, Hq), 128, 0, st>>>(part_o, part_lse, T, Hq, d_v, splits,
+                                                             out, lse);
+        DSA_LAUNCH_CHECK("lse_combine_kernel");
+    }
+    return DSA_OK;
+}
+
+}  // namespace
+
+// ===================================================================== C ABI
+
+extern "C" {
+
+int dsa_abi_version(void) { return 1; }
+
+uint64_t dsa_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+const char* dsa_last_error(void) { return g_err; }
+
+size_t dsa_workspace_size(int T, int S, int H_I, int d_I, int k, int Hq, int d_qk, int d_v)
+{
+    (void)H_I;
+    (void)d_I;
+    (void)d_qk;
+    if (T <= 0 || S <= 0 || k <= 0 || Hq <= 0 || d_v <= 0) return 0;
+    return std::max(indexer_workspace(T, S), attn_workspace(T, Hq, d_v, k));
+}
+
+int dsa_indexer_topk(const void* q_idx, const float* w, const void* k_idx, const int32_t* pos,
+                     const int32_t* k_base, int T, int S, int H_I, int d_I, int k, int32_t* idx,
+                     void* workspace, size_t ws_bytes, void* stream)
+{
+    g_err[0] = 0;
+    if (int rc = check_indexer(q_idx, w, k_idx, pos, k_base, T, S, H_I, d_I, k, idx)) return rc;
+    const size_t need = indexer_workspace(T, S);
+    if (need && (!workspace || ws_bytes < need || !al16(workspace)))
+        return fail(DSA_ERR_WORKSPACE, "indexer needs %zu workspace bytes (got %zu)", need, ws_bytes);
+    return indexer_scan_select(reinterpret_cast<const uint8_t*>(q_idx), w,
+                               reinterpret_cast<const uint8_t*>(k_idx), pos, k_base, T, S, H_I, d_I,
+                               k, idx, workspace, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int dsa_sparse_mla_attn(const void* q, const void* kv, const int32_t* idx, const int32_t* pos,
+                        const int32_t* k_base, int T, int S, int Hq, int d_qk, int d_v, int k,
+                        float scale, void* out, float* lse, void* workspace, size_t ws_bytes,
+                        void* stream)
+{
+    g_err[0] = 0;
+    if (int rc = check_attn(q, kv, idx, pos, k_base, T, S, Hq, d_qk, d_v, k, out, lse)) return rc;
+    const size_t need = attn_workspace(T, Hq, d_v, k);
+    if (need && (!workspace || ws_bytes < need || !al16(workspace)))
+        return fail(DSA_ERR_WORKSPACE, "attention needs %zu workspace bytes (got %zu)", need,
+                    ws_bytes);
+    return attn_simple(reinterpret_cast<const __nv_bfloat16*>(q),
+                       reinterpret_cast<const __nv_bfloat16*>(kv), idx, pos, k_base, T, S, Hq,
+                       d_qk, d_v, k, scale, reinterpret_cast<__nv_bfloat16*>(out), lse, workspace,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+int dsa_forward(const void* q_idx, const float* w, const void* k_idx, const void* q,
+                const void* kv, const int32_t* pos, const int32_t* k_base, int T, int S, int H_I,
+                int d_I, int Hq, int d_qk, int d_v, int k, float scale, int32_t* idx, void* out,
+                float* lse, void* workspace, size_t ws_bytes, void* stream)
+{
+    g_err[0] = 0;
+    if (int rc = check_indexer(q_idx, w, k_idx, pos, k_base, T, S, H_I, d_I, k, idx)) return rc;
+    if (int rc = check_attn(q, kv, idx, pos, k_base, T, S, Hq, d_qk, d_v, k, out, lse)) return rc;
+    if (int rc = dsa_indexer_topk(q_idx, w, k_idx, pos, k_base, T, S, H_I, d_I, k, idx, workspace,
+                                  ws_bytes, stream))
+        return rc;
+    return dsa_sparse_mla_attn(q, kv, idx, pos, k_base, T, S, Hq, d_qk, d_v, k, scale, out, lse,
+                               workspace, ws_bytes, stream);
+}
+
+int dsa_device_status(void* stream)
+{
+    cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    int v = 0;
+    e = cudaMemcpyFromSymbol(&v, dsa::g_status, sizeof v);
+    if (e != cudaSuccess) return cuda_fail(e, "read device status");
+    if (v != 0) {
+        const int zero = 0;
+        cudaMemcpyToSymbol(dsa::g_status, &zero, sizeof zero);
+        return fail(v, "a kernel reported status %d (bounded wait gave up)", v);
+    }
+    return DSA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,192 @@
+// Exact per-row Top-k selection ("Top-k selector on I_{t,s}", section 2 of
+// "Paper Breakdown: DeepSeek-V3.2") over scores that are already in memory.
+//
+// One CTA per row. The k-th largest score is found by an MSD radix select on
+// the order-preserving 32-bit key of the fp32 score (four 8-bit digits, one
+// pass over the row each, per-warp shared-memory histograms). Equal scores are
+// broken towards the lower index: if more entries tie at the k-th score than
+// slots are left, a second radix select over the candidates' indices finds the
+// cut. The emitted set is therefore the unique Top-k under (score desc, s asc).
+#pragma once
+#include "common.cuh"
+
+namespace dsa {
+
+template <int THREADS>
+struct SelectSmem {
+    uint32_t hist[THREADS / 32][256];
+    uint32_t total[256];
+    int misc[4];
+    int counter[2];
+};
+
+// Scores stored densely: entry i is candidate s = i.
+struct DenseScores {
+    const float* p;
+    __device__ __forceinline__ uint32_t key(int i) const { return score_key(p[i]); }
+    __device__ __forceinline__ int s(int i) const { return i; }
+};
+
+// Candidates stored as (fp32 score bits, s) pairs.
+struct PairScores {
+    const uint2* p;
+    __device__ __forceinline__ uint32_t key(int i) const { return score_key(__uint_as_float(p[i].x)); }
+    __device__ __forceinline__ int s(int i) const { return (int)p[i].y; }
+};
+
+// Merge the per-warp histograms into total[], then find the digit whose bin
+// holds the need-th entry counted from the top (descending) or from the
+// bottom (ascending). Results: misc[0] = digit, misc[1] = rank inside the bin
+// (1-based), misc[2] = entries in the bin.
+template <int THREADS>
+__device__ __forceinline__ void select_digit(SelectSmem<THREADS>& sm, int need, bool descending)
+{
+    constexpr int W = THREADS / 32;
+    for (int b = threadIdx.x; b < 256; b += THREADS) {
+        uint32_t s = 0;
+#pragma unroll 8
+        for (int w = 0; w < W; ++w) s += sm.hist[w][b];
+        sm.total[b] = s;
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        // lane owns 8 bins; in the descending case lane 0 owns the top bins
+        uint32_t c[8];
+        uint32_t local = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int b = descending ? 255 - (lane * 8 + j) : lane * 8 + j;
+            c[j] = sm.total[b];
+            local += c[j];
+        }
+        uint32_t incl = local;  // inclusive prefix over lanes 0..lane
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const uint32_t v = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += v;
+        }
+        const uint32_t before = incl - local;
+        if (before < (uint32_t)need && incl >= (uint32_t)need) {
+            uint32_t cum = before;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                if (cum + c[j] >= (uint32_t)need) {
+                    sm.misc[0] = descending ? 255 - (lane * 8 + j) : lane * 8 + j;
+                    sm.misc[1] = need - (int)cum;
+                    sm.misc[2] = (int)c[j];
+                    break;
+                }
+                cum += c[j];
+            }
+        }
+    }
+    __syncthreads();
+}
+
+template <int THREADS>
+__device__ __forceinline__ void clear_hist(SelectSmem<THREADS>& sm)
+{
+    uint32_t* h = &sm.hist[0][0];
+    for (int i = threadIdx.x; i < (THREADS / 32) * 256; i += THREADS) h[i] = 0u;
+    __syncthreads();
+}
+
+// Returns the key of the k-th largest entry; *take_eq = entries equal to it
+// that belong to the Top-k, *count_eq = entries equal to it. Requires n > k.
+template <int THREADS, class Row>
+__device__ uint32_t radix_kth_key(const Row& row, int n, int k, SelectSmem<THREADS>& sm,
+                                  int* take_eq, int* count_eq)
+{
+    const int warp = threadIdx.x >> 5;
+    uint32_t prefix = 0u, mask = 0u;
+    int need = k, cnt = 0;
+#pragma unroll 1
+    for (int shift = 24; shift >= 0; shift -= 8) {
+        clear_hist(sm);
+        for (int i = threadIdx.x; i < n; i += THREADS) {
+            const uint32_t key = row.key(i);
+            if ((key & mask) == prefix) atomicAdd(&sm.hist[warp][(key >> shift) & 255u], 1u);
+        }
+        __syncthreads();
+        select_digit(sm, need, true);
+        prefix |= (uint32_t)sm.misc[0] << shift;
+        mask |= 255u << shift;
+        need = sm.misc[1];
+        cnt = sm.misc[2];
+        __syncthreads();
+    }
+    *take_eq = need;
+    *count_eq = cnt;
+    return prefix;
+}
+
+// Writes the Top-k of `row` (n entries) to out[0..k): the entries above the
+// k-th key in any order, then the lowest-index entries equal to it.
+template <int THREADS, class Row>
+__device__ void block_topk(const Row& row, int n, int k, int32_t* __restrict__ out,
+                           SelectSmem<THREADS>& sm)
+{
+    if (n <= k) {
+        for (int i = threadIdx.x; i < k; i += THREADS) out[i] = i < n ? row.s(i) : -1;
+        return;
+    }
+    int take_eq, count_eq;
+    const uint32_t kth = radix_kth_key<THREADS>(row, n, k, sm, &take_eq, &count_eq);
+    const int warp = threadIdx.x >> 5;
+    // Index cut among the ties: the take_eq-th smallest s with key == kth.
+    uint32_t s_cut = 0xFFFFFFFFu;
+    if (count_eq > take_eq) {
+        uint32_t prefix = 0u, mask = 0u;
+        int need = take_eq;
+#pragma unroll 1
+        for (int shift = 24; shift >= 0; shift -= 8) {
+            clear_hist(sm);
+            for (int i = threadIdx.x; i < n; i += THREADS) {
+                if (row.key(i) != kth) continue;
+                const uint32_t s = (uint32_t)row.s(i);
+                if ((s & mask) == prefix) atomicAdd(&sm.hist[warp][(s >> shift) & 255u], 1u);
+            }
+            __syncthreads();
+            select_digit(sm, need, false);
+            prefix |= (uint32_t)sm.misc[0] << shift;
+            mask |= 255u << shift;
+            need = sm.misc[1];
+            __syncthreads();
+        }
+        s_cut = prefix;
+    }
+    if (threadIdx.x == 0) {
+        sm.counter[0] = 0;
+        sm.counter[1] = 0;
+    }
+    __syncthreads();
+    const int n_gt = k - take_eq;
+    for (int i = threadIdx.x; i < n; i += THREADS) {
+        const uint32_t key = row.key(i);
+        if (key > kth) {
+            out[atomicAdd(&sm.counter[0], 1)] = row.s(i);
+        } else if (key == kth) {
+            const int s = row.s(i);
+            if ((uint32_t)s <= s_cut) out[n_gt + atomicAdd(&sm.counter[1], 1)] = s;
+        }
+    }
+}
+
+constexpr int kSelectThreads = 1024;
+
+// One CTA per query row t = row0 + blockIdx.x; its scores are row blockIdx.x
+// of `scores` (dense, s = 0..pos[t]).
+template <int THREADS>
+__global__ void __launch_bounds__(THREADS)
+topk_dense_rows_kernel(const float* __restrict__ scores, long long ld, const int* __restrict__ pos,
+                       int T, int S, int row0, int k, int32_t* __restrict__ idx)
+{
+    __shared__ SelectSmem<THREADS> sm;
+    const int t = row0 + blockIdx.x;
+    const int n = (pos ? pos[t] : t + S - T) + 1;
+    DenseScores row{scores + (size_t)blockIdx.x * ld};
+    block_topk<THREADS>(row, n, k, idx + (size_t)t * k, sm);
+}
+
+}  // namespace dsa

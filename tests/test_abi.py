@@ -1,0 +1,119 @@
+"""Host-side checks of the C-ABI library (no GPU): it builds for sm_100a, loads,
+exports every symbol include/dsa.h declares, sizes workspaces, and rejects bad
+arguments before launching anything."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from conftest import ROOT
+
+import sparse_attention_20_b200 as dsa
+from sparse_attention_20_b200 import build as dsa_build
+
+HEADER = os.path.join(ROOT, "include", "dsa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    dsa_build.build()
+    return dsa.load_library()
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(dsa_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_exports():
+    assert _declared() == sorted(dsa.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", dsa.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\s[TW]\s+(\w+)$", out, flags=re.M))
+    for name in _declared():
+        assert name in exported, name
+        assert hasattr(lib, name)
+
+
+def test_build_targets_sm100a():
+    flags = " ".join(dsa_build.NVCC_FLAGS)
+    assert "arch=compute_100a,code=sm_100a" in flags
+
+
+def test_abi_version_and_empty_error(lib):
+    assert lib.dsa_abi_version() == 1
+    assert isinstance(lib.dsa_last_error(), bytes)
+
+
+def test_workspace_sizes(lib):
+    # 128K prefill: score blocks of <= 1 GiB
+    ws = dsa.workspace_size(131072, 131072, 8, 128, 2048, 128, 576, 512)
+    assert 0 < ws <= (1 << 30) + 4096
+    assert dsa.workspace_size(0, 10, 8, 128, 2048, 128, 576, 512) == 0
+    small = dsa.workspace_size(256, 256, 4, 32, 32, 4, 80, 64)
+    assert small >= 256 * 256 * 4
+
+
+FAKE = ctypes.c_void_p(0x10000)          # aligned, never dereferenced: checks fail first
+ODD = ctypes.c_void_p(0x10004)
+
+
+def test_indexer_rejects_bad_arguments(lib):
+    f = lib.dsa_indexer_topk
+    ws = ctypes.c_size_t(1 << 20)
+    # NULL pointer
+    assert f(None, FAKE, FAKE, None, None, 4, 4, 8, 128, 2, FAKE, FAKE, ws, None) == -1
+    assert b"NULL" in lib.dsa_last_error()
+    # misaligned
+    assert f(ODD, FAKE, FAKE, None, None, 4, 4, 8, 128, 2, FAKE, FAKE, ws, None) == -1
+    # sizes
+    assert f(FAKE, FAKE, FAKE, None, None, 0, 4, 8, 128, 2, FAKE, FAKE, ws, None) == -1
+    assert f(FAKE, FAKE, FAKE, None, None, 8, 4, 8, 128, 2, FAKE, FAKE, ws, None) == -1  # T > S
+    # unsupported dims
+    assert f(FAKE, FAKE, FAKE, None, None, 4, 4, 17, 128, 2, FAKE, FAKE, ws, None) == -2
+    assert f(FAKE, FAKE, FAKE, None, None, 4, 4, 8, 96, 2, FAKE, FAKE, ws, None) == -2
+    assert f(FAKE, FAKE, FAKE, None, None, 4, 4, 8, 128, 4097, FAKE, FAKE, ws, None) == -2
+    # workspace too small
+    assert f(FAKE, FAKE, FAKE, None, None, 4, 4, 8, 128, 2, FAKE, FAKE, ctypes.c_size_t(8),
+             None) == -5
+
+
+def test_attention_rejects_bad_arguments(lib):
+    f = lib.dsa_sparse_mla_attn
+    ws = ctypes.c_size_t(1 << 20)
+    sc = ctypes.c_float(0.1)
+    assert f(FAKE, None, FAKE, None, None, 4, 4, 128, 576, 512, 64, sc, FAKE, FAKE, FAKE, ws,
+             None) == -1
+    assert f(FAKE, FAKE, FAKE, None, None, 4, 4, 128, 570, 512, 64, sc, FAKE, FAKE, FAKE, ws,
+             None) == -2
+    assert f(FAKE, FAKE, FAKE, None, None, 4, 4, 128, 576, 577, 64, sc, FAKE, FAKE, FAKE, ws,
+             None) == -2
+    assert f(FAKE, FAKE, FAKE, None, None, 4, 4, 2000, 576, 512, 64, sc, FAKE, FAKE, FAKE, ws,
+             None) == -2
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    x = torch.zeros((4, 8, 128), dtype=torch.uint8)
+    with pytest.raises(ValueError):
+        dsa.indexer_topk(x, torch.zeros(4, 8), torch.zeros((4, 128), dtype=torch.uint8), 2)
+
+
+def test_product_and_oracle_share_no_code():
+    pkg = os.path.join(ROOT, "sparse_attention_20_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for fn in files:
+            if fn.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, fn)).read()
+                assert "oracle" not in text.lower(), fn
+    for fn in os.listdir(os.path.join(ROOT, "oracle")):
+        if fn.endswith((".py", ".c", ".h")):
+            text = open(os.path.join(ROOT, "oracle", fn)).read()
+            assert "import sparse_attention_20_b200" not in text
+            assert "dsa.h" not in text

@@ -1,0 +1,198 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle on B200.
+
+Sizes: small cases run the oracle on every row (several tiles, ragged tails);
+the full-size workloads (32K, 128K prefill, 64-sequence decode) check sampled
+rows in the exact launch configuration bench.py times.
+"""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+import sparse_attention_20_b200 as dsa
+from sparse_attention_20_b200 import build as dsa_build
+from parity import check_attention, check_indexer, host_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    dsa_build.build()
+    dsa.load_library()
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    yield
+    torch.cuda.synchronize()
+    assert dsa.device_status() == 0
+
+
+def _run(x, **kw):
+    idx, out, lse = dsa.forward(x.q_idx, x.w, x.k_idx, x.q, x.kv, x.k, x.scale, x.d_v, pos=x.pos,
+                                k_base=x.k_base, **kw)
+    torch.cuda.synchronize()
+    return idx, out, lse
+
+
+def _take(t, rows):
+    return t[torch.tensor(rows, device=t.device)].cpu()
+
+
+# ----------------------------------------------------------- small, full check
+
+def test_tiny_indexer_bit_exact_and_attention_all_rows():
+    x = synth.prefill_inputs("tiny", device="cuda", seed=0)
+    idx, out, lse = _run(x)
+    rows = list(range(x.T))
+    h = host_inputs(x, rows)
+    check_indexer(x, idx.cpu(), rows, exact=True, h=h)
+    check_attention(x, idx.cpu(), out.cpu(), lse.cpu(), rows, h=h)
+
+
+def test_forward_equals_separate_calls():
+    x = synth.prefill_inputs("tiny", device="cuda", seed=1)
+    idx, out, lse = _run(x)
+    idx2 = dsa.indexer_topk(x.q_idx, x.w, x.k_idx, x.k, pos=x.pos, k_base=x.k_base)
+    out2, lse2 = dsa.sparse_mla_attn(x.q, x.kv, idx2, x.scale, x.d_v, pos=x.pos, k_base=x.k_base)
+    torch.cuda.synchronize()
+    assert torch.equal(torch.sort(idx, 1)[0], torch.sort(idx2, 1)[0])
+    assert torch.equal(out, out2) and torch.equal(lse, lse2)
+
+
+@pytest.mark.parametrize("L,k", [(333, 64), (130, 200)])
+def test_small_realistic_all_rows(L, k):
+    x = synth.prefill_inputs("prefill4k", device="cuda", seed=2, L=L, overrides=dict(k=k))
+    idx, out, lse = _run(x)
+    rows = list(range(x.T))
+    h = host_inputs(x, rows)
+    check_indexer(x, idx.cpu(), rows, exact=False, h=h)
+    check_attention(x, idx.cpu(), out.cpu(), lse.cpu(), rows, h=h)
+
+
+def test_integer_indexer_bit_exact_d128():
+    x = synth.prefill_inputs("prefill32k_int", device="cuda", seed=3, L=1500,
+                             overrides=dict(k=300))
+    idx = dsa.indexer_topk(x.q_idx, x.w, x.k_idx, x.k)
+    torch.cuda.synchronize()
+    rows = list(range(0, x.T, 3)) + [x.T - 1]
+    check_indexer(x, _take(idx, rows), rows, exact=True)
+
+
+def test_explicit_pos_and_k_base_packed_rows():
+    """Queries of three sequences in one packed cache, with ragged lengths."""
+    x = synth.decode_inputs("decode", device="cuda", seed=4, B=5, ctx=[1, 17, 300, 129, 2050],
+                            overrides=dict(k=128))
+    idx, out, lse = _run(x)
+    rows = list(range(x.T))
+    h = host_inputs(x, rows)
+    check_indexer(x, idx.cpu(), rows, exact=False, h=h)
+    check_attention(x, idx.cpu(), out.cpu(), lse.cpu(), rows, h=h)
+
+
+def test_decode_integer_inputs_bit_exact():
+    x = synth.decode_inputs("decode", device="cuda", seed=5, B=6, ctx=[40, 1000, 3000, 64, 65, 5000],
+                            overrides=dict(indexer="int", k=256))
+    idx = dsa.indexer_topk(x.q_idx, x.w, x.k_idx, x.k, pos=x.pos, k_base=x.k_base)
+    torch.cuda.synchronize()
+    check_indexer(x, idx.cpu(), list(range(x.T)), exact=True)
+
+
+def test_k_at_least_L_selects_every_past_token():
+    x = synth.prefill_inputs("tiny", device="cuda", seed=6, L=100, overrides=dict(k=128))
+    idx, out, lse = _run(x)
+    for t in range(x.T):
+        row = idx[t].cpu().numpy()
+        assert sorted(row[: t + 1].tolist()) == list(range(t + 1))
+        assert (row[t + 1:] == -1).all()
+    check_attention(x, idx.cpu(), out.cpu(), lse.cpu(), list(range(x.T)))
+
+
+def test_k_equals_one_and_single_row():
+    x = synth.prefill_inputs("tiny", device="cuda", seed=7, overrides=dict(k=1))
+    pos = torch.tensor([200], dtype=torch.int32, device="cuda")
+    idx = dsa.indexer_topk(x.q_idx[200:201].contiguous(), x.w[200:201].contiguous(), x.k_idx, 1,
+                           pos=pos)
+    torch.cuda.synchronize()
+    full = dsa.indexer_topk(x.q_idx, x.w, x.k_idx, 1)
+    torch.cuda.synchronize()
+    assert idx[0, 0].item() == full[200, 0].item()
+    check_indexer(x, full.cpu(), list(range(x.T)), exact=True)
+
+
+def test_attention_splits_and_lse_merge(monkeypatch):
+    x = synth.prefill_inputs("prefill4k", device="cuda", seed=8, L=96, overrides=dict(k=80))
+    idx = dsa.indexer_topk(x.q_idx, x.w, x.k_idx, x.k)
+    out1, lse1 = dsa.sparse_mla_attn(x.q, x.kv, idx, x.scale, x.d_v)
+    monkeypatch.setenv("DSA_ATTN_SPLITS", "5")
+    out5, lse5 = dsa.sparse_mla_attn(x.q, x.kv, idx, x.scale, x.d_v)
+    torch.cuda.synchronize()
+    rows = list(range(x.T))
+    check_attention(x, idx.cpu(), out5.cpu(), lse5.cpu(), rows)
+    assert (out1.float() - out5.float()).abs().max().item() < 2e-2
+
+
+def test_invalid_entries_are_ignored():
+    """-1 padding and s > pos inside the read range do not contribute."""
+    x = synth.prefill_inputs("tiny", device="cuda", seed=9)
+    t = 100
+    idx = torch.full((x.T, x.k), -1, dtype=torch.int32, device="cuda")
+    idx[t, :4] = torch.tensor([5, 250, 7, -1], dtype=torch.int32)
+    out, lse = dsa.sparse_mla_attn(x.q, x.kv, idx, x.scale, x.d_v)
+    torch.cuda.synchronize()
+    ref_idx = torch.full_like(idx, -1)
+    ref_idx[t, :2] = torch.tensor([5, 7], dtype=torch.int32)
+    check_attention(x, ref_idx[[t]].cpu(), out[[t]].cpu(), lse[[t]].cpu(), [t])
+
+
+# ----------------------------------------------------- full-size workloads
+
+def _sampled(T, k, n):
+    return synth.sample_rows(T, k, n, seed=0)
+
+
+def test_prefill4k_all_rows_indexer_sampled_attention():
+    x = synth.prefill_inputs("prefill4k", device="cuda", seed=0)
+    idx, out, lse = _run(x)
+    rows = list(range(x.T))
+    check_indexer(x, idx.cpu(), rows, exact=False)
+    srows = _sampled(x.T, x.k, 48)
+    check_attention(x, _take(idx, srows), _take(out, srows), _take(lse, srows), srows)
+
+
+def test_prefill32k_integer_indexer_bit_exact_sampled():
+    x = synth.prefill_inputs("prefill32k_int", device="cuda", seed=0)
+    idx, out, lse = _run(x)
+    rows = _sampled(x.T, x.k, 160)
+    check_indexer(x, _take(idx, rows), rows, exact=True)
+    srows = rows[:: max(1, len(rows) // 12)]
+    check_attention(x, _take(idx, srows), _take(out, srows), _take(lse, srows), srows)
+
+
+def test_prefill32k_sampled():
+    x = synth.prefill_inputs("prefill32k", device="cuda", seed=0)
+    idx, out, lse = _run(x)
+    rows = _sampled(x.T, x.k, 48)
+    check_indexer(x, _take(idx, rows), rows, exact=False)
+    srows = rows[:: max(1, len(rows) // 12)]
+    check_attention(x, _take(idx, srows), _take(out, srows), _take(lse, srows), srows)
+
+
+def test_prefill128k_sampled():
+    x = synth.prefill_inputs("prefill128k", device="cuda", seed=0)
+    idx, out, lse = _run(x)
+    rows = _sampled(x.T, x.k, 24)
+    check_indexer(x, _take(idx, rows), rows, exact=False)
+    srows = rows[:: max(1, len(rows) // 8)]
+    check_attention(x, _take(idx, srows), _take(out, srows), _take(lse, srows), srows)
+    del x, idx, out, lse
+    torch.cuda.empty_cache()
+
+
+def test_decode_64_sequences():
+    x = synth.decode_inputs("decode", device="cuda", seed=0)
+    idx, out, lse = _run(x)
+    rows = list(range(x.T))
+    check_indexer(x, idx.cpu(), rows, exact=False)
+    srows = rows[::4]
+    check_attention(x, _take(idx, srows), _take(out, srows), _take(lse, srows), srows)
