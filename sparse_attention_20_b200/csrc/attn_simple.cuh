@@ -47,9 +47,10 @@ sparse_attn_simple_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat
     const int h0 = blockIdx.y * kAttnHeads;
     const int split = blockIdx.z, splits = gridDim.z;
     const int nh = min(kAttnHeads, Hq - h0);
-    const int p = pos ? pos[t] : t + S - T;
-    const long long base = k_base ? k_base[t] : 0;
-    const int n_row = min(k, p + 1);
+    long long base;
+    const int n_cand = row_candidates(pos, k_base, t, T, S, &base);
+    const int p = n_cand - 1;   // last valid s
+    const int n_row = min(k, n_cand);
     const int per = ceil_div(n_row, splits);
     const int i0 = min(n_row, split * per), i1 = min(n_row, i0 + per);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;

@@ -50,4 +50,17 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 
 __host__ __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
+// Candidate range of query row t: s = 0..n-1 at cache rows base + s. Rows that
+// would reach outside the cache (a caller error) are clipped to it, so no
+// kernel ever reads out of bounds.
+__device__ __forceinline__ int row_candidates(const int* pos, const int* k_base, int t, int T,
+                                              int S, long long* base_out)
+{
+    const long long base = k_base ? k_base[t] : 0;
+    const long long p = pos ? pos[t] : (long long)t + S - T;
+    *base_out = base;
+    if (base < 0 || base >= S || p < 0) return 0;
+    return (int)min(p + 1, (long long)S - base);
+}
+
 }  // namespace dsa

@@ -182,7 +182,7 @@ int indexer_scan_select(const uint8_t* q_idx, const float* w, const uint8_t* k_i
         scores_fn(grid, st, q_idx, w, k_idx, pos, k_base, T, S, H_I, row0, scores, ld, kKeysPerCta);
         DSA_LAUNCH_CHECK("indexer_scores_kernel");
         dsa::topk_dense_rows_kernel<dsa::kSelectThreads>
-            <<<rb, dsa::kSelectThreads, 0, st>>>(scores, ld, pos, T, S, row0, k, idx);
+            <<<rb, dsa::kSelectThreads, 0, st>>>(scores, ld, pos, k_base, T, S, row0, k, idx);
         DSA_LAUNCH_CHECK("topk_dense_rows_kernel");
     }
     return DSA_OK;

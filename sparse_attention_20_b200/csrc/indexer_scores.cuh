@@ -68,8 +68,8 @@ indexer_scores_kernel(const uint8_t* __restrict__ q_idx, const float* __restrict
     constexpr int KSTEPS = DI / 32;
     const int r = blockIdx.y;
     const int t = row0 + r;
-    const int n = (pos ? pos[t] : t + S - T) + 1;
-    const long long base = k_base ? k_base[t] : 0;
+    long long base;
+    const int n = row_candidates(pos, k_base, t, T, S, &base);
     const int s_begin = blockIdx.x * keys_per_cta;
     if (s_begin >= n) return;
     const int s_end = min(n, s_begin + keys_per_cta);

@@ -165,10 +165,14 @@ __device__ void block_topk(const Row& row, int n, int k, int32_t* __restrict__ o
     for (int i = threadIdx.x; i < n; i += THREADS) {
         const uint32_t key = row.key(i);
         if (key > kth) {
-            out[atomicAdd(&sm.counter[0], 1)] = row.s(i);
+            const int slot = atomicAdd(&sm.counter[0], 1);
+            if (slot < n_gt) out[slot] = row.s(i);
         } else if (key == kth) {
             const int s = row.s(i);
-            if ((uint32_t)s <= s_cut) out[n_gt + atomicAdd(&sm.counter[1], 1)] = s;
+            if ((uint32_t)s <= s_cut) {
+                const int slot = atomicAdd(&sm.counter[1], 1);
+                if (slot < take_eq) out[n_gt + slot] = s;
+            }
         }
     }
 }
@@ -180,11 +184,13 @@ constexpr int kSelectThreads = 1024;
 template <int THREADS>
 __global__ void __launch_bounds__(THREADS)
 topk_dense_rows_kernel(const float* __restrict__ scores, long long ld, const int* __restrict__ pos,
-                       int T, int S, int row0, int k, int32_t* __restrict__ idx)
+                       const int* __restrict__ k_base, int T, int S, int row0, int k,
+                       int32_t* __restrict__ idx)
 {
     __shared__ SelectSmem<THREADS> sm;
     const int t = row0 + blockIdx.x;
-    const int n = (pos ? pos[t] : t + S - T) + 1;
+    long long base;
+    const int n = row_candidates(pos, k_base, t, T, S, &base);
     DenseScores row{scores + (size_t)blockIdx.x * ld};
     block_topk<THREADS>(row, n, k, idx + (size_t)t * k, sm);
 }
