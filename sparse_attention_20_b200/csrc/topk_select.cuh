@@ -121,8 +121,8 @@ __device__ uint32_t radix_kth_key(const Row& row, int n, int k, SelectSmem<THREA
     return prefix;
 }
 
-// Writes the Top-k of `row` (n entries) to out[0..k): the entries above the
-// k-th key in any order, then the lowest-index entries equal to it.
+// Writes the Top-k of `row` (n entries) to out[0..k) in storage order (for
+// dense rows: ascending s), so the result is deterministic.
 template <int THREADS, class Row>
 __device__ void block_topk(const Row& row, int n, int k, int32_t* __restrict__ out,
                            SelectSmem<THREADS>& sm)
@@ -156,24 +156,33 @@ __device__ void block_topk(const Row& row, int n, int k, int32_t* __restrict__ o
         }
         s_cut = prefix;
     }
-    if (threadIdx.x == 0) {
-        sm.counter[0] = 0;
-        sm.counter[1] = 0;
-    }
+    // Emit in storage order (ascending s for dense rows): ordered compaction.
+    if (threadIdx.x == 0) sm.counter[0] = 0;
     __syncthreads();
-    const int n_gt = k - take_eq;
-    for (int i = threadIdx.x; i < n; i += THREADS) {
-        const uint32_t key = row.key(i);
-        if (key > kth) {
-            const int slot = atomicAdd(&sm.counter[0], 1);
-            if (slot < n_gt) out[slot] = row.s(i);
-        } else if (key == kth) {
-            const int s = row.s(i);
-            if ((uint32_t)s <= s_cut) {
-                const int slot = atomicAdd(&sm.counter[1], 1);
-                if (slot < take_eq) out[n_gt + slot] = s;
-            }
+    const int lane = threadIdx.x & 31;
+    for (int c0 = 0; c0 < n; c0 += THREADS) {
+        const int i = c0 + threadIdx.x;
+        bool take = false;
+        int s = 0;
+        if (i < n) {
+            const uint32_t key = row.key(i);
+            s = row.s(i);
+            take = key > kth || (key == kth && (uint32_t)s <= s_cut);
         }
+        const unsigned m = __ballot_sync(0xffffffffu, take);
+        if (lane == 0) sm.hist[0][warp] = __popc(m);
+        __syncthreads();
+        int off = sm.counter[0];
+        for (int w = 0; w < warp; ++w) off += (int)sm.hist[0][w];
+        const int slot = off + __popc(m & ((1u << lane) - 1u));
+        if (take && slot < k) out[slot] = s;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            int tot = 0;
+            for (int w = 0; w < THREADS / 32; ++w) tot += (int)sm.hist[0][w];
+            sm.counter[0] += tot;
+        }
+        __syncthreads();
     }
 }
 
