@@ -115,6 +115,28 @@ int dsa_forward(const void* q_idx, const float* w, const void* k_idx, const void
                 float* lse, void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * dsa_indexer_topk without a workspace argument. The paper has no
+ * counterpart: this entry point exists for callers that cannot give the
+ * library device memory -- code that must not call cudaMalloc (whose implicit
+ * device synchronisation can stall other work, or which a host framework's
+ * memory pool forbids) and has no spare buffer of its own to lend.
+ *
+ * Same arguments, result and limits as dsa_indexer_topk, minus the workspace;
+ * it allocates nothing. Its scratch is a 16 MiB array (4,194,304 fp32 scores)
+ * that the library holds in the device memory of every GPU it is loaded on,
+ * until the process exits. Calls with S > 4,194,304 are rejected with
+ * DSA_ERR_UNSUPPORTED before any launch. The first call on a device looks up
+ * the array's device address for that device; make that first call before
+ * any stream capture. Every call on a device shares the one array, so calls
+ * whose kernels overlap on the GPU (two streams, two host threads) race and
+ * must be serialised by the caller; nothing in the array has to start at
+ * zero, and it keeps whatever the last call wrote.
+ */
+int dsa_indexer_topk_noalloc(const void* q_idx, const float* w, const void* k_idx,
+                             const int32_t* pos, const int32_t* k_base, int T, int S, int H_I,
+                             int d_I, int k, int32_t* idx, void* stream);
+
+/*
  * Waits for `stream`, then returns and clears the device status word:
  * DSA_OK, DSA_ERR_TIMEOUT (a kernel gave up a bounded wait) or DSA_ERR_CUDA
  * (an asynchronous CUDA error; its text is in dsa_last_error()).

@@ -30,7 +30,8 @@ STATUS_NAMES = {0: "DSA_OK", -1: "DSA_ERR_ARG", -2: "DSA_ERR_UNSUPPORTED", -3: "
 
 # Every symbol include/dsa.h declares.
 EXPORTS = ("dsa_workspace_size", "dsa_indexer_topk", "dsa_sparse_mla_attn", "dsa_forward",
-           "dsa_device_status", "dsa_last_error", "dsa_abi_version", "dsa_launch_count")
+           "dsa_device_status", "dsa_last_error", "dsa_abi_version", "dsa_launch_count",
+           "dsa_indexer_topk_noalloc")
 
 
 class DSAError(RuntimeError):
@@ -65,6 +66,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.dsa_last_error.restype = ctypes.c_char_p
         lib.dsa_abi_version.restype = I
         lib.dsa_launch_count.restype = ctypes.c_uint64
+        lib.dsa_indexer_topk_noalloc.argtypes = [P, P, P, P, P, I, I, I, I, I, P, P]
+        lib.dsa_indexer_topk_noalloc.restype = I
         _lib = lib
     return _lib
 

@@ -9,6 +9,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 
 #include "dsa.h"
 #include "attn_simple.cuh"
@@ -303,3 +304,75 @@ int dsa_device_status(void* stream)
 }
 
 }  // extern "C"
+
+// ============================================== indexer with library-held scratch
+//
+// dsa_indexer_topk_noalloc runs the same two kernels as dsa_indexer_topk, but
+// its score scratch is a fixed array that the library itself holds in device
+// memory, so the caller passes no workspace and nothing is allocated per call.
+
+namespace {
+
+// 4,194,304 fp32 scores = 16 MiB. Every GPU on which the library is loaded
+// holds this array until the process exits.
+constexpr size_t kStaticScoreFloats = size_t(4) << 20;
+static __device__ __align__(256) float g_static_scores[kStaticScoreFloats];
+
+// In host code `g_static_scores` only names a host-side stand-in for the
+// array, not a device address; kernels get the address that
+// cudaGetSymbolAddress returns, looked up once per device with that device
+// current.
+constexpr int kMaxDevices = 64;
+std::mutex g_static_mu;
+float* g_static_ptr[kMaxDevices] = {nullptr};
+
+int static_scores_on_current_device(float** out)
+{
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return fail(DSA_ERR_UNSUPPORTED, "device %d", dev);
+    std::lock_guard<std::mutex> lock(g_static_mu);
+    if (!g_static_ptr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_static_scores);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(g_static_scores)");
+        g_static_ptr[dev] = reinterpret_cast<float*>(p);
+    }
+    *out = g_static_ptr[dev];
+    return DSA_OK;
+}
+
+}  // namespace
+
+extern "C" int dsa_indexer_topk_noalloc(const void* q_idx, const float* w, const void* k_idx,
+                                        const int32_t* pos, const int32_t* k_base, int T, int S,
+                                        int H_I, int d_I, int k, int32_t* idx, void* stream)
+{
+    g_err[0] = 0;
+    if (int rc = check_indexer(q_idx, w, k_idx, pos, k_base, T, S, H_I, d_I, k, idx)) return rc;
+    if ((size_t)S > kStaticScoreFloats)
+        return fail(DSA_ERR_UNSUPPORTED,
+                    "S=%d: the library-held scratch takes at most %zu candidate keys", S,
+                    kStaticScoreFloats);
+    float* scores = nullptr;
+    if (int rc = static_scores_on_current_device(&scores)) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int RB = (int)std::min<size_t>((size_t)T, kStaticScoreFloats / (size_t)S);
+    const long long ld = S;
+    constexpr int kKeysPerCta = 2048;
+    ScoresFn scores_fn = pick_scores(H_I, d_I);
+    const uint8_t* q8 = reinterpret_cast<const uint8_t*>(q_idx);
+    const uint8_t* k8 = reinterpret_cast<const uint8_t*>(k_idx);
+    for (int row0 = 0; row0 < T; row0 += RB) {
+        const int rb = std::min(RB, T - row0);
+        const int n_max = pos ? S : std::min(S, row0 + rb + S - T);
+        dim3 grid(dsa::ceil_div(n_max, kKeysPerCta), rb);
+        scores_fn(grid, st, q8, w, k8, pos, k_base, T, S, H_I, row0, scores, ld, kKeysPerCta);
+        DSA_LAUNCH_CHECK("indexer_scores_kernel");
+        dsa::topk_dense_rows_kernel<dsa::kSelectThreads>
+            <<<rb, dsa::kSelectThreads, 0, st>>>(scores, ld, pos, k_base, T, S, row0, k, idx);
+        DSA_LAUNCH_CHECK("topk_dense_rows_kernel");
+    }
+    return DSA_OK;
+}

@@ -1,0 +1,54 @@
+"""dsa_indexer_topk_noalloc: the indexer entry point for callers that cannot
+give the library device memory (no workspace argument; its scratch is an
+array the library holds). Called through the C ABI and compared with
+dsa_indexer_topk on the same inputs, twice in a row, because the shared
+scratch keeps the previous call's contents. Collected last on purpose."""
+import ctypes
+
+import pytest
+import torch
+
+import synth
+import sparse_attention_20_b200 as dsa
+from sparse_attention_20_b200 import build as dsa_build
+
+STATIC_MAX_S = 4 << 20
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def test_noalloc_rejects_S_beyond_its_scratch():
+    dsa_build.build()
+    lib = dsa.load_library()
+    fake = ctypes.c_void_p(0x10000)
+    rc = lib.dsa_indexer_topk_noalloc(fake, fake, fake, None, None, 4, STATIC_MAX_S + 1, 8, 128,
+                                      2048, fake, None)
+    assert rc == -2 and b"scratch" in lib.dsa_last_error()
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("case", ["decode", "prefill"])
+def test_noalloc_matches_workspace_entry_point_twice(case):
+    dsa_build.build()
+    lib = dsa.load_library()
+    if case == "decode":
+        x = synth.decode_inputs("decode", device="cuda", seed=21, B=12,
+                                ctx=[131072, 9000, 70000, 8192, 120001, 33333, 4096, 100000,
+                                     65536, 12345, 98765, 131071])
+    else:
+        x = synth.prefill_inputs("prefill4k", device="cuda", seed=22)
+    assert x.S <= STATIC_MAX_S
+    T, H_I, d_I = x.q_idx.shape
+    ref = dsa.indexer_topk(x.q_idx, x.w, x.k_idx, x.k, pos=x.pos, k_base=x.k_base)
+    torch.cuda.synchronize()
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    for _ in range(2):
+        got = torch.full_like(ref, -7)
+        rc = lib.dsa_indexer_topk_noalloc(_p(x.q_idx), _p(x.w), _p(x.k_idx), _p(x.pos),
+                                          _p(x.k_base), T, x.S, H_I, d_I, x.k, _p(got), stream)
+        assert rc == 0, lib.dsa_last_error()
+        torch.cuda.synchronize()
+        assert torch.equal(got, ref)
+    assert dsa.device_status() == 0
