@@ -13,6 +13,7 @@
 
 #include "dsa.h"
 #include "attn_simple.cuh"
+#include "attn_tc.cuh"
 #include "common.cuh"
 #include "indexer_scores.cuh"
 #include "topk_select.cuh"
@@ -221,6 +222,59 @@ int attn_simple(const __nv_bfloat16* q, const __nv_bfloat16* kv, const int32_t* 
     return DSA_OK;
 }
 
+// Tensor-core path: one 2-CTA cluster per query row (Hq=128, d_qk=576, d_v=512).
+bool attn_tc_supported(int Hq, int d_qk, int d_v, int k)
+{
+    if (const char* e = getenv("DSA_ATTN_IMPL"))
+        if (strcmp(e, "simple") == 0) return false;
+    if (getenv("DSA_ATTN_SPLITS")) return false;
+    return Hq == dsa::attn_tc::kHeads && d_qk == dsa::attn_tc::kDqk && d_v == dsa::attn_tc::kDv &&
+           k % 4 == 0;
+}
+
+// 2D bf16 tensor map over a row-major [rows, cols] matrix, box [box_rows, box_cols].
+int make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows,
+                   uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle sw)
+{
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * 2};
+    const cuuint32_t box[2] = {box_cols, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = cuTensorMapEncodeTiled(
+        m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+        CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return DSA_OK;
+}
+
+int attn_tc(const __nv_bfloat16* q, const __nv_bfloat16* kv, const int32_t* idx,
+            const int32_t* pos, const int32_t* k_base, int T, int S, int k, float scale,
+            __nv_bfloat16* out, float* lse, cudaStream_t st)
+{
+    using namespace dsa::attn_tc;
+    cudaError_t e = cudaFuncSetAttribute(sparse_mla_attn_tc_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(sparse_mla_attn_tc_kernel)");
+    // Q as [T*128, 576]: one 128-head box per slab; KV as [S, 576]: one-row
+    // boxes for tile::gather4. 64-column slabs use 128B swizzle, the 32-column
+    // rope slab 64B swizzle.
+    CUtensorMap tq128, tq64, tkv128, tkv64;
+    if (int rc = make_tmap_bf16(&tq128, q, kDqk, (uint64_t)T * kHeads, 64, kHeads,
+                                CU_TENSOR_MAP_SWIZZLE_128B)) return rc;
+    if (int rc = make_tmap_bf16(&tq64, q, kDqk, (uint64_t)T * kHeads, 32, kHeads,
+                                CU_TENSOR_MAP_SWIZZLE_64B)) return rc;
+    if (int rc = make_tmap_bf16(&tkv128, kv, kDqk, (uint64_t)S, 64, 1, CU_TENSOR_MAP_SWIZZLE_128B))
+        return rc;
+    if (int rc = make_tmap_bf16(&tkv64, kv, kDqk, (uint64_t)S, 32, 1, CU_TENSOR_MAP_SWIZZLE_64B))
+        return rc;
+    const float scale_log2 = scale * 1.4426950408889634f;
+    sparse_mla_attn_tc_kernel<<<dim3(2 * T), kThreads, kSmemBytes, st>>>(
+        tq128, tq64, tkv128, tkv64, idx, pos, k_base, T, S, k, scale_log2, out, lse);
+    DSA_LAUNCH_CHECK("sparse_mla_attn_tc_kernel");
+    return DSA_OK;
+}
+
 }  // namespace
 
 // ===================================================================== C ABI
@@ -263,6 +317,11 @@ int dsa_sparse_mla_attn(const void* q, const void* kv, const int32_t* idx, const
 {
     g_err[0] = 0;
     if (int rc = check_attn(q, kv, idx, pos, k_base, T, S, Hq, d_qk, d_v, k, out, lse)) return rc;
+    if (attn_tc_supported(Hq, d_qk, d_v, k))
+        return attn_tc(reinterpret_cast<const __nv_bfloat16*>(q),
+                       reinterpret_cast<const __nv_bfloat16*>(kv), idx, pos, k_base, T, S, k, scale,
+                       reinterpret_cast<__nv_bfloat16*>(out), lse,
+                       reinterpret_cast<cudaStream_t>(stream));
     const size_t need = attn_workspace(T, Hq, d_v, k);
     if (need && (!workspace || ws_bytes < need || !al16(workspace)))
         return fail(DSA_ERR_WORKSPACE, "attention needs %zu workspace bytes (got %zu)", need,
