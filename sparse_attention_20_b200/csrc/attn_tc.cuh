@@ -19,13 +19,15 @@
 // gathered rows read MN-major, N = 256). No flop is done twice and every
 // selected row crosses HBM/L2 once per query.
 //
-// Warp roles (256 threads per CTA): warp 0 allocates TMEM and issues MMAs
-// (one thread); warp 1 loads Q with TMA tiles and gathers the selected rows
-// with TMA tile::gather4 (four rows per instruction, 128B/64B swizzle applied
-// by the TMA unit) into a 3-stage ring of 64-row chunks; warps 4-7 (one thread
-// per head = TMEM lane) run the softmax, the exchange (st.async into the
-// peer's shared memory, counted on the peer's mbarrier) and the epilogue;
-// warps 2-3 only take part in set-up and tear-down.
+// Warp roles (416 threads per CTA): warp 0 allocates TMEM and issues the QK
+// MMAs (one thread); warp 12 issues the PV MMAs (one thread), so a late chunk
+// never holds back the PV of the previous one; warps 1-3 load Q (TMA tiles)
+// and gather the selected rows with 16-byte cp.async into 128B/64B-swizzled
+// shared memory (3-stage ring of 64-row chunks; completion is counted on the
+// stage's mbarrier, so the gather runs up to three chunks ahead); warps 4-11
+// (two per TMEM lane quarter, each taking 32 of a chunk's 64 keys) run the
+// softmax, the exchange (st.async into the peer's shared memory, counted on
+// the peer's mbarrier) and the epilogue.
 // Shared memory per CTA: Q slice 72 KB + 3 x 36 KB ring + 2 x 16 KB exchange.
 // TMEM: O cols [0,256), S double buffer [256,384), P (bf16 pairs) [384,448).
 #pragma once
@@ -43,7 +45,8 @@ constexpr int kDqk = 576;
 constexpr int kDv = 512;
 constexpr int kKeys = 64;
 constexpr int kStages = 3;
-constexpr int kThreads = 256;
+constexpr int kThreads = 416;               // 13 warps: QK, 3 gather, 8 softmax, PV
+constexpr int kGatherThreads = 96;
 
 constexpr int kQSlab = kHeads * 128;        // 64 columns x 128 rows, 128B swizzle
 constexpr int kQBytes = 4 * kQSlab + kHeads * 64;
@@ -55,14 +58,17 @@ constexpr int kOffKV = kOffQ + kQBytes;
 constexpr int kOffX = kOffKV + kStages * kStageBytes;
 constexpr int kOffBar = kOffX + 2 * kXBytes;
 constexpr int kOffMask = kOffBar + 256;                 // [kStages][2] validity bits
-constexpr int kSmemBytes = kOffMask + kStages * 8 + 1024;  // + 1 KB alignment slack
+constexpr int kOffRed = kOffMask + 64;                  // [2 parity][2 halves][128] row maxima
+constexpr int kOffLsum = kOffRed + 2 * 2 * kHeads * 4;  // [2 halves][128] row sums
+constexpr int kOffRows = kOffLsum + 2 * kHeads * 4;     // [3 gather warps][64] row byte offsets
+constexpr int kSmemBytes = kOffRows + 3 * kKeys * 8 + 1024;  // + 1 KB alignment slack
 
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 0, kColS = 256, kColP = 384;
 
 enum : int {
     B_Q = 0, B_FULL = 1, B_EMPTY = 4, B_SFULL = 7, B_SFREE = 9, B_PFULL = 11, B_PVDONE = 13,
-    B_XFULL = 15, B_XFREE = 17, B_DRAIN = 19, B_COUNT = 20
+    B_XFULL = 15, B_XFREE = 17, B_DRAIN = 19, B_RED = 20, B_LSUM = 22, B_COUNT = 23
 };
 
 static_assert(kOffKV % 1024 == 0 && kStageBytes % 1024 == 0 && kOffX % 1024 == 0, "alignment");
@@ -79,11 +85,25 @@ __device__ __forceinline__ float2 unpack_half2(uint32_t v)
     return __half22float2(h);
 }
 
+// Destination of 16-byte piece j (0..35) of gathered row r in a stage: pieces
+// 0..31 go to four 128B-swizzled slabs of 64 columns, 32..35 to one
+// 64B-swizzled slab of 32 columns (the layouts the MMA descriptors name).
+__device__ __forceinline__ uint32_t piece_dst(uint32_t stage, int r, int j)
+{
+    if (j < 32) return stage + (j >> 3) * kKSlab + r * 128 + (((j & 7) ^ (r & 7)) << 4);
+    return stage + 4 * kKSlab + r * 64 + (((j - 32) ^ ((r >> 1) & 3)) << 4);
+}
+
+// Source column of piece j for CTA `rank`.
+__device__ __forceinline__ int piece_col(uint32_t rank, int j)
+{
+    return j < 32 ? (int)rank * 256 + j * 8 : 512 + (int)rank * 32 + (j - 32) * 8;
+}
+
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
                           const __grid_constant__ CUtensorMap tm_q64,
-                          const __grid_constant__ CUtensorMap tm_kv128,
-                          const __grid_constant__ CUtensorMap tm_kv64,
+                          const __nv_bfloat16* __restrict__ kv,
                           const int* __restrict__ idx, const int* __restrict__ pos,
                           const int* __restrict__ k_base, int T, int S, int k, float scale_log2,
                           __nv_bfloat16* __restrict__ out, float* __restrict__ lse)
@@ -110,18 +130,21 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
     if (threadIdx.x == 0) {
         mbar_init(bar(B_Q), 1);
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(bar(B_FULL + s), 1);
+            // every gather thread's cp.async arrival + the mask publisher
+            mbar_init(bar(B_FULL + s), kGatherThreads + 1);
             mbar_init(bar(B_EMPTY + s), 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(bar(B_SFULL + b), 1);
-            mbar_init(bar(B_SFREE + b), 4);
-            mbar_init(bar(B_PFULL + b), 4);
+            mbar_init(bar(B_SFREE + b), 8);   // one arrival per softmax warp
+            mbar_init(bar(B_PFULL + b), 8);
             mbar_init(bar(B_PVDONE + b), 1);
             mbar_init(bar(B_XFULL + b), 1);   // receiver's expect_tx + the peer's bytes
-            mbar_init(bar(B_XFREE + b), 4);   // one arrival per softmax warp of the peer
+            mbar_init(bar(B_XFREE + b), 8);   // one arrival per softmax warp of the peer
+            mbar_init(bar(B_RED + b), 8);
         }
-        mbar_init(bar(B_DRAIN), 1);
+        mbar_init(bar(B_DRAIN), 2);     // QK and PV issuers
+        mbar_init(bar(B_LSUM), 8);
         *abort_flag = 0;
         fence_mbar_init_cluster();
     }
@@ -137,32 +160,19 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
     const uint32_t qs = sbase + kOffQ;
 
     if (warp == 0) {
-        // ------------------------------------------------------------- MMA
+        // --------------------------------------------------------- QK MMAs
         if (lane == 0 && NC > 0) {
             const uint32_t id_qk = idesc_bf16(128, kKeys, false);
-            const uint32_t id_pv = idesc_bf16(128, 256, true);
-            bool ok = mbar_wait(bar(B_Q), 0, abort_flag);
-            auto pv = [&](int c) -> bool {
-                if (!mbar_wait(bar(B_PFULL + (c & 1)), (c >> 1) & 1, abort_flag)) return false;
-                tc_fence_after();
-                const uint32_t kvs = sbase + kOffKV + (c % kStages) * kStageBytes;
-#pragma unroll
-                for (int kk = 0; kk < kKeys / 16; ++kk) {
-                    // B = gathered rows read MN-major: 64 values per 128-byte row,
-                    // LBO = next 64 columns (slab), SBO = next 8 keys.
-                    const uint64_t bd = smem_desc(kvs + kk * 16 * 128, kKSlab, 1024, kSwizzle128B);
-                    mma_f16_ts(tmem + kColO, tmem + kColP + (c & 1) * 32 + kk * 8, bd, id_pv,
-                               (c > 0 || kk > 0) ? 1u : 0u);
-                }
-                mma_commit(bar(B_PVDONE + (c & 1)));
-                mma_commit(bar(B_EMPTY + (c % kStages)));
-                return true;
-            };
+            bool ok = mbar_wait(bar(B_Q), 0, abort_flag, B_Q, 0);
             for (int c = 0; ok && c < NC; ++c) {
                 const int st = c % kStages;
-                ok = mbar_wait(bar(B_FULL + st), (c / kStages) & 1, abort_flag);
-                if (ok && c >= 2) ok = mbar_wait(bar(B_SFREE + (c & 1)), ((c - 2) >> 1) & 1, abort_flag);
+                ok = mbar_wait(bar(B_FULL + st), (c / kStages) & 1, abort_flag, B_FULL, c);
+                if (ok && c >= 2)
+                    ok = mbar_wait(bar(B_SFREE + (c & 1)), ((c - 2) >> 1) & 1, abort_flag, B_SFREE, c);
                 if (!ok) break;
+                // the stage was written by cp.async (generic proxy); the MMA
+                // reads it through the async proxy
+                fence_proxy_async_smem();
                 tc_fence_after();
                 const uint32_t kvs = sbase + kOffKV + st * kStageBytes;
                 const uint32_t d = tmem + kColS + (c & 1) * kKeys;
@@ -183,23 +193,41 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
                     mma_f16_ss(d, ad, bd, id_qk, 1u);
                 }
                 mma_commit(bar(B_SFULL + (c & 1)));
-                if (c >= 1) ok = pv(c - 1);
-            }
-            if (ok) pv(NC - 1);
-            // drain: every MMA issued above completes before TMEM is released
-            mma_commit(bar(B_DRAIN));
-            const uint64_t t0 = globaltimer_ns();
-            while (!mbar_try_wait(bar(B_DRAIN), 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
             }
         }
-        __syncwarp();
-    } else if (warp == 1) {
-        // ------------------------------------------------------ TMA loads
-        if (lane == 0) {
+    } else if (warp == 12) {
+        // --------------------------------------------------------- PV MMAs
+        if (lane == 0 && NC > 0) {
+            const uint32_t id_pv = idesc_bf16(128, 256, true);
+            for (int c = 0; c < NC; ++c) {
+                if (!mbar_wait(bar(B_PFULL + (c & 1)), (c >> 1) & 1, abort_flag, B_PFULL, c)) break;
+                tc_fence_after();
+                const uint32_t kvs = sbase + kOffKV + (c % kStages) * kStageBytes;
+#pragma unroll
+                for (int kk = 0; kk < kKeys / 16; ++kk) {
+                    // B = gathered rows read MN-major: 64 values per 128-byte row,
+                    // LBO = next 64 columns (slab), SBO = next 8 keys.
+                    const uint64_t bd = smem_desc(kvs + kk * 16 * 128, kKSlab, 1024, kSwizzle128B);
+                    mma_f16_ts(tmem + kColO, tmem + kColP + (c & 1) * 32 + kk * 8, bd, id_pv,
+                               (c > 0 || kk > 0) ? 1u : 0u);
+                }
+                mma_commit(bar(B_PVDONE + (c & 1)));
+                mma_commit(bar(B_EMPTY + (c % kStages)));
+            }
+        }
+    } else if (warp <= 3) {
+        // ---------------------------------------------------------- gather
+        // The 64 x 36 sixteen-byte pieces of a chunk are spread evenly over the
+        // 96 gather threads: piece e = it*96 + g is row e/36, piece e%36. The
+        // (row, piece) pattern of a thread repeats every three iterations with
+        // the row advanced by 8, which keeps the swizzle phase, so a copy costs
+        // one table load and one cp.async. Each warp keeps its own table of the
+        // chunk's row byte offsets (-1 = masked entry, read as zeros).
+        const int gw = warp - 1;
+        const int g = threadIdx.x - 32;
+        if (gw == 0 && lane == 0) {
             prefetch_tmap(&tm_q128);
             prefetch_tmap(&tm_q64);
-            prefetch_tmap(&tm_kv128);
-            prefetch_tmap(&tm_kv64);
             mbar_arrive_expect_tx(bar(B_Q), kQBytes);
             for (int j = 0; j < 4; ++j)
                 tma_load_2d(qs + j * kQSlab, &tm_q128, (int)rank * 256 + j * 64, t * kHeads, bar(B_Q));
@@ -207,201 +235,245 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
         }
         const int* idx_row = idx + (size_t)t * k;
         uint32_t* smask = reinterpret_cast<uint32_t*>(sgen + kOffMask);
-        // lane holds entries lane and lane + 32 of the next chunk (one chunk ahead)
+        long long* rows_tab = reinterpret_cast<long long*>(sgen + kOffRows) + gw * kKeys;
+        int r_q[3];
+        uint32_t d_q[3], dstep_q[3];
+        int col_q[3];
+#pragma unroll
+        for (int q3 = 0; q3 < 3; ++q3) {
+            const int e = q3 * kGatherThreads + g;
+            const int r = e / 36, j = e - r * 36;
+            r_q[q3] = r;
+            d_q[q3] = piece_dst(0, r, j);
+            dstep_q[q3] = j < 32 ? 8 * 128 : 8 * 64;
+            col_q[q3] = piece_col(rank, j) * 2;   // bytes
+        }
+        const char* kvb = reinterpret_cast<const char*>(kv);
         int sa = lane < n_row ? __ldg(idx_row + lane) : -1;
         int sb = lane + 32 < n_row ? __ldg(idx_row + lane + 32) : -1;
-        int issued = 0;
         for (int c = 0; c < NC; ++c) {
             const int st = c % kStages;
-            if (c >= kStages && !mbar_wait(bar(B_EMPTY + st), ((c - kStages) / kStages) & 1, abort_flag))
-                break;
+            if (c >= kStages) {
+                const bool got = mbar_wait(bar(B_EMPTY + st), ((c - kStages) / kStages) & 1,
+                                           abort_flag, 100 + B_EMPTY, c);
+                if (!__all_sync(0xffffffffu, got)) break;   // warp-uniform exit
+            }
             const bool va = sa >= 0 && sa <= p_last, vb = sb >= 0 && sb <= p_last;
-            // masked entries load row 0 of the sequence (finite data, weight 0)
-            const int ra = va ? sa : 0, rb = vb ? sb : 0;
-            const unsigned ma = __ballot_sync(0xffffffffu, va), mb = __ballot_sync(0xffffffffu, vb);
-            if (lane == 0) {
-                smask[st * 2] = ma;
-                smask[st * 2 + 1] = mb;
+            rows_tab[lane] = va ? (base + sa) * (long long)(kDqk * 2) : -1ll;
+            rows_tab[lane + 32] = vb ? (base + sb) * (long long)(kDqk * 2) : -1ll;
+            if (gw == 0) {
+                const unsigned ma = __ballot_sync(0xffffffffu, va), mb = __ballot_sync(0xffffffffu, vb);
+                if (lane == 0) {
+                    smask[st * 2] = ma;
+                    smask[st * 2 + 1] = mb;
+                }
             }
             const int i_next = (c + 1) * kKeys + lane;
             sa = i_next < n_row ? __ldg(idx_row + i_next) : -1;
             sb = i_next + 32 < n_row ? __ldg(idx_row + i_next + 32) : -1;
-            int y[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int key = 4 * (lane & 15) + e;
-                const int from_a = __shfl_sync(0xffffffffu, ra, key & 31);
-                const int from_b = __shfl_sync(0xffffffffu, rb, key & 31);
-                y[e] = (int)(base + (key < 32 ? from_a : from_b));
-            }
             __syncwarp();
-            if (lane == 0) mbar_arrive_expect_tx(bar(B_FULL + st), kStageBytes);
-            __syncwarp();
-            if (lane < 16) {
-                const uint32_t kvs = sbase + kOffKV + st * kStageBytes;
-                const int r0 = 4 * lane;
+            const uint32_t kvs = sbase + kOffKV + st * kStageBytes;
 #pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    tma_gather4(kvs + j * kKSlab + r0 * 128, &tm_kv128, (int)rank * 256 + j * 64,
-                                y[0], y[1], y[2], y[3], bar(B_FULL + st));
-                tma_gather4(kvs + 4 * kKSlab + r0 * 64, &tm_kv64, 512 + (int)rank * 32, y[0], y[1],
-                            y[2], y[3], bar(B_FULL + st));
-            }
-            issued = c + 1;
-        }
-        if (issued < NC) {
-            // aborted: let the loads already issued land before the CTA ends
-            for (int c = issued > kStages ? issued - kStages : 0; c < issued; ++c) {
-                const uint64_t t0 = globaltimer_ns();
-                while (!mbar_try_wait(bar(B_FULL + c % kStages), (c / kStages) & 1) &&
-                       globaltimer_ns() - t0 < kWaitLimitNs) {
+            for (int m = 0; m < 8; ++m)
+#pragma unroll
+                for (int q3 = 0; q3 < 3; ++q3) {
+                    const long long off = rows_tab[r_q[q3] + 8 * m];
+                    const void* src = off >= 0 ? kvb + off + col_q[q3] : kvb;
+                    cp_async16(kvs + d_q[q3] + m * dstep_q[q3], src, off >= 0 ? 16u : 0u);
                 }
-            }
+            cp_async_arrive_noinc(bar(B_FULL + st));
+            if (gw == 0 && lane == 0) mbar_arrive(bar(B_FULL + st));   // publishes the mask
+            __syncwarp();   // the table is rewritten for the next chunk
         }
+        cp_async_wait_all();
     } else if (warp >= 4) {
         // --------------------------------------------- softmax + epilogue
-        const int i = threadIdx.x - 128;                       // head = TMEM lane
+        // Warps 4-11: two warps per TMEM lane quarter; warp half hs takes keys
+        // [32hs, 32hs+32) of every chunk and output columns [128hs, 128hs+128).
+        const int hs = (warp - 4) >> 2;
+        const int i = (warp & 3) * 32 + lane;                  // head = TMEM lane
         const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
         const uint32_t xs = sbase + kOffX;
         const uint32_t x_peer = mapa(xs, peer);
         const uint32_t xfull_peer = mapa(bar(B_XFULL), peer);
         const uint32_t xfree_peer = mapa(bar(B_XFREE), peer);
         const uint32_t* smask = reinterpret_cast<const uint32_t*>(sgen + kOffMask);
+        float* red = reinterpret_cast<float*>(sgen + kOffRed);
+        float* lsum_s = reinterpret_cast<float*>(sgen + kOffLsum);
         float m_use = -INFINITY, l = 0.f;
         bool ok = true;
-
-        // this CTA's partial logits of chunk c, scaled, as fp16 pairs
-        auto load_partial = [&](int c, uint32_t (&h)[32]) {
-            uint32_t s0[32], s1[32];
-            tmem_ld32(tmem + lane_addr + kColS + (c & 1) * kKeys, s0);
-            tmem_ld32(tmem + lane_addr + kColS + (c & 1) * kKeys + 32, s1);
-            tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                h[j] = pack_half2(__uint_as_float(s0[2 * j]) * scale_log2,
-                                  __uint_as_float(s0[2 * j + 1]) * scale_log2);
-                h[16 + j] = pack_half2(__uint_as_float(s1[2 * j]) * scale_log2,
-                                       __uint_as_float(s1[2 * j + 1]) * scale_log2);
-            }
+        // bounded wait whose outcome is the same for the whole warp
+        auto wait_w = [&](uint32_t b_addr, uint32_t par, int tag, int c, bool cluster) -> bool {
+            const bool got = cluster ? mbar_wait<true>(b_addr, par, abort_flag, tag, c)
+                                     : mbar_wait(b_addr, par, abort_flag, tag, c);
+            return __all_sync(0xffffffffu, got);
         };
-        // send chunk c's partial into the peer's exchange slot
+
+        // Send this CTA's partial logits of chunk c (scaled, fp16) to the peer.
         auto send = [&](int c) -> bool {
             const int b = c & 1;
-            if (!mbar_wait(bar(B_SFULL + b), (c >> 1) & 1, abort_flag)) return false;
+            if (!wait_w(bar(B_SFULL + b), (c >> 1) & 1, 200 + B_SFULL, c, false)) return false;
             tc_fence_after();
-            uint32_t h[32];
-            load_partial(c, h);
-            if (c >= 2 && !mbar_wait<true>(bar(B_XFREE + b), ((c - 2) >> 1) & 1, abort_flag)) return false;
+            uint32_t sr[32];
+            tmem_ld32(tmem + lane_addr + kColS + b * kKeys + 32 * hs, sr);
+            tmem_wait_ld();
+            uint32_t h[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+                h[j] = pack_half2(__uint_as_float(sr[2 * j]) * scale_log2,
+                                  __uint_as_float(sr[2 * j + 1]) * scale_log2);
+            if (c >= 2 && !wait_w(bar(B_XFREE + b), ((c - 2) >> 1) & 1, 200 + B_XFREE, c, true)) return false;
             const uint32_t xr_peer = x_peer + b * kXBytes + i * 128;
 #pragma unroll
-            for (int m = 0; m < 8; ++m)
-                st_async_v4(xr_peer + (((m + i) & 7) << 4),
+            for (int m = 0; m < 4; ++m)
+                st_async_v4(xr_peer + (((4 * hs + m + i) & 7) << 4),
                             make_uint4(h[4 * m], h[4 * m + 1], h[4 * m + 2], h[4 * m + 3]),
                             xfull_peer + 8u * b);
             return true;
         };
 
-        if (NC > 0) ok = send(0);
+        int sent = 0;                       // chunks whose partial logits went out
+        if (NC > 0) {
+            ok = send(0);
+            sent = 1;
+        }
         for (int c = 0; ok && c < NC; ++c) {
             const int b = c & 1;
-            // the next chunk's exchange overlaps this chunk's softmax
-            if (c + 1 < NC && !send(c + 1)) { ok = false; break; }
-            if (i == 0) mbar_arrive_expect_tx(bar(B_XFULL + b), kXBytes);
-            if (!mbar_wait<true>(bar(B_XFULL + b), (c >> 1) & 1, abort_flag)) { ok = false; break; }
-            uint32_t g[32], h[32];
+            // send the next chunk's partial now if its logits are already in
+            // TMEM (the exchange then overlaps this chunk's softmax); never
+            // wait for them here
+            if (c + 1 < NC && sent == c + 1 &&
+                __all_sync(0xffffffffu, mbar_test_wait(bar(B_SFULL + ((c + 1) & 1)), ((c + 1) >> 1) & 1))) {
+                if (!send(c + 1)) { ok = false; break; }
+                sent = c + 2;
+            }
+            if (i == 0 && hs == 0) mbar_arrive_expect_tx(bar(B_XFULL + b), kXBytes);
+            if (!wait_w(bar(B_XFULL + b), (c >> 1) & 1, 200 + B_XFULL, c, true)) { ok = false; break; }
+            uint32_t g[16];
             const uint32_t xr = xs + b * kXBytes + i * 128;
 #pragma unroll
-            for (int m = 0; m < 8; ++m) {
-                const uint4 v = ld_shared_v4(xr + (((m + i) & 7) << 4));
+            for (int m = 0; m < 4; ++m) {
+                const uint4 v = ld_shared_v4(xr + (((4 * hs + m + i) & 7) << 4));
                 g[4 * m] = v.x; g[4 * m + 1] = v.y; g[4 * m + 2] = v.z; g[4 * m + 3] = v.w;
             }
-            load_partial(c, h);                     // same rounding as what was sent
+            uint32_t sr[32];
+            tmem_ld32(tmem + lane_addr + kColS + b * kKeys + 32 * hs, sr);
+            tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_SFREE + b));
-            // validity of the chunk's entries (published by the gather warps)
-            if (!mbar_wait(bar(B_FULL + c % kStages), (c / kStages) & 1, abort_flag)) { ok = false; break; }
-            const uint32_t mlo = smask[(c % kStages) * 2], mhi = smask[(c % kStages) * 2 + 1];
-
-            // full logits (log2 domain), masked entries -> -inf
-            float x[kKeys];
+            if (!wait_w(bar(B_FULL + c % kStages), (c / kStages) & 1, 200 + B_FULL, c, false)) { ok = false; break; }
+            const uint32_t mw = smask[(c % kStages) * 2 + hs];
+            // logit (log2 domain) = own partial (fp32) + peer partial (fp16); masked -> -inf
+            float x[32];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const float2 a = unpack_half2(h[j]), o = unpack_half2(g[j]);
-                const uint32_t mw = j < 16 ? mlo : mhi;
-                x[2 * j] = (mw >> ((2 * j) & 31)) & 1u ? a.x + o.x : -INFINITY;
-                x[2 * j + 1] = (mw >> ((2 * j + 1) & 31)) & 1u ? a.y + o.y : -INFINITY;
+            for (int j = 0; j < 16; ++j) {
+                const float2 o = unpack_half2(g[j]);
+                x[2 * j] = (mw >> (2 * j)) & 1u ? fmaf(__uint_as_float(sr[2 * j]), scale_log2, o.x)
+                                                : -INFINITY;
+                x[2 * j + 1] = (mw >> (2 * j + 1)) & 1u
+                                   ? fmaf(__uint_as_float(sr[2 * j + 1]), scale_log2, o.y)
+                                   : -INFINITY;
             }
             // the peer may refill this exchange slot once every warp has used it
             __syncwarp();
             if (lane == 0) mbar_arrive_remote(xfree_peer + 8u * b);
-            float mc = -INFINITY;
+            float mx[16];
 #pragma unroll
-            for (int j = 0; j < kKeys; ++j) mc = fmaxf(mc, x[j]);
+            for (int j = 0; j < 16; ++j) mx[j] = fmaxf(x[j], x[j + 16]);
+#pragma unroll
+            for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+                for (int j = 0; j < w; ++j) mx[j] = fmaxf(mx[j], mx[j + w]);
+            // row maximum over both key halves (the other half lives in warp +-4)
+            red[(b * 2 + hs) * kHeads + i] = mx[0];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(B_RED + b));
+            if (!wait_w(bar(B_RED + b), (c >> 1) & 1, 200 + B_RED, c, false)) { ok = false; break; }
+            const float mc = fmaxf(mx[0], red[(b * 2 + (hs ^ 1)) * kHeads + i]);
             const float m_new = fmaxf(m_use, mc);
-            if (m_new > m_use + 8.f) {
-                if (m_use != -INFINITY) {
-                    // O holds earlier chunks: rescale once PV(c-1) has landed
-                    const float f = ex2(m_use - m_new);
-                    l *= f;
-                    if (!mbar_wait(bar(B_PVDONE + ((c - 1) & 1)), ((c - 1) >> 1) & 1, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-#pragma unroll 1
-                    for (int q8 = 0; q8 < 8; ++q8) {
-                        uint32_t o[32];
-                        tmem_ld32(tmem + lane_addr + kColO + q8 * 32, o);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
-                        tmem_st32(tmem + lane_addr + kColO + q8 * 32, o);
-                    }
-                    tmem_wait_st();
+            const bool raise = m_new > m_use + 8.f;
+            const bool rescale = raise && m_use != -INFINITY;
+            const float f = rescale ? ex2(m_use - m_new) : 1.f;
+            if (__any_sync(0xffffffffu, rescale)) {
+                // O holds earlier chunks: rescale once PV(c-1) has landed. TMEM
+                // loads/stores are warp-wide, so every lane takes part (f = 1
+                // for rows whose maximum did not move).
+                if (!wait_w(bar(B_PVDONE + ((c - 1) & 1)), ((c - 1) >> 1) & 1, 400 + B_PVDONE, c, false)) {
+                    ok = false;
+                    break;
                 }
-                m_use = m_new;
-            }
-            const float msub = m_use == -INFINITY ? 0.f : m_use;
-            uint32_t pk[32];
-            float lsum = 0.f;
+                tc_fence_after();
+#pragma unroll 1
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    uint32_t o[32];
+                    const uint32_t ta = tmem + lane_addr + kColO + 128 * hs + q4 * 32;
+                    tmem_ld32(ta, o);
+                    tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
+                    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+                    tmem_st32(ta, o);
+                }
+                tmem_wait_st();
+            }
+            l *= f;
+            if (raise) m_use = m_new;
+            const float msub = m_use == -INFINITY ? 0.f : m_use;
+            uint32_t pk[16];
+            float ps[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
                 const float p0 = ex2(x[2 * j] - msub), p1 = ex2(x[2 * j + 1] - msub);
-                lsum += p0 + p1;
+                ps[j] = p0 + p1;
                 pk[j] = pack_bf16x2(p0, p1);
             }
-            l += lsum;
-            if (c >= 2 && !mbar_wait(bar(B_PVDONE + b), ((c - 2) >> 1) & 1, abort_flag)) {
+#pragma unroll
+            for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+                for (int j = 0; j < w; ++j) ps[j] += ps[j + w];
+            l += ps[0];
+            if (c >= 2 && !wait_w(bar(B_PVDONE + b), ((c - 2) >> 1) & 1, 200 + B_PVDONE, c, false)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            tmem_st32(tmem + lane_addr + kColP + b * 32, pk);
+            tmem_st16(tmem + lane_addr + kColP + b * 32 + 16 * hs, pk);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_PFULL + b));
+            if (c + 1 < NC && sent == c + 1) {
+                if (!send(c + 1)) { ok = false; break; }
+                sent = c + 2;
+            }
         }
-        // epilogue: O / l -> bf16, this CTA's 256 columns of head i
-        __nv_bfloat16* orow = out + ((size_t)t * kHeads + i) * kDv + rank * 256;
+        // row sum over both key halves
+        if (ok) {
+            lsum_s[hs * kHeads + i] = l;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(B_LSUM));
+            ok = wait_w(bar(B_LSUM), 0, 200 + B_LSUM, 0, false);
+            if (ok) l += lsum_s[(hs ^ 1) * kHeads + i];
+        }
+        // epilogue: O / l -> bf16, columns [128hs, 128hs+128) of this CTA's half
+        __nv_bfloat16* orow = out + ((size_t)t * kHeads + i) * kDv + rank * 256 + 128 * hs;
         if (ok && NC > 0) {
             const int c = NC - 1;
-            ok = mbar_wait(bar(B_PVDONE + (c & 1)), (c >> 1) & 1, abort_flag);
+            ok = wait_w(bar(B_PVDONE + (c & 1)), (c >> 1) & 1, 300 + B_PVDONE, c, false);
             if (ok) {
                 tc_fence_after();
                 const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll 1
-                for (int q8 = 0; q8 < 8; ++q8) {
+                for (int q4 = 0; q4 < 4; ++q4) {
                     uint32_t o[32];
-                    tmem_ld32(tmem + lane_addr + kColO + q8 * 32, o);
+                    tmem_ld32(tmem + lane_addr + kColO + 128 * hs + q4 * 32, o);
                     tmem_wait_ld();
                     uint32_t w[16];
 #pragma unroll
                     for (int e = 0; e < 16; ++e)
                         w[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv,
                                            __uint_as_float(o[2 * e + 1]) * inv);
-                    uint4* dst = reinterpret_cast<uint4*>(orow + q8 * 32);
+                    uint4* dst = reinterpret_cast<uint4*>(orow + q4 * 32);
 #pragma unroll
                     for (int v = 0; v < 4; ++v)
                         dst[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
@@ -409,12 +481,19 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
             }
         } else if (NC == 0) {
             uint4* dst = reinterpret_cast<uint4*>(orow);
-            for (int v = 0; v < 32; ++v) dst[v] = make_uint4(0u, 0u, 0u, 0u);
+            for (int v = 0; v < 16; ++v) dst[v] = make_uint4(0u, 0u, 0u, 0u);
         }
-        if (rank == 0 && (ok || NC == 0))
+        if (rank == 0 && hs == 0 && (ok || NC == 0))
             lse[(size_t)t * kHeads + i] = l > 0.f ? (m_use + __log2f(l)) * 0.69314718055994531f : -INFINITY;
     }
 
+    if ((warp == 0 || warp == 12) && lane == 0 && NC > 0) {
+        // every MMA this thread issued completes before TMEM is released
+        mma_commit(bar(B_DRAIN));
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(bar(B_DRAIN), 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
+        }
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();

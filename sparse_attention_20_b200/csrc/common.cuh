@@ -8,12 +8,26 @@
 
 namespace dsa {
 
+enum : int { kStatusOk = 0, kStatusTimeout = -4 };
+
 // Device status word: kernels record the first failure here (never trap).
 __device__ int g_status = 0;
 
-enum : int { kStatusOk = 0, kStatusTimeout = -4 };
+// Where the first bounded wait gave up: {tag, chunk, block, parity}.
+__device__ int g_timeout_info[4] = {0, 0, 0, 0};
 
 __device__ __forceinline__ void report_status(int code) { atomicCAS(&g_status, 0, code); }
+
+__device__ __forceinline__ void report_timeout(int tag, int chunk, int parity)
+{
+    if (atomicCAS(&g_status, 0, kStatusTimeout) == 0) {
+        g_timeout_info[0] = tag;
+        g_timeout_info[1] = chunk;
+        g_timeout_info[2] = (int)blockIdx.x;
+        g_timeout_info[3] = parity;
+        __threadfence();
+    }
+}
 
 // Order-preserving map fp32 -> uint32 (a > b  <=>  key(a) > key(b)); -0 is
 // folded onto +0 so that equal scores compare equal.

@@ -256,21 +256,16 @@ int attn_tc(const __nv_bfloat16* q, const __nv_bfloat16* kv, const int32_t* idx,
     cudaError_t e = cudaFuncSetAttribute(sparse_mla_attn_tc_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(sparse_mla_attn_tc_kernel)");
-    // Q as [T*128, 576]: one 128-head box per slab; KV as [S, 576]: one-row
-    // boxes for tile::gather4. 64-column slabs use 128B swizzle, the 32-column
-    // rope slab 64B swizzle.
-    CUtensorMap tq128, tq64, tkv128, tkv64;
+    // Q as [T*128, 576]: one 128-head box per slab; 64-column slabs use 128B
+    // swizzle, the 32-column rope slab 64B swizzle.
+    CUtensorMap tq128, tq64;
     if (int rc = make_tmap_bf16(&tq128, q, kDqk, (uint64_t)T * kHeads, 64, kHeads,
                                 CU_TENSOR_MAP_SWIZZLE_128B)) return rc;
     if (int rc = make_tmap_bf16(&tq64, q, kDqk, (uint64_t)T * kHeads, 32, kHeads,
                                 CU_TENSOR_MAP_SWIZZLE_64B)) return rc;
-    if (int rc = make_tmap_bf16(&tkv128, kv, kDqk, (uint64_t)S, 64, 1, CU_TENSOR_MAP_SWIZZLE_128B))
-        return rc;
-    if (int rc = make_tmap_bf16(&tkv64, kv, kDqk, (uint64_t)S, 32, 1, CU_TENSOR_MAP_SWIZZLE_64B))
-        return rc;
     const float scale_log2 = scale * 1.4426950408889634f;
     sparse_mla_attn_tc_kernel<<<dim3(2 * T), kThreads, kSmemBytes, st>>>(
-        tq128, tq64, tkv128, tkv64, idx, pos, k_base, T, S, k, scale_log2, out, lse);
+        tq128, tq64, kv, idx, pos, k_base, T, S, k, scale_log2, out, lse);
     DSA_LAUNCH_CHECK("sparse_mla_attn_tc_kernel");
     return DSA_OK;
 }
@@ -355,9 +350,12 @@ int dsa_device_status(void* stream)
     e = cudaMemcpyFromSymbol(&v, dsa::g_status, sizeof v);
     if (e != cudaSuccess) return cuda_fail(e, "read device status");
     if (v != 0) {
+        int info[4] = {0, 0, 0, 0};
+        cudaMemcpyFromSymbol(info, dsa::g_timeout_info, sizeof info);
         const int zero = 0;
         cudaMemcpyToSymbol(dsa::g_status, &zero, sizeof zero);
-        return fail(v, "a kernel reported status %d (bounded wait gave up)", v);
+        return fail(v, "a kernel reported status %d: bounded wait gave up (barrier tag %d, chunk %d, "
+                       "block %d, parity %d)", v, info[0], info[1], info[2], info[3]);
     }
     return DSA_OK;
 }
