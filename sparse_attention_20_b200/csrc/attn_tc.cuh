@@ -44,17 +44,16 @@ constexpr int kHeads = 128;
 constexpr int kDqk = 576;
 constexpr int kDv = 512;
 constexpr int kKeys = 64;
-constexpr int kStages = 3;
+constexpr int kStages = 4;
 constexpr int kThreads = 416;               // 13 warps: QK, 3 gather, 8 softmax, PV
 constexpr int kGatherThreads = 96;
 
-constexpr int kQSlab = kHeads * 128;        // 64 columns x 128 rows, 128B swizzle
-constexpr int kQBytes = 4 * kQSlab + kHeads * 64;
+constexpr int kQBytes = kHeads * 64;       // rope slice of Q: 32 columns, 64B swizzle
 constexpr int kKSlab = kKeys * 128;
 constexpr int kStageBytes = 4 * kKSlab + kKeys * 64;
 constexpr int kXBytes = kHeads * 128;       // 64 fp16 partial logits per head
 constexpr int kOffQ = 0;
-constexpr int kOffKV = kOffQ + kQBytes;
+constexpr int kOffKV = kOffQ + 8192;       // (kQBytes, rounded to 1 KB)
 constexpr int kOffX = kOffKV + kStages * kStageBytes;
 constexpr int kOffBar = kOffX + 2 * kXBytes;
 constexpr int kOffMask = kOffBar + 256;                 // [kStages][2] validity bits
@@ -64,11 +63,13 @@ constexpr int kOffRows = kOffLsum + 2 * kHeads * 4;     // [3 gather warps][64] 
 constexpr int kSmemBytes = kOffRows + 3 * kKeys * 8 + 1024;  // + 1 KB alignment slack
 
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColO = 0, kColS = 256, kColP = 384;
+// O [0,256); S double buffer [256,384) (P(c) overwrites the first half of
+// each key half's S columns once read); latent Q slice [384,512).
+constexpr uint32_t kColO = 0, kColS = 256, kColQ = 384;
 
 enum : int {
-    B_Q = 0, B_FULL = 1, B_EMPTY = 4, B_SFULL = 7, B_SFREE = 9, B_PFULL = 11, B_PVDONE = 13,
-    B_XFULL = 15, B_XFREE = 17, B_DRAIN = 19, B_RED = 20, B_LSUM = 22, B_COUNT = 23
+    B_Q = 0, B_QT = 1, B_FULL = 2, B_EMPTY = 6, B_SFULL = 10, B_PFULL = 12, B_PVDONE = 14,
+    B_XFULL = 16, B_XFREE = 18, B_DRAIN = 20, B_RED = 21, B_LSUM = 23, B_COUNT = 24
 };
 
 static_assert(kOffKV % 1024 == 0 && kStageBytes % 1024 == 0 && kOffX % 1024 == 0, "alignment");
@@ -101,8 +102,8 @@ __device__ __forceinline__ int piece_col(uint32_t rank, int j)
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
-                          const __grid_constant__ CUtensorMap tm_q64,
+sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q64,
+                          const __nv_bfloat16* __restrict__ q,
                           const __nv_bfloat16* __restrict__ kv,
                           const int* __restrict__ idx, const int* __restrict__ pos,
                           const int* __restrict__ k_base, int T, int S, int k, float scale_log2,
@@ -129,6 +130,7 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
 
     if (threadIdx.x == 0) {
         mbar_init(bar(B_Q), 1);
+        mbar_init(bar(B_QT), 8);        // latent Q written to TMEM by the softmax warps
         for (int s = 0; s < kStages; ++s) {
             // every gather thread's cp.async arrival + the mask publisher
             mbar_init(bar(B_FULL + s), kGatherThreads + 1);
@@ -136,7 +138,6 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(bar(B_SFULL + b), 1);
-            mbar_init(bar(B_SFREE + b), 8);   // one arrival per softmax warp
             mbar_init(bar(B_PFULL + b), 8);
             mbar_init(bar(B_PVDONE + b), 1);
             mbar_init(bar(B_XFULL + b), 1);   // receiver's expect_tx + the peer's bytes
@@ -163,12 +164,14 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
         // --------------------------------------------------------- QK MMAs
         if (lane == 0 && NC > 0) {
             const uint32_t id_qk = idesc_bf16(128, kKeys, false);
-            bool ok = mbar_wait(bar(B_Q), 0, abort_flag, B_Q, 0);
+            bool ok = mbar_wait(bar(B_Q), 0, abort_flag, B_Q, 0) &&
+                      mbar_wait(bar(B_QT), 0, abort_flag, B_QT, 0);
             for (int c = 0; ok && c < NC; ++c) {
                 const int st = c % kStages;
                 ok = mbar_wait(bar(B_FULL + st), (c / kStages) & 1, abort_flag, B_FULL, c);
+                // S(c) reuses the buffer of chunk c-2, whose P that PV(c-2) read
                 if (ok && c >= 2)
-                    ok = mbar_wait(bar(B_SFREE + (c & 1)), ((c - 2) >> 1) & 1, abort_flag, B_SFREE, c);
+                    ok = mbar_wait(bar(B_PVDONE + (c & 1)), ((c - 2) >> 1) & 1, abort_flag, B_PVDONE, c);
                 if (!ok) break;
                 // the stage was written by cp.async (generic proxy); the MMA
                 // reads it through the async proxy
@@ -176,19 +179,16 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
                 tc_fence_after();
                 const uint32_t kvs = sbase + kOffKV + st * kStageBytes;
                 const uint32_t d = tmem + kColS + (c & 1) * kKeys;
-                uint32_t acc = 0;
+                // latent part: A = Q slice in TMEM (16 K-steps of 16 columns)
 #pragma unroll
-                for (int slab = 0; slab < 4; ++slab)
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) {
-                        const uint64_t ad = smem_desc(qs + slab * kQSlab + kk * 32, 16, 1024, kSwizzle128B);
-                        const uint64_t bd = smem_desc(kvs + slab * kKSlab + kk * 32, 16, 1024, kSwizzle128B);
-                        mma_f16_ss(d, ad, bd, id_qk, acc);
-                        acc = 1;
-                    }
+                for (int kk = 0; kk < 16; ++kk) {
+                    const uint64_t bd = smem_desc(kvs + (kk >> 2) * kKSlab + (kk & 3) * 32, 16, 1024, kSwizzle128B);
+                    mma_f16_ts(d, tmem + kColQ + kk * 8, bd, id_qk, kk > 0 ? 1u : 0u);
+                }
+                // rope part: A = Q rope slice in shared memory
 #pragma unroll
                 for (int kk = 0; kk < 2; ++kk) {
-                    const uint64_t ad = smem_desc(qs + 4 * kQSlab + kk * 32, 16, 512, kSwizzle64B);
+                    const uint64_t ad = smem_desc(qs + kk * 32, 16, 512, kSwizzle64B);
                     const uint64_t bd = smem_desc(kvs + 4 * kKSlab + kk * 32, 16, 512, kSwizzle64B);
                     mma_f16_ss(d, ad, bd, id_qk, 1u);
                 }
@@ -208,7 +208,8 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
                     // B = gathered rows read MN-major: 64 values per 128-byte row,
                     // LBO = next 64 columns (slab), SBO = next 8 keys.
                     const uint64_t bd = smem_desc(kvs + kk * 16 * 128, kKSlab, 1024, kSwizzle128B);
-                    mma_f16_ts(tmem + kColO, tmem + kColP + (c & 1) * 32 + kk * 8, bd, id_pv,
+                    // P of keys [32h, 32h+32) sits in the first 16 columns of that half's S
+                    mma_f16_ts(tmem + kColO, tmem + kColS + (c & 1) * kKeys + (kk >> 1) * 32 + (kk & 1) * 8, bd, id_pv,
                                (c > 0 || kk > 0) ? 1u : 0u);
                 }
                 mma_commit(bar(B_PVDONE + (c & 1)));
@@ -226,12 +227,9 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
         const int gw = warp - 1;
         const int g = threadIdx.x - 32;
         if (gw == 0 && lane == 0) {
-            prefetch_tmap(&tm_q128);
             prefetch_tmap(&tm_q64);
             mbar_arrive_expect_tx(bar(B_Q), kQBytes);
-            for (int j = 0; j < 4; ++j)
-                tma_load_2d(qs + j * kQSlab, &tm_q128, (int)rank * 256 + j * 64, t * kHeads, bar(B_Q));
-            tma_load_2d(qs + 4 * kQSlab, &tm_q64, 512 + (int)rank * 32, t * kHeads, bar(B_Q));
+            tma_load_2d(qs, &tm_q64, 512 + (int)rank * 32, t * kHeads, bar(B_Q));
         }
         const int* idx_row = idx + (size_t)t * k;
         uint32_t* smask = reinterpret_cast<uint32_t*>(sgen + kOffMask);
@@ -332,6 +330,26 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
             return true;
         };
 
+        {
+            // latent Q slice of head i into TMEM (A operand of the QK MMAs):
+            // this half's 128 columns, two bf16 per 32-bit column
+            const uint4* qsrc = reinterpret_cast<const uint4*>(
+                q + ((size_t)t * kHeads + i) * kDqk + rank * 256 + 128 * hs);
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {
+                uint32_t w[32];
+#pragma unroll
+                for (int v = 0; v < 8; ++v) {
+                    const uint4 x = __ldg(qsrc + part * 8 + v);
+                    w[4 * v] = x.x; w[4 * v + 1] = x.y; w[4 * v + 2] = x.z; w[4 * v + 3] = x.w;
+                }
+                tmem_st32(tmem + lane_addr + kColQ + 64 * hs + 32 * part, w);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(B_QT));
+        }
         int sent = 0;                       // chunks whose partial logits went out
         if (NC > 0) {
             ok = send(0);
@@ -359,9 +377,6 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
             uint32_t sr[32];
             tmem_ld32(tmem + lane_addr + kColS + b * kKeys + 32 * hs, sr);
             tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(B_SFREE + b));
             if (!wait_w(bar(B_FULL + c % kStages), (c / kStages) & 1, 200 + B_FULL, c, false)) { ok = false; break; }
             const uint32_t mw = smask[(c % kStages) * 2 + hs];
             // logit (log2 domain) = own partial (fp32) + peer partial (fp16); masked -> -inf
@@ -432,12 +447,8 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
 #pragma unroll
                 for (int j = 0; j < w; ++j) ps[j] += ps[j + w];
             l += ps[0];
-            if (c >= 2 && !wait_w(bar(B_PVDONE + b), ((c - 2) >> 1) & 1, 200 + B_PVDONE, c, false)) {
-                ok = false;
-                break;
-            }
             tc_fence_after();
-            tmem_st16(tmem + lane_addr + kColP + b * 32 + 16 * hs, pk);
+            tmem_st16(tmem + lane_addr + kColS + b * kKeys + 32 * hs, pk);   // over this half's S
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
