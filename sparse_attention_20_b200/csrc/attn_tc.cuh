@@ -320,7 +320,8 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q64,
             for (int j = 0; j < 16; ++j)
                 h[j] = pack_half2(__uint_as_float(sr[2 * j]) * scale_log2,
                                   __uint_as_float(sr[2 * j + 1]) * scale_log2);
-            if (c >= 2 && !wait_w(bar(B_XFREE + b), ((c - 2) >> 1) & 1, 200 + B_XFREE, c, true)) return false;
+            // the peer has consumed chunk c-2 from this slot (a pure signal)
+            if (c >= 2 && !wait_w(bar(B_XFREE + b), ((c - 2) >> 1) & 1, 200 + B_XFREE, c, false)) return false;
             const uint32_t xr_peer = x_peer + b * kXBytes + i * 128;
 #pragma unroll
             for (int m = 0; m < 4; ++m)
@@ -366,7 +367,8 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q64,
                 sent = c + 2;
             }
             if (i == 0 && hs == 0) mbar_arrive_expect_tx(bar(B_XFULL + b), kXBytes);
-            if (!wait_w(bar(B_XFULL + b), (c >> 1) & 1, 200 + B_XFULL, c, true)) { ok = false; break; }
+            // the peer's bytes arrive by st.async, counted on this local barrier
+            if (!wait_w(bar(B_XFULL + b), (c >> 1) & 1, 200 + B_XFULL, c, false)) { ok = false; break; }
             uint32_t g[16];
             const uint32_t xr = xs + b * kXBytes + i * 128;
 #pragma unroll
@@ -391,8 +393,9 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q64,
                                    : -INFINITY;
             }
             // the peer may refill this exchange slot once every warp has used it
+            // (the loaded values are consumed above, so a relaxed signal suffices)
             __syncwarp();
-            if (lane == 0) mbar_arrive_remote(xfree_peer + 8u * b);
+            if (lane == 0) mbar_arrive_remote_relaxed(xfree_peer + 8u * b);
             float mx[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) mx[j] = fmaxf(x[j], x[j + 16]);

@@ -44,6 +44,15 @@ __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_bar)
                  : "memory");
 }
 
+// Relaxed remote arrival: a pure signal that orders no memory operation.
+// Used where the signalled fact is already settled by data dependence (for
+// example "this thread has consumed those values").
+__device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t cluster_bar)
+{
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar)
+                 : "memory");
+}
+
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
 {
     uint32_t ok;
