@@ -409,6 +409,12 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q64,
             if (lane == 0) mbar_arrive(bar(B_RED + b));
             if (!wait_w(bar(B_RED + b), (c >> 1) & 1, 200 + B_RED, c, false)) { ok = false; break; }
             const float mc = fmaxf(mx[0], red[(b * 2 + (hs ^ 1)) * kHeads + i]);
+            // second chance to send the next chunk's partial before this chunk's exps
+            if (c + 1 < NC && sent == c + 1 &&
+                __all_sync(0xffffffffu, mbar_test_wait(bar(B_SFULL + ((c + 1) & 1)), ((c + 1) >> 1) & 1))) {
+                if (!send(c + 1)) { ok = false; break; }
+                sent = c + 2;
+            }
             const float m_new = fmaxf(m_use, mc);
             const bool raise = m_new > m_use + 8.f;
             const bool rescale = raise && m_use != -INFINITY;
