@@ -16,6 +16,7 @@
 #include "attn_tc.cuh"
 #include "common.cuh"
 #include "indexer_scores.cuh"
+#include "indexer_tc.cuh"
 #include "topk_select.cuh"
 
 namespace {
@@ -61,9 +62,34 @@ int index_rows_per_block(int T, int S)
     return (int)std::min<size_t>((size_t)T, rows);
 }
 
-size_t indexer_workspace(int T, int S)
+// Streaming (tensor-core) indexer: query rows per launch block and the
+// per-row buffers it needs.
+constexpr int kFusedRowsPerBlock = 32768;
+
+struct FusedPlan {
+    int RB, samp_ld, cap;
+    size_t off_samp, off_tau, off_cand, off_cnt, bytes;
+};
+
+FusedPlan fused_plan(int T, int S, int k)
 {
-    return align_up((size_t)index_rows_per_block(T, S) * (size_t)S * sizeof(float));
+    using namespace dsa::idx_tc;
+    FusedPlan p;
+    p.RB = std::min(T, kFusedRowsPerBlock);
+    p.samp_ld = ((num_tiles(S) + kSampleStride - 1) / kSampleStride) * kKeys;
+    p.cap = 2 * kAlpha * k;
+    p.off_samp = 0;
+    p.off_tau = align_up(p.off_samp + (size_t)p.RB * p.samp_ld * sizeof(float));
+    p.off_cand = align_up(p.off_tau + (size_t)p.RB * sizeof(float));
+    p.off_cnt = align_up(p.off_cand + (size_t)p.RB * p.cap * sizeof(uint2));
+    p.bytes = align_up(p.off_cnt + (size_t)p.RB * sizeof(int));
+    return p;
+}
+
+size_t indexer_workspace(int T, int S, int k = 1)
+{
+    const size_t general = align_up((size_t)index_rows_per_block(T, S) * (size_t)S * sizeof(float));
+    return std::max(general, fused_plan(T, S, k).bytes);
 }
 
 int num_sms()
@@ -190,6 +216,64 @@ int indexer_scan_select(const uint8_t* q_idx, const float* w, const uint8_t* k_i
     return DSA_OK;
 }
 
+// One causal sequence (pos and k_base NULL), H_I = 8, d_I = 128: streamed
+// FP8 tensor-core scan with sampled thresholds (indexer_tc.cuh).
+bool indexer_fused_supported(const int32_t* pos, const int32_t* k_base, int H_I, int d_I)
+{
+    if (const char* e = getenv("DSA_INDEXER_IMPL"))
+        if (strcmp(e, "general") == 0) return false;
+    return !pos && !k_base && H_I == dsa::idx_tc::kHI && d_I == dsa::idx_tc::kDI;
+}
+
+int make_tmap_u8(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t rows,
+                 uint32_t box_rows)
+{
+    const cuuint64_t dims[2] = {row_bytes, rows};
+    const cuuint64_t strides[1] = {row_bytes};
+    const cuuint32_t box[2] = {(cuuint32_t)row_bytes, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = cuTensorMapEncodeTiled(
+        m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return DSA_OK;
+}
+
+int indexer_fused(const uint8_t* q_idx, const float* w, const uint8_t* k_idx, int T, int S, int k,
+                  int32_t* idx, void* workspace, cudaStream_t st)
+{
+    using namespace dsa::idx_tc;
+    const FusedPlan p = fused_plan(T, S, k);
+    char* ws = reinterpret_cast<char*>(workspace);
+    float* samp = reinterpret_cast<float*>(ws + p.off_samp);
+    float* tau = reinterpret_cast<float*>(ws + p.off_tau);
+    uint2* cand = reinterpret_cast<uint2*>(ws + p.off_cand);
+    int* cnt = reinterpret_cast<int*>(ws + p.off_cnt);
+    CUtensorMap tq, tk;
+    if (int rc = make_tmap_u8(&tq, q_idx, kDI, (uint64_t)T * kHI, kN)) return rc;
+    if (int rc = make_tmap_u8(&tk, k_idx, kDI, (uint64_t)S, kKeys)) return rc;
+    for (auto* f : {indexer_scan_kernel<true>, indexer_scan_kernel<false>}) {
+        cudaError_t e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(indexer_scan_kernel)");
+    }
+    for (int row0 = 0; row0 < T; row0 += p.RB) {
+        const int rows = std::min(p.RB, T - row0);
+        ScanArgs a{w, T, S, k, row0, rows, samp, p.samp_ld, tau, cand, cnt, p.cap};
+        const int ctas = (rows + kRows - 1) / kRows;
+        indexer_scan_kernel<true><<<ctas, kThreads, kSmemBytes, st>>>(tq, tk, a);
+        DSA_LAUNCH_CHECK("indexer_scan_kernel<sample>");
+        indexer_tau_kernel<512><<<rows, 512, 0, st>>>(samp, p.samp_ld, T, S, k, row0, tau);
+        DSA_LAUNCH_CHECK("indexer_tau_kernel");
+        indexer_scan_kernel<false><<<ctas, kThreads, kSmemBytes, st>>>(tq, tk, a);
+        DSA_LAUNCH_CHECK("indexer_scan_kernel<filter>");
+        indexer_select_kernel<dsa::kSelectThreads><<<rows, dsa::kSelectThreads, 0, st>>>(
+            cand, cnt, p.cap, q_idx, w, k_idx, T, S, k, row0, idx);
+        DSA_LAUNCH_CHECK("indexer_select_kernel");
+    }
+    return DSA_OK;
+}
+
 // --------------------------------------------------------------- attention
 
 int attn_simple(const __nv_bfloat16* q, const __nv_bfloat16* kv, const int32_t* idx,
@@ -287,7 +371,7 @@ size_t dsa_workspace_size(int T, int S, int H_I, int d_I, int k, int Hq, int d_q
     (void)d_I;
     (void)d_qk;
     if (T <= 0 || S <= 0 || k <= 0 || Hq <= 0 || d_v <= 0) return 0;
-    return std::max(indexer_workspace(T, S), attn_workspace(T, Hq, d_v, k));
+    return std::max(indexer_workspace(T, S, k), attn_workspace(T, Hq, d_v, k));
 }
 
 int dsa_indexer_topk(const void* q_idx, const float* w, const void* k_idx, const int32_t* pos,
@@ -296,9 +380,13 @@ int dsa_indexer_topk(const void* q_idx, const float* w, const void* k_idx, const
 {
     g_err[0] = 0;
     if (int rc = check_indexer(q_idx, w, k_idx, pos, k_base, T, S, H_I, d_I, k, idx)) return rc;
-    const size_t need = indexer_workspace(T, S);
+    const size_t need = indexer_workspace(T, S, k);
     if (need && (!workspace || ws_bytes < need || !al16(workspace)))
         return fail(DSA_ERR_WORKSPACE, "indexer needs %zu workspace bytes (got %zu)", need, ws_bytes);
+    if (indexer_fused_supported(pos, k_base, H_I, d_I))
+        return indexer_fused(reinterpret_cast<const uint8_t*>(q_idx), w,
+                             reinterpret_cast<const uint8_t*>(k_idx), T, S, k, idx, workspace,
+                             reinterpret_cast<cudaStream_t>(stream));
     return indexer_scan_select(reinterpret_cast<const uint8_t*>(q_idx), w,
                                reinterpret_cast<const uint8_t*>(k_idx), pos, k_base, T, S, H_I, d_I,
                                k, idx, workspace, reinterpret_cast<cudaStream_t>(stream));

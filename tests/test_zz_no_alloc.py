@@ -38,7 +38,9 @@ def test_noalloc_matches_workspace_entry_point_twice(case):
                                 ctx=[131072, 9000, 70000, 8192, 120001, 33333, 4096, 100000,
                                      65536, 12345, 98765, 131071])
     else:
-        x = synth.prefill_inputs("prefill4k", device="cuda", seed=22)
+        # integer-valued FP8 inputs: every score is exact, so any two correct
+        # Top-k implementations select the same set
+        x = synth.prefill_inputs("prefill32k_int", device="cuda", seed=22, L=4096)
     assert x.S <= STATIC_MAX_S
     T, H_I, d_I = x.q_idx.shape
     ref = dsa.indexer_topk(x.q_idx, x.w, x.k_idx, x.k, pos=x.pos, k_base=x.k_base)
@@ -50,5 +52,6 @@ def test_noalloc_matches_workspace_entry_point_twice(case):
                                           _p(x.k_base), T, x.S, H_I, d_I, x.k, _p(got), stream)
         assert rc == 0, lib.dsa_last_error()
         torch.cuda.synchronize()
-        assert torch.equal(got, ref)
+        # each row is a set: compare in sorted order
+        assert torch.equal(torch.sort(got, dim=1)[0], torch.sort(ref, dim=1)[0])
     assert dsa.device_status() == 0
