@@ -53,7 +53,7 @@ def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
         return LIB
     tmp = LIB + f".tmp{os.getpid()}"
     cmd = [nvcc(), *NVCC_FLAGS, *extra_flags, "-I", INCLUDE, "-I", CSRC,
-           os.path.join(CSRC, "dsa.cu"), "-o", tmp, "-lcuda"]
+           os.path.join(CSRC, "dsa.cu"), "-o", tmp]
     if verbose:
         print(" ".join(cmd), flush=True)
     subprocess.run(cmd, check=True)

@@ -40,6 +40,26 @@ int cuda_fail(cudaError_t e, const char* where)
     return fail(DSA_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
 }
 
+// cuTensorMapEncodeTiled, looked up through the runtime so the library does
+// not link the driver library directly (it loads on machines without a GPU).
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled()
+{
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess && q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
 #define DSA_LAUNCH_CHECK(where)                                      \
     do {                                                             \
         g_launches.fetch_add(1, std::memory_order_relaxed);          \
@@ -232,7 +252,9 @@ int make_tmap_u8(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t 
     const cuuint64_t strides[1] = {row_bytes};
     const cuuint32_t box[2] = {(cuuint32_t)row_bytes, box_rows};
     const cuuint32_t estr[2] = {1, 1};
-    const CUresult r = cuTensorMapEncodeTiled(
+    EncodeTiledFn enc = encode_tiled();
+    if (!enc) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+    const CUresult r = enc(
         m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -324,7 +346,9 @@ int make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t cols, uint64_t row
     const cuuint64_t strides[1] = {cols * 2};
     const cuuint32_t box[2] = {box_cols, box_rows};
     const cuuint32_t estr[2] = {1, 1};
-    const CUresult r = cuTensorMapEncodeTiled(
+    EncodeTiledFn enc = encode_tiled();
+    if (!enc) return fail(DSA_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+    const CUresult r = enc(
         m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
         CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);

@@ -52,9 +52,10 @@ def test_abi_version_and_empty_error(lib):
 
 
 def test_workspace_sizes(lib):
-    # 128K prefill: score blocks of <= 1 GiB
+    # 128K prefill: bounded per block of query rows (sampled scores + candidate
+    # buffers of 32768 rows: 32768 * (4096 * 4 + 8192 * 8) bytes)
     ws = dsa.workspace_size(131072, 131072, 8, 128, 2048, 128, 576, 512)
-    assert 0 < ws <= (1 << 30) + 4096
+    assert 0 < ws <= 32768 * (4096 * 4 + 8192 * 8) + (1 << 20)
     assert dsa.workspace_size(0, 10, 8, 128, 2048, 128, 576, 512) == 0
     small = dsa.workspace_size(256, 256, 4, 32, 32, 4, 80, 64)
     assert small >= 256 * 256 * 4
