@@ -285,12 +285,13 @@ int indexer_fused(const uint8_t* q_idx, const float* w, const uint8_t* k_idx, in
         const int ctas = (rows + kRows - 1) / kRows;
         indexer_scan_kernel<true><<<ctas, kThreads, kSmemBytes, st>>>(tq, tk, a);
         DSA_LAUNCH_CHECK("indexer_scan_kernel<sample>");
-        indexer_tau_kernel<512><<<rows, 512, 0, st>>>(samp, p.samp_ld, T, S, k, row0, tau);
+        indexer_tau_kernel<256><<<rows, 256, 0, st>>>(samp, p.samp_ld, T, S, k, row0, tau);
         DSA_LAUNCH_CHECK("indexer_tau_kernel");
         indexer_scan_kernel<false><<<ctas, kThreads, kSmemBytes, st>>>(tq, tk, a);
         DSA_LAUNCH_CHECK("indexer_scan_kernel<filter>");
-        indexer_select_kernel<dsa::kSelectThreads><<<rows, dsa::kSelectThreads, 0, st>>>(
-            cand, cnt, p.cap, q_idx, w, k_idx, T, S, k, row0, idx);
+        // ~2k candidates per row: 256 threads keep the radix passes busy
+        indexer_select_kernel<256><<<rows, 256, 0, st>>>(cand, cnt, p.cap, q_idx, w, k_idx, T, S, k,
+                                                         row0, idx);
         DSA_LAUNCH_CHECK("indexer_select_kernel");
     }
     return DSA_OK;

@@ -21,9 +21,10 @@
 // high) or overflowed are recomputed exactly in the same select kernel, so
 // the result never depends on the sampling.
 //
-// Warp roles (384 threads): warp 0 TMA, warp 1 MMA (one thread), warps 4-11
-// two epilogue groups of four warps, each owning one of the two TMEM buffers
-// (alternate key tiles).
+// Warp roles (640 threads): warp 0 TMA, warp 1 MMA (one thread), warps 4-19
+// four epilogue groups of four warps: groups 0/1 share TMEM buffer 0 (even
+// key tiles), groups 2/3 buffer 1 (odd tiles); within a pair each group takes
+// 16 of the 32 query rows.
 #pragma once
 #include <cuda.h>
 
@@ -41,7 +42,7 @@ constexpr int kRows = 32;         // query rows per CTA (N = 32 * 8 = 256)
 constexpr int kN = kRows * kHI;
 constexpr int kKeys = 128;        // keys per tile (M)
 constexpr int kStages = 6;
-constexpr int kThreads = 384;
+constexpr int kThreads = 640;            // 20 warps: TMA, MMA, 2 idle, 16 epilogue
 constexpr int kQBytes = kN * kDI;             // 32 KB
 constexpr int kTileBytes = kKeys * kDI;       // 16 KB
 constexpr int kOffQ = 0;
@@ -58,6 +59,7 @@ enum : int { B_Q = 0, B_KFULL = 1, B_KEMPTY = 1 + kStages, B_DFULL = 1 + 2 * kSt
 
 static_assert(kOffK % 1024 == 0 && kTileBytes % 1024 == 0, "alignment");
 static_assert(kSmemBytes <= 232448, "shared memory");
+static_assert(kThreads == 32 * (4 + 16), "four role warps + four epilogue groups of four warps");
 
 // Sampling: every kSampleStride-th key tile is scored in the sample pass; a
 // row keeps about kAlpha * k candidates in the filter pass.
@@ -119,7 +121,7 @@ indexer_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(bar(B_DFULL + b), 1);
-            mbar_init(bar(B_DEMPTY + b), 4);
+            mbar_init(bar(B_DEMPTY + b), 8);   // two groups of four warps per buffer
         }
         mbar_init(bar(B_DRAIN), 1);
         *abort_flag = 0;
@@ -190,7 +192,9 @@ indexer_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
     } else if (warp >= 4) {
         // -------------------------------------------------------- epilogue
-        const int g = (warp - 4) >> 2;                     // TMEM buffer / tile parity
+        const int grp = (warp - 4) >> 2;                   // epilogue group 0..3
+        const int g = grp >> 1;                            // TMEM buffer / tile parity
+        const int rh = grp & 1;                            // row half: rows [16rh, 16rh+16)
         const int key_lane = (warp & 3) * 32 + lane;       // key within the tile
         const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
         for (int it = g; it < NIT; it += 2) {
@@ -201,12 +205,12 @@ indexer_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             // eight rows at a time: two TMEM loads (4 rows x 8 heads each), the
             // weighted ReLU head-sums, then the rows' mask / sample / filter step
 #pragma unroll 1
-            for (int q8 = 0; q8 < kRows / 4; q8 += 2) {
+            for (int q8 = 4 * rh; q8 < 4 * rh + 4; q8 += 2) {
                 uint32_t v0[32], v1[32];
                 tmem_ld32(tmem + lane_addr + g * 256 + q8 * 32, v0);
                 tmem_ld32(tmem + lane_addr + g * 256 + q8 * 32 + 32, v1);
                 tmem_wait_ld();
-                if (q8 == kRows / 4 - 2) {
+                if (q8 == 4 * rh + 2) {
                     // every column of this buffer has been read: hand it back
                     tc_fence_before();
                     __syncwarp();
