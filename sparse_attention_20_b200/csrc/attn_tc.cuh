@@ -48,12 +48,16 @@ constexpr int kStages = 4;
 constexpr int kThreads = 416;               // 13 warps: QK, 3 gather, 8 softmax, PV
 constexpr int kGatherThreads = 96;
 
-constexpr int kQBytes = kHeads * 64;       // rope slice of Q: 32 columns, 64B swizzle
+constexpr int kQSlab = kHeads * 128;        // 64 latent columns x 128 heads, 128B swizzle
+// Q in shared memory: latent columns [128, 256) of this CTA's slice (two
+// slabs) and the rope slice (32 columns, 64B swizzle). Latent columns [0, 128)
+// live in TMEM.
+constexpr int kQBytes = 2 * kQSlab + kHeads * 64;
 constexpr int kKSlab = kKeys * 128;
 constexpr int kStageBytes = 4 * kKSlab + kKeys * 64;
 constexpr int kXBytes = kHeads * 128;       // 64 fp16 partial logits per head
 constexpr int kOffQ = 0;
-constexpr int kOffKV = kOffQ + 8192;       // (kQBytes, rounded to 1 KB)
+constexpr int kOffKV = kOffQ + kQBytes;
 constexpr int kOffX = kOffKV + kStages * kStageBytes;
 constexpr int kOffBar = kOffX + 2 * kXBytes;
 constexpr int kOffMask = kOffBar + 256;                 // [kStages][2] validity bits
@@ -63,16 +67,17 @@ constexpr int kOffRows = kOffLsum + 2 * kHeads * 4;     // [3 gather warps][64] 
 constexpr int kSmemBytes = kOffRows + 3 * kKeys * 8 + 1024;  // + 1 KB alignment slack
 
 constexpr uint32_t kTmemCols = 512;
-// O [0,256); S double buffer [256,384) (P(c) overwrites the first half of
-// each key half's S columns once read); latent Q slice [384,512).
-constexpr uint32_t kColO = 0, kColS = 256, kColQ = 384;
+// O [0,256); S double buffer [256,384); latent Q columns [0,128) of the
+// slice [384,448); P double buffer (bf16 pairs) [448,512).
+constexpr uint32_t kColO = 0, kColS = 256, kColQ = 384, kColP = 448;
 
 enum : int {
     B_Q = 0, B_QT = 1, B_FULL = 2, B_EMPTY = 6, B_SFULL = 10, B_PFULL = 12, B_PVDONE = 14,
-    B_XFULL = 16, B_XFREE = 18, B_DRAIN = 20, B_RED = 21, B_LSUM = 23, B_COUNT = 24
+    B_XFULL = 16, B_XFREE = 18, B_DRAIN = 20, B_RED = 21, B_LSUM = 23, B_SFREE = 24, B_COUNT = 26
 };
 
 static_assert(kOffKV % 1024 == 0 && kStageBytes % 1024 == 0 && kOffX % 1024 == 0, "alignment");
+static_assert(8 * B_COUNT + 16 <= 256, "barrier area");
 static_assert(kSmemBytes <= 232448, "shared memory");
 
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi)
@@ -102,7 +107,8 @@ __device__ __forceinline__ int piece_col(uint32_t rank, int j)
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q64,
+sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
+                          const __grid_constant__ CUtensorMap tm_q64,
                           const __nv_bfloat16* __restrict__ q,
                           const __nv_bfloat16* __restrict__ kv,
                           const int* __restrict__ idx, const int* __restrict__ pos,
@@ -131,6 +137,7 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q64,
     if (threadIdx.x == 0) {
         mbar_init(bar(B_Q), 1);
         mbar_init(bar(B_QT), 8);        // latent Q written to TMEM by the softmax warps
+        for (int b = 0; b < 2; ++b) mbar_init(bar(B_SFREE + b), 8);   // S(c) read by every softmax warp
         for (int s = 0; s < kStages; ++s) {
             // every gather thread's cp.async arrival + the mask publisher
             mbar_init(bar(B_FULL + s), kGatherThreads + 1);
@@ -169,9 +176,9 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q64,
             for (int c = 0; ok && c < NC; ++c) {
                 const int st = c % kStages;
                 ok = mbar_wait(bar(B_FULL + st), (c / kStages) & 1, abort_flag, B_FULL, c);
-                // S(c) reuses the buffer of chunk c-2, whose P that PV(c-2) read
+                // S(c) reuses the buffer of chunk c-2 once the softmax has read it
                 if (ok && c >= 2)
-                    ok = mbar_wait(bar(B_PVDONE + (c & 1)), ((c - 2) >> 1) & 1, abort_flag, B_PVDONE, c);
+                    ok = mbar_wait(bar(B_SFREE + (c & 1)), ((c - 2) >> 1) & 1, abort_flag, B_SFREE, c);
                 if (!ok) break;
                 // the stage was written by cp.async (generic proxy); the MMA
                 // reads it through the async proxy
@@ -179,16 +186,23 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q64,
                 tc_fence_after();
                 const uint32_t kvs = sbase + kOffKV + st * kStageBytes;
                 const uint32_t d = tmem + kColS + (c & 1) * kKeys;
-                // latent part: A = Q slice in TMEM (16 K-steps of 16 columns)
+                // latent columns [0,128) of the slice: A = Q in TMEM (8 K-steps)
 #pragma unroll
-                for (int kk = 0; kk < 16; ++kk) {
+                for (int kk = 0; kk < 8; ++kk) {
                     const uint64_t bd = smem_desc(kvs + (kk >> 2) * kKSlab + (kk & 3) * 32, 16, 1024, kSwizzle128B);
                     mma_f16_ts(d, tmem + kColQ + kk * 8, bd, id_qk, kk > 0 ? 1u : 0u);
+                }
+                // latent columns [128,256): A = Q in shared memory (8 K-steps)
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint64_t ad = smem_desc(qs + (kk >> 2) * kQSlab + (kk & 3) * 32, 16, 1024, kSwizzle128B);
+                    const uint64_t bd = smem_desc(kvs + (2 + (kk >> 2)) * kKSlab + (kk & 3) * 32, 16, 1024, kSwizzle128B);
+                    mma_f16_ss(d, ad, bd, id_qk, 1u);
                 }
                 // rope part: A = Q rope slice in shared memory
 #pragma unroll
                 for (int kk = 0; kk < 2; ++kk) {
-                    const uint64_t ad = smem_desc(qs + kk * 32, 16, 512, kSwizzle64B);
+                    const uint64_t ad = smem_desc(qs + 2 * kQSlab + kk * 32, 16, 512, kSwizzle64B);
                     const uint64_t bd = smem_desc(kvs + 4 * kKSlab + kk * 32, 16, 512, kSwizzle64B);
                     mma_f16_ss(d, ad, bd, id_qk, 1u);
                 }
@@ -208,8 +222,7 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q64,
                     // B = gathered rows read MN-major: 64 values per 128-byte row,
                     // LBO = next 64 columns (slab), SBO = next 8 keys.
                     const uint64_t bd = smem_desc(kvs + kk * 16 * 128, kKSlab, 1024, kSwizzle128B);
-                    // P of keys [32h, 32h+32) sits in the first 16 columns of that half's S
-                    mma_f16_ts(tmem + kColO, tmem + kColS + (c & 1) * kKeys + (kk >> 1) * 32 + (kk & 1) * 8, bd, id_pv,
+                    mma_f16_ts(tmem + kColO, tmem + kColP + (c & 1) * 32 + kk * 8, bd, id_pv,
                                (c > 0 || kk > 0) ? 1u : 0u);
                 }
                 mma_commit(bar(B_PVDONE + (c & 1)));
@@ -227,9 +240,12 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q64,
         const int gw = warp - 1;
         const int g = threadIdx.x - 32;
         if (gw == 0 && lane == 0) {
+            prefetch_tmap(&tm_q128);
             prefetch_tmap(&tm_q64);
             mbar_arrive_expect_tx(bar(B_Q), kQBytes);
-            tma_load_2d(qs, &tm_q64, 512 + (int)rank * 32, t * kHeads, bar(B_Q));
+            for (int j = 0; j < 2; ++j)
+                tma_load_2d(qs + j * kQSlab, &tm_q128, (int)rank * 256 + 128 + j * 64, t * kHeads, bar(B_Q));
+            tma_load_2d(qs + 2 * kQSlab, &tm_q64, 512 + (int)rank * 32, t * kHeads, bar(B_Q));
         }
         const int* idx_row = idx + (size_t)t * k;
         uint32_t* smask = reinterpret_cast<uint32_t*>(sgen + kOffMask);
@@ -332,20 +348,18 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q64,
         };
 
         {
-            // latent Q slice of head i into TMEM (A operand of the QK MMAs):
-            // this half's 128 columns, two bf16 per 32-bit column
+            // latent Q columns [0,128) of the slice for head i into TMEM (A
+            // operand of the QK MMAs): this half's 64 columns, two bf16 per
+            // 32-bit TMEM column
             const uint4* qsrc = reinterpret_cast<const uint4*>(
-                q + ((size_t)t * kHeads + i) * kDqk + rank * 256 + 128 * hs);
+                q + ((size_t)t * kHeads + i) * kDqk + rank * 256 + 64 * hs);
+            uint32_t w[32];
 #pragma unroll
-            for (int part = 0; part < 2; ++part) {
-                uint32_t w[32];
-#pragma unroll
-                for (int v = 0; v < 8; ++v) {
-                    const uint4 x = __ldg(qsrc + part * 8 + v);
-                    w[4 * v] = x.x; w[4 * v + 1] = x.y; w[4 * v + 2] = x.z; w[4 * v + 3] = x.w;
-                }
-                tmem_st32(tmem + lane_addr + kColQ + 64 * hs + 32 * part, w);
+            for (int v = 0; v < 8; ++v) {
+                const uint4 x = __ldg(qsrc + v);
+                w[4 * v] = x.x; w[4 * v + 1] = x.y; w[4 * v + 2] = x.z; w[4 * v + 3] = x.w;
             }
+            tmem_st32(tmem + lane_addr + kColQ + 32 * hs, w);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
@@ -379,6 +393,9 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q64,
             uint32_t sr[32];
             tmem_ld32(tmem + lane_addr + kColS + b * kKeys + 32 * hs, sr);
             tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(B_SFREE + b));   // S(c) fully read by this warp
             if (!wait_w(bar(B_FULL + c % kStages), (c / kStages) & 1, 200 + B_FULL, c, false)) { ok = false; break; }
             const uint32_t mw = smask[(c % kStages) * 2 + hs];
             // logit (log2 domain) = own partial (fp32) + peer partial (fp16); masked -> -inf
@@ -456,8 +473,13 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q64,
 #pragma unroll
                 for (int j = 0; j < w; ++j) ps[j] += ps[j + w];
             l += ps[0];
+            // P buffer b is free once PV(c-2) has read it
+            if (c >= 2 && !wait_w(bar(B_PVDONE + b), ((c - 2) >> 1) & 1, 200 + B_PVDONE, c, false)) {
+                ok = false;
+                break;
+            }
             tc_fence_after();
-            tmem_st16(tmem + lane_addr + kColS + b * kKeys + 32 * hs, pk);   // over this half's S
+            tmem_st16(tmem + lane_addr + kColP + b * 32 + 16 * hs, pk);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();

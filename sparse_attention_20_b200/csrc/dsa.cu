@@ -365,15 +365,17 @@ int attn_tc(const __nv_bfloat16* q, const __nv_bfloat16* kv, const int32_t* idx,
     cudaError_t e = cudaFuncSetAttribute(sparse_mla_attn_tc_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(sparse_mla_attn_tc_kernel)");
-    // Q as [T*128, 576]; the rope slice goes to shared memory by TMA (one
-    // 128-head box of 32 columns, 64B swizzle); the latent slice is written
-    // to TMEM by the kernel itself.
-    CUtensorMap tq64;
+    // Q as [T*128, 576]: TMA boxes of 128 heads; 64 latent columns with 128B
+    // swizzle, the 32 rope columns with 64B swizzle. Half of the latent slice
+    // is written to TMEM by the kernel itself.
+    CUtensorMap tq128, tq64;
+    if (int rc = make_tmap_bf16(&tq128, q, kDqk, (uint64_t)T * kHeads, 64, kHeads,
+                                CU_TENSOR_MAP_SWIZZLE_128B)) return rc;
     if (int rc = make_tmap_bf16(&tq64, q, kDqk, (uint64_t)T * kHeads, 32, kHeads,
                                 CU_TENSOR_MAP_SWIZZLE_64B)) return rc;
     const float scale_log2 = scale * 1.4426950408889634f;
     sparse_mla_attn_tc_kernel<<<dim3(2 * T), kThreads, kSmemBytes, st>>>(
-        tq64, q, kv, idx, pos, k_base, T, S, k, scale_log2, out, lse);
+        tq128, tq64, q, kv, idx, pos, k_base, T, S, k, scale_log2, out, lse);
     DSA_LAUNCH_CHECK("sparse_mla_attn_tc_kernel");
     return DSA_OK;
 }
