@@ -26,10 +26,13 @@
 // shared memory (3-stage ring of 64-row chunks; completion is counted on the
 // stage's mbarrier, so the gather runs up to three chunks ahead); warps 4-11
 // (two per TMEM lane quarter, each taking 32 of a chunk's 64 keys) run the
-// softmax, the exchange (st.async into the peer's shared memory, counted on
-// the peer's mbarrier) and the epilogue.
-// Shared memory per CTA: Q slice 72 KB + 3 x 36 KB ring + 2 x 16 KB exchange.
-// TMEM: O cols [0,256), S double buffer [256,384), P (bf16 pairs) [384,448).
+// softmax, the exchange (each warp stages its fp16 partial logits locally and
+// sends them with one bulk copy into the peer's shared memory, counted on the
+// peer's mbarrier) and the epilogue.
+// Shared memory per CTA: Q 40 KB (latent columns 128..255 of the slice and the
+// rope slice) + 3 x 36 KB ring + 2 x 16 KB receive slots + 2 x 16 KB staging.
+// TMEM: O cols [0,256), S double buffer [256,384), latent Q [384,448), P
+// (bf16 pairs) double buffer [448,512).
 #pragma once
 #include <cuda.h>
 
@@ -44,7 +47,7 @@ constexpr int kHeads = 128;
 constexpr int kDqk = 576;
 constexpr int kDv = 512;
 constexpr int kKeys = 64;
-constexpr int kStages = 4;
+constexpr int kStages = 3;
 constexpr int kThreads = 416;               // 13 warps: QK, 3 gather, 8 softmax, PV
 constexpr int kGatherThreads = 96;
 
@@ -55,11 +58,17 @@ constexpr int kQSlab = kHeads * 128;        // 64 latent columns x 128 heads, 12
 constexpr int kQBytes = 2 * kQSlab + kHeads * 64;
 constexpr int kKSlab = kKeys * 128;
 constexpr int kStageBytes = 4 * kKSlab + kKeys * 64;
-constexpr int kXBytes = kHeads * 128;       // 64 fp16 partial logits per head
+// Exchange slot: fp16 partial logits of one chunk, [key half][head][32 keys],
+// 64 B per head and half with the four 16 B pieces rotated by (head >> 1).
+// One softmax warp owns a contiguous 2 KB run (one half, 32 heads), sent as a
+// single bulk copy.
+constexpr int kXBytes = kHeads * 128;
+constexpr int kXWarpBytes = 32 * 64;
 constexpr int kOffQ = 0;
 constexpr int kOffKV = kOffQ + kQBytes;
 constexpr int kOffX = kOffKV + kStages * kStageBytes;
-constexpr int kOffBar = kOffX + 2 * kXBytes;
+constexpr int kOffXS = kOffX + 2 * kXBytes;               // staging of outgoing slots
+constexpr int kOffBar = kOffXS + 2 * kXBytes;
 constexpr int kOffMask = kOffBar + 256;                 // [kStages][2] validity bits
 constexpr int kOffRed = kOffMask + 64;                  // [2 parity][2 halves][128] row maxima
 constexpr int kOffLsum = kOffRed + 2 * 2 * kHeads * 4;  // [2 halves][128] row sums
@@ -309,6 +318,10 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
         const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
         const uint32_t xs = sbase + kOffX;
         const uint32_t x_peer = mapa(xs, peer);
+        // this warp's 2 KB run inside a slot; head i's 64 B row within it
+        const uint32_t xwarp = (uint32_t)(hs * 4 + (warp & 3)) * kXWarpBytes;
+        const uint32_t xrow = xwarp + (uint32_t)lane * 64;
+        const uint32_t xstage = sbase + kOffXS;
         const uint32_t xfull_peer = mapa(bar(B_XFULL), peer);
         const uint32_t xfree_peer = mapa(bar(B_XFREE), peer);
         const uint32_t* smask = reinterpret_cast<const uint32_t*>(sgen + kOffMask);
@@ -336,14 +349,18 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
             for (int j = 0; j < 16; ++j)
                 h[j] = pack_half2(__uint_as_float(sr[2 * j]) * scale_log2,
                                   __uint_as_float(sr[2 * j + 1]) * scale_log2);
-            // the peer has consumed chunk c-2 from this slot (a pure signal)
+            // The peer has consumed chunk c-2 from its slot b, so the bulk copy
+            // of c-2 has landed: it has also finished reading staging slot b.
             if (c >= 2 && !wait_w(bar(B_XFREE + b), ((c - 2) >> 1) & 1, 200 + B_XFREE, c, false)) return false;
-            const uint32_t xr_peer = x_peer + b * kXBytes + i * 128;
+            const uint32_t stg = xstage + b * kXBytes;
 #pragma unroll
             for (int m = 0; m < 4; ++m)
-                st_async_v4(xr_peer + (((4 * hs + m + i) & 7) << 4),
-                            make_uint4(h[4 * m], h[4 * m + 1], h[4 * m + 2], h[4 * m + 3]),
-                            xfull_peer + 8u * b);
+                st_shared_v4(stg + xrow + (((m + (lane >> 1)) & 3) << 4),
+                             make_uint4(h[4 * m], h[4 * m + 1], h[4 * m + 2], h[4 * m + 3]));
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0)
+                bulk_s2cluster(x_peer + b * kXBytes + xwarp, stg + xwarp, kXWarpBytes, xfull_peer + 8u * b);
             return true;
         };
 
@@ -381,13 +398,13 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
                 sent = c + 2;
             }
             if (i == 0 && hs == 0) mbar_arrive_expect_tx(bar(B_XFULL + b), kXBytes);
-            // the peer's bytes arrive by st.async, counted on this local barrier
+            // the peer's bytes arrive by bulk copy, counted on this local barrier
             if (!wait_w(bar(B_XFULL + b), (c >> 1) & 1, 200 + B_XFULL, c, false)) { ok = false; break; }
             uint32_t g[16];
-            const uint32_t xr = xs + b * kXBytes + i * 128;
+            const uint32_t xr = xs + b * kXBytes + xrow;
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
-                const uint4 v = ld_shared_v4(xr + (((4 * hs + m + i) & 7) << 4));
+                const uint4 v = ld_shared_v4(xr + (((m + (lane >> 1)) & 3) << 4));
                 g[4 * m] = v.x; g[4 * m + 1] = v.y; g[4 * m + 2] = v.z; g[4 * m + 3] = v.w;
             }
             uint32_t sr[32];
