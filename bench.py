@@ -44,6 +44,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--prefill", default="prefill128k")
     ap.add_argument("--decode", default="decode")
+    ap.add_argument("--seq-len", type=int, default=None,
+                    help="override L of the prefill workload (smaller cases for profiling)")
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -246,7 +248,8 @@ def bench_ours(args, world, rank, local):
     barrier(world)
     dsa.load_library()
     dev = torch.device("cuda", torch.cuda.current_device())
-    xp = synth.make_inputs(args.prefill, device=dev, seed=args.seed + rank)
+    xp = synth.make_inputs(args.prefill, device=dev, seed=args.seed + rank,
+                           **({"L": args.seq_len} if args.seq_len else {}))
     xd = synth.make_inputs(args.decode, device=dev, seed=args.seed + rank)
     bp, bd = Batch(xp, dsa), Batch(xd, dsa)
     stream = torch.cuda.current_stream()
@@ -310,8 +313,9 @@ def bench_ours(args, world, rank, local):
         "data": "synthetic (seeded; shapes and distributions of the pages' 128K workloads)",
         "config": {"workload": f"{args.prefill} causal prefill (L={xp.T}, H_I={bp.H_I}, "
                                f"d_I={bp.d_I}, k={xp.k}, Hq={bp.Hq}, d_qk={bp.d_qk}, "
-                               f"d_v={xp.d_v}) + {args.decode} step ({xd.T} seqs, "
-                               f"ctx U[8192,131072])",
+                               f"d_v={xp.d_v}) + {args.decode} step ({xd.T} "
+                               + ("seqs, ctx U[8192,131072])" if args.decode == "decode"
+                                  else "rows)"),
                    "global_batch": world, "seq_len": xp.T, "parallelism": f"replicas{world}",
                    "l2": "inputs larger than L2 (19 GB of queries, 151 MB latent cache)"},
         "prefill_tokens_per_s": tokens / (prefill_ms * 1e-3),
@@ -400,7 +404,8 @@ def bench_reference(args, world, rank):
     """The CPU oracle as the reference arm, on bounded samples of the same workload."""
     import oracle
     dev = "cuda" if torch.cuda.is_available() else "cpu"
-    x = synth.make_inputs(args.prefill, device=dev, seed=args.seed)
+    x = synth.make_inputs(args.prefill, device=dev, seed=args.seed,
+                          **({"L": args.seq_len} if args.seq_len else {}))
     threads = oracle.num_threads()
     g = torch.Generator().manual_seed(args.seed)
     per_step = max(2, threads)

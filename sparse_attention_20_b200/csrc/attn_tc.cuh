@@ -19,16 +19,17 @@
 // gathered rows read MN-major, N = 256). No flop is done twice and every
 // selected row crosses HBM/L2 once per query.
 //
-// Warp roles (416 threads per CTA): warp 0 allocates TMEM and issues the QK
-// MMAs (one thread); warp 12 issues the PV MMAs (one thread), so a late chunk
-// never holds back the PV of the previous one; warps 1-3 load Q (TMA tiles)
+// Warp roles (512 threads per CTA): warp 0 allocates TMEM and issues the QK
+// and PV MMAs (one thread polling both kinds of readiness, so a late chunk
+// never holds back the PV of the previous one); warps 1-3 load Q (TMA tiles)
 // and gather the selected rows with 16-byte cp.async into 128B/64B-swizzled
 // shared memory (3-stage ring of 64-row chunks; completion is counted on the
-// stage's mbarrier, so the gather runs up to three chunks ahead); warps 4-11
-// (two per TMEM lane quarter, each taking 32 of a chunk's 64 keys) run the
-// softmax, the exchange (each warp stages its fp16 partial logits locally and
-// sends them with one bulk copy into the peer's shared memory, counted on the
-// peer's mbarrier) and the epilogue.
+// stage's mbarrier, so the gather runs up to three chunks ahead); warps 12-15
+// (one per TMEM lane quarter) run the exchange: they stage the chunk's fp16
+// partial logits locally and send them with one bulk copy per warp into the
+// peer's shared memory, counted on the peer's mbarrier; warps 4-11 (two per
+// lane quarter, each taking 32 of a chunk's 64 keys) run the softmax and the
+// epilogue.
 // Shared memory per CTA: Q 40 KB (latent columns 128..255 of the slice and the
 // rope slice) + 3 x 36 KB ring + 2 x 16 KB receive slots + 2 x 16 KB staging.
 // TMEM: O cols [0,256), S double buffer [256,384), latent Q [384,448), P
@@ -48,7 +49,7 @@ constexpr int kDqk = 576;
 constexpr int kDv = 512;
 constexpr int kKeys = 64;
 constexpr int kStages = 3;
-constexpr int kThreads = 416;               // 13 warps: QK, 3 gather, 8 softmax, PV
+constexpr int kThreads = 512;               // 16 warps: MMA, 3 gather, 8 softmax, 4 senders
 constexpr int kGatherThreads = 96;
 
 constexpr int kQSlab = kHeads * 128;        // 64 latent columns x 128 heads, 128B swizzle
@@ -58,12 +59,11 @@ constexpr int kQSlab = kHeads * 128;        // 64 latent columns x 128 heads, 12
 constexpr int kQBytes = 2 * kQSlab + kHeads * 64;
 constexpr int kKSlab = kKeys * 128;
 constexpr int kStageBytes = 4 * kKSlab + kKeys * 64;
-// Exchange slot: fp16 partial logits of one chunk, [key half][head][32 keys],
-// 64 B per head and half with the four 16 B pieces rotated by (head >> 1).
-// One softmax warp owns a contiguous 2 KB run (one half, 32 heads), sent as a
-// single bulk copy.
+// Exchange slot: fp16 partial logits of one chunk, [head][64 keys], 128 B per
+// head with the eight 16 B pieces rotated by the head index. One sender warp
+// owns the contiguous 4 KB of its 32 heads and sends them as one bulk copy.
 constexpr int kXBytes = kHeads * 128;
-constexpr int kXWarpBytes = 32 * 64;
+constexpr int kXWarpBytes = 32 * 128;
 constexpr int kOffQ = 0;
 constexpr int kOffKV = kOffQ + kQBytes;
 constexpr int kOffX = kOffKV + kStages * kStageBytes;
@@ -115,6 +115,13 @@ __device__ __forceinline__ int piece_col(uint32_t rank, int j)
     return j < 32 ? (int)rank * 256 + j * 8 : 512 + (int)rank * 32 + (j - 32) * 8;
 }
 
+// Bounded wait whose outcome is the same for the whole warp.
+__device__ __forceinline__ bool wait_warp(uint32_t b_addr, uint32_t par, volatile int* abort_flag,
+                                          int tag, int c)
+{
+    return __all_sync(0xffffffffu, mbar_wait(b_addr, par, abort_flag, tag, c));
+}
+
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
                           const __grid_constant__ CUtensorMap tm_q64,
@@ -146,7 +153,8 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
     if (threadIdx.x == 0) {
         mbar_init(bar(B_Q), 1);
         mbar_init(bar(B_QT), 8);        // latent Q written to TMEM by the softmax warps
-        for (int b = 0; b < 2; ++b) mbar_init(bar(B_SFREE + b), 8);   // S(c) read by every softmax warp
+        // S(c) read by every softmax and sender warp
+        for (int b = 0; b < 2; ++b) mbar_init(bar(B_SFREE + b), 12);
         for (int s = 0; s < kStages; ++s) {
             // every gather thread's cp.async arrival + the mask publisher
             mbar_init(bar(B_FULL + s), kGatherThreads + 1);
@@ -156,11 +164,11 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
             mbar_init(bar(B_SFULL + b), 1);
             mbar_init(bar(B_PFULL + b), 8);
             mbar_init(bar(B_PVDONE + b), 1);
-            mbar_init(bar(B_XFULL + b), 1);   // receiver's expect_tx + the peer's bytes
+            mbar_init(bar(B_XFULL + b), 1);   // receiver's expect_tx + the peer senders' bytes
             mbar_init(bar(B_XFREE + b), 8);   // one arrival per softmax warp of the peer
             mbar_init(bar(B_RED + b), 8);
         }
-        mbar_init(bar(B_DRAIN), 2);     // QK and PV issuers
+        mbar_init(bar(B_DRAIN), 1);     // the MMA issuer
         mbar_init(bar(B_LSUM), 8);
         *abort_flag = 0;
         fence_mbar_init_cluster();
@@ -177,65 +185,77 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
     const uint32_t qs = sbase + kOffQ;
 
     if (warp == 0) {
-        // --------------------------------------------------------- QK MMAs
+        // ------------------------------------------------- QK and PV MMAs
+        // One thread issues both: QK(c) once chunk c is gathered and its S
+        // buffer has been read (chunk c-2), PV(c) once the softmax has written
+        // P(c). Readiness is polled without blocking so that neither kind of
+        // MMA waits behind the other; the tensor pipe runs them in issue order.
         if (lane == 0 && NC > 0) {
             const uint32_t id_qk = idesc_bf16(128, kKeys, false);
+            const uint32_t id_pv = idesc_bf16(128, 256, true);
             bool ok = mbar_wait(bar(B_Q), 0, abort_flag, B_Q, 0) &&
                       mbar_wait(bar(B_QT), 0, abort_flag, B_QT, 0);
-            for (int c = 0; ok && c < NC; ++c) {
-                const int st = c % kStages;
-                ok = mbar_wait(bar(B_FULL + st), (c / kStages) & 1, abort_flag, B_FULL, c);
-                // S(c) reuses the buffer of chunk c-2 once the softmax has read it
-                if (ok && c >= 2)
-                    ok = mbar_wait(bar(B_SFREE + (c & 1)), ((c - 2) >> 1) & 1, abort_flag, B_SFREE, c);
-                if (!ok) break;
-                // the stage was written by cp.async (generic proxy); the MMA
-                // reads it through the async proxy
-                fence_proxy_async_smem();
-                tc_fence_after();
-                const uint32_t kvs = sbase + kOffKV + st * kStageBytes;
-                const uint32_t d = tmem + kColS + (c & 1) * kKeys;
-                // latent columns [0,128) of the slice: A = Q in TMEM (8 K-steps)
+            int cq = 0, cp = 0;              // next chunk for QK / for PV
+            uint64_t t_idle = globaltimer_ns();
+            while (ok && cp < NC) {
+                bool progressed = false;
+                if (cq < NC && mbar_test_wait(bar(B_FULL + cq % kStages), (cq / kStages) & 1) &&
+                    (cq < 2 || mbar_test_wait(bar(B_SFREE + (cq & 1)), ((cq - 2) >> 1) & 1))) {
+                    const int c = cq++;
+                    // the stage was written by cp.async (generic proxy); the MMA
+                    // reads it through the async proxy
+                    fence_proxy_async_smem();
+                    tc_fence_after();
+                    const uint32_t kvs = sbase + kOffKV + (c % kStages) * kStageBytes;
+                    const uint32_t d = tmem + kColS + (c & 1) * kKeys;
+                    // latent columns [0,128) of the slice: A = Q in TMEM (8 K-steps)
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint64_t bd = smem_desc(kvs + (kk >> 2) * kKSlab + (kk & 3) * 32, 16, 1024, kSwizzle128B);
-                    mma_f16_ts(d, tmem + kColQ + kk * 8, bd, id_qk, kk > 0 ? 1u : 0u);
-                }
-                // latent columns [128,256): A = Q in shared memory (8 K-steps)
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint64_t bd = smem_desc(kvs + (kk >> 2) * kKSlab + (kk & 3) * 32, 16, 1024, kSwizzle128B);
+                        mma_f16_ts(d, tmem + kColQ + kk * 8, bd, id_qk, kk > 0 ? 1u : 0u);
+                    }
+                    // latent columns [128,256): A = Q in shared memory (8 K-steps)
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint64_t ad = smem_desc(qs + (kk >> 2) * kQSlab + (kk & 3) * 32, 16, 1024, kSwizzle128B);
-                    const uint64_t bd = smem_desc(kvs + (2 + (kk >> 2)) * kKSlab + (kk & 3) * 32, 16, 1024, kSwizzle128B);
-                    mma_f16_ss(d, ad, bd, id_qk, 1u);
-                }
-                // rope part: A = Q rope slice in shared memory
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint64_t ad = smem_desc(qs + (kk >> 2) * kQSlab + (kk & 3) * 32, 16, 1024, kSwizzle128B);
+                        const uint64_t bd = smem_desc(kvs + (2 + (kk >> 2)) * kKSlab + (kk & 3) * 32, 16, 1024, kSwizzle128B);
+                        mma_f16_ss(d, ad, bd, id_qk, 1u);
+                    }
+                    // rope part: A = Q rope slice in shared memory
 #pragma unroll
-                for (int kk = 0; kk < 2; ++kk) {
-                    const uint64_t ad = smem_desc(qs + 2 * kQSlab + kk * 32, 16, 512, kSwizzle64B);
-                    const uint64_t bd = smem_desc(kvs + 4 * kKSlab + kk * 32, 16, 512, kSwizzle64B);
-                    mma_f16_ss(d, ad, bd, id_qk, 1u);
+                    for (int kk = 0; kk < 2; ++kk) {
+                        const uint64_t ad = smem_desc(qs + 2 * kQSlab + kk * 32, 16, 512, kSwizzle64B);
+                        const uint64_t bd = smem_desc(kvs + 4 * kKSlab + kk * 32, 16, 512, kSwizzle64B);
+                        mma_f16_ss(d, ad, bd, id_qk, 1u);
+                    }
+                    mma_commit(bar(B_SFULL + (c & 1)));
+                    progressed = true;
                 }
-                mma_commit(bar(B_SFULL + (c & 1)));
-            }
-        }
-    } else if (warp == 12) {
-        // --------------------------------------------------------- PV MMAs
-        if (lane == 0 && NC > 0) {
-            const uint32_t id_pv = idesc_bf16(128, 256, true);
-            for (int c = 0; c < NC; ++c) {
-                if (!mbar_wait(bar(B_PFULL + (c & 1)), (c >> 1) & 1, abort_flag, B_PFULL, c)) break;
-                tc_fence_after();
-                const uint32_t kvs = sbase + kOffKV + (c % kStages) * kStageBytes;
+                if (cp < cq && mbar_test_wait(bar(B_PFULL + (cp & 1)), (cp >> 1) & 1)) {
+                    const int c = cp++;
+                    tc_fence_after();
+                    const uint32_t kvs = sbase + kOffKV + (c % kStages) * kStageBytes;
 #pragma unroll
-                for (int kk = 0; kk < kKeys / 16; ++kk) {
-                    // B = gathered rows read MN-major: 64 values per 128-byte row,
-                    // LBO = next 64 columns (slab), SBO = next 8 keys.
-                    const uint64_t bd = smem_desc(kvs + kk * 16 * 128, kKSlab, 1024, kSwizzle128B);
-                    mma_f16_ts(tmem + kColO, tmem + kColP + (c & 1) * 32 + kk * 8, bd, id_pv,
-                               (c > 0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < kKeys / 16; ++kk) {
+                        // B = gathered rows read MN-major: 64 values per 128-byte row,
+                        // LBO = next 64 columns (slab), SBO = next 8 keys.
+                        const uint64_t bd = smem_desc(kvs + kk * 16 * 128, kKSlab, 1024, kSwizzle128B);
+                        mma_f16_ts(tmem + kColO, tmem + kColP + (c & 1) * 32 + kk * 8, bd, id_pv,
+                                   (c > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    mma_commit(bar(B_PVDONE + (c & 1)));
+                    mma_commit(bar(B_EMPTY + (c % kStages)));
+                    progressed = true;
                 }
-                mma_commit(bar(B_PVDONE + (c & 1)));
-                mma_commit(bar(B_EMPTY + (c % kStages)));
+                if (progressed) {
+                    t_idle = globaltimer_ns();
+                } else if (*abort_flag) {
+                    ok = false;
+                } else if (globaltimer_ns() - t_idle > kWaitLimitNs) {
+                    *abort_flag = 1;
+                    report_timeout(cq < NC ? B_FULL : B_PFULL, cq < NC ? cq : cp, 0);
+                    ok = false;
+                }
             }
         }
     } else if (warp <= 3) {
@@ -309,6 +329,52 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
             __syncwarp();   // the table is rewritten for the next chunk
         }
         cp_async_wait_all();
+    } else if (warp >= 12) {
+        // ------------------------------------------------------- senders
+        // Warps 12-15, one per TMEM lane quarter: ship this CTA's partial
+        // logits of each chunk (scaled to log2 units, fp16) to the peer. A warp
+        // stages its 32 heads x 64 keys locally and sends the 4 KB with one
+        // bulk copy, counted in bytes on the peer's XFULL barrier.
+        const int qd = warp & 3;
+        const uint32_t lane_addr = (uint32_t)(qd * 32) << 16;
+        const uint32_t xwarp = (uint32_t)qd * kXWarpBytes;
+        const uint32_t xrow = xwarp + (uint32_t)lane * 128;
+        const uint32_t x_peer = mapa(sbase + kOffX, peer);
+        const uint32_t xfull_peer = mapa(bar(B_XFULL), peer);
+        const uint32_t xstage = sbase + kOffXS;
+        for (int c = 0; c < NC; ++c) {
+            const int b = c & 1;
+            if (!wait_warp(bar(B_SFULL + b), (c >> 1) & 1, abort_flag, 500 + B_SFULL, c)) break;
+            tc_fence_after();
+            uint32_t s0[32], s1[32];
+            tmem_ld32(tmem + lane_addr + kColS + b * kKeys, s0);
+            tmem_ld32(tmem + lane_addr + kColS + b * kKeys + 32, s1);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(B_SFREE + b));
+            uint32_t h[32];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                h[j] = pack_half2(__uint_as_float(s0[2 * j]) * scale_log2,
+                                  __uint_as_float(s0[2 * j + 1]) * scale_log2);
+                h[16 + j] = pack_half2(__uint_as_float(s1[2 * j]) * scale_log2,
+                                       __uint_as_float(s1[2 * j + 1]) * scale_log2);
+            }
+            // The peer has consumed chunk c-2 from its slot b, so the bulk copy
+            // of c-2 has landed: it has also finished reading staging slot b.
+            if (c >= 2 && !wait_warp(bar(B_XFREE + b), ((c - 2) >> 1) & 1, abort_flag, 500 + B_XFREE, c))
+                break;
+            const uint32_t stg = xstage + b * kXBytes;
+#pragma unroll
+            for (int m = 0; m < 8; ++m)
+                st_shared_v4(stg + xrow + (((m + lane) & 7) << 4),
+                             make_uint4(h[4 * m], h[4 * m + 1], h[4 * m + 2], h[4 * m + 3]));
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0)
+                bulk_s2cluster(x_peer + b * kXBytes + xwarp, stg + xwarp, kXWarpBytes, xfull_peer + 8u * b);
+        }
     } else if (warp >= 4) {
         // --------------------------------------------- softmax + epilogue
         // Warps 4-11: two warps per TMEM lane quarter; warp half hs takes keys
@@ -316,52 +382,16 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
         const int hs = (warp - 4) >> 2;
         const int i = (warp & 3) * 32 + lane;                  // head = TMEM lane
         const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
-        const uint32_t xs = sbase + kOffX;
-        const uint32_t x_peer = mapa(xs, peer);
-        // this warp's 2 KB run inside a slot; head i's 64 B row within it
-        const uint32_t xwarp = (uint32_t)(hs * 4 + (warp & 3)) * kXWarpBytes;
-        const uint32_t xrow = xwarp + (uint32_t)lane * 64;
-        const uint32_t xstage = sbase + kOffXS;
-        const uint32_t xfull_peer = mapa(bar(B_XFULL), peer);
+        // head i's 128 B row of an exchange slot
+        const uint32_t xs = sbase + kOffX + (uint32_t)i * 128;
         const uint32_t xfree_peer = mapa(bar(B_XFREE), peer);
         const uint32_t* smask = reinterpret_cast<const uint32_t*>(sgen + kOffMask);
         float* red = reinterpret_cast<float*>(sgen + kOffRed);
         float* lsum_s = reinterpret_cast<float*>(sgen + kOffLsum);
         float m_use = -INFINITY, l = 0.f;
         bool ok = true;
-        // bounded wait whose outcome is the same for the whole warp
-        auto wait_w = [&](uint32_t b_addr, uint32_t par, int tag, int c, bool cluster) -> bool {
-            const bool got = cluster ? mbar_wait<true>(b_addr, par, abort_flag, tag, c)
-                                     : mbar_wait(b_addr, par, abort_flag, tag, c);
-            return __all_sync(0xffffffffu, got);
-        };
-
-        // Send this CTA's partial logits of chunk c (scaled, fp16) to the peer.
-        auto send = [&](int c) -> bool {
-            const int b = c & 1;
-            if (!wait_w(bar(B_SFULL + b), (c >> 1) & 1, 200 + B_SFULL, c, false)) return false;
-            tc_fence_after();
-            uint32_t sr[32];
-            tmem_ld32(tmem + lane_addr + kColS + b * kKeys + 32 * hs, sr);
-            tmem_wait_ld();
-            uint32_t h[16];
-#pragma unroll
-            for (int j = 0; j < 16; ++j)
-                h[j] = pack_half2(__uint_as_float(sr[2 * j]) * scale_log2,
-                                  __uint_as_float(sr[2 * j + 1]) * scale_log2);
-            // The peer has consumed chunk c-2 from its slot b, so the bulk copy
-            // of c-2 has landed: it has also finished reading staging slot b.
-            if (c >= 2 && !wait_w(bar(B_XFREE + b), ((c - 2) >> 1) & 1, 200 + B_XFREE, c, false)) return false;
-            const uint32_t stg = xstage + b * kXBytes;
-#pragma unroll
-            for (int m = 0; m < 4; ++m)
-                st_shared_v4(stg + xrow + (((m + (lane >> 1)) & 3) << 4),
-                             make_uint4(h[4 * m], h[4 * m + 1], h[4 * m + 2], h[4 * m + 3]));
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0)
-                bulk_s2cluster(x_peer + b * kXBytes + xwarp, stg + xwarp, kXWarpBytes, xfull_peer + 8u * b);
-            return true;
+        auto wait_w = [&](uint32_t b_addr, uint32_t par, int tag, int c) -> bool {
+            return wait_warp(b_addr, par, abort_flag, tag, c);
         };
 
         {
@@ -382,38 +412,31 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_QT));
         }
-        int sent = 0;                       // chunks whose partial logits went out
-        if (NC > 0) {
-            ok = send(0);
-            sent = 1;
-        }
         for (int c = 0; ok && c < NC; ++c) {
             const int b = c & 1;
-            // send the next chunk's partial now if its logits are already in
-            // TMEM (the exchange then overlaps this chunk's softmax); never
-            // wait for them here
-            if (c + 1 < NC && sent == c + 1 &&
-                __all_sync(0xffffffffu, mbar_test_wait(bar(B_SFULL + ((c + 1) & 1)), ((c + 1) >> 1) & 1))) {
-                if (!send(c + 1)) { ok = false; break; }
-                sent = c + 2;
-            }
             if (i == 0 && hs == 0) mbar_arrive_expect_tx(bar(B_XFULL + b), kXBytes);
-            // the peer's bytes arrive by bulk copy, counted on this local barrier
-            if (!wait_w(bar(B_XFULL + b), (c >> 1) & 1, 200 + B_XFULL, c, false)) { ok = false; break; }
-            uint32_t g[16];
-            const uint32_t xr = xs + b * kXBytes + xrow;
-#pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                const uint4 v = ld_shared_v4(xr + (((m + (lane >> 1)) & 3) << 4));
-                g[4 * m] = v.x; g[4 * m + 1] = v.y; g[4 * m + 2] = v.z; g[4 * m + 3] = v.w;
-            }
+            // this CTA's partial logits of chunk c (fp32, TMEM)
+            if (!wait_w(bar(B_SFULL + b), (c >> 1) & 1, 200 + B_SFULL, c)) { ok = false; break; }
+            tc_fence_after();
             uint32_t sr[32];
             tmem_ld32(tmem + lane_addr + kColS + b * kKeys + 32 * hs, sr);
+            // the peer's (fp16, scaled) arrive by bulk copy, counted on this local barrier
+            if (!wait_w(bar(B_XFULL + b), (c >> 1) & 1, 200 + B_XFULL, c)) {
+                tmem_wait_ld();
+                ok = false;
+                break;
+            }
+            uint32_t g[16];
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const uint4 v = ld_shared_v4(xs + b * kXBytes + (((4 * hs + m + lane) & 7) << 4));
+                g[4 * m] = v.x; g[4 * m + 1] = v.y; g[4 * m + 2] = v.z; g[4 * m + 3] = v.w;
+            }
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_SFREE + b));   // S(c) fully read by this warp
-            if (!wait_w(bar(B_FULL + c % kStages), (c / kStages) & 1, 200 + B_FULL, c, false)) { ok = false; break; }
+            if (!wait_w(bar(B_FULL + c % kStages), (c / kStages) & 1, 200 + B_FULL, c)) { ok = false; break; }
             const uint32_t mw = smask[(c % kStages) * 2 + hs];
             // logit (log2 domain) = own partial (fp32) + peer partial (fp16); masked -> -inf
             float x[32];
@@ -441,14 +464,8 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
             red[(b * 2 + hs) * kHeads + i] = mx[0];
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_RED + b));
-            if (!wait_w(bar(B_RED + b), (c >> 1) & 1, 200 + B_RED, c, false)) { ok = false; break; }
+            if (!wait_w(bar(B_RED + b), (c >> 1) & 1, 200 + B_RED, c)) { ok = false; break; }
             const float mc = fmaxf(mx[0], red[(b * 2 + (hs ^ 1)) * kHeads + i]);
-            // second chance to send the next chunk's partial before this chunk's exps
-            if (c + 1 < NC && sent == c + 1 &&
-                __all_sync(0xffffffffu, mbar_test_wait(bar(B_SFULL + ((c + 1) & 1)), ((c + 1) >> 1) & 1))) {
-                if (!send(c + 1)) { ok = false; break; }
-                sent = c + 2;
-            }
             const float m_new = fmaxf(m_use, mc);
             const bool raise = m_new > m_use + 8.f;
             const bool rescale = raise && m_use != -INFINITY;
@@ -457,7 +474,7 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
                 // O holds earlier chunks: rescale once PV(c-1) has landed. TMEM
                 // loads/stores are warp-wide, so every lane takes part (f = 1
                 // for rows whose maximum did not move).
-                if (!wait_w(bar(B_PVDONE + ((c - 1) & 1)), ((c - 1) >> 1) & 1, 400 + B_PVDONE, c, false)) {
+                if (!wait_w(bar(B_PVDONE + ((c - 1) & 1)), ((c - 1) >> 1) & 1, 400 + B_PVDONE, c)) {
                     ok = false;
                     break;
                 }
@@ -491,7 +508,7 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
                 for (int j = 0; j < w; ++j) ps[j] += ps[j + w];
             l += ps[0];
             // P buffer b is free once PV(c-2) has read it
-            if (c >= 2 && !wait_w(bar(B_PVDONE + b), ((c - 2) >> 1) & 1, 200 + B_PVDONE, c, false)) {
+            if (c >= 2 && !wait_w(bar(B_PVDONE + b), ((c - 2) >> 1) & 1, 200 + B_PVDONE, c)) {
                 ok = false;
                 break;
             }
@@ -501,24 +518,20 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_PFULL + b));
-            if (c + 1 < NC && sent == c + 1) {
-                if (!send(c + 1)) { ok = false; break; }
-                sent = c + 2;
-            }
         }
         // row sum over both key halves
         if (ok) {
             lsum_s[hs * kHeads + i] = l;
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_LSUM));
-            ok = wait_w(bar(B_LSUM), 0, 200 + B_LSUM, 0, false);
+            ok = wait_w(bar(B_LSUM), 0, 200 + B_LSUM, 0);
             if (ok) l += lsum_s[(hs ^ 1) * kHeads + i];
         }
         // epilogue: O / l -> bf16, columns [128hs, 128hs+128) of this CTA's half
         __nv_bfloat16* orow = out + ((size_t)t * kHeads + i) * kDv + rank * 256 + 128 * hs;
         if (ok && NC > 0) {
             const int c = NC - 1;
-            ok = wait_w(bar(B_PVDONE + (c & 1)), (c >> 1) & 1, 300 + B_PVDONE, c, false);
+            ok = wait_w(bar(B_PVDONE + (c & 1)), (c >> 1) & 1, 300 + B_PVDONE, c);
             if (ok) {
                 tc_fence_after();
                 const float inv = l > 0.f ? 1.f / l : 0.f;
@@ -546,8 +559,8 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
             lse[(size_t)t * kHeads + i] = l > 0.f ? (m_use + __log2f(l)) * 0.69314718055994531f : -INFINITY;
     }
 
-    if ((warp == 0 || warp == 12) && lane == 0 && NC > 0) {
-        // every MMA this thread issued completes before TMEM is released
+    if (warp == 0 && lane == 0 && NC > 0) {
+        // every MMA issued completes before TMEM is released
         mma_commit(bar(B_DRAIN));
         const uint64_t t0 = globaltimer_ns();
         while (!mbar_try_wait(bar(B_DRAIN), 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
