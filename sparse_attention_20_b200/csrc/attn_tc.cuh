@@ -23,15 +23,15 @@
 // and PV MMAs (one thread polling both kinds of readiness, so a late chunk
 // never holds back the PV of the previous one); warps 1-3 load Q (TMA tiles)
 // and gather the selected rows with 16-byte cp.async into 128B/64B-swizzled
-// shared memory (3-stage ring of 64-row chunks; completion is counted on the
-// stage's mbarrier, so the gather runs up to three chunks ahead); warps 12-15
+// shared memory (4-stage ring of 64-row chunks; completion is counted on the
+// stage's mbarrier, so the gather runs up to four chunks ahead); warps 12-15
 // (one per TMEM lane quarter) run the exchange: they stage the chunk's fp16
 // partial logits locally and send them with one bulk copy per warp into the
 // peer's shared memory, counted on the peer's mbarrier; warps 4-11 (two per
 // lane quarter, each taking 32 of a chunk's 64 keys) run the softmax and the
 // epilogue.
 // Shared memory per CTA: Q 40 KB (latent columns 128..255 of the slice and the
-// rope slice) + 3 x 36 KB ring + 2 x 16 KB receive slots + 2 x 16 KB staging.
+// rope slice) + 4 x 36 KB ring + 16 KB receive slot + 16 KB staging.
 // TMEM: O cols [0,256), S double buffer [256,384), latent Q [384,448), P
 // (bf16 pairs) double buffer [448,512).
 #pragma once
@@ -48,7 +48,7 @@ constexpr int kHeads = 128;
 constexpr int kDqk = 576;
 constexpr int kDv = 512;
 constexpr int kKeys = 64;
-constexpr int kStages = 3;
+constexpr int kStages = 4;
 constexpr int kThreads = 512;               // 16 warps: MMA, 3 gather, 8 softmax, 4 senders
 constexpr int kGatherThreads = 96;
 
@@ -63,12 +63,16 @@ constexpr int kStageBytes = 4 * kKSlab + kKeys * 64;
 // head with the eight 16 B pieces rotated by the head index. One sender warp
 // owns the contiguous 4 KB of its 32 heads and sends them as one bulk copy.
 constexpr int kXBytes = kHeads * 128;
+// One receive slot and one staging slot: chunk c+1 is staged and sent once
+// the peer has taken chunk c out of its slot, which also proves that the
+// bulk copy of c has finished reading the staging slot.
+constexpr int kXSlots = 1;
 constexpr int kXWarpBytes = 32 * 128;
 constexpr int kOffQ = 0;
 constexpr int kOffKV = kOffQ + kQBytes;
 constexpr int kOffX = kOffKV + kStages * kStageBytes;
-constexpr int kOffXS = kOffX + 2 * kXBytes;               // staging of outgoing slots
-constexpr int kOffBar = kOffXS + 2 * kXBytes;
+constexpr int kOffXS = kOffX + kXSlots * kXBytes;         // staging of outgoing slots
+constexpr int kOffBar = kOffXS + kXSlots * kXBytes;
 constexpr int kOffMask = kOffBar + 256;                 // [kStages][2] validity bits
 constexpr int kOffRed = kOffMask + 64;                  // [2 parity][2 halves][128] row maxima
 constexpr int kOffLsum = kOffRed + 2 * 2 * kHeads * 4;  // [2 halves][128] row sums
@@ -164,8 +168,10 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
             mbar_init(bar(B_SFULL + b), 1);
             mbar_init(bar(B_PFULL + b), 8);
             mbar_init(bar(B_PVDONE + b), 1);
-            mbar_init(bar(B_XFULL + b), 1);   // receiver's expect_tx + the peer senders' bytes
-            mbar_init(bar(B_XFREE + b), 8);   // one arrival per softmax warp of the peer
+            if (b < kXSlots) {
+                mbar_init(bar(B_XFULL + b), 1);   // receiver's expect_tx + the peer senders' bytes
+                mbar_init(bar(B_XFREE + b), 8);   // one arrival per softmax warp of the peer
+            }
             mbar_init(bar(B_RED + b), 8);
         }
         mbar_init(bar(B_DRAIN), 1);     // the MMA issuer
@@ -361,11 +367,14 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
                 h[16 + j] = pack_half2(__uint_as_float(s1[2 * j]) * scale_log2,
                                        __uint_as_float(s1[2 * j + 1]) * scale_log2);
             }
-            // The peer has consumed chunk c-2 from its slot b, so the bulk copy
-            // of c-2 has landed: it has also finished reading staging slot b.
-            if (c >= 2 && !wait_warp(bar(B_XFREE + b), ((c - 2) >> 1) & 1, abort_flag, 500 + B_XFREE, c))
+            // The peer has consumed chunk c-kXSlots from slot xb, so the bulk
+            // copy of that chunk has landed: it has also finished reading
+            // staging slot xb.
+            const int xb = c % kXSlots;
+            if (c >= kXSlots && !wait_warp(bar(B_XFREE + xb), ((c - kXSlots) / kXSlots) & 1, abort_flag,
+                                           500 + B_XFREE, c))
                 break;
-            const uint32_t stg = xstage + b * kXBytes;
+            const uint32_t stg = xstage + xb * kXBytes;
 #pragma unroll
             for (int m = 0; m < 8; ++m)
                 st_shared_v4(stg + xrow + (((m + lane) & 7) << 4),
@@ -373,7 +382,7 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0)
-                bulk_s2cluster(x_peer + b * kXBytes + xwarp, stg + xwarp, kXWarpBytes, xfull_peer + 8u * b);
+                bulk_s2cluster(x_peer + xb * kXBytes + xwarp, stg + xwarp, kXWarpBytes, xfull_peer + 8u * xb);
         }
     } else if (warp >= 4) {
         // --------------------------------------------- softmax + epilogue
@@ -414,14 +423,15 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
         }
         for (int c = 0; ok && c < NC; ++c) {
             const int b = c & 1;
-            if (i == 0 && hs == 0) mbar_arrive_expect_tx(bar(B_XFULL + b), kXBytes);
+            const int xb = c % kXSlots;
+            if (i == 0 && hs == 0) mbar_arrive_expect_tx(bar(B_XFULL + xb), kXBytes);
             // this CTA's partial logits of chunk c (fp32, TMEM)
             if (!wait_w(bar(B_SFULL + b), (c >> 1) & 1, 200 + B_SFULL, c)) { ok = false; break; }
             tc_fence_after();
             uint32_t sr[32];
             tmem_ld32(tmem + lane_addr + kColS + b * kKeys + 32 * hs, sr);
             // the peer's (fp16, scaled) arrive by bulk copy, counted on this local barrier
-            if (!wait_w(bar(B_XFULL + b), (c >> 1) & 1, 200 + B_XFULL, c)) {
+            if (!wait_w(bar(B_XFULL + xb), (c / kXSlots) & 1, 200 + B_XFULL, c)) {
                 tmem_wait_ld();
                 ok = false;
                 break;
@@ -429,7 +439,7 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
             uint32_t g[16];
 #pragma unroll
             for (int m = 0; m < 4; ++m) {
-                const uint4 v = ld_shared_v4(xs + b * kXBytes + (((4 * hs + m + lane) & 7) << 4));
+                const uint4 v = ld_shared_v4(xs + xb * kXBytes + (((4 * hs + m + lane) & 7) << 4));
                 g[4 * m] = v.x; g[4 * m + 1] = v.y; g[4 * m + 2] = v.z; g[4 * m + 3] = v.w;
             }
             tmem_wait_ld();
@@ -452,7 +462,7 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
             // the peer may refill this exchange slot once every warp has used it
             // (the loaded values are consumed above, so a relaxed signal suffices)
             __syncwarp();
-            if (lane == 0) mbar_arrive_remote_relaxed(xfree_peer + 8u * b);
+            if (lane == 0) mbar_arrive_remote_relaxed(xfree_peer + 8u * xb);
             float mx[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) mx[j] = fmaxf(x[j], x[j + 16]);
