@@ -15,6 +15,7 @@
 #include "attn_simple.cuh"
 #include "attn_tc.cuh"
 #include "common.cuh"
+#include "indexer_chunked.cuh"
 #include "indexer_scores.cuh"
 #include "indexer_tc.cuh"
 #include "topk_select.cuh"
@@ -75,11 +76,26 @@ constexpr size_t kScoreBlockBytes = size_t(1) << 30;  // score rows kept per blo
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 // Query rows whose full score rows fit in one block of the score buffer.
-int index_rows_per_block(int T, int S)
+// Chunked indexer (per-row key ranges): rows per launch block, the pair
+// stride of a row (its most chunks times k) and the buffers it needs.
+struct ChunkPlan {
+    int RB, max_chunks;
+    long long cand_ld;
+    size_t off_work, off_cand, bytes;
+};
+
+ChunkPlan chunk_plan(int T, int S, int k)
 {
-    const size_t per_row = (size_t)S * sizeof(float);
-    const size_t rows = std::max<size_t>(1, kScoreBlockBytes / per_row);
-    return (int)std::min<size_t>((size_t)T, rows);
+    using namespace dsa::idx_chunk;
+    ChunkPlan p;
+    p.max_chunks = dsa::ceil_div(S, kChunkKeys);
+    p.cand_ld = p.max_chunks > 1 ? (long long)p.max_chunks * k : 0;
+    const size_t per_row = (size_t)p.cand_ld * sizeof(uint2) + sizeof(int);
+    p.RB = (int)std::min<size_t>((size_t)T, std::max<size_t>(1, kScoreBlockBytes / per_row));
+    p.off_work = 0;
+    p.off_cand = align_up((size_t)(p.RB + 1) * sizeof(int));
+    p.bytes = align_up(p.off_cand + (size_t)p.RB * p.cand_ld * sizeof(uint2));
+    return p;
 }
 
 // Streaming (tensor-core) indexer: query rows per launch block and the
@@ -108,8 +124,7 @@ FusedPlan fused_plan(int T, int S, int k)
 
 size_t indexer_workspace(int T, int S, int k = 1)
 {
-    const size_t general = align_up((size_t)index_rows_per_block(T, S) * (size_t)S * sizeof(float));
-    return std::max(general, fused_plan(T, S, k).bytes);
+    return std::max(chunk_plan(T, S, k).bytes, fused_plan(T, S, k).bytes);
 }
 
 int num_sms()
@@ -213,25 +228,61 @@ ScoresFn pick_scores(int H_I, int d_I)
     }
 }
 
-int indexer_scan_select(const uint8_t* q_idx, const float* w, const uint8_t* k_idx,
-                        const int32_t* pos, const int32_t* k_base, int T, int S, int H_I, int d_I,
-                        int k, int32_t* idx, void* workspace, cudaStream_t st)
+template <int NT, int DI>
+void launch_chunk_topk(int grid, cudaStream_t st, const uint8_t* q_idx, const float* w,
+                       const uint8_t* k_idx, const int* pos, const int* k_base, int T, int S, int H_I,
+                       int row0, int rows, int k, const int* work_off, uint2* cand, long long cand_ld,
+                       int32_t* idx)
 {
-    const int RB = index_rows_per_block(T, S);
-    float* scores = reinterpret_cast<float*>(workspace);
-    const long long ld = S;
-    constexpr int kKeysPerCta = 2048;
-    ScoresFn scores_fn = pick_scores(H_I, d_I);
-    for (int row0 = 0; row0 < T; row0 += RB) {
-        const int rb = std::min(RB, T - row0);
-        // longest candidate range in this block of rows
-        const int n_max = pos ? S : std::min(S, row0 + rb + S - T);
-        dim3 grid(dsa::ceil_div(n_max, kKeysPerCta), rb);
-        scores_fn(grid, st, q_idx, w, k_idx, pos, k_base, T, S, H_I, row0, scores, ld, kKeysPerCta);
-        DSA_LAUNCH_CHECK("indexer_scores_kernel");
-        dsa::topk_dense_rows_kernel<dsa::kSelectThreads>
-            <<<rb, dsa::kSelectThreads, 0, st>>>(scores, ld, pos, k_base, T, S, row0, k, idx);
-        DSA_LAUNCH_CHECK("topk_dense_rows_kernel");
+    using namespace dsa::idx_chunk;
+    cudaFuncSetAttribute(chunk_topk_kernel<NT, DI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)kSmemBytes);
+    chunk_topk_kernel<NT, DI><<<grid, kThreads, kSmemBytes, st>>>(
+        q_idx, w, k_idx, pos, k_base, T, S, H_I, row0, rows, k, work_off, cand, cand_ld, idx);
+}
+
+using ChunkFn = void (*)(int, cudaStream_t, const uint8_t*, const float*, const uint8_t*, const int*,
+                         const int*, int, int, int, int, int, int, const int*, uint2*, long long,
+                         int32_t*);
+
+ChunkFn pick_chunk(int H_I, int d_I)
+{
+    const bool two = H_I > 8;
+    switch (d_I) {
+        case 32: return two ? launch_chunk_topk<2, 32> : launch_chunk_topk<1, 32>;
+        case 64: return two ? launch_chunk_topk<2, 64> : launch_chunk_topk<1, 64>;
+        case 128: return two ? launch_chunk_topk<2, 128> : launch_chunk_topk<1, 128>;
+        default: return two ? launch_chunk_topk<2, 256> : launch_chunk_topk<1, 256>;
+    }
+}
+
+// Rows with their own key ranges: chunk scores + chunk Top-k, then the merge
+// of the chunks' pairs (indexer_chunked.cuh).
+int indexer_chunked(const uint8_t* q_idx, const float* w, const uint8_t* k_idx, const int32_t* pos,
+                    const int32_t* k_base, int T, int S, int H_I, int d_I, int k, int32_t* idx,
+                    void* workspace, cudaStream_t st)
+{
+    using namespace dsa::idx_chunk;
+    const ChunkPlan p = chunk_plan(T, S, k);
+    char* ws = reinterpret_cast<char*>(workspace);
+    int* work_off = reinterpret_cast<int*>(ws + p.off_work);
+    uint2* cand = reinterpret_cast<uint2*>(ws + p.off_cand);
+    ChunkFn chunk_fn = pick_chunk(H_I, d_I);
+    const int resident = kCtasPerSm * num_sms();
+    for (int row0 = 0; row0 < T; row0 += p.RB) {
+        const int rows = std::min(p.RB, T - row0);
+        const int n_max = pos ? S : std::min(S, row0 + rows + S - T);
+        const long long items_max = (long long)rows * std::max(1, dsa::ceil_div(n_max, kChunkKeys));
+        chunk_plan_kernel<<<1, kPlanThreads, 0, st>>>(pos, k_base, T, S, row0, rows, work_off);
+        DSA_LAUNCH_CHECK("chunk_plan_kernel");
+        chunk_fn((int)std::min<long long>(items_max, resident), st, q_idx, w, k_idx, pos, k_base, T, S,
+                 H_I, row0, rows, k, work_off, cand, p.cand_ld, idx);
+        DSA_LAUNCH_CHECK("chunk_topk_kernel");
+        if (n_max > kChunkKeys) {
+            merge_topk_kernel<kMergeThreads><<<rows, kMergeThreads, 0, st>>>(
+                cand, p.cand_ld, pos, k_base, T, S, row0, k, idx);
+            DSA_LAUNCH_CHECK("merge_topk_kernel");
+        }
     }
     return DSA_OK;
 }
@@ -414,9 +465,9 @@ int dsa_indexer_topk(const void* q_idx, const float* w, const void* k_idx, const
         return indexer_fused(reinterpret_cast<const uint8_t*>(q_idx), w,
                              reinterpret_cast<const uint8_t*>(k_idx), T, S, k, idx, workspace,
                              reinterpret_cast<cudaStream_t>(stream));
-    return indexer_scan_select(reinterpret_cast<const uint8_t*>(q_idx), w,
-                               reinterpret_cast<const uint8_t*>(k_idx), pos, k_base, T, S, H_I, d_I,
-                               k, idx, workspace, reinterpret_cast<cudaStream_t>(stream));
+    return indexer_chunked(reinterpret_cast<const uint8_t*>(q_idx), w,
+                           reinterpret_cast<const uint8_t*>(k_idx), pos, k_base, T, S, H_I, d_I, k,
+                           idx, workspace, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int dsa_sparse_mla_attn(const void* q, const void* kv, const int32_t* idx, const int32_t* pos,

@@ -27,6 +27,14 @@ struct DenseScores {
     __device__ __forceinline__ int s(int i) const { return i; }
 };
 
+// Scores of keys s0, s0+1, ... held in shared memory.
+struct SmemScores {
+    const float* p;
+    int s0;
+    __device__ __forceinline__ uint32_t key(int i) const { return score_key(p[i]); }
+    __device__ __forceinline__ int s(int i) const { return s0 + i; }
+};
+
 // Candidates stored as (fp32 score bits, s) pairs.
 struct PairScores {
     const uint2* p;
@@ -121,16 +129,12 @@ __device__ uint32_t radix_kth_key(const Row& row, int n, int k, SelectSmem<THREA
     return prefix;
 }
 
-// Writes the Top-k of `row` (n entries) to out[0..k) in storage order (for
-// dense rows: ascending s), so the result is deterministic.
-template <int THREADS, class Row>
-__device__ void block_topk(const Row& row, int n, int k, int32_t* __restrict__ out,
-                           SelectSmem<THREADS>& sm)
+// Emits the Top-k of `row` (n > k entries) as emit(slot, i) for slots
+// 0..k-1 in storage order (for dense rows: ascending s), so the result is
+// deterministic.
+template <int THREADS, class Row, class Emit>
+__device__ void block_select(const Row& row, int n, int k, const Emit& emit, SelectSmem<THREADS>& sm)
 {
-    if (n <= k) {
-        for (int i = threadIdx.x; i < k; i += THREADS) out[i] = i < n ? row.s(i) : -1;
-        return;
-    }
     int take_eq, count_eq;
     const uint32_t kth = radix_kth_key<THREADS>(row, n, k, sm, &take_eq, &count_eq);
     const int warp = threadIdx.x >> 5;
@@ -175,7 +179,7 @@ __device__ void block_topk(const Row& row, int n, int k, int32_t* __restrict__ o
         int off = sm.counter[0];
         for (int w = 0; w < warp; ++w) off += (int)sm.hist[0][w];
         const int slot = off + __popc(m & ((1u << lane) - 1u));
-        if (take && slot < k) out[slot] = s;
+        if (take && slot < k) emit(slot, i);
         __syncthreads();
         if (threadIdx.x == 0) {
             int tot = 0;
@@ -184,6 +188,19 @@ __device__ void block_topk(const Row& row, int n, int k, int32_t* __restrict__ o
         }
         __syncthreads();
     }
+}
+
+// Writes the Top-k of `row` (n entries) to out[0..k) in storage order; slots
+// beyond n (n < k) get -1.
+template <int THREADS, class Row>
+__device__ void block_topk(const Row& row, int n, int k, int32_t* __restrict__ out,
+                           SelectSmem<THREADS>& sm)
+{
+    if (n <= k) {
+        for (int i = threadIdx.x; i < k; i += THREADS) out[i] = i < n ? row.s(i) : -1;
+        return;
+    }
+    block_select<THREADS>(row, n, k, [&](int slot, int i) { out[slot] = row.s(i); }, sm);
 }
 
 constexpr int kSelectThreads = 1024;
