@@ -76,25 +76,35 @@ constexpr size_t kScoreBlockBytes = size_t(1) << 30;  // score rows kept per blo
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 // Query rows whose full score rows fit in one block of the score buffer.
-// Chunked indexer (per-row key ranges): rows per launch block, the pair
-// stride of a row (its most chunks times k) and the buffers it needs.
+// Chunked indexer (per-row key ranges): rows per launch block, the per-row
+// strides (most chunks of a row times k pairs, times the sampled positions)
+// and the buffers it needs.
 struct ChunkPlan {
     int RB, max_chunks;
-    long long cand_ld;
-    size_t off_work, off_cand, bytes;
+    long long cand_ld, samp_ld;
+    size_t off_work, off_flags, off_tau, off_ccnt, off_samp, off_cand, bytes;
 };
+
+constexpr int kMaxChunksPerRow = 32768;   // S <= 2^28 keys on this path
 
 ChunkPlan chunk_plan(int T, int S, int k)
 {
     using namespace dsa::idx_chunk;
     ChunkPlan p;
     p.max_chunks = dsa::ceil_div(S, kChunkKeys);
-    p.cand_ld = p.max_chunks > 1 ? (long long)p.max_chunks * k : 0;
-    const size_t per_row = (size_t)p.cand_ld * sizeof(uint2) + sizeof(int);
+    const bool multi = p.max_chunks > 1;
+    p.cand_ld = multi ? (long long)p.max_chunks * k : 0;
+    p.samp_ld = multi ? (long long)p.max_chunks * kSamplesPerChunk : 0;
+    const size_t per_row = (size_t)p.cand_ld * sizeof(uint2) + (size_t)p.samp_ld * sizeof(float) +
+                           (size_t)p.max_chunks * sizeof(int) + 3 * sizeof(int);
     p.RB = (int)std::min<size_t>((size_t)T, std::max<size_t>(1, kScoreBlockBytes / per_row));
     p.off_work = 0;
-    p.off_cand = align_up((size_t)(p.RB + 1) * sizeof(int));
-    p.bytes = align_up(p.off_cand + (size_t)p.RB * p.cand_ld * sizeof(uint2));
+    p.off_flags = align_up((size_t)(p.RB + 1) * sizeof(int));
+    p.off_tau = p.off_flags + align_up((size_t)p.RB * sizeof(int));
+    p.off_ccnt = p.off_tau + align_up((size_t)p.RB * sizeof(uint32_t));
+    p.off_samp = p.off_ccnt + align_up((size_t)p.RB * p.max_chunks * sizeof(int));
+    p.off_cand = p.off_samp + align_up((size_t)p.RB * p.samp_ld * sizeof(float));
+    p.bytes = p.off_cand + align_up((size_t)p.RB * p.cand_ld * sizeof(uint2));
     return p;
 }
 
@@ -228,61 +238,117 @@ ScoresFn pick_scores(int H_I, int d_I)
     }
 }
 
+struct ChunkArgs {
+    const uint8_t* q_idx;
+    const float* w;
+    const uint8_t* k_idx;
+    const int* pos;
+    const int* k_base;
+    int T, S, H_I, k, row0, rows;
+    const int* work_off;
+};
+
 template <int NT, int DI>
-void launch_chunk_topk(int grid, cudaStream_t st, const uint8_t* q_idx, const float* w,
-                       const uint8_t* k_idx, const int* pos, const int* k_base, int T, int S, int H_I,
-                       int row0, int rows, int k, const int* work_off, uint2* cand, long long cand_ld,
-                       int32_t* idx)
+struct ChunkKernels {
+    static void sample(int grid, cudaStream_t st, const ChunkArgs& a, float* samp, long long samp_ld)
+    {
+        using namespace dsa::idx_chunk;
+        chunk_sample_kernel<NT, DI><<<grid, kThreads, 0, st>>>(a.q_idx, a.w, a.k_idx, a.pos, a.k_base, a.T,
+                                                              a.S, a.H_I, a.row0, a.rows, a.work_off,
+                                                              samp, samp_ld);
+    }
+    static void topk(int grid, cudaStream_t st, const ChunkArgs& a, const uint32_t* tau, uint2* cand,
+                     long long cand_ld, int* ccnt, int max_chunks, int32_t* idx)
+    {
+        using namespace dsa::idx_chunk;
+        cudaFuncSetAttribute(chunk_topk_kernel<NT, DI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kSmemBytes);
+        chunk_topk_kernel<NT, DI><<<grid, kThreads, kSmemBytes, st>>>(
+            a.q_idx, a.w, a.k_idx, a.pos, a.k_base, a.T, a.S, a.H_I, a.row0, a.rows, a.k, a.work_off,
+            tau, cand, cand_ld, ccnt, max_chunks, idx);
+    }
+};
+
+struct ChunkFns {
+    void (*sample)(int, cudaStream_t, const ChunkArgs&, float*, long long);
+    void (*topk)(int, cudaStream_t, const ChunkArgs&, const uint32_t*, uint2*, long long, int*, int,
+                 int32_t*);
+};
+
+template <int NT, int DI>
+ChunkFns chunk_fns()
 {
-    using namespace dsa::idx_chunk;
-    cudaFuncSetAttribute(chunk_topk_kernel<NT, DI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)kSmemBytes);
-    chunk_topk_kernel<NT, DI><<<grid, kThreads, kSmemBytes, st>>>(
-        q_idx, w, k_idx, pos, k_base, T, S, H_I, row0, rows, k, work_off, cand, cand_ld, idx);
+    return {ChunkKernels<NT, DI>::sample, ChunkKernels<NT, DI>::topk};
 }
 
-using ChunkFn = void (*)(int, cudaStream_t, const uint8_t*, const float*, const uint8_t*, const int*,
-                         const int*, int, int, int, int, int, int, const int*, uint2*, long long,
-                         int32_t*);
-
-ChunkFn pick_chunk(int H_I, int d_I)
+ChunkFns pick_chunk(int H_I, int d_I)
 {
     const bool two = H_I > 8;
     switch (d_I) {
-        case 32: return two ? launch_chunk_topk<2, 32> : launch_chunk_topk<1, 32>;
-        case 64: return two ? launch_chunk_topk<2, 64> : launch_chunk_topk<1, 64>;
-        case 128: return two ? launch_chunk_topk<2, 128> : launch_chunk_topk<1, 128>;
-        default: return two ? launch_chunk_topk<2, 256> : launch_chunk_topk<1, 256>;
+        case 32: return two ? chunk_fns<2, 32>() : chunk_fns<1, 32>();
+        case 64: return two ? chunk_fns<2, 64>() : chunk_fns<1, 64>();
+        case 128: return two ? chunk_fns<2, 128>() : chunk_fns<1, 128>();
+        default: return two ? chunk_fns<2, 256>() : chunk_fns<1, 256>();
     }
 }
 
-// Rows with their own key ranges: chunk scores + chunk Top-k, then the merge
-// of the chunks' pairs (indexer_chunked.cuh).
+// Rows with their own key ranges (indexer_chunked.cuh): chunk scores and
+// sampled thresholds, chunk filters, the merge of the chunks' pairs, and the
+// rerun without threshold of any row the merge flags.
 int indexer_chunked(const uint8_t* q_idx, const float* w, const uint8_t* k_idx, const int32_t* pos,
                     const int32_t* k_base, int T, int S, int H_I, int d_I, int k, int32_t* idx,
                     void* workspace, cudaStream_t st)
 {
     using namespace dsa::idx_chunk;
     const ChunkPlan p = chunk_plan(T, S, k);
+    if (p.max_chunks > kMaxChunksPerRow)
+        return fail(DSA_ERR_UNSUPPORTED, "S=%d: at most %d keys per row on this path", S,
+                    kMaxChunksPerRow * kChunkKeys);
     char* ws = reinterpret_cast<char*>(workspace);
     int* work_off = reinterpret_cast<int*>(ws + p.off_work);
+    int* flags = reinterpret_cast<int*>(ws + p.off_flags);
+    uint32_t* tau = reinterpret_cast<uint32_t*>(ws + p.off_tau);
+    int* ccnt = reinterpret_cast<int*>(ws + p.off_ccnt);
+    float* samp = reinterpret_cast<float*>(ws + p.off_samp);
     uint2* cand = reinterpret_cast<uint2*>(ws + p.off_cand);
-    ChunkFn chunk_fn = pick_chunk(H_I, d_I);
+    const ChunkFns fn = pick_chunk(H_I, d_I);
     const int resident = kCtasPerSm * num_sms();
+    const size_t merge_smem = (size_t)(p.max_chunks + 1) * sizeof(int);
+    if (merge_smem > 8192) {
+        cudaError_t e = cudaFuncSetAttribute(merge_topk_kernel<kMergeThreads>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)merge_smem);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(merge_topk_kernel)");
+    }
     for (int row0 = 0; row0 < T; row0 += p.RB) {
         const int rows = std::min(p.RB, T - row0);
         const int n_max = pos ? S : std::min(S, row0 + rows + S - T);
-        const long long items_max = (long long)rows * std::max(1, dsa::ceil_div(n_max, kChunkKeys));
-        chunk_plan_kernel<<<1, kPlanThreads, 0, st>>>(pos, k_base, T, S, row0, rows, work_off);
+        const bool multi = n_max > kChunkKeys;
+        const int grid = (int)std::min<long long>(
+            (long long)rows * std::max(1, dsa::ceil_div(n_max, kChunkKeys)), resident);
+        const ChunkArgs a{q_idx, w, k_idx, pos, k_base, T, S, H_I, k, row0, rows, work_off};
+        chunk_plan_kernel<<<1, kPlanThreads, 0, st>>>(pos, k_base, T, S, row0, rows, 0, flags, work_off);
         DSA_LAUNCH_CHECK("chunk_plan_kernel");
-        chunk_fn((int)std::min<long long>(items_max, resident), st, q_idx, w, k_idx, pos, k_base, T, S,
-                 H_I, row0, rows, k, work_off, cand, p.cand_ld, idx);
-        DSA_LAUNCH_CHECK("chunk_topk_kernel");
-        if (n_max > kChunkKeys) {
-            merge_topk_kernel<kMergeThreads><<<rows, kMergeThreads, 0, st>>>(
-                cand, p.cand_ld, pos, k_base, T, S, row0, k, idx);
-            DSA_LAUNCH_CHECK("merge_topk_kernel");
+        if (multi) {
+            fn.sample(grid, st, a, samp, p.samp_ld);
+            DSA_LAUNCH_CHECK("chunk_sample_kernel");
+            chunk_tau_kernel<kTauThreads><<<rows, kTauThreads, 0, st>>>(samp, p.samp_ld, pos, k_base, T, S,
+                                                                       row0, k, tau);
+            DSA_LAUNCH_CHECK("chunk_tau_kernel");
         }
+        fn.topk(grid, st, a, multi ? tau : nullptr, cand, p.cand_ld, ccnt, p.max_chunks, idx);
+        DSA_LAUNCH_CHECK("chunk_topk_kernel");
+        if (!multi) continue;
+        merge_topk_kernel<kMergeThreads><<<rows, kMergeThreads, merge_smem, st>>>(
+            cand, p.cand_ld, ccnt, p.max_chunks, pos, k_base, T, S, row0, k, 0, flags, idx);
+        DSA_LAUNCH_CHECK("merge_topk_kernel");
+        // rows the threshold left short of k: again without it
+        chunk_plan_kernel<<<1, kPlanThreads, 0, st>>>(pos, k_base, T, S, row0, rows, 1, flags, work_off);
+        DSA_LAUNCH_CHECK("chunk_plan_kernel");
+        fn.topk(grid, st, a, nullptr, cand, p.cand_ld, ccnt, p.max_chunks, idx);
+        DSA_LAUNCH_CHECK("chunk_topk_kernel");
+        merge_topk_kernel<kMergeThreads><<<rows, kMergeThreads, merge_smem, st>>>(
+            cand, p.cand_ld, ccnt, p.max_chunks, pos, k_base, T, S, row0, k, 1, flags, idx);
+        DSA_LAUNCH_CHECK("merge_topk_kernel");
     }
     return DSA_OK;
 }

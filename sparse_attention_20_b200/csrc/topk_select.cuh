@@ -129,6 +129,38 @@ __device__ uint32_t radix_kth_key(const Row& row, int n, int k, SelectSmem<THREA
     return prefix;
 }
 
+// Ordered compaction: emit(slot, i) for the entries i < n with pred(i), in
+// storage order, for slots below cap. Returns the number of such entries
+// (which may exceed cap). Every thread of the CTA takes part.
+template <int THREADS, class Pred, class Emit>
+__device__ int block_emit_if(int n, const Pred& pred, const Emit& emit, int cap, SelectSmem<THREADS>& sm)
+{
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) sm.counter[0] = 0;
+    __syncthreads();
+    for (int c0 = 0; c0 < n; c0 += THREADS) {
+        const int i = c0 + threadIdx.x;
+        const bool take = i < n && pred(i);
+        const unsigned m = __ballot_sync(0xffffffffu, take);
+        if (lane == 0) sm.hist[0][warp] = __popc(m);
+        __syncthreads();
+        int off = sm.counter[0];
+        for (int w = 0; w < warp; ++w) off += (int)sm.hist[0][w];
+        const int slot = off + __popc(m & ((1u << lane) - 1u));
+        if (take && slot < cap) emit(slot, i);
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            int tot = 0;
+            for (int w = 0; w < THREADS / 32; ++w) tot += (int)sm.hist[0][w];
+            sm.counter[0] += tot;
+        }
+        __syncthreads();
+    }
+    const int total = sm.counter[0];
+    __syncthreads();
+    return total;
+}
+
 // Emits the Top-k of `row` (n > k entries) as emit(slot, i) for slots
 // 0..k-1 in storage order (for dense rows: ascending s), so the result is
 // deterministic.
@@ -161,33 +193,13 @@ __device__ void block_select(const Row& row, int n, int k, const Emit& emit, Sel
         s_cut = prefix;
     }
     // Emit in storage order (ascending s for dense rows): ordered compaction.
-    if (threadIdx.x == 0) sm.counter[0] = 0;
-    __syncthreads();
-    const int lane = threadIdx.x & 31;
-    for (int c0 = 0; c0 < n; c0 += THREADS) {
-        const int i = c0 + threadIdx.x;
-        bool take = false;
-        int s = 0;
-        if (i < n) {
+    block_emit_if<THREADS>(
+        n,
+        [&](int i) {
             const uint32_t key = row.key(i);
-            s = row.s(i);
-            take = key > kth || (key == kth && (uint32_t)s <= s_cut);
-        }
-        const unsigned m = __ballot_sync(0xffffffffu, take);
-        if (lane == 0) sm.hist[0][warp] = __popc(m);
-        __syncthreads();
-        int off = sm.counter[0];
-        for (int w = 0; w < warp; ++w) off += (int)sm.hist[0][w];
-        const int slot = off + __popc(m & ((1u << lane) - 1u));
-        if (take && slot < k) emit(slot, i);
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            int tot = 0;
-            for (int w = 0; w < THREADS / 32; ++w) tot += (int)sm.hist[0][w];
-            sm.counter[0] += tot;
-        }
-        __syncthreads();
-    }
+            return key > kth || (key == kth && (uint32_t)row.s(i) <= s_cut);
+        },
+        emit, k, sm);
 }
 
 // Writes the Top-k of `row` (n entries) to out[0..k) in storage order; slots

@@ -98,6 +98,34 @@ def test_decode_integer_inputs_bit_exact():
     check_indexer(x, idx.cpu(), list(range(x.T)), exact=True)
 
 
+def test_decode_multi_chunk_integer_bit_exact():
+    """Rows of one to five 8192-key chunks (chunk Top-k, sampled threshold and
+    merge); integer FP8-exact inputs make many scores tie across chunks."""
+    x = synth.decode_inputs("decode", device="cuda", seed=9, B=5, ctx=[8193, 16384, 20000, 40000, 9000],
+                            overrides=dict(indexer="int", k=2048))
+    idx = dsa.indexer_topk(x.q_idx, x.w, x.k_idx, x.k, pos=x.pos, k_base=x.k_base)
+    torch.cuda.synchronize()
+    check_indexer(x, idx.cpu(), list(range(x.T)), exact=True)
+
+
+def test_decode_threshold_overshoot_still_exact():
+    """Only keys on a regular grid (s mod 4096 < 128) are non-zero, so a
+    threshold sampled on that grid keeps far fewer than k keys; the rows must
+    still get their exact Top-k (ties at score 0 go to the lowest s)."""
+    x = synth.decode_inputs("decode", device="cuda", seed=10, B=3, ctx=[30000, 50000, 12000],
+                            overrides=dict(indexer="int", k=2048))
+    base = x.bases().cpu().long()
+    pos = x.positions().cpu().long()
+    keep = torch.zeros(x.k_idx.shape[0], dtype=torch.bool)
+    for b, p in zip(base.tolist(), pos.tolist()):
+        s = torch.arange(p + 1)
+        keep[b + s[(s % 4096) < 128]] = True
+    x.k_idx[~keep.to(x.k_idx.device)] = 0
+    idx = dsa.indexer_topk(x.q_idx, x.w, x.k_idx, x.k, pos=x.pos, k_base=x.k_base)
+    torch.cuda.synchronize()
+    check_indexer(x, idx.cpu(), list(range(x.T)), exact=True)
+
+
 def test_k_at_least_L_selects_every_past_token():
     x = synth.prefill_inputs("tiny", device="cuda", seed=6, L=100, overrides=dict(k=128))
     idx, out, lse = _run(x)
