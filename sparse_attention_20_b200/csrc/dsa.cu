@@ -238,6 +238,8 @@ ScoresFn pick_scores(int H_I, int d_I)
     }
 }
 
+int make_tmap_u8(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t rows, uint32_t box_rows);
+
 struct ChunkArgs {
     const uint8_t* q_idx;
     const float* w;
@@ -269,16 +271,33 @@ struct ChunkKernels {
     }
 };
 
+// d_I = 128: key rows streamed by TMA (tm_k over k_idx, 128-key boxes)
+template <int NT>
+void chunk_topk_tma(int grid, cudaStream_t st, const CUtensorMap& tm_k, const ChunkArgs& a,
+                    const uint32_t* tau, uint2* cand, long long cand_ld, int* ccnt, int max_chunks,
+                    int32_t* idx)
+{
+    using namespace dsa::idx_chunk;
+    cudaFuncSetAttribute(chunk_topk_tma_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         tma::kSmemBytes);
+    chunk_topk_tma_kernel<NT><<<grid, tma::kThreads, tma::kSmemBytes, st>>>(
+        tm_k, a.q_idx, a.w, a.pos, a.k_base, a.T, a.S, a.H_I, a.row0, a.rows, a.k, a.work_off, tau, cand,
+        cand_ld, ccnt, max_chunks, idx);
+}
+
 struct ChunkFns {
     void (*sample)(int, cudaStream_t, const ChunkArgs&, float*, long long);
     void (*topk)(int, cudaStream_t, const ChunkArgs&, const uint32_t*, uint2*, long long, int*, int,
                  int32_t*);
+    void (*topk_tma)(int, cudaStream_t, const CUtensorMap&, const ChunkArgs&, const uint32_t*, uint2*,
+                     long long, int*, int, int32_t*);
 };
 
 template <int NT, int DI>
 ChunkFns chunk_fns()
 {
-    return {ChunkKernels<NT, DI>::sample, ChunkKernels<NT, DI>::topk};
+    return {ChunkKernels<NT, DI>::sample, ChunkKernels<NT, DI>::topk,
+            DI == 128 ? chunk_topk_tma<NT> : nullptr};
 }
 
 ChunkFns pick_chunk(int H_I, int d_I)
@@ -312,7 +331,16 @@ int indexer_chunked(const uint8_t* q_idx, const float* w, const uint8_t* k_idx, 
     float* samp = reinterpret_cast<float*>(ws + p.off_samp);
     uint2* cand = reinterpret_cast<uint2*>(ws + p.off_cand);
     const ChunkFns fn = pick_chunk(H_I, d_I);
-    const int resident = kCtasPerSm * num_sms();
+    CUtensorMap tm_k;
+    if (fn.topk_tma)
+        if (int rc = make_tmap_u8(&tm_k, k_idx, 128, (uint64_t)S, tma::kTileKeys)) return rc;
+    const int resident = (fn.topk_tma ? tma::kCtasPerSm : kCtasPerSm) * num_sms();
+    auto topk = [&](const ChunkArgs& a, int grid, const uint32_t* tk) {
+        if (fn.topk_tma)
+            fn.topk_tma(grid, st, tm_k, a, tk, cand, p.cand_ld, ccnt, p.max_chunks, idx);
+        else
+            fn.topk(grid, st, a, tk, cand, p.cand_ld, ccnt, p.max_chunks, idx);
+    };
     const size_t merge_smem = (size_t)(p.max_chunks + 1) * sizeof(int);
     if (merge_smem > 8192) {
         cudaError_t e = cudaFuncSetAttribute(merge_topk_kernel<kMergeThreads>,
@@ -335,7 +363,7 @@ int indexer_chunked(const uint8_t* q_idx, const float* w, const uint8_t* k_idx, 
                                                                        row0, k, tau);
             DSA_LAUNCH_CHECK("chunk_tau_kernel");
         }
-        fn.topk(grid, st, a, multi ? tau : nullptr, cand, p.cand_ld, ccnt, p.max_chunks, idx);
+        topk(a, grid, multi ? tau : nullptr);
         DSA_LAUNCH_CHECK("chunk_topk_kernel");
         if (!multi) continue;
         merge_topk_kernel<kMergeThreads><<<rows, kMergeThreads, merge_smem, st>>>(
@@ -344,7 +372,7 @@ int indexer_chunked(const uint8_t* q_idx, const float* w, const uint8_t* k_idx, 
         // rows the threshold left short of k: again without it
         chunk_plan_kernel<<<1, kPlanThreads, 0, st>>>(pos, k_base, T, S, row0, rows, 1, flags, work_off);
         DSA_LAUNCH_CHECK("chunk_plan_kernel");
-        fn.topk(grid, st, a, nullptr, cand, p.cand_ld, ccnt, p.max_chunks, idx);
+        topk(a, grid, nullptr);
         DSA_LAUNCH_CHECK("chunk_topk_kernel");
         merge_topk_kernel<kMergeThreads><<<rows, kMergeThreads, merge_smem, st>>>(
             cand, p.cand_ld, ccnt, p.max_chunks, pos, k_base, T, S, row0, k, 1, flags, idx);

@@ -26,6 +26,7 @@
 #pragma once
 #include "common.cuh"
 #include "indexer_scores.cuh"
+#include "sm100.cuh"
 #include "topk_select.cuh"
 
 namespace dsa {
@@ -194,6 +195,30 @@ chunk_tau_kernel(const float* __restrict__ samp, long long samp_ld, const int* _
     if (threadIdx.x == 0) tau[r] = key;
 }
 
+// Keeps the pairs of chunk c0.. of local row r (scores sc[0..m)) and writes
+// their count; a single-chunk row instead writes its final indices.
+template <int THREADS>
+__device__ __forceinline__ void chunk_keep(const float* sc, int m, int c0, int chunk, int nchunks, int r,
+                                           int t, int k, uint32_t tk, uint2* __restrict__ cand,
+                                           long long cand_ld, int* __restrict__ ccnt, int max_chunks,
+                                           int32_t* __restrict__ idx, SelectSmem<THREADS>& sm)
+{
+    if (nchunks == 1) {
+        block_topk<THREADS>(SmemScores{sc, 0}, m, k, idx + (size_t)t * k, sm);
+        return;
+    }
+    uint2* out = cand + (size_t)r * cand_ld + (size_t)chunk * k;
+    auto emit = [&](int slot, int i) { out[slot] = make_uint2(__float_as_uint(sc[i]), (uint32_t)(c0 + i)); };
+    // entries >= tau in s order (all entries when tau is 0)
+    int kept = block_emit_if<THREADS>(m, [&](int i) { return score_key(sc[i]) >= tk; }, emit, k, sm);
+    if (kept > k) {
+        // more than k pass: the chunk's own Top-k
+        block_select<THREADS>(SmemScores{sc, c0}, m, k, emit, sm);
+        kept = k;
+    }
+    if (threadIdx.x == 0) ccnt[(size_t)r * max_chunks + chunk] = kept;
+}
+
 // Persistent CTAs over the work items of rows row0 .. row0+rows-1. Chunk c of
 // local row r keeps its pairs at cand[r * cand_ld + c * k ...] and their count
 // at ccnt[r * max_chunks + c]; tau == NULL: no filtering. A single-chunk row
@@ -226,23 +251,152 @@ chunk_topk_kernel(const uint8_t* __restrict__ q_idx, const float* __restrict__ w
         qf.load(q_idx, w, t, H_I, lane);
         score_chunk<NT, DI, kThreads>(qf, k_idx + (size_t)(base + c0) * DI + tid4 * (DI / 4), m, sc);
         __syncthreads();
-        if (nchunks == 1) {
-            block_topk<kThreads>(SmemScores{sc, 0}, m, k, idx + (size_t)t * k, sm);
-        } else {
-            uint2* out = cand + (size_t)r * cand_ld + (size_t)chunk * k;
-            auto emit = [&](int slot, int i) {
-                out[slot] = make_uint2(__float_as_uint(sc[i]), (uint32_t)(c0 + i));
-            };
-            const uint32_t tk = tau ? tau[r] : 0u;
-            // entries >= tau in s order (all entries when tau is 0)
-            int kept = block_emit_if<kThreads>(m, [&](int i) { return score_key(sc[i]) >= tk; }, emit, k, sm);
-            if (kept > k) {
-                // more than k pass: the chunk's own Top-k
-                block_select<kThreads>(SmemScores{sc, c0}, m, k, emit, sm);
-                kept = k;
-            }
-            if (threadIdx.x == 0) ccnt[(size_t)r * max_chunks + chunk] = kept;
+        chunk_keep<kThreads>(sc, m, c0, chunk, nchunks, r, t, k, tau ? tau[r] : 0u, cand, cand_ld, ccnt,
+                             max_chunks, idx, sm);
+        __syncthreads();   // sc and sm are reused by the next item
+    }
+}
+
+// d_I = 128: the same work with the key rows streamed by TMA (128-key tiles,
+// 128B-swizzled, a 4-stage ring per CTA) so that many tiles are in flight
+// without holding registers. Warps 0-7 score (16 keys each per tile), warp 8
+// issues the copies; all nine take part in the selection.
+namespace tma {
+constexpr int kTileKeys = 128;
+constexpr int kTileBytes = kTileKeys * 128;
+constexpr int kStages = 4;
+constexpr int kScoreWarps = 8;
+constexpr int kThreads = (kScoreWarps + 1) * 32;
+constexpr int kCtasPerSm = 2;
+constexpr int kOffScores = kStages * kTileBytes;
+constexpr int kOffSel = kOffScores + kChunkKeys * 4;
+constexpr int kOffBar = kOffSel + (int)((sizeof(SelectSmem<kThreads>) + 15) / 16 * 16);
+constexpr int kSmemBytes = kOffBar + 128 + 1024;   // + alignment slack
+enum : int { B_FULL = 0, B_EMPTY = kStages, B_COUNT = 2 * kStages };
+static_assert(kTileKeys == kScoreWarps * 16, "one 16-key MMA block per scoring warp and tile");
+}  // namespace tma
+
+template <int NT>
+__global__ void __launch_bounds__(tma::kThreads, tma::kCtasPerSm)
+chunk_topk_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const uint8_t* __restrict__ q_idx,
+                      const float* __restrict__ w, const int* __restrict__ pos,
+                      const int* __restrict__ k_base, int T, int S, int H_I, int row0, int rows, int k,
+                      const int* __restrict__ work_off, const uint32_t* __restrict__ tau,
+                      uint2* __restrict__ cand, long long cand_ld, int* __restrict__ ccnt, int max_chunks,
+                      int32_t* __restrict__ idx)
+{
+    using namespace sm100;
+    constexpr int DI = 128;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t sbase = (raw + 1023u) & ~1023u;
+    uint8_t* sgen = smem_raw + (sbase - raw);
+    float* sc = reinterpret_cast<float*>(sgen + tma::kOffScores);
+    SelectSmem<tma::kThreads>& sm = *reinterpret_cast<SelectSmem<tma::kThreads>*>(sgen + tma::kOffSel);
+    const uint32_t bar0 = sbase + tma::kOffBar;
+    auto bar = [&](int i) -> uint32_t { return bar0 + 8u * (uint32_t)i; };
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sgen + tma::kOffBar + 8 * tma::B_COUNT);
+    int* stop_s = reinterpret_cast<int*>(sgen + tma::kOffBar + 8 * tma::B_COUNT + 4);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int gid = lane >> 2, tid4 = lane & 3;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < tma::kStages; ++s) {
+            mbar_init(bar(tma::B_FULL + s), 1);
+            mbar_init(bar(tma::B_EMPTY + s), tma::kScoreWarps);
         }
+        *abort_flag = 0;
+        fence_mbar_init_cluster();
+        prefetch_tmap(&tm_k);
+    }
+    __syncthreads();
+    const int total = work_off[rows];
+    struct Item {
+        int r, t, chunk, n, nchunks, c0, m, ntiles;
+        long long base;
+    };
+    auto item_info = [&](int item) {
+        Item it;
+        it.r = item_row(work_off, rows, item);
+        it.t = row0 + it.r;
+        it.chunk = item - work_off[it.r];
+        it.n = row_candidates(pos, k_base, it.t, T, S, &it.base);
+        it.nchunks = row_chunks(it.n);
+        it.c0 = it.chunk * kChunkKeys;
+        it.m = min(it.n - it.c0, kChunkKeys);   // 0 for an empty row
+        it.ntiles = ceil_div(max(it.m, 0), tma::kTileKeys);
+        return it;
+    };
+    // Copy warp: tiles [j0, j1) of item `it`, whose first tile is ring
+    // position g0 of this CTA.
+    auto issue = [&](const Item& it, int g0, int j0, int j1) -> bool {
+        for (int j = j0; j < j1; ++j) {
+            const int g = g0 + j, st = g % tma::kStages;
+            if (g >= tma::kStages &&
+                !mbar_wait(bar(tma::B_EMPTY + st), ((g - tma::kStages) / tma::kStages) & 1, abort_flag,
+                           600 + tma::B_EMPTY, j))
+                return false;
+            mbar_arrive_expect_tx(bar(tma::B_FULL + st), tma::kTileBytes);
+            tma_load_2d(sbase + st * tma::kTileBytes, &tm_k, 0, (int)(it.base + it.c0 + j * tma::kTileKeys),
+                        bar(tma::B_FULL + st));
+        }
+        return true;
+    };
+    const bool producer = warp == tma::kScoreWarps && lane == 0;
+    int gt = 0;   // tiles of this CTA so far (ring position and phase)
+    // the first tiles of each item are issued ahead, while the previous item
+    // is still being selected
+    if (producer && (int)blockIdx.x < total) {
+        const Item it = item_info(blockIdx.x);
+        issue(it, 0, 0, min(it.ntiles, tma::kStages));
+    }
+    for (int item = blockIdx.x; item < total; item += gridDim.x) {
+        const Item it = item_info(item);
+        if (warp == tma::kScoreWarps) {
+            if (lane == 0) issue(it, gt, min(it.ntiles, tma::kStages), it.ntiles);
+        } else {
+            QueryFrag<NT, DI> qf;
+            qf.load(q_idx, w, it.t, H_I, lane);
+            const int ra = warp * 16 + gid, rb = ra + 8;   // tile rows; both are gid mod 8
+            for (int j = 0; j < it.ntiles; ++j) {
+                const int g = gt + j, st = g % tma::kStages;
+                const bool got = mbar_wait(bar(tma::B_FULL + st), (g / tma::kStages) & 1, abort_flag,
+                                           600 + tma::B_FULL, j);
+                if (!__all_sync(0xffffffffu, got)) break;
+                const uint32_t ts = sbase + st * tma::kTileBytes;
+                KeyQuarter<DI> A, B;
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    // 16-byte chunk 2*tid4+h of the row, 128B swizzle: chunk ^ (row & 7)
+                    const uint32_t col = (uint32_t)(((2 * tid4 + h) ^ gid) << 4);
+                    const uint4 va = ld_shared_v4(ts + ra * 128 + col);
+                    const uint4 vb = ld_shared_v4(ts + rb * 128 + col);
+                    A.v[4 * h] = va.x; A.v[4 * h + 1] = va.y; A.v[4 * h + 2] = va.z; A.v[4 * h + 3] = va.w;
+                    B.v[4 * h] = vb.x; B.v[4 * h + 1] = vb.y; B.v[4 * h + 2] = vb.z; B.v[4 * h + 3] = vb.w;
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(tma::B_EMPTY + st));
+                float ia, ib;
+                qf.score(A, B, ia, ib);
+                const int a = j * tma::kTileKeys + ra, b = a + 8;
+                if (tid4 == 0) {
+                    if (a < it.m) sc[a] = ia;
+                    if (b < it.m) sc[b] = ib;
+                }
+            }
+        }
+        gt += it.ntiles;
+        __syncthreads();
+        if (threadIdx.x == 0) *stop_s = *abort_flag;
+        __syncthreads();
+        if (*stop_s) break;
+        if (producer && item + (int)gridDim.x < total) {
+            // every stage is free now: start the next item's copies
+            const Item nx = item_info(item + gridDim.x);
+            issue(nx, gt, 0, min(nx.ntiles, tma::kStages));
+        }
+        chunk_keep<tma::kThreads>(sc, it.m, it.c0, it.chunk, it.nchunks, it.r, it.t, k, tau ? tau[it.r] : 0u,
+                                  cand, cand_ld, ccnt, max_chunks, idx, sm);
         __syncthreads();   // sc and sm are reused by the next item
     }
 }

@@ -131,34 +131,48 @@ __device__ uint32_t radix_kth_key(const Row& row, int n, int k, SelectSmem<THREA
 
 // Ordered compaction: emit(slot, i) for the entries i < n with pred(i), in
 // storage order, for slots below cap. Returns the number of such entries
-// (which may exceed cap). Every thread of the CTA takes part.
+// (which may exceed cap). Every thread of the CTA takes part; thread j looks
+// at kEmitPer consecutive entries of each batch of THREADS * kEmitPer.
+constexpr int kEmitPer = 4;
+
 template <int THREADS, class Pred, class Emit>
 __device__ int block_emit_if(int n, const Pred& pred, const Emit& emit, int cap, SelectSmem<THREADS>& sm)
 {
+    constexpr int W = THREADS / 32;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (threadIdx.x == 0) sm.counter[0] = 0;
-    __syncthreads();
-    for (int c0 = 0; c0 < n; c0 += THREADS) {
-        const int i = c0 + threadIdx.x;
-        const bool take = i < n && pred(i);
-        const unsigned m = __ballot_sync(0xffffffffu, take);
-        if (lane == 0) sm.hist[0][warp] = __popc(m);
-        __syncthreads();
-        int off = sm.counter[0];
-        for (int w = 0; w < warp; ++w) off += (int)sm.hist[0][w];
-        const int slot = off + __popc(m & ((1u << lane) - 1u));
-        if (take && slot < cap) emit(slot, i);
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            int tot = 0;
-            for (int w = 0; w < THREADS / 32; ++w) tot += (int)sm.hist[0][w];
-            sm.counter[0] += tot;
+    int running = 0;
+    for (int b0 = 0; b0 < n; b0 += THREADS * kEmitPer) {
+        const int i0 = b0 + threadIdx.x * kEmitPer;
+        uint32_t bits = 0u;
+#pragma unroll
+        for (int e = 0; e < kEmitPer; ++e)
+            if (i0 + e < n && pred(i0 + e)) bits |= 1u << e;
+        const int cnt = __popc(bits);
+        int incl = cnt;   // inclusive prefix over the lanes of the warp
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += v;
         }
+        if (lane == 31) sm.hist[0][warp] = (uint32_t)incl;
         __syncthreads();
+        int slot = running + incl - cnt, total = 0;
+#pragma unroll 4
+        for (int w = 0; w < W; ++w) {
+            const int v = (int)sm.hist[0][w];
+            if (w < warp) slot += v;
+            total += v;
+        }
+#pragma unroll
+        for (int e = 0; e < kEmitPer; ++e)
+            if (bits >> e & 1u) {
+                if (slot < cap) emit(slot, i0 + e);
+                ++slot;
+            }
+        running += total;
+        __syncthreads();   // hist[0] is rewritten by the next batch
     }
-    const int total = sm.counter[0];
-    __syncthreads();
-    return total;
+    return running;
 }
 
 // Emits the Top-k of `row` (n > k entries) as emit(slot, i) for slots
