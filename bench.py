@@ -18,6 +18,7 @@ from __future__ import annotations
 
 import argparse
 import json
+import re
 import math
 import os
 import statistics
@@ -189,6 +190,24 @@ def run_attn(dsa, b, stream):
                         lse=b.lse, workspace=b.ws, stream=stream)
 
 
+def attn_traffic():
+    """DRAM bytes per prefill attention launch from the committed ncu summary,
+    or None once the kernel source has changed since those counters were taken."""
+    import hashlib
+    prof = os.path.join(ROOT, "profiles", "dram_bench_prefill128k_decode64.md")
+    csrc = os.path.join(ROOT, "sparse_attention_20_b200", "csrc")
+    try:
+        text = open(prof).read()
+        want = re.search(r"attn_source_sha256_16:\s*([0-9a-f]+)", text).group(1)
+        value = float(re.search(r"attn_traffic_bytes_per_launch:\s*([0-9.e+]+)", text).group(1))
+        h = hashlib.sha256()
+        for f in ("attn_tc.cuh", "sm100.cuh", "common.cuh"):
+            h.update(open(os.path.join(csrc, f), "rb").read())
+    except (OSError, AttributeError, ValueError):
+        return None
+    return value if h.hexdigest()[:16] == want else None
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -329,7 +348,8 @@ def bench_ours(args, world, rank, local):
         "roofline": {"bound": "tensor", "kernel": "prefill sparse MLA attention",
                      "achieved": attn_tflops, "peak": peaks["bf16_sustained"],
                      "unit": "TFLOP/s", "frac": attn_tflops / peaks["bf16_sustained"],
-                     "traffic": None,
+                     "traffic": attn_traffic() if xp.config == "prefill128k" and xp.T == 131072
+                     else None,
                      "peak_source": f"{peaks['source']} bf16 sustained"},
         "rooflines": {
             "prefill_indexer_topk": {"bound": "tensor", "unit": "TFLOP/s",
