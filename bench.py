@@ -163,6 +163,20 @@ def algorithmic_work(x):
                 attn_bytes=attn_bytes)
 
 
+def workload_config(args, xp, world):
+    """The `config` of the JSON line, the same for both arms."""
+    H_I, d_I = xp.q_idx.shape[1], xp.q_idx.shape[2]
+    Hq, d_qk = xp.q.shape[1], xp.q.shape[2]
+    dc = synth.CONFIGS[args.decode]
+    decode = (f"{dc['B']} seqs, ctx U[{dc['ctx_lo']},{dc['ctx_hi']}]" if dc["kind"] == "decode"
+              else f"{dc['L']} rows")
+    return {"workload": f"{args.prefill} causal prefill (L={xp.T}, H_I={H_I}, d_I={d_I}, k={xp.k}, "
+                        f"Hq={Hq}, d_qk={d_qk}, d_v={xp.d_v}) + {args.decode} step ({decode})",
+            "global_batch": world, "seq_len": xp.T, "parallelism": f"replicas{world}",
+            "l2": f"inputs larger than L2: {xp.T * Hq * d_qk * 2 / 1e9:.1f} GB of queries, "
+                  f"{xp.S * d_qk * 2 / 1e6:.0f} MB latent cache (L2 126 MB)"}
+
+
 class Batch:
     def __init__(self, x, dsa):
         self.x = x
@@ -246,9 +260,11 @@ def cpu_baseline(x, seed=0, target_s=15.0):
     n = max(4, threads)
     rows = sorted(torch.randperm(x.T, generator=g)[:n].tolist())
     dt, cores = time_oracle_sample(x, rows)
-    # grow once towards the target duration if the first sample was short
-    if dt < target_s / 4:
-        n2 = min(x.T, int(n * min(8.0, target_s / max(dt, 1e-3))))
+    # grow towards the target duration (at most twice) while the sample is short
+    for _ in range(2):
+        if dt >= target_s / 2 or len(rows) >= x.T:
+            break
+        n2 = min(x.T, int(len(rows) * min(64.0, target_s / max(dt, 1e-3))))
         rows = sorted(torch.randperm(x.T, generator=g)[:n2].tolist())
         dt, cores = time_oracle_sample(x, rows)
     return dict(value=len(rows) / dt, unit="tokens/s", cores=cores, kind="oracle",
@@ -330,13 +346,7 @@ def bench_ours(args, world, rank, local):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded; shapes and distributions of the pages' 128K workloads)",
-        "config": {"workload": f"{args.prefill} causal prefill (L={xp.T}, H_I={bp.H_I}, "
-                               f"d_I={bp.d_I}, k={xp.k}, Hq={bp.Hq}, d_qk={bp.d_qk}, "
-                               f"d_v={xp.d_v}) + {args.decode} step ({xd.T} "
-                               + ("seqs, ctx U[8192,131072])" if args.decode == "decode"
-                                  else "rows)"),
-                   "global_batch": world, "seq_len": xp.T, "parallelism": f"replicas{world}",
-                   "l2": "inputs larger than L2 (19 GB of queries, 151 MB latent cache)"},
+        "config": workload_config(args, xp, world),
         "prefill_tokens_per_s": tokens / (prefill_ms * 1e-3),
         "decode": {"value": world * xd.T / (decode_ms * 1e-3), "unit": "seqs/s",
                    "ms_per_step": decode_ms,
@@ -445,7 +455,7 @@ def bench_reference(args, world, rank):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": f"{args.prefill} causal prefill (sampled rows)", "seq_len": x.T},
+        "config": workload_config(args, x, world),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
