@@ -76,7 +76,9 @@ size_t dsa_workspace_size(int T, int S, int H_I, int d_I, int k, int Hq, int d_q
  *
  * Scores are formed in fp32 (FP8 products are exact in fp32). Among equal
  * scores the lower s is selected first, so the result is unique.
- * Supported: H_I <= 16, d_I in {32, 64, 128, 256}, 1 <= k <= 4096.
+ * Supported: H_I <= 16, d_I in {32, 64, 128, 256}, 1 <= k <= 4096; with pos
+ * or k_base given, or H_I != 8, or d_I != 128, S <= 2^27 (DSA_ERR_UNSUPPORTED
+ * beyond, before any launch).
  */
 int dsa_indexer_topk(const void* q_idx, const float* w, const void* k_idx, const int32_t* pos,
                      const int32_t* k_base, int T, int S, int H_I, int d_I, int k, int32_t* idx,

@@ -85,7 +85,7 @@ struct ChunkPlan {
     size_t off_work, off_flags, off_tau, off_ccnt, off_samp, off_cand, bytes;
 };
 
-constexpr int kMaxChunksPerRow = 32768;   // S <= 2^28 keys on this path
+constexpr int kMaxChunksPerRow = 16384;   // S <= 2^27 keys on this path
 
 ChunkPlan chunk_plan(int T, int S, int k)
 {
@@ -341,8 +341,9 @@ int indexer_chunked(const uint8_t* q_idx, const float* w, const uint8_t* k_idx, 
         else
             fn.topk(grid, st, a, tk, cand, p.cand_ld, ccnt, p.max_chunks, idx);
     };
-    const size_t merge_smem = (size_t)(p.max_chunks + 1) * sizeof(int);
-    if (merge_smem > 8192) {
+    const size_t merge_smem = (size_t)((p.max_chunks + 2) & ~1) * sizeof(int) +
+                              (size_t)kMergeSmemPairs * sizeof(uint2);
+    {
         cudaError_t e = cudaFuncSetAttribute(merge_topk_kernel<kMergeThreads>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)merge_smem);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(merge_topk_kernel)");

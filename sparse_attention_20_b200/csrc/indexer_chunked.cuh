@@ -36,8 +36,10 @@ constexpr int kChunkKeys = 8192;
 constexpr int kThreads = 512;
 constexpr int kCtasPerSm = 2;
 constexpr int kMergeThreads = 1024;
+constexpr int kMergeSmemPairs = 8192;   // 64 KB of staged (score, s) pairs
 constexpr int kPlanThreads = 1024;
-constexpr int kTauThreads = 256;
+constexpr int kTauThreads = 512;
+constexpr int kTauSmemSamples = 6144;   // rows up to 24 chunks stage their samples
 constexpr size_t kSmemBytes = kChunkKeys * sizeof(float) + sizeof(SelectSmem<kThreads>);
 // sampling: tiles of 128 keys, every 32nd tile of a row (two per chunk)
 constexpr int kSampleTile = 128;
@@ -127,7 +129,8 @@ __device__ __forceinline__ void score_chunk(const QueryFrag<NT, DI>& qf, const u
 }
 
 // Sample tiles of every chunk of multi-chunk rows: samp[r * samp_ld +
-// chunk * kSamplesPerChunk + j]; positions beyond the row hold -inf.
+// chunk * kSamplesPerChunk + j]; positions beyond the row hold -inf. The
+// chunk's sample keys (two tiles of 128) are one 16-key block per warp.
 template <int NT, int DI>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 chunk_sample_kernel(const uint8_t* __restrict__ q_idx, const float* __restrict__ w,
@@ -135,30 +138,32 @@ chunk_sample_kernel(const uint8_t* __restrict__ q_idx, const float* __restrict__
                     const int* __restrict__ k_base, int T, int S, int H_I, int row0, int rows,
                     const int* __restrict__ work_off, float* __restrict__ samp, long long samp_ld)
 {
-    __shared__ float sc[kSamplesPerChunk];
-    const int lane = threadIdx.x & 31;
+    static_assert(kSamplesPerChunk == 16 * (kThreads / 32), "one 16-key block per warp");
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int gid = lane >> 2, tid4 = lane & 3;
     const int total = work_off[rows];
     for (int item = blockIdx.x; item < total; item += gridDim.x) {
         const int r = item_row(work_off, rows, item), t = row0 + r;
         const int chunk = item - work_off[r];
         long long base;
         const int n = row_candidates(pos, k_base, t, T, S, &base);
-        if (row_chunks(n) < 2) continue;   // uniform over the CTA
+        if (row_chunks(n) < 2) continue;
         QueryFrag<NT, DI> qf;
         qf.load(q_idx, w, t, H_I, lane);
-        const int tid4 = lane & 3;
-#pragma unroll 1
-        for (int u = 0; u < kSamplesPerChunk / kSampleTile; ++u) {
-            const int s0 = chunk * kChunkKeys + u * kSampleStride;
-            const int m = max(0, min(kSampleTile, n - s0));
-            score_chunk<NT, DI, kThreads>(qf, k_idx + (size_t)(base + s0) * DI + tid4 * (DI / 4), m,
-                                          sc + u * kSampleTile);
-            for (int j = m + (int)threadIdx.x; j < kSampleTile; j += kThreads) sc[u * kSampleTile + j] = -INFINITY;
+        // sample position j of this chunk: tile j / 128, key j % 128 of the tile
+        const int j0 = warp * 16;
+        const int s0 = chunk * kChunkKeys + (j0 / kSampleTile) * kSampleStride + (j0 % kSampleTile);
+        const int sa = s0 + gid, sb = sa + 8;
+        KeyQuarter<DI> A, B;
+        if (sa < n) A.load(k_idx + (size_t)(base + sa) * DI + tid4 * (DI / 4)); else A.zero();
+        if (sb < n) B.load(k_idx + (size_t)(base + sb) * DI + tid4 * (DI / 4)); else B.zero();
+        float ia, ib;
+        qf.score(A, B, ia, ib);
+        if (tid4 == 0) {
+            float* out = samp + (size_t)r * samp_ld + (size_t)chunk * kSamplesPerChunk + j0;
+            out[gid] = sa < n ? ia : -INFINITY;
+            out[gid + 8] = sb < n ? ib : -INFINITY;
         }
-        __syncthreads();
-        float* out = samp + (size_t)r * samp_ld + (size_t)chunk * kSamplesPerChunk;
-        for (int j = threadIdx.x; j < kSamplesPerChunk; j += kThreads) out[j] = sc[j];
-        __syncthreads();
     }
 }
 
@@ -189,9 +194,18 @@ chunk_tau_kernel(const float* __restrict__ samp, long long samp_ld, const int* _
         if (threadIdx.x == 0) tau[r] = 0u;
         return;
     }
+    // the row's samples, staged in shared memory when they fit
+    __shared__ float ss[kTauSmemSamples];
+    const float* src = samp + (size_t)r * samp_ld;
     int take_eq, count_eq;
-    const uint32_t key = radix_kth_key<THREADS>(DenseScores{samp + (size_t)r * samp_ld}, n_s, (int)want,
-                                                sm, &take_eq, &count_eq);
+    uint32_t key;
+    if (n_s <= kTauSmemSamples) {
+        for (int j = threadIdx.x; j < n_s; j += THREADS) ss[j] = src[j];
+        __syncthreads();
+        key = radix_kth_key<THREADS>(SmemScores{ss, 0}, n_s, (int)want, sm, &take_eq, &count_eq);
+    } else {
+        key = radix_kth_key<THREADS>(DenseScores{src}, n_s, (int)want, sm, &take_eq, &count_eq);
+    }
     if (threadIdx.x == 0) tau[r] = key;
 }
 
@@ -423,7 +437,8 @@ struct ChunkPairs {
 // Row Top-k from the chunks' pairs (rows of two or more chunks). mode 0: a row
 // whose chunks kept fewer than k pairs in all is flagged for the rerun; mode 1:
 // only flagged rows. Pairs are in ascending s, and so is the emitted row.
-// Dynamic shared memory: (max_chunks + 1) ints.
+// Dynamic shared memory: (max_chunks + 2) ints (rounded to even) for the
+// prefix, then kMergeSmemPairs pairs.
 template <int THREADS>
 __global__ void __launch_bounds__(THREADS)
 merge_topk_kernel(const uint2* __restrict__ cand, long long cand_ld, const int* __restrict__ ccnt,
@@ -452,8 +467,19 @@ merge_topk_kernel(const uint2* __restrict__ cand, long long cand_ld, const int* 
         if (threadIdx.x == 0) flags[r] = 1;
         return;
     }
-    block_topk<THREADS>(ChunkPairs{cand + (size_t)r * cand_ld, pre, nchunks, k}, n_pairs, k,
-                        idx + (size_t)t * k, sm);
+    const ChunkPairs pairs{cand + (size_t)r * cand_ld, pre, nchunks, k};
+    if (n_pairs <= kMergeSmemPairs) {
+        // gather the kept pairs in chunk order into shared memory first
+        uint2* ps = reinterpret_cast<uint2*>(pre + ((max_chunks + 2) & ~1));
+        for (int c = 0; c < nchunks; ++c) {
+            const uint2* src = cand + (size_t)r * cand_ld + (size_t)c * k;
+            for (int j = threadIdx.x; j < pre[c + 1] - pre[c]; j += THREADS) ps[pre[c] + j] = src[j];
+        }
+        __syncthreads();
+        block_topk<THREADS>(PairScores{ps}, n_pairs, k, idx + (size_t)t * k, sm);
+    } else {
+        block_topk<THREADS>(pairs, n_pairs, k, idx + (size_t)t * k, sm);
+    }
 }
 
 }  // namespace idx_chunk
