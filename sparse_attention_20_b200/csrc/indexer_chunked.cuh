@@ -138,7 +138,7 @@ chunk_sample_kernel(const uint8_t* __restrict__ q_idx, const float* __restrict__
                     const int* __restrict__ k_base, int T, int S, int H_I, int row0, int rows,
                     const int* __restrict__ work_off, float* __restrict__ samp, long long samp_ld)
 {
-    static_assert(kSamplesPerChunk == 16 * (kThreads / 32), "one 16-key block per warp");
+    static_assert(kSamplesPerChunk <= 16 * (kThreads / 32), "one 16-key block per warp");
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gid = lane >> 2, tid4 = lane & 3;
     const int total = work_off[rows];
@@ -147,11 +147,11 @@ chunk_sample_kernel(const uint8_t* __restrict__ q_idx, const float* __restrict__
         const int chunk = item - work_off[r];
         long long base;
         const int n = row_candidates(pos, k_base, t, T, S, &base);
-        if (row_chunks(n) < 2) continue;
+        const int j0 = warp * 16;   // this warp's sample positions [j0, j0 + 16)
+        if (row_chunks(n) < 2 || j0 >= kSamplesPerChunk) continue;
         QueryFrag<NT, DI> qf;
         qf.load(q_idx, w, t, H_I, lane);
         // sample position j of this chunk: tile j / 128, key j % 128 of the tile
-        const int j0 = warp * 16;
         const int s0 = chunk * kChunkKeys + (j0 / kSampleTile) * kSampleStride + (j0 % kSampleTile);
         const int sa = s0 + gid, sb = sa + 8;
         KeyQuarter<DI> A, B;
