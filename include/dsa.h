@@ -151,6 +151,17 @@ const char* dsa_last_error(void);
 /* ABI version: bumped on any change of a signature or a convention. */
 int dsa_abi_version(void);
 
+/*
+ * Failure-detection self-test (no counterpart in the method). Launches one
+ * warp that waits on a barrier nothing ever signals, with the library's
+ * bounded wait shortened to limit_ms (1..2000): the wait gives up, records
+ * DSA_ERR_TIMEOUT (barrier tag 999) in the device status word, and the kernel
+ * returns; the context stays usable. Returns DSA_OK once the launch is issued
+ * (DSA_ERR_ARG for a limit outside 1..2000); read the outcome with
+ * dsa_device_status (expected: DSA_ERR_TIMEOUT, then DSA_OK on the next call).
+ */
+int dsa_selftest_bounded_wait(int limit_ms, void* stream);
+
 /* Number of kernels this process has launched through the library so far
  * (all threads, all devices): a diagnostic for launch accounting. */
 uint64_t dsa_launch_count(void);

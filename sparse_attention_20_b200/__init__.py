@@ -31,7 +31,7 @@ STATUS_NAMES = {0: "DSA_OK", -1: "DSA_ERR_ARG", -2: "DSA_ERR_UNSUPPORTED", -3: "
 # Every symbol include/dsa.h declares.
 EXPORTS = ("dsa_workspace_size", "dsa_indexer_topk", "dsa_sparse_mla_attn", "dsa_forward",
            "dsa_device_status", "dsa_last_error", "dsa_abi_version", "dsa_launch_count",
-           "dsa_indexer_topk_noalloc")
+           "dsa_indexer_topk_noalloc", "dsa_selftest_bounded_wait")
 
 
 class DSAError(RuntimeError):
@@ -68,6 +68,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.dsa_launch_count.restype = ctypes.c_uint64
         lib.dsa_indexer_topk_noalloc.argtypes = [P, P, P, P, P, I, I, I, I, I, P, P]
         lib.dsa_indexer_topk_noalloc.restype = I
+        lib.dsa_selftest_bounded_wait.argtypes = [I, P]
+        lib.dsa_selftest_bounded_wait.restype = I
         _lib = lib
     return _lib
 
@@ -199,6 +201,13 @@ def forward(q_idx, w, k_idx, q, kv, k: int, scale: float, d_v: int, pos=None, k_
 def device_status(stream=None) -> int:
     """Wait for the stream and return (and clear) the device status word."""
     return int(load_library().dsa_device_status(_stream(stream)))
+
+
+def selftest_bounded_wait(limit_ms: int = 100, stream=None) -> int:
+    """Run the failure-detection self-test and return the device status it left
+    (DSA_ERR_TIMEOUT = -4 when the bounded wait gave up as it should)."""
+    _check(load_library().dsa_selftest_bounded_wait(int(limit_ms), _stream(stream)))
+    return device_status(stream)
 
 
 def abi_version() -> int:

@@ -20,6 +20,29 @@
 #include "indexer_tc.cuh"
 #include "topk_select.cuh"
 
+namespace dsa {
+
+// One warp waits on a barrier that nothing ever signals: the bounded wait
+// gives up after limit_ns, records DSA_ERR_TIMEOUT (barrier tag 999) in the
+// device status word and the kernel returns. Exercises the failure-detection
+// path without faulting or hanging the GPU.
+__global__ void bounded_wait_selftest_kernel(uint64_t limit_ns)
+{
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    const uint32_t b = sm100::smem_u32(&bar);
+    if (threadIdx.x == 0) {
+        sm100::mbar_init(b, 1);
+        abort_flag = 0;
+    }
+    __syncthreads();
+    const bool got = sm100::mbar_wait(b, 0, &abort_flag, 999, 0, limit_ns);
+    __syncwarp();
+    (void)got;
+}
+
+}  // namespace dsa
+
 namespace {
 
 thread_local char g_err[512] = {0};
@@ -533,6 +556,16 @@ int attn_tc(const __nv_bfloat16* q, const __nv_bfloat16* kv, const int32_t* idx,
 extern "C" {
 
 int dsa_abi_version(void) { return 1; }
+
+int dsa_selftest_bounded_wait(int limit_ms, void* stream)
+{
+    g_err[0] = 0;
+    if (limit_ms < 1 || limit_ms > 2000) return fail(DSA_ERR_ARG, "limit_ms=%d (1..2000)", limit_ms);
+    dsa::bounded_wait_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        (uint64_t)limit_ms * 1000000ull);
+    DSA_LAUNCH_CHECK("bounded_wait_selftest_kernel");
+    return DSA_OK;
+}
 
 uint64_t dsa_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 

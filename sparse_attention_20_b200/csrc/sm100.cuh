@@ -100,14 +100,14 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
 template <bool kCluster = false>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          int tag = 0, int chunk = 0)
+                                          int tag = 0, int chunk = 0, uint64_t limit_ns = kWaitLimitNs)
 {
     if (kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     while (true) {
         if (kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
         if (*abort_flag) return false;
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        if (globaltimer_ns() - t0 > limit_ns) {
             *abort_flag = 1;
             report_timeout(tag, chunk, (int)parity);
             return false;

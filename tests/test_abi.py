@@ -58,7 +58,10 @@ def test_workspace_sizes(lib):
     assert 0 < ws <= 32768 * (4096 * 4 + 8192 * 8) + (1 << 20)
     assert dsa.workspace_size(0, 10, 8, 128, 2048, 128, 576, 512) == 0
     small = dsa.workspace_size(256, 256, 4, 32, 32, 4, 80, 64)
-    assert small >= 256 * 256 * 4
+    assert 0 < small < 1 << 20
+    # decode-like: 64 rows over a 4.5M-key packed cache stay within one block
+    dec = dsa.workspace_size(64, 4_500_000, 8, 128, 2048, 128, 576, 512)
+    assert 0 < dec <= 1 << 30
 
 
 FAKE = ctypes.c_void_p(0x10000)          # aligned, never dereferenced: checks fail first
@@ -118,3 +121,10 @@ def test_product_and_oracle_share_no_code():
             text = open(os.path.join(ROOT, "oracle", fn)).read()
             assert "import sparse_attention_20_b200" not in text
             assert "dsa.h" not in text
+
+
+def test_selftest_rejects_bad_limit(lib):
+    # the argument check comes before any launch
+    assert lib.dsa_selftest_bounded_wait(0, None) == -1
+    assert lib.dsa_selftest_bounded_wait(2001, None) == -1
+    assert b"limit_ms" in lib.dsa_last_error()

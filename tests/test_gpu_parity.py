@@ -197,6 +197,21 @@ def test_prefill32k_integer_indexer_bit_exact_sampled():
     check_attention(x, _take(idx, srows), _take(out, srows), _take(lse, srows), srows)
 
 
+def test_prefill_threshold_overshoot_falls_back_exactly():
+    """Causal prefill through the streaming tensor-core indexer with keys that
+    are non-zero only on every 32nd 128-key tile (where the threshold is
+    sampled): far fewer than k keys pass the sampled threshold, the select
+    kernel's exact recompute must give the oracle's Top-k (ties at score 0 go
+    to the lowest s)."""
+    x = synth.prefill_inputs("prefill32k_int", device="cuda", seed=11, L=12288)
+    s = torch.arange(x.S, device=x.k_idx.device)
+    x.k_idx[(s // 128) % 32 != 0] = 0
+    idx = dsa.indexer_topk(x.q_idx, x.w, x.k_idx, x.k)
+    torch.cuda.synchronize()
+    rows = _sampled(x.T, x.k, 48) + [x.T - 2, 4096, 4097, 8191]
+    check_indexer(x, _take(idx, rows), rows, exact=True)
+
+
 def test_prefill32k_sampled():
     x = synth.prefill_inputs("prefill32k", device="cuda", seed=0)
     idx, out, lse = _run(x)
