@@ -47,6 +47,9 @@ def parse():
     ap.add_argument("--decode", default="decode")
     ap.add_argument("--seq-len", type=int, default=None,
                     help="override L of the prefill workload (smaller cases for profiling)")
+    ap.add_argument("--rows", type=int, default=None,
+                    help="prefill only the last ROWS tokens of the sequence (long rows, small "
+                         "footprint: profiling)")
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -163,6 +166,15 @@ def algorithmic_work(x):
                 attn_bytes=attn_bytes)
 
 
+def prefill_kw(args):
+    kw = {}
+    if args.seq_len:
+        kw["L"] = args.seq_len
+    if args.rows:
+        kw["T"] = args.rows
+    return kw
+
+
 def workload_config(args, xp, world):
     """The `config` of the JSON line, the same for both arms."""
     H_I, d_I = xp.q_idx.shape[1], xp.q_idx.shape[2]
@@ -170,7 +182,8 @@ def workload_config(args, xp, world):
     dc = synth.CONFIGS[args.decode]
     decode = (f"{dc['B']} seqs, ctx U[{dc['ctx_lo']},{dc['ctx_hi']}]" if dc["kind"] == "decode"
               else f"{dc['L']} rows")
-    return {"workload": f"{args.prefill} causal prefill (L={xp.T}, H_I={H_I}, d_I={d_I}, k={xp.k}, "
+    rows = f"L={xp.T}" if xp.T == xp.S else f"last {xp.T} of L={xp.S}"
+    return {"workload": f"{args.prefill} causal prefill ({rows}, H_I={H_I}, d_I={d_I}, k={xp.k}, "
                         f"Hq={Hq}, d_qk={d_qk}, d_v={xp.d_v}) + {args.decode} step ({decode})",
             "global_batch": world, "seq_len": xp.T, "parallelism": f"replicas{world}",
             "l2": f"inputs larger than L2: {xp.T * Hq * d_qk * 2 / 1e9:.1f} GB of queries, "
@@ -283,8 +296,7 @@ def bench_ours(args, world, rank, local):
     barrier(world)
     dsa.load_library()
     dev = torch.device("cuda", torch.cuda.current_device())
-    xp = synth.make_inputs(args.prefill, device=dev, seed=args.seed + rank,
-                           **({"L": args.seq_len} if args.seq_len else {}))
+    xp = synth.make_inputs(args.prefill, device=dev, seed=args.seed + rank, **prefill_kw(args))
     xd = synth.make_inputs(args.decode, device=dev, seed=args.seed + rank)
     bp, bd = Batch(xp, dsa), Batch(xd, dsa)
     stream = torch.cuda.current_stream()
@@ -434,8 +446,7 @@ def bench_reference(args, world, rank):
     """The CPU oracle as the reference arm, on bounded samples of the same workload."""
     import oracle
     dev = "cuda" if torch.cuda.is_available() else "cpu"
-    x = synth.make_inputs(args.prefill, device=dev, seed=args.seed,
-                          **({"L": args.seq_len} if args.seq_len else {}))
+    x = synth.make_inputs(args.prefill, device=dev, seed=args.seed, **prefill_kw(args))
     threads = oracle.num_threads()
     g = torch.Generator().manual_seed(args.seed)
     per_step = max(2, threads)

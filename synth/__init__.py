@@ -165,16 +165,20 @@ def _indexer_tensors(cfg, name, T, S, base, device, with_main=True):
 
 
 def prefill_inputs(name: str = "prefill4k", device="cpu", seed: int = 0, L: int = None,
-                   overrides: dict = None) -> DSAInputs:
-    """One causal prefill sequence: T = S = L, pos[t] = t, k_base = 0."""
+                   overrides: dict = None, T: int = None) -> DSAInputs:
+    """One causal prefill sequence of L tokens: S = L keys; the queries are its
+    last T tokens (T = L by default; T < L is a chunked prefill of the tail),
+    pos[t] = t + L - T, k_base = 0."""
     cfg = dict(CONFIGS[name])
     if overrides:
         cfg.update(overrides)
     if L is not None:
         cfg["L"] = L
     L = cfg["L"]
-    q_idx, w, k_idx = _indexer_tensors(cfg, name, L, L, seed, device)
-    q = normal((L, cfg["Hq"], cfg["d_qk"]), seed, name, "q", device, dtype=torch.bfloat16)
+    T = L if T is None else int(T)
+    assert 0 < T <= L
+    q_idx, w, k_idx = _indexer_tensors(cfg, name, T, L, seed, device)
+    q = normal((T, cfg["Hq"], cfg["d_qk"]), seed, name, "q", device, dtype=torch.bfloat16)
     kv = normal((L, cfg["d_qk"]), seed, name, "kv", device, dtype=torch.bfloat16)
     return DSAInputs(name, q_idx, w, k_idx, q, kv, None, None, cfg["k"],
                      1.0 / math.sqrt(cfg["d_qk"]), cfg["d_v"], meta=cfg)

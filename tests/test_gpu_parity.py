@@ -197,6 +197,18 @@ def test_prefill32k_integer_indexer_bit_exact_sampled():
     check_attention(x, _take(idx, srows), _take(out, srows), _take(lse, srows), srows)
 
 
+def test_tail_prefill_last_rows_of_a_longer_sequence():
+    """Chunked prefill: the last 700 query rows of a 6000-token sequence (pos
+    implied as t + S - T, no explicit pos): streaming indexer and tensor-core
+    attention with every row's range starting past its own index."""
+    x = synth.prefill_inputs("prefill4k", device="cuda", seed=12, L=6000, T=700)
+    idx, out, lse = _run(x)
+    rows = list(range(x.T))
+    check_indexer(x, idx.cpu(), rows, exact=False)
+    srows = rows[::50] + [x.T - 1]
+    check_attention(x, _take(idx, srows), _take(out, srows), _take(lse, srows), srows)
+
+
 def test_prefill_threshold_overshoot_falls_back_exactly():
     """Causal prefill through the streaming tensor-core indexer with keys that
     are non-zero only on every 32nd 128-key tile (where the threshold is
