@@ -20,6 +20,22 @@ struct SelectSmem {
     int counter[2];
 };
 
+// Threads that run a block-level selection together: the whole CTA (the
+// default) or a warp-aligned subset meeting at a named barrier.
+struct CtaGroup {
+    __device__ static __forceinline__ int tid() { return (int)threadIdx.x; }
+    __device__ static __forceinline__ void sync() { __syncthreads(); }
+};
+template <int ID, int NTHREADS, int FIRST>
+struct NamedGroup {
+    static_assert(NTHREADS % 32 == 0 && FIRST % 32 == 0, "warp-aligned group");
+    __device__ static __forceinline__ int tid() { return (int)threadIdx.x - FIRST; }
+    __device__ static __forceinline__ void sync()
+    {
+        asm volatile("bar.sync %0, %1;" ::"n"(ID), "n"(NTHREADS) : "memory");
+    }
+};
+
 // Scores stored densely: entry i is candidate s = i.
 struct DenseScores {
     const float* p;
@@ -46,19 +62,19 @@ struct PairScores {
 // holds the need-th entry counted from the top (descending) or from the
 // bottom (ascending). Results: misc[0] = digit, misc[1] = rank inside the bin
 // (1-based), misc[2] = entries in the bin.
-template <int THREADS>
+template <int THREADS, class G = CtaGroup>
 __device__ __forceinline__ void select_digit(SelectSmem<THREADS>& sm, int need, bool descending)
 {
     constexpr int W = THREADS / 32;
-    for (int b = threadIdx.x; b < 256; b += THREADS) {
+    for (int b = G::tid(); b < 256; b += THREADS) {
         uint32_t s = 0;
 #pragma unroll 8
         for (int w = 0; w < W; ++w) s += sm.hist[w][b];
         sm.total[b] = s;
     }
-    __syncthreads();
-    if (threadIdx.x < 32) {
-        const int lane = threadIdx.x;
+    G::sync();
+    if (G::tid() < 32) {
+        const int lane = G::tid();
         // lane owns 8 bins; in the descending case lane 0 owns the top bins
         uint32_t c[8];
         uint32_t local = 0;
@@ -89,40 +105,40 @@ __device__ __forceinline__ void select_digit(SelectSmem<THREADS>& sm, int need, 
             }
         }
     }
-    __syncthreads();
+    G::sync();
 }
 
-template <int THREADS>
+template <int THREADS, class G = CtaGroup>
 __device__ __forceinline__ void clear_hist(SelectSmem<THREADS>& sm)
 {
     uint32_t* h = &sm.hist[0][0];
-    for (int i = threadIdx.x; i < (THREADS / 32) * 256; i += THREADS) h[i] = 0u;
-    __syncthreads();
+    for (int i = G::tid(); i < (THREADS / 32) * 256; i += THREADS) h[i] = 0u;
+    G::sync();
 }
 
 // Returns the key of the k-th largest entry; *take_eq = entries equal to it
 // that belong to the Top-k, *count_eq = entries equal to it. Requires n > k.
-template <int THREADS, class Row>
+template <int THREADS, class G = CtaGroup, class Row>
 __device__ uint32_t radix_kth_key(const Row& row, int n, int k, SelectSmem<THREADS>& sm,
                                   int* take_eq, int* count_eq)
 {
-    const int warp = threadIdx.x >> 5;
+    const int warp = G::tid() >> 5;
     uint32_t prefix = 0u, mask = 0u;
     int need = k, cnt = 0;
 #pragma unroll 1
     for (int shift = 24; shift >= 0; shift -= 8) {
-        clear_hist(sm);
-        for (int i = threadIdx.x; i < n; i += THREADS) {
+        clear_hist<THREADS, G>(sm);
+        for (int i = G::tid(); i < n; i += THREADS) {
             const uint32_t key = row.key(i);
             if ((key & mask) == prefix) atomicAdd(&sm.hist[warp][(key >> shift) & 255u], 1u);
         }
-        __syncthreads();
-        select_digit(sm, need, true);
+        G::sync();
+        select_digit<THREADS, G>(sm, need, true);
         prefix |= (uint32_t)sm.misc[0] << shift;
         mask |= 255u << shift;
         need = sm.misc[1];
         cnt = sm.misc[2];
-        __syncthreads();
+        G::sync();
     }
     *take_eq = need;
     *count_eq = cnt;
@@ -135,14 +151,14 @@ __device__ uint32_t radix_kth_key(const Row& row, int n, int k, SelectSmem<THREA
 // at kEmitPer consecutive entries of each batch of THREADS * kEmitPer.
 constexpr int kEmitPer = 4;
 
-template <int THREADS, class Pred, class Emit>
+template <int THREADS, class G = CtaGroup, class Pred, class Emit>
 __device__ int block_emit_if(int n, const Pred& pred, const Emit& emit, int cap, SelectSmem<THREADS>& sm)
 {
     constexpr int W = THREADS / 32;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int warp = G::tid() >> 5, lane = G::tid() & 31;
     int running = 0;
     for (int b0 = 0; b0 < n; b0 += THREADS * kEmitPer) {
-        const int i0 = b0 + threadIdx.x * kEmitPer;
+        const int i0 = b0 + G::tid() * kEmitPer;
         uint32_t bits = 0u;
 #pragma unroll
         for (int e = 0; e < kEmitPer; ++e)
@@ -155,7 +171,7 @@ __device__ int block_emit_if(int n, const Pred& pred, const Emit& emit, int cap,
             if (lane >= off) incl += v;
         }
         if (lane == 31) sm.hist[0][warp] = (uint32_t)incl;
-        __syncthreads();
+        G::sync();
         int slot = running + incl - cnt, total = 0;
 #pragma unroll 4
         for (int w = 0; w < W; ++w) {
@@ -170,7 +186,7 @@ __device__ int block_emit_if(int n, const Pred& pred, const Emit& emit, int cap,
                 ++slot;
             }
         running += total;
-        __syncthreads();   // hist[0] is rewritten by the next batch
+        G::sync();   // hist[0] is rewritten by the next batch
     }
     return running;
 }
@@ -178,12 +194,12 @@ __device__ int block_emit_if(int n, const Pred& pred, const Emit& emit, int cap,
 // Emits the Top-k of `row` (n > k entries) as emit(slot, i) for slots
 // 0..k-1 in storage order (for dense rows: ascending s), so the result is
 // deterministic.
-template <int THREADS, class Row, class Emit>
+template <int THREADS, class G = CtaGroup, class Row, class Emit>
 __device__ void block_select(const Row& row, int n, int k, const Emit& emit, SelectSmem<THREADS>& sm)
 {
     int take_eq, count_eq;
-    const uint32_t kth = radix_kth_key<THREADS>(row, n, k, sm, &take_eq, &count_eq);
-    const int warp = threadIdx.x >> 5;
+    const uint32_t kth = radix_kth_key<THREADS, G>(row, n, k, sm, &take_eq, &count_eq);
+    const int warp = G::tid() >> 5;
     // Index cut among the ties: the take_eq-th smallest s with key == kth.
     uint32_t s_cut = 0xFFFFFFFFu;
     if (count_eq > take_eq) {
@@ -191,23 +207,23 @@ __device__ void block_select(const Row& row, int n, int k, const Emit& emit, Sel
         int need = take_eq;
 #pragma unroll 1
         for (int shift = 24; shift >= 0; shift -= 8) {
-            clear_hist(sm);
-            for (int i = threadIdx.x; i < n; i += THREADS) {
+            clear_hist<THREADS, G>(sm);
+            for (int i = G::tid(); i < n; i += THREADS) {
                 if (row.key(i) != kth) continue;
                 const uint32_t s = (uint32_t)row.s(i);
                 if ((s & mask) == prefix) atomicAdd(&sm.hist[warp][(s >> shift) & 255u], 1u);
             }
-            __syncthreads();
-            select_digit(sm, need, false);
+            G::sync();
+            select_digit<THREADS, G>(sm, need, false);
             prefix |= (uint32_t)sm.misc[0] << shift;
             mask |= 255u << shift;
             need = sm.misc[1];
-            __syncthreads();
+            G::sync();
         }
         s_cut = prefix;
     }
     // Emit in storage order (ascending s for dense rows): ordered compaction.
-    block_emit_if<THREADS>(
+    block_emit_if<THREADS, G>(
         n,
         [&](int i) {
             const uint32_t key = row.key(i);
@@ -218,15 +234,15 @@ __device__ void block_select(const Row& row, int n, int k, const Emit& emit, Sel
 
 // Writes the Top-k of `row` (n entries) to out[0..k) in storage order; slots
 // beyond n (n < k) get -1.
-template <int THREADS, class Row>
+template <int THREADS, class G = CtaGroup, class Row>
 __device__ void block_topk(const Row& row, int n, int k, int32_t* __restrict__ out,
                            SelectSmem<THREADS>& sm)
 {
     if (n <= k) {
-        for (int i = threadIdx.x; i < k; i += THREADS) out[i] = i < n ? row.s(i) : -1;
+        for (int i = G::tid(); i < k; i += THREADS) out[i] = i < n ? row.s(i) : -1;
         return;
     }
-    block_select<THREADS>(row, n, k, [&](int slot, int i) { out[slot] = row.s(i); }, sm);
+    block_select<THREADS, G>(row, n, k, [&](int slot, int i) { out[slot] = row.s(i); }, sm);
 }
 
 constexpr int kSelectThreads = 1024;
