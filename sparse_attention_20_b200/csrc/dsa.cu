@@ -105,7 +105,7 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 struct ChunkPlan {
     int RB, max_chunks;
     long long cand_ld, samp_ld;
-    size_t off_work, off_flags, off_tau, off_ccnt, off_samp, off_cand, bytes;
+    size_t off_work, off_tau, off_ccnt, off_samp, off_cand, bytes;
 };
 
 constexpr int kMaxChunksPerRow = 16384;   // S <= 2^27 keys on this path
@@ -119,11 +119,10 @@ ChunkPlan chunk_plan(int T, int S, int k)
     p.cand_ld = multi ? (long long)p.max_chunks * k : 0;
     p.samp_ld = multi ? (long long)p.max_chunks * kSamplesPerChunk : 0;
     const size_t per_row = (size_t)p.cand_ld * sizeof(uint2) + (size_t)p.samp_ld * sizeof(float) +
-                           (size_t)p.max_chunks * sizeof(int) + 3 * sizeof(int);
+                           (size_t)p.max_chunks * sizeof(int) + 2 * sizeof(int);
     p.RB = (int)std::min<size_t>((size_t)T, std::max<size_t>(1, kScoreBlockBytes / per_row));
     p.off_work = 0;
-    p.off_flags = align_up((size_t)(p.RB + 1) * sizeof(int));
-    p.off_tau = p.off_flags + align_up((size_t)p.RB * sizeof(int));
+    p.off_tau = align_up((size_t)(p.RB + 1) * sizeof(int));
     p.off_ccnt = p.off_tau + align_up((size_t)p.RB * sizeof(uint32_t));
     p.off_samp = p.off_ccnt + align_up((size_t)p.RB * p.max_chunks * sizeof(int));
     p.off_cand = p.off_samp + align_up((size_t)p.RB * p.samp_ld * sizeof(float));
@@ -335,8 +334,8 @@ ChunkFns pick_chunk(int H_I, int d_I)
 }
 
 // Rows with their own key ranges (indexer_chunked.cuh): chunk scores and
-// sampled thresholds, chunk filters, the merge of the chunks' pairs, and the
-// rerun without threshold of any row the merge flags.
+// sampled thresholds, chunk filters, and the merge of the chunks' pairs (with
+// the exact fallback for a row the threshold left short).
 int indexer_chunked(const uint8_t* q_idx, const float* w, const uint8_t* k_idx, const int32_t* pos,
                     const int32_t* k_base, int T, int S, int H_I, int d_I, int k, int32_t* idx,
                     void* workspace, cudaStream_t st)
@@ -348,7 +347,6 @@ int indexer_chunked(const uint8_t* q_idx, const float* w, const uint8_t* k_idx, 
                     kMaxChunksPerRow * kChunkKeys);
     char* ws = reinterpret_cast<char*>(workspace);
     int* work_off = reinterpret_cast<int*>(ws + p.off_work);
-    int* flags = reinterpret_cast<int*>(ws + p.off_flags);
     uint32_t* tau = reinterpret_cast<uint32_t*>(ws + p.off_tau);
     int* ccnt = reinterpret_cast<int*>(ws + p.off_ccnt);
     float* samp = reinterpret_cast<float*>(ws + p.off_samp);
@@ -378,7 +376,7 @@ int indexer_chunked(const uint8_t* q_idx, const float* w, const uint8_t* k_idx, 
         const int grid = (int)std::min<long long>(
             (long long)rows * std::max(1, dsa::ceil_div(n_max, kChunkKeys)), resident);
         const ChunkArgs a{q_idx, w, k_idx, pos, k_base, T, S, H_I, k, row0, rows, work_off};
-        chunk_plan_kernel<<<1, kPlanThreads, 0, st>>>(pos, k_base, T, S, row0, rows, 0, flags, work_off);
+        chunk_plan_kernel<<<1, kPlanThreads, 0, st>>>(pos, k_base, T, S, row0, rows, work_off);
         DSA_LAUNCH_CHECK("chunk_plan_kernel");
         if (multi) {
             fn.sample(grid, st, a, samp, p.samp_ld);
@@ -391,15 +389,8 @@ int indexer_chunked(const uint8_t* q_idx, const float* w, const uint8_t* k_idx, 
         DSA_LAUNCH_CHECK("chunk_topk_kernel");
         if (!multi) continue;
         merge_topk_kernel<kMergeThreads><<<rows, kMergeThreads, merge_smem, st>>>(
-            cand, p.cand_ld, ccnt, p.max_chunks, pos, k_base, T, S, row0, k, 0, flags, idx);
-        DSA_LAUNCH_CHECK("merge_topk_kernel");
-        // rows the threshold left short of k: again without it
-        chunk_plan_kernel<<<1, kPlanThreads, 0, st>>>(pos, k_base, T, S, row0, rows, 1, flags, work_off);
-        DSA_LAUNCH_CHECK("chunk_plan_kernel");
-        topk(a, grid, nullptr);
-        DSA_LAUNCH_CHECK("chunk_topk_kernel");
-        merge_topk_kernel<kMergeThreads><<<rows, kMergeThreads, merge_smem, st>>>(
-            cand, p.cand_ld, ccnt, p.max_chunks, pos, k_base, T, S, row0, k, 1, flags, idx);
+            cand, p.cand_ld, ccnt, p.max_chunks, q_idx, w, k_idx, H_I, d_I, pos, k_base, T, S, row0, k,
+            idx);
         DSA_LAUNCH_CHECK("merge_topk_kernel");
     }
     return DSA_OK;

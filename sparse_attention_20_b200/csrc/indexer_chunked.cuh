@@ -17,8 +17,9 @@
 // order; if more than k pass, it keeps its own Top-k instead. Under the total
 // order (score descending, s ascending) both keep every member of the row's
 // Top-k whenever at least k entries of the row pass tau; the merge checks that
-// count, and a row short of it is run again without tau, where each chunk
-// keeps its own Top-k. The result is the row's exact Top-k either way.
+// count, and for a row short of it selects the exact Top-k of the whole row
+// from scores it recomputes itself. The result is the row's exact Top-k
+// either way.
 //
 // Work items (row, chunk) are numbered through a per-row prefix of chunk
 // counts computed on the device, so a fixed grid of persistent CTAs covers
@@ -50,19 +51,16 @@ constexpr int kAlpha = 2;   // tau aims at about kAlpha * k entries of the row
 __device__ __forceinline__ int row_chunks(int n) { return n <= kChunkKeys ? 1 : ceil_div(n, kChunkKeys); }
 
 // work_off[r] = number of work items of rows row0 .. row0+r-1, r = 0..rows.
-// mode 0: every row has row_chunks(n) items and flags[r] is cleared;
-// mode 1: only rows with flags[r] set have items.
 __global__ void __launch_bounds__(kPlanThreads)
 chunk_plan_kernel(const int* __restrict__ pos, const int* __restrict__ k_base, int T, int S, int row0,
-                  int rows, int mode, int* __restrict__ flags, int* __restrict__ work_off)
+                  int rows, int* __restrict__ work_off)
 {
     __shared__ int part[kPlanThreads];
     const int per = ceil_div(rows, kPlanThreads);
     const int r0 = threadIdx.x * per, r1 = min(rows, r0 + per);
     auto items = [&](int r) -> int {
         long long base;
-        const int c = row_chunks(row_candidates(pos, k_base, row0 + r, T, S, &base));
-        return mode == 0 ? c : (flags[r] ? c : 0);
+        return row_chunks(row_candidates(pos, k_base, row0 + r, T, S, &base));
     };
     int sum = 0;
     for (int r = r0; r < r1; ++r) sum += items(r);
@@ -79,7 +77,6 @@ chunk_plan_kernel(const int* __restrict__ pos, const int* __restrict__ k_base, i
     for (int r = r0; r < r1; ++r) {
         work_off[r] = acc;
         acc += items(r);
-        if (mode == 0) flags[r] = 0;
     }
     if (threadIdx.x == kPlanThreads - 1) work_off[rows] = part[kPlanThreads - 1];
 }
@@ -415,6 +412,46 @@ chunk_topk_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const uint8_t* _
     }
 }
 
+// Scores recomputed from the key rows (the merge's exact fallback): q^I of the
+// row as fp32 in shared memory, up to 16 heads.
+struct RecomputedRow {
+    const float* qf;      // [H_I][d_I]
+    const float* wf;      // [H_I]
+    const uint8_t* keys;  // key 0 of the row's range
+    int H_I, d_I;
+    __device__ uint32_t key(int i) const
+    {
+        const uint8_t* kr = keys + (size_t)i * d_I;
+        float dot[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) dot[j] = 0.f;
+        for (int c = 0; c < d_I; c += 16) {
+            const uint4 x = __ldg(reinterpret_cast<const uint4*>(kr + c));
+            const uint32_t wds[4] = {x.x, x.y, x.z, x.w};
+            float kf[16];
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                const float2 lo = e4m3x2_to_float2((uint16_t)(wds[h] & 0xFFFFu));
+                const float2 hi = e4m3x2_to_float2((uint16_t)(wds[h] >> 16));
+                kf[4 * h] = lo.x; kf[4 * h + 1] = lo.y; kf[4 * h + 2] = hi.x; kf[4 * h + 3] = hi.y;
+            }
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                if (j >= H_I) break;
+                const float* qj = qf + j * d_I + c;
+#pragma unroll
+                for (int e = 0; e < 16; ++e) dot[j] = fmaf(qj[e], kf[e], dot[j]);
+            }
+        }
+        float sc = 0.f;
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            if (j < H_I) sc = fmaf(wf[j], fmaxf(dot[j], 0.f), sc);
+        return score_key(sc);
+    }
+    __device__ int s(int i) const { return i; }
+};
+
 // The pairs of a row: chunk c's ccnt[c] pairs at c * k; entry i of the
 // concatenation is found through the prefix pre[] (shared memory).
 struct ChunkPairs {
@@ -434,16 +471,18 @@ struct ChunkPairs {
     __device__ __forceinline__ int s(int i) const { return (int)at(i).y; }
 };
 
-// Row Top-k from the chunks' pairs (rows of two or more chunks). mode 0: a row
-// whose chunks kept fewer than k pairs in all is flagged for the rerun; mode 1:
-// only flagged rows. Pairs are in ascending s, and so is the emitted row.
-// Dynamic shared memory: (max_chunks + 2) ints (rounded to even) for the
-// prefix, then kMergeSmemPairs pairs.
+// Row Top-k from the chunks' pairs (rows of two or more chunks). Pairs are in
+// ascending s, and so is the emitted row. A row whose chunks kept fewer than
+// k pairs in all (tau overshot) gets the exact Top-k of all its keys from
+// recomputed scores instead. Dynamic shared memory: (max_chunks + 2) ints
+// (rounded to even) for the prefix, then kMergeSmemPairs pairs (or the row's
+// q^I and w as fp32 for the fallback).
 template <int THREADS>
 __global__ void __launch_bounds__(THREADS)
 merge_topk_kernel(const uint2* __restrict__ cand, long long cand_ld, const int* __restrict__ ccnt,
-                  int max_chunks, const int* __restrict__ pos, const int* __restrict__ k_base, int T,
-                  int S, int row0, int k, int mode, int* __restrict__ flags, int32_t* __restrict__ idx)
+                  int max_chunks, const uint8_t* __restrict__ q_idx, const float* __restrict__ w,
+                  const uint8_t* __restrict__ k_idx, int H_I, int d_I, const int* __restrict__ pos,
+                  const int* __restrict__ k_base, int T, int S, int row0, int k, int32_t* __restrict__ idx)
 {
     __shared__ SelectSmem<THREADS> sm;
     extern __shared__ int pre[];
@@ -451,7 +490,7 @@ merge_topk_kernel(const uint2* __restrict__ cand, long long cand_ld, const int* 
     long long base;
     const int n = row_candidates(pos, k_base, t, T, S, &base);
     const int nchunks = row_chunks(n);
-    if (nchunks < 2 || (mode == 1 && !flags[r])) return;
+    if (nchunks < 2) return;
     if (threadIdx.x == 0) {
         int acc = 0;
         for (int c = 0; c < nchunks; ++c) {
@@ -462,15 +501,21 @@ merge_topk_kernel(const uint2* __restrict__ cand, long long cand_ld, const int* 
     }
     __syncthreads();
     const int n_pairs = pre[nchunks];
+    uint2* ps = reinterpret_cast<uint2*>(pre + ((max_chunks + 2) & ~1));
     if (n_pairs < k) {
-        // fewer than k entries passed tau: rerun this row without it
-        if (threadIdx.x == 0) flags[r] = 1;
+        // fewer than k entries passed tau: exact Top-k of the whole row
+        float* qf = reinterpret_cast<float*>(ps);
+        float* wf = qf + H_I * d_I;
+        const uint8_t* qrow = q_idx + (size_t)t * H_I * d_I;
+        for (int e = threadIdx.x; e < H_I * d_I; e += THREADS) qf[e] = e4m3x2_to_float2((uint16_t)qrow[e]).x;
+        for (int j = threadIdx.x; j < H_I; j += THREADS) wf[j] = w[(size_t)t * H_I + j];
+        __syncthreads();
+        block_topk<THREADS>(RecomputedRow{qf, wf, k_idx + (size_t)base * d_I, H_I, d_I}, n, k,
+                            idx + (size_t)t * k, sm);
         return;
     }
-    const ChunkPairs pairs{cand + (size_t)r * cand_ld, pre, nchunks, k};
     if (n_pairs <= kMergeSmemPairs) {
         // gather the kept pairs in chunk order into shared memory first
-        uint2* ps = reinterpret_cast<uint2*>(pre + ((max_chunks + 2) & ~1));
         for (int c = 0; c < nchunks; ++c) {
             const uint2* src = cand + (size_t)r * cand_ld + (size_t)c * k;
             for (int j = threadIdx.x; j < pre[c + 1] - pre[c]; j += THREADS) ps[pre[c] + j] = src[j];
@@ -478,7 +523,8 @@ merge_topk_kernel(const uint2* __restrict__ cand, long long cand_ld, const int* 
         __syncthreads();
         block_topk<THREADS>(PairScores{ps}, n_pairs, k, idx + (size_t)t * k, sm);
     } else {
-        block_topk<THREADS>(pairs, n_pairs, k, idx + (size_t)t * k, sm);
+        block_topk<THREADS>(ChunkPairs{cand + (size_t)r * cand_ld, pre, nchunks, k}, n_pairs, k,
+                            idx + (size_t)t * k, sm);
     }
 }
 
