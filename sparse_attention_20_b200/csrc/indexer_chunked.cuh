@@ -197,6 +197,7 @@ chunk_tau_kernel(const float* __restrict__ samp, long long samp_ld, const int* _
     int take_eq, count_eq;
     uint32_t key;
     if (n_s <= kTauSmemSamples) {
+#pragma unroll 4
         for (int j = threadIdx.x; j < n_s; j += THREADS) ss[j] = src[j];
         __syncthreads();
         key = radix_kth_key<THREADS>(SmemScores{ss, 0}, n_s, (int)want, sm, &take_eq, &count_eq);
@@ -491,13 +492,12 @@ merge_topk_kernel(const uint2* __restrict__ cand, long long cand_ld, const int* 
     const int n = row_candidates(pos, k_base, t, T, S, &base);
     const int nchunks = row_chunks(n);
     if (nchunks < 2) return;
+    // chunk counts loaded in parallel, then their prefix
+    for (int c = threadIdx.x; c < nchunks; c += THREADS) pre[c + 1] = ccnt[(size_t)r * max_chunks + c];
+    __syncthreads();
     if (threadIdx.x == 0) {
-        int acc = 0;
-        for (int c = 0; c < nchunks; ++c) {
-            pre[c] = acc;
-            acc += ccnt[(size_t)r * max_chunks + c];
-        }
-        pre[nchunks] = acc;
+        pre[0] = 0;
+        for (int c = 0; c < nchunks; ++c) pre[c + 1] += pre[c];
     }
     __syncthreads();
     const int n_pairs = pre[nchunks];
@@ -514,17 +514,16 @@ merge_topk_kernel(const uint2* __restrict__ cand, long long cand_ld, const int* 
                             idx + (size_t)t * k, sm);
         return;
     }
+    const ChunkPairs pairs{cand + (size_t)r * cand_ld, pre, nchunks, k};
     if (n_pairs <= kMergeSmemPairs) {
-        // gather the kept pairs in chunk order into shared memory first
-        for (int c = 0; c < nchunks; ++c) {
-            const uint2* src = cand + (size_t)r * cand_ld + (size_t)c * k;
-            for (int j = threadIdx.x; j < pre[c + 1] - pre[c]; j += THREADS) ps[pre[c] + j] = src[j];
-        }
+        // gather the kept pairs in chunk order into shared memory first (one
+        // flat loop: every load is independent)
+#pragma unroll 4
+        for (int i = threadIdx.x; i < n_pairs; i += THREADS) ps[i] = pairs.at(i);
         __syncthreads();
         block_topk<THREADS>(PairScores{ps}, n_pairs, k, idx + (size_t)t * k, sm);
     } else {
-        block_topk<THREADS>(ChunkPairs{cand + (size_t)r * cand_ld, pre, nchunks, k}, n_pairs, k,
-                            idx + (size_t)t * k, sm);
+        block_topk<THREADS>(pairs, n_pairs, k, idx + (size_t)t * k, sm);
     }
 }
 
