@@ -47,6 +47,9 @@ def parse():
     ap.add_argument("--decode", default="decode")
     ap.add_argument("--seq-len", type=int, default=None,
                     help="override L of the prefill workload (smaller cases for profiling)")
+    ap.add_argument("--varlen", default=None,
+                    help="comma-separated sequence lengths: time a packed batch of causal prefills "
+                         "(varlen indexer + attention) instead of the default step")
     ap.add_argument("--rows", type=int, default=None,
                     help="prefill only the last ROWS tokens of the sequence (long rows, small "
                          "footprint: profiling)")
@@ -516,6 +519,79 @@ def bench_reference(args, world, rank):
     }
 
 
+def bench_varlen(args, world, rank, local):
+    """Batched (variable-length) prefill: packed causal sequences of the
+    prefill128k shapes, indexer per sequence + attention with pos / k_base."""
+    import sparse_attention_20_b200 as dsa
+    from sparse_attention_20_b200 import build as dsa_build
+    if rank == 0:
+        dsa_build.build()
+    barrier(world)
+    dsa.load_library()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    lens = [int(v) for v in args.varlen.split(",")]
+    x = synth.varlen_prefill_inputs(args.prefill, device=dev, seed=args.seed + rank, lens=lens)
+    cu = x.meta["cu"]
+    H_I, d_I = x.q_idx.shape[1], x.q_idx.shape[2]
+    ws = dsa.alloc_workspace(max(lens), max(lens), H_I, d_I, x.k, x.q.shape[1], x.q.shape[2], x.d_v, dev)
+    idx = torch.empty((x.T, x.k), dtype=torch.int32, device=dev)
+    out = torch.empty((x.T, x.q.shape[1], x.d_v), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((x.T, x.q.shape[1]), dtype=torch.float32, device=dev)
+    pos, base = dsa.varlen_rows(cu, cu, dev)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev is not None: ev[0].record(stream)
+        dsa.indexer_topk_varlen(x.q_idx, x.w, x.k_idx, cu, cu, x.k, idx=idx, workspace=ws, stream=stream)
+        if ev is not None: ev[1].record(stream)
+        dsa.sparse_mla_attn(x.q, x.kv, idx, x.scale, x.d_v, pos=pos, k_base=base, out=out, lse=lse,
+                            workspace=ws, stream=stream)
+        if ev is not None: ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert dsa.device_status() == 0, dsa.last_error()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    n0 = dsa.launch_count()
+    start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    end.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    launches = dsa.launch_count() - n0
+    clk = clocks.stop()
+    ms_step = max_over_ranks(world, start.elapsed_time(end)) / args.steps
+    t_idx = max_over_ranks(world, statistics.mean(e[0].elapsed_time(e[1]) for e in evs))
+    t_attn = max_over_ranks(world, statistics.mean(e[1].elapsed_time(e[2]) for e in evs))
+    assert dsa.device_status() == 0, dsa.last_error()
+    work = algorithmic_work(x)
+    peaks = measured_peaks()
+    attn_tf = work["attn_flops"] / (t_attn * 1e-3) / 1e12
+    return {
+        "metric": "DSA batched prefill tokens/s (packed causal sequences)",
+        "value": job_throughput(world, x.T, ms_step), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{args.prefill} shapes, {len(lens)} packed sequences of {lens} tokens",
+                   "global_batch": world * len(lens), "seq_len": max(lens),
+                   "parallelism": f"replicas{world}"},
+        "kernels_ms": {"indexer_topk_varlen": t_idx, "sparse_attn": t_attn},
+        "roofline": {"bound": "tensor", "kernel": "sparse MLA attention", "achieved": attn_tf,
+                     "peak": peaks["bf16_sustained"], "unit": "TFLOP/s",
+                     "frac": attn_tf / peaks["bf16_sustained"], "traffic": None,
+                     "peak_source": f"{peaks['source']} bf16 sustained"},
+        "indexer_tflops": work["idx_flops"] / (t_idx * 1e-3) / 1e12,
+        "gpu_launches": launches, "clocks": clk,
+    }
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -525,7 +601,7 @@ def main():
             print(json.dumps(bench_reference(args, world, 0)), flush=True)
         return
     world, rank, local = dist_setup(args)
-    res = bench_ours(args, world, rank, local)
+    res = (bench_varlen if args.varlen else bench_ours)(args, world, rank, local)
     if rank == 0:
         print(json.dumps(res), flush=True)
     if world > 1:

@@ -85,6 +85,29 @@ int dsa_indexer_topk(const void* q_idx, const float* w, const void* k_idx, const
                      void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * Indexer + Top-k for a batch of packed causal sequences (variable-length
+ * prefill; the serving form of dsa_indexer_topk, no counterpart on the pages
+ * beyond the per-sequence definition).
+ *
+ *   cu_q   int32 [n_seqs+1], HOST memory: sequence b owns query rows
+ *          [cu_q[b], cu_q[b+1]) of q_idx, w and idx
+ *   cu_k   int32 [n_seqs+1], HOST memory: sequence b owns key rows
+ *          [cu_k[b], cu_k[b+1]) of k_idx
+ *
+ * Each sequence is a suffix-aligned causal prefill: its j-th query row sees
+ * keys s <= j + (S_b - T_b) of its own keys (T_b <= S_b), and idx values are
+ * relative to cu_k[b]. Equivalent to dsa_indexer_topk with
+ * pos[t] = j + S_b - T_b and k_base[t] = cu_k[b], but each sequence runs the
+ * streaming tensor-core path. cu_q[0] = cu_k[0] = 0; cu_q[b] * H_I * 4 and
+ * cu_q[b] * k * 4 must be multiples of 16 (always so for H_I = 8 and k % 4 ==
+ * 0). Workspace: dsa_workspace_size(max_b T_b, max_b S_b, ...) suffices.
+ * Sequences run one after another on `stream`.
+ */
+int dsa_indexer_topk_varlen(const void* q_idx, const float* w, const void* k_idx, const int32_t* cu_q,
+                            const int32_t* cu_k, int n_seqs, int H_I, int d_I, int k, int32_t* idx,
+                            void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * Sparse MQA attention over the selected latent rows ("Attention" and "DSA
  * under MLA (MQA Mode)", section 2 of "Paper Breakdown: DeepSeek-V3.2").
  *

@@ -31,7 +31,7 @@ STATUS_NAMES = {0: "DSA_OK", -1: "DSA_ERR_ARG", -2: "DSA_ERR_UNSUPPORTED", -3: "
 # Every symbol include/dsa.h declares.
 EXPORTS = ("dsa_workspace_size", "dsa_indexer_topk", "dsa_sparse_mla_attn", "dsa_forward",
            "dsa_device_status", "dsa_last_error", "dsa_abi_version", "dsa_launch_count",
-           "dsa_indexer_topk_noalloc", "dsa_selftest_bounded_wait")
+           "dsa_indexer_topk_noalloc", "dsa_selftest_bounded_wait", "dsa_indexer_topk_varlen")
 
 
 class DSAError(RuntimeError):
@@ -68,6 +68,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.dsa_launch_count.restype = ctypes.c_uint64
         lib.dsa_indexer_topk_noalloc.argtypes = [P, P, P, P, P, I, I, I, I, I, P, P]
         lib.dsa_indexer_topk_noalloc.restype = I
+        lib.dsa_indexer_topk_varlen.argtypes = [P, P, P, P, P, I, I, I, I, P, P, Z, P]
+        lib.dsa_indexer_topk_varlen.restype = I
         lib.dsa_selftest_bounded_wait.argtypes = [I, P]
         lib.dsa_selftest_bounded_wait.restype = I
         _lib = lib
@@ -145,6 +147,48 @@ def indexer_topk(q_idx, w, k_idx, k: int, pos=None, k_base=None, idx=None, works
     _check(lib.dsa_indexer_topk(_ptr(q_idx), _ptr(w), _ptr(k_idx), _ptr(pos), _ptr(k_base), T, S,
                                 H_I, d_I, k, _ptr(idx), _ptr(workspace), workspace.numel(),
                                 _stream(stream)))
+    return idx
+
+
+def varlen_rows(cu_q, cu_k, device):
+    """(pos, k_base) int32 [T] of a packed batch of suffix-aligned causal
+    sequences (cu_q / cu_k: host offsets): what dsa_sparse_mla_attn needs for
+    the same rows."""
+    cu_q = [int(v) for v in cu_q]
+    cu_k = [int(v) for v in cu_k]
+    pos, base = [], []
+    for b in range(len(cu_q) - 1):
+        Tb, Sb = cu_q[b + 1] - cu_q[b], cu_k[b + 1] - cu_k[b]
+        pos.extend(range(Sb - Tb, Sb))
+        base.extend([cu_k[b]] * Tb)
+    return (torch.tensor(pos, dtype=torch.int32, device=device),
+            torch.tensor(base, dtype=torch.int32, device=device))
+
+
+def indexer_topk_varlen(q_idx, w, k_idx, cu_q, cu_k, k: int, idx=None, workspace=None,
+                        stream=None) -> torch.Tensor:
+    """idx [T, k] int32 for a packed batch of causal sequences; cu_q / cu_k are
+    host offsets (lists or CPU tensors) of each sequence's query and key rows."""
+    q_idx = _fp8(q_idx, "q_idx")
+    k_idx = _fp8(k_idx, "k_idx")
+    w = _dev(w, "w")
+    if w.dtype != torch.float32:
+        raise TypeError("w must be float32")
+    T, H_I, d_I = q_idx.shape
+    cq = (ctypes.c_int32 * len(cu_q))(*[int(v) for v in cu_q])
+    ck = (ctypes.c_int32 * len(cu_k))(*[int(v) for v in cu_k])
+    if len(cu_q) != len(cu_k) or len(cu_q) < 2:
+        raise ValueError("cu_q and cu_k need n_seqs + 1 >= 2 entries each")
+    n = len(cu_q) - 1
+    if idx is None:
+        idx = torch.empty((T, k), dtype=torch.int32, device=q_idx.device)
+    if workspace is None:
+        t_max = max(cq[b + 1] - cq[b] for b in range(n))
+        s_max = max(ck[b + 1] - ck[b] for b in range(n))
+        workspace = alloc_workspace(max(t_max, 1), max(s_max, 1), H_I, d_I, k, 1, 8, 2, q_idx.device)
+    _check(load_library().dsa_indexer_topk_varlen(
+        _ptr(q_idx), _ptr(w), _ptr(k_idx), ctypes.cast(cq, ctypes.c_void_p), ctypes.cast(ck, ctypes.c_void_p),
+        n, H_I, d_I, k, _ptr(idx), _ptr(workspace), workspace.numel(), _stream(stream)))
     return idx
 
 

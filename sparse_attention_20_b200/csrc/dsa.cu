@@ -589,6 +589,47 @@ int dsa_indexer_topk(const void* q_idx, const float* w, const void* k_idx, const
                            idx, workspace, reinterpret_cast<cudaStream_t>(stream));
 }
 
+int dsa_indexer_topk_varlen(const void* q_idx, const float* w, const void* k_idx, const int32_t* cu_q,
+                            const int32_t* cu_k, int n_seqs, int H_I, int d_I, int k, int32_t* idx,
+                            void* workspace, size_t ws_bytes, void* stream)
+{
+    g_err[0] = 0;
+    if (!cu_q || !cu_k || n_seqs <= 0) return fail(DSA_ERR_ARG, "cu_q, cu_k NULL or n_seqs=%d", n_seqs);
+    if (cu_q[0] != 0 || cu_k[0] != 0) return fail(DSA_ERR_ARG, "cu_q[0] and cu_k[0] must be 0");
+    size_t need = 0;
+    for (int b = 0; b < n_seqs; ++b) {
+        const int Tb = cu_q[b + 1] - cu_q[b], Sb = cu_k[b + 1] - cu_k[b];
+        if (Tb < 0 || Sb < 0 || Tb > Sb)
+            return fail(DSA_ERR_ARG, "sequence %d: %d query rows over %d keys (need 0 <= T <= S)", b, Tb, Sb);
+        if (Tb > 0) need = std::max(need, indexer_workspace(Tb, Sb, k));
+    }
+    const int T = cu_q[n_seqs], S = cu_k[n_seqs];
+    if (int rc = check_indexer(q_idx, w, k_idx, nullptr, nullptr, T, S, H_I, d_I, k, idx)) return rc;
+    if (need && (!workspace || ws_bytes < need || !al16(workspace)))
+        return fail(DSA_ERR_WORKSPACE, "indexer needs %zu workspace bytes (got %zu)", need, ws_bytes);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const uint8_t* q8 = reinterpret_cast<const uint8_t*>(q_idx);
+    const uint8_t* k8 = reinterpret_cast<const uint8_t*>(k_idx);
+    for (int b = 0; b < n_seqs; ++b) {
+        const int Tb = cu_q[b + 1] - cu_q[b], Sb = cu_k[b + 1] - cu_k[b];
+        if (Tb == 0) continue;
+        const uint8_t* qb = q8 + (size_t)cu_q[b] * H_I * d_I;
+        const float* wb = w + (size_t)cu_q[b] * H_I;
+        const uint8_t* kb = k8 + (size_t)cu_k[b] * d_I;
+        int32_t* ib = idx + (size_t)cu_q[b] * k;
+        if (!al16(qb) || !al16(wb) || !al16(kb) || !al16(ib))
+            return fail(DSA_ERR_ARG, "sequence %d: its rows of q_idx, w, k_idx or idx are not 16-byte "
+                                     "aligned (cu_q[b] * H_I * 4 and cu_q[b] * k * 4 must be multiples "
+                                     "of 16)", b);
+        const int rc = indexer_fused_supported(nullptr, nullptr, H_I, d_I)
+                           ? indexer_fused(qb, wb, kb, Tb, Sb, k, ib, workspace, st)
+                           : indexer_chunked(qb, wb, kb, nullptr, nullptr, Tb, Sb, H_I, d_I, k, ib,
+                                             workspace, st);
+        if (rc) return rc;
+    }
+    return DSA_OK;
+}
+
 int dsa_sparse_mla_attn(const void* q, const void* kv, const int32_t* idx, const int32_t* pos,
                         const int32_t* k_base, int T, int S, int Hq, int d_qk, int d_v, int k,
                         float scale, void* out, float* lse, void* workspace, size_t ws_bytes,

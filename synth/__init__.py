@@ -184,6 +184,30 @@ def prefill_inputs(name: str = "prefill4k", device="cpu", seed: int = 0, L: int 
                      1.0 / math.sqrt(cfg["d_qk"]), cfg["d_v"], meta=cfg)
 
 
+def varlen_prefill_inputs(name: str = "prefill4k", device="cpu", seed: int = 0, lens=(700, 1500),
+                          overrides: dict = None) -> DSAInputs:
+    """A packed batch of causal prefill sequences (full prefill: each sequence's
+    queries are all of its tokens). Sequence b owns rows [cu[b], cu[b+1]) of the
+    query tensors and of the key caches; pos[t] is the row's index within its
+    sequence and k_base[t] = cu[b]. meta["cu"] holds the offsets."""
+    cfg = dict(CONFIGS[name])
+    if overrides:
+        cfg.update(overrides)
+    lens = [int(v) for v in lens]
+    cu = [0]
+    for n in lens:
+        cu.append(cu[-1] + n)
+    total = cu[-1]
+    q_idx, w, k_idx = _indexer_tensors(cfg, name + ":varlen", total, total, seed, device)
+    q = normal((total, cfg["Hq"], cfg["d_qk"]), seed, name + ":varlen", "q", device, dtype=torch.bfloat16)
+    kv = normal((total, cfg["d_qk"]), seed, name + ":varlen", "kv", device, dtype=torch.bfloat16)
+    pos = torch.cat([torch.arange(n, dtype=torch.int32) for n in lens]).to(device)
+    k_base = torch.cat([torch.full((n,), c, dtype=torch.int32) for n, c in zip(lens, cu)]).to(device)
+    meta = dict(cfg, cu=cu)
+    return DSAInputs(name + ":varlen", q_idx, w, k_idx, q, kv, pos, k_base, cfg["k"],
+                     1.0 / math.sqrt(cfg["d_qk"]), cfg["d_v"], meta=meta)
+
+
 def decode_inputs(name: str = "decode", device="cpu", seed: int = 0, B: int = None,
                   ctx: list = None, overrides: dict = None) -> DSAInputs:
     """B sequences with one query each, keys packed per sequence in one cache.

@@ -128,3 +128,18 @@ def test_selftest_rejects_bad_limit(lib):
     assert lib.dsa_selftest_bounded_wait(0, None) == -1
     assert lib.dsa_selftest_bounded_wait(2001, None) == -1
     assert b"limit_ms" in lib.dsa_last_error()
+
+
+def test_varlen_rejects_bad_offsets(lib):
+    f = lib.dsa_indexer_topk_varlen
+    ws = ctypes.c_size_t(1 << 20)
+    good = (ctypes.c_int32 * 3)(0, 4, 8)
+    bad0 = (ctypes.c_int32 * 3)(1, 4, 8)
+    fewer_keys = (ctypes.c_int32 * 3)(0, 4, 6)     # second sequence: 4 rows over 2 keys
+    cq = (ctypes.c_int32 * 3)(0, 4, 8)
+    P = lambda a: ctypes.cast(a, ctypes.c_void_p)
+    assert f(FAKE, FAKE, FAKE, None, P(good), 2, 8, 128, 2, FAKE, FAKE, ws, None) == -1
+    assert f(FAKE, FAKE, FAKE, P(bad0), P(good), 2, 8, 128, 2, FAKE, FAKE, ws, None) == -1
+    assert f(FAKE, FAKE, FAKE, P(cq), P(fewer_keys), 2, 8, 128, 2, FAKE, FAKE, ws, None) == -1
+    assert b"sequence 1" in lib.dsa_last_error()
+    assert f(FAKE, FAKE, FAKE, P(cq), P(good), 0, 8, 128, 2, FAKE, FAKE, ws, None) == -1
