@@ -108,6 +108,40 @@ int dsa_indexer_topk_varlen(const void* q_idx, const float* w, const void* k_idx
                             void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * Paged caches (the serving form of the decode path; the method itself is
+ * defined per sequence). A sequence's cache rows are pages of page_size rows
+ * (a multiple of 64) in a pool of num_pages pages:
+ *
+ *   block_table int32 [n_seqs, max_pages] (device): entry [b, j] is the pool
+ *               page holding logical keys [j*page_size, (j+1)*page_size) of
+ *               sequence b
+ *   seq         int32 [T] (device): the sequence of query row t
+ *   pos         int32 [T] (device): the last logical key row t sees
+ *
+ * idx values are logical positions within the row's sequence. Block-table
+ * entries outside [0, num_pages) are read as page 0 (no access outside the
+ * pool, wrong values); a row whose seq is outside [0, n_seqs) has no keys.
+ *
+ * dsa_indexer_topk_paged: k_pages e4m3 [num_pages * page_size, d_I], d_I = 128
+ * (H_I <= 16, k as dsa_indexer_topk); workspace as dsa_workspace_size(T,
+ * max_pages * page_size, ...).
+ */
+int dsa_indexer_topk_paged(const void* q_idx, const float* w, const void* k_pages, int num_pages,
+                           int page_size, const int32_t* block_table, int n_seqs, int max_pages,
+                           const int32_t* seq, const int32_t* pos, int T, int H_I, int d_I, int k,
+                           int32_t* idx, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * dsa_sparse_mla_attn over a paged latent cache: kv_pages bf16
+ * [num_pages * page_size, d_qk]; Hq = 128, d_qk = 576, d_v = 512 (other
+ * arguments as dsa_sparse_mla_attn; no workspace).
+ */
+int dsa_sparse_mla_attn_paged(const void* q, const void* kv_pages, int num_pages, int page_size,
+                              const int32_t* block_table, int n_seqs, int max_pages, const int32_t* seq,
+                              const int32_t* pos, const int32_t* idx, int T, int Hq, int d_qk, int d_v,
+                              int k, float scale, void* out, float* lse, void* stream);
+
+/*
  * Sparse MQA attention over the selected latent rows ("Attention" and "DSA
  * under MLA (MQA Mode)", section 2 of "Paper Breakdown: DeepSeek-V3.2").
  *

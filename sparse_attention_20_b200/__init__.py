@@ -31,7 +31,8 @@ STATUS_NAMES = {0: "DSA_OK", -1: "DSA_ERR_ARG", -2: "DSA_ERR_UNSUPPORTED", -3: "
 # Every symbol include/dsa.h declares.
 EXPORTS = ("dsa_workspace_size", "dsa_indexer_topk", "dsa_sparse_mla_attn", "dsa_forward",
            "dsa_device_status", "dsa_last_error", "dsa_abi_version", "dsa_launch_count",
-           "dsa_indexer_topk_noalloc", "dsa_selftest_bounded_wait", "dsa_indexer_topk_varlen")
+           "dsa_indexer_topk_noalloc", "dsa_selftest_bounded_wait", "dsa_indexer_topk_varlen",
+           "dsa_indexer_topk_paged", "dsa_sparse_mla_attn_paged")
 
 
 class DSAError(RuntimeError):
@@ -70,6 +71,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.dsa_indexer_topk_noalloc.restype = I
         lib.dsa_indexer_topk_varlen.argtypes = [P, P, P, P, P, I, I, I, I, P, P, Z, P]
         lib.dsa_indexer_topk_varlen.restype = I
+        lib.dsa_indexer_topk_paged.argtypes = [P, P, P, I, I, P, I, I, P, P, I, I, I, I, P, P, Z, P]
+        lib.dsa_indexer_topk_paged.restype = I
+        lib.dsa_sparse_mla_attn_paged.argtypes = [P, P, I, I, P, I, I, P, P, P, I, I, I, I, I, F, P, P, P]
+        lib.dsa_sparse_mla_attn_paged.restype = I
         lib.dsa_selftest_bounded_wait.argtypes = [I, P]
         lib.dsa_selftest_bounded_wait.restype = I
         _lib = lib
@@ -190,6 +195,49 @@ def indexer_topk_varlen(q_idx, w, k_idx, cu_q, cu_k, k: int, idx=None, workspace
         _ptr(q_idx), _ptr(w), _ptr(k_idx), ctypes.cast(cq, ctypes.c_void_p), ctypes.cast(ck, ctypes.c_void_p),
         n, H_I, d_I, k, _ptr(idx), _ptr(workspace), workspace.numel(), _stream(stream)))
     return idx
+
+
+def indexer_topk_paged(q_idx, w, k_pages, page_size: int, block_table, seq, pos, k: int, idx=None,
+                       workspace=None, stream=None) -> torch.Tensor:
+    """idx [T, k] over a paged FP8 key cache (k_pages [num_pages*page_size, d_I],
+    block_table [n_seqs, max_pages], seq / pos [T]; see include/dsa.h)."""
+    q_idx, k_pages = _fp8(q_idx, "q_idx"), _fp8(k_pages, "k_pages")
+    w = _dev(w, "w")
+    block_table, seq, pos = _i32(block_table, "block_table"), _i32(seq, "seq"), _i32(pos, "pos")
+    T, H_I, d_I = q_idx.shape
+    num_pages = k_pages.shape[0] // page_size
+    n_seqs, max_pages = block_table.shape
+    if idx is None:
+        idx = torch.empty((T, k), dtype=torch.int32, device=q_idx.device)
+    if workspace is None:
+        workspace = alloc_workspace(T, max_pages * page_size, H_I, d_I, k, 1, 8, 2, q_idx.device)
+    _check(load_library().dsa_indexer_topk_paged(
+        _ptr(q_idx), _ptr(w), _ptr(k_pages), num_pages, page_size, _ptr(block_table), n_seqs, max_pages,
+        _ptr(seq), _ptr(pos), T, H_I, d_I, k, _ptr(idx), _ptr(workspace), workspace.numel(),
+        _stream(stream)))
+    return idx
+
+
+def sparse_mla_attn_paged(q, kv_pages, page_size: int, block_table, seq, pos, idx, scale: float,
+                          d_v: int, out=None, lse=None, stream=None):
+    """(out, lse) of sparse MQA attention over a paged latent cache."""
+    q, kv_pages = _dev(q, "q"), _dev(kv_pages, "kv_pages")
+    if q.dtype != torch.bfloat16 or kv_pages.dtype != torch.bfloat16:
+        raise TypeError("q and kv_pages must be bfloat16")
+    block_table, seq, pos = _i32(block_table, "block_table"), _i32(seq, "seq"), _i32(pos, "pos")
+    idx = _i32(idx, "idx")
+    T, Hq, d_qk = q.shape
+    num_pages = kv_pages.shape[0] // page_size
+    n_seqs, max_pages = block_table.shape
+    if out is None:
+        out = torch.empty((T, Hq, d_v), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((T, Hq), dtype=torch.float32, device=q.device)
+    _check(load_library().dsa_sparse_mla_attn_paged(
+        _ptr(q), _ptr(kv_pages), num_pages, page_size, _ptr(block_table), n_seqs, max_pages, _ptr(seq),
+        _ptr(pos), _ptr(idx), T, Hq, d_qk, d_v, idx.shape[1], float(scale), _ptr(out), _ptr(lse),
+        _stream(stream)))
+    return out, lse
 
 
 def sparse_mla_attn(q, kv, idx, scale: float, d_v: int, pos=None, k_base=None, out=None,

@@ -133,7 +133,7 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
                           const __nv_bfloat16* __restrict__ kv,
                           const int* __restrict__ idx, const int* __restrict__ pos,
                           const int* __restrict__ k_base, int T, int S, int k, float scale_log2,
-                          __nv_bfloat16* __restrict__ out, float* __restrict__ lse)
+                          __nv_bfloat16* __restrict__ out, float* __restrict__ lse, const PagedRows pg)
 {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -149,7 +149,8 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
     const uint32_t peer = rank ^ 1u;
     const int t = T - 1 - (int)(blockIdx.x >> 1);   // long rows first
     long long base;
-    const int n_cand = row_candidates(pos, k_base, t, T, S, &base);
+    const int* bt;   // block-table line of a paged cache, else NULL
+    const int n_cand = row_keys(pg, pos, k_base, t, T, S, &base, &bt);
     const int p_last = n_cand - 1;
     const int n_row = min(k, n_cand);
     const int NC = ceil_div(n_row, kKeys);
@@ -308,8 +309,8 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
                 if (!__all_sync(0xffffffffu, got)) break;   // warp-uniform exit
             }
             const bool va = sa >= 0 && sa <= p_last, vb = sb >= 0 && sb <= p_last;
-            rows_tab[lane] = va ? (base + sa) * (long long)(kDqk * 2) : -1ll;
-            rows_tab[lane + 32] = vb ? (base + sb) * (long long)(kDqk * 2) : -1ll;
+            rows_tab[lane] = va ? key_row(pg, bt, base, sa) * (long long)(kDqk * 2) : -1ll;
+            rows_tab[lane + 32] = vb ? key_row(pg, bt, base, sb) * (long long)(kDqk * 2) : -1ll;
             if (gw == 0) {
                 const unsigned ma = __ballot_sync(0xffffffffu, va), mb = __ballot_sync(0xffffffffu, vb);
                 if (lane == 0) {

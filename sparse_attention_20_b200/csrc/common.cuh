@@ -77,4 +77,42 @@ __device__ __forceinline__ int row_candidates(const int* pos, const int* k_base,
     return (int)min(p + 1, (long long)S - base);
 }
 
+// A paged cache (serving form): logical key s of query row t lives at physical
+// row block_table[seq[t] * max_pages + s / page_size] * page_size + s % page_size.
+// block_table == NULL: keys are contiguous from k_base[t] (row_candidates).
+struct PagedRows {
+    const int* block_table = nullptr;
+    const int* seq = nullptr;
+    int n_seqs = 0, max_pages = 0, page_size = 1, num_pages = 0;
+};
+
+// Key count of row t; *base and *bt say where its keys live (key_row).
+__device__ __forceinline__ int row_keys(const PagedRows& pg, const int* pos, const int* k_base, int t,
+                                        int T, int S, long long* base, const int** bt)
+{
+    if (!pg.block_table) {
+        *bt = nullptr;
+        return row_candidates(pos, k_base, t, T, S, base);
+    }
+    *base = 0;
+    const int sq = pg.seq[t];
+    const long long p = pos[t];
+    if (sq < 0 || sq >= pg.n_seqs || p < 0) {
+        *bt = nullptr;
+        return 0;
+    }
+    *bt = pg.block_table + (size_t)sq * pg.max_pages;
+    return (int)min(p + 1, (long long)pg.max_pages * pg.page_size);
+}
+
+// Physical row of logical key s (0 <= s < row_keys). A block-table entry out
+// of range reads page 0: wrong values, but no access outside the cache.
+__device__ __forceinline__ long long key_row(const PagedRows& pg, const int* bt, long long base, int s)
+{
+    if (!bt) return base + s;
+    int page = bt[s / pg.page_size];
+    if ((unsigned)page >= (unsigned)pg.num_pages) page = 0;
+    return (long long)page * pg.page_size + s % pg.page_size;
+}
+
 }  // namespace dsa

@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <climits>
 #include <atomic>
 #include <cstdarg>
 #include <cstdio>
@@ -270,6 +271,7 @@ struct ChunkArgs {
     const int* k_base;
     int T, S, H_I, k, row0, rows;
     const int* work_off;
+    dsa::PagedRows pg;
 };
 
 template <int NT, int DI>
@@ -279,7 +281,7 @@ struct ChunkKernels {
         using namespace dsa::idx_chunk;
         chunk_sample_kernel<NT, DI><<<grid, kThreads, 0, st>>>(a.q_idx, a.w, a.k_idx, a.pos, a.k_base, a.T,
                                                               a.S, a.H_I, a.row0, a.rows, a.work_off,
-                                                              samp, samp_ld);
+                                                              samp, samp_ld, a.pg);
     }
     static void topk(int grid, cudaStream_t st, const ChunkArgs& a, const uint32_t* tau, uint2* cand,
                      long long cand_ld, int* ccnt, int max_chunks, int32_t* idx)
@@ -304,7 +306,7 @@ void chunk_topk_tma(int grid, cudaStream_t st, const CUtensorMap& tm_k, const Ch
                          tma::kSmemBytes);
     chunk_topk_tma_kernel<NT><<<grid, tma::kThreads, tma::kSmemBytes, st>>>(
         tm_k, a.q_idx, a.w, a.pos, a.k_base, a.T, a.S, a.H_I, a.row0, a.rows, a.k, a.work_off, tau, cand,
-        cand_ld, ccnt, max_chunks, idx);
+        cand_ld, ccnt, max_chunks, idx, a.pg);
 }
 
 struct ChunkFns {
@@ -336,9 +338,11 @@ ChunkFns pick_chunk(int H_I, int d_I)
 // Rows with their own key ranges (indexer_chunked.cuh): chunk scores and
 // sampled thresholds, chunk filters, and the merge of the chunks' pairs (with
 // the exact fallback for a row the threshold left short).
+// S: the most keys a row can have; a paged cache (pg.block_table) holds
+// pg.num_pages * pg.page_size key rows.
 int indexer_chunked(const uint8_t* q_idx, const float* w, const uint8_t* k_idx, const int32_t* pos,
                     const int32_t* k_base, int T, int S, int H_I, int d_I, int k, int32_t* idx,
-                    void* workspace, cudaStream_t st)
+                    void* workspace, cudaStream_t st, const dsa::PagedRows& pg = {})
 {
     using namespace dsa::idx_chunk;
     const ChunkPlan p = chunk_plan(T, S, k);
@@ -352,9 +356,15 @@ int indexer_chunked(const uint8_t* q_idx, const float* w, const uint8_t* k_idx, 
     float* samp = reinterpret_cast<float*>(ws + p.off_samp);
     uint2* cand = reinterpret_cast<uint2*>(ws + p.off_cand);
     const ChunkFns fn = pick_chunk(H_I, d_I);
+    const bool paged = pg.block_table != nullptr;
+    if (paged && !fn.topk_tma)
+        return fail(DSA_ERR_UNSUPPORTED, "a paged key cache needs d_I = 128 (got %d)", d_I);
     CUtensorMap tm_k;
-    if (fn.topk_tma)
-        if (int rc = make_tmap_u8(&tm_k, k_idx, 128, (uint64_t)S, tma::kTileKeys)) return rc;
+    if (fn.topk_tma) {
+        const uint64_t key_rows = paged ? (uint64_t)pg.num_pages * pg.page_size : (uint64_t)S;
+        if (int rc = make_tmap_u8(&tm_k, k_idx, 128, key_rows, paged ? tma::kTileKeys / 2 : tma::kTileKeys))
+            return rc;
+    }
     const int resident = (fn.topk_tma ? tma::kCtasPerSm : kCtasPerSm) * num_sms();
     auto topk = [&](const ChunkArgs& a, int grid, const uint32_t* tk) {
         if (fn.topk_tma)
@@ -375,14 +385,14 @@ int indexer_chunked(const uint8_t* q_idx, const float* w, const uint8_t* k_idx, 
         const bool multi = n_max > kChunkKeys;
         const int grid = (int)std::min<long long>(
             (long long)rows * std::max(1, dsa::ceil_div(n_max, kChunkKeys)), resident);
-        const ChunkArgs a{q_idx, w, k_idx, pos, k_base, T, S, H_I, k, row0, rows, work_off};
-        chunk_plan_kernel<<<1, kPlanThreads, 0, st>>>(pos, k_base, T, S, row0, rows, work_off);
+        const ChunkArgs a{q_idx, w, k_idx, pos, k_base, T, S, H_I, k, row0, rows, work_off, pg};
+        chunk_plan_kernel<<<1, kPlanThreads, 0, st>>>(pos, k_base, T, S, row0, rows, work_off, pg);
         DSA_LAUNCH_CHECK("chunk_plan_kernel");
         if (multi) {
             fn.sample(grid, st, a, samp, p.samp_ld);
             DSA_LAUNCH_CHECK("chunk_sample_kernel");
             chunk_tau_kernel<kTauThreads><<<rows, kTauThreads, 0, st>>>(samp, p.samp_ld, pos, k_base, T, S,
-                                                                       row0, k, tau);
+                                                                       row0, k, tau, pg);
             DSA_LAUNCH_CHECK("chunk_tau_kernel");
         }
         topk(a, grid, multi ? tau : nullptr);
@@ -390,7 +400,7 @@ int indexer_chunked(const uint8_t* q_idx, const float* w, const uint8_t* k_idx, 
         if (!multi) continue;
         merge_topk_kernel<kMergeThreads><<<rows, kMergeThreads, merge_smem, st>>>(
             cand, p.cand_ld, ccnt, p.max_chunks, q_idx, w, k_idx, H_I, d_I, pos, k_base, T, S, row0, k,
-            idx);
+            idx, pg);
         DSA_LAUNCH_CHECK("merge_topk_kernel");
     }
     return DSA_OK;
@@ -519,7 +529,7 @@ int make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t cols, uint64_t row
 
 int attn_tc(const __nv_bfloat16* q, const __nv_bfloat16* kv, const int32_t* idx,
             const int32_t* pos, const int32_t* k_base, int T, int S, int k, float scale,
-            __nv_bfloat16* out, float* lse, cudaStream_t st)
+            __nv_bfloat16* out, float* lse, cudaStream_t st, const dsa::PagedRows& pg = {})
 {
     using namespace dsa::attn_tc;
     cudaError_t e = cudaFuncSetAttribute(sparse_mla_attn_tc_kernel,
@@ -535,7 +545,7 @@ int attn_tc(const __nv_bfloat16* q, const __nv_bfloat16* kv, const int32_t* idx,
                                 CU_TENSOR_MAP_SWIZZLE_64B)) return rc;
     const float scale_log2 = scale * 1.4426950408889634f;
     sparse_mla_attn_tc_kernel<<<dim3(2 * T), kThreads, kSmemBytes, st>>>(
-        tq128, tq64, q, kv, idx, pos, k_base, T, S, k, scale_log2, out, lse);
+        tq128, tq64, q, kv, idx, pos, k_base, T, S, k, scale_log2, out, lse, pg);
     DSA_LAUNCH_CHECK("sparse_mla_attn_tc_kernel");
     return DSA_OK;
 }
@@ -628,6 +638,74 @@ int dsa_indexer_topk_varlen(const void* q_idx, const float* w, const void* k_idx
         if (rc) return rc;
     }
     return DSA_OK;
+}
+
+namespace {
+int check_paged(const void* cache, int num_pages, int page_size, const int32_t* block_table, int n_seqs,
+                int max_pages, const int32_t* seq, const int32_t* pos, int T)
+{
+    if (!cache || !block_table || !seq || !pos) return fail(DSA_ERR_ARG, "NULL cache, block_table, seq or pos");
+    if (!al16(cache) || !al16(block_table) || !al16(seq) || !al16(pos))
+        return fail(DSA_ERR_ARG, "cache, block_table, seq and pos must be 16-byte aligned");
+    if (T <= 0 || num_pages <= 0 || n_seqs <= 0 || max_pages <= 0)
+        return fail(DSA_ERR_ARG, "T=%d, num_pages=%d, n_seqs=%d, max_pages=%d must be positive", T,
+                    num_pages, n_seqs, max_pages);
+    if (page_size <= 0 || page_size % 64 != 0)
+        return fail(DSA_ERR_UNSUPPORTED, "page_size=%d (supported: multiples of 64)", page_size);
+    if ((long long)num_pages * page_size > INT32_MAX || (long long)max_pages * page_size > INT32_MAX)
+        return fail(DSA_ERR_UNSUPPORTED, "cache of more than 2^31 rows");
+    return DSA_OK;
+}
+}  // namespace
+
+int dsa_indexer_topk_paged(const void* q_idx, const float* w, const void* k_pages, int num_pages,
+                           int page_size, const int32_t* block_table, int n_seqs, int max_pages,
+                           const int32_t* seq, const int32_t* pos, int T, int H_I, int d_I, int k,
+                           int32_t* idx, void* workspace, size_t ws_bytes, void* stream)
+{
+    g_err[0] = 0;
+    if (int rc = check_paged(k_pages, num_pages, page_size, block_table, n_seqs, max_pages, seq, pos, T))
+        return rc;
+    const int S = max_pages * page_size;   // the most keys a row can have
+    if (int rc = check_indexer(q_idx, w, k_pages, pos, nullptr, T, S, H_I, d_I, k, idx)) return rc;
+    if (d_I != 128) return fail(DSA_ERR_UNSUPPORTED, "a paged key cache needs d_I = 128 (got %d)", d_I);
+    const size_t need = indexer_workspace(T, S, k);
+    if (need && (!workspace || ws_bytes < need || !al16(workspace)))
+        return fail(DSA_ERR_WORKSPACE, "indexer needs %zu workspace bytes (got %zu)", need, ws_bytes);
+    dsa::PagedRows pg;
+    pg.block_table = block_table;
+    pg.seq = seq;
+    pg.n_seqs = n_seqs;
+    pg.max_pages = max_pages;
+    pg.page_size = page_size;
+    pg.num_pages = num_pages;
+    return indexer_chunked(reinterpret_cast<const uint8_t*>(q_idx), w,
+                           reinterpret_cast<const uint8_t*>(k_pages), pos, nullptr, T, S, H_I, d_I, k, idx,
+                           workspace, reinterpret_cast<cudaStream_t>(stream), pg);
+}
+
+int dsa_sparse_mla_attn_paged(const void* q, const void* kv_pages, int num_pages, int page_size,
+                              const int32_t* block_table, int n_seqs, int max_pages, const int32_t* seq,
+                              const int32_t* pos, const int32_t* idx, int T, int Hq, int d_qk, int d_v,
+                              int k, float scale, void* out, float* lse, void* stream)
+{
+    g_err[0] = 0;
+    if (int rc = check_paged(kv_pages, num_pages, page_size, block_table, n_seqs, max_pages, seq, pos, T))
+        return rc;
+    const int S = num_pages * page_size;
+    if (int rc = check_attn(q, kv_pages, idx, pos, nullptr, T, S, Hq, d_qk, d_v, k, out, lse)) return rc;
+    if (!attn_tc_supported(Hq, d_qk, d_v, k))
+        return fail(DSA_ERR_UNSUPPORTED, "a paged latent cache needs Hq = 128, d_qk = 576, d_v = 512");
+    dsa::PagedRows pg;
+    pg.block_table = block_table;
+    pg.seq = seq;
+    pg.n_seqs = n_seqs;
+    pg.max_pages = max_pages;
+    pg.page_size = page_size;
+    pg.num_pages = num_pages;
+    return attn_tc(reinterpret_cast<const __nv_bfloat16*>(q), reinterpret_cast<const __nv_bfloat16*>(kv_pages),
+                   idx, pos, nullptr, T, S, k, scale, reinterpret_cast<__nv_bfloat16*>(out), lse,
+                   reinterpret_cast<cudaStream_t>(stream), pg);
 }
 
 int dsa_sparse_mla_attn(const void* q, const void* kv, const int32_t* idx, const int32_t* pos,

@@ -53,14 +53,15 @@ __device__ __forceinline__ int row_chunks(int n) { return n <= kChunkKeys ? 1 : 
 // work_off[r] = number of work items of rows row0 .. row0+r-1, r = 0..rows.
 __global__ void __launch_bounds__(kPlanThreads)
 chunk_plan_kernel(const int* __restrict__ pos, const int* __restrict__ k_base, int T, int S, int row0,
-                  int rows, int* __restrict__ work_off)
+                  int rows, int* __restrict__ work_off, const PagedRows pg)
 {
     __shared__ int part[kPlanThreads];
     const int per = ceil_div(rows, kPlanThreads);
     const int r0 = threadIdx.x * per, r1 = min(rows, r0 + per);
     auto items = [&](int r) -> int {
         long long base;
-        return row_chunks(row_candidates(pos, k_base, row0 + r, T, S, &base));
+        const int* bt;
+        return row_chunks(row_keys(pg, pos, k_base, row0 + r, T, S, &base, &bt));
     };
     int sum = 0;
     for (int r = r0; r < r1; ++r) sum += items(r);
@@ -133,7 +134,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 chunk_sample_kernel(const uint8_t* __restrict__ q_idx, const float* __restrict__ w,
                     const uint8_t* __restrict__ k_idx, const int* __restrict__ pos,
                     const int* __restrict__ k_base, int T, int S, int H_I, int row0, int rows,
-                    const int* __restrict__ work_off, float* __restrict__ samp, long long samp_ld)
+                    const int* __restrict__ work_off, float* __restrict__ samp, long long samp_ld,
+                    const PagedRows pg)
 {
     static_assert(kSamplesPerChunk <= 16 * (kThreads / 32), "one 16-key block per warp");
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -143,7 +145,8 @@ chunk_sample_kernel(const uint8_t* __restrict__ q_idx, const float* __restrict__
         const int r = item_row(work_off, rows, item), t = row0 + r;
         const int chunk = item - work_off[r];
         long long base;
-        const int n = row_candidates(pos, k_base, t, T, S, &base);
+        const int* bt;
+        const int n = row_keys(pg, pos, k_base, t, T, S, &base, &bt);
         const int j0 = warp * 16;   // this warp's sample positions [j0, j0 + 16)
         if (row_chunks(n) < 2 || j0 >= kSamplesPerChunk) continue;
         QueryFrag<NT, DI> qf;
@@ -152,8 +155,8 @@ chunk_sample_kernel(const uint8_t* __restrict__ q_idx, const float* __restrict__
         const int s0 = chunk * kChunkKeys + (j0 / kSampleTile) * kSampleStride + (j0 % kSampleTile);
         const int sa = s0 + gid, sb = sa + 8;
         KeyQuarter<DI> A, B;
-        if (sa < n) A.load(k_idx + (size_t)(base + sa) * DI + tid4 * (DI / 4)); else A.zero();
-        if (sb < n) B.load(k_idx + (size_t)(base + sb) * DI + tid4 * (DI / 4)); else B.zero();
+        if (sa < n) A.load(k_idx + (size_t)key_row(pg, bt, base, sa) * DI + tid4 * (DI / 4)); else A.zero();
+        if (sb < n) B.load(k_idx + (size_t)key_row(pg, bt, base, sb) * DI + tid4 * (DI / 4)); else B.zero();
         float ia, ib;
         qf.score(A, B, ia, ib);
         if (tid4 == 0) {
@@ -177,12 +180,13 @@ template <int THREADS>
 __global__ void __launch_bounds__(THREADS)
 chunk_tau_kernel(const float* __restrict__ samp, long long samp_ld, const int* __restrict__ pos,
                  const int* __restrict__ k_base, int T, int S, int row0, int k,
-                 uint32_t* __restrict__ tau)
+                 uint32_t* __restrict__ tau, const PagedRows pg)
 {
     __shared__ SelectSmem<THREADS> sm;
     const int r = blockIdx.x, t = row0 + r;
     long long base;
-    const int n = row_candidates(pos, k_base, t, T, S, &base);
+    const int* bt;
+    const int n = row_keys(pg, pos, k_base, t, T, S, &base, &bt);
     const int nchunks = row_chunks(n);
     const int m = row_samples(n);
     const long long want = ((long long)kAlpha * k * m + n - 1) / n;
@@ -244,6 +248,7 @@ chunk_topk_kernel(const uint8_t* __restrict__ q_idx, const float* __restrict__ w
                   uint2* __restrict__ cand, long long cand_ld, int* __restrict__ ccnt, int max_chunks,
                   int32_t* __restrict__ idx)
 {
+    // contiguous key ranges only (a paged cache takes the TMA kernel below)
     extern __shared__ __align__(16) uint8_t smem[];
     float* sc = reinterpret_cast<float*>(smem);
     SelectSmem<kThreads>& sm = *reinterpret_cast<SelectSmem<kThreads>*>(smem + kChunkKeys * sizeof(float));
@@ -295,8 +300,10 @@ chunk_topk_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const uint8_t* _
                       const int* __restrict__ k_base, int T, int S, int H_I, int row0, int rows, int k,
                       const int* __restrict__ work_off, const uint32_t* __restrict__ tau,
                       uint2* __restrict__ cand, long long cand_ld, int* __restrict__ ccnt, int max_chunks,
-                      int32_t* __restrict__ idx)
+                      int32_t* __restrict__ idx, const PagedRows pg)
 {
+    // tm_k boxes: 128 key rows (contiguous ranges) or 64 (paged cache: a tile
+    // is two half-tiles, each inside one page of a multiple of 64 keys)
     using namespace sm100;
     constexpr int DI = 128;
     extern __shared__ uint8_t smem_raw[];
@@ -326,13 +333,14 @@ chunk_topk_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const uint8_t* _
     struct Item {
         int r, t, chunk, n, nchunks, c0, m, ntiles;
         long long base;
+        const int* bt;
     };
     auto item_info = [&](int item) {
         Item it;
         it.r = item_row(work_off, rows, item);
         it.t = row0 + it.r;
         it.chunk = item - work_off[it.r];
-        it.n = row_candidates(pos, k_base, it.t, T, S, &it.base);
+        it.n = row_keys(pg, pos, k_base, it.t, T, S, &it.base, &it.bt);
         it.nchunks = row_chunks(it.n);
         it.c0 = it.chunk * kChunkKeys;
         it.m = min(it.n - it.c0, kChunkKeys);   // 0 for an empty row
@@ -349,8 +357,19 @@ chunk_topk_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const uint8_t* _
                            600 + tma::B_EMPTY, j))
                 return false;
             mbar_arrive_expect_tx(bar(tma::B_FULL + st), tma::kTileBytes);
-            tma_load_2d(sbase + st * tma::kTileBytes, &tm_k, 0, (int)(it.base + it.c0 + j * tma::kTileKeys),
-                        bar(tma::B_FULL + st));
+            const int s0 = it.c0 + j * tma::kTileKeys;
+            if (it.bt) {
+                tma_load_2d(sbase + st * tma::kTileBytes, &tm_k, 0, (int)key_row(pg, it.bt, 0, s0),
+                            bar(tma::B_FULL + st));
+                // a second half that starts past the row's keys reloads the
+                // first half (never scored) instead of naming a page the row
+                // does not have
+                const int s1 = s0 + tma::kTileKeys / 2 < it.n ? s0 + tma::kTileKeys / 2 : s0;
+                tma_load_2d(sbase + st * tma::kTileBytes + tma::kTileBytes / 2, &tm_k, 0,
+                            (int)key_row(pg, it.bt, 0, s1), bar(tma::B_FULL + st));
+            } else {
+                tma_load_2d(sbase + st * tma::kTileBytes, &tm_k, 0, (int)(it.base + s0), bar(tma::B_FULL + st));
+            }
         }
         return true;
     };
@@ -418,11 +437,14 @@ chunk_topk_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const uint8_t* _
 struct RecomputedRow {
     const float* qf;      // [H_I][d_I]
     const float* wf;      // [H_I]
-    const uint8_t* keys;  // key 0 of the row's range
+    const uint8_t* k_idx; // the key cache
+    PagedRows pg;
+    const int* bt;        // the row's block-table line (paged), else NULL
+    long long base;       // first key of the row's range (contiguous)
     int H_I, d_I;
     __device__ uint32_t key(int i) const
     {
-        const uint8_t* kr = keys + (size_t)i * d_I;
+        const uint8_t* kr = k_idx + (size_t)key_row(pg, bt, base, i) * d_I;
         float dot[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) dot[j] = 0.f;
@@ -483,13 +505,15 @@ __global__ void __launch_bounds__(THREADS)
 merge_topk_kernel(const uint2* __restrict__ cand, long long cand_ld, const int* __restrict__ ccnt,
                   int max_chunks, const uint8_t* __restrict__ q_idx, const float* __restrict__ w,
                   const uint8_t* __restrict__ k_idx, int H_I, int d_I, const int* __restrict__ pos,
-                  const int* __restrict__ k_base, int T, int S, int row0, int k, int32_t* __restrict__ idx)
+                  const int* __restrict__ k_base, int T, int S, int row0, int k, int32_t* __restrict__ idx,
+                  const PagedRows pg)
 {
     __shared__ SelectSmem<THREADS> sm;
     extern __shared__ int pre[];
     const int r = blockIdx.x, t = row0 + r;
     long long base;
-    const int n = row_candidates(pos, k_base, t, T, S, &base);
+    const int* bt;
+    const int n = row_keys(pg, pos, k_base, t, T, S, &base, &bt);
     const int nchunks = row_chunks(n);
     if (nchunks < 2) return;
     // chunk counts loaded in parallel, then their prefix
@@ -510,7 +534,7 @@ merge_topk_kernel(const uint2* __restrict__ cand, long long cand_ld, const int* 
         for (int e = threadIdx.x; e < H_I * d_I; e += THREADS) qf[e] = e4m3x2_to_float2((uint16_t)qrow[e]).x;
         for (int j = threadIdx.x; j < H_I; j += THREADS) wf[j] = w[(size_t)t * H_I + j];
         __syncthreads();
-        block_topk<THREADS>(RecomputedRow{qf, wf, k_idx + (size_t)base * d_I, H_I, d_I}, n, k,
+        block_topk<THREADS>(RecomputedRow{qf, wf, k_idx, pg, bt, base, H_I, d_I}, n, k,
                             idx + (size_t)t * k, sm);
         return;
     }

@@ -208,6 +208,35 @@ def varlen_prefill_inputs(name: str = "prefill4k", device="cpu", seed: int = 0, 
                      1.0 / math.sqrt(cfg["d_qk"]), cfg["d_v"], meta=meta)
 
 
+def page_caches(x: DSAInputs, page_size: int, seed: int = 0, spare_pages: int = 3):
+    """Scatter the per-sequence caches of decode/packed inputs x (rows
+    [k_base, k_base + pos + 1) per query row, one row per sequence) into a
+    shuffled pool of pages. Returns (k_pages, kv_pages, block_table [n_seqs,
+    max_pages], seq [T]); unused block-table entries are -1."""
+    base = x.bases().cpu().long().tolist()
+    n = (x.positions().cpu().long() + 1).tolist()
+    pages = [(c + page_size - 1) // page_size for c in n]
+    total = sum(pages) + spare_pages
+    g = _gen("cpu", tensor_seed(seed, x.config, f"pages{page_size}"))
+    perm = torch.randperm(total, generator=g).tolist()
+    dev = x.k_idx.device
+    k_pages = torch.zeros((total * page_size, x.k_idx.shape[1]), dtype=x.k_idx.dtype, device=dev)
+    kv_pages = torch.zeros((total * page_size, x.kv.shape[1]), dtype=x.kv.dtype, device=dev)
+    max_pages = max(pages)
+    table = torch.full((len(n), max_pages), -1, dtype=torch.int32)
+    nxt = 0
+    for b, (b0, c, npg) in enumerate(zip(base, n, pages)):
+        for j in range(npg):
+            pid = perm[nxt]
+            nxt += 1
+            table[b, j] = pid
+            lo, hi = j * page_size, min(c, (j + 1) * page_size)
+            k_pages[pid * page_size: pid * page_size + hi - lo] = x.k_idx[b0 + lo: b0 + hi]
+            kv_pages[pid * page_size: pid * page_size + hi - lo] = x.kv[b0 + lo: b0 + hi]
+    seq = torch.arange(len(n), dtype=torch.int32, device=dev)
+    return k_pages, kv_pages, table.to(dev), seq
+
+
 def decode_inputs(name: str = "decode", device="cpu", seed: int = 0, B: int = None,
                   ctx: list = None, overrides: dict = None) -> DSAInputs:
     """B sequences with one query each, keys packed per sequence in one cache.

@@ -143,3 +143,20 @@ def test_varlen_rejects_bad_offsets(lib):
     assert f(FAKE, FAKE, FAKE, P(cq), P(fewer_keys), 2, 8, 128, 2, FAKE, FAKE, ws, None) == -1
     assert b"sequence 1" in lib.dsa_last_error()
     assert f(FAKE, FAKE, FAKE, P(cq), P(good), 0, 8, 128, 2, FAKE, FAKE, ws, None) == -1
+
+
+def test_paged_rejects_bad_arguments(lib):
+    f = lib.dsa_indexer_topk_paged
+    ws = ctypes.c_size_t(1 << 20)
+    # page size not a multiple of 64
+    assert f(FAKE, FAKE, FAKE, 4, 48, FAKE, 1, 2, FAKE, FAKE, 1, 8, 128, 2, FAKE, FAKE, ws, None) == -2
+    # NULL block table
+    assert f(FAKE, FAKE, FAKE, 4, 64, None, 1, 2, FAKE, FAKE, 1, 8, 128, 2, FAKE, FAKE, ws, None) == -1
+    # d_I other than 128
+    assert f(FAKE, FAKE, FAKE, 4, 64, FAKE, 1, 2, FAKE, FAKE, 1, 8, 64, 2, FAKE, FAKE, ws, None) == -2
+    g = lib.dsa_sparse_mla_attn_paged
+    sc = ctypes.c_float(0.1)
+    assert g(FAKE, FAKE, 4, 64, FAKE, 1, 2, FAKE, FAKE, FAKE, 1, 4, 80, 64, 32, sc, FAKE, FAKE,
+             None) == -2   # tensor-core shapes only
+    assert g(FAKE, FAKE, 0, 64, FAKE, 1, 2, FAKE, FAKE, FAKE, 1, 128, 576, 512, 32, sc, FAKE, FAKE,
+             None) == -1
