@@ -50,6 +50,8 @@ def parse():
     ap.add_argument("--varlen", default=None,
                     help="comma-separated sequence lengths: time a packed batch of causal prefills "
                          "(varlen indexer + attention) instead of the default step")
+    ap.add_argument("--decode-page-size", type=int, default=None,
+                    help="run the decode step over paged caches (block table, pages of this size)")
     ap.add_argument("--rows", type=int, default=None,
                     help="prefill only the last ROWS tokens of the sequence (long rows, small "
                          "footprint: profiling)")
@@ -193,6 +195,8 @@ def workload_config(args, xp, world):
     dc = synth.CONFIGS[args.decode]
     decode = (f"{dc['B']} seqs, ctx U[{dc['ctx_lo']},{dc['ctx_hi']}]" if dc["kind"] == "decode"
               else f"{dc['L']} rows")
+    if getattr(args, "decode_page_size", None):
+        decode += f", paged caches of {args.decode_page_size}-row pages"
     rows = f"L={xp.T}" if xp.T == xp.S else f"last {xp.T} of L={xp.S}"
     return {"workload": f"{args.prefill} causal prefill ({rows}, H_I={H_I}, d_I={d_I}, k={xp.k}, "
                         f"Hq={Hq}, d_qk={d_qk}, d_v={xp.d_v}) + {args.decode} step ({decode})",
@@ -214,16 +218,27 @@ class Batch:
         self.ws = dsa.alloc_workspace(self.T, self.S, self.H_I, self.d_I, x.k, self.Hq,
                                       self.d_qk, x.d_v, dev)
         self.work = algorithmic_work(x)
+        self.paged = None   # (k_pages, kv_pages, block_table, seq, page_size) for a paged cache
 
 
 def run_indexer(dsa, b, stream):
     x = b.x
+    if b.paged is not None:
+        kp, vp, bt, seq, ps = b.paged
+        dsa.indexer_topk_paged(x.q_idx, x.w, kp, ps, bt, seq, x.pos, x.k, idx=b.idx, workspace=b.ws,
+                               stream=stream)
+        return
     dsa.indexer_topk(x.q_idx, x.w, x.k_idx, x.k, pos=x.pos, k_base=x.k_base, idx=b.idx,
                      workspace=b.ws, stream=stream)
 
 
 def run_attn(dsa, b, stream):
     x = b.x
+    if b.paged is not None:
+        kp, vp, bt, seq, ps = b.paged
+        dsa.sparse_mla_attn_paged(x.q, vp, ps, bt, seq, x.pos, b.idx, x.scale, x.d_v, out=b.out,
+                                  lse=b.lse, stream=stream)
+        return
     dsa.sparse_mla_attn(x.q, x.kv, b.idx, x.scale, x.d_v, pos=x.pos, k_base=x.k_base, out=b.out,
                         lse=b.lse, workspace=b.ws, stream=stream)
 
@@ -335,6 +350,12 @@ def bench_ours(args, world, rank, local):
     xp = synth.make_inputs(args.prefill, device=dev, seed=args.seed + rank, **prefill_kw(args))
     xd = synth.make_inputs(args.decode, device=dev, seed=args.seed + rank)
     bp, bd = Batch(xp, dsa), Batch(xd, dsa)
+    if args.decode_page_size:
+        ps = args.decode_page_size
+        kp, vp, bt, seq = synth.page_caches(xd, ps, seed=args.seed)
+        bd.paged = (kp, vp, bt, seq, ps)
+        bd.ws = dsa.alloc_workspace(xd.T, bt.shape[1] * ps, bd.H_I, bd.d_I, xd.k, bd.Hq, bd.d_qk, xd.d_v,
+                                    dev)
     stream = torch.cuda.current_stream()
 
     def step(ev=None):
