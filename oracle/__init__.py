@@ -55,6 +55,8 @@ def _load():
                                                     P, P]
             lib.oracle_dense_attn_row.argtypes = [P, P, i64, i64, i32, i32, i32, dbl, P, P]
             lib.oracle_lse_merge.argtypes = [P, P, i32, i32, i32, P, P]
+            lib.oracle_sparse_attn_bwd_rows.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, dbl,
+                                                        P, P, P]
             _lib = lib
     return _lib
 
@@ -174,6 +176,26 @@ def sparse_attn(q, kv, idx, pos, k_base, scale: float, d_v: int, rows=None, idx_
                                     out.ctypes.data_as(ctypes.c_void_p),
                                     lse.ctypes.data_as(ctypes.c_void_p))
     return out, lse
+
+
+def sparse_attn_bwd(q, kv, idx, pos, k_base, scale: float, d_v: int, dout):
+    """Gradients of sum(dout * out) of the sparse attention of every row of q
+    (bf16 [T, Hq, d_qk]) over its idx entries: (dq fp64 [T, Hq, d_qk],
+    dkv fp64 [S, d_qk]); dout bf16 [T, Hq, d_v]. pos / k_base int32 [T]."""
+    q_r, qp = _c(_u16(q), np.uint16)
+    kvu, kvp = _c(_u16(kv), np.uint16)
+    i_r, ip = _c(_np(idx, np.int32), np.int32)
+    p_r, pp = _c(_np(pos, np.int32), np.int32)
+    b_r, bp = _c(_np(k_base, np.int32), np.int32)
+    g_r, gp = _c(_u16(dout), np.uint16)
+    R, Hq, d_qk = q_r.shape
+    k = i_r.shape[1]
+    dq = np.zeros((R, Hq, d_qk), np.float64)
+    dkv = np.zeros((kvu.shape[0], d_qk), np.float64)
+    _load().oracle_sparse_attn_bwd_rows(qp, kvp, ip, pp, bp, R, k, Hq, d_qk, int(d_v), float(scale), gp,
+                                        dq.ctypes.data_as(ctypes.c_void_p),
+                                        dkv.ctypes.data_as(ctypes.c_void_p))
+    return dq, dkv
 
 
 def dense_attn_row(q_row, kv, pos: int, k_base: int, scale: float, d_v: int):

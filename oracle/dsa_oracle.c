@@ -346,3 +346,84 @@ void oracle_lse_merge(const double* o_parts, const double* lse_parts, int P, int
         lse[h] = total;
     }
 }
+
+/* Backward of the sparse MQA attention: the sparse training stage trains the
+ * main model with the LM loss through the selected entries only ("Paper
+ * Breakdown: DeepSeek-V3.2", "Continued Pre-Training (2.1.1)" table, row
+ * "Sparse Training"). The gradient is that of u_t = Attn(h_t, {c_s}) of the
+ * forward above, by the chain rule through softmax.
+ * For query row t with selected set sel and each head h (z_s = scale q_h.c_s,
+ * p = softmax(z) over sel, o_h = sum_s p_s c_s[0:d_v]), given dout_h:
+ *   dp_s = dout_h . c_s[0:d_v]
+ *   D    = sum_s p_s dp_s                       (= dout_h . o_h)
+ *   dz_s = p_s (dp_s - D)
+ *   dq_h = scale sum_s dz_s c_s                 (all d_qk columns)
+ *   dc_s += scale dz_s q_h  (all d_qk columns)  +  p_s dout_h  (first d_v)
+ * dkv accumulates over rows and heads (a scatter-add over idx); the caller
+ * zeroes it. Rows run one after another so the sums are deterministic. */
+void oracle_sparse_attn_bwd_rows(const uint16_t* q_rows, const uint16_t* kv, const int32_t* idx_rows,
+                                 const int32_t* pos_rows, const int32_t* base_rows, int R, int k,
+                                 int Hq, int d_qk, int d_v, double scale, const uint16_t* dout_rows,
+                                 double* dq, double* dkv)
+{
+    int32_t* sel = (int32_t*)malloc(sizeof(int32_t) * (size_t)(k > 0 ? k : 1));
+    double* z = (double*)malloc(sizeof(double) * (size_t)(k > 0 ? k : 1));
+    double* dp = (double*)malloc(sizeof(double) * (size_t)(k > 0 ? k : 1));
+    double* qh = (double*)malloc(sizeof(double) * (size_t)d_qk);
+    double* gh = (double*)malloc(sizeof(double) * (size_t)d_v);
+    for (int r = 0; r < R; ++r) {
+        const int32_t* idx_row = idx_rows + (size_t)r * k;
+        const int64_t pos = pos_rows[r], k_base = base_rows[r];
+        int n = 0;
+        for (int i = 0; i < k; ++i)
+            if (idx_row[i] >= 0 && idx_row[i] <= pos)
+                sel[n++] = idx_row[i];
+        for (int h = 0; h < Hq; ++h) {
+            double* dqh = dq + ((size_t)r * Hq + h) * d_qk;
+            for (int d = 0; d < d_qk; ++d)
+                dqh[d] = 0.0;
+            if (n == 0)
+                continue;
+            for (int d = 0; d < d_qk; ++d)
+                qh[d] = bf16_decode(q_rows[((size_t)r * Hq + h) * d_qk + d]);
+            for (int c = 0; c < d_v; ++c)
+                gh[c] = bf16_decode(dout_rows[((size_t)r * Hq + h) * d_v + c]);
+            double m = -INFINITY;
+            for (int i = 0; i < n; ++i) {
+                const uint16_t* c_s = kv + (size_t)(k_base + sel[i]) * d_qk;
+                double dot = 0.0, dg = 0.0;
+                for (int d = 0; d < d_qk; ++d)
+                    dot += qh[d] * bf16_decode(c_s[d]);
+                for (int c = 0; c < d_v; ++c)
+                    dg += gh[c] * bf16_decode(c_s[c]);
+                z[i] = scale * dot;
+                dp[i] = dg;
+                if (z[i] > m)
+                    m = z[i];
+            }
+            double l = 0.0;
+            for (int i = 0; i < n; ++i)
+                l += exp(z[i] - m);
+            double D = 0.0;
+            for (int i = 0; i < n; ++i)
+                D += exp(z[i] - m) / l * dp[i];
+            for (int i = 0; i < n; ++i) {
+                const double p = exp(z[i] - m) / l;
+                const double dz = p * (dp[i] - D);
+                const uint16_t* c_s = kv + (size_t)(k_base + sel[i]) * d_qk;
+                double* dc = dkv + (size_t)(k_base + sel[i]) * d_qk;
+                for (int d = 0; d < d_qk; ++d) {
+                    dqh[d] += scale * dz * bf16_decode(c_s[d]);
+                    dc[d] += scale * dz * qh[d];
+                }
+                for (int c = 0; c < d_v; ++c)
+                    dc[c] += p * gh[c];
+            }
+        }
+    }
+    free(gh);
+    free(qh);
+    free(dp);
+    free(z);
+    free(sel);
+}
