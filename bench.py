@@ -55,6 +55,9 @@ def parse():
     ap.add_argument("--rows", type=int, default=None,
                     help="prefill only the last ROWS tokens of the sequence (long rows, small "
                          "footprint: profiling)")
+    ap.add_argument("--bwd", nargs="?", const="prefill32k", default=None,
+                    help="time the sparse attention backward on this prefill workload "
+                         "(default prefill32k) instead of the default step")
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -613,6 +616,89 @@ def bench_varlen(args, world, rank, local):
     }
 
 
+def bench_bwd(args, world, rank, local):
+    """Sparse attention backward: dq and dkv of one causal prefill (all rows, k
+    selected latent rows each) from the forward's out / lse and a seeded dout.
+    The selection is the GPU indexer's Top-k (real overlap between rows, so
+    the dkv scatter sees realistic contention); it and the forward run once,
+    untimed. A step is zeroing dkv plus the backward call."""
+    import sparse_attention_20_b200 as dsa
+    from sparse_attention_20_b200 import build as dsa_build
+    if rank == 0:
+        dsa_build.build()
+    barrier(world)
+    dsa.load_library()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    x = synth.prefill_inputs(args.bwd, device=dev, seed=args.seed + rank, L=args.seq_len)
+    Hq, d_qk, d_v = x.q.shape[1], x.q.shape[2], x.d_v
+    idx, out, lse = dsa.forward(x.q_idx, x.w, x.k_idx, x.q, x.kv, x.k, x.scale, d_v)
+    dout = synth.grad_out(x, args.seed + rank)
+    dq = torch.empty((x.T, Hq, d_qk), dtype=torch.float32, device=dev)
+    dkv = torch.empty((x.S, d_qk), dtype=torch.float32, device=dev)
+    lib = dsa.load_library()
+    ws = torch.empty(int(lib.dsa_sparse_mla_attn_bwd_workspace_size(x.T, Hq, x.k)), dtype=torch.uint8,
+                     device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        dkv.zero_()
+        dsa.sparse_mla_attn_bwd(x.q, x.kv, idx, out, lse, dout, x.scale, dq=dq, dkv=dkv, workspace=ws,
+                                stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert dsa.device_status() == 0, dsa.last_error()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    n0 = dsa.launch_count()
+    start.record(stream)
+    for _ in range(args.steps):
+        step()
+    end.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    launches = dsa.launch_count() - n0
+    clk = clocks.stop()
+    ms_step = max_over_ranks(world, start.elapsed_time(end)) / args.steps
+    assert dsa.device_status() == 0, dsa.last_error()
+    # bf16 MMA flops per (row, valid slot, head): z (d_qk), dp (d_v), dq (d_qk), dkv (d_qk + d_v)
+    sel = torch.clamp(x.positions().cpu().long() + 1, max=x.k)
+    flops = float(sel.sum().item()) * Hq * 2 * (3 * d_qk + 2 * d_v)
+    peaks = measured_peaks()
+    tf = flops / (ms_step * 1e-3) / 1e12
+    res = {
+        "metric": "sparse MLA attention backward tokens/s (dq + dkv)",
+        "value": job_throughput(world, x.T, ms_step), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{args.bwd} causal prefill backward, L={x.T}, k={x.k}, Hq={Hq}, "
+                               f"d_qk={d_qk}, d_v={d_v}; inputs larger than L2, no flush",
+                   "global_batch": world, "seq_len": x.T, "parallelism": f"replicas{world}"},
+        "roofline": {"bound": "tensor", "kernel": "attention backward (dkv + dq kernels, one call)",
+                     "achieved": tf, "peak": peaks["bf16_sustained"], "unit": "TFLOP/s",
+                     "frac": tf / peaks["bf16_sustained"], "traffic": None,
+                     "peak_source": f"{peaks['source']} bf16 sustained"},
+        "gpu_launches": launches, "clocks": clk,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        import oracle
+        g = torch.Generator().manual_seed(args.seed)
+        rows = sorted(torch.randperm(x.T, generator=g)[:8].tolist())
+        r = torch.tensor(rows, device=dev)
+        t0 = time.perf_counter()
+        oracle.sparse_attn_bwd(x.q[r].cpu(), x.kv.cpu(), idx[r].cpu(), x.positions()[r].cpu(),
+                               torch.zeros(len(rows), dtype=torch.int32), x.scale, d_v, dout[r].cpu())
+        dt = time.perf_counter() - t0
+        res["cpu_baseline"] = {"value": len(rows) / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                               "sample": f"{len(rows)} uniformly drawn query rows of the {args.bwd} "
+                                         f"backward (fp64, one thread); {dt:.1f} s"}
+    return res
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -622,7 +708,8 @@ def main():
             print(json.dumps(bench_reference(args, world, 0)), flush=True)
         return
     world, rank, local = dist_setup(args)
-    res = (bench_varlen if args.varlen else bench_ours)(args, world, rank, local)
+    mode = bench_bwd if args.bwd else bench_varlen if args.varlen else bench_ours
+    res = mode(args, world, rank, local)
     if rank == 0:
         print(json.dumps(res), flush=True)
     if world > 1:

@@ -164,6 +164,39 @@ int dsa_sparse_mla_attn(const void* q, const void* kv, const int32_t* idx, const
                         void* stream);
 
 /*
+ * Backward of dsa_sparse_mla_attn: the gradients through the selected latent
+ * rows only, as the sparse training stage trains the main model ("Paper
+ * Breakdown: DeepSeek-V3.2", table "Continued Pre-Training (2.1.1)", row
+ * "Sparse Training"). With p_s = exp(scale q_h.c_s - lse_h) over row t's
+ * valid entries, dp_s = dout_h.c_s[0:d_v] and D_h = dout_h.out_h:
+ *   dq[t,h]        = scale sum_s p_s (dp_s - D_h) c_s
+ *   dkv[base + s] += scale sum_h p_s (dp_s - D_h) q_h + sum_h p_s dout_h
+ *                    (the second term on the first d_v columns only)
+ * Inputs as dsa_sparse_mla_attn, plus the forward's results for the same
+ * idx:
+ *   out    bf16 [T, Hq, d_v]   forward output (gives D_h)
+ *   lse    fp32 [T, Hq]        forward log-sum-exp
+ *   dout   bf16 [T, Hq, d_v]   gradient of the loss with respect to out
+ * Outputs (device memory, caller-owned):
+ *   dq     fp32 [T, Hq, d_qk]  written in full
+ *   dkv    fp32 [S, d_qk]      ACCUMULATED into (atomic adds, so the order of
+ *                              the adds and the last bits vary run to run);
+ *                              zero it for a fresh gradient
+ * workspace: at least one row of scratch (dsa_sparse_mla_attn_bwd_workspace_size
+ * with T = 1); more lets the call take more rows per pass (up to 8192 per
+ * pass, DSA_ERR_WORKSPACE below one row). Rows are processed in passes of
+ * that many rows on `stream`; the workspace holds the bf16 scale*dz of one
+ * pass between its two kernels.
+ * Supported: Hq <= 128, d_qk % 16 == 0, d_qk <= 576, d_v % 16 == 0,
+ * d_v <= d_qk, 1 <= k <= 4096 (DSA_ERR_UNSUPPORTED otherwise).
+ */
+size_t dsa_sparse_mla_attn_bwd_workspace_size(int T, int Hq, int k);
+int dsa_sparse_mla_attn_bwd(const void* q, const void* kv, const int32_t* idx, const int32_t* pos,
+                            const int32_t* k_base, const void* out, const float* lse, const void* dout,
+                            int T, int S, int Hq, int d_qk, int d_v, int k, float scale, float* dq,
+                            float* dkv, void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * The whole hot path: dsa_indexer_topk followed by dsa_sparse_mla_attn on the
  * same stream. `idx` is an output the caller keeps (it is also the input of
  * the attention step). Argument meanings and limits as above.

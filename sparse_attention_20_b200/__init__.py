@@ -32,7 +32,8 @@ STATUS_NAMES = {0: "DSA_OK", -1: "DSA_ERR_ARG", -2: "DSA_ERR_UNSUPPORTED", -3: "
 EXPORTS = ("dsa_workspace_size", "dsa_indexer_topk", "dsa_sparse_mla_attn", "dsa_forward",
            "dsa_device_status", "dsa_last_error", "dsa_abi_version", "dsa_launch_count",
            "dsa_indexer_topk_noalloc", "dsa_selftest_bounded_wait", "dsa_indexer_topk_varlen",
-           "dsa_indexer_topk_paged", "dsa_sparse_mla_attn_paged")
+           "dsa_indexer_topk_paged", "dsa_sparse_mla_attn_paged", "dsa_sparse_mla_attn_bwd",
+           "dsa_sparse_mla_attn_bwd_workspace_size")
 
 
 class DSAError(RuntimeError):
@@ -75,6 +76,11 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.dsa_indexer_topk_paged.restype = I
         lib.dsa_sparse_mla_attn_paged.argtypes = [P, P, I, I, P, I, I, P, P, P, I, I, I, I, I, F, P, P, P]
         lib.dsa_sparse_mla_attn_paged.restype = I
+        lib.dsa_sparse_mla_attn_bwd_workspace_size.argtypes = [I, I, I]
+        lib.dsa_sparse_mla_attn_bwd_workspace_size.restype = Z
+        lib.dsa_sparse_mla_attn_bwd.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, P, P, P, Z,
+                                                P]
+        lib.dsa_sparse_mla_attn_bwd.restype = I
         lib.dsa_selftest_bounded_wait.argtypes = [I, P]
         lib.dsa_selftest_bounded_wait.restype = I
         _lib = lib
@@ -262,6 +268,35 @@ def sparse_mla_attn(q, kv, idx, scale: float, d_v: int, pos=None, k_base=None, o
                                    d_qk, d_v, k, float(scale), _ptr(out), _ptr(lse),
                                    _ptr(workspace), workspace.numel(), _stream(stream)))
     return out, lse
+
+
+def sparse_mla_attn_bwd(q, kv, idx, out, lse, dout, scale: float, pos=None, k_base=None, dq=None,
+                        dkv=None, workspace=None, stream=None):
+    """(dq fp32 [T, Hq, d_qk], dkv fp32 [S, d_qk]) of sparse MQA attention over idx.
+
+    out / lse are the forward's results for the same idx; dout is bf16
+    [T, Hq, d_v]. dkv is accumulated into (a new zeroed tensor when None)."""
+    q, kv = _dev(q, "q"), _dev(kv, "kv")
+    out, dout, lse = _dev(out, "out"), _dev(dout, "dout"), _dev(lse, "lse")
+    if any(t.dtype != torch.bfloat16 for t in (q, kv, out, dout)):
+        raise TypeError("q, kv, out and dout must be bfloat16")
+    idx = _i32(idx, "idx")
+    T, Hq, d_qk = q.shape
+    S, d_v, k = kv.shape[0], out.shape[2], idx.shape[1]
+    pos, k_base = _i32(pos, "pos"), _i32(k_base, "k_base")
+    if dq is None:
+        dq = torch.empty((T, Hq, d_qk), dtype=torch.float32, device=q.device)
+    if dkv is None:
+        dkv = torch.zeros((S, d_qk), dtype=torch.float32, device=q.device)
+    lib = load_library()
+    if workspace is None:
+        workspace = torch.empty(int(lib.dsa_sparse_mla_attn_bwd_workspace_size(T, Hq, k)),
+                                dtype=torch.uint8, device=q.device)
+    _check(lib.dsa_sparse_mla_attn_bwd(_ptr(q), _ptr(kv), _ptr(idx), _ptr(pos), _ptr(k_base), _ptr(out),
+                                       _ptr(lse), _ptr(dout), T, S, Hq, d_qk, d_v, k, float(scale),
+                                       _ptr(dq), _ptr(dkv), _ptr(workspace), workspace.numel(),
+                                       _stream(stream)))
+    return dq, dkv
 
 
 def forward(q_idx, w, k_idx, q, kv, k: int, scale: float, d_v: int, pos=None, k_base=None,

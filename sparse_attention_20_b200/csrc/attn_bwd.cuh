@@ -1,0 +1,396 @@
+// Backward of the sparse MQA attention: the gradients that train the main
+// model through the selected latent rows only (the sparse training stage of
+// "Paper Breakdown: DeepSeek-V3.2", table "Continued Pre-Training (2.1.1)").
+//
+// Forward, per query row t and head h over the selected set (MQA: one latent
+// row c_s serves every head): z_s = scale q_h.c_s, p = softmax(z),
+// o_h = sum_s p_s c_s[0:d_v], lse_h = log sum_s exp(z_s). Given dout:
+//   dp_s = dout_h . c_s[0:d_v]          D_h  = dout_h . o_h
+//   dz_s = p_s (dp_s - D_h)             p_s  = exp(z_s - lse_h)
+//   dq_h = scale sum_s dz_s c_s
+//   dkv[row of s] += scale sum_h dz_{h,s} q_h + sum_h p_{h,s} dout_h[0:d_v]
+//
+// Two kernels, both on warp-level bf16 MMAs (m16n8k16, fp32 accumulate):
+//  - attn_bwd_dkv_kernel, one CTA per (row, 64 selected slots): recomputes z
+//    and dp for all heads against the 64 gathered rows, forms p and
+//    g = scale dz (bf16), adds g^T q + p^T dout into dkv (fp32 atomics, one
+//    add per (slot, column)) and stores g for the next kernel;
+//  - attn_bwd_dq_kernel, one CTA per (row, 64 columns): dq = g . C over the
+//    row's selected rows, no atomics.
+// p and g are rounded to bf16 before they enter an MMA, as the forward rounds
+// its probabilities; D comes from the forward's bf16 output.
+#pragma once
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace dsa {
+namespace bwd {
+
+using sm100::smem_u32;
+
+constexpr int kSlots = 64;      // selected slots per CTA of the dkv kernel
+constexpr int kCols = 64;       // column slice of the dC and dq tiles
+constexpr int kThreads = 256;   // 8 warps
+constexpr int kWarps = kThreads / 32;
+constexpr int kMaxHeads = 128;  // 8 warps x 16 heads
+constexpr int kMaxDqk = 576;
+constexpr int kPS = kCols + 8;  // row stride (bf16) of the [head][64] tiles: 144 B, conflict-free ldmatrix
+
+__host__ __device__ inline int heads_pad(int Hq) { return (Hq + 15) / 16 * 16; }
+__host__ __device__ inline int slots_pad(int k) { return (k + kSlots - 1) / kSlots * kSlots; }
+
+// shared memory of the dkv kernel
+__host__ __device__ inline size_t dkv_smem(int Hq, int d_qk)
+{
+    const size_t hp = heads_pad(Hq);
+    return sizeof(__nv_bfloat16) * ((size_t)kSlots * (d_qk + 8) + 4 * hp * kPS) +
+           sizeof(long long) * kSlots + 2 * sizeof(float) * hp;
+}
+
+__host__ __device__ inline size_t dq_smem(int Hq)
+{
+    return sizeof(__nv_bfloat16) * ((size_t)kSlots * kPS + (size_t)heads_pad(Hq) * kPS) +
+           sizeof(long long) * kSlots;
+}
+
+// ------------------------------------------------------ warp-level helpers
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4])
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4])
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
+// d += a (16x16, row) * b (16x8, col); bf16 inputs, fp32 accumulators
+__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Lane addresses of the four 8x8 matrices of one ldmatrix.x4 (lane l feeds row l % 8 of
+// matrix l / 8), for the three operand forms used here. Shared tiles are row-major with
+// a row stride of `ld` bf16.
+// A fragment (16 x 16 at r0, c0) of a row-major [m][k] tile.
+__device__ __forceinline__ uint32_t a_addr(uint32_t base, int ld, int r0, int c0, int lane)
+{
+    return base + 2u * (uint32_t)((r0 + (lane & 15)) * ld + c0 + (lane >> 4) * 8);
+}
+// A fragment of the transpose of a [k][m] tile (m0 = first m, k0 = first k); use with .trans.
+__device__ __forceinline__ uint32_t at_addr(uint32_t base, int ld, int m0, int k0, int lane)
+{
+    return base + 2u * (uint32_t)((k0 + (lane & 7) + (lane >> 4) * 8) * ld + m0 + ((lane >> 3) & 1) * 8);
+}
+// B fragments of two n8 tiles (n0, n0 + 8) from a [n][k] tile (non-trans).
+__device__ __forceinline__ uint32_t bn_addr(uint32_t base, int ld, int n0, int k0, int lane)
+{
+    return base + 2u * (uint32_t)((n0 + (lane & 7) + (lane >> 4) * 8) * ld + k0 + ((lane >> 3) & 1) * 8);
+}
+// B fragments of two n8 tiles (n0, n0 + 8) from a [k][n] tile; use with .trans.
+__device__ __forceinline__ uint32_t bk_addr(uint32_t base, int ld, int n0, int k0, int lane)
+{
+    return base + 2u * (uint32_t)((k0 + (lane & 7) + ((lane >> 3) & 1) * 8) * ld + n0 + (lane >> 4) * 8);
+}
+
+__device__ __forceinline__ uint32_t ld_pair(const __nv_bfloat16* p) { return __ldg(reinterpret_cast<const uint32_t*>(p)); }
+
+// Cache row of slot i of row t (-1: not a candidate).
+__device__ __forceinline__ long long slot_row(const int* idx, int k, int t, int i, long long base, int n_cand)
+{
+    if (i >= k) return -1;
+    const int s = idx[(size_t)t * k + i];
+    return (s >= 0 && s < n_cand) ? base + s : -1;
+}
+
+// ------------------------------------------------------------- dkv kernel
+
+// grid: x = slot chunk (64 slots), y = query row within the batch [r0, r0 + gridDim.y).
+// g_ws: bf16 [rows][heads_pad(Hq)][slots_pad(k)], g = scale * dz for every slot.
+__global__ void __launch_bounds__(kThreads)
+attn_bwd_dkv_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kv,
+                    const int* __restrict__ idx, const int* __restrict__ pos, const int* __restrict__ k_base,
+                    const __nv_bfloat16* __restrict__ out, const float* __restrict__ lse,
+                    const __nv_bfloat16* __restrict__ dout, int r0, int T, int S, int Hq, int d_qk, int d_v,
+                    int k, float scale, float* __restrict__ dkv, __nv_bfloat16* __restrict__ g_ws)
+{
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    const int hp = heads_pad(Hq), ldc = d_qk + 8, kp = slots_pad(k);
+    __nv_bfloat16* cs = reinterpret_cast<__nv_bfloat16*>(smem_raw);   // [64][ldc] gathered rows
+    __nv_bfloat16* ps = cs + (size_t)kSlots * ldc;                    // [hp][kPS] p
+    __nv_bfloat16* gs = ps + (size_t)hp * kPS;                        // [hp][kPS] g = scale dz
+    __nv_bfloat16* qsl = gs + (size_t)hp * kPS;                       // [hp][kPS] q columns slice
+    __nv_bfloat16* osl = qsl + (size_t)hp * kPS;                      // [hp][kPS] dout columns slice
+    long long* rows = reinterpret_cast<long long*>(osl + (size_t)hp * kPS);  // [64]
+    float* Dh = reinterpret_cast<float*>(rows + kSlots);              // [hp]
+    float* lse2 = Dh + hp;                                            // [hp]
+
+    const int tl = blockIdx.y, t = r0 + tl, i0 = blockIdx.x * kSlots;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int gq = lane >> 2, tq = lane & 3;
+    constexpr float kLog2e = 1.4426950408889634f;
+    long long base;
+    const int n_cand = row_candidates(pos, k_base, t, T, S, &base);
+
+    if (threadIdx.x < kSlots) rows[threadIdx.x] = slot_row(idx, k, t, i0 + threadIdx.x, base, n_cand);
+    // D_h = dout_h . o_h and lse in base 2, one warp per head
+    for (int h = warp; h < hp; h += kWarps) {
+        float acc = 0.f;
+        if (h < Hq) {
+            const __nv_bfloat16* gr = dout + ((size_t)t * Hq + h) * d_v;
+            const __nv_bfloat16* orow = out + ((size_t)t * Hq + h) * d_v;
+            for (int c = 2 * lane; c < d_v; c += 64) {
+                const uint32_t a = ld_pair(gr + c), b = ld_pair(orow + c);
+                acc = fmaf(bf16_lo(a), bf16_lo(b), fmaf(bf16_hi(a), bf16_hi(b), acc));
+            }
+        }
+#pragma unroll
+        for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (lane == 0) {
+            Dh[h] = acc;
+            lse2[h] = h < Hq ? lse[(size_t)t * Hq + h] * kLog2e : 0.f;
+        }
+    }
+    __syncthreads();
+    // gather the 64 selected rows (zeros for non-candidates)
+    {
+        const int v8 = d_qk / 8;
+        for (int e = threadIdx.x; e < kSlots * v8; e += kThreads) {
+            const int j = e / v8, c8 = e - j * v8;
+            const long long r = rows[j];
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (r >= 0) v = __ldg(reinterpret_cast<const uint4*>(kv + (size_t)r * d_qk) + c8);
+            *reinterpret_cast<uint4*>(cs + (size_t)j * ldc + c8 * 8) = v;
+        }
+    }
+    __syncthreads();
+
+    const uint32_t cs_u = smem_u32(cs), ps_u = smem_u32(ps), gs_u = smem_u32(gs);
+    const uint32_t qsl_u = smem_u32(qsl), osl_u = smem_u32(osl);
+
+    // z and dp for 16 heads x 64 slots per warp; then p and g
+    for (int ht = warp; ht * 16 < hp; ht += kWarps) {
+        const int h0 = ht * 16;
+        float z[8][4], dp[8][4];
+#pragma unroll
+        for (int n = 0; n < 8; ++n)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) z[n][e] = dp[n][e] = 0.f;
+        const bool lo_ok = h0 + gq < Hq, hi_ok = h0 + gq + 8 < Hq;
+        const __nv_bfloat16* qlo = q + ((size_t)t * Hq + h0 + gq) * d_qk + 2 * tq;
+        const __nv_bfloat16* qhi = qlo + (size_t)8 * d_qk;
+        for (int k0 = 0; k0 < d_qk; k0 += 16) {
+            uint32_t a[4];
+            a[0] = lo_ok ? ld_pair(qlo + k0) : 0u;
+            a[1] = hi_ok ? ld_pair(qhi + k0) : 0u;
+            a[2] = lo_ok ? ld_pair(qlo + k0 + 8) : 0u;
+            a[3] = hi_ok ? ld_pair(qhi + k0 + 8) : 0u;
+#pragma unroll
+            for (int np = 0; np < 4; ++np) {
+                uint32_t b[4];
+                ldsm_x4(bn_addr(cs_u, ldc, np * 16, k0, lane), b);
+                mma_bf16(z[2 * np], a, b[0], b[1]);
+                mma_bf16(z[2 * np + 1], a, b[2], b[3]);
+            }
+        }
+        const __nv_bfloat16* glo = dout + ((size_t)t * Hq + h0 + gq) * d_v + 2 * tq;
+        const __nv_bfloat16* ghi = glo + (size_t)8 * d_v;
+        for (int k0 = 0; k0 < d_v; k0 += 16) {
+            uint32_t a[4];
+            a[0] = lo_ok ? ld_pair(glo + k0) : 0u;
+            a[1] = hi_ok ? ld_pair(ghi + k0) : 0u;
+            a[2] = lo_ok ? ld_pair(glo + k0 + 8) : 0u;
+            a[3] = hi_ok ? ld_pair(ghi + k0 + 8) : 0u;
+#pragma unroll
+            for (int np = 0; np < 4; ++np) {
+                uint32_t b[4];
+                ldsm_x4(bn_addr(cs_u, ldc, np * 16, k0, lane), b);
+                mma_bf16(dp[2 * np], a, b[0], b[1]);
+                mma_bf16(dp[2 * np + 1], a, b[2], b[3]);
+            }
+        }
+        const float zs = scale * kLog2e;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            const int hl = h0 + gq + 8 * half;
+            const bool hok = hl < Hq;
+            const float l2 = lse2[hl], D = Dh[hl];
+            __nv_bfloat16* gw = g_ws + ((size_t)tl * hp + hl) * kp + i0;
+#pragma unroll
+            for (int n = 0; n < 8; ++n) {
+                const int j = n * 8 + 2 * tq;
+                float pv[2], gv[2];
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const bool ok = hok && rows[j + e] >= 0;
+                    const float p = ok ? exp2f(fmaf(z[n][2 * half + e], zs, -l2)) : 0.f;
+                    pv[e] = p;
+                    gv[e] = ok ? scale * p * (dp[n][2 * half + e] - D) : 0.f;
+                }
+                const uint32_t pp = pack_bf16x2(pv[0], pv[1]), gg = pack_bf16x2(gv[0], gv[1]);
+                *reinterpret_cast<uint32_t*>(ps + (size_t)hl * kPS + j) = pp;
+                *reinterpret_cast<uint32_t*>(gs + (size_t)hl * kPS + j) = gg;
+                *reinterpret_cast<uint32_t*>(gw + j) = gg;
+            }
+        }
+    }
+    __syncthreads();
+
+    // dC (64 slots x d_qk) = g^T q + p^T dout, 64 columns at a time; warp w owns
+    // slots 16 (w % 4) .. + 16 and columns 32 (w / 4) .. + 32 of the slice.
+    const int mt = warp & 3, nh = warp >> 2;
+    for (int c0 = 0; c0 < d_qk; c0 += kCols) {
+        const int nc = min(kCols, d_qk - c0);   // multiple of 16
+        const bool with_v = c0 < d_v;
+        for (int e = threadIdx.x; e < hp * (kCols / 8); e += kThreads) {
+            const int h = e >> 3, c8 = (e & 7) * 8;
+            uint4 vq = make_uint4(0, 0, 0, 0), vg = make_uint4(0, 0, 0, 0);
+            if (h < Hq && c8 < nc) {
+                vq = __ldg(reinterpret_cast<const uint4*>(q + ((size_t)t * Hq + h) * d_qk + c0 + c8));
+                if (c0 + c8 < d_v)
+                    vg = __ldg(reinterpret_cast<const uint4*>(dout + ((size_t)t * Hq + h) * d_v + c0 + c8));
+            }
+            *reinterpret_cast<uint4*>(qsl + (size_t)h * kPS + c8) = vq;
+            *reinterpret_cast<uint4*>(osl + (size_t)h * kPS + c8) = vg;
+        }
+        __syncthreads();
+        if (nh * 32 < nc) {
+            float acc[4][4];
+#pragma unroll
+            for (int n = 0; n < 4; ++n)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) acc[n][e] = 0.f;
+            const int npairs = min(2, (nc - nh * 32) / 16);
+            for (int k0 = 0; k0 < hp; k0 += 16) {
+                uint32_t a[4];
+                ldsm_x4_t(at_addr(gs_u, kPS, mt * 16, k0, lane), a);
+#pragma unroll
+                for (int np = 0; np < 2; ++np) {
+                    if (np < npairs) {
+                        uint32_t b[4];
+                        ldsm_x4_t(bk_addr(qsl_u, kPS, nh * 32 + np * 16, k0, lane), b);
+                        mma_bf16(acc[2 * np], a, b[0], b[1]);
+                        mma_bf16(acc[2 * np + 1], a, b[2], b[3]);
+                    }
+                }
+                if (with_v) {
+                    ldsm_x4_t(at_addr(ps_u, kPS, mt * 16, k0, lane), a);
+#pragma unroll
+                    for (int np = 0; np < 2; ++np) {
+                        if (np < npairs) {
+                            uint32_t b[4];
+                            ldsm_x4_t(bk_addr(osl_u, kPS, nh * 32 + np * 16, k0, lane), b);
+                            mma_bf16(acc[2 * np], a, b[0], b[1]);
+                            mma_bf16(acc[2 * np + 1], a, b[2], b[3]);
+                        }
+                    }
+                }
+            }
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                const long long r = rows[mt * 16 + gq + 8 * half];
+                if (r < 0) continue;
+                float* dst = dkv + (size_t)r * d_qk + c0 + nh * 32 + 2 * tq;
+#pragma unroll
+                for (int n = 0; n < 4; ++n) {
+                    if (n < 2 * npairs) {
+                        atomicAdd(dst + n * 8, acc[n][2 * half]);
+                        atomicAdd(dst + n * 8 + 1, acc[n][2 * half + 1]);
+                    }
+                }
+            }
+        }
+        __syncthreads();
+    }
+}
+
+// -------------------------------------------------------------- dq kernel
+
+// grid: x = 64-column slice of d_qk, y = query row within the batch.
+// dq fp32 [T][Hq][d_qk] = sum over the row's slots of g (from g_ws) times the row.
+__global__ void __launch_bounds__(kThreads)
+attn_bwd_dq_kernel(const __nv_bfloat16* __restrict__ kv, const int* __restrict__ idx,
+                   const int* __restrict__ pos, const int* __restrict__ k_base,
+                   const __nv_bfloat16* __restrict__ g_ws, int r0, int T, int S, int Hq, int d_qk, int k,
+                   float* __restrict__ dq)
+{
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    const int hp = heads_pad(Hq), kp = slots_pad(k);
+    __nv_bfloat16* csl = reinterpret_cast<__nv_bfloat16*>(smem_raw);  // [64 slots][kPS] columns slice
+    __nv_bfloat16* gsm = csl + (size_t)kSlots * kPS;                   // [hp][kPS] g of 64 slots
+    long long* rows = reinterpret_cast<long long*>(gsm + (size_t)hp * kPS);
+
+    const int tl = blockIdx.y, t = r0 + tl, c0 = blockIdx.x * kCols;
+    const int nc = min(kCols, d_qk - c0);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int gq = lane >> 2, tq = lane & 3;
+    long long base;
+    const int n_cand = row_candidates(pos, k_base, t, T, S, &base);
+    const uint32_t csl_u = smem_u32(csl), gsm_u = smem_u32(gsm);
+    const int h0 = warp * 16;
+    const bool active = h0 < hp;
+    float acc[8][4];
+#pragma unroll
+    for (int n = 0; n < 8; ++n)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[n][e] = 0.f;
+
+    for (int i0 = 0; i0 < kp; i0 += kSlots) {
+        if (threadIdx.x < kSlots) rows[threadIdx.x] = slot_row(idx, k, t, i0 + threadIdx.x, base, n_cand);
+        __syncthreads();
+        for (int e = threadIdx.x; e < kSlots * (kCols / 8); e += kThreads) {
+            const int j = e >> 3, c8 = (e & 7) * 8;
+            const long long r = rows[j];
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (r >= 0 && c8 < nc) v = __ldg(reinterpret_cast<const uint4*>(kv + (size_t)r * d_qk + c0 + c8));
+            *reinterpret_cast<uint4*>(csl + (size_t)j * kPS + c8) = v;
+        }
+        for (int e = threadIdx.x; e < hp * (kSlots / 8); e += kThreads) {
+            const int h = e >> 3, j8 = (e & 7) * 8;
+            *reinterpret_cast<uint4*>(gsm + (size_t)h * kPS + j8) =
+                __ldg(reinterpret_cast<const uint4*>(g_ws + ((size_t)tl * hp + h) * kp + i0 + j8));
+        }
+        __syncthreads();
+        if (active) {
+#pragma unroll
+            for (int k0 = 0; k0 < kSlots; k0 += 16) {
+                uint32_t a[4];
+                ldsm_x4(a_addr(gsm_u, kPS, h0, k0, lane), a);
+#pragma unroll
+                for (int np = 0; np < 4; ++np) {
+                    if (np * 16 < nc) {
+                        uint32_t b[4];
+                        ldsm_x4_t(bk_addr(csl_u, kPS, np * 16, k0, lane), b);
+                        mma_bf16(acc[2 * np], a, b[0], b[1]);
+                        mma_bf16(acc[2 * np + 1], a, b[2], b[3]);
+                    }
+                }
+            }
+        }
+        __syncthreads();
+    }
+    if (!active) return;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+        const int h = h0 + gq + 8 * half;
+        if (h >= Hq) continue;
+        float* dst = dq + ((size_t)t * Hq + h) * d_qk + c0 + 2 * tq;
+#pragma unroll
+        for (int n = 0; n < 8; ++n)
+            if (n * 8 < nc)
+                *reinterpret_cast<float2*>(dst + n * 8) = make_float2(acc[n][2 * half], acc[n][2 * half + 1]);
+    }
+}
+
+}  // namespace bwd
+}  // namespace dsa

@@ -13,6 +13,7 @@
 #include <mutex>
 
 #include "dsa.h"
+#include "attn_bwd.cuh"
 #include "attn_simple.cuh"
 #include "attn_tc.cuh"
 #include "common.cuh"
@@ -550,6 +551,60 @@ int attn_tc(const __nv_bfloat16* q, const __nv_bfloat16* kv, const int32_t* idx,
     return DSA_OK;
 }
 
+// ---------------------------------------------------------- attention backward
+
+constexpr int kBwdRowsMax = 8192;   // query rows per pass of the backward (workspace size)
+
+size_t attn_bwd_row_bytes(int Hq, int k)
+{
+    return (size_t)dsa::bwd::heads_pad(Hq) * dsa::bwd::slots_pad(k) * sizeof(__nv_bfloat16);
+}
+
+int check_attn_bwd(const void* q, const void* kv, const int32_t* idx, const int32_t* pos,
+                   const int32_t* k_base, const void* out, const float* lse, const void* dout, int T,
+                   int S, int Hq, int d_qk, int d_v, int k, const float* dq, const float* dkv)
+{
+    if (int rc = check_attn(q, kv, idx, pos, k_base, T, S, Hq, d_qk, d_v, k, out, lse)) return rc;
+    if (!dout || !dq || !dkv) return fail(DSA_ERR_ARG, "NULL dout, dq or dkv");
+    if (!al16(dout) || !al16(dq) || !al16(dkv))
+        return fail(DSA_ERR_ARG, "dout, dq and dkv must be 16-byte aligned");
+    if (Hq > dsa::bwd::kMaxHeads)
+        return fail(DSA_ERR_UNSUPPORTED, "Hq=%d (backward supports 1..%d)", Hq, dsa::bwd::kMaxHeads);
+    if (d_qk % 16 || d_qk > dsa::bwd::kMaxDqk || d_v % 16)
+        return fail(DSA_ERR_UNSUPPORTED, "d_qk=%d, d_v=%d (backward: multiples of 16, d_qk <= %d)", d_qk,
+                    d_v, dsa::bwd::kMaxDqk);
+    return DSA_OK;
+}
+
+int attn_bwd(const __nv_bfloat16* q, const __nv_bfloat16* kv, const int32_t* idx, const int32_t* pos,
+             const int32_t* k_base, const __nv_bfloat16* out, const float* lse,
+             const __nv_bfloat16* dout, int T, int S, int Hq, int d_qk, int d_v, int k, float scale,
+             float* dq, float* dkv, void* workspace, size_t ws_bytes, cudaStream_t st)
+{
+    using namespace dsa::bwd;
+    const size_t row_bytes = attn_bwd_row_bytes(Hq, k);
+    const size_t fit = workspace && al16(workspace) ? ws_bytes / row_bytes : 0;
+    if (fit < 1)
+        return fail(DSA_ERR_WORKSPACE, "attention backward needs %zu workspace bytes per row (got %zu)",
+                    row_bytes, ws_bytes);
+    const int rows = (int)std::min<size_t>(std::min<size_t>(fit, (size_t)T), 65535);
+    const size_t s_dkv = dkv_smem(Hq, d_qk), s_dq = dq_smem(Hq);
+    cudaError_t e = cudaFuncSetAttribute(attn_bwd_dkv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)s_dkv);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(attn_bwd_dkv_kernel)");
+    __nv_bfloat16* g_ws = reinterpret_cast<__nv_bfloat16*>(workspace);
+    for (int r0 = 0; r0 < T; r0 += rows) {
+        const int n = std::min(rows, T - r0);
+        attn_bwd_dkv_kernel<<<dim3(slots_pad(k) / kSlots, n), kThreads, s_dkv, st>>>(
+            q, kv, idx, pos, k_base, out, lse, dout, r0, T, S, Hq, d_qk, d_v, k, scale, dkv, g_ws);
+        DSA_LAUNCH_CHECK("attn_bwd_dkv_kernel");
+        attn_bwd_dq_kernel<<<dim3(dsa::ceil_div(d_qk, kCols), n), kThreads, s_dq, st>>>(
+            kv, idx, pos, k_base, g_ws, r0, T, S, Hq, d_qk, k, dq);
+        DSA_LAUNCH_CHECK("attn_bwd_dq_kernel");
+    }
+    return DSA_OK;
+}
+
 }  // namespace
 
 // ===================================================================== C ABI
@@ -728,6 +783,26 @@ int dsa_sparse_mla_attn(const void* q, const void* kv, const int32_t* idx, const
                        reinterpret_cast<const __nv_bfloat16*>(kv), idx, pos, k_base, T, S, Hq,
                        d_qk, d_v, k, scale, reinterpret_cast<__nv_bfloat16*>(out), lse, workspace,
                        reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t dsa_sparse_mla_attn_bwd_workspace_size(int T, int Hq, int k)
+{
+    if (T <= 0 || Hq <= 0 || k <= 0) return 0;
+    return (size_t)std::min(T, kBwdRowsMax) * attn_bwd_row_bytes(Hq, k);
+}
+
+int dsa_sparse_mla_attn_bwd(const void* q, const void* kv, const int32_t* idx, const int32_t* pos,
+                            const int32_t* k_base, const void* out, const float* lse, const void* dout,
+                            int T, int S, int Hq, int d_qk, int d_v, int k, float scale, float* dq,
+                            float* dkv, void* workspace, size_t ws_bytes, void* stream)
+{
+    g_err[0] = 0;
+    if (int rc = check_attn_bwd(q, kv, idx, pos, k_base, out, lse, dout, T, S, Hq, d_qk, d_v, k, dq, dkv))
+        return rc;
+    using bf = __nv_bfloat16;
+    return attn_bwd(reinterpret_cast<const bf*>(q), reinterpret_cast<const bf*>(kv), idx, pos, k_base,
+                    reinterpret_cast<const bf*>(out), lse, reinterpret_cast<const bf*>(dout), T, S, Hq,
+                    d_qk, d_v, k, scale, dq, dkv, workspace, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int dsa_forward(const void* q_idx, const float* w, const void* k_idx, const void* q,

@@ -33,6 +33,7 @@ import zlib
 from dataclasses import dataclass, field
 from typing import Optional
 
+import numpy as np
 import torch
 
 E4M3_MAX = 448.0
@@ -287,3 +288,34 @@ def sample_rows(T: int, k: int, n: int, seed: int = 0) -> list:
         if len(out) >= max(n, len(fixed)):
             break
     return sorted(out)
+
+
+def selection(pos, k: int, seed: int = 0) -> torch.Tensor:
+    """A valid selection for every query row that depends on no score: int32
+    [T, k] (CPU) holding min(k, n_t) distinct s in [0, n_t) first and -1 after,
+    n_t = pos[t] + 1. Row t takes s_i = (a_t * i + b_t) mod n_t, i = 0, 1, ...,
+    with a_t drawn coprime to n_t (so the s_i are distinct) and b_t uniform."""
+    pos = np.asarray(pos.cpu() if hasattr(pos, "cpu") else pos, dtype=np.int64)
+    T = pos.shape[0]
+    out = np.full((T, k), -1, np.int32)
+    rng = np.random.default_rng(tensor_seed(seed, "selection", str(k)))
+    n = np.maximum(pos + 1, 0)
+    a = rng.integers(1, np.maximum(n, 1) + 1)
+    bad = np.gcd(a, np.maximum(n, 1)) != 1
+    while bad.any():
+        a[bad] = rng.integers(1, n[bad] + 1)
+        bad = np.gcd(a, np.maximum(n, 1)) != 1
+    b = rng.integers(0, np.maximum(n, 1))
+    i = np.arange(k, dtype=np.int64)
+    step = max(1, (1 << 24) // max(k, 1))
+    for r0 in range(0, T, step):
+        r1 = min(T, r0 + step)
+        nn = n[r0:r1, None]
+        s = (a[r0:r1, None] * i[None, :] + b[r0:r1, None]) % np.maximum(nn, 1)
+        out[r0:r1] = np.where(i[None, :] < nn, s, -1)
+    return torch.from_numpy(out)
+
+
+def grad_out(x: DSAInputs, seed: int = 0) -> torch.Tensor:
+    """dL/dout of the attention output: bf16 N(0, 1) [T, Hq, d_v] on x's device."""
+    return normal((x.T, x.q.shape[1], x.d_v), seed, x.config, "dout", x.q.device, dtype=torch.bfloat16)

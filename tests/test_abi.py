@@ -102,6 +102,27 @@ def test_attention_rejects_bad_arguments(lib):
              None) == -2
 
 
+def test_attention_backward_rejects_bad_arguments(lib):
+    f = lib.dsa_sparse_mla_attn_bwd
+    sc = ctypes.c_float(0.1)
+    ws = ctypes.c_size_t(1 << 20)
+
+    def call(Hq=128, d_qk=576, d_v=512, k=64, dout=FAKE, wsb=ws, wsp=FAKE):
+        return f(FAKE, FAKE, FAKE, None, None, FAKE, FAKE, dout, 4, 4, Hq, d_qk, d_v, k, sc, FAKE, FAKE,
+                 wsp, wsb, None)
+
+    assert call(dout=None) == -1
+    assert call(Hq=129) == -2            # more heads than the backward takes
+    assert call(d_qk=584, d_v=512) == -2  # d_qk above 576
+    assert call(d_qk=576, d_v=504) == -2  # d_v not a multiple of 16
+    assert call(wsb=ctypes.c_size_t(100)) == -5
+    assert call(wsp=None) == -5
+    # one row of scratch: heads padded to 16, slots to 64, bf16
+    assert lib.dsa_sparse_mla_attn_bwd_workspace_size(1, 4, 32) == 16 * 64 * 2
+    assert lib.dsa_sparse_mla_attn_bwd_workspace_size(100000, 128, 2048) == 8192 * 128 * 2048 * 2
+    assert lib.dsa_sparse_mla_attn_bwd_workspace_size(0, 128, 2048) == 0
+
+
 def test_binding_refuses_cpu_tensors():
     import torch
     x = torch.zeros((4, 8, 128), dtype=torch.uint8)

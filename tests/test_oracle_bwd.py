@@ -165,3 +165,13 @@ def test_finite_difference_pin_catches_a_dropped_term():
         bad[r] = scale * (p * (gf[r] @ C[:, :d_v].T)) @ C
     fd = _central_diff(qf, lambda: _loss(qf, kvf, gf, idx, pos, base, scale, d_v))
     assert not np.allclose(bad, fd, rtol=1e-7, atol=1e-8)
+
+
+def test_backward_column_sums_of_dkv():
+    """sum_s p_s = 1 and sum_s dz_s = 0 per row and head, so summed over the cache
+    rows dkv[:, :d_v] = sum over rows and heads of dout, and dkv[:, d_v:] sums to 0."""
+    q, kv, dout, idx, pos, base, scale, d_v = _case(9, R=4, Hq=3, d_qk=16, d_v=8, S=30, k=12)
+    dq, dkv = oracle.sparse_attn_bwd(q, kv, idx, pos, base, scale, d_v, dout)
+    col = dkv.sum(axis=0)
+    assert np.allclose(col[:d_v], _f64(dout).sum(axis=(0, 1)), rtol=1e-12, atol=1e-12)
+    assert np.allclose(col[d_v:], 0.0, atol=1e-12)
