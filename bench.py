@@ -629,7 +629,7 @@ def bench_bwd(args, world, rank, local):
     barrier(world)
     dsa.load_library()
     dev = torch.device("cuda", torch.cuda.current_device())
-    x = synth.prefill_inputs(args.bwd, device=dev, seed=args.seed + rank, L=args.seq_len)
+    x = synth.prefill_inputs(args.bwd, device=dev, seed=args.seed + rank, L=args.seq_len, T=args.rows)
     Hq, d_qk, d_v = x.q.shape[1], x.q.shape[2], x.d_v
     idx, out, lse = dsa.forward(x.q_idx, x.w, x.k_idx, x.q, x.kv, x.k, x.scale, d_v)
     dout = synth.grad_out(x, args.seed + rank)
@@ -675,7 +675,7 @@ def bench_bwd(args, world, rank, local):
         "value": job_throughput(world, x.T, ms_step), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": f"{args.bwd} causal prefill backward, L={x.T}, k={x.k}, Hq={Hq}, "
+        "config": {"workload": f"{args.bwd} causal prefill backward, L={x.S}, rows={x.T}, k={x.k}, Hq={Hq}, "
                                f"d_qk={d_qk}, d_v={d_v}; inputs larger than L2, no flush",
                    "global_batch": world, "seq_len": x.T, "parallelism": f"replicas{world}"},
         "roofline": {"bound": "tensor", "kernel": "attention backward (dkv + dq kernels, one call)",

@@ -592,6 +592,8 @@ int attn_bwd(const __nv_bfloat16* q, const __nv_bfloat16* kv, const int32_t* idx
     cudaError_t e = cudaFuncSetAttribute(attn_bwd_dkv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)s_dkv);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(attn_bwd_dkv_kernel)");
+    e = cudaFuncSetAttribute(attn_bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s_dq);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(attn_bwd_dq_kernel)");
     __nv_bfloat16* g_ws = reinterpret_cast<__nv_bfloat16*>(workspace);
     for (int r0 = 0; r0 < T; r0 += rows) {
         const int n = std::min(rows, T - r0);
