@@ -57,6 +57,8 @@ def _load():
             lib.oracle_lse_merge.argtypes = [P, P, i32, i32, i32, P, P]
             lib.oracle_sparse_attn_bwd_rows.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, dbl,
                                                         P, P, P]
+            lib.oracle_indexer_kl_rows.argtypes = [P, P, P, P, P, i32, i32, i32, i32, dbl, P, P, P, i32,
+                                                   i32, P, P, P, P]
             _lib = lib
     return _lib
 
@@ -196,6 +198,32 @@ def sparse_attn_bwd(q, kv, idx, pos, k_base, scale: float, d_v: int, dout):
                                         dq.ctypes.data_as(ctypes.c_void_p),
                                         dkv.ctypes.data_as(ctypes.c_void_p))
     return dq, dkv
+
+
+def indexer_kl(q, kv, idx, pos, k_base, scale: float, q_idx, w, k_idx):
+    """Indexer KL loss over each row's selected set and its gradient:
+    (loss fp64 [T], dw fp64 [T, H_I], dq_idx fp64 [T, H_I, d_I], dk_idx fp64 [S, d_I]).
+    q bf16 [T, Hq, d_qk], kv bf16 [S, d_qk], q_idx e4m3 [T, H_I, d_I], w fp32 [T, H_I],
+    k_idx e4m3 [S, d_I], idx/pos/k_base int32."""
+    q_r, qp = _c(_u16(q), np.uint16)
+    kvu, kvp = _c(_u16(kv), np.uint16)
+    i_r, ip = _c(_np(idx, np.int32), np.int32)
+    p_r, pp = _c(_np(pos, np.int32), np.int32)
+    b_r, bp = _c(_np(k_base, np.int32), np.int32)
+    qi, qip = _c(_u8(q_idx), np.uint8)
+    w_r, wp = _c(_np(w, np.float32), np.float32)
+    ki, kip = _c(_u8(k_idx), np.uint8)
+    R, Hq, d_qk = q_r.shape
+    _, H_I, d_I = qi.shape
+    k = i_r.shape[1]
+    loss = np.zeros(R, np.float64)
+    dw = np.zeros((R, H_I), np.float64)
+    dq = np.zeros((R, H_I, d_I), np.float64)
+    dk = np.zeros((ki.shape[0], d_I), np.float64)
+    vp = lambda a: a.ctypes.data_as(ctypes.c_void_p)
+    _load().oracle_indexer_kl_rows(qp, kvp, ip, pp, bp, R, k, Hq, d_qk, float(scale), qip, wp, kip, H_I,
+                                   d_I, vp(loss), vp(dw), vp(dq), vp(dk))
+    return loss, dw, dq, dk
 
 
 def dense_attn_row(q_row, kv, pos: int, k_base: int, scale: float, d_v: int):

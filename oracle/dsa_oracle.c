@@ -427,3 +427,131 @@ void oracle_sparse_attn_bwd_rows(const uint16_t* q_rows, const uint16_t* kv, con
     free(z);
     free(sel);
 }
+
+/* Indexer KL loss and its gradient with respect to the indexer's inputs.
+ * "Paper Breakdown: DeepSeek-V3.2", "Continued Pre-Training (2.1.1)" table:
+ * the dense warm-up trains the indexer with L^I = sum_t D_KL(p_{t,:} || Softmax(I_{t,:}))
+ * with the main model frozen; the sparse stage keeps the KL on the selected set
+ * S_t, with the indexer's input detached (no gradient into the main model).
+ * The pages leave p_{t,:} undefined; reading: the main attention distribution
+ * of row t summed over the query heads and L1-normalised over the keys, so
+ * over the set S_t (the dense stage is S_t = every s <= pos[t]):
+ *   P_{h,s} = softmax over S_t of scale q_h.c_s        (one distribution per head)
+ *   p_s     = sum_h P_{h,s} / sum_{s', h} P_{h,s'}
+ *   u_{j,s} = q^I_j.k^I_s,  I_s = sum_j w_j ReLU(u_{j,s})   (index score, unrounded)
+ *   L_t     = sum_s p_s (log p_s - log softmax_S(I)_s)     (0 log 0 = 0)
+ * p is a constant (detached). With dI_s = softmax_S(I)_s - p_s:
+ *   dw_j     = sum_s dI_s ReLU(u_{j,s})
+ *   dq^I_j   = sum_s dI_s w_j [u_{j,s} > 0] k^I_s
+ *   dk^I_s  += sum_j dI_s w_j [u_{j,s} > 0] q^I_j          (over rows; caller zeroes)
+ * ReLU'(0) is taken as 0. S_t = the entries of idx_row that are >= 0 and <= pos.
+ * Rows run one after another (dk accumulates deterministically). */
+void oracle_indexer_kl_rows(const uint16_t* q_rows, const uint16_t* kv, const int32_t* idx_rows,
+                            const int32_t* pos_rows, const int32_t* base_rows, int R, int k, int Hq,
+                            int d_qk, double scale, const uint8_t* qi_rows, const float* w_rows,
+                            const uint8_t* k_idx, int H_I, int d_I, double* loss, double* dw,
+                            double* dqi, double* dki)
+{
+    e4m3_init();
+    const size_t kk = (size_t)(k > 0 ? k : 1);
+    int32_t* sel = (int32_t*)malloc(sizeof(int32_t) * kk);
+    double* z = (double*)malloc(sizeof(double) * kk);
+    double* p = (double*)malloc(sizeof(double) * kk);
+    double* I = (double*)malloc(sizeof(double) * kk);
+    double* u = (double*)malloc(sizeof(double) * kk * (size_t)H_I);
+    double* qh = (double*)malloc(sizeof(double) * (size_t)d_qk);
+    for (int r = 0; r < R; ++r) {
+        const int32_t* idx_row = idx_rows + (size_t)r * k;
+        const int64_t pos = pos_rows[r], k_base = base_rows[r];
+        const uint8_t* qi = qi_rows + (size_t)r * H_I * d_I;
+        const float* w = w_rows + (size_t)r * H_I;
+        double* dw_r = dw + (size_t)r * H_I;
+        double* dq_r = dqi + (size_t)r * H_I * d_I;
+        for (int j = 0; j < H_I; ++j)
+            dw_r[j] = 0.0;
+        for (int e = 0; e < H_I * d_I; ++e)
+            dq_r[e] = 0.0;
+        loss[r] = 0.0;
+        int n = 0;
+        for (int i = 0; i < k; ++i)
+            if (idx_row[i] >= 0 && idx_row[i] <= pos)
+                sel[n++] = idx_row[i];
+        if (n == 0)
+            continue;
+        /* target: head-summed main attention over S_t, L1-normalised */
+        for (int i = 0; i < n; ++i)
+            p[i] = 0.0;
+        for (int h = 0; h < Hq; ++h) {
+            for (int d = 0; d < d_qk; ++d)
+                qh[d] = bf16_decode(q_rows[((size_t)r * Hq + h) * d_qk + d]);
+            double m = -INFINITY;
+            for (int i = 0; i < n; ++i) {
+                const uint16_t* c_s = kv + (size_t)(k_base + sel[i]) * d_qk;
+                double dot = 0.0;
+                for (int d = 0; d < d_qk; ++d)
+                    dot += qh[d] * bf16_decode(c_s[d]);
+                z[i] = scale * dot;
+                if (z[i] > m)
+                    m = z[i];
+            }
+            double l = 0.0;
+            for (int i = 0; i < n; ++i)
+                l += exp(z[i] - m);
+            for (int i = 0; i < n; ++i)
+                p[i] += exp(z[i] - m) / l;
+        }
+        double psum = 0.0;
+        for (int i = 0; i < n; ++i)
+            psum += p[i];
+        for (int i = 0; i < n; ++i)
+            p[i] /= psum;
+        /* index scores over S_t and their log-softmax */
+        double mI = -INFINITY;
+        for (int i = 0; i < n; ++i) {
+            const uint8_t* ks = k_idx + (size_t)(k_base + sel[i]) * d_I;
+            double acc = 0.0;
+            for (int j = 0; j < H_I; ++j) {
+                double dot = 0.0;
+                for (int d = 0; d < d_I; ++d)
+                    dot += E4M3[qi[(size_t)j * d_I + d]] * E4M3[ks[d]];
+                u[(size_t)i * H_I + j] = dot;
+                acc += (double)w[j] * (dot > 0.0 ? dot : 0.0);
+            }
+            I[i] = acc;
+            if (acc > mI)
+                mI = acc;
+        }
+        double lI = 0.0;
+        for (int i = 0; i < n; ++i)
+            lI += exp(I[i] - mI);
+        const double lseI = mI + log(lI);
+        double L = 0.0;
+        for (int i = 0; i < n; ++i)
+            if (p[i] > 0.0)
+                L += p[i] * (log(p[i]) - (I[i] - lseI));
+        loss[r] = L;
+        /* gradients through the index score */
+        for (int i = 0; i < n; ++i) {
+            const double dI = exp(I[i] - lseI) - p[i];
+            const uint8_t* ks = k_idx + (size_t)(k_base + sel[i]) * d_I;
+            double* dk_s = dki + (size_t)(k_base + sel[i]) * d_I;
+            for (int j = 0; j < H_I; ++j) {
+                const double uj = u[(size_t)i * H_I + j];
+                dw_r[j] += dI * (uj > 0.0 ? uj : 0.0);
+                if (uj > 0.0) {
+                    const double c = dI * (double)w[j];
+                    for (int d = 0; d < d_I; ++d) {
+                        dq_r[(size_t)j * d_I + d] += c * E4M3[ks[d]];
+                        dk_s[d] += c * E4M3[qi[(size_t)j * d_I + d]];
+                    }
+                }
+            }
+        }
+    }
+    free(qh);
+    free(u);
+    free(I);
+    free(p);
+    free(z);
+    free(sel);
+}
