@@ -58,6 +58,9 @@ def parse():
     ap.add_argument("--bwd", nargs="?", const="prefill32k", default=None,
                     help="time the sparse attention backward on this prefill workload "
                          "(default prefill32k) instead of the default step")
+    ap.add_argument("--kl", nargs="?", const="prefill32k", default=None,
+                    help="time the indexer KL loss and its gradient on this prefill workload "
+                         "(default prefill32k) instead of the default step")
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -699,6 +702,90 @@ def bench_bwd(args, world, rank, local):
     return res
 
 
+def bench_kl(args, world, rank, local):
+    """Indexer KL loss over the selected sets (the sparse training stage's
+    indexer objective) and its gradient to w, q^I, k^I, for every row of one
+    causal prefill. The selected sets are the GPU indexer's Top-k and lse the
+    attention forward's, both computed once, untimed. A step is zeroing dk_idx
+    plus the loss call."""
+    import sparse_attention_20_b200 as dsa
+    from sparse_attention_20_b200 import build as dsa_build
+    if rank == 0:
+        dsa_build.build()
+    barrier(world)
+    dsa.load_library()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    x = synth.prefill_inputs(args.kl, device=dev, seed=args.seed + rank, L=args.seq_len, T=args.rows)
+    Hq, d_qk = x.q.shape[1], x.q.shape[2]
+    H_I, d_I = x.q_idx.shape[1], x.q_idx.shape[2]
+    idx, _, lse = dsa.forward(x.q_idx, x.w, x.k_idx, x.q, x.kv, x.k, x.scale, x.d_v)
+    dk = torch.empty((x.S, d_I), dtype=torch.float32, device=dev)
+    lib = dsa.load_library()
+    ws = torch.empty(int(lib.dsa_indexer_kl_workspace_size(x.T, x.k)), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        dk.zero_()
+        return dsa.indexer_kl(x.q, x.kv, idx, lse, x.q_idx, x.w, x.k_idx, x.scale, dk_idx=dk, workspace=ws,
+                              stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert dsa.device_status() == 0, dsa.last_error()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    n0 = dsa.launch_count()
+    start.record(stream)
+    for _ in range(args.steps):
+        res = step()
+    end.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    launches = dsa.launch_count() - n0
+    clk = clocks.stop()
+    ms_step = max_over_ranks(world, start.elapsed_time(end)) / args.steps
+    assert dsa.device_status() == 0, dsa.last_error()
+    assert torch.isfinite(res[0]).all()
+    # bf16 MMA flops of the head-summed probabilities: 2 Hq d_qk per (row, selected slot)
+    sel = torch.clamp(x.positions().cpu().long() + 1, max=x.k)
+    flops = float(sel.sum().item()) * 2 * Hq * d_qk
+    peaks = measured_peaks()
+    tf = flops / (ms_step * 1e-3) / 1e12
+    out = {
+        "metric": "indexer KL loss + gradient tokens/s (selected sets)",
+        "value": job_throughput(world, x.T, ms_step), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{args.kl} causal prefill, L={x.S}, rows={x.T}, k={x.k}, Hq={Hq}, d_qk={d_qk}, "
+                               f"H_I={H_I}, d_I={d_I}; inputs larger than L2, no flush",
+                   "global_batch": world, "seq_len": x.T, "parallelism": f"replicas{world}"},
+        "roofline": {"bound": "tensor", "kernel": "head-summed attention probabilities + per-row loss (one call)",
+                     "achieved": tf, "peak": peaks["bf16_sustained"], "unit": "TFLOP/s",
+                     "frac": tf / peaks["bf16_sustained"], "traffic": None,
+                     "peak_source": f"{peaks['source']} bf16 sustained"},
+        "mean_loss": float(res[0].mean().item()),
+        "gpu_launches": launches, "clocks": clk,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        import oracle
+        g = torch.Generator().manual_seed(args.seed)
+        rows = sorted(torch.randperm(x.T, generator=g)[:8].tolist())
+        r = torch.tensor(rows, device=dev)
+        t0 = time.perf_counter()
+        oracle.indexer_kl(x.q[r].cpu(), x.kv.cpu(), idx[r].cpu(), x.positions()[r].cpu(),
+                          torch.zeros(len(rows), dtype=torch.int32), x.scale, x.q_idx[r].cpu(), x.w[r].cpu(),
+                          x.k_idx.cpu())
+        dt = time.perf_counter() - t0
+        out["cpu_baseline"] = {"value": len(rows) / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                               "sample": f"{len(rows)} uniformly drawn query rows of the {args.kl} KL loss "
+                                         f"(fp64, one thread); {dt:.1f} s"}
+    return out
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -708,7 +795,8 @@ def main():
             print(json.dumps(bench_reference(args, world, 0)), flush=True)
         return
     world, rank, local = dist_setup(args)
-    mode = bench_bwd if args.bwd else bench_varlen if args.varlen else bench_ours
+    mode = (bench_bwd if args.bwd else bench_kl if args.kl else bench_varlen if args.varlen
+            else bench_ours)
     res = mode(args, world, rank, local)
     if rank == 0:
         print(json.dumps(res), flush=True)

@@ -197,6 +197,42 @@ int dsa_sparse_mla_attn_bwd(const void* q, const void* kv, const int32_t* idx, c
                             float* dkv, void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * Indexer KL loss over each row's selected set and its gradient with respect
+ * to the indexer's inputs: the objective that trains the lightning indexer
+ * toward the main attention ("Paper Breakdown: DeepSeek-V3.2", table
+ * "Continued Pre-Training (2.1.1)": dense warm-up L^I = sum_t
+ * D_KL(p_{t,:} || Softmax(I_{t,:})) with the main model frozen; sparse stage:
+ * the same KL over the selected set S_t, indexer input detached). The pages
+ * leave p_{t,:} undefined; here it is the main attention of row t summed over
+ * the query heads and L1-normalised over S_t:
+ *   p_s  = sum_h exp(scale q_h.c_s - lse_h) / (sum over s' in S_t and h)
+ *   I_s  = sum_j w_j ReLU(q^I_j.k^I_s)          (unrounded fp32)
+ *   loss[t] = sum_{s in S_t} p_s (log p_s - log softmax_{S_t}(I)_s)
+ * and, with dI_s = softmax_{S_t}(I)_s - p_s (p is a constant):
+ *   dw[t,j]       = sum_s dI_s ReLU(q^I_j.k^I_s)
+ *   dq_idx[t,j,:] = sum_s dI_s w_j [q^I_j.k^I_s > 0] k^I_s
+ *   dk_idx[s,:]  += sum_t sum_j dI_s w_j [q^I_j.k^I_s > 0] q^I_j
+ * S_t is row t's idx entries (valid entries first; only the first
+ * min(k, pos[t]+1) are read, negatives and entries > pos[t] ignored). The
+ * dense warm-up loss is this call with every s <= pos[t] in idx (k >= L).
+ * Inputs: q, kv, idx, pos, k_base, scale as dsa_sparse_mla_attn; lse fp32
+ * [T, Hq] its log-sum-exp for the same idx; q_idx, w, k_idx as
+ * dsa_indexer_topk (e4m3, fp32, e4m3).
+ * Outputs (device, caller-owned): loss fp32 [T]; dw fp32 [T, H_I]; dq_idx
+ * fp32 [T, H_I, d_I] (written); dk_idx fp32 [S, d_I] ACCUMULATED (atomic
+ * adds; zero it for a fresh gradient). A row without entries gives 0.
+ * workspace: at least dsa_indexer_kl_workspace_size(1, k) bytes; up to 8192
+ * rows per pass (DSA_ERR_WORKSPACE below one row).
+ * Supported: Hq <= 128, d_qk % 16 == 0 and <= 576, H_I <= 16, d_I % 16 == 0
+ * and <= 256, H_I * d_I <= 4096, 1 <= k <= 4096 (DSA_ERR_UNSUPPORTED).
+ */
+size_t dsa_indexer_kl_workspace_size(int T, int k);
+int dsa_indexer_kl(const void* q, const void* kv, const int32_t* idx, const int32_t* pos, const int32_t* k_base,
+                   const float* lse, const void* q_idx, const float* w, const void* k_idx, int T, int S, int Hq,
+                   int d_qk, int H_I, int d_I, int k, float scale, float* loss, float* dw, float* dq_idx,
+                   float* dk_idx, void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * The whole hot path: dsa_indexer_topk followed by dsa_sparse_mla_attn on the
  * same stream. `idx` is an output the caller keeps (it is also the input of
  * the attention step). Argument meanings and limits as above.

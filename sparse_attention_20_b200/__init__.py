@@ -33,7 +33,7 @@ EXPORTS = ("dsa_workspace_size", "dsa_indexer_topk", "dsa_sparse_mla_attn", "dsa
            "dsa_device_status", "dsa_last_error", "dsa_abi_version", "dsa_launch_count",
            "dsa_indexer_topk_noalloc", "dsa_selftest_bounded_wait", "dsa_indexer_topk_varlen",
            "dsa_indexer_topk_paged", "dsa_sparse_mla_attn_paged", "dsa_sparse_mla_attn_bwd",
-           "dsa_sparse_mla_attn_bwd_workspace_size")
+           "dsa_sparse_mla_attn_bwd_workspace_size", "dsa_indexer_kl", "dsa_indexer_kl_workspace_size")
 
 
 class DSAError(RuntimeError):
@@ -81,6 +81,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.dsa_sparse_mla_attn_bwd.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, P, P, P, Z,
                                                 P]
         lib.dsa_sparse_mla_attn_bwd.restype = I
+        lib.dsa_indexer_kl_workspace_size.argtypes = [I, I]
+        lib.dsa_indexer_kl_workspace_size.restype = Z
+        lib.dsa_indexer_kl.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, F, P, P, P, P, P, Z, P]
+        lib.dsa_indexer_kl.restype = I
         lib.dsa_selftest_bounded_wait.argtypes = [I, P]
         lib.dsa_selftest_bounded_wait.restype = I
         _lib = lib
@@ -297,6 +301,38 @@ def sparse_mla_attn_bwd(q, kv, idx, out, lse, dout, scale: float, pos=None, k_ba
                                        _ptr(dq), _ptr(dkv), _ptr(workspace), workspace.numel(),
                                        _stream(stream)))
     return dq, dkv
+
+
+def indexer_kl(q, kv, idx, lse, q_idx, w, k_idx, scale: float, pos=None, k_base=None, dk_idx=None,
+               workspace=None, stream=None):
+    """Indexer KL loss over each row's selected set and its gradient:
+    (loss fp32 [T], dw fp32 [T, H_I], dq_idx fp32 [T, H_I, d_I], dk_idx fp32 [S, d_I]).
+
+    lse is the attention forward's log-sum-exp for the same idx. dk_idx is
+    accumulated into (a new zeroed tensor when None)."""
+    q, kv, lse, w = _dev(q, "q"), _dev(kv, "kv"), _dev(lse, "lse"), _dev(w, "w")
+    q_idx, k_idx = _fp8(q_idx, "q_idx"), _fp8(k_idx, "k_idx")
+    if q.dtype != torch.bfloat16 or kv.dtype != torch.bfloat16:
+        raise TypeError("q and kv must be bfloat16")
+    idx = _i32(idx, "idx")
+    T, Hq, d_qk = q.shape
+    _, H_I, d_I = q_idx.shape
+    S, k = kv.shape[0], idx.shape[1]
+    pos, k_base = _i32(pos, "pos"), _i32(k_base, "k_base")
+    dev = q.device
+    loss = torch.empty(T, dtype=torch.float32, device=dev)
+    dw = torch.empty((T, H_I), dtype=torch.float32, device=dev)
+    dq_idx = torch.empty((T, H_I, d_I), dtype=torch.float32, device=dev)
+    if dk_idx is None:
+        dk_idx = torch.zeros((S, d_I), dtype=torch.float32, device=dev)
+    lib = load_library()
+    if workspace is None:
+        workspace = torch.empty(int(lib.dsa_indexer_kl_workspace_size(T, k)), dtype=torch.uint8, device=dev)
+    _check(lib.dsa_indexer_kl(_ptr(q), _ptr(kv), _ptr(idx), _ptr(pos), _ptr(k_base), _ptr(lse), _ptr(q_idx),
+                              _ptr(w), _ptr(k_idx), T, S, Hq, d_qk, H_I, d_I, k, float(scale), _ptr(loss),
+                              _ptr(dw), _ptr(dq_idx), _ptr(dk_idx), _ptr(workspace), workspace.numel(),
+                              _stream(stream)))
+    return loss, dw, dq_idx, dk_idx
 
 
 def forward(q_idx, w, k_idx, q, kv, k: int, scale: float, d_v: int, pos=None, k_base=None,

@@ -18,6 +18,7 @@
 #include "attn_tc.cuh"
 #include "common.cuh"
 #include "indexer_chunked.cuh"
+#include "indexer_kl.cuh"
 #include "indexer_scores.cuh"
 #include "indexer_tc.cuh"
 #include "topk_select.cuh"
@@ -607,6 +608,65 @@ int attn_bwd(const __nv_bfloat16* q, const __nv_bfloat16* kv, const int32_t* idx
     return DSA_OK;
 }
 
+// ------------------------------------------------------------ indexer KL loss
+
+constexpr int kKlRowsMax = 8192;   // query rows per pass (workspace size)
+
+size_t kl_row_bytes(int k) { return (size_t)dsa::bwd::slots_pad(k) * sizeof(float); }
+
+int check_kl(const void* q, const void* kv, const int32_t* idx, const int32_t* pos, const int32_t* k_base,
+             const float* lse, const void* q_idx, const float* w, const void* k_idx, int T, int S, int Hq,
+             int d_qk, int H_I, int d_I, int k, const float* loss, const float* dw, const float* dqi,
+             const float* dki)
+{
+    if (!q || !kv || !idx || !lse || !q_idx || !w || !k_idx || !loss || !dw || !dqi || !dki)
+        return fail(DSA_ERR_ARG, "NULL argument");
+    if (!al16(q) || !al16(kv) || !al16(idx) || !al16(lse) || !al16(q_idx) || !al16(w) || !al16(k_idx) ||
+        !al16(loss) || !al16(dw) || !al16(dqi) || !al16(dki))
+        return fail(DSA_ERR_ARG, "every array must be 16-byte aligned");
+    if (int rc = check_rows(pos, k_base, T, S)) return rc;
+    if (Hq <= 0 || Hq > dsa::bwd::kMaxHeads || d_qk <= 0 || d_qk % 16 || d_qk > dsa::bwd::kMaxDqk)
+        return fail(DSA_ERR_UNSUPPORTED, "Hq=%d, d_qk=%d (supported: Hq <= 128, d_qk a multiple of 16 <= 576)",
+                    Hq, d_qk);
+    if (H_I <= 0 || H_I > dsa::kl::kMaxHI || d_I <= 0 || d_I % 16 || d_I > dsa::kl::kMaxDI ||
+        H_I * d_I > dsa::kl::kMaxQElems)
+        return fail(DSA_ERR_UNSUPPORTED, "H_I=%d, d_I=%d (supported: H_I <= 16, d_I a multiple of 16 <= 256, "
+                    "H_I * d_I <= 4096)", H_I, d_I);
+    if (k <= 0 || k > 4096) return fail(DSA_ERR_UNSUPPORTED, "k=%d (supported: 1..4096)", k);
+    return DSA_OK;
+}
+
+int indexer_kl(const __nv_bfloat16* q, const __nv_bfloat16* kv, const int32_t* idx, const int32_t* pos,
+               const int32_t* k_base, const float* lse, const uint8_t* q_idx, const float* w,
+               const uint8_t* k_idx, int T, int S, int Hq, int d_qk, int H_I, int d_I, int k, float scale,
+               float* loss, float* dw, float* dqi, float* dki, void* workspace, size_t ws_bytes, cudaStream_t st)
+{
+    using namespace dsa::kl;
+    const size_t row_bytes = kl_row_bytes(k);
+    const size_t fit = workspace && al16(workspace) ? ws_bytes / row_bytes : 0;
+    if (fit < 1)
+        return fail(DSA_ERR_WORKSPACE, "indexer KL loss needs %zu workspace bytes per row (got %zu)", row_bytes,
+                    ws_bytes);
+    const int rows = (int)std::min<size_t>(std::min<size_t>(fit, (size_t)T), 65535);
+    const size_t s_prob = prob_smem(Hq, d_qk), s_row = row_smem(H_I, d_I, k);
+    cudaError_t e = cudaFuncSetAttribute(head_prob_sum_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)s_prob);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(head_prob_sum_kernel)");
+    e = cudaFuncSetAttribute(indexer_kl_row_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s_row);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(indexer_kl_row_kernel)");
+    float* psum = reinterpret_cast<float*>(workspace);
+    for (int r0 = 0; r0 < T; r0 += rows) {
+        const int n = std::min(rows, T - r0);
+        head_prob_sum_kernel<<<dim3(dsa::bwd::slots_pad(k) / dsa::bwd::kSlots, n), dsa::bwd::kThreads, s_prob,
+                               st>>>(q, kv, idx, pos, k_base, lse, r0, T, S, Hq, d_qk, k, scale, psum);
+        DSA_LAUNCH_CHECK("head_prob_sum_kernel");
+        indexer_kl_row_kernel<<<n, kRowThreads, s_row, st>>>(q_idx, w, k_idx, idx, pos, k_base, psum, r0, T, S,
+                                                             H_I, d_I, k, loss, dw, dqi, dki);
+        DSA_LAUNCH_CHECK("indexer_kl_row_kernel");
+    }
+    return DSA_OK;
+}
+
 }  // namespace
 
 // ===================================================================== C ABI
@@ -805,6 +865,28 @@ int dsa_sparse_mla_attn_bwd(const void* q, const void* kv, const int32_t* idx, c
     return attn_bwd(reinterpret_cast<const bf*>(q), reinterpret_cast<const bf*>(kv), idx, pos, k_base,
                     reinterpret_cast<const bf*>(out), lse, reinterpret_cast<const bf*>(dout), T, S, Hq,
                     d_qk, d_v, k, scale, dq, dkv, workspace, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t dsa_indexer_kl_workspace_size(int T, int k)
+{
+    if (T <= 0 || k <= 0) return 0;
+    return (size_t)std::min(T, kKlRowsMax) * kl_row_bytes(k);
+}
+
+int dsa_indexer_kl(const void* q, const void* kv, const int32_t* idx, const int32_t* pos, const int32_t* k_base,
+                   const float* lse, const void* q_idx, const float* w, const void* k_idx, int T, int S, int Hq,
+                   int d_qk, int H_I, int d_I, int k, float scale, float* loss, float* dw, float* dq_idx,
+                   float* dk_idx, void* workspace, size_t ws_bytes, void* stream)
+{
+    g_err[0] = 0;
+    if (int rc = check_kl(q, kv, idx, pos, k_base, lse, q_idx, w, k_idx, T, S, Hq, d_qk, H_I, d_I, k, loss, dw,
+                          dq_idx, dk_idx))
+        return rc;
+    using bf = __nv_bfloat16;
+    return indexer_kl(reinterpret_cast<const bf*>(q), reinterpret_cast<const bf*>(kv), idx, pos, k_base, lse,
+                      reinterpret_cast<const uint8_t*>(q_idx), w, reinterpret_cast<const uint8_t*>(k_idx), T, S,
+                      Hq, d_qk, H_I, d_I, k, scale, loss, dw, dq_idx, dk_idx, workspace, ws_bytes,
+                      reinterpret_cast<cudaStream_t>(stream));
 }
 
 int dsa_forward(const void* q_idx, const float* w, const void* k_idx, const void* q,

@@ -123,6 +123,26 @@ def test_attention_backward_rejects_bad_arguments(lib):
     assert lib.dsa_sparse_mla_attn_bwd_workspace_size(0, 128, 2048) == 0
 
 
+def test_indexer_kl_rejects_bad_arguments(lib):
+    f = lib.dsa_indexer_kl
+    sc = ctypes.c_float(0.1)
+
+    def call(Hq=128, d_qk=576, H_I=8, d_I=128, k=64, lse=FAKE, wsb=ctypes.c_size_t(1 << 20), wsp=FAKE):
+        return f(FAKE, FAKE, FAKE, None, None, lse, FAKE, FAKE, FAKE, 4, 4, Hq, d_qk, H_I, d_I, k, sc, FAKE,
+                 FAKE, FAKE, FAKE, wsp, wsb, None)
+
+    assert call(lse=None) == -1
+    assert call(Hq=256) == -2
+    assert call(H_I=17) == -2
+    assert call(d_I=136) == -2          # not a multiple of 16
+    assert call(H_I=16, d_I=512) == -2  # above 256
+    assert call(k=5000) == -2
+    assert call(wsb=ctypes.c_size_t(16)) == -5
+    assert lib.dsa_indexer_kl_workspace_size(1, 2048) == 2048 * 4
+    assert lib.dsa_indexer_kl_workspace_size(50000, 100) == 8192 * 128 * 4
+    assert lib.dsa_indexer_kl_workspace_size(0, 100) == 0
+
+
 def test_binding_refuses_cpu_tensors():
     import torch
     x = torch.zeros((4, 8, 128), dtype=torch.uint8)
