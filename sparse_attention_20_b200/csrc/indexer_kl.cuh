@@ -276,10 +276,16 @@ indexer_kl_row_kernel(const uint8_t* __restrict__ q_idx, const float* __restrict
 #pragma unroll
             for (int j = 0; j < kMaxHI; ++j) {
                 if (j < H_I) {
-                    const float* qj = qf + j * d_I + part * 16;
+                    const float4* qj = reinterpret_cast<const float4*>(qf + j * d_I + part * 16);
                     float s = u[j];
 #pragma unroll
-                    for (int m = 0; m < 16; ++m) s = fmaf(qj[m], kf[m], s);
+                    for (int m = 0; m < 4; ++m) {
+                        const float4 qv = qj[m];
+                        s = fmaf(qv.x, kf[4 * m], s);
+                        s = fmaf(qv.y, kf[4 * m + 1], s);
+                        s = fmaf(qv.z, kf[4 * m + 2], s);
+                        s = fmaf(qv.w, kf[4 * m + 3], s);
+                    }
                     u[j] = s;
                 }
             }
@@ -329,10 +335,13 @@ indexer_kl_row_kernel(const uint8_t* __restrict__ q_idx, const float* __restrict
     L = block_sum(L, red + 24);
     if (tid == 0) loss[t] = any ? L : 0.f;
 
-    // pass B: gradients
-    float acc[kMaxQElems / kRowThreads];
+    // pass B: gradients. dq: thread owns groups g = tid + 256 e of four
+    // consecutive d of one head j (g < H_I d_I / 4)
+    constexpr int kGroups = kMaxQElems / 4 / kRowThreads;
+    float4 acc[kGroups];
 #pragma unroll
-    for (int e = 0; e < kMaxQElems / kRowThreads; ++e) acc[e] = 0.f;
+    for (int e = 0; e < kGroups; ++e) acc[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+    const int d4 = d_I / 4, nq4 = nq / 4;
     float dwp[kMaxHI];
 #pragma unroll
     for (int j = 0; j < kMaxHI; ++j) dwp[j] = 0.f;
@@ -377,20 +386,29 @@ indexer_kl_row_kernel(const uint8_t* __restrict__ q_idx, const float* __restrict
         __syncthreads();
         const int ns = min(kRowThreads, n_row - c0);
 #pragma unroll
-        for (int e = 0; e < kMaxQElems / kRowThreads; ++e) {
-            const int o = tid + e * kRowThreads;
-            if (o < nq) {
-                const int j = o / d_I, d = o - j * d_I;
-                float s = acc[e];
-                for (int sl = 0; sl < ns; ++sl) s = fmaf(cch[sl * H_I + j], lut[kch[(size_t)sl * d_I + d]], s);
-                acc[e] = s;
+        for (int e = 0; e < kGroups; ++e) {
+            const int g = tid + e * kRowThreads;
+            if (g < nq4) {
+                const int j = g / d4, d0 = 4 * (g - j * d4);
+                float4 a = acc[e];
+                for (int sl = 0; sl < ns; ++sl) {
+                    const float cj = cch[sl * H_I + j];
+                    const uint32_t kb = *reinterpret_cast<const uint32_t*>(kch + (size_t)sl * d_I + d0);
+                    const float2 lo = e4m3x2_to_float2((uint16_t)(kb & 0xFFFFu));
+                    const float2 hi = e4m3x2_to_float2((uint16_t)(kb >> 16));
+                    a.x = fmaf(cj, lo.x, a.x);
+                    a.y = fmaf(cj, lo.y, a.y);
+                    a.z = fmaf(cj, hi.x, a.z);
+                    a.w = fmaf(cj, hi.y, a.w);
+                }
+                acc[e] = a;
             }
         }
     }
 #pragma unroll
-    for (int e = 0; e < kMaxQElems / kRowThreads; ++e) {
-        const int o = tid + e * kRowThreads;
-        if (o < nq) dqi[(size_t)t * nq + o] = acc[e];
+    for (int e = 0; e < kGroups; ++e) {
+        const int g = tid + e * kRowThreads;
+        if (g < nq4) *reinterpret_cast<float4*>(dqi + (size_t)t * nq + 4 * g) = acc[e];
     }
     // dw: per-thread partials summed over the block, one head at a time
     for (int j = 0; j < H_I; ++j) {
