@@ -57,6 +57,7 @@ def _load():
             lib.oracle_lse_merge.argtypes = [P, P, i32, i32, i32, P, P]
             lib.oracle_sparse_attn_bwd_rows.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, dbl,
                                                         P, P, P]
+            lib.oracle_mha_attn_rows.argtypes = [P, P, P, P, P, i32, i32, i32, i32, dbl, P, P]
             lib.oracle_indexer_kl_rows.argtypes = [P, P, P, P, P, i32, i32, i32, i32, dbl, P, P, P, i32,
                                                    i32, P, P, P, P]
             _lib = lib
@@ -224,6 +225,24 @@ def indexer_kl(q, kv, idx, pos, k_base, scale: float, q_idx, w, k_idx):
     _load().oracle_indexer_kl_rows(qp, kvp, ip, pp, bp, R, k, Hq, d_qk, float(scale), qip, wp, kip, H_I,
                                    d_I, vp(loss), vp(dw), vp(dq), vp(dk))
     return loss, dw, dq, dk
+
+
+def mha_attn(q, k, v, pos, k_base, scale: float):
+    """Dense causal attention with per-head keys and values (MLA in MHA mode):
+    (out fp64 [R, Hq, d_hv], lse fp64 [R, Hq]). q bf16 [R, Hq, d_h], k bf16
+    [S, Hq, d_h], v bf16 [S, Hq, d_hv]; row r sees keys k_base[r] + 0..pos[r]."""
+    q_r, qp = _c(_u16(q), np.uint16)
+    k_r, kp = _c(_u16(k), np.uint16)
+    v_r, vp = _c(_u16(v), np.uint16)
+    p_r, pp = _c(_np(pos, np.int32), np.int32)
+    b_r, bp = _c(_np(k_base, np.int32), np.int32)
+    R, Hq, d_h = q_r.shape
+    d_hv = v_r.shape[2]
+    out = np.zeros((R, Hq, d_hv), np.float64)
+    lse = np.zeros((R, Hq), np.float64)
+    _load().oracle_mha_attn_rows(qp, kp, vp, pp, bp, R, Hq, d_h, d_hv, float(scale),
+                                 out.ctypes.data_as(ctypes.c_void_p), lse.ctypes.data_as(ctypes.c_void_p))
+    return out, lse
 
 
 def dense_attn_row(q_row, kv, pos: int, k_base: int, scale: float, d_v: int):

@@ -555,3 +555,55 @@ void oracle_indexer_kl_rows(const uint16_t* q_rows, const uint16_t* kv, const in
     free(z);
     free(sel);
 }
+
+/* MLA in MHA mode over a causal sequence (the bilingual paper summary's list of
+ * sections, "Appendix A MHA and MQA Modes of MLA", title only; "Paper
+ * Breakdown: DeepSeek-V3.2", section 2, "DSA under MLA (MQA Mode)"). Reading:
+ * in MHA mode every head has its own key and value rows (the latent row
+ * expanded per head), where MQA mode shares one latent row across heads. For a
+ * short prefill (L <= k) the selector keeps every causal key, so the mode is
+ * dense causal attention, per row t and head h over s = 0..pos:
+ *   z_s = scale q_{t,h}.k_{s,h},  o_{t,h} = sum_s softmax(z)_s v_{s,h},
+ *   lse = log sum_s exp(z_s)
+ * q [R, Hq, d_h] (row r at position pos_rows[r]), k [S, Hq, d_h], v [S, Hq, d_hv]
+ * (bf16); keys of row r at base_rows[r] + s. */
+void oracle_mha_attn_rows(const uint16_t* q_rows, const uint16_t* k, const uint16_t* v,
+                          const int32_t* pos_rows, const int32_t* base_rows, int R, int Hq, int d_h,
+                          int d_hv, double scale, double* out, double* lse)
+{
+    for (int r = 0; r < R; ++r) {
+        const int64_t n = (int64_t)pos_rows[r] + 1, base = base_rows[r];
+        double* z = (double*)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
+        for (int h = 0; h < Hq; ++h) {
+            double* o = out + ((size_t)r * Hq + h) * d_hv;
+            for (int c = 0; c < d_hv; ++c)
+                o[c] = 0.0;
+            if (n <= 0) {
+                lse[(size_t)r * Hq + h] = -INFINITY;
+                continue;
+            }
+            const uint16_t* qh = q_rows + ((size_t)r * Hq + h) * d_h;
+            double m = -INFINITY;
+            for (int64_t s = 0; s < n; ++s) {
+                const uint16_t* ks = k + ((size_t)(base + s) * Hq + h) * d_h;
+                double dot = 0.0;
+                for (int d = 0; d < d_h; ++d)
+                    dot += bf16_decode(qh[d]) * bf16_decode(ks[d]);
+                z[s] = scale * dot;
+                if (z[s] > m)
+                    m = z[s];
+            }
+            double l = 0.0;
+            for (int64_t s = 0; s < n; ++s)
+                l += exp(z[s] - m);
+            for (int64_t s = 0; s < n; ++s) {
+                const double p = exp(z[s] - m) / l;
+                const uint16_t* vs = v + ((size_t)(base + s) * Hq + h) * d_hv;
+                for (int c = 0; c < d_hv; ++c)
+                    o[c] += p * bf16_decode(vs[c]);
+            }
+            lse[(size_t)r * Hq + h] = m + log(l);
+        }
+        free(z);
+    }
+}
