@@ -61,6 +61,9 @@ def parse():
     ap.add_argument("--kl", nargs="?", const="prefill32k", default=None,
                     help="time the indexer KL loss and its gradient on this prefill workload "
                          "(default prefill32k) instead of the default step")
+    ap.add_argument("--mha", nargs="?", const="mha_short", default=None,
+                    help="time MLA MHA-mode dense causal attention (short prefill, default "
+                         "mha_short: 2048 tokens, 128 heads, d_h 192, d_hv 128) instead of the default step")
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -786,6 +789,76 @@ def bench_kl(args, world, rank, local):
     return out
 
 
+def bench_mha(args, world, rank, local):
+    """MLA in MHA mode on a short prefill (every causal key kept): dense causal
+    attention with per-head keys and values. A step is one call."""
+    import sparse_attention_20_b200 as dsa
+    from sparse_attention_20_b200 import build as dsa_build
+    if rank == 0:
+        dsa_build.build()
+    barrier(world)
+    dsa.load_library()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    q, k, v, scale = synth.mha_inputs(args.mha, device=dev, seed=args.seed + rank, L=args.seq_len)
+    T, Hq, d_h = q.shape
+    S, d_hv = k.shape[0], v.shape[2]
+    out = torch.empty((T, Hq, d_hv), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((T, Hq), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    step = lambda: dsa.mla_mha_attn(q, k, v, scale, out=out, lse=lse, stream=stream)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert dsa.device_status() == 0, dsa.last_error()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    n0 = dsa.launch_count()
+    start.record(stream)
+    for _ in range(args.steps):
+        step()
+    end.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    launches = dsa.launch_count() - n0
+    clk = clocks.stop()
+    ms_step = max_over_ranks(world, start.elapsed_time(end)) / args.steps
+    assert dsa.device_status() == 0, dsa.last_error()
+    pairs = sum(min(S, t + S - T + 1) for t in range(T))
+    flops = float(pairs) * Hq * 2 * (d_h + d_hv)
+    peaks = measured_peaks()
+    tf = flops / (ms_step * 1e-3) / 1e12
+    res = {
+        "metric": "MLA MHA-mode causal attention tokens/s (short prefill)",
+        "value": job_throughput(world, T, ms_step), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{args.mha}: L={S}, rows={T}, Hq={Hq}, d_h={d_h}, d_hv={d_hv}, dense causal; "
+                               f"inputs larger than L2, no flush",
+                   "global_batch": world, "seq_len": S, "parallelism": f"replicas{world}"},
+        "roofline": {"bound": "tensor", "kernel": "mha_causal_kernel", "achieved": tf,
+                     "peak": peaks["bf16_sustained"], "unit": "TFLOP/s", "frac": tf / peaks["bf16_sustained"],
+                     "traffic": None, "peak_source": f"{peaks['source']} bf16 sustained"},
+        "gpu_launches": launches, "clocks": clk,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        import numpy as np
+        import oracle
+        g = torch.Generator().manual_seed(args.seed)
+        rows = sorted(torch.randperm(T, generator=g)[:8].tolist())
+        r = torch.tensor(rows)
+        t0 = time.perf_counter()
+        oracle.mha_attn(q.cpu()[r], k.cpu(), v.cpu(), (r + S - T).int().numpy(), np.zeros(len(rows), np.int32),
+                        scale)
+        dt = time.perf_counter() - t0
+        res["cpu_baseline"] = {"value": len(rows) / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                               "sample": f"{len(rows)} uniformly drawn query rows of {args.mha} (fp64, one "
+                                         f"thread); {dt:.1f} s"}
+    return res
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -795,8 +868,8 @@ def main():
             print(json.dumps(bench_reference(args, world, 0)), flush=True)
         return
     world, rank, local = dist_setup(args)
-    mode = (bench_bwd if args.bwd else bench_kl if args.kl else bench_varlen if args.varlen
-            else bench_ours)
+    mode = (bench_bwd if args.bwd else bench_kl if args.kl else bench_mha if args.mha
+            else bench_varlen if args.varlen else bench_ours)
     res = mode(args, world, rank, local)
     if rank == 0:
         print(json.dumps(res), flush=True)

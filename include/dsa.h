@@ -233,6 +233,27 @@ int dsa_indexer_kl(const void* q, const void* kv, const int32_t* idx, const int3
                    float* dk_idx, void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * MLA in MHA mode over one causal sequence: every head has its own key and
+ * value rows (the latent row expanded per head), where the sparse path's MQA
+ * mode shares one latent row across heads (the bilingual paper summary's
+ * section list, "Appendix A MHA and MQA Modes of MLA", title only; "Paper
+ * Breakdown: DeepSeek-V3.2", section 2, "DSA under MLA (MQA Mode)"). On a
+ * short prefill (L <= k) the selector keeps every causal key, so this is dense
+ * causal attention: for query row t (position pos[t] = t + S - T) and head h,
+ *   out[t,h] = sum_{s <= pos[t]} softmax_s(scale q[t,h].k[s,h]) v[s,h]
+ *   lse[t,h] = log sum_{s <= pos[t]} exp(scale q[t,h].k[s,h])
+ * Arguments (device memory, caller-owned, row-major, 16-byte aligned):
+ *   q   bf16 [T, Hq, d_h]     queries of the last T tokens
+ *   k   bf16 [S, Hq, d_h]     per-head keys of all S tokens
+ *   v   bf16 [S, Hq, d_hv]    per-head values
+ *   out bf16 [T, Hq, d_hv] (out), lse fp32 [T, Hq] (out, natural log)
+ * Supported: (d_h, d_hv) in {(192, 128), (64, 64)}, 0 < T <= S, Hq <= 65535.
+ * Asynchronous on `stream`; no workspace.
+ */
+int dsa_mla_mha_attn(const void* q, const void* k, const void* v, int T, int S, int Hq, int d_h, int d_hv,
+                     float scale, void* out, float* lse, void* stream);
+
+/*
  * The whole hot path: dsa_indexer_topk followed by dsa_sparse_mla_attn on the
  * same stream. `idx` is an output the caller keeps (it is also the input of
  * the attention step). Argument meanings and limits as above.

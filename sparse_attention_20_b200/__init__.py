@@ -33,7 +33,8 @@ EXPORTS = ("dsa_workspace_size", "dsa_indexer_topk", "dsa_sparse_mla_attn", "dsa
            "dsa_device_status", "dsa_last_error", "dsa_abi_version", "dsa_launch_count",
            "dsa_indexer_topk_noalloc", "dsa_selftest_bounded_wait", "dsa_indexer_topk_varlen",
            "dsa_indexer_topk_paged", "dsa_sparse_mla_attn_paged", "dsa_sparse_mla_attn_bwd",
-           "dsa_sparse_mla_attn_bwd_workspace_size", "dsa_indexer_kl", "dsa_indexer_kl_workspace_size")
+           "dsa_sparse_mla_attn_bwd_workspace_size", "dsa_indexer_kl", "dsa_indexer_kl_workspace_size",
+           "dsa_mla_mha_attn")
 
 
 class DSAError(RuntimeError):
@@ -85,6 +86,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.dsa_indexer_kl_workspace_size.restype = Z
         lib.dsa_indexer_kl.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, F, P, P, P, P, P, Z, P]
         lib.dsa_indexer_kl.restype = I
+        lib.dsa_mla_mha_attn.argtypes = [P, P, P, I, I, I, I, I, F, P, P, P]
+        lib.dsa_mla_mha_attn.restype = I
         lib.dsa_selftest_bounded_wait.argtypes = [I, P]
         lib.dsa_selftest_bounded_wait.restype = I
         _lib = lib
@@ -333,6 +336,24 @@ def indexer_kl(q, kv, idx, lse, q_idx, w, k_idx, scale: float, pos=None, k_base=
                               _ptr(dw), _ptr(dq_idx), _ptr(dk_idx), _ptr(workspace), workspace.numel(),
                               _stream(stream)))
     return loss, dw, dq_idx, dk_idx
+
+
+def mla_mha_attn(q, k, v, scale: float, out=None, lse=None, stream=None):
+    """MLA in MHA mode, dense causal over one sequence: (out bf16 [T, Hq, d_hv],
+    lse fp32 [T, Hq]); q [T, Hq, d_h], k [S, Hq, d_h], v [S, Hq, d_hv] bf16, the
+    queries being the last T of the S tokens."""
+    q, k, v = _dev(q, "q"), _dev(k, "k"), _dev(v, "v")
+    if any(t.dtype != torch.bfloat16 for t in (q, k, v)):
+        raise TypeError("q, k and v must be bfloat16")
+    T, Hq, d_h = q.shape
+    S, d_hv = k.shape[0], v.shape[2]
+    if out is None:
+        out = torch.empty((T, Hq, d_hv), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((T, Hq), dtype=torch.float32, device=q.device)
+    _check(load_library().dsa_mla_mha_attn(_ptr(q), _ptr(k), _ptr(v), T, S, Hq, d_h, d_hv, float(scale),
+                                           _ptr(out), _ptr(lse), _stream(stream)))
+    return out, lse
 
 
 def forward(q_idx, w, k_idx, q, kv, k: int, scale: float, d_v: int, pos=None, k_base=None,

@@ -21,6 +21,7 @@
 #include "indexer_kl.cuh"
 #include "indexer_scores.cuh"
 #include "indexer_tc.cuh"
+#include "mha_attn.cuh"
 #include "topk_select.cuh"
 
 namespace dsa {
@@ -667,6 +668,23 @@ int indexer_kl(const __nv_bfloat16* q, const __nv_bfloat16* kv, const int32_t* i
     return DSA_OK;
 }
 
+// ------------------------------------------------------------- MLA MHA mode
+
+template <int DH, int DV>
+int mha_launch(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, int T, int S, int Hq,
+               float scale, __nv_bfloat16* out, float* lse, cudaStream_t st)
+{
+    using namespace dsa::mha;
+    auto kern = mha_causal_kernel<DH, DV>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)Shape<DH, DV>::kSmem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(mha_causal_kernel)");
+    kern<<<dim3(dsa::ceil_div(T, kRows), Hq), kThreads, Shape<DH, DV>::kSmem, st>>>(q, k, v, T, S, Hq, scale,
+                                                                                   out, lse);
+    DSA_LAUNCH_CHECK("mha_causal_kernel");
+    return DSA_OK;
+}
+
 }  // namespace
 
 // ===================================================================== C ABI
@@ -887,6 +905,25 @@ int dsa_indexer_kl(const void* q, const void* kv, const int32_t* idx, const int3
                       reinterpret_cast<const uint8_t*>(q_idx), w, reinterpret_cast<const uint8_t*>(k_idx), T, S,
                       Hq, d_qk, H_I, d_I, k, scale, loss, dw, dq_idx, dk_idx, workspace, ws_bytes,
                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+int dsa_mla_mha_attn(const void* q, const void* k, const void* v, int T, int S, int Hq, int d_h, int d_hv,
+                     float scale, void* out, float* lse, void* stream)
+{
+    g_err[0] = 0;
+    if (!q || !k || !v || !out || !lse) return fail(DSA_ERR_ARG, "NULL q, k, v, out or lse");
+    if (!al16(q) || !al16(k) || !al16(v) || !al16(out) || !al16(lse))
+        return fail(DSA_ERR_ARG, "q, k, v, out and lse must be 16-byte aligned");
+    if (T <= 0 || S <= 0 || T > S) return fail(DSA_ERR_ARG, "T=%d, S=%d (need 0 < T <= S)", T, S);
+    if (Hq <= 0 || Hq > 65535) return fail(DSA_ERR_UNSUPPORTED, "Hq=%d (supported: 1..65535)", Hq);
+    using bf = __nv_bfloat16;
+    auto st = reinterpret_cast<cudaStream_t>(stream);
+    const bf *qq = reinterpret_cast<const bf*>(q), *kk = reinterpret_cast<const bf*>(k),
+             *vv = reinterpret_cast<const bf*>(v);
+    bf* oo = reinterpret_cast<bf*>(out);
+    if (d_h == 192 && d_hv == 128) return mha_launch<192, 128>(qq, kk, vv, T, S, Hq, scale, oo, lse, st);
+    if (d_h == 64 && d_hv == 64) return mha_launch<64, 64>(qq, kk, vv, T, S, Hq, scale, oo, lse, st);
+    return fail(DSA_ERR_UNSUPPORTED, "d_h=%d, d_hv=%d (supported: (192, 128), (64, 64))", d_h, d_hv);
 }
 
 int dsa_forward(const void* q_idx, const float* w, const void* k_idx, const void* q,

@@ -319,3 +319,28 @@ def selection(pos, k: int, seed: int = 0) -> torch.Tensor:
 def grad_out(x: DSAInputs, seed: int = 0) -> torch.Tensor:
     """dL/dout of the attention output: bf16 N(0, 1) [T, Hq, d_v] on x's device."""
     return normal((x.T, x.q.shape[1], x.d_v), seed, x.config, "dout", x.q.device, dtype=torch.bfloat16)
+
+
+# MLA in MHA mode: per-head query/key dims 192 (128 expanded from the latent
+# row + the 64 rope dims) and value dims 128, for a short prefill (L <= k).
+MHA_CONFIGS = {
+    "mha_short": dict(L=2048, Hq=128, d_h=192, d_hv=128),
+    "mha_small": dict(L=300, Hq=4, d_h=64, d_hv=64),
+}
+
+
+def mha_inputs(name: str = "mha_short", device="cpu", seed: int = 0, L: int = None, T: int = None,
+               Hq: int = None):
+    """(q [T, Hq, d_h], k [L, Hq, d_h], v [L, Hq, d_hv], scale): bf16 N(0, 1),
+    the queries being the last T of the L tokens; scale 1/sqrt(d_h)."""
+    cfg = dict(MHA_CONFIGS[name])
+    if L is not None:
+        cfg["L"] = L
+    if Hq is not None:
+        cfg["Hq"] = Hq
+    L, H, dh, dv = cfg["L"], cfg["Hq"], cfg["d_h"], cfg["d_hv"]
+    T = L if T is None else int(T)
+    q = normal((T, H, dh), seed, name, "q", device, dtype=torch.bfloat16)
+    k = normal((L, H, dh), seed, name, "k", device, dtype=torch.bfloat16)
+    v = normal((L, H, dv), seed, name, "v", device, dtype=torch.bfloat16)
+    return q, k, v, 1.0 / math.sqrt(dh)

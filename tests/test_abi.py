@@ -143,6 +143,14 @@ def test_indexer_kl_rejects_bad_arguments(lib):
     assert lib.dsa_indexer_kl_workspace_size(0, 100) == 0
 
 
+def test_mha_rejects_bad_arguments(lib):
+    f = lib.dsa_mla_mha_attn
+    sc = ctypes.c_float(0.1)
+    assert f(FAKE, None, FAKE, 4, 4, 8, 192, 128, sc, FAKE, FAKE, None) == -1
+    assert f(FAKE, FAKE, FAKE, 5, 4, 8, 192, 128, sc, FAKE, FAKE, None) == -1   # T > S
+    assert f(FAKE, FAKE, FAKE, 4, 4, 8, 128, 128, sc, FAKE, FAKE, None) == -2   # head dims
+
+
 def test_binding_refuses_cpu_tensors():
     import torch
     x = torch.zeros((4, 8, 128), dtype=torch.uint8)
