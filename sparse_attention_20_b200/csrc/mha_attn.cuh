@@ -56,7 +56,9 @@ mha_causal_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __re
     extern __shared__ __align__(16) unsigned char smem_raw[];
     __nv_bfloat16* stage0 = reinterpret_cast<__nv_bfloat16*>(smem_raw);
 
-    const int t0 = blockIdx.x * kRows, h = blockIdx.y;
+    // the last query tiles see the most keys: launch them first so the short
+    // tiles fill the tail of the grid
+    const int t0 = (gridDim.x - 1 - blockIdx.x) * kRows, h = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gq = lane >> 2, tq = lane & 3;
     const int rA = t0 + warp * 16 + gq, rB = rA + 8;
