@@ -1,6 +1,7 @@
-"""Host-side helpers of the serving forms (no GPU): the page-pool builder
-places every key of every sequence where the block table says, and the
-varlen row maps give each packed row its sequence's range."""
+"""Host-side helpers (no GPU): the page-pool builder places every key of every
+sequence where the block table says, the varlen row maps give each packed row
+its sequence's range, the score-free selection is a valid set per row, and the
+MHA-mode inputs have their shapes."""
 import torch
 
 import synth
@@ -36,3 +37,27 @@ def test_varlen_rows_and_inputs_agree():
     # suffix-aligned tails: 2 of 5 keys in the first sequence, 3 of 7 in the second
     pos2, base2 = dsa.varlen_rows([0, 2, 5], [0, 5, 12], "cpu")
     assert pos2.tolist() == [3, 4, 4, 5, 6] and base2.tolist() == [0, 0, 5, 5, 5]
+
+
+def test_selection_rows_are_valid_sets():
+    """synth.selection: min(k, pos+1) distinct in-range entries first, -1 after,
+    for rows shorter and longer than k, an empty row and a one-key row."""
+    import numpy as np
+    pos = np.array([-1, 0, 5, 63, 64, 1000, 4095])
+    for k in (1, 64, 100):
+        sel = synth.selection(pos, k, seed=3).numpy()
+        assert sel.shape == (len(pos), k) and sel.dtype == np.int32
+        for row, p in zip(sel, pos):
+            n = min(k, int(p) + 1) if p >= 0 else 0
+            assert (row[n:] == -1).all()
+            v = row[:n]
+            assert len(set(v.tolist())) == n and ((v >= 0) & (v <= p)).all()
+    a = synth.selection(pos, 64, seed=3)
+    assert torch.equal(a, synth.selection(pos, 64, seed=3))          # seeded
+    assert not torch.equal(a, synth.selection(pos, 64, seed=4))
+
+
+def test_mha_inputs_shapes_and_tail():
+    q, k, v, scale = synth.mha_inputs("mha_small", L=50, T=20)
+    assert q.shape == (20, 4, 64) and k.shape == (50, 4, 64) and v.shape == (50, 4, 64)
+    assert q.dtype == k.dtype == v.dtype == torch.bfloat16 and abs(scale - 0.125) < 1e-12
