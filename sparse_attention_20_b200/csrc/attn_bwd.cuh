@@ -13,8 +13,8 @@
 // Two kernels, both on warp-level bf16 MMAs (m16n8k16, fp32 accumulate):
 //  - attn_bwd_dkv_kernel, one CTA per (row, 64 selected slots): recomputes z
 //    and dp for all heads against the 64 gathered rows, forms p and
-//    g = scale dz (bf16), adds g^T q + p^T dout into dkv (fp32 atomics, one
-//    add per (slot, column)) and stores g for the next kernel;
+//    g = scale dz (bf16), adds g^T q + p^T dout into dkv (float4 fp32
+//    atomics, one per four columns of a slot) and stores g for the next kernel;
 //  - attn_bwd_dq_kernel, one CTA per (row, 64 columns): dq = g . C over the
 //    row's selected rows, no atomics.
 // p and g are rounded to bf16 before they enter an MMA, as the forward rounds
