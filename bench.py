@@ -252,22 +252,32 @@ def run_attn(dsa, b, stream):
                         lse=b.lse, workspace=b.ws, stream=stream)
 
 
-def attn_traffic():
-    """DRAM bytes per prefill attention launch from the committed ncu summary,
-    or None once the kernel source has changed since those counters were taken."""
+def profiled_traffic(profile: str, key: str, sources) -> float | None:
+    """DRAM bytes per launch recorded in a committed ncu summary (`profiles/`),
+    or None once any of the kernel's source files has changed since those
+    counters were taken (the summary records a sha256 prefix of them)."""
     import hashlib
-    prof = os.path.join(ROOT, "profiles", "dram_bench_prefill128k_decode64.md")
+    prof = os.path.join(ROOT, "profiles", profile)
     csrc = os.path.join(ROOT, "sparse_attention_20_b200", "csrc")
     try:
         text = open(prof).read()
-        want = re.search(r"attn_source_sha256_16:\s*([0-9a-f]+)", text).group(1)
-        value = float(re.search(r"attn_traffic_bytes_per_launch:\s*([0-9.e+]+)", text).group(1))
+        want = re.search(key + r"_source_sha256_16:\s*([0-9a-f]+)", text).group(1)
+        value = float(re.search(key + r"_traffic_bytes_per_launch:\s*([0-9.e+]+)", text).group(1))
         h = hashlib.sha256()
-        for f in ("attn_tc.cuh", "sm100.cuh", "common.cuh"):
+        for f in sources:
             h.update(open(os.path.join(csrc, f), "rb").read())
     except (OSError, AttributeError, ValueError):
         return None
     return value if h.hexdigest()[:16] == want else None
+
+
+def attn_traffic():
+    """DRAM bytes per prefill attention launch (128K workload)."""
+    return profiled_traffic("dram_bench_prefill128k_decode64.md", "attn",
+                            ("attn_tc.cuh", "sm100.cuh", "common.cuh"))
+
+
+MHA_SOURCES = ("mha_attn.cuh", "attn_bwd.cuh", "sm100.cuh", "common.cuh")
 
 
 def fp8_gemm_tflops(n=8192, reps=10):
@@ -840,7 +850,9 @@ def bench_mha(args, world, rank, local):
                    "global_batch": world, "seq_len": S, "parallelism": f"replicas{world}"},
         "roofline": {"bound": "tensor", "kernel": "mha_causal_kernel", "achieved": tf,
                      "peak": peaks["bf16_sustained"], "unit": "TFLOP/s", "frac": tf / peaks["bf16_sustained"],
-                     "traffic": None, "peak_source": f"{peaks['source']} bf16 sustained"},
+                     "traffic": (profiled_traffic("mha_causal_short_prefill2k.md", "mha", MHA_SOURCES)
+                                 if args.mha == "mha_short" and args.seq_len is None else None),
+                     "peak_source": f"{peaks['source']} bf16 sustained"},
         "gpu_launches": launches, "clocks": clk,
     }
     if rank == 0 and not args.no_cpu_baseline:
