@@ -156,6 +156,17 @@ def test_binding_refuses_cpu_tensors():
     x = torch.zeros((4, 8, 128), dtype=torch.uint8)
     with pytest.raises(ValueError):
         dsa.indexer_topk(x, torch.zeros(4, 8), torch.zeros((4, 128), dtype=torch.uint8), 2)
+    q = torch.zeros((4, 2, 64), dtype=torch.bfloat16)
+    kv = torch.zeros((4, 64), dtype=torch.bfloat16)
+    idx = torch.zeros((4, 2), dtype=torch.int32)
+    out = torch.zeros((4, 2, 32), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        dsa.sparse_mla_attn_bwd(q, kv, idx, out, torch.zeros(4, 2), out, 0.1)
+    with pytest.raises(ValueError):
+        dsa.indexer_kl(q, kv, idx, torch.zeros(4, 2), x, torch.zeros(4, 8), torch.zeros((4, 128), dtype=torch.uint8),
+                       0.1)
+    with pytest.raises(ValueError):
+        dsa.mla_mha_attn(q, q, q, 0.1)
 
 
 def test_product_and_oracle_share_no_code():
