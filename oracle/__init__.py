@@ -49,6 +49,7 @@ def _load():
             lib.oracle_set_threads.argtypes = [i32]
             lib.oracle_indexer_row.argtypes = [P, P, P, i64, i64, i32, i32, P]
             lib.oracle_topk_row.argtypes = [P, i64, i32, P]
+            lib.oracle_indexer_scores_rows.argtypes = [P, P, P, P, P, i32, i32, i32, i64, P]
             lib.oracle_indexer_topk_rows.argtypes = [P, P, P, P, P, i32, i32, i32, i32, P]
             lib.oracle_sparse_attn_row.argtypes = [P, P, i64, i64, P, i32, i32, i32, i32, dbl, P, P]
             lib.oracle_sparse_attn_rows.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, dbl,
@@ -119,6 +120,23 @@ def indexer_scores(q_row, w_row, keys, n: int, k_base: int = 0) -> np.ndarray:
     out = np.empty(int(n), np.float32)
     _load().oracle_indexer_row(qp, wp, kp, int(k_base), int(n), H_I, d_I,
                                out.ctypes.data_as(ctypes.c_void_p))
+    return out
+
+
+def indexer_scores_rows(q_rows, w_rows, keys, pos, k_base) -> np.ndarray:
+    """I_{t,s} of R query rows at once (rows in parallel): float32 [R, max(pos)+1],
+    row r valid for s <= pos[r] and NaN past it. q_rows e4m3 [R, H_I, d_I],
+    w_rows [R, H_I], keys e4m3 [*, d_I], pos / k_base int [R]."""
+    q, qp = _c(_u8(q_rows), np.uint8)
+    w, wp = _c(_np(w_rows, np.float32), np.float32)
+    kk, kp = _c(_u8(keys), np.uint8)
+    p, pp = _c(_np(pos, np.int32), np.int32)
+    b, bp = _c(_np(k_base, np.int32), np.int32)
+    R, H_I, d_I = q.shape
+    ld = int(p.max()) + 1 if R else 1
+    out = np.full((R, ld), np.nan, np.float32)
+    _load().oracle_indexer_scores_rows(qp, wp, kp, pp, bp, R, H_I, d_I, ld,
+                                       out.ctypes.data_as(ctypes.c_void_p))
     return out
 
 

@@ -607,3 +607,21 @@ void oracle_mha_attn_rows(const uint16_t* q_rows, const uint16_t* k, const uint1
         free(z);
     }
 }
+
+/* ------------------------------------------- index scores of many rows */
+
+/* I_{t,s} of a list of query rows, one oracle_indexer_row per row (rows run
+ * in parallel; the arithmetic is that function's):
+ *   q_rows [R, H_I, d_I] e4m3, w_rows [R, H_I], pos_rows [R], base_rows [R];
+ *   out [R, ld] fp32: row r holds s = 0..pos_rows[r]; entries past that are
+ *   left untouched (ld >= max pos + 1). */
+void oracle_indexer_scores_rows(const uint8_t* q_rows, const float* w_rows, const uint8_t* keys,
+                                const int32_t* pos_rows, const int32_t* base_rows, int R, int H_I,
+                                int d_I, int64_t ld, float* out)
+{
+    e4m3_init();
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int r = 0; r < R; ++r)
+        oracle_indexer_row(q_rows + (size_t)r * H_I * d_I, w_rows + (size_t)r * H_I, keys,
+                           base_rows[r], (int64_t)pos_rows[r] + 1, H_I, d_I, out + (size_t)r * ld);
+}

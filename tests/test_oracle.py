@@ -93,6 +93,22 @@ def test_indexer_int64_brute_force_tiny():
         assert (got.astype(np.int64) == want).all() and (got == want).all()
 
 
+def test_indexer_scores_rows_int64_brute_force_packed():
+    """The many-rows form (rows in parallel, ragged pos, packed k_base) equals
+    integer brute force row by row and leaves NaN past each row's pos."""
+    x = synth.decode_inputs("decode", seed=4, B=4, ctx=[1, 60, 300, 129],
+                            overrides=dict(H_I=4, d_I=32, indexer="int", k=16))
+    q_idx, k_idx, w = x.q_idx.numpy(), x.k_idx.numpy(), x.w.numpy()
+    pos, base = x.pos.numpy(), x.k_base.numpy()
+    got = oracle.indexer_scores_rows(q_idx, w, k_idx, pos, base)
+    assert got.shape == (4, int(pos.max()) + 1)
+    for b in range(4):
+        n = int(pos[b]) + 1
+        want = _brute_int64(q_idx, w, k_idx[base[b]:], b, n)
+        assert (got[b, :n] == want).all()
+        assert np.isnan(got[b, n:]).all()
+
+
 def test_indexer_relu_identity():
     """ReLU(x) - ReLU(-x) = x: negating head j changes I by exactly w_j (q_j . k)."""
     x = synth.prefill_inputs("tiny", seed=5)
