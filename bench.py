@@ -64,6 +64,9 @@ def parse():
     ap.add_argument("--mha", nargs="?", const="mha_short", default=None,
                     help="time MLA MHA-mode dense causal attention (short prefill, default "
                          "mha_short: 2048 tokens, 128 heads, d_h 192, d_hv 128) instead of the default step")
+    ap.add_argument("--replicas", action="store_true",
+                    help="with several ranks, run the whole workload on every rank (weak scaling) "
+                         "instead of splitting its query rows and sequences between them")
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -103,6 +106,42 @@ def max_over_ranks(world, x: float) -> float:
     t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def shard_prefill_rows(world: int, rank: int, T: int, S: int, k: int, H_I: int, d_I: int, Hq: int,
+                       d_qk: int, d_v: int):
+    """This rank's query rows [t0, t1) of one causal prefill: contiguous ranges of
+    equal modelled work from the library's partition (host-only call)."""
+    import sparse_attention_20_b200 as dsa
+    b = dsa.partition_prefill_rows(T, S, k, H_I, d_I, Hq, d_qk, d_v, world)
+    return b[rank], b[rank + 1]
+
+
+def shard_decode_seqs(world: int, rank: int, ctx, k: int, d_I: int, d_qk: int):
+    """This rank's decode sequences [b0, b1) (contiguous, equal modelled bytes)."""
+    import sparse_attention_20_b200 as dsa
+    b = dsa.partition_decode_seqs(ctx, k, d_I, d_qk, world)
+    return b[rank], b[rank + 1]
+
+
+def shard_inputs(x, world: int, rank: int):
+    """The part of batch x this rank runs. A causal prefill (pos / k_base NULL)
+    keeps rows [t0, t1) as the tail prefill of its first t1 + S - T tokens (the
+    row slices of q_idx, w, q and a prefix of the caches); a decode batch keeps
+    sequences [b0, b1) with their pos / k_base over the whole caches."""
+    import synth
+    H_I, d_I = x.q_idx.shape[1], x.q_idx.shape[2]
+    Hq, d_qk = x.q.shape[1], x.q.shape[2]
+    if x.pos is None and x.k_base is None:
+        t0, t1 = shard_prefill_rows(world, rank, x.T, x.S, x.k, H_I, d_I, Hq, d_qk, x.d_v)
+        s1 = t1 + x.S - x.T
+        return synth.DSAInputs(x.config, x.q_idx[t0:t1], x.w[t0:t1], x.k_idx[:s1], x.q[t0:t1], x.kv[:s1],
+                               None, None, x.k, x.scale, x.d_v, dict(x.meta, rows=(t0, t1)))
+    ctx = (x.positions() + 1).cpu().tolist()
+    b0, b1 = shard_decode_seqs(world, rank, ctx, x.k, d_I, d_qk)
+    return synth.DSAInputs(x.config, x.q_idx[b0:b1], x.w[b0:b1], x.k_idx, x.q[b0:b1], x.kv,
+                           x.positions()[b0:b1], x.bases()[b0:b1], x.k, x.scale, x.d_v,
+                           dict(x.meta, rows=(b0, b1)))
 
 
 def job_throughput(world: int, units_per_rank: int, ms_max: float) -> float:
@@ -197,6 +236,11 @@ def prefill_kw(args):
     return kw
 
 
+def sharded(args, world) -> bool:
+    """Several ranks split one workload (strong scaling) unless --replicas."""
+    return world > 1 and not getattr(args, "replicas", False)
+
+
 def workload_config(args, xp, world):
     """The `config` of the JSON line, the same for both arms."""
     H_I, d_I = xp.q_idx.shape[1], xp.q_idx.shape[2]
@@ -209,7 +253,9 @@ def workload_config(args, xp, world):
     rows = f"L={xp.T}" if xp.T == xp.S else f"last {xp.T} of L={xp.S}"
     return {"workload": f"{args.prefill} causal prefill ({rows}, H_I={H_I}, d_I={d_I}, k={xp.k}, "
                         f"Hq={Hq}, d_qk={d_qk}, d_v={xp.d_v}) + {args.decode} step ({decode})",
-            "global_batch": world, "seq_len": xp.T, "parallelism": f"replicas{world}",
+            "global_batch": 1 if sharded(args, world) else world, "seq_len": xp.T,
+            "parallelism": (f"rows{world} (query rows and decode sequences split, no exchange)"
+                            if sharded(args, world) else f"replicas{world}"),
             "l2": f"inputs larger than L2: {xp.T * Hq * d_qk * 2 / 1e9:.1f} GB of queries, "
                   f"{xp.S * d_qk * 2 / 1e6:.0f} MB latent cache (L2 126 MB)"}
 
@@ -274,10 +320,10 @@ def profiled_traffic(profile: str, key: str, sources) -> float | None:
 def attn_traffic():
     """DRAM bytes per prefill attention launch (128K workload)."""
     return profiled_traffic("dram_bench_prefill128k_decode64.md", "attn",
-                            ("attn_tc.cuh", "sm100.cuh", "common.cuh"))
+                            ("attn_tc.cuh", "sm100.cuh", "common.cuh", "dsa.cu"))
 
 
-MHA_SOURCES = ("mha_attn.cuh", "attn_bwd.cuh", "sm100.cuh", "common.cuh")
+MHA_SOURCES = ("mha_attn.cuh", "attn_bwd.cuh", "sm100.cuh", "common.cuh", "dsa.cu")
 
 
 def fp8_gemm_tflops(n=8192, reps=10):
@@ -366,8 +412,15 @@ def bench_ours(args, world, rank, local):
     barrier(world)
     dsa.load_library()
     dev = torch.device("cuda", torch.cuda.current_device())
-    xp = synth.make_inputs(args.prefill, device=dev, seed=args.seed + rank, **prefill_kw(args))
-    xd = synth.make_inputs(args.decode, device=dev, seed=args.seed + rank)
+    split = sharded(args, world)
+    # split: every rank draws the same workload and runs its part of it;
+    # replicas: every rank runs a whole workload of its own
+    seed = args.seed if split else args.seed + rank
+    xp = synth.make_inputs(args.prefill, device=dev, seed=seed, **prefill_kw(args))
+    xd = synth.make_inputs(args.decode, device=dev, seed=seed)
+    xp_full, xd_full = xp, xd
+    if split:
+        xp, xd = shard_inputs(xp, world, rank), shard_inputs(xd, world, rank)
     bp, bd = Batch(xp, dsa), Batch(xd, dsa)
     if args.decode_page_size:
         ps = args.decode_page_size
@@ -416,36 +469,40 @@ def bench_ours(args, world, rank, local):
     ms_step = total_ms / args.steps
     prefill_ms = p_idx + p_attn
     decode_ms = d_idx + d_attn
-    tokens = world * xp.T   # every rank runs the same workload (weak scaling)
+    # whole-job units: the full workload once (split) or once per rank (replicas)
+    tokens = xp_full.T if split else world * xp.T
+    seqs = xd_full.T if split else world * xd.T
     peaks = measured_peaks()
     wp, wd = bp.work, bd.work
     attn_tflops = wp["attn_flops"] / (p_attn * 1e-3) / 1e12
-    # FP8: measured burst here, scaled like bf16 from burst to sustained (the
-    # indexer runs inside a long step); else 2 x bf16 sustained (nominal ratio)
+    # Denominators: each kernel is one launch of tens of milliseconds at most,
+    # timed on its own, so its peak is the burst figure (bf16 from
+    # MEASURED_PEAKS.json; FP8 measured here by a cuBLAS GEMM, else 2 x bf16
+    # burst, the nominal ratio). The sustained figures are reported beside them.
     fp8_burst = fp8_gemm_tflops()
     if fp8_burst:
-        fp8_peak = fp8_burst * peaks["bf16_sustained"] / peaks["bf16"]
-        fp8_source = (f"measured FP8 GEMM {fp8_burst:.0f} TF/s burst x bf16 sustained/burst "
-                      f"({peaks['source']} bf16)")
+        fp8_peak = fp8_burst
+        fp8_source = f"measured FP8 GEMM burst (cuBLAS e4m3 8192^3, this run)"
     else:
-        fp8_peak = 2.0 * peaks["bf16_sustained"]
-        fp8_source = "2 x measured bf16 sustained (fp8 ratio)"
+        fp8_peak = 2.0 * peaks["bf16"]
+        fp8_source = f"2 x {peaks['source']} bf16 burst (nominal FP8 ratio)"
+    fp8_sustained = fp8_peak * peaks["bf16_sustained"] / peaks["bf16"]
     result = {
         "metric": METRIC,
-        "value": job_throughput(world, xp.T, ms_step),
+        "value": tokens / (ms_step * 1e-3),
         "unit": "tokens/s",
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
         "ms_per_step": ms_step,
         "higher_is_better": True,
-        "scaling": "weak",
+        "scaling": "strong" if split else "weak",
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded; shapes and distributions of the pages' 128K workloads)",
-        "config": workload_config(args, xp, world),
+        "config": workload_config(args, xp_full, world),
         "prefill_tokens_per_s": tokens / (prefill_ms * 1e-3),
-        "decode": {"value": world * xd.T / (decode_ms * 1e-3), "unit": "seqs/s",
+        "decode": {"value": seqs / (decode_ms * 1e-3), "unit": "seqs/s",
                    "ms_per_step": decode_ms,
                    "hbm_gbs": (wd["idx_bytes"] + wd["attn_bytes"]) / (decode_ms * 1e-3) / 1e9,
                    "hbm_frac": (wd["idx_bytes"] + wd["attn_bytes"]) / (decode_ms * 1e-3) / 1e9
@@ -453,32 +510,65 @@ def bench_ours(args, world, rank, local):
         "kernels_ms": {"prefill_indexer_topk": p_idx, "prefill_sparse_attn": p_attn,
                        "decode_indexer_topk": d_idx, "decode_sparse_attn": d_attn},
         "roofline": {"bound": "tensor", "kernel": "prefill sparse MLA attention",
-                     "achieved": attn_tflops, "peak": peaks["bf16_sustained"],
-                     "unit": "TFLOP/s", "frac": attn_tflops / peaks["bf16_sustained"],
+                     "achieved": attn_tflops, "peak": peaks["bf16"],
+                     "unit": "TFLOP/s", "frac": attn_tflops / peaks["bf16"],
                      "traffic": attn_traffic() if xp.config == "prefill128k" and xp.T == 131072
                      else None,
-                     "peak_source": f"{peaks['source']} bf16 sustained"},
+                     "peak_source": f"{peaks['source']} bf16 burst",
+                     "frac_of_sustained": attn_tflops / peaks["bf16_sustained"]},
         "rooflines": {
             "prefill_indexer_topk": {"bound": "tensor", "unit": "TFLOP/s",
                                      "achieved": wp["idx_flops"] / (p_idx * 1e-3) / 1e12,
                                      "peak": fp8_peak,
                                      "frac": wp["idx_flops"] / (p_idx * 1e-3) / 1e12 / fp8_peak,
-                                     "peak_source": fp8_source},
+                                     "peak_source": fp8_source,
+                                     "frac_of_sustained": wp["idx_flops"] / (p_idx * 1e-3) / 1e12
+                                     / fp8_sustained},
             "decode_step": {"bound": "hbm", "unit": "GB/s",
                             "achieved": (wd["idx_bytes"] + wd["attn_bytes"]) / (decode_ms * 1e-3)
-                            / 1e9, "peak": peaks["hbm"]},
+                            / 1e9, "peak": peaks["hbm"],
+                            "frac": (wd["idx_bytes"] + wd["attn_bytes"]) / (decode_ms * 1e-3) / 1e9
+                            / peaks["hbm"], "peak_source": f"{peaks['source']} HBM copy"},
         },
         "gpu_launches": launches,
         "clocks": clk,
     }
+    result["topk"] = topk_phases(dsa, bp, bd, stream)
+    if split:
+        result["shard"] = {"prefill_rows": list(xp.meta["rows"]), "decode_seqs": list(xd.meta["rows"]),
+                           "rank": rank}
     if not args.no_e2e:
-        result["e2e"] = bench_e2e(args, world, dsa, bp, bd, stream)
+        result["e2e"] = bench_e2e(args, world, dsa, bp, bd, stream, tokens)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(xp, seed=args.seed)
     return result
 
 
-def bench_e2e(args, world, dsa, bp, bd, stream):
+def topk_phases(dsa, bp, bd, stream):
+    """The indexer's phases timed on their own (one extra step after the timed
+    region, CUDA events around each phase inside the library): the Top-k
+    selection alone, reported as GB/s over its candidate traffic. Candidate
+    bytes per row that needs a selection (n > k): the threshold keeps about
+    2k (score, s) pairs of 8 bytes (all n when n <= 2k), read once, plus the
+    k int32 indices written."""
+    out = {}
+    for name, b in (("prefill", bp), ("decode", bd)):
+        dsa.phase_timing(True)
+        run_indexer(dsa, b, stream)
+        torch.cuda.synchronize()
+        ph = dsa.phase_times()
+        dsa.phase_timing(False)
+        n = b.x.positions().cpu().long() + 1
+        k = b.x.k
+        sel = n > k
+        cand_bytes = float((torch.clamp(n[sel], max=2 * k) * 8).sum().item() + int(sel.sum().item()) * k * 4)
+        out[name] = {"scores_ms": ph["scores"], "threshold_ms": ph["threshold"], "select_ms": ph["select"],
+                     "select_candidate_bytes": cand_bytes,
+                     "select_gbs": cand_bytes / (ph["select"] * 1e-3) / 1e9 if ph["select"] > 0 else None}
+    return out
+
+
+def bench_e2e(args, world, dsa, bp, bd, stream, tokens):
     """Same step through the C ABI with inputs in pinned host memory: every step
     copies its inputs host->device and reads idx/out/lse back."""
     def host(t):
@@ -520,7 +610,7 @@ def bench_e2e(args, world, dsa, bp, bd, stream):
     end.record(stream)
     torch.cuda.synchronize()
     ms = max_over_ranks(world, start.elapsed_time(end)) / args.e2e_steps
-    return {"value": world * bp.T / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
+    return {"value": tokens / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "pinned": all(h.is_pinned() for h, _ in pairs_in + pairs_out)}
 
@@ -624,9 +714,10 @@ def bench_varlen(args, world, rank, local):
                    "parallelism": f"replicas{world}"},
         "kernels_ms": {"indexer_topk_varlen": t_idx, "sparse_attn": t_attn},
         "roofline": {"bound": "tensor", "kernel": "sparse MLA attention", "achieved": attn_tf,
-                     "peak": peaks["bf16_sustained"], "unit": "TFLOP/s",
-                     "frac": attn_tf / peaks["bf16_sustained"], "traffic": None,
-                     "peak_source": f"{peaks['source']} bf16 sustained"},
+                     "peak": peaks["bf16"], "unit": "TFLOP/s",
+                     "frac": attn_tf / peaks["bf16"], "traffic": None,
+                     "peak_source": f"{peaks['source']} bf16 burst",
+                     "frac_of_sustained": attn_tf / peaks["bf16_sustained"]},
         "indexer_tflops": work["idx_flops"] / (t_idx * 1e-3) / 1e12,
         "gpu_launches": launches, "clocks": clk,
     }
@@ -695,9 +786,10 @@ def bench_bwd(args, world, rank, local):
                                f"d_qk={d_qk}, d_v={d_v}; inputs larger than L2, no flush",
                    "global_batch": world, "seq_len": x.T, "parallelism": f"replicas{world}"},
         "roofline": {"bound": "tensor", "kernel": "attention backward (dkv + dq kernels, one call)",
-                     "achieved": tf, "peak": peaks["bf16_sustained"], "unit": "TFLOP/s",
-                     "frac": tf / peaks["bf16_sustained"], "traffic": None,
-                     "peak_source": f"{peaks['source']} bf16 sustained"},
+                     "achieved": tf, "peak": peaks["bf16"], "unit": "TFLOP/s",
+                     "frac": tf / peaks["bf16"], "traffic": None,
+                     "peak_source": f"{peaks['source']} bf16 burst",
+                     "frac_of_sustained": tf / peaks["bf16_sustained"]},
         "gpu_launches": launches, "clocks": clk,
     }
     if rank == 0 and not args.no_cpu_baseline:
@@ -777,9 +869,10 @@ def bench_kl(args, world, rank, local):
                                f"H_I={H_I}, d_I={d_I}; inputs larger than L2, no flush",
                    "global_batch": world, "seq_len": x.T, "parallelism": f"replicas{world}"},
         "roofline": {"bound": "tensor", "kernel": "head-summed attention probabilities + per-row loss (one call)",
-                     "achieved": tf, "peak": peaks["bf16_sustained"], "unit": "TFLOP/s",
-                     "frac": tf / peaks["bf16_sustained"], "traffic": None,
-                     "peak_source": f"{peaks['source']} bf16 sustained"},
+                     "achieved": tf, "peak": peaks["bf16"], "unit": "TFLOP/s",
+                     "frac": tf / peaks["bf16"], "traffic": None,
+                     "peak_source": f"{peaks['source']} bf16 burst",
+                     "frac_of_sustained": tf / peaks["bf16_sustained"]},
         "mean_loss": float(res[0].mean().item()),
         "gpu_launches": launches, "clocks": clk,
     }
@@ -849,10 +942,11 @@ def bench_mha(args, world, rank, local):
                                f"inputs larger than L2, no flush",
                    "global_batch": world, "seq_len": S, "parallelism": f"replicas{world}"},
         "roofline": {"bound": "tensor", "kernel": "mha_causal_kernel", "achieved": tf,
-                     "peak": peaks["bf16_sustained"], "unit": "TFLOP/s", "frac": tf / peaks["bf16_sustained"],
+                     "peak": peaks["bf16"], "unit": "TFLOP/s", "frac": tf / peaks["bf16"],
+                     "frac_of_sustained": tf / peaks["bf16_sustained"],
                      "traffic": (profiled_traffic("mha_causal_short_prefill2k.md", "mha", MHA_SOURCES)
                                  if args.mha == "mha_short" and args.seq_len is None else None),
-                     "peak_source": f"{peaks['source']} bf16 sustained"},
+                     "peak_source": f"{peaks['source']} bf16 burst"},
         "gpu_launches": launches, "clocks": clk,
     }
     if rank == 0 and not args.no_cpu_baseline:

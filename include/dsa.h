@@ -48,7 +48,8 @@ typedef enum {
     DSA_ERR_UNSUPPORTED = -2, /* a dimension outside the supported set (below) */
     DSA_ERR_CUDA = -3,        /* a CUDA runtime error at launch (or an earlier asynchronous one) */
     DSA_ERR_TIMEOUT = -4,     /* a kernel gave up a bounded wait (see dsa_device_status) */
-    DSA_ERR_WORKSPACE = -5    /* workspace NULL or smaller than dsa_workspace_size() */
+    DSA_ERR_WORKSPACE = -5,   /* workspace NULL or smaller than dsa_workspace_size() */
+    DSA_ERR_CHECK = -6        /* debug build only: a device check counted invalid index-set entries */
 } dsa_status;
 
 /*
@@ -162,6 +163,30 @@ int dsa_sparse_mla_attn(const void* q, const void* kv, const int32_t* idx, const
                         const int32_t* k_base, int T, int S, int Hq, int d_qk, int d_v, int k,
                         float scale, void* out, float* lse, void* workspace, size_t ws_bytes,
                         void* stream);
+
+/*
+ * dsa_sparse_mla_attn with the number of parts each row's selected set is
+ * split into chosen by the caller (the decode form: one query token per
+ * sequence, so few rows must fill the GPU). The row's valid entries are cut
+ * into `splits` contiguous ranges of whole 64-entry chunks; each range is
+ * attended by its own CTAs, which write the part's output normalised by its
+ * own softmax sum and its log-sum-exp, and a merge kernel combines the parts:
+ *   lse = log sum_z exp(lse_z),   out = sum_z exp(lse_z - lse) out_z
+ * (the split of the selected set across CTAs with a log-sum-exp merge:
+ * "DeepSeek-V3.2: Pushing the Frontier of Open Large Language Models",
+ * "2.3 Inference Costs"). splits = 0 is the library's own choice (what
+ * dsa_sparse_mla_attn uses: parts only where they add no wave of work);
+ * 1..16 forces that many (a part may be empty). The result equals the
+ * unsplit one up to fp32 rounding of the merge.
+ * workspace: dsa_sparse_mla_attn_split_workspace_size(T, Hq, d_v, splits)
+ * bytes (0 for splits = 1; for splits = 0 use dsa_workspace_size).
+ * Other arguments and limits as dsa_sparse_mla_attn; DSA_ERR_ARG for splits
+ * outside 0..16.
+ */
+size_t dsa_sparse_mla_attn_split_workspace_size(int T, int Hq, int d_v, int splits);
+int dsa_sparse_mla_attn_split(const void* q, const void* kv, const int32_t* idx, const int32_t* pos,
+                              const int32_t* k_base, int T, int S, int Hq, int d_qk, int d_v, int k, float scale,
+                              int splits, void* out, float* lse, void* workspace, size_t ws_bytes, void* stream);
 
 /*
  * Backward of dsa_sparse_mla_attn: the gradients through the selected latent
@@ -286,11 +311,78 @@ int dsa_indexer_topk_noalloc(const void* q_idx, const float* w, const void* k_id
                              int d_I, int k, int32_t* idx, void* stream);
 
 /*
+ * Multi-GPU partition (host-only; no device memory, no launch). The path
+ * shards with no exchange between ranks: query rows of one causal prefill
+ * are independent once every rank holds the key and latent caches, and
+ * decode sequences are independent altogether. These functions give rank r
+ * the contiguous range [bounds[r], bounds[r+1]) with about equal modelled
+ * work (bounds: caller-owned HOST int32 [parts + 1]; bounds[0] = 0,
+ * bounds[parts] = the item count; a range may be empty when parts exceeds
+ * the items).
+ *
+ * dsa_partition_prefill_rows: the T query rows of one causal sequence of S
+ * tokens (row t at position t + S - T). Row cost: when it has n > k
+ * candidates, the indexer's n (row, key) pairs at 2 H_I d_I FP8 flop each,
+ * counted at half weight (FP8 runs at twice the BF16 rate; rows with n <= k
+ * need no scores), plus min(n, k) selected rows at 2 Hq (d_qk + d_v) BF16
+ * flop each. The causal cost grows with t (the indexer's O(L^2) term: "Paper
+ * Breakdown: DeepSeek-V3.2", "Efficiency (Fig 3)"), so the ranges shrink
+ * toward the end of the sequence. A rank runs its rows [t0, t1) as the tail
+ * prefill of the first t1 + S - T tokens: dsa_forward with T' = t1 - t0,
+ * S' = t1 + S - T, pos = k_base = NULL and the row slices of q_idx, w, q, idx,
+ * out and lse; the results equal the one-call results bit for bit.
+ *
+ * dsa_partition_decode_seqs: n_seqs decode sequences with context lengths
+ * ctx (HOST int32 [n_seqs]); cost = ctx d_I key bytes + min(ctx, k) 2 d_qk
+ * gathered bytes.
+ *
+ * DSA_ERR_ARG for NULL pointers or sizes out of range (T <= 0, S < T,
+ * parts <= 0, a negative ctx).
+ */
+int dsa_partition_prefill_rows(int T, int S, int k, int H_I, int d_I, int Hq, int d_qk, int d_v, int parts,
+                               int32_t* bounds);
+int dsa_partition_decode_seqs(const int32_t* ctx, int n_seqs, int k, int d_I, int d_qk, int parts,
+                              int32_t* bounds);
+
+/*
  * Waits for `stream`, then returns and clears the device status word:
  * DSA_OK, DSA_ERR_TIMEOUT (a kernel gave up a bounded wait) or DSA_ERR_CUDA
  * (an asynchronous CUDA error; its text is in dsa_last_error()).
  */
 int dsa_device_status(void* stream);
+
+/*
+ * Debug build. libdsa_debug.so is the same library compiled with -DDSA_DEBUG
+ * (no counterpart in the method: a stand-in for an external memory checker).
+ * Every entry point that produces or reads an index set then also validates
+ * it on the device, per row t with n = pos[t] + 1 candidates and m =
+ * min(k, n) entries read, and counts (never traps):
+ *   [0] entries in [0, m) greater than pos[t]   (ignored by the attention)
+ *   [1] entries in [0, m) below 0               (ignored by the attention)
+ *   [2] valid entries at or past m              (not read by the attention)
+ *   [3] repeated valid entries in [0, m)
+ *   [4] valid entries whose block-table page is outside the pool (paged calls)
+ *   [5] selector results that are not min(k, n) distinct valid entries then -1
+ * A call that counts any sets the status word to DSA_ERR_CHECK
+ * (dsa_device_status). dsa_debug_build() is 1 in that build, 0 otherwise;
+ * dsa_debug_counters copies the first n (<= 6) totals to HOST memory after a
+ * device synchronisation and, with reset != 0, clears them. The release build
+ * counts nothing (all totals stay 0).
+ */
+int dsa_debug_build(void);
+int dsa_debug_counters(uint64_t* out, int n, int reset);
+
+/*
+ * Phase timing (a diagnostic, no counterpart in the method). With
+ * dsa_phase_timing(1), every indexer call brackets each of its phases with a
+ * pair of CUDA events on its stream: [0] the scores (the sampled and filter
+ * scans, or the chunk passes), [1] the threshold (the sampled tau), [2] the
+ * Top-k selection (the select or merge kernels). dsa_phase_times copies the
+ * first n (<= 3) sums in milliseconds to HOST memory, waiting for the events,
+ * and starts new sums. Off by default; when off nothing is recorded.
+ */
+int dsa_phase_timing(int enable);
+int dsa_phase_times(double* ms, int n);
 
 /* Text of the last error on the calling thread ("" when none). */
 const char* dsa_last_error(void);

@@ -41,27 +41,35 @@ def _sources():
                   + glob.glob(os.path.join(INCLUDE, "*.h")))
 
 
-def stale() -> bool:
-    if not os.path.exists(LIB):
+# The debug build: the same source with the device-side index-set checks
+# (csrc/debug_checks.cuh) compiled in.
+DEBUG_LIB = os.path.join(PKG, "libdsa_debug.so")
+
+
+def stale(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return any(os.path.getmtime(s) > t for s in _sources())
 
 
-def build(force: bool = False, verbose: bool = False, extra_flags=()) -> str:
-    if not force and not stale():
-        return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc(), *NVCC_FLAGS, *extra_flags, "-I", INCLUDE, "-I", CSRC,
+def build(force: bool = False, verbose: bool = False, extra_flags=(), debug: bool = False) -> str:
+    """Compile libdsa.so (or, with debug=True, libdsa_debug.so with -DDSA_DEBUG)
+    when a source is newer than it; returns its path."""
+    lib = DEBUG_LIB if debug else LIB
+    if not force and not stale(lib):
+        return lib
+    tmp = lib + f".tmp{os.getpid()}"
+    cmd = [nvcc(), *NVCC_FLAGS, *(["-DDSA_DEBUG"] if debug else []), *extra_flags, "-I", INCLUDE, "-I", CSRC,
            os.path.join(CSRC, "dsa.cu"), "-o", tmp]
     if verbose:
         print(" ".join(cmd), flush=True)
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
     force = "--force" in sys.argv
     extra = ["-Xptxas", "-v"] if "--ptxas-v" in sys.argv else []
-    print(build(force=force or bool(extra), verbose=True, extra_flags=extra))
+    print(build(force=force or bool(extra), verbose=True, extra_flags=extra, debug="--debug" in sys.argv))

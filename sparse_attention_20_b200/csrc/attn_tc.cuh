@@ -19,6 +19,14 @@
 // gathered rows read MN-major, N = 256). No flop is done twice and every
 // selected row crosses HBM/L2 once per query.
 //
+// Decode variant (few rows): the selected set of a row can be split across
+// `splits` clusters, each taking a contiguous range of the row's chunks; a
+// cluster then writes its partial output normalised by its own softmax sum
+// (fp32) and its log-sum-exp, and lse_merge_kernel combines the parts
+// ("DeepSeek-V3.2: Pushing the Frontier of Open Large Language Models",
+// section "2.3 Inference Costs": decoding reads the cache, so the work of one
+// query token is spread over more SMs).
+//
 // Warp roles (512 threads per CTA): warp 0 allocates TMEM and issues the QK
 // and PV MMAs (one thread polling both kinds of readiness, so a late chunk
 // never holds back the PV of the previous one); warps 1-3 load Q (TMA tiles)
@@ -133,7 +141,8 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
                           const __nv_bfloat16* __restrict__ kv,
                           const int* __restrict__ idx, const int* __restrict__ pos,
                           const int* __restrict__ k_base, int T, int S, int k, float scale_log2,
-                          __nv_bfloat16* __restrict__ out, float* __restrict__ lse, const PagedRows pg)
+                          __nv_bfloat16* __restrict__ out, float* __restrict__ lse, const PagedRows pg,
+                          int splits, float* __restrict__ part_o, float* __restrict__ part_lse)
 {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -147,12 +156,21 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();
     const uint32_t peer = rank ^ 1u;
-    const int t = T - 1 - (int)(blockIdx.x >> 1);   // long rows first
+    griddep_wait();
+    const int cid = (int)(blockIdx.x >> 1);
+    const int t = T - 1 - cid / splits;             // long rows first
+    const int part = cid % splits;
     long long base;
     const int* bt;   // block-table line of a paged cache, else NULL
     const int n_cand = row_keys(pg, pos, k_base, t, T, S, &base, &bt);
     const int p_last = n_cand - 1;
-    const int n_row = min(k, n_cand);
+    // this cluster's entries of the row: chunks [c0, c1) of its ceil(n/64)
+    const int n_all = min(k, n_cand);
+    const int nc_all = ceil_div(n_all, kKeys);
+    const int c0 = (int)((long long)nc_all * part / splits);
+    const int c1 = (int)((long long)nc_all * (part + 1) / splits);
+    const int e0 = c0 * kKeys;
+    const int n_row = max(0, min(c1 * kKeys, n_all) - e0);
     const int NC = ceil_div(n_row, kKeys);
 
     if (threadIdx.x == 0) {
@@ -283,7 +301,7 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
                 tma_load_2d(qs + j * kQSlab, &tm_q128, (int)rank * 256 + 128 + j * 64, t * kHeads, bar(B_Q));
             tma_load_2d(qs + 2 * kQSlab, &tm_q64, 512 + (int)rank * 32, t * kHeads, bar(B_Q));
         }
-        const int* idx_row = idx + (size_t)t * k;
+        const int* idx_row = idx + (size_t)t * k + e0;
         uint32_t* smask = reinterpret_cast<uint32_t*>(sgen + kOffMask);
         long long* rows_tab = reinterpret_cast<long long*>(sgen + kOffRows) + gw * kKeys;
         int r_q[3];
@@ -538,8 +556,11 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
             ok = wait_w(bar(B_LSUM), 0, 200 + B_LSUM, 0);
             if (ok) l += lsum_s[(hs ^ 1) * kHeads + i];
         }
-        // epilogue: O / l -> bf16, columns [128hs, 128hs+128) of this CTA's half
+        // epilogue: O / l -> bf16 (or, for a part of a split row, fp32 into
+        // the parts buffer), columns [128hs, 128hs+128) of this CTA's half
+        const size_t prow = ((size_t)t * splits + part) * kHeads + i;   // parts layout [T, splits, 128]
         __nv_bfloat16* orow = out + ((size_t)t * kHeads + i) * kDv + rank * 256 + 128 * hs;
+        float* porow = splits > 1 ? part_o + prow * kDv + rank * 256 + 128 * hs : nullptr;
         if (ok && NC > 0) {
             const int c = NC - 1;
             ok = wait_w(bar(B_PVDONE + (c & 1)), (c >> 1) & 1, 300 + B_PVDONE, c);
@@ -551,6 +572,15 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
                     uint32_t o[32];
                     tmem_ld32(tmem + lane_addr + kColO + 128 * hs + q4 * 32, o);
                     tmem_wait_ld();
+                    if (porow) {
+                        float4* dst = reinterpret_cast<float4*>(porow + q4 * 32);
+#pragma unroll
+                        for (int v = 0; v < 8; ++v)
+                            dst[v] = make_float4(__uint_as_float(o[4 * v]) * inv, __uint_as_float(o[4 * v + 1]) * inv,
+                                                 __uint_as_float(o[4 * v + 2]) * inv,
+                                                 __uint_as_float(o[4 * v + 3]) * inv);
+                        continue;
+                    }
                     uint32_t w[16];
 #pragma unroll
                     for (int e = 0; e < 16; ++e)
@@ -563,11 +593,21 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
                 }
             }
         } else if (NC == 0) {
-            uint4* dst = reinterpret_cast<uint4*>(orow);
-            for (int v = 0; v < 16; ++v) dst[v] = make_uint4(0u, 0u, 0u, 0u);
+            if (porow) {
+                float4* dst = reinterpret_cast<float4*>(porow);
+                for (int v = 0; v < 32; ++v) dst[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+            } else {
+                uint4* dst = reinterpret_cast<uint4*>(orow);
+                for (int v = 0; v < 16; ++v) dst[v] = make_uint4(0u, 0u, 0u, 0u);
+            }
         }
-        if (rank == 0 && hs == 0 && (ok || NC == 0))
-            lse[(size_t)t * kHeads + i] = l > 0.f ? (m_use + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+        if (rank == 0 && hs == 0 && (ok || NC == 0)) {
+            const float lv = l > 0.f ? (m_use + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+            if (splits > 1)
+                part_lse[prow] = lv;
+            else
+                lse[(size_t)t * kHeads + i] = lv;
+        }
     }
 
     if (warp == 0 && lane == 0 && NC > 0) {
@@ -583,6 +623,61 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
     if (warp == 0) tmem_dealloc(tmem, kTmemCols);
     cluster_sync();   // no CTA leaves while its peer may still touch its shared memory
 }
+
+// Log-sum-exp merge of a split row's parts (decode variant): for row t and
+// head h, with parts z of (o_z normalised by its own softmax sum, lse_z),
+//   lse = log sum_z exp(lse_z),  out = sum_z exp(lse_z - lse) o_z.
+// One CTA of 128 threads per (row, 8 heads); each thread owns four
+// consecutive columns of one head at a time (float4 loads of every part).
+constexpr int kMergeHeads = 8;
+
+__global__ void __launch_bounds__(128)
+lse_merge_kernel(const float* __restrict__ part_o, const float* __restrict__ part_lse, int T, int splits,
+                 __nv_bfloat16* __restrict__ out, float* __restrict__ lse)
+{
+    __shared__ float wz[kMergeHeads][16];
+    griddep_wait();
+    const int t = blockIdx.x;
+    const int h0 = blockIdx.y * kMergeHeads;
+    if (threadIdx.x < kMergeHeads) {
+        const int h = h0 + threadIdx.x;
+        float m = -INFINITY;
+        for (int z = 0; z < splits; ++z) m = fmaxf(m, part_lse[((size_t)t * splits + z) * kHeads + h]);
+        float total = -INFINITY;
+        if (m != -INFINITY) {
+            float l = 0.f;
+            for (int z = 0; z < splits; ++z) l += expf(part_lse[((size_t)t * splits + z) * kHeads + h] - m);
+            total = m + logf(l);
+        }
+        for (int z = 0; z < splits; ++z) {
+            const float lz = part_lse[((size_t)t * splits + z) * kHeads + h];
+            wz[threadIdx.x][z] = (total == -INFINITY || lz == -INFINITY) ? 0.f : expf(lz - total);
+        }
+        lse[(size_t)t * kHeads + h] = total;
+    }
+    __syncthreads();
+    // 8 heads x 512 columns = 1024 float4 groups, 8 per thread
+    for (int e = threadIdx.x; e < kMergeHeads * kDv / 4; e += 128) {
+        const int hh = e / (kDv / 4), c4 = e % (kDv / 4);
+        const int h = h0 + hh;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int z = 0; z < splits; ++z) {
+            const float wgt = wz[hh][z];
+            const float4 v = reinterpret_cast<const float4*>(
+                part_o + (((size_t)t * splits + z) * kHeads + h) * kDv)[c4];
+            acc.x = fmaf(wgt, v.x, acc.x);
+            acc.y = fmaf(wgt, v.y, acc.y);
+            acc.z = fmaf(wgt, v.z, acc.z);
+            acc.w = fmaf(wgt, v.w, acc.w);
+        }
+        uint2 pk = make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
+        reinterpret_cast<uint2*>(out + ((size_t)t * kHeads + h) * kDv)[c4] = pk;
+    }
+}
+
+// Most parts a row is split into (the merge keeps one weight per part in
+// shared memory).
+constexpr int kMaxSplits = 16;
 
 }  // namespace attn_tc
 }  // namespace dsa

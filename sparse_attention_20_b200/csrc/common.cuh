@@ -64,6 +64,13 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 
 __host__ __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start while the previous kernel on its stream is still
+// running; it waits here, before its first read of global memory, until that
+// kernel has completed and its writes are visible. (A no-op for a kernel
+// launched without the attribute.)
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // Candidate range of query row t: s = 0..n-1 at cache rows base + s. Rows that
 // would reach outside the cache (a caller error) are clipped to it, so no
 // kernel ever reads out of bounds.

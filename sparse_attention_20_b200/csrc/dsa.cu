@@ -11,12 +11,14 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "dsa.h"
 #include "attn_bwd.cuh"
 #include "attn_simple.cuh"
 #include "attn_tc.cuh"
 #include "common.cuh"
+#include "debug_checks.cuh"
 #include "indexer_chunked.cuh"
 #include "indexer_kl.cuh"
 #include "indexer_scores.cuh"
@@ -95,6 +97,87 @@ EncodeTiledFn encode_tiled()
         if (e_ != cudaSuccess) return cuda_fail(e_, where);          \
     } while (0)
 
+// Debug build (-DDSA_DEBUG): validate an index set on the device (counts
+// violations, never traps; debug_checks.cuh). `selector`: the set is a
+// selector result. The release build launches nothing here.
+int debug_check(const int32_t* idx, const int32_t* pos, const int32_t* k_base, int T, int S, int k,
+                const dsa::PagedRows& pg, bool selector, cudaStream_t st)
+{
+#ifdef DSA_DEBUG
+    dsa::debug_check_idx_kernel<<<T, dsa::kCheckThreads, 0, st>>>(idx, pos, k_base, T, S, k, pg, selector ? 1 : 0);
+    DSA_LAUNCH_CHECK("debug_check_idx_kernel");
+#else
+    (void)idx; (void)pos; (void)k_base; (void)T; (void)S; (void)k; (void)pg; (void)selector; (void)st;
+#endif
+    return DSA_OK;
+}
+
+// ------------------------------------------------------------ phase timing
+//
+// Diagnostic: with timing on, the indexer brackets each of its phases with a
+// pair of CUDA events on the caller's stream; dsa_phase_times() sums them.
+enum Phase : int { kPhaseScores = 0, kPhaseThreshold = 1, kPhaseSelect = 2, kNumPhases = 3 };
+
+struct PhaseRec {
+    int phase;
+    cudaEvent_t a, b;
+};
+std::mutex g_phase_mu;
+std::atomic<bool> g_phase_on{false};
+std::vector<PhaseRec> g_phase_recs;
+
+// Records the start of a phase; the returned handle closes it.
+struct PhaseMark {
+    int phase = -1;
+    cudaEvent_t a = nullptr;
+    cudaStream_t st = nullptr;
+};
+
+PhaseMark phase_begin(int phase, cudaStream_t st)
+{
+    PhaseMark m;
+    if (!g_phase_on.load(std::memory_order_relaxed)) return m;
+    if (cudaEventCreate(&m.a) != cudaSuccess) return PhaseMark{};
+    cudaEventRecord(m.a, st);
+    m.phase = phase;
+    m.st = st;
+    return m;
+}
+
+void phase_end(const PhaseMark& m)
+{
+    if (m.phase < 0) return;
+    cudaEvent_t b;
+    if (cudaEventCreate(&b) != cudaSuccess) {
+        cudaEventDestroy(m.a);
+        return;
+    }
+    cudaEventRecord(b, m.st);
+    std::lock_guard<std::mutex> lock(g_phase_mu);
+    g_phase_recs.push_back({m.phase, m.a, b});
+}
+
+// Launch with programmatic stream serialization: the kernel may start while
+// the previous kernel on the stream drains (it calls griddep_wait() before
+// reading global memory), which hides the launch gap between the short
+// kernels of a decode step.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 // ------------------------------------------------------------ workspace plan
 
 constexpr size_t kAlign = 256;
@@ -158,9 +241,13 @@ FusedPlan fused_plan(int T, int S, int k)
     return p;
 }
 
-size_t indexer_workspace(int T, int S, int k = 1)
+// Workspace of the indexer paths these head shapes can take (the streaming
+// tensor-core path exists for H_I = 8, d_I = 128 only).
+size_t indexer_workspace(int T, int S, int k, int H_I, int d_I)
 {
-    return std::max(chunk_plan(T, S, k).bytes, fused_plan(T, S, k).bytes);
+    const size_t chunked = chunk_plan(T, S, k).bytes;
+    if (H_I != dsa::idx_tc::kHI || d_I != dsa::idx_tc::kDI) return chunked;
+    return std::max(chunked, fused_plan(T, S, k).bytes);
 }
 
 int num_sms()
@@ -175,26 +262,43 @@ int num_sms()
     return sms;
 }
 
-// Splits of each row's selected set so that few rows still fill the GPU.
-int attn_splits(int T, int Hq, int k)
+// Tensor-core attention: one 2-CTA cluster per query row (Hq=128, d_qk=576,
+// d_v=512, k a multiple of 4).
+bool attn_tc_supported(int Hq, int d_qk, int d_v, int k)
 {
-    if (const char* e = getenv("DSA_ATTN_SPLITS")) {
-        const int v = atoi(e);
-        if (v >= 1) return std::min(v, std::max(1, k));
+    return Hq == dsa::attn_tc::kHeads && d_qk == dsa::attn_tc::kDqk && d_v == dsa::attn_tc::kDv &&
+           k % 4 == 0;
+}
+
+// Parts each row's selected set is split into when the caller leaves it to
+// the library: only as many as add no wave of work. CUDA-core kernel: CTAs
+// of 8 heads, two per SM; tensor-core kernel: one cluster per SM pair.
+int attn_auto_splits(int T, int Hq, int d_qk, int d_v, int k)
+{
+    const int max_split = std::max(1, std::min(16, k / 64));
+    if (attn_tc_supported(Hq, d_qk, d_v, k)) {
+        const int slots = num_sms() / 2;
+        if (T >= slots) return 1;
+        return std::max(1, std::min(max_split, slots / T));
     }
     const long long ctas = (long long)T * dsa::ceil_div(Hq, dsa::kAttnHeads);
     const long long want = 2LL * num_sms();
     if (ctas >= want) return 1;
     const int s = (int)((want + ctas - 1) / ctas);
-    return std::max(1, std::min({s, 16, std::max(1, k / 64)}));
+    return std::max(1, std::min(s, max_split));
 }
 
-size_t attn_workspace(int T, int Hq, int d_v, int k)
+// Workspace of a split attention: the parts' fp32 outputs and log-sum-exps.
+size_t attn_split_workspace(int T, int Hq, int d_v, int splits)
 {
-    const int splits = attn_splits(T, Hq, k);
-    if (splits == 1) return 0;
+    if (splits <= 1) return 0;
     return align_up((size_t)T * splits * Hq * d_v * sizeof(float)) +
            align_up((size_t)T * splits * Hq * sizeof(float));
+}
+
+size_t attn_workspace(int T, int Hq, int d_qk, int d_v, int k)
+{
+    return attn_split_workspace(T, Hq, d_v, attn_auto_splits(T, Hq, d_qk, d_v, k));
 }
 
 // ---------------------------------------------------------- argument checks
@@ -282,9 +386,8 @@ struct ChunkKernels {
     static void sample(int grid, cudaStream_t st, const ChunkArgs& a, float* samp, long long samp_ld)
     {
         using namespace dsa::idx_chunk;
-        chunk_sample_kernel<NT, DI><<<grid, kThreads, 0, st>>>(a.q_idx, a.w, a.k_idx, a.pos, a.k_base, a.T,
-                                                              a.S, a.H_I, a.row0, a.rows, a.work_off,
-                                                              samp, samp_ld, a.pg);
+        launch_pdl(chunk_sample_kernel<NT, DI>, dim3(grid), dim3(kThreads), 0, st, a.q_idx, a.w, a.k_idx, a.pos,
+                   a.k_base, a.T, a.S, a.H_I, a.row0, a.rows, a.work_off, samp, samp_ld, a.pg);
     }
     static void topk(int grid, cudaStream_t st, const ChunkArgs& a, const uint32_t* tau, uint2* cand,
                      long long cand_ld, int* ccnt, int max_chunks, int32_t* idx)
@@ -292,9 +395,9 @@ struct ChunkKernels {
         using namespace dsa::idx_chunk;
         cudaFuncSetAttribute(chunk_topk_kernel<NT, DI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kSmemBytes);
-        chunk_topk_kernel<NT, DI><<<grid, kThreads, kSmemBytes, st>>>(
-            a.q_idx, a.w, a.k_idx, a.pos, a.k_base, a.T, a.S, a.H_I, a.row0, a.rows, a.k, a.work_off,
-            tau, cand, cand_ld, ccnt, max_chunks, idx);
+        launch_pdl(chunk_topk_kernel<NT, DI>, dim3(grid), dim3(kThreads), kSmemBytes, st, a.q_idx, a.w, a.k_idx,
+                   a.pos, a.k_base, a.T, a.S, a.H_I, a.row0, a.rows, a.k, a.work_off, tau, cand, cand_ld, ccnt,
+                   max_chunks, idx);
     }
 };
 
@@ -307,9 +410,9 @@ void chunk_topk_tma(int grid, cudaStream_t st, const CUtensorMap& tm_k, const Ch
     using namespace dsa::idx_chunk;
     cudaFuncSetAttribute(chunk_topk_tma_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          tma::kSmemBytes);
-    chunk_topk_tma_kernel<NT><<<grid, tma::kThreads, tma::kSmemBytes, st>>>(
-        tm_k, a.q_idx, a.w, a.pos, a.k_base, a.T, a.S, a.H_I, a.row0, a.rows, a.k, a.work_off, tau, cand,
-        cand_ld, ccnt, max_chunks, idx, a.pg);
+    launch_pdl(chunk_topk_tma_kernel<NT>, dim3(grid), dim3(tma::kThreads), tma::kSmemBytes, st, tm_k, a.q_idx,
+               a.w, a.pos, a.k_base, a.T, a.S, a.H_I, a.row0, a.rows, a.k, a.work_off, tau, cand, cand_ld, ccnt,
+               max_chunks, idx, a.pg);
 }
 
 struct ChunkFns {
@@ -389,33 +492,46 @@ int indexer_chunked(const uint8_t* q_idx, const float* w, const uint8_t* k_idx, 
         const int grid = (int)std::min<long long>(
             (long long)rows * std::max(1, dsa::ceil_div(n_max, kChunkKeys)), resident);
         const ChunkArgs a{q_idx, w, k_idx, pos, k_base, T, S, H_I, k, row0, rows, work_off, pg};
-        chunk_plan_kernel<<<1, kPlanThreads, 0, st>>>(pos, k_base, T, S, row0, rows, work_off, pg);
+        PhaseMark ph = phase_begin(kPhaseThreshold, st);
+        launch_pdl(chunk_plan_kernel, dim3(1), dim3(kPlanThreads), 0, st, pos, k_base, T, S, row0, rows, work_off,
+                   pg);
         DSA_LAUNCH_CHECK("chunk_plan_kernel");
         if (multi) {
             fn.sample(grid, st, a, samp, p.samp_ld);
             DSA_LAUNCH_CHECK("chunk_sample_kernel");
-            chunk_tau_kernel<kTauThreads><<<rows, kTauThreads, 0, st>>>(samp, p.samp_ld, pos, k_base, T, S,
-                                                                       row0, k, tau, pg);
+            launch_pdl(chunk_tau_kernel<kTauThreads>, dim3(rows), dim3(kTauThreads), 0, st, samp, p.samp_ld, pos,
+                       k_base, T, S, row0, k, tau, pg);
             DSA_LAUNCH_CHECK("chunk_tau_kernel");
         }
+        phase_end(ph);
+        ph = phase_begin(kPhaseScores, st);
         topk(a, grid, multi ? tau : nullptr);
         DSA_LAUNCH_CHECK("chunk_topk_kernel");
+        phase_end(ph);
         if (!multi) continue;
-        merge_topk_kernel<kMergeThreads><<<rows, kMergeThreads, merge_smem, st>>>(
-            cand, p.cand_ld, ccnt, p.max_chunks, q_idx, w, k_idx, H_I, d_I, pos, k_base, T, S, row0, k,
-            idx, pg);
+        ph = phase_begin(kPhaseSelect, st);
+        launch_pdl(merge_topk_kernel<kMergeThreads>, dim3(rows), dim3(kMergeThreads), merge_smem, st, cand,
+                   p.cand_ld, ccnt, p.max_chunks, q_idx, w, k_idx, H_I, d_I, pos, k_base, T, S, row0, k, idx, pg);
         DSA_LAUNCH_CHECK("merge_topk_kernel");
+        phase_end(ph);
     }
     return DSA_OK;
 }
 
-// One causal sequence (pos and k_base NULL), H_I = 8, d_I = 128: streamed
-// FP8 tensor-core scan with sampled thresholds (indexer_tc.cuh).
-bool indexer_fused_supported(const int32_t* pos, const int32_t* k_base, int H_I, int d_I)
+// Shared memory the streaming indexer's threshold and select kernels stage a
+// row in (its samples, its candidates).
+constexpr size_t kFusedStageMax = 200 * 1024;
+
+// One causal sequence (pos and k_base NULL), H_I = 8, d_I = 128, and a row's
+// samples and candidates fit the select kernels' shared memory: streamed FP8
+// tensor-core scan with sampled thresholds (indexer_tc.cuh).
+bool indexer_fused_supported(const int32_t* pos, const int32_t* k_base, int H_I, int d_I, int S, int k)
 {
-    if (const char* e = getenv("DSA_INDEXER_IMPL"))
-        if (strcmp(e, "general") == 0) return false;
-    return !pos && !k_base && H_I == dsa::idx_tc::kHI && d_I == dsa::idx_tc::kDI;
+    using namespace dsa::idx_tc;
+    if (pos || k_base || H_I != kHI || d_I != kDI) return false;
+    const size_t samp_bytes = (size_t)((num_tiles(S) + kSampleStride - 1) / kSampleStride) * kKeys * sizeof(float);
+    const size_t cand_bytes = (size_t)2 * kAlpha * k * sizeof(uint2) + (size_t)dsa::pow2_ceil(k) * sizeof(int);
+    return samp_bytes <= kFusedStageMax && cand_bytes <= kFusedStageMax;
 }
 
 int make_tmap_u8(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t rows,
@@ -452,20 +568,39 @@ int indexer_fused(const uint8_t* q_idx, const float* w, const uint8_t* k_idx, in
         cudaError_t e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(indexer_scan_kernel)");
     }
+    // staged samples (tau) and candidates (select) of one row
+    const size_t tau_smem = (size_t)p.samp_ld * sizeof(float);
+    const size_t sel_smem = (size_t)p.cap * sizeof(uint2) + (size_t)dsa::pow2_ceil(k) * sizeof(int);
+    {
+        cudaError_t e = cudaFuncSetAttribute(indexer_tau_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)tau_smem);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(indexer_select_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)sel_smem);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(indexer_tau/select_kernel)");
+    }
     for (int row0 = 0; row0 < T; row0 += p.RB) {
         const int rows = std::min(p.RB, T - row0);
         ScanArgs a{w, T, S, k, row0, rows, samp, p.samp_ld, tau, cand, cnt, p.cap};
         const int ctas = (rows + kRows - 1) / kRows;
+        PhaseMark ph = phase_begin(kPhaseScores, st);
         indexer_scan_kernel<true><<<ctas, kThreads, kSmemBytes, st>>>(tq, tk, a);
         DSA_LAUNCH_CHECK("indexer_scan_kernel<sample>");
-        indexer_tau_kernel<256><<<rows, 256, 0, st>>>(samp, p.samp_ld, T, S, k, row0, tau);
+        phase_end(ph);
+        ph = phase_begin(kPhaseThreshold, st);
+        indexer_tau_kernel<256><<<rows, 256, tau_smem, st>>>(samp, p.samp_ld, T, S, k, row0, tau);
         DSA_LAUNCH_CHECK("indexer_tau_kernel");
+        phase_end(ph);
+        ph = phase_begin(kPhaseScores, st);
         indexer_scan_kernel<false><<<ctas, kThreads, kSmemBytes, st>>>(tq, tk, a);
         DSA_LAUNCH_CHECK("indexer_scan_kernel<filter>");
+        phase_end(ph);
         // ~2k candidates per row: 256 threads keep the radix passes busy
-        indexer_select_kernel<256><<<rows, 256, 0, st>>>(cand, cnt, p.cap, q_idx, w, k_idx, T, S, k,
-                                                         row0, idx);
+        ph = phase_begin(kPhaseSelect, st);
+        indexer_select_kernel<256><<<rows, 256, sel_smem, st>>>(cand, cnt, p.cap, q_idx, w, k_idx, T, S, k,
+                                                                row0, idx);
         DSA_LAUNCH_CHECK("indexer_select_kernel");
+        phase_end(ph);
     }
     return DSA_OK;
 }
@@ -474,10 +609,9 @@ int indexer_fused(const uint8_t* q_idx, const float* w, const uint8_t* k_idx, in
 
 int attn_simple(const __nv_bfloat16* q, const __nv_bfloat16* kv, const int32_t* idx,
                 const int32_t* pos, const int32_t* k_base, int T, int S, int Hq, int d_qk,
-                int d_v, int k, float scale, __nv_bfloat16* out, float* lse, void* workspace,
+                int d_v, int k, float scale, int splits, __nv_bfloat16* out, float* lse, void* workspace,
                 cudaStream_t st)
 {
-    const int splits = attn_splits(T, Hq, k);
     const int kcap = dsa::ceil_div(k, splits);
     const size_t smem = dsa::attn_simple_smem(d_qk, kcap);
     cudaError_t e = cudaFuncSetAttribute(dsa::sparse_attn_simple_kernel,
@@ -502,16 +636,6 @@ int attn_simple(const __nv_bfloat16* q, const __nv_bfloat16* kv, const int32_t* 
     return DSA_OK;
 }
 
-// Tensor-core path: one 2-CTA cluster per query row (Hq=128, d_qk=576, d_v=512).
-bool attn_tc_supported(int Hq, int d_qk, int d_v, int k)
-{
-    if (const char* e = getenv("DSA_ATTN_IMPL"))
-        if (strcmp(e, "simple") == 0) return false;
-    if (getenv("DSA_ATTN_SPLITS")) return false;
-    return Hq == dsa::attn_tc::kHeads && d_qk == dsa::attn_tc::kDqk && d_v == dsa::attn_tc::kDv &&
-           k % 4 == 0;
-}
-
 // 2D bf16 tensor map over a row-major [rows, cols] matrix, box [box_rows, box_cols].
 int make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows,
                    uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle sw)
@@ -532,7 +656,8 @@ int make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t cols, uint64_t row
 
 int attn_tc(const __nv_bfloat16* q, const __nv_bfloat16* kv, const int32_t* idx,
             const int32_t* pos, const int32_t* k_base, int T, int S, int k, float scale,
-            __nv_bfloat16* out, float* lse, cudaStream_t st, const dsa::PagedRows& pg = {})
+            __nv_bfloat16* out, float* lse, cudaStream_t st, const dsa::PagedRows& pg = {},
+            int splits = 1, void* workspace = nullptr)
 {
     using namespace dsa::attn_tc;
     cudaError_t e = cudaFuncSetAttribute(sparse_mla_attn_tc_kernel,
@@ -547,10 +672,47 @@ int attn_tc(const __nv_bfloat16* q, const __nv_bfloat16* kv, const int32_t* idx,
     if (int rc = make_tmap_bf16(&tq64, q, kDqk, (uint64_t)T * kHeads, 32, kHeads,
                                 CU_TENSOR_MAP_SWIZZLE_64B)) return rc;
     const float scale_log2 = scale * 1.4426950408889634f;
-    sparse_mla_attn_tc_kernel<<<dim3(2 * T), kThreads, kSmemBytes, st>>>(
-        tq128, tq64, q, kv, idx, pos, k_base, T, S, k, scale_log2, out, lse, pg);
+    float* part_o = nullptr;
+    float* part_lse = nullptr;
+    if (splits > 1) {
+        part_o = reinterpret_cast<float*>(workspace);
+        part_lse = reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) +
+                                            align_up((size_t)T * splits * kHeads * kDv * sizeof(float)));
+    }
+    launch_pdl(sparse_mla_attn_tc_kernel, dim3(2 * T * splits), dim3(kThreads), kSmemBytes, st, tq128, tq64, q,
+               kv, idx, pos, k_base, T, S, k, scale_log2, out, lse, pg, splits, part_o, part_lse);
     DSA_LAUNCH_CHECK("sparse_mla_attn_tc_kernel");
+    if (splits > 1) {
+        launch_pdl(lse_merge_kernel, dim3(T, kHeads / kMergeHeads), dim3(128), 0, st, part_o, part_lse, T, splits,
+                   out, lse);
+        DSA_LAUNCH_CHECK("lse_merge_kernel");
+    }
     return DSA_OK;
+}
+
+// Sparse attention with `splits` parts per row (0: the library's choice).
+int attn_dispatch(const void* q, const void* kv, const int32_t* idx, const int32_t* pos, const int32_t* k_base,
+                  int T, int S, int Hq, int d_qk, int d_v, int k, float scale, int splits, void* out, float* lse,
+                  void* workspace, size_t ws_bytes, void* stream)
+{
+    using bf = __nv_bfloat16;
+    if (splits < 0 || splits > dsa::attn_tc::kMaxSplits)
+        return fail(DSA_ERR_ARG, "splits=%d (supported: 0..%d)", splits, dsa::attn_tc::kMaxSplits);
+    if (splits == 0) splits = attn_auto_splits(T, Hq, d_qk, d_v, k);
+    const size_t need = attn_split_workspace(T, Hq, d_v, splits);
+    if (need && (!workspace || ws_bytes < need || !al16(workspace)))
+        return fail(DSA_ERR_WORKSPACE, "attention with %d parts per row needs %zu workspace bytes (got %zu)",
+                    splits, need, ws_bytes);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (int rc = debug_check(idx, pos, k_base, T, S, k, {}, false, st)) return rc;
+    if (attn_tc_supported(Hq, d_qk, d_v, k)) {
+        if ((long long)T * splits > 0x3FFFFFFF)
+            return fail(DSA_ERR_UNSUPPORTED, "T * splits = %lld clusters", (long long)T * splits);
+        return attn_tc(reinterpret_cast<const bf*>(q), reinterpret_cast<const bf*>(kv), idx, pos, k_base, T, S,
+                       k, scale, reinterpret_cast<bf*>(out), lse, st, {}, splits, workspace);
+    }
+    return attn_simple(reinterpret_cast<const bf*>(q), reinterpret_cast<const bf*>(kv), idx, pos, k_base, T, S,
+                       Hq, d_qk, d_v, k, scale, splits, reinterpret_cast<bf*>(out), lse, workspace, st);
 }
 
 // ---------------------------------------------------------- attention backward
@@ -709,11 +871,8 @@ const char* dsa_last_error(void) { return g_err; }
 
 size_t dsa_workspace_size(int T, int S, int H_I, int d_I, int k, int Hq, int d_qk, int d_v)
 {
-    (void)H_I;
-    (void)d_I;
-    (void)d_qk;
     if (T <= 0 || S <= 0 || k <= 0 || Hq <= 0 || d_v <= 0) return 0;
-    return std::max(indexer_workspace(T, S, k), attn_workspace(T, Hq, d_v, k));
+    return std::max(indexer_workspace(T, S, k, H_I, d_I), attn_workspace(T, Hq, d_qk, d_v, k));
 }
 
 int dsa_indexer_topk(const void* q_idx, const float* w, const void* k_idx, const int32_t* pos,
@@ -722,16 +881,18 @@ int dsa_indexer_topk(const void* q_idx, const float* w, const void* k_idx, const
 {
     g_err[0] = 0;
     if (int rc = check_indexer(q_idx, w, k_idx, pos, k_base, T, S, H_I, d_I, k, idx)) return rc;
-    const size_t need = indexer_workspace(T, S, k);
+    const size_t need = indexer_workspace(T, S, k, H_I, d_I);
     if (need && (!workspace || ws_bytes < need || !al16(workspace)))
         return fail(DSA_ERR_WORKSPACE, "indexer needs %zu workspace bytes (got %zu)", need, ws_bytes);
-    if (indexer_fused_supported(pos, k_base, H_I, d_I))
-        return indexer_fused(reinterpret_cast<const uint8_t*>(q_idx), w,
-                             reinterpret_cast<const uint8_t*>(k_idx), T, S, k, idx, workspace,
-                             reinterpret_cast<cudaStream_t>(stream));
-    return indexer_chunked(reinterpret_cast<const uint8_t*>(q_idx), w,
-                           reinterpret_cast<const uint8_t*>(k_idx), pos, k_base, T, S, H_I, d_I, k,
-                           idx, workspace, reinterpret_cast<cudaStream_t>(stream));
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int rc = indexer_fused_supported(pos, k_base, H_I, d_I, S, k)
+                       ? indexer_fused(reinterpret_cast<const uint8_t*>(q_idx), w,
+                                       reinterpret_cast<const uint8_t*>(k_idx), T, S, k, idx, workspace, st)
+                       : indexer_chunked(reinterpret_cast<const uint8_t*>(q_idx), w,
+                                         reinterpret_cast<const uint8_t*>(k_idx), pos, k_base, T, S, H_I, d_I, k,
+                                         idx, workspace, st);
+    if (rc) return rc;
+    return debug_check(idx, pos, k_base, T, S, k, {}, true, st);
 }
 
 int dsa_indexer_topk_varlen(const void* q_idx, const float* w, const void* k_idx, const int32_t* cu_q,
@@ -746,7 +907,7 @@ int dsa_indexer_topk_varlen(const void* q_idx, const float* w, const void* k_idx
         const int Tb = cu_q[b + 1] - cu_q[b], Sb = cu_k[b + 1] - cu_k[b];
         if (Tb < 0 || Sb < 0 || Tb > Sb)
             return fail(DSA_ERR_ARG, "sequence %d: %d query rows over %d keys (need 0 <= T <= S)", b, Tb, Sb);
-        if (Tb > 0) need = std::max(need, indexer_workspace(Tb, Sb, k));
+        if (Tb > 0) need = std::max(need, indexer_workspace(Tb, Sb, k, H_I, d_I));
     }
     const int T = cu_q[n_seqs], S = cu_k[n_seqs];
     if (int rc = check_indexer(q_idx, w, k_idx, nullptr, nullptr, T, S, H_I, d_I, k, idx)) return rc;
@@ -766,11 +927,12 @@ int dsa_indexer_topk_varlen(const void* q_idx, const float* w, const void* k_idx
             return fail(DSA_ERR_ARG, "sequence %d: its rows of q_idx, w, k_idx or idx are not 16-byte "
                                      "aligned (cu_q[b] * H_I * 4 and cu_q[b] * k * 4 must be multiples "
                                      "of 16)", b);
-        const int rc = indexer_fused_supported(nullptr, nullptr, H_I, d_I)
+        const int rc = indexer_fused_supported(nullptr, nullptr, H_I, d_I, Sb, k)
                            ? indexer_fused(qb, wb, kb, Tb, Sb, k, ib, workspace, st)
                            : indexer_chunked(qb, wb, kb, nullptr, nullptr, Tb, Sb, H_I, d_I, k, ib,
                                              workspace, st);
         if (rc) return rc;
+        if (int rc2 = debug_check(ib, nullptr, nullptr, Tb, Sb, k, {}, true, st)) return rc2;
     }
     return DSA_OK;
 }
@@ -804,7 +966,7 @@ int dsa_indexer_topk_paged(const void* q_idx, const float* w, const void* k_page
     const int S = max_pages * page_size;   // the most keys a row can have
     if (int rc = check_indexer(q_idx, w, k_pages, pos, nullptr, T, S, H_I, d_I, k, idx)) return rc;
     if (d_I != 128) return fail(DSA_ERR_UNSUPPORTED, "a paged key cache needs d_I = 128 (got %d)", d_I);
-    const size_t need = indexer_workspace(T, S, k);
+    const size_t need = indexer_workspace(T, S, k, H_I, d_I);
     if (need && (!workspace || ws_bytes < need || !al16(workspace)))
         return fail(DSA_ERR_WORKSPACE, "indexer needs %zu workspace bytes (got %zu)", need, ws_bytes);
     dsa::PagedRows pg;
@@ -814,9 +976,12 @@ int dsa_indexer_topk_paged(const void* q_idx, const float* w, const void* k_page
     pg.max_pages = max_pages;
     pg.page_size = page_size;
     pg.num_pages = num_pages;
-    return indexer_chunked(reinterpret_cast<const uint8_t*>(q_idx), w,
-                           reinterpret_cast<const uint8_t*>(k_pages), pos, nullptr, T, S, H_I, d_I, k, idx,
-                           workspace, reinterpret_cast<cudaStream_t>(stream), pg);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (int rc = indexer_chunked(reinterpret_cast<const uint8_t*>(q_idx), w,
+                                 reinterpret_cast<const uint8_t*>(k_pages), pos, nullptr, T, S, H_I, d_I, k, idx,
+                                 workspace, st, pg))
+        return rc;
+    return debug_check(idx, pos, nullptr, T, S, k, pg, true, st);
 }
 
 int dsa_sparse_mla_attn_paged(const void* q, const void* kv_pages, int num_pages, int page_size,
@@ -838,9 +1003,10 @@ int dsa_sparse_mla_attn_paged(const void* q, const void* kv_pages, int num_pages
     pg.max_pages = max_pages;
     pg.page_size = page_size;
     pg.num_pages = num_pages;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (int rc = debug_check(idx, pos, nullptr, T, S, k, pg, false, st)) return rc;
     return attn_tc(reinterpret_cast<const __nv_bfloat16*>(q), reinterpret_cast<const __nv_bfloat16*>(kv_pages),
-                   idx, pos, nullptr, T, S, k, scale, reinterpret_cast<__nv_bfloat16*>(out), lse,
-                   reinterpret_cast<cudaStream_t>(stream), pg);
+                   idx, pos, nullptr, T, S, k, scale, reinterpret_cast<__nv_bfloat16*>(out), lse, st, pg);
 }
 
 int dsa_sparse_mla_attn(const void* q, const void* kv, const int32_t* idx, const int32_t* pos,
@@ -850,19 +1016,24 @@ int dsa_sparse_mla_attn(const void* q, const void* kv, const int32_t* idx, const
 {
     g_err[0] = 0;
     if (int rc = check_attn(q, kv, idx, pos, k_base, T, S, Hq, d_qk, d_v, k, out, lse)) return rc;
-    if (attn_tc_supported(Hq, d_qk, d_v, k))
-        return attn_tc(reinterpret_cast<const __nv_bfloat16*>(q),
-                       reinterpret_cast<const __nv_bfloat16*>(kv), idx, pos, k_base, T, S, k, scale,
-                       reinterpret_cast<__nv_bfloat16*>(out), lse,
-                       reinterpret_cast<cudaStream_t>(stream));
-    const size_t need = attn_workspace(T, Hq, d_v, k);
-    if (need && (!workspace || ws_bytes < need || !al16(workspace)))
-        return fail(DSA_ERR_WORKSPACE, "attention needs %zu workspace bytes (got %zu)", need,
-                    ws_bytes);
-    return attn_simple(reinterpret_cast<const __nv_bfloat16*>(q),
-                       reinterpret_cast<const __nv_bfloat16*>(kv), idx, pos, k_base, T, S, Hq,
-                       d_qk, d_v, k, scale, reinterpret_cast<__nv_bfloat16*>(out), lse, workspace,
-                       reinterpret_cast<cudaStream_t>(stream));
+    return attn_dispatch(q, kv, idx, pos, k_base, T, S, Hq, d_qk, d_v, k, scale, 0, out, lse, workspace, ws_bytes,
+                         stream);
+}
+
+size_t dsa_sparse_mla_attn_split_workspace_size(int T, int Hq, int d_v, int splits)
+{
+    if (T <= 0 || Hq <= 0 || d_v <= 0 || splits < 0) return 0;
+    return attn_split_workspace(T, Hq, d_v, splits);
+}
+
+int dsa_sparse_mla_attn_split(const void* q, const void* kv, const int32_t* idx, const int32_t* pos,
+                              const int32_t* k_base, int T, int S, int Hq, int d_qk, int d_v, int k, float scale,
+                              int splits, void* out, float* lse, void* workspace, size_t ws_bytes, void* stream)
+{
+    g_err[0] = 0;
+    if (int rc = check_attn(q, kv, idx, pos, k_base, T, S, Hq, d_qk, d_v, k, out, lse)) return rc;
+    return attn_dispatch(q, kv, idx, pos, k_base, T, S, Hq, d_qk, d_v, k, scale, splits, out, lse, workspace,
+                         ws_bytes, stream);
 }
 
 size_t dsa_sparse_mla_attn_bwd_workspace_size(int T, int Hq, int k)
@@ -941,6 +1112,74 @@ int dsa_forward(const void* q_idx, const float* w, const void* k_idx, const void
                                workspace, ws_bytes, stream);
 }
 
+// ------------------------------------------------------- multi-GPU partition
+//
+// The path shards by query rows and by sequences with no exchange between
+// ranks; these host-only functions pick the contiguous ranges.
+
+namespace {
+
+// Split items with costs c[0..n) into `parts` contiguous ranges of about
+// equal total cost: range r ends at the first item where the running cost
+// reaches (r+1)/parts of the total. bounds[0] = 0, bounds[parts] = n.
+void balanced_bounds(const double* prefix, int n, int parts, int32_t* bounds)
+{
+    const double total = prefix[n];
+    bounds[0] = 0;
+    int i = 0;
+    for (int r = 1; r < parts; ++r) {
+        const double goal = total * r / parts;
+        while (i < n && prefix[i + 1] < goal) ++i;
+        // item i straddles the goal: end the range before or after it,
+        // whichever lands closer
+        int b = i;
+        if (i < n && prefix[i + 1] - goal < goal - prefix[i]) b = i + 1;
+        bounds[r] = std::max(b, (int)bounds[r - 1]);
+    }
+    bounds[parts] = n;
+}
+
+}  // namespace
+
+int dsa_partition_prefill_rows(int T, int S, int k, int H_I, int d_I, int Hq, int d_qk, int d_v, int parts,
+                               int32_t* bounds)
+{
+    g_err[0] = 0;
+    if (!bounds) return fail(DSA_ERR_ARG, "NULL bounds");
+    if (T <= 0 || S < T || k <= 0 || H_I <= 0 || d_I <= 0 || Hq <= 0 || d_qk <= 0 || d_v <= 0 || parts <= 0)
+        return fail(DSA_ERR_ARG, "T=%d, S=%d, k=%d, H_I=%d, d_I=%d, Hq=%d, d_qk=%d, d_v=%d, parts=%d",
+                    T, S, k, H_I, d_I, Hq, d_qk, d_v, parts);
+    // modelled time of row t (position p = t + S - T, n = p + 1 candidates):
+    // indexer FP8 MMA work over its n keys when n > k (FP8 at twice the BF16
+    // rate), then the BF16 attention work over min(n, k) selected rows
+    std::vector<double> prefix((size_t)T + 1, 0.0);
+    const double w_idx = 2.0 * H_I * d_I / 2.0, w_attn = 2.0 * Hq * (double)(d_qk + d_v);
+    for (int t = 0; t < T; ++t) {
+        const double n = (double)t + (S - T) + 1;
+        prefix[t + 1] = prefix[t] + (n > k ? n * w_idx : 0.0) + std::min(n, (double)k) * w_attn;
+    }
+    balanced_bounds(prefix.data(), T, parts, bounds);
+    return DSA_OK;
+}
+
+int dsa_partition_decode_seqs(const int32_t* ctx, int n_seqs, int k, int d_I, int d_qk, int parts,
+                              int32_t* bounds)
+{
+    g_err[0] = 0;
+    if (!ctx || !bounds) return fail(DSA_ERR_ARG, "NULL ctx or bounds");
+    if (n_seqs <= 0 || k <= 0 || d_I <= 0 || d_qk <= 0 || parts <= 0)
+        return fail(DSA_ERR_ARG, "n_seqs=%d, k=%d, d_I=%d, d_qk=%d, parts=%d", n_seqs, k, d_I, d_qk, parts);
+    // modelled time of a sequence: the bytes its step reads (every cached
+    // indexer key once, the selected latent rows once)
+    std::vector<double> prefix((size_t)n_seqs + 1, 0.0);
+    for (int b = 0; b < n_seqs; ++b) {
+        if (ctx[b] < 0) return fail(DSA_ERR_ARG, "ctx[%d] = %d", b, ctx[b]);
+        prefix[b + 1] = prefix[b] + (double)ctx[b] * d_I + std::min(ctx[b], k) * 2.0 * d_qk;
+    }
+    balanced_bounds(prefix.data(), n_seqs, parts, bounds);
+    return DSA_OK;
+}
+
 int dsa_device_status(void* stream)
 {
     cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
@@ -949,12 +1188,74 @@ int dsa_device_status(void* stream)
     e = cudaMemcpyFromSymbol(&v, dsa::g_status, sizeof v);
     if (e != cudaSuccess) return cuda_fail(e, "read device status");
     if (v != 0) {
+        const int zero = 0;
+        if (v == dsa::kStatusCheck) {
+            cudaMemcpyToSymbol(dsa::g_status, &zero, sizeof zero);
+            return fail(v, "a debug-build check counted invalid index-set entries (dsa_debug_counters)");
+        }
         int info[4] = {0, 0, 0, 0};
         cudaMemcpyFromSymbol(info, dsa::g_timeout_info, sizeof info);
-        const int zero = 0;
         cudaMemcpyToSymbol(dsa::g_status, &zero, sizeof zero);
         return fail(v, "a kernel reported status %d: bounded wait gave up (barrier tag %d, chunk %d, "
                        "block %d, parity %d)", v, info[0], info[1], info[2], info[3]);
+    }
+    return DSA_OK;
+}
+
+int dsa_phase_timing(int enable)
+{
+    g_phase_on.store(enable != 0, std::memory_order_relaxed);
+    return DSA_OK;
+}
+
+int dsa_phase_times(double* ms, int n)
+{
+    g_err[0] = 0;
+    if (!ms || n < 0 || n > kNumPhases) return fail(DSA_ERR_ARG, "ms NULL or n=%d outside 0..%d", n, (int)kNumPhases);
+    std::vector<PhaseRec> recs;
+    {
+        std::lock_guard<std::mutex> lock(g_phase_mu);
+        recs.swap(g_phase_recs);
+    }
+    double sum[kNumPhases] = {0.0, 0.0, 0.0};
+    int rc = DSA_OK;
+    for (const PhaseRec& r : recs) {
+        float t = 0.f;
+        cudaError_t e = cudaEventSynchronize(r.b);
+        if (e == cudaSuccess) e = cudaEventElapsedTime(&t, r.a, r.b);
+        if (e != cudaSuccess && rc == DSA_OK) rc = cuda_fail(e, "phase timing events");
+        sum[r.phase] += t;
+        cudaEventDestroy(r.a);
+        cudaEventDestroy(r.b);
+    }
+    for (int i = 0; i < n; ++i) ms[i] = sum[i];
+    return rc;
+}
+
+int dsa_debug_build(void)
+{
+#ifdef DSA_DEBUG
+    return 1;
+#else
+    return 0;
+#endif
+}
+
+int dsa_debug_counters(uint64_t* out, int n, int reset)
+{
+    g_err[0] = 0;
+    if (!out || n < 0 || n > dsa::kNumDebugCounts)
+        return fail(DSA_ERR_ARG, "out NULL or n=%d outside 0..%d", n, (int)dsa::kNumDebugCounts);
+    unsigned long long v[dsa::kNumDebugCounts] = {0};
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+    e = cudaMemcpyFromSymbol(v, dsa::g_debug_counts, sizeof v);
+    if (e != cudaSuccess) return cuda_fail(e, "read debug counters");
+    for (int i = 0; i < n; ++i) out[i] = v[i];
+    if (reset) {
+        const unsigned long long z[dsa::kNumDebugCounts] = {0};
+        e = cudaMemcpyToSymbol(dsa::g_debug_counts, z, sizeof z);
+        if (e != cudaSuccess) return cuda_fail(e, "clear debug counters");
     }
     return DSA_OK;
 }
@@ -1014,7 +1315,9 @@ extern "C" int dsa_indexer_topk_noalloc(const void* q_idx, const float* w, const
     float* scores = nullptr;
     if (int rc = static_scores_on_current_device(&scores)) return rc;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    const int RB = (int)std::min<size_t>((size_t)T, kStaticScoreFloats / (size_t)S);
+    // rows per block: as many score rows as the array holds, at most 65535
+    // (the launches below put the block's rows on gridDim.y)
+    const int RB = (int)std::min<size_t>({(size_t)T, kStaticScoreFloats / (size_t)S, (size_t)65535});
     const long long ld = S;
     constexpr int kKeysPerCta = 2048;
     ScoresFn scores_fn = pick_scores(H_I, d_I);
@@ -1030,5 +1333,5 @@ extern "C" int dsa_indexer_topk_noalloc(const void* q_idx, const float* w, const
             <<<rb, dsa::kSelectThreads, 0, st>>>(scores, ld, pos, k_base, T, S, row0, k, idx);
         DSA_LAUNCH_CHECK("topk_dense_rows_kernel");
     }
-    return DSA_OK;
+    return debug_check(idx, pos, k_base, T, S, k, {}, true, st);
 }

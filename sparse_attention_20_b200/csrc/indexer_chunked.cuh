@@ -56,6 +56,7 @@ chunk_plan_kernel(const int* __restrict__ pos, const int* __restrict__ k_base, i
                   int rows, int* __restrict__ work_off, const PagedRows pg)
 {
     __shared__ int part[kPlanThreads];
+    griddep_wait();
     const int per = ceil_div(rows, kPlanThreads);
     const int r0 = threadIdx.x * per, r1 = min(rows, r0 + per);
     auto items = [&](int r) -> int {
@@ -138,6 +139,7 @@ chunk_sample_kernel(const uint8_t* __restrict__ q_idx, const float* __restrict__
                     const PagedRows pg)
 {
     static_assert(kSamplesPerChunk <= 16 * (kThreads / 32), "one 16-key block per warp");
+    griddep_wait();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gid = lane >> 2, tid4 = lane & 3;
     const int total = work_off[rows];
@@ -183,6 +185,7 @@ chunk_tau_kernel(const float* __restrict__ samp, long long samp_ld, const int* _
                  uint32_t* __restrict__ tau, const PagedRows pg)
 {
     __shared__ SelectSmem<THREADS> sm;
+    griddep_wait();
     const int r = blockIdx.x, t = row0 + r;
     long long base;
     const int* bt;
@@ -253,6 +256,7 @@ chunk_topk_kernel(const uint8_t* __restrict__ q_idx, const float* __restrict__ w
     float* sc = reinterpret_cast<float*>(smem);
     SelectSmem<kThreads>& sm = *reinterpret_cast<SelectSmem<kThreads>*>(smem + kChunkKeys * sizeof(float));
     const int lane = threadIdx.x & 31, tid4 = lane & 3;
+    griddep_wait();
     const int total = work_off[rows];
 
     for (int item = blockIdx.x; item < total; item += gridDim.x) {
@@ -329,6 +333,7 @@ chunk_topk_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const uint8_t* _
         prefetch_tmap(&tm_k);
     }
     __syncthreads();
+    griddep_wait();
     const int total = work_off[rows];
     struct Item {
         int r, t, chunk, n, nchunks, c0, m, ntiles;
@@ -510,6 +515,7 @@ merge_topk_kernel(const uint2* __restrict__ cand, long long cand_ld, const int* 
 {
     __shared__ SelectSmem<THREADS> sm;
     extern __shared__ int pre[];
+    griddep_wait();
     const int r = blockIdx.x, t = row0 + r;
     long long base;
     const int* bt;

@@ -264,13 +264,16 @@ __device__ __forceinline__ int sampled_valid(int n)
 }
 
 // tau_t: the r-th largest sampled score with r = ceil(alpha * k * m / n); rows
-// that can keep every candidate get -inf.
+// that can keep every candidate get -inf. The row's samples are staged in
+// shared memory (dynamic, samp_ld floats) so the radix passes read them once
+// from global memory.
 template <int THREADS>
 __global__ void __launch_bounds__(THREADS)
 indexer_tau_kernel(const float* __restrict__ samp, int samp_ld, int T, int S, int k, int row0,
                    float* __restrict__ tau)
 {
     __shared__ SelectSmem<THREADS> sm;
+    extern __shared__ float samp_s[];
     const int rl = blockIdx.x;
     const int t = row0 + rl;
     const int n = min(S, t + (S - T) + 1);
@@ -280,9 +283,12 @@ indexer_tau_kernel(const float* __restrict__ samp, int samp_ld, int T, int S, in
         const long long r = ((long long)kAlpha * k * m + n - 1) / n;
         const int stored = ((num_tiles(n) + kSampleStride - 1) / kSampleStride) * kKeys;
         if (r < m) {
+            const float4* src = reinterpret_cast<const float4*>(samp + (size_t)rl * samp_ld);
+            for (int i = threadIdx.x; i < stored / 4; i += THREADS) reinterpret_cast<float4*>(samp_s)[i] = src[i];
+            __syncthreads();
             int take_eq, count_eq;
-            DenseScores row{samp + (size_t)rl * samp_ld};
-            const uint32_t kth = radix_kth_key<THREADS>(row, stored, (int)r, sm, &take_eq, &count_eq);
+            const uint32_t kth = radix_kth_key<THREADS>(SmemScores{samp_s, 0}, stored, (int)r, sm, &take_eq,
+                                                        &count_eq);
             out = key_score(kth);
         }
     }
@@ -331,6 +337,11 @@ struct CandScores {
     __device__ __forceinline__ int s(int i) const { return (int)p[i].y; }
 };
 
+// The row's candidates are staged in shared memory (dynamic: cap pairs, then
+// pow2_ceil(k) ints) so the radix passes read them once from global memory.
+// The candidates arrive in no fixed order (appended by the scan's atomics), so
+// the selected set is sorted before it is written: every row comes out in
+// ascending s, deterministically (and attention over it sums in a fixed order).
 template <int THREADS>
 __global__ void __launch_bounds__(THREADS)
 indexer_select_kernel(const uint2* __restrict__ cand, const int* __restrict__ cnt, int cap,
@@ -339,6 +350,7 @@ indexer_select_kernel(const uint2* __restrict__ cand, const int* __restrict__ cn
                       int32_t* __restrict__ idx)
 {
     __shared__ SelectSmem<THREADS> sm;
+    extern __shared__ uint2 staged[];
     __shared__ float qf[kHI * kDI];
     __shared__ float wf[kHI];
     const int rl = blockIdx.x;
@@ -351,7 +363,16 @@ indexer_select_kernel(const uint2* __restrict__ cand, const int* __restrict__ cn
     }
     const int c = cnt[rl];
     if (c >= k && c <= cap) {
-        block_topk<THREADS>(CandScores{cand + (size_t)rl * cap}, c, k, out, sm);
+        const uint4* src = reinterpret_cast<const uint4*>(cand + (size_t)rl * cap);
+        for (int i = threadIdx.x; i < c / 2; i += THREADS) reinterpret_cast<uint4*>(staged)[i] = src[i];
+        if ((c & 1) && threadIdx.x == 0) staged[c - 1] = cand[(size_t)rl * cap + c - 1];
+        __syncthreads();
+        int* sel = reinterpret_cast<int*>(staged + cap);
+        const CandScores row{staged};
+        block_select<THREADS>(row, c, k, [&](int slot, int i) { sel[slot] = row.s(i); }, sm);
+        __syncthreads();
+        block_sort_ascending(sel, k, pow2_ceil(k));
+        for (int i = threadIdx.x; i < k; i += THREADS) out[i] = sel[i];
         return;
     }
     // threshold too high (fewer than k candidates) or buffer overflow: exact

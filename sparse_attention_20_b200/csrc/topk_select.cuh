@@ -245,6 +245,37 @@ __device__ void block_topk(const Row& row, int n, int k, int32_t* __restrict__ o
     block_select<THREADS, G>(row, n, k, [&](int slot, int i) { out[slot] = row.s(i); }, sm);
 }
 
+// Sorts v[0..n) ascending in shared memory (bitonic network over cap, a power
+// of two >= n; the tail is padded with INT_MAX). Every thread of the CTA takes
+// part.
+__device__ __forceinline__ void block_sort_ascending(int* v, int n, int cap)
+{
+    for (int i = n + (int)threadIdx.x; i < cap; i += blockDim.x) v[i] = 0x7FFFFFFF;
+    __syncthreads();
+    for (int size = 2; size <= cap; size <<= 1)
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            for (int i = threadIdx.x; i < cap / 2; i += blockDim.x) {
+                // i-th compare-exchange pair of this stage: (lo, lo + stride)
+                const int lo = 2 * i - (i & (stride - 1));
+                const int hi = lo + stride;
+                const bool up = (lo & size) == 0;
+                const int a = v[lo], b = v[hi];
+                if ((a > b) == up) {
+                    v[lo] = b;
+                    v[hi] = a;
+                }
+            }
+            __syncthreads();
+        }
+}
+
+__host__ __device__ __forceinline__ int pow2_ceil(int x)
+{
+    int p = 1;
+    while (p < x) p <<= 1;
+    return p;
+}
+
 constexpr int kSelectThreads = 1024;
 
 // One CTA per query row t = row0 + blockIdx.x; its scores are row blockIdx.x

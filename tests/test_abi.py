@@ -102,6 +102,22 @@ def test_attention_rejects_bad_arguments(lib):
              None) == -2
 
 
+def test_split_attention_arguments_and_workspace(lib):
+    f = lib.dsa_sparse_mla_attn_split
+    ws = ctypes.c_size_t(1 << 30)
+    sc = ctypes.c_float(0.1)
+    for bad in (-1, 17):
+        assert f(FAKE, FAKE, FAKE, None, None, 4, 4, 128, 576, 512, 64, sc, bad, FAKE, FAKE, FAKE, ws,
+                 None) == -1
+        assert b"splits" in lib.dsa_last_error()
+    # 4 parts of 64 rows need room for every part's fp32 output and log-sum-exp
+    need = lib.dsa_sparse_mla_attn_split_workspace_size(64, 128, 512, 4)
+    assert need >= 64 * 4 * 128 * (512 + 1) * 4
+    assert lib.dsa_sparse_mla_attn_split_workspace_size(64, 128, 512, 1) == 0
+    assert f(FAKE, FAKE, FAKE, None, None, 64, 64, 128, 576, 512, 64, sc, 4, FAKE, FAKE, FAKE,
+             ctypes.c_size_t(need - 1), None) == -5
+
+
 def test_attention_backward_rejects_bad_arguments(lib):
     f = lib.dsa_sparse_mla_attn_bwd
     sc = ctypes.c_float(0.1)

@@ -148,16 +148,53 @@ def test_k_equals_one_and_single_row():
     check_indexer(x, full.cpu(), list(range(x.T)), exact=True)
 
 
-def test_attention_splits_and_lse_merge(monkeypatch):
-    x = synth.prefill_inputs("prefill4k", device="cuda", seed=8, L=96, overrides=dict(k=80))
+@pytest.mark.parametrize("splits", [2, 5, 16])
+def test_attention_splits_and_lse_merge_cuda_core(splits):
+    """CUDA-core kernel (Hq = 4, d_qk = 80) with each row's set split into
+    parts and merged by log-sum-exp; parts of short rows are empty."""
+    x = synth.prefill_inputs("tiny", device="cuda", seed=8, L=200, overrides=dict(k=96))
     idx = dsa.indexer_topk(x.q_idx, x.w, x.k_idx, x.k)
-    out1, lse1 = dsa.sparse_mla_attn(x.q, x.kv, idx, x.scale, x.d_v)
-    monkeypatch.setenv("DSA_ATTN_SPLITS", "5")
-    out5, lse5 = dsa.sparse_mla_attn(x.q, x.kv, idx, x.scale, x.d_v)
+    out1, lse1 = dsa.sparse_mla_attn_split(x.q, x.kv, idx, x.scale, x.d_v, 1)
+    outs, lses = dsa.sparse_mla_attn_split(x.q, x.kv, idx, x.scale, x.d_v, splits)
     torch.cuda.synchronize()
     rows = list(range(x.T))
-    check_attention(x, idx.cpu(), out5.cpu(), lse5.cpu(), rows)
-    assert (out1.float() - out5.float()).abs().max().item() < 2e-2
+    check_attention(x, idx.cpu(), outs.cpu(), lses.cpu(), rows)
+    assert (out1.float() - outs.float()).abs().max().item() < 2e-2
+
+
+@pytest.mark.parametrize("splits", [2, 3, 5, 16])
+def test_decode_split_tensor_core_matches_oracle(splits):
+    """The decode variant on the tensor-core kernel: each row's selected set
+    split across clusters (ranges of whole 64-entry chunks; with short rows
+    and 16 parts some parts are empty), parts merged by log-sum-exp. Every row
+    against the oracle, and against the unsplit kernel."""
+    x = synth.decode_inputs("decode", device="cuda", seed=13, B=9,
+                            ctx=[9000, 1, 63, 64, 65, 700, 2047, 131072, 40000])
+    idx = dsa.indexer_topk(x.q_idx, x.w, x.k_idx, x.k, pos=x.pos, k_base=x.k_base)
+    out1, lse1 = dsa.sparse_mla_attn_split(x.q, x.kv, idx, x.scale, x.d_v, 1, pos=x.pos, k_base=x.k_base)
+    outs, lses = dsa.sparse_mla_attn_split(x.q, x.kv, idx, x.scale, x.d_v, splits, pos=x.pos,
+                                           k_base=x.k_base)
+    torch.cuda.synchronize()
+    assert dsa.device_status() == 0
+    rows = list(range(x.T))
+    h = host_inputs(x, rows)
+    check_attention(x, idx.cpu(), outs.cpu(), lses.cpu(), rows, h=h)
+    assert (out1.float() - outs.float()).abs().max().item() < 2e-2
+    assert (lse1 - lses).abs().max().item() < 1e-3
+
+
+def test_decode_64_sequences_split_launch():
+    """The 64-sequence decode step with its rows split in two (every row
+    against the oracle) and the library's own choice of parts."""
+    x = synth.decode_inputs("decode", device="cuda", seed=0)
+    idx = dsa.indexer_topk(x.q_idx, x.w, x.k_idx, x.k, pos=x.pos, k_base=x.k_base)
+    rows = list(range(x.T))
+    h = host_inputs(x, rows)
+    for splits in (0, 2):
+        out, lse = dsa.sparse_mla_attn_split(x.q, x.kv, idx, x.scale, x.d_v, splits, pos=x.pos,
+                                             k_base=x.k_base)
+        torch.cuda.synchronize()
+        check_attention(x, idx.cpu(), out.cpu(), lse.cpu(), rows, h=h)
 
 
 def test_invalid_entries_are_ignored():
@@ -188,13 +225,19 @@ def test_prefill4k_all_rows_indexer_sampled_attention():
     check_attention(x, _take(idx, srows), _take(out, srows), _take(lse, srows), srows)
 
 
+# Full-size configurations: 256 sampled query rows (rows 0, k-1, k, L-1 and a
+# seeded random set), every one checked for both the indexer and attention.
+N_SAMPLED = 256
+
+
 def test_prefill32k_integer_indexer_bit_exact_sampled():
     x = synth.prefill_inputs("prefill32k_int", device="cuda", seed=0)
     idx, out, lse = _run(x)
-    rows = _sampled(x.T, x.k, 160)
-    check_indexer(x, _take(idx, rows), rows, exact=True)
-    srows = rows[:: max(1, len(rows) // 12)]
-    check_attention(x, _take(idx, srows), _take(out, srows), _take(lse, srows), srows)
+    rows = _sampled(x.T, x.k, N_SAMPLED)
+    assert len(rows) == N_SAMPLED
+    h = host_inputs(x, rows)
+    check_indexer(x, _take(idx, rows), rows, exact=True, h=h)
+    check_attention(x, _take(idx, rows), _take(out, rows), _take(lse, rows), rows, h=h)
 
 
 def test_tail_prefill_last_rows_of_a_longer_sequence():
@@ -227,19 +270,23 @@ def test_prefill_threshold_overshoot_falls_back_exactly():
 def test_prefill32k_sampled():
     x = synth.prefill_inputs("prefill32k", device="cuda", seed=0)
     idx, out, lse = _run(x)
-    rows = _sampled(x.T, x.k, 48)
-    check_indexer(x, _take(idx, rows), rows, exact=False)
-    srows = rows[:: max(1, len(rows) // 12)]
-    check_attention(x, _take(idx, srows), _take(out, srows), _take(lse, srows), srows)
+    rows = _sampled(x.T, x.k, N_SAMPLED)
+    assert len(rows) == N_SAMPLED
+    h = host_inputs(x, rows)
+    check_indexer(x, _take(idx, rows), rows, exact=False, h=h)
+    check_attention(x, _take(idx, rows), _take(out, rows), _take(lse, rows), rows, h=h)
 
 
 def test_prefill128k_sampled():
+    """The 128K prefill in bench.py's launch configuration (one indexer call
+    over all 131072 rows, one attention call)."""
     x = synth.prefill_inputs("prefill128k", device="cuda", seed=0)
     idx, out, lse = _run(x)
-    rows = _sampled(x.T, x.k, 24)
-    check_indexer(x, _take(idx, rows), rows, exact=False)
-    srows = rows[:: max(1, len(rows) // 8)]
-    check_attention(x, _take(idx, srows), _take(out, srows), _take(lse, srows), srows)
+    rows = _sampled(x.T, x.k, N_SAMPLED)
+    assert len(rows) == N_SAMPLED
+    h = host_inputs(x, rows)
+    check_indexer(x, _take(idx, rows), rows, exact=False, h=h)
+    check_attention(x, _take(idx, rows), _take(out, rows), _take(lse, rows), rows, h=h)
     del x, idx, out, lse
     torch.cuda.empty_cache()
 
@@ -248,6 +295,39 @@ def test_decode_64_sequences():
     x = synth.decode_inputs("decode", device="cuda", seed=0)
     idx, out, lse = _run(x)
     rows = list(range(x.T))
-    check_indexer(x, idx.cpu(), rows, exact=False)
-    srows = rows[::4]
-    check_attention(x, _take(idx, srows), _take(out, srows), _take(lse, srows), srows)
+    h = host_inputs(x, rows)
+    check_indexer(x, idx.cpu(), rows, exact=False, h=h)
+    check_attention(x, idx.cpu(), out.cpu(), lse.cpu(), rows, h=h)
+
+
+def test_streaming_indexer_rows_are_ascending_and_repeatable():
+    """The streaming indexer writes each row in ascending s, the same on every
+    call (so attention over it sums in a fixed order and repeats bit for bit)."""
+    x = synth.prefill_inputs("prefill4k", device="cuda", seed=14, L=3000)
+    a = dsa.indexer_topk(x.q_idx, x.w, x.k_idx, x.k)
+    b = dsa.indexer_topk(x.q_idx, x.w, x.k_idx, x.k)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+    n = torch.clamp(x.positions().long() + 1, max=x.k)
+    v = a.long()
+    valid = torch.arange(x.k, device="cuda")[None, :] < n[:, None]
+    assert ((v[:, 1:] > v[:, :-1]) | ~valid[:, 1:]).all()
+    o1, l1 = dsa.sparse_mla_attn(x.q, x.kv, a, x.scale, x.d_v)
+    o2, l2 = dsa.sparse_mla_attn(x.q, x.kv, b, x.scale, x.d_v)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_phase_timing_reports_the_indexer_phases():
+    x = synth.prefill_inputs("prefill4k", device="cuda", seed=15)
+    dsa.phase_timing(True)
+    try:
+        dsa.indexer_topk(x.q_idx, x.w, x.k_idx, x.k)
+        torch.cuda.synchronize()
+        ph = dsa.phase_times()
+    finally:
+        dsa.phase_timing(False)
+    assert ph["scores"] > 0 and ph["threshold"] > 0 and ph["select"] > 0
+    dsa.indexer_topk(x.q_idx, x.w, x.k_idx, x.k)
+    torch.cuda.synchronize()
+    assert all(v == 0 for v in dsa.phase_times().values())   # off: nothing recorded

@@ -2,7 +2,8 @@
 give the library device memory (no workspace argument; its scratch is an
 array the library holds). Called through the C ABI and compared with
 dsa_indexer_topk on the same inputs, twice in a row, because the shared
-scratch keeps the previous call's contents. Collected last on purpose."""
+scratch keeps the previous call's contents, and with the CPU oracle.
+Collected last on purpose."""
 import ctypes
 
 import pytest
@@ -10,6 +11,7 @@ import torch
 
 import synth
 import sparse_attention_20_b200 as dsa
+from parity import check_indexer
 from sparse_attention_20_b200 import build as dsa_build
 
 STATIC_MAX_S = 4 << 20
@@ -55,3 +57,33 @@ def test_noalloc_matches_workspace_entry_point_twice(case):
         # each row is a set: compare in sorted order
         assert torch.equal(torch.sort(got, dim=1)[0], torch.sort(ref, dim=1)[0])
     assert dsa.device_status() == 0
+    # and against the oracle: exact sets on integer inputs, the tolerance rule
+    # on realistic ones (every row of the decode case, sampled prefill rows)
+    rows = list(range(T)) if case == "decode" else synth.sample_rows(T, x.k, 64, seed=3)
+    r = torch.tensor(rows, device=got.device)
+    check_indexer(x, got[r].cpu(), rows, exact=(case == "prefill"))
+
+
+@pytest.mark.gpu
+def test_noalloc_many_rows_over_few_keys():
+    """T = 70000 query rows over S = 64 keys: the scratch holds 65536 score
+    rows, so the call works through the rows in blocks of at most 65535 (the
+    grid's y limit); every row must still get its exact Top-k."""
+    dsa_build.build()
+    dsa.load_library()
+    x = synth.decode_inputs("decode", device="cuda", seed=23, B=1, ctx=[64],
+                            overrides=dict(indexer="int", k=16))
+    T = 70000
+    q_idx = x.q_idx.expand(T, -1, -1).contiguous()
+    w = synth.integers((T, x.w.shape[1]), -2, 2, 23, "noalloc_rows", "w", "cuda")
+    pos = synth.integers((T,), 0, 63, 23, "noalloc_rows", "pos", "cuda").to(torch.int32)
+    ref = dsa.indexer_topk(q_idx, w, x.k_idx, x.k, pos=pos)
+    got = dsa.indexer_topk_noalloc(q_idx, w, x.k_idx, x.k, pos=pos)
+    torch.cuda.synchronize()
+    assert dsa.device_status() == 0
+    assert torch.equal(torch.sort(got, dim=1)[0], torch.sort(ref, dim=1)[0])
+    rows = [0, 1, 65534, 65535, 65536, T - 1] + list(range(100, T, 7919))
+    r = torch.tensor(rows, device="cuda")
+    h = dict(q_idx=q_idx[r].cpu().numpy(), w=w[r].cpu().numpy(), k_idx=x.k_idx.cpu().numpy(),
+             pos=pos[r].cpu().numpy(), base=torch.zeros(len(rows), dtype=torch.int32).numpy())
+    check_indexer(x, got[r].cpu(), rows, exact=True, h=h)
