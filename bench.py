@@ -139,8 +139,9 @@ def shard_inputs(x, world: int, rank: int):
                                None, None, x.k, x.scale, x.d_v, dict(x.meta, rows=(t0, t1)))
     ctx = (x.positions() + 1).cpu().tolist()
     b0, b1 = shard_decode_seqs(world, rank, ctx, x.k, d_I, d_qk)
+    # pos / k_base slices are copied: the library wants 16-byte aligned arrays
     return synth.DSAInputs(x.config, x.q_idx[b0:b1], x.w[b0:b1], x.k_idx, x.q[b0:b1], x.kv,
-                           x.positions()[b0:b1], x.bases()[b0:b1], x.k, x.scale, x.d_v,
+                           x.positions()[b0:b1].clone(), x.bases()[b0:b1].clone(), x.k, x.scale, x.d_v,
                            dict(x.meta, rows=(b0, b1)))
 
 

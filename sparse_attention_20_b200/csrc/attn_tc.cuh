@@ -444,6 +444,9 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
             const int b = c & 1;
             const int xb = c % kXSlots;
             if (i == 0 && hs == 0) mbar_arrive_expect_tx(bar(B_XFULL + xb), kXBytes);
+            // the chunk's validity bits (its gather completed long before S(c))
+            if (!wait_w(bar(B_FULL + c % kStages), (c / kStages) & 1, 200 + B_FULL, c)) { ok = false; break; }
+            const uint32_t mw = smask[(c % kStages) * 2 + hs];
             // this CTA's partial logits of chunk c (fp32, TMEM)
             if (!wait_w(bar(B_SFULL + b), (c >> 1) & 1, 200 + B_SFULL, c)) { ok = false; break; }
             tc_fence_after();
@@ -465,8 +468,6 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_SFREE + b));   // S(c) fully read by this warp
-            if (!wait_w(bar(B_FULL + c % kStages), (c / kStages) & 1, 200 + B_FULL, c)) { ok = false; break; }
-            const uint32_t mw = smask[(c % kStages) * 2 + hs];
             // logit (log2 domain) = own partial (fp32) + peer partial (fp16); masked -> -inf
             float x[32];
 #pragma unroll

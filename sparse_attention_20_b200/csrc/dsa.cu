@@ -383,11 +383,14 @@ struct ChunkArgs {
 
 template <int NT, int DI>
 struct ChunkKernels {
-    static void sample(int grid, cudaStream_t st, const ChunkArgs& a, float* samp, long long samp_ld)
+    // plan + sampled scores + threshold in one launch
+    static void sample_tau(cudaStream_t st, const ChunkArgs& a, int* work_off, float* samp, long long samp_ld,
+                           uint32_t* tau)
     {
         using namespace dsa::idx_chunk;
-        launch_pdl(chunk_sample_kernel<NT, DI>, dim3(grid), dim3(kThreads), 0, st, a.q_idx, a.w, a.k_idx, a.pos,
-                   a.k_base, a.T, a.S, a.H_I, a.row0, a.rows, a.work_off, samp, samp_ld, a.pg);
+        launch_pdl(chunk_sample_tau_kernel<NT, DI>, dim3(a.rows), dim3(kFusedTauThreads), 0, st, a.q_idx, a.w,
+                   a.k_idx, a.pos, a.k_base, a.T, a.S, a.H_I, a.row0, a.rows, a.k, work_off, samp, samp_ld, tau,
+                   a.pg);
     }
     static void topk(int grid, cudaStream_t st, const ChunkArgs& a, const uint32_t* tau, uint2* cand,
                      long long cand_ld, int* ccnt, int max_chunks, int32_t* idx)
@@ -416,7 +419,7 @@ void chunk_topk_tma(int grid, cudaStream_t st, const CUtensorMap& tm_k, const Ch
 }
 
 struct ChunkFns {
-    void (*sample)(int, cudaStream_t, const ChunkArgs&, float*, long long);
+    void (*sample_tau)(cudaStream_t, const ChunkArgs&, int*, float*, long long, uint32_t*);
     void (*topk)(int, cudaStream_t, const ChunkArgs&, const uint32_t*, uint2*, long long, int*, int,
                  int32_t*);
     void (*topk_tma)(int, cudaStream_t, const CUtensorMap&, const ChunkArgs&, const uint32_t*, uint2*,
@@ -426,7 +429,7 @@ struct ChunkFns {
 template <int NT, int DI>
 ChunkFns chunk_fns()
 {
-    return {ChunkKernels<NT, DI>::sample, ChunkKernels<NT, DI>::topk,
+    return {ChunkKernels<NT, DI>::sample_tau, ChunkKernels<NT, DI>::topk,
             DI == 128 ? chunk_topk_tma<NT> : nullptr};
 }
 
@@ -493,15 +496,14 @@ int indexer_chunked(const uint8_t* q_idx, const float* w, const uint8_t* k_idx, 
             (long long)rows * std::max(1, dsa::ceil_div(n_max, kChunkKeys)), resident);
         const ChunkArgs a{q_idx, w, k_idx, pos, k_base, T, S, H_I, k, row0, rows, work_off, pg};
         PhaseMark ph = phase_begin(kPhaseThreshold, st);
-        launch_pdl(chunk_plan_kernel, dim3(1), dim3(kPlanThreads), 0, st, pos, k_base, T, S, row0, rows, work_off,
-                   pg);
-        DSA_LAUNCH_CHECK("chunk_plan_kernel");
         if (multi) {
-            fn.sample(grid, st, a, samp, p.samp_ld);
-            DSA_LAUNCH_CHECK("chunk_sample_kernel");
-            launch_pdl(chunk_tau_kernel<kTauThreads>, dim3(rows), dim3(kTauThreads), 0, st, samp, p.samp_ld, pos,
-                       k_base, T, S, row0, k, tau, pg);
-            DSA_LAUNCH_CHECK("chunk_tau_kernel");
+            // plan, sampled scores and threshold in one launch
+            fn.sample_tau(st, a, work_off, samp, p.samp_ld, tau);
+            DSA_LAUNCH_CHECK("chunk_sample_tau_kernel");
+        } else {
+            launch_pdl(chunk_plan_kernel, dim3(1), dim3(kPlanThreads), 0, st, pos, k_base, T, S, row0, rows,
+                       work_off, pg);
+            DSA_LAUNCH_CHECK("chunk_plan_kernel");
         }
         phase_end(ph);
         ph = phase_begin(kPhaseScores, st);
@@ -530,8 +532,8 @@ bool indexer_fused_supported(const int32_t* pos, const int32_t* k_base, int H_I,
     using namespace dsa::idx_tc;
     if (pos || k_base || H_I != kHI || d_I != kDI) return false;
     const size_t samp_bytes = (size_t)((num_tiles(S) + kSampleStride - 1) / kSampleStride) * kKeys * sizeof(float);
-    const size_t cand_bytes = (size_t)2 * kAlpha * k * sizeof(uint2) + (size_t)dsa::pow2_ceil(k) * sizeof(int);
-    return samp_bytes <= kFusedStageMax && cand_bytes <= kFusedStageMax;
+    const size_t bitmap_bytes = (size_t)std::max((S + 31) / 32, dsa::pow2_ceil(k)) * sizeof(uint32_t);
+    return samp_bytes <= kFusedStageMax && bitmap_bytes <= kFusedStageMax;
 }
 
 int make_tmap_u8(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t rows,
@@ -570,7 +572,10 @@ int indexer_fused(const uint8_t* q_idx, const float* w, const uint8_t* k_idx, in
     }
     // staged samples (tau) and candidates (select) of one row
     const size_t tau_smem = (size_t)p.samp_ld * sizeof(float);
-    const size_t sel_smem = (size_t)p.cap * sizeof(uint2) + (size_t)dsa::pow2_ceil(k) * sizeof(int);
+    // select: a bitmap over the row's keys (S bits), at least pow2_ceil(k)
+    // ints for the sort a longer row falls back to
+    const int bitmap_words = std::max((S + 31) / 32, dsa::pow2_ceil(k));
+    const size_t sel_smem = (size_t)bitmap_words * sizeof(uint32_t);
     {
         cudaError_t e = cudaFuncSetAttribute(indexer_tau_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)tau_smem);
@@ -598,7 +603,7 @@ int indexer_fused(const uint8_t* q_idx, const float* w, const uint8_t* k_idx, in
         // ~2k candidates per row: 256 threads keep the radix passes busy
         ph = phase_begin(kPhaseSelect, st);
         indexer_select_kernel<256><<<rows, 256, sel_smem, st>>>(cand, cnt, p.cap, q_idx, w, k_idx, T, S, k,
-                                                                row0, idx);
+                                                                row0, idx, bitmap_words);
         DSA_LAUNCH_CHECK("indexer_select_kernel");
         phase_end(ph);
     }

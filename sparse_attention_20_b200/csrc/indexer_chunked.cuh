@@ -39,7 +39,6 @@ constexpr int kCtasPerSm = 2;
 constexpr int kMergeThreads = 1024;
 constexpr int kMergeSmemPairs = 8192;   // 64 KB of staged (score, s) pairs
 constexpr int kPlanThreads = 1024;
-constexpr int kTauThreads = 512;
 constexpr int kTauSmemSamples = 6144;   // rows up to 24 chunks stage their samples
 constexpr size_t kSmemBytes = kChunkKeys * sizeof(float) + sizeof(SelectSmem<kThreads>);
 // sampling: tiles of 128 keys, every 32nd tile of a row (two per chunk)
@@ -127,48 +126,6 @@ __device__ __forceinline__ void score_chunk(const QueryFrag<NT, DI>& qf, const u
     }
 }
 
-// Sample tiles of every chunk of multi-chunk rows: samp[r * samp_ld +
-// chunk * kSamplesPerChunk + j]; positions beyond the row hold -inf. The
-// chunk's sample keys (two tiles of 128) are one 16-key block per warp.
-template <int NT, int DI>
-__global__ void __launch_bounds__(kThreads, kCtasPerSm)
-chunk_sample_kernel(const uint8_t* __restrict__ q_idx, const float* __restrict__ w,
-                    const uint8_t* __restrict__ k_idx, const int* __restrict__ pos,
-                    const int* __restrict__ k_base, int T, int S, int H_I, int row0, int rows,
-                    const int* __restrict__ work_off, float* __restrict__ samp, long long samp_ld,
-                    const PagedRows pg)
-{
-    static_assert(kSamplesPerChunk <= 16 * (kThreads / 32), "one 16-key block per warp");
-    griddep_wait();
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int gid = lane >> 2, tid4 = lane & 3;
-    const int total = work_off[rows];
-    for (int item = blockIdx.x; item < total; item += gridDim.x) {
-        const int r = item_row(work_off, rows, item), t = row0 + r;
-        const int chunk = item - work_off[r];
-        long long base;
-        const int* bt;
-        const int n = row_keys(pg, pos, k_base, t, T, S, &base, &bt);
-        const int j0 = warp * 16;   // this warp's sample positions [j0, j0 + 16)
-        if (row_chunks(n) < 2 || j0 >= kSamplesPerChunk) continue;
-        QueryFrag<NT, DI> qf;
-        qf.load(q_idx, w, t, H_I, lane);
-        // sample position j of this chunk: tile j / 128, key j % 128 of the tile
-        const int s0 = chunk * kChunkKeys + (j0 / kSampleTile) * kSampleStride + (j0 % kSampleTile);
-        const int sa = s0 + gid, sb = sa + 8;
-        KeyQuarter<DI> A, B;
-        if (sa < n) A.load(k_idx + (size_t)key_row(pg, bt, base, sa) * DI + tid4 * (DI / 4)); else A.zero();
-        if (sb < n) B.load(k_idx + (size_t)key_row(pg, bt, base, sb) * DI + tid4 * (DI / 4)); else B.zero();
-        float ia, ib;
-        qf.score(A, B, ia, ib);
-        if (tid4 == 0) {
-            float* out = samp + (size_t)r * samp_ld + (size_t)chunk * kSamplesPerChunk + j0;
-            out[gid] = sa < n ? ia : -INFINITY;
-            out[gid + 8] = sb < n ? ib : -INFINITY;
-        }
-    }
-}
-
 // Number of sampled positions inside a row of n keys.
 __device__ __forceinline__ int row_samples(int n)
 {
@@ -176,16 +133,55 @@ __device__ __forceinline__ int row_samples(int n)
     return full * kSampleTile + min(kSampleTile, n - full * kSampleStride);
 }
 
-// tau[r] = order key of the sample of rank ceil(kAlpha * k * m / n) (m valid
-// samples), or 0 (no filtering) where that rank is out of reach.
-template <int THREADS>
-__global__ void __launch_bounds__(THREADS)
-chunk_tau_kernel(const float* __restrict__ samp, long long samp_ld, const int* __restrict__ pos,
-                 const int* __restrict__ k_base, int T, int S, int row0, int k,
-                 uint32_t* __restrict__ tau, const PagedRows pg)
+// One CTA per row: the work plan of the chunk kernel (block 0, as
+// chunk_plan_kernel), then the row's sampled scores (every 32nd 128-key tile)
+// and its threshold tau[r] = the order key of the sample of rank
+// ceil(kAlpha * k * m / n) (m valid samples), or 0 (no filtering) where that
+// rank is out of reach. The samples of a row of up to 24 chunks (196608 keys,
+// every decode row of the 128K workload) stay in shared memory; a longer
+// row's go to samp[r * samp_ld ...] in global memory.
+constexpr int kFusedTauThreads = 512;
+
+template <int NT, int DI>
+__global__ void __launch_bounds__(kFusedTauThreads)
+chunk_sample_tau_kernel(const uint8_t* __restrict__ q_idx, const float* __restrict__ w,
+                        const uint8_t* __restrict__ k_idx, const int* __restrict__ pos,
+                        const int* __restrict__ k_base, int T, int S, int H_I, int row0, int rows, int k,
+                        int* __restrict__ work_off, float* __restrict__ samp, long long samp_ld,
+                        uint32_t* __restrict__ tau, const PagedRows pg)
 {
-    __shared__ SelectSmem<THREADS> sm;
+    __shared__ SelectSmem<kFusedTauThreads> sm;
+    __shared__ float ss[kTauSmemSamples];
+    __shared__ int part[kFusedTauThreads];
     griddep_wait();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int gid = lane >> 2, tid4 = lane & 3;
+    if (blockIdx.x == 0) {
+        // work_off[r] = work items of rows row0 .. row0+r-1 (chunk_plan_kernel)
+        const int per = ceil_div(rows, kFusedTauThreads);
+        const int a0 = threadIdx.x * per, a1 = min(rows, a0 + per);
+        auto items = [&](int r) -> int {
+            long long base;
+            const int* bt;
+            return row_chunks(row_keys(pg, pos, k_base, row0 + r, T, S, &base, &bt));
+        };
+        int sum = 0;
+        for (int r = a0; r < a1; ++r) sum += items(r);
+        part[threadIdx.x] = sum;
+        __syncthreads();
+        for (int off = 1; off < kFusedTauThreads; off <<= 1) {
+            const int v = threadIdx.x >= off ? part[threadIdx.x - off] : 0;
+            __syncthreads();
+            part[threadIdx.x] += v;
+            __syncthreads();
+        }
+        int acc = part[threadIdx.x] - sum;
+        for (int r = a0; r < a1; ++r) {
+            work_off[r] = acc;
+            acc += items(r);
+        }
+        if (threadIdx.x == kFusedTauThreads - 1) work_off[rows] = part[kFusedTauThreads - 1];
+    }
     const int r = blockIdx.x, t = row0 + r;
     long long base;
     const int* bt;
@@ -198,19 +194,42 @@ chunk_tau_kernel(const float* __restrict__ samp, long long samp_ld, const int* _
         if (threadIdx.x == 0) tau[r] = 0u;
         return;
     }
-    // the row's samples, staged in shared memory when they fit
-    __shared__ float ss[kTauSmemSamples];
-    const float* src = samp + (size_t)r * samp_ld;
-    int take_eq, count_eq;
-    uint32_t key;
-    if (n_s <= kTauSmemSamples) {
-#pragma unroll 4
-        for (int j = threadIdx.x; j < n_s; j += THREADS) ss[j] = src[j];
-        __syncthreads();
-        key = radix_kth_key<THREADS>(SmemScores{ss, 0}, n_s, (int)want, sm, &take_eq, &count_eq);
-    } else {
-        key = radix_kth_key<THREADS>(DenseScores{src}, n_s, (int)want, sm, &take_eq, &count_eq);
+    float* dst = n_s <= kTauSmemSamples ? ss : samp + (size_t)r * samp_ld;
+    // sample position j: chunk j / 256, tile (j % 256) / 128 of the chunk's
+    // every-32nd tiles, key j % 128; each warp scores 16 consecutive positions
+    // per step, with the loads of two steps issued before their MMAs
+    QueryFrag<NT, DI> qf;
+    qf.load(q_idx, w, t, H_I, lane);
+    constexpr int kStep = 16 * (kFusedTauThreads / 32);
+    auto key_of = [&](int j) -> int {
+        const int c = j / kSamplesPerChunk, jj = j % kSamplesPerChunk;
+        return c * kChunkKeys + (jj / kSampleTile) * kSampleStride + jj % kSampleTile;
+    };
+    for (int j0 = warp * 16; j0 < n_s; j0 += 2 * kStep) {
+        KeyQuarter<DI> A[2], B[2];
+        int sa[2], sb[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int ja = j0 + u * kStep + gid;
+            sa[u] = ja < n_s ? key_of(ja) : n;
+            sb[u] = ja + 8 < n_s ? key_of(ja + 8) : n;
+            if (sa[u] < n) A[u].load(k_idx + (size_t)key_row(pg, bt, base, sa[u]) * DI + tid4 * (DI / 4)); else A[u].zero();
+            if (sb[u] < n) B[u].load(k_idx + (size_t)key_row(pg, bt, base, sb[u]) * DI + tid4 * (DI / 4)); else B[u].zero();
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            float ia, ib;
+            qf.score(A[u], B[u], ia, ib);
+            const int ja = j0 + u * kStep + gid;
+            if (tid4 == 0) {
+                if (ja < n_s) dst[ja] = sa[u] < n ? ia : -INFINITY;
+                if (ja + 8 < n_s) dst[ja + 8] = sb[u] < n ? ib : -INFINITY;
+            }
+        }
     }
+    __syncthreads();
+    int take_eq, count_eq;
+    const uint32_t key = radix_kth_key<kFusedTauThreads>(DenseScores{dst}, n_s, (int)want, sm, &take_eq, &count_eq);
     if (threadIdx.x == 0) tau[r] = key;
 }
 

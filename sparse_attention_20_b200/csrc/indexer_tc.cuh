@@ -31,6 +31,8 @@
 #include "sm100.cuh"
 #include "topk_select.cuh"
 
+#include <type_traits>
+
 namespace dsa {
 namespace idx_tc {
 
@@ -202,6 +204,10 @@ indexer_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             if (!__all_sync(0xffffffffu, got)) break;
             tc_fence_after();
             const int s = it * tile_step * kKeys + key_lane;     // this thread's key
+            // every row of the CTA exists and sees every key of this warp: no
+            // per-row validity test (the common case on long rows)
+            const bool full = r0 + kRows <= a.rows &&
+                              it * tile_step * kKeys + (warp & 3) * 32 + 31 <= t0 + shift;
             // eight rows at a time: two TMEM loads (4 rows x 8 heads each), the
             // weighted ReLU head-sums, then the rows' mask / sample / filter step
 #pragma unroll 1
@@ -216,33 +222,51 @@ indexer_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     __syncwarp();
                     if (lane == 0) mbar_arrive(bar(B_DEMPTY + g));
                 }
+                auto rows8 = [&](auto full_tag) {
+                    constexpr bool kFull = decltype(full_tag)::value;
+                    float accs[8];
+                    uint32_t pass = 0u;                        // bit rr: row q8 * 4 + rr passes
 #pragma unroll
-                for (int rr = 0; rr < 8; ++rr) {
-                    const uint32_t* v = rr < 4 ? v0 : v1;
-                    const int rb = (rr & 3) * 8;
-                    const int r = q8 * 4 + rr;
-                    const float4 wa = *reinterpret_cast<const float4*>(w_s + r * kHI);
-                    const float4 wb = *reinterpret_cast<const float4*>(w_s + r * kHI + 4);
-                    float acc = wa.x * fmaxf(__uint_as_float(v[rb + 0]), 0.f);
-                    acc = fmaf(wa.y, fmaxf(__uint_as_float(v[rb + 1]), 0.f), acc);
-                    acc = fmaf(wa.z, fmaxf(__uint_as_float(v[rb + 2]), 0.f), acc);
-                    acc = fmaf(wa.w, fmaxf(__uint_as_float(v[rb + 3]), 0.f), acc);
-                    acc = fmaf(wb.x, fmaxf(__uint_as_float(v[rb + 4]), 0.f), acc);
-                    acc = fmaf(wb.y, fmaxf(__uint_as_float(v[rb + 5]), 0.f), acc);
-                    acc = fmaf(wb.z, fmaxf(__uint_as_float(v[rb + 6]), 0.f), acc);
-                    acc = fmaf(wb.w, fmaxf(__uint_as_float(v[rb + 7]), 0.f), acc);
-                    const int rl = r0 + r;                   // launch-relative row
-                    const int t = t0 + r;
-                    const bool valid = rl < a.rows && t < a.T && s <= t + shift && s < a.S;
-                    if (kSample) {
-                        if (rl < a.rows)
-                            a.samp[(size_t)rl * a.samp_ld + it * kKeys + key_lane] = valid ? acc : -INFINITY;
-                    } else if (valid && acc >= tau_s[r]) {
-                        const int slot = atomicAdd(&cnt_s[r], 1);
-                        if (slot < a.cap)
-                            a.cand[(size_t)rl * a.cap + slot] = make_uint2(__float_as_uint(acc), (uint32_t)s);
+                    for (int rr = 0; rr < 8; ++rr) {
+                        const uint32_t* v = rr < 4 ? v0 : v1;
+                        const int rb = (rr & 3) * 8;
+                        const int r = q8 * 4 + rr;
+                        const float4 wa = *reinterpret_cast<const float4*>(w_s + r * kHI);
+                        const float4 wb = *reinterpret_cast<const float4*>(w_s + r * kHI + 4);
+                        float acc = wa.x * fmaxf(__uint_as_float(v[rb + 0]), 0.f);
+                        acc = fmaf(wa.y, fmaxf(__uint_as_float(v[rb + 1]), 0.f), acc);
+                        acc = fmaf(wa.z, fmaxf(__uint_as_float(v[rb + 2]), 0.f), acc);
+                        acc = fmaf(wa.w, fmaxf(__uint_as_float(v[rb + 3]), 0.f), acc);
+                        acc = fmaf(wb.x, fmaxf(__uint_as_float(v[rb + 4]), 0.f), acc);
+                        acc = fmaf(wb.y, fmaxf(__uint_as_float(v[rb + 5]), 0.f), acc);
+                        acc = fmaf(wb.z, fmaxf(__uint_as_float(v[rb + 6]), 0.f), acc);
+                        acc = fmaf(wb.w, fmaxf(__uint_as_float(v[rb + 7]), 0.f), acc);
+                        const int rl = r0 + r;                   // launch-relative row
+                        const int t = t0 + r;
+                        const bool valid = kFull || (rl < a.rows && t < a.T && s <= t + shift && s < a.S);
+                        if (kSample) {
+                            if (kFull || rl < a.rows)
+                                a.samp[(size_t)rl * a.samp_ld + it * kKeys + key_lane] = valid ? acc : -INFINITY;
+                        } else {
+                            accs[rr] = acc;
+                            if (valid && acc >= tau_s[r]) pass |= 1u << rr;
+                        }
                     }
-                }
+                    // the rows' appends, once per eight rows (about 3% of the
+                    // pairs pass on long rows)
+                    if (!kSample) {
+                        while (pass) {
+                            const int rr = __ffs(pass) - 1;
+                            pass &= pass - 1u;
+                            const int r = q8 * 4 + rr;
+                            const int slot = atomicAdd(&cnt_s[r], 1);
+                            if (slot < a.cap)
+                                a.cand[(size_t)(r0 + r) * a.cap + slot] =
+                                    make_uint2(__float_as_uint(accs[rr]), (uint32_t)s);
+                        }
+                    }
+                };
+                if (full) rows8(std::true_type{}); else rows8(std::false_type{});
             }
         }
     }
@@ -332,25 +356,27 @@ struct RecomputedScores {
 
 // Candidate buffer of a row viewed as one array.
 struct CandScores {
-    const uint2* p;
+    const uint2* p;    // the row's candidate pairs
     __device__ __forceinline__ uint32_t key(int i) const { return score_key(__uint_as_float(p[i].x)); }
     __device__ __forceinline__ int s(int i) const { return (int)p[i].y; }
 };
 
-// The row's candidates are staged in shared memory (dynamic: cap pairs, then
-// pow2_ceil(k) ints) so the radix passes read them once from global memory.
 // The candidates arrive in no fixed order (appended by the scan's atomics), so
-// the selected set is sorted before it is written: every row comes out in
-// ascending s, deterministically (and attention over it sums in a fixed order).
+// the selected set is not written in the order it is found: each selected s
+// sets its bit in a shared-memory bitmap over the row's keys (dynamic shared
+// memory, bitmap_words words), and the row is written from the bitmap in
+// ascending s, deterministically (attention over it then sums in a fixed
+// order). A row longer than the bitmap sorts its k values instead
+// (bitmap_words >= k required for that buffer).
 template <int THREADS>
 __global__ void __launch_bounds__(THREADS)
 indexer_select_kernel(const uint2* __restrict__ cand, const int* __restrict__ cnt, int cap,
                       const uint8_t* __restrict__ q_idx, const float* __restrict__ w,
                       const uint8_t* __restrict__ k_idx, int T, int S, int k, int row0,
-                      int32_t* __restrict__ idx)
+                      int32_t* __restrict__ idx, int bitmap_words)
 {
     __shared__ SelectSmem<THREADS> sm;
-    extern __shared__ uint2 staged[];
+    extern __shared__ uint32_t bitmap[];
     __shared__ float qf[kHI * kDI];
     __shared__ float wf[kHI];
     const int rl = blockIdx.x;
@@ -363,16 +389,25 @@ indexer_select_kernel(const uint2* __restrict__ cand, const int* __restrict__ cn
     }
     const int c = cnt[rl];
     if (c >= k && c <= cap) {
-        const uint4* src = reinterpret_cast<const uint4*>(cand + (size_t)rl * cap);
-        for (int i = threadIdx.x; i < c / 2; i += THREADS) reinterpret_cast<uint4*>(staged)[i] = src[i];
-        if ((c & 1) && threadIdx.x == 0) staged[c - 1] = cand[(size_t)rl * cap + c - 1];
-        __syncthreads();
-        int* sel = reinterpret_cast<int*>(staged + cap);
-        const CandScores row{staged};
-        block_select<THREADS>(row, c, k, [&](int slot, int i) { sel[slot] = row.s(i); }, sm);
-        __syncthreads();
-        block_sort_ascending(sel, k, pow2_ceil(k));
-        for (int i = threadIdx.x; i < k; i += THREADS) out[i] = sel[i];
+        const CandScores row{cand + (size_t)rl * cap};
+        if (n <= bitmap_words * 32) {
+            for (int i = threadIdx.x; i < (n + 31) / 32; i += THREADS) bitmap[i] = 0u;
+            __syncthreads();
+            block_select<THREADS>(row, c, k,
+                                  [&](int, int i) {
+                                      const int s = row.s(i);
+                                      atomicOr(&bitmap[s >> 5], 1u << (s & 31));
+                                  },
+                                  sm);
+            __syncthreads();
+            block_emit_bitmap<THREADS>(bitmap, n, out, reinterpret_cast<int*>(sm.hist[0]));
+        } else {
+            int* sel = reinterpret_cast<int*>(bitmap);
+            block_select<THREADS>(row, c, k, [&](int slot, int i) { sel[slot] = row.s(i); }, sm);
+            __syncthreads();
+            block_sort_ascending(sel, k, pow2_ceil(k));
+            for (int i = threadIdx.x; i < k; i += THREADS) out[i] = sel[i];
+        }
         return;
     }
     // threshold too high (fewer than k candidates) or buffer overflow: exact

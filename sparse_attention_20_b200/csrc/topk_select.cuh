@@ -269,6 +269,34 @@ __device__ __forceinline__ void block_sort_ascending(int* v, int n, int cap)
         }
 }
 
+// Writes the positions of the set bits of bm (words covering [0, n)) to
+// out[0..) in ascending order: every thread emits the set bits of its run of
+// words at an offset from a block-wide prefix of their counts. warp_sums
+// holds THREADS / 32 ints of shared memory. Every thread of the CTA takes
+// part.
+template <int THREADS>
+__device__ void block_emit_bitmap(const uint32_t* bm, int n, int* out, int* warp_sums)
+{
+    const int words = (n + 31) >> 5;
+    const int per = (words + THREADS - 1) / THREADS;
+    const int w0 = min(words, (int)threadIdx.x * per), w1 = min(words, w0 + per);
+    int cnt = 0;
+    for (int i = w0; i < w1; ++i) cnt += __popc(bm[i]);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    int incl = cnt;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += v;
+    }
+    if (lane == 31) warp_sums[warp] = incl;
+    __syncthreads();
+    int pos = incl - cnt;
+    for (int q = 0; q < warp; ++q) pos += warp_sums[q];
+    for (int i = w0; i < w1; ++i)
+        for (uint32_t b = bm[i]; b; b &= b - 1u) out[pos++] = (i << 5) + __ffs(b) - 1;
+}
+
 __host__ __device__ __forceinline__ int pow2_ceil(int x)
 {
     int p = 1;

@@ -331,3 +331,14 @@ def test_phase_timing_reports_the_indexer_phases():
     dsa.indexer_topk(x.q_idx, x.w, x.k_idx, x.k)
     torch.cuda.synchronize()
     assert all(v == 0 for v in dsa.phase_times().values())   # off: nothing recorded
+
+
+def test_decode_rows_beyond_the_fused_threshold_path():
+    """Rows longer than 24 chunks of 8192 keys keep their sampled scores in
+    global memory (shorter rows in shared memory); both kinds in one call,
+    integer inputs, bit-exact."""
+    x = synth.decode_inputs("decode", device="cuda", seed=16, B=3, ctx=[200000, 9000, 300001],
+                            overrides=dict(indexer="int", k=2048))
+    idx = dsa.indexer_topk(x.q_idx, x.w, x.k_idx, x.k, pos=x.pos, k_base=x.k_base)
+    torch.cuda.synchronize()
+    check_indexer(x, idx.cpu(), list(range(x.T)), exact=True)
