@@ -320,7 +320,7 @@ def profiled_traffic(profile: str, key: str, sources) -> float | None:
 
 def attn_traffic():
     """DRAM bytes per prefill attention launch (128K workload)."""
-    return profiled_traffic("dram_bench_prefill128k_decode64.md", "attn",
+    return profiled_traffic("sparse_mla_attn_tc_prefill128k.md", "attn",
                             ("attn_tc.cuh", "sm100.cuh", "common.cuh", "dsa.cu"))
 
 
