@@ -393,12 +393,13 @@ indexer_select_kernel(const uint2* __restrict__ cand, const int* __restrict__ cn
         if (n <= bitmap_words * 32) {
             for (int i = threadIdx.x; i < (n + 31) / 32; i += THREADS) bitmap[i] = 0u;
             __syncthreads();
-            block_select<THREADS>(row, c, k,
-                                  [&](int, int i) {
-                                      const int s = row.s(i);
-                                      atomicOr(&bitmap[s >> 5], 1u << (s & 31));
-                                  },
-                                  sm);
+            if (!range_select_bitmap<THREADS>(row, c, k, bitmap, sm))
+                block_select<THREADS>(row, c, k,
+                                      [&](int, int i) {
+                                          const int s = row.s(i);
+                                          atomicOr(&bitmap[s >> 5], 1u << (s & 31));
+                                      },
+                                      sm);
             __syncthreads();
             block_emit_bitmap<THREADS>(bitmap, n, out, reinterpret_cast<int*>(sm.hist[0]));
         } else {

@@ -232,6 +232,119 @@ __device__ void block_select(const Row& row, int n, int k, const Emit& emit, Sel
         emit, k, sm);
 }
 
+// Exact Top-k of `row` (n >= k entries; order: key descending, then s
+// ascending) marked in a bitmap over s, in three reads of the row: the key
+// range, a histogram of kRangeBins equal-width bins over that range, and a
+// pass that marks every entry of a bin above the one holding the k-th entry
+// and collects that bin's entries, which are then ranked in shared memory.
+// Returns false, with the bitmap untouched, when every key is equal or the
+// boundary bin holds more than kRangeListCap entries (the caller then takes
+// the radix path). The caller synchronises before reading the bitmap.
+constexpr int kRangeBins = 2048;
+constexpr int kRangeListCap = 128;   // uint2 entries in SelectSmem::total
+
+template <int THREADS, class Row>
+__device__ bool range_select_bitmap(const Row& row, int n, int k, uint32_t* bm, SelectSmem<THREADS>& sm)
+{
+    constexpr int W = THREADS / 32;
+    constexpr int PER = kRangeBins / THREADS;
+    static_assert(W * 256 >= kRangeBins && kRangeBins % THREADS == 0, "histogram space");
+    static_assert(2 * kRangeListCap <= 256 && 2 * W <= 256, "list space");
+    __shared__ uint32_t wsum[W];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    uint32_t* h = &sm.hist[0][0];
+    // 1. key range
+    uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+    for (int i = tid; i < n; i += THREADS) {
+        const uint32_t key = row.key(i);
+        lo = min(lo, key);
+        hi = max(hi, key);
+    }
+#pragma unroll
+    for (int off = 16; off; off >>= 1) {
+        lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, off));
+        hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, off));
+    }
+    if (lane == 0) {
+        sm.total[warp] = lo;
+        sm.total[W + warp] = hi;
+    }
+    for (int b = tid; b < kRangeBins; b += THREADS) h[b] = 0u;
+    __syncthreads();
+    lo = sm.total[0];
+    hi = sm.total[W];
+#pragma unroll
+    for (int w = 1; w < W; ++w) {
+        lo = min(lo, sm.total[w]);
+        hi = max(hi, sm.total[W + w]);
+    }
+    if (lo == hi) return false;
+    const int shift = max(0, 32 - __clz(hi - lo) - 11);   // (hi - lo) >> shift < 2048
+    // 2. histogram
+    for (int i = tid; i < n; i += THREADS) atomicAdd(&h[(row.key(i) - lo) >> shift], 1u);
+    __syncthreads();
+    // 3. the bin of the k-th entry from the top: thread j owns the PER bins
+    //    just below the top j * PER
+    uint32_t c[PER], local = 0u;
+#pragma unroll
+    for (int j = 0; j < PER; ++j) {
+        c[j] = h[kRangeBins - 1 - (tid * PER + j)];
+        local += c[j];
+    }
+    uint32_t incl = local;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += v;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    if (tid == 0) sm.counter[0] = 0;
+    __syncthreads();
+    uint32_t before = incl - local;
+    for (int w = 0; w < warp; ++w) before += wsum[w];
+    if (before < (uint32_t)k && before + local >= (uint32_t)k) {
+        uint32_t cum = before;
+#pragma unroll
+        for (int j = 0; j < PER; ++j) {
+            if (cum + c[j] >= (uint32_t)k) {
+                sm.misc[0] = kRangeBins - 1 - (tid * PER + j);
+                sm.misc[1] = k - (int)cum;
+                sm.misc[2] = (int)c[j];
+                break;
+            }
+            cum += c[j];
+        }
+    }
+    __syncthreads();
+    const uint32_t kb = (uint32_t)sm.misc[0];
+    const int need = sm.misc[1], inb = sm.misc[2];
+    if (inb > kRangeListCap) return false;
+    // 4. mark the entries above bin kb, collect bin kb
+    uint2* list = reinterpret_cast<uint2*>(sm.total);
+    for (int i = tid; i < n; i += THREADS) {
+        const uint32_t key = row.key(i);
+        const uint32_t b = (key - lo) >> shift;
+        if (b > kb) {
+            const uint32_t s = (uint32_t)row.s(i);
+            atomicOr(&bm[s >> 5], 1u << (s & 31));
+        } else if (b == kb) {
+            list[atomicAdd(&sm.counter[0], 1)] = make_uint2(key, (uint32_t)row.s(i));
+        }
+    }
+    __syncthreads();
+    // 5. the first `need` entries of the bin by (key descending, s ascending)
+    for (int j = tid; j < inb; j += THREADS) {
+        const uint2 e = list[j];
+        int rank = 0;
+        for (int q = 0; q < inb; ++q) {
+            const uint2 f = list[q];
+            rank += (f.x > e.x) || (f.x == e.x && f.y < e.y);
+        }
+        if (rank < need) atomicOr(&bm[e.y >> 5], 1u << (e.y & 31));
+    }
+    return true;
+}
+
 // Writes the Top-k of `row` (n entries) to out[0..k) in storage order; slots
 // beyond n (n < k) get -1.
 template <int THREADS, class G = CtaGroup, class Row>

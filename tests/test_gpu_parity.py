@@ -267,6 +267,29 @@ def test_prefill_threshold_overshoot_falls_back_exactly():
     check_indexer(x, _take(idx, rows), rows, exact=True)
 
 
+def test_prefill_select_ties_take_the_radix_path_exactly():
+    """The prefill Top-k select ranks a row's candidates through a histogram
+    over their key range and falls back to the radix select when every
+    candidate ties or the bin holding the k-th entry holds more than 128
+    entries. Keys repeating four distinct rows give four distinct scores per
+    query row (boundary bins of hundreds of ties); keys all equal give rows
+    whose candidates all tie. Either way the result is the oracle's Top-k
+    (ties to the lowest s)."""
+    for distinct, seed in ((4, 13), (1, 14)):
+        x = synth.prefill_inputs("prefill32k_int", device="cuda", seed=seed, L=6144)
+        s = torch.arange(x.S, device=x.k_idx.device)
+        x.k_idx[:] = x.k_idx[s % distinct]
+        idx = dsa.indexer_topk(x.q_idx, x.w, x.k_idx, x.k)
+        torch.cuda.synchronize()
+        rows = _sampled(x.T, x.k, 24) + [x.k, x.k + 1, 4095, x.T - 1]
+        check_indexer(x, _take(idx, rows), rows, exact=True)
+        if distinct == 1:
+            # every score equal: the lowest k positions, in ascending order
+            want = torch.arange(x.k, dtype=torch.int32)
+            for t in (x.k, 4095, x.T - 1):
+                assert torch.equal(idx[t].cpu(), want)
+
+
 def test_prefill32k_sampled():
     x = synth.prefill_inputs("prefill32k", device="cuda", seed=0)
     idx, out, lse = _run(x)
