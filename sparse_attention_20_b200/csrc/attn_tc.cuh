@@ -27,17 +27,27 @@
 // section "2.3 Inference Costs": decoding reads the cache, so the work of one
 // query token is spread over more SMs).
 //
+// The kernel is persistent: one cluster per pair of SMs walks the work units
+// (row, part) cid, cid + clusters, ... in order of decreasing row length. Every
+// per-chunk barrier counts chunks across units, so the gather ring, the QK
+// MMAs and the exchange run on into the next unit while the softmax warps
+// finish the current one (its last chunk, the row-sum exchange, the
+// epilogue): the per-row setup (barriers, TMEM, the first gathers and Q
+// loads) is paid once per cluster, not once per row.
+//
 // Warp roles (512 threads per CTA): warp 0 allocates TMEM and issues the QK
-// and PV MMAs (one thread polling both kinds of readiness, so a late chunk
-// never holds back the PV of the previous one); warps 1-3 load Q (TMA tiles)
-// and gather the selected rows with 16-byte cp.async into 128B/64B-swizzled
-// shared memory (4-stage ring of 64-row chunks; completion is counted on the
-// stage's mbarrier, so the gather runs up to four chunks ahead); warps 12-15
+// and PV MMAs and the Q TMA loads (one thread polling every kind of
+// readiness, so a late chunk never holds back the PV of the previous one);
+// warps 1-3 gather the selected rows with 16-byte cp.async into
+// 128B/64B-swizzled shared memory (4-stage ring of 64-row chunks; completion
+// is counted on the stage's mbarrier, so the gather runs up to four chunks
+// ahead); warps 12-15
 // (one per TMEM lane quarter) run the exchange: they stage the chunk's fp16
 // partial logits locally and send them with one bulk copy per warp into the
 // peer's shared memory, counted on the peer's mbarrier; warps 4-11 (two per
-// lane quarter, each taking 32 of a chunk's 64 keys) run the softmax and the
-// epilogue.
+// lane quarter, each taking 32 of a chunk's 64 keys) run the softmax, write
+// the next unit's latent Q columns into TMEM once the current unit's last
+// QK has completed, and run the epilogue.
 // Shared memory per CTA: Q 40 KB (latent columns 128..255 of the slice and the
 // rope slice) + 4 x 36 KB ring + 16 KB receive slot + 16 KB staging.
 // TMEM: O cols [0,256), S double buffer [256,384), latent Q [384,448), P
@@ -83,8 +93,8 @@ constexpr int kOffXS = kOffX + kXSlots * kXBytes;         // staging of outgoing
 constexpr int kOffBar = kOffXS + kXSlots * kXBytes;
 constexpr int kOffMask = kOffBar + 256;                 // [kStages][2] validity bits
 constexpr int kOffRed = kOffMask + 64;                  // [2 parity][2 halves][128] row maxima
-constexpr int kOffLsum = kOffRed + 2 * 2 * kHeads * 4;  // [2 halves][128] row sums
-constexpr int kOffRows = kOffLsum + 2 * kHeads * 4;     // [3 gather warps][64] row byte offsets
+constexpr int kOffLsum = kOffRed + 2 * 2 * kHeads * 4;  // [2 unit parities][2 halves][128] row sums
+constexpr int kOffRows = kOffLsum + 2 * 2 * kHeads * 4;     // [3 gather warps][64] row byte offsets
 constexpr int kSmemBytes = kOffRows + 3 * kKeys * 8 + 1024;  // + 1 KB alignment slack
 
 constexpr uint32_t kTmemCols = 512;
@@ -134,6 +144,33 @@ __device__ __forceinline__ bool wait_warp(uint32_t b_addr, uint32_t par, volatil
     return __all_sync(0xffffffffu, mbar_wait(b_addr, par, abort_flag, tag, c));
 }
 
+// A work unit of the persistent kernel: part `part` of query row t's
+// selected set (unit u: t = T-1-u/splits, long rows first).
+struct Unit {
+    int t, part, e0, n_row, NC, p_last;
+    long long base;
+    const int* bt;   // block-table line of a paged cache, else NULL
+};
+
+__device__ __forceinline__ Unit unit_of(int u, const PagedRows& pg, const int* pos, const int* k_base, int T,
+                                        int S, int k, int splits)
+{
+    Unit w;
+    w.t = T - 1 - u / splits;
+    w.part = u % splits;
+    const int n_cand = row_keys(pg, pos, k_base, w.t, T, S, &w.base, &w.bt);
+    w.p_last = n_cand - 1;
+    // this unit's entries of the row: chunks [c0, c1) of its ceil(n/64)
+    const int n_all = min(k, n_cand);
+    const int nc_all = ceil_div(n_all, kKeys);
+    const int c0 = (int)((long long)nc_all * w.part / splits);
+    const int c1 = (int)((long long)nc_all * (w.part + 1) / splits);
+    w.e0 = c0 * kKeys;
+    w.n_row = max(0, min(c1 * kKeys, n_all) - w.e0);
+    w.NC = ceil_div(w.n_row, kKeys);
+    return w;
+}
+
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
                           const __grid_constant__ CUtensorMap tm_q64,
@@ -157,21 +194,12 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
     const uint32_t rank = cluster_ctarank();
     const uint32_t peer = rank ^ 1u;
     griddep_wait();
-    const int cid = (int)(blockIdx.x >> 1);
-    const int t = T - 1 - cid / splits;             // long rows first
-    const int part = cid % splits;
-    long long base;
-    const int* bt;   // block-table line of a paged cache, else NULL
-    const int n_cand = row_keys(pg, pos, k_base, t, T, S, &base, &bt);
-    const int p_last = n_cand - 1;
-    // this cluster's entries of the row: chunks [c0, c1) of its ceil(n/64)
-    const int n_all = min(k, n_cand);
-    const int nc_all = ceil_div(n_all, kKeys);
-    const int c0 = (int)((long long)nc_all * part / splits);
-    const int c1 = (int)((long long)nc_all * (part + 1) / splits);
-    const int e0 = c0 * kKeys;
-    const int n_row = max(0, min(c1 * kKeys, n_all) - e0);
-    const int NC = ceil_div(n_row, kKeys);
+    // units cid, cid + ncl, ... of the T * splits (every role walks the same
+    // sequence; per-chunk barrier phases count chunks across units)
+    const int cid = (int)(blockIdx.x >> 1), ncl = (int)(gridDim.x >> 1);
+    const int n_units_all = T * splits;
+    const int n_units = cid < n_units_all ? (n_units_all - cid + ncl - 1) / ncl : 0;
+    auto unit = [&](int j) -> Unit { return unit_of(cid + j * ncl, pg, pos, k_base, T, S, k, splits); };
 
     if (threadIdx.x == 0) {
         mbar_init(bar(B_Q), 1);
@@ -208,31 +236,63 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
     tc_fence_after();
     const uint32_t tmem = *taddr_slot;
     const uint32_t qs = sbase + kOffQ;
+    bool issued_any = false;
 
     if (warp == 0) {
         // ------------------------------------------------- QK and PV MMAs
-        // One thread issues both: QK(c) once chunk c is gathered and its S
-        // buffer has been read (chunk c-2), PV(c) once the softmax has written
-        // P(c). Readiness is polled without blocking so that neither kind of
-        // MMA waits behind the other; the tensor pipe runs them in issue order.
-        if (lane == 0 && NC > 0) {
+        // One thread issues both: QK(g) once chunk g is gathered and its S
+        // buffer has been read (chunk g-2), PV(g) once the softmax has written
+        // P(g); g counts chunks across this cluster's units. The Q tiles of a
+        // unit are loaded once every QK of the previous unit has completed.
+        // Readiness is polled without blocking so that neither kind of MMA
+        // waits behind the other; the tensor pipe runs them in issue order.
+        if (lane == 0) {
+            prefetch_tmap(&tm_q128);
+            prefetch_tmap(&tm_q64);
             const uint32_t id_qk = idesc_bf16(128, kKeys, false);
             const uint32_t id_pv = idesc_bf16(128, 256, true);
-            bool ok = mbar_wait(bar(B_Q), 0, abort_flag, B_Q, 0) &&
-                      mbar_wait(bar(B_QT), 0, abort_flag, B_QT, 0);
-            int cq = 0, cp = 0;              // next chunk for QK / for PV
+            bool ok = true;
+            Unit qu{}, pu{};
+            int qj = 0, qc = 0, qg = 0, qq = 0;   // QK cursor: unit, local chunk, global chunk, Q index
+            int pj = 0, pc = 0, pgl = 0;          // PV cursor
+            auto seek = [&](int& j, Unit& w) {
+                for (; j < n_units; ++j) {
+                    w = unit(j);
+                    if (w.NC > 0) return;
+                }
+            };
+            seek(qj, qu);
+            pj = qj;
+            pu = qu;
+            int q_issued = 0;         // Q loads issued (units with entries)
+            int g_prev_last = -1;     // last QK of the previous unit with entries
             uint64_t t_idle = globaltimer_ns();
-            while (ok && cp < NC) {
+            while (ok && pj < n_units) {
                 bool progressed = false;
-                if (cq < NC && mbar_test_wait(bar(B_FULL + cq % kStages), (cq / kStages) & 1) &&
-                    (cq < 2 || mbar_test_wait(bar(B_SFREE + (cq & 1)), ((cq - 2) >> 1) & 1))) {
-                    const int c = cq++;
+                if (qj < n_units && q_issued == qq &&
+                    (g_prev_last < 0 ||
+                     mbar_test_wait(bar(B_SFULL + (g_prev_last & 1)), (g_prev_last >> 1) & 1))) {
+                    // Q of the unit at the QK cursor: latent columns [128,256) of
+                    // the slice and the rope slice
+                    mbar_arrive_expect_tx(bar(B_Q), kQBytes);
+                    for (int j = 0; j < 2; ++j)
+                        tma_load_2d(qs + j * kQSlab, &tm_q128, (int)rank * 256 + 128 + j * 64, qu.t * kHeads,
+                                    bar(B_Q));
+                    tma_load_2d(qs + 2 * kQSlab, &tm_q64, 512 + (int)rank * 32, qu.t * kHeads, bar(B_Q));
+                    ++q_issued;
+                    progressed = true;
+                }
+                if (qj < n_units && q_issued > qq &&
+                    mbar_test_wait(bar(B_FULL + qg % kStages), (qg / kStages) & 1) &&
+                    (qg < 2 || mbar_test_wait(bar(B_SFREE + (qg & 1)), ((qg - 2) >> 1) & 1)) &&
+                    (qc > 0 || (mbar_test_wait(bar(B_Q), qq & 1) && mbar_test_wait(bar(B_QT), qq & 1)))) {
+                    const int g = qg;
                     // the stage was written by cp.async (generic proxy); the MMA
                     // reads it through the async proxy
                     fence_proxy_async_smem();
                     tc_fence_after();
-                    const uint32_t kvs = sbase + kOffKV + (c % kStages) * kStageBytes;
-                    const uint32_t d = tmem + kColS + (c & 1) * kKeys;
+                    const uint32_t kvs = sbase + kOffKV + (g % kStages) * kStageBytes;
+                    const uint32_t d = tmem + kColS + (g & 1) * kKeys;
                     // latent columns [0,128) of the slice: A = Q in TMEM (8 K-steps)
 #pragma unroll
                     for (int kk = 0; kk < 8; ++kk) {
@@ -253,23 +313,38 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
                         const uint64_t bd = smem_desc(kvs + 4 * kKSlab + kk * 32, 16, 512, kSwizzle64B);
                         mma_f16_ss(d, ad, bd, id_qk, 1u);
                     }
-                    mma_commit(bar(B_SFULL + (c & 1)));
+                    mma_commit(bar(B_SFULL + (g & 1)));
+                    issued_any = true;
+                    ++qg;
+                    if (++qc == qu.NC) {
+                        g_prev_last = g;
+                        ++qq;
+                        qc = 0;
+                        ++qj;
+                        seek(qj, qu);
+                    }
                     progressed = true;
                 }
-                if (cp < cq && mbar_test_wait(bar(B_PFULL + (cp & 1)), (cp >> 1) & 1)) {
-                    const int c = cp++;
+                if (pgl < qg && mbar_test_wait(bar(B_PFULL + (pgl & 1)), (pgl >> 1) & 1)) {
+                    const int g = pgl;
                     tc_fence_after();
-                    const uint32_t kvs = sbase + kOffKV + (c % kStages) * kStageBytes;
+                    const uint32_t kvs = sbase + kOffKV + (g % kStages) * kStageBytes;
 #pragma unroll
                     for (int kk = 0; kk < kKeys / 16; ++kk) {
                         // B = gathered rows read MN-major: 64 values per 128-byte row,
                         // LBO = next 64 columns (slab), SBO = next 8 keys.
                         const uint64_t bd = smem_desc(kvs + kk * 16 * 128, kKSlab, 1024, kSwizzle128B);
-                        mma_f16_ts(tmem + kColO, tmem + kColP + (c & 1) * 32 + kk * 8, bd, id_pv,
-                                   (c > 0 || kk > 0) ? 1u : 0u);
+                        mma_f16_ts(tmem + kColO, tmem + kColP + (g & 1) * 32 + kk * 8, bd, id_pv,
+                                   (pc > 0 || kk > 0) ? 1u : 0u);
                     }
-                    mma_commit(bar(B_PVDONE + (c & 1)));
-                    mma_commit(bar(B_EMPTY + (c % kStages)));
+                    mma_commit(bar(B_PVDONE + (g & 1)));
+                    mma_commit(bar(B_EMPTY + (g % kStages)));
+                    ++pgl;
+                    if (++pc == pu.NC) {
+                        pc = 0;
+                        ++pj;
+                        seek(pj, pu);
+                    }
                     progressed = true;
                 }
                 if (progressed) {
@@ -278,7 +353,7 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
                     ok = false;
                 } else if (globaltimer_ns() - t_idle > kWaitLimitNs) {
                     *abort_flag = 1;
-                    report_timeout(cq < NC ? B_FULL : B_PFULL, cq < NC ? cq : cp, 0);
+                    report_timeout(B_PFULL, pgl, 0);
                     ok = false;
                 }
             }
@@ -290,18 +365,11 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
         // (row, piece) pattern of a thread repeats every three iterations with
         // the row advanced by 8, which keeps the swizzle phase, so a copy costs
         // one table load and one cp.async. Each warp keeps its own table of the
-        // chunk's row byte offsets (-1 = masked entry, read as zeros).
+        // chunk's row byte offsets (-1 = masked entry, read as zeros). The ring
+        // runs on across units: the next unit's first chunks are gathered
+        // while the current one finishes.
         const int gw = warp - 1;
         const int g = threadIdx.x - 32;
-        if (gw == 0 && lane == 0) {
-            prefetch_tmap(&tm_q128);
-            prefetch_tmap(&tm_q64);
-            mbar_arrive_expect_tx(bar(B_Q), kQBytes);
-            for (int j = 0; j < 2; ++j)
-                tma_load_2d(qs + j * kQSlab, &tm_q128, (int)rank * 256 + 128 + j * 64, t * kHeads, bar(B_Q));
-            tma_load_2d(qs + 2 * kQSlab, &tm_q64, 512 + (int)rank * 32, t * kHeads, bar(B_Q));
-        }
-        const int* idx_row = idx + (size_t)t * k + e0;
         uint32_t* smask = reinterpret_cast<uint32_t*>(sgen + kOffMask);
         long long* rows_tab = reinterpret_cast<long long*>(sgen + kOffRows) + gw * kKeys;
         int r_q[3];
@@ -317,41 +385,51 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
             col_q[q3] = piece_col(rank, j) * 2;   // bytes
         }
         const char* kvb = reinterpret_cast<const char*>(kv);
-        int sa = lane < n_row ? __ldg(idx_row + lane) : -1;
-        int sb = lane + 32 < n_row ? __ldg(idx_row + lane + 32) : -1;
-        for (int c = 0; c < NC; ++c) {
-            const int st = c % kStages;
-            if (c >= kStages) {
-                const bool got = mbar_wait(bar(B_EMPTY + st), ((c - kStages) / kStages) & 1,
-                                           abort_flag, 100 + B_EMPTY, c);
-                if (!__all_sync(0xffffffffu, got)) break;   // warp-uniform exit
-            }
-            const bool va = sa >= 0 && sa <= p_last, vb = sb >= 0 && sb <= p_last;
-            rows_tab[lane] = va ? key_row(pg, bt, base, sa) * (long long)(kDqk * 2) : -1ll;
-            rows_tab[lane + 32] = vb ? key_row(pg, bt, base, sb) * (long long)(kDqk * 2) : -1ll;
-            if (gw == 0) {
-                const unsigned ma = __ballot_sync(0xffffffffu, va), mb = __ballot_sync(0xffffffffu, vb);
-                if (lane == 0) {
-                    smask[st * 2] = ma;
-                    smask[st * 2 + 1] = mb;
+        int gg = 0;
+        bool ok = true;
+        for (int j = 0; ok && j < n_units; ++j) {
+            const Unit w = unit(j);
+            if (w.NC == 0) continue;
+            const int* idx_row = idx + (size_t)w.t * k + w.e0;
+            int sa = lane < w.n_row ? __ldg(idx_row + lane) : -1;
+            int sb = lane + 32 < w.n_row ? __ldg(idx_row + lane + 32) : -1;
+            for (int c = 0; c < w.NC; ++c, ++gg) {
+                const int st = gg % kStages;
+                if (gg >= kStages) {
+                    const bool got = mbar_wait(bar(B_EMPTY + st), ((gg - kStages) / kStages) & 1,
+                                               abort_flag, 100 + B_EMPTY, gg);
+                    if (!__all_sync(0xffffffffu, got)) {   // warp-uniform exit
+                        ok = false;
+                        break;
+                    }
                 }
-            }
-            const int i_next = (c + 1) * kKeys + lane;
-            sa = i_next < n_row ? __ldg(idx_row + i_next) : -1;
-            sb = i_next + 32 < n_row ? __ldg(idx_row + i_next + 32) : -1;
-            __syncwarp();
-            const uint32_t kvs = sbase + kOffKV + st * kStageBytes;
-#pragma unroll
-            for (int m = 0; m < 8; ++m)
-#pragma unroll
-                for (int q3 = 0; q3 < 3; ++q3) {
-                    const long long off = rows_tab[r_q[q3] + 8 * m];
-                    const void* src = off >= 0 ? kvb + off + col_q[q3] : kvb;
-                    cp_async16(kvs + d_q[q3] + m * dstep_q[q3], src, off >= 0 ? 16u : 0u);
+                const bool va = sa >= 0 && sa <= w.p_last, vb = sb >= 0 && sb <= w.p_last;
+                rows_tab[lane] = va ? key_row(pg, w.bt, w.base, sa) * (long long)(kDqk * 2) : -1ll;
+                rows_tab[lane + 32] = vb ? key_row(pg, w.bt, w.base, sb) * (long long)(kDqk * 2) : -1ll;
+                if (gw == 0) {
+                    const unsigned ma = __ballot_sync(0xffffffffu, va), mb = __ballot_sync(0xffffffffu, vb);
+                    if (lane == 0) {
+                        smask[st * 2] = ma;
+                        smask[st * 2 + 1] = mb;
+                    }
                 }
-            cp_async_arrive_noinc(bar(B_FULL + st));
-            if (gw == 0 && lane == 0) mbar_arrive(bar(B_FULL + st));   // publishes the mask
-            __syncwarp();   // the table is rewritten for the next chunk
+                const int i_next = (c + 1) * kKeys + lane;
+                sa = i_next < w.n_row ? __ldg(idx_row + i_next) : -1;
+                sb = i_next + 32 < w.n_row ? __ldg(idx_row + i_next + 32) : -1;
+                __syncwarp();
+                const uint32_t kvs = sbase + kOffKV + st * kStageBytes;
+#pragma unroll
+                for (int m = 0; m < 8; ++m)
+#pragma unroll
+                    for (int q3 = 0; q3 < 3; ++q3) {
+                        const long long off = rows_tab[r_q[q3] + 8 * m];
+                        const void* src = off >= 0 ? kvb + off + col_q[q3] : kvb;
+                        cp_async16(kvs + d_q[q3] + m * dstep_q[q3], src, off >= 0 ? 16u : 0u);
+                    }
+                cp_async_arrive_noinc(bar(B_FULL + st));
+                if (gw == 0 && lane == 0) mbar_arrive(bar(B_FULL + st));   // publishes the mask
+                __syncwarp();   // the table is rewritten for the next chunk
+            }
         }
         cp_async_wait_all();
     } else if (warp >= 12) {
@@ -367,41 +445,51 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
         const uint32_t x_peer = mapa(sbase + kOffX, peer);
         const uint32_t xfull_peer = mapa(bar(B_XFULL), peer);
         const uint32_t xstage = sbase + kOffXS;
-        for (int c = 0; c < NC; ++c) {
-            const int b = c & 1;
-            if (!wait_warp(bar(B_SFULL + b), (c >> 1) & 1, abort_flag, 500 + B_SFULL, c)) break;
-            tc_fence_after();
-            uint32_t s0[32], s1[32];
-            tmem_ld32(tmem + lane_addr + kColS + b * kKeys, s0);
-            tmem_ld32(tmem + lane_addr + kColS + b * kKeys + 32, s1);
-            tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(B_SFREE + b));
-            uint32_t h[32];
+        int gs = 0;
+        bool ok = true;
+        for (int j = 0; ok && j < n_units; ++j) {
+            const int NC = unit(j).NC;
+            for (int c = 0; c < NC; ++c, ++gs) {
+                const int b = gs & 1;
+                if (!wait_warp(bar(B_SFULL + b), (gs >> 1) & 1, abort_flag, 500 + B_SFULL, gs)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                uint32_t s0[32], s1[32];
+                tmem_ld32(tmem + lane_addr + kColS + b * kKeys, s0);
+                tmem_ld32(tmem + lane_addr + kColS + b * kKeys + 32, s1);
+                tmem_wait_ld();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(B_SFREE + b));
+                uint32_t h[32];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                h[j] = pack_half2(__uint_as_float(s0[2 * j]) * scale_log2,
-                                  __uint_as_float(s0[2 * j + 1]) * scale_log2);
-                h[16 + j] = pack_half2(__uint_as_float(s1[2 * j]) * scale_log2,
-                                       __uint_as_float(s1[2 * j + 1]) * scale_log2);
+                for (int jj = 0; jj < 16; ++jj) {
+                    h[jj] = pack_half2(__uint_as_float(s0[2 * jj]) * scale_log2,
+                                       __uint_as_float(s0[2 * jj + 1]) * scale_log2);
+                    h[16 + jj] = pack_half2(__uint_as_float(s1[2 * jj]) * scale_log2,
+                                            __uint_as_float(s1[2 * jj + 1]) * scale_log2);
+                }
+                // The peer has consumed chunk gs-kXSlots from slot xb, so the bulk
+                // copy of that chunk has landed: it has also finished reading
+                // staging slot xb.
+                const int xb = gs % kXSlots;
+                if (gs >= kXSlots && !wait_warp(bar(B_XFREE + xb), ((gs - kXSlots) / kXSlots) & 1, abort_flag,
+                                                500 + B_XFREE, gs)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t stg = xstage + xb * kXBytes;
+#pragma unroll
+                for (int m = 0; m < 8; ++m)
+                    st_shared_v4(stg + xrow + (((m + lane) & 7) << 4),
+                                 make_uint4(h[4 * m], h[4 * m + 1], h[4 * m + 2], h[4 * m + 3]));
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0)
+                    bulk_s2cluster(x_peer + xb * kXBytes + xwarp, stg + xwarp, kXWarpBytes, xfull_peer + 8u * xb);
             }
-            // The peer has consumed chunk c-kXSlots from slot xb, so the bulk
-            // copy of that chunk has landed: it has also finished reading
-            // staging slot xb.
-            const int xb = c % kXSlots;
-            if (c >= kXSlots && !wait_warp(bar(B_XFREE + xb), ((c - kXSlots) / kXSlots) & 1, abort_flag,
-                                           500 + B_XFREE, c))
-                break;
-            const uint32_t stg = xstage + xb * kXBytes;
-#pragma unroll
-            for (int m = 0; m < 8; ++m)
-                st_shared_v4(stg + xrow + (((m + lane) & 7) << 4),
-                             make_uint4(h[4 * m], h[4 * m + 1], h[4 * m + 2], h[4 * m + 3]));
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0)
-                bulk_s2cluster(x_peer + xb * kXBytes + xwarp, stg + xwarp, kXWarpBytes, xfull_peer + 8u * xb);
         }
     } else if (warp >= 4) {
         // --------------------------------------------- softmax + epilogue
@@ -416,16 +504,14 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
         const uint32_t* smask = reinterpret_cast<const uint32_t*>(sgen + kOffMask);
         float* red = reinterpret_cast<float*>(sgen + kOffRed);
         float* lsum_s = reinterpret_cast<float*>(sgen + kOffLsum);
-        float m_use = -INFINITY, l = 0.f;
         bool ok = true;
         auto wait_w = [&](uint32_t b_addr, uint32_t par, int tag, int c) -> bool {
             return wait_warp(b_addr, par, abort_flag, tag, c);
         };
-
-        {
-            // latent Q columns [0,128) of the slice for head i into TMEM (A
-            // operand of the QK MMAs): this half's 64 columns, two bf16 per
-            // 32-bit TMEM column
+        // latent Q columns [0,128) of a unit's row for head i into TMEM (A
+        // operand of the QK MMAs): this half's 64 columns, two bf16 per 32-bit
+        // TMEM column
+        auto write_q = [&](int t) {
             const uint4* qsrc = reinterpret_cast<const uint4*>(
                 q + ((size_t)t * kHeads + i) * kDqk + rank * 256 + 64 * hs);
             uint32_t w[32];
@@ -439,179 +525,213 @@ sparse_mla_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q128,
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar(B_QT));
+        };
+        // the next unit with entries after iteration j (n_units if none)
+        auto next_with_entries = [&](int j, int* t_out) -> int {
+            for (++j; j < n_units; ++j) {
+                const Unit w = unit(j);
+                if (w.NC > 0) {
+                    *t_out = w.t;
+                    return j;
+                }
+            }
+            return n_units;
+        };
+        {
+            int t_first;
+            if (next_with_entries(-1, &t_first) < n_units) write_q(t_first);
         }
-        for (int c = 0; ok && c < NC; ++c) {
-            const int b = c & 1;
-            const int xb = c % kXSlots;
-            if (i == 0 && hs == 0) mbar_arrive_expect_tx(bar(B_XFULL + xb), kXBytes);
-            // the chunk's validity bits (its gather completed long before S(c))
-            if (!wait_w(bar(B_FULL + c % kStages), (c / kStages) & 1, 200 + B_FULL, c)) { ok = false; break; }
-            const uint32_t mw = smask[(c % kStages) * 2 + hs];
-            // this CTA's partial logits of chunk c (fp32, TMEM)
-            if (!wait_w(bar(B_SFULL + b), (c >> 1) & 1, 200 + B_SFULL, c)) { ok = false; break; }
-            tc_fence_after();
-            uint32_t sr[32];
-            tmem_ld32(tmem + lane_addr + kColS + b * kKeys + 32 * hs, sr);
-            // the peer's (fp16, scaled) arrive by bulk copy, counted on this local barrier
-            if (!wait_w(bar(B_XFULL + xb), (c / kXSlots) & 1, 200 + B_XFULL, c)) {
+        int g0 = 0;
+        for (int j = 0; j < n_units; ++j) {
+            const Unit w = unit(j);
+            const int NC = w.NC, t = w.t, part = w.part;
+            float m_use = -INFINITY, l = 0.f;
+            for (int c = 0; ok && c < NC; ++c) {
+                const int gc = g0 + c;
+                const int b = gc & 1;
+                const int xb = gc % kXSlots;
+                if (i == 0 && hs == 0) mbar_arrive_expect_tx(bar(B_XFULL + xb), kXBytes);
+                // the chunk's validity bits (its gather completed long before S(c))
+                if (!wait_w(bar(B_FULL + gc % kStages), (gc / kStages) & 1, 200 + B_FULL, gc)) { ok = false; break; }
+                const uint32_t mw = smask[(gc % kStages) * 2 + hs];
+                // this CTA's partial logits of chunk c (fp32, TMEM)
+                if (!wait_w(bar(B_SFULL + b), (gc >> 1) & 1, 200 + B_SFULL, gc)) { ok = false; break; }
+                tc_fence_after();
+                uint32_t sr[32];
+                tmem_ld32(tmem + lane_addr + kColS + b * kKeys + 32 * hs, sr);
+                // the peer's (fp16, scaled) arrive by bulk copy, counted on this local barrier
+                if (!wait_w(bar(B_XFULL + xb), (gc / kXSlots) & 1, 200 + B_XFULL, gc)) {
+                    tmem_wait_ld();
+                    ok = false;
+                    break;
+                }
+                uint32_t gx[16];
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    const uint4 v = ld_shared_v4(xs + xb * kXBytes + (((4 * hs + m + lane) & 7) << 4));
+                    gx[4 * m] = v.x; gx[4 * m + 1] = v.y; gx[4 * m + 2] = v.z; gx[4 * m + 3] = v.w;
+                }
                 tmem_wait_ld();
-                ok = false;
-                break;
-            }
-            uint32_t g[16];
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(B_SFREE + b));   // S(c) fully read by this warp
+                // logit (log2 domain) = own partial (fp32) + peer partial (fp16); masked -> -inf
+                float x[32];
 #pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                const uint4 v = ld_shared_v4(xs + xb * kXBytes + (((4 * hs + m + lane) & 7) << 4));
-                g[4 * m] = v.x; g[4 * m + 1] = v.y; g[4 * m + 2] = v.z; g[4 * m + 3] = v.w;
-            }
-            tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(B_SFREE + b));   // S(c) fully read by this warp
-            // logit (log2 domain) = own partial (fp32) + peer partial (fp16); masked -> -inf
-            float x[32];
+                for (int jj = 0; jj < 16; ++jj) {
+                    const float2 o = unpack_half2(gx[jj]);
+                    x[2 * jj] = (mw >> (2 * jj)) & 1u ? fmaf(__uint_as_float(sr[2 * jj]), scale_log2, o.x)
+                                                      : -INFINITY;
+                    x[2 * jj + 1] = (mw >> (2 * jj + 1)) & 1u
+                                        ? fmaf(__uint_as_float(sr[2 * jj + 1]), scale_log2, o.y)
+                                        : -INFINITY;
+                }
+                // the peer may refill this exchange slot once every warp has used it
+                // (the loaded values are consumed above, so a relaxed signal suffices)
+                __syncwarp();
+                if (lane == 0) mbar_arrive_remote_relaxed(xfree_peer + 8u * xb);
+                float mx[16];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                const float2 o = unpack_half2(g[j]);
-                x[2 * j] = (mw >> (2 * j)) & 1u ? fmaf(__uint_as_float(sr[2 * j]), scale_log2, o.x)
-                                                : -INFINITY;
-                x[2 * j + 1] = (mw >> (2 * j + 1)) & 1u
-                                   ? fmaf(__uint_as_float(sr[2 * j + 1]), scale_log2, o.y)
-                                   : -INFINITY;
-            }
-            // the peer may refill this exchange slot once every warp has used it
-            // (the loaded values are consumed above, so a relaxed signal suffices)
-            __syncwarp();
-            if (lane == 0) mbar_arrive_remote_relaxed(xfree_peer + 8u * xb);
-            float mx[16];
+                for (int jj = 0; jj < 16; ++jj) mx[jj] = fmaxf(x[jj], x[jj + 16]);
 #pragma unroll
-            for (int j = 0; j < 16; ++j) mx[j] = fmaxf(x[j], x[j + 16]);
+                for (int ww = 8; ww >= 1; ww >>= 1)
 #pragma unroll
-            for (int w = 8; w >= 1; w >>= 1)
+                    for (int jj = 0; jj < ww; ++jj) mx[jj] = fmaxf(mx[jj], mx[jj + ww]);
+                // row maximum over both key halves (the other half lives in warp +-4)
+                red[(b * 2 + hs) * kHeads + i] = mx[0];
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(B_RED + b));
+                if (!wait_w(bar(B_RED + b), (gc >> 1) & 1, 200 + B_RED, gc)) { ok = false; break; }
+                const float mc = fmaxf(mx[0], red[(b * 2 + (hs ^ 1)) * kHeads + i]);
+                const float m_new = fmaxf(m_use, mc);
+                const bool raise = m_new > m_use + 8.f;
+                const bool rescale = raise && m_use != -INFINITY;
+                const float f = rescale ? ex2(m_use - m_new) : 1.f;
+                if (__any_sync(0xffffffffu, rescale)) {
+                    // O holds earlier chunks of this unit: rescale once PV(c-1)
+                    // has landed. TMEM loads/stores are warp-wide, so every lane
+                    // takes part (f = 1 for rows whose maximum did not move).
+                    if (!wait_w(bar(B_PVDONE + ((gc - 1) & 1)), ((gc - 1) >> 1) & 1, 400 + B_PVDONE, gc)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+#pragma unroll 1
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        uint32_t o[32];
+                        const uint32_t ta = tmem + lane_addr + kColO + 128 * hs + q4 * 32;
+                        tmem_ld32(ta, o);
+                        tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < w; ++j) mx[j] = fmaxf(mx[j], mx[j + w]);
-            // row maximum over both key halves (the other half lives in warp +-4)
-            red[(b * 2 + hs) * kHeads + i] = mx[0];
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(B_RED + b));
-            if (!wait_w(bar(B_RED + b), (c >> 1) & 1, 200 + B_RED, c)) { ok = false; break; }
-            const float mc = fmaxf(mx[0], red[(b * 2 + (hs ^ 1)) * kHeads + i]);
-            const float m_new = fmaxf(m_use, mc);
-            const bool raise = m_new > m_use + 8.f;
-            const bool rescale = raise && m_use != -INFINITY;
-            const float f = rescale ? ex2(m_use - m_new) : 1.f;
-            if (__any_sync(0xffffffffu, rescale)) {
-                // O holds earlier chunks: rescale once PV(c-1) has landed. TMEM
-                // loads/stores are warp-wide, so every lane takes part (f = 1
-                // for rows whose maximum did not move).
-                if (!wait_w(bar(B_PVDONE + ((c - 1) & 1)), ((c - 1) >> 1) & 1, 400 + B_PVDONE, c)) {
+                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+                        tmem_st32(ta, o);
+                    }
+                    tmem_wait_st();
+                }
+                l *= f;
+                if (raise) m_use = m_new;
+                const float msub = m_use == -INFINITY ? 0.f : m_use;
+                uint32_t pk[16];
+                float ps[16];
+#pragma unroll
+                for (int jj = 0; jj < 16; ++jj) {
+                    const float p0 = ex2(x[2 * jj] - msub), p1 = ex2(x[2 * jj + 1] - msub);
+                    ps[jj] = p0 + p1;
+                    pk[jj] = pack_bf16x2(p0, p1);
+                }
+#pragma unroll
+                for (int ww = 8; ww >= 1; ww >>= 1)
+#pragma unroll
+                    for (int jj = 0; jj < ww; ++jj) ps[jj] += ps[jj + ww];
+                l += ps[0];
+                // P buffer b is free once PV(g-2) has read it
+                if (gc >= 2 && !wait_w(bar(B_PVDONE + b), ((gc - 2) >> 1) & 1, 200 + B_PVDONE, gc)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-#pragma unroll 1
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    uint32_t o[32];
-                    const uint32_t ta = tmem + lane_addr + kColO + 128 * hs + q4 * 32;
-                    tmem_ld32(ta, o);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
-                    tmem_st32(ta, o);
-                }
+                tmem_st16(tmem + lane_addr + kColP + b * 32 + 16 * hs, pk);
                 tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(B_PFULL + b));
             }
-            l *= f;
-            if (raise) m_use = m_new;
-            const float msub = m_use == -INFINITY ? 0.f : m_use;
-            uint32_t pk[16];
-            float ps[16];
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                const float p0 = ex2(x[2 * j] - msub), p1 = ex2(x[2 * j + 1] - msub);
-                ps[j] = p0 + p1;
-                pk[j] = pack_bf16x2(p0, p1);
+            // every QK of this unit has completed (its last S was read): the
+            // next unit's Q goes into TMEM now, so its first QKs overlap this
+            // unit's epilogue
+            if (ok && NC > 0) {
+                int t_next;
+                if (next_with_entries(j, &t_next) < n_units) write_q(t_next);
             }
-#pragma unroll
-            for (int w = 8; w >= 1; w >>= 1)
-#pragma unroll
-                for (int j = 0; j < w; ++j) ps[j] += ps[j + w];
-            l += ps[0];
-            // P buffer b is free once PV(c-2) has read it
-            if (c >= 2 && !wait_w(bar(B_PVDONE + b), ((c - 2) >> 1) & 1, 200 + B_PVDONE, c)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            tmem_st16(tmem + lane_addr + kColP + b * 32 + 16 * hs, pk);
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(B_PFULL + b));
-        }
-        // row sum over both key halves
-        if (ok) {
-            lsum_s[hs * kHeads + i] = l;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(B_LSUM));
-            ok = wait_w(bar(B_LSUM), 0, 200 + B_LSUM, 0);
-            if (ok) l += lsum_s[(hs ^ 1) * kHeads + i];
-        }
-        // epilogue: O / l -> bf16 (or, for a part of a split row, fp32 into
-        // the parts buffer), columns [128hs, 128hs+128) of this CTA's half
-        const size_t prow = ((size_t)t * splits + part) * kHeads + i;   // parts layout [T, splits, 128]
-        __nv_bfloat16* orow = out + ((size_t)t * kHeads + i) * kDv + rank * 256 + 128 * hs;
-        float* porow = splits > 1 ? part_o + prow * kDv + rank * 256 + 128 * hs : nullptr;
-        if (ok && NC > 0) {
-            const int c = NC - 1;
-            ok = wait_w(bar(B_PVDONE + (c & 1)), (c >> 1) & 1, 300 + B_PVDONE, c);
+            // row sum over both key halves (buffer j & 1)
             if (ok) {
-                tc_fence_after();
-                const float inv = l > 0.f ? 1.f / l : 0.f;
+                lsum_s[((j & 1) * 2 + hs) * kHeads + i] = l;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(B_LSUM));
+                ok = wait_w(bar(B_LSUM), j & 1, 200 + B_LSUM, j);
+                if (ok) l += lsum_s[((j & 1) * 2 + (hs ^ 1)) * kHeads + i];
+            }
+            // epilogue: O / l -> bf16 (or, for a part of a split row, fp32 into
+            // the parts buffer), columns [128hs, 128hs+128) of this CTA's half
+            const size_t prow = ((size_t)t * splits + part) * kHeads + i;   // parts layout [T, splits, 128]
+            __nv_bfloat16* orow = out + ((size_t)t * kHeads + i) * kDv + rank * 256 + 128 * hs;
+            float* porow = splits > 1 ? part_o + prow * kDv + rank * 256 + 128 * hs : nullptr;
+            if (ok && NC > 0) {
+                const int gl = g0 + NC - 1;
+                ok = wait_w(bar(B_PVDONE + (gl & 1)), (gl >> 1) & 1, 300 + B_PVDONE, gl);
+                if (ok) {
+                    tc_fence_after();
+                    const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll 1
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    uint32_t o[32];
-                    tmem_ld32(tmem + lane_addr + kColO + 128 * hs + q4 * 32, o);
-                    tmem_wait_ld();
-                    if (porow) {
-                        float4* dst = reinterpret_cast<float4*>(porow + q4 * 32);
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        uint32_t o[32];
+                        tmem_ld32(tmem + lane_addr + kColO + 128 * hs + q4 * 32, o);
+                        tmem_wait_ld();
+                        if (porow) {
+                            float4* dst = reinterpret_cast<float4*>(porow + q4 * 32);
 #pragma unroll
-                        for (int v = 0; v < 8; ++v)
-                            dst[v] = make_float4(__uint_as_float(o[4 * v]) * inv, __uint_as_float(o[4 * v + 1]) * inv,
-                                                 __uint_as_float(o[4 * v + 2]) * inv,
-                                                 __uint_as_float(o[4 * v + 3]) * inv);
-                        continue;
+                            for (int v = 0; v < 8; ++v)
+                                dst[v] = make_float4(__uint_as_float(o[4 * v]) * inv, __uint_as_float(o[4 * v + 1]) * inv,
+                                                     __uint_as_float(o[4 * v + 2]) * inv,
+                                                     __uint_as_float(o[4 * v + 3]) * inv);
+                            continue;
+                        }
+                        uint32_t wv[16];
+#pragma unroll
+                        for (int e = 0; e < 16; ++e)
+                            wv[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv,
+                                                __uint_as_float(o[2 * e + 1]) * inv);
+                        uint4* dst = reinterpret_cast<uint4*>(orow + q4 * 32);
+#pragma unroll
+                        for (int v = 0; v < 4; ++v)
+                            dst[v] = make_uint4(wv[4 * v], wv[4 * v + 1], wv[4 * v + 2], wv[4 * v + 3]);
                     }
-                    uint32_t w[16];
-#pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        w[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv,
-                                           __uint_as_float(o[2 * e + 1]) * inv);
-                    uint4* dst = reinterpret_cast<uint4*>(orow + q4 * 32);
-#pragma unroll
-                    for (int v = 0; v < 4; ++v)
-                        dst[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+                    // O is read: the next unit's first PV may overwrite it (its
+                    // P arrives only after this warp's next chunk)
+                    tc_fence_before();
+                }
+            } else if (NC == 0) {
+                if (porow) {
+                    float4* dst = reinterpret_cast<float4*>(porow);
+                    for (int v = 0; v < 32; ++v) dst[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+                } else {
+                    uint4* dst = reinterpret_cast<uint4*>(orow);
+                    for (int v = 0; v < 16; ++v) dst[v] = make_uint4(0u, 0u, 0u, 0u);
                 }
             }
-        } else if (NC == 0) {
-            if (porow) {
-                float4* dst = reinterpret_cast<float4*>(porow);
-                for (int v = 0; v < 32; ++v) dst[v] = make_float4(0.f, 0.f, 0.f, 0.f);
-            } else {
-                uint4* dst = reinterpret_cast<uint4*>(orow);
-                for (int v = 0; v < 16; ++v) dst[v] = make_uint4(0u, 0u, 0u, 0u);
+            if (rank == 0 && hs == 0 && (ok || NC == 0)) {
+                const float lv = l > 0.f ? (m_use + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+                if (splits > 1)
+                    part_lse[prow] = lv;
+                else
+                    lse[(size_t)t * kHeads + i] = lv;
             }
-        }
-        if (rank == 0 && hs == 0 && (ok || NC == 0)) {
-            const float lv = l > 0.f ? (m_use + __log2f(l)) * 0.69314718055994531f : -INFINITY;
-            if (splits > 1)
-                part_lse[prow] = lv;
-            else
-                lse[(size_t)t * kHeads + i] = lv;
+            g0 += NC;
+            if (!ok) break;
         }
     }
 
-    if (warp == 0 && lane == 0 && NC > 0) {
+    if (warp == 0 && lane == 0 && issued_any) {
         // every MMA issued completes before TMEM is released
         mma_commit(bar(B_DRAIN));
         const uint64_t t0 = globaltimer_ns();

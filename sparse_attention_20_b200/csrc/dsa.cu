@@ -684,7 +684,9 @@ int attn_tc(const __nv_bfloat16* q, const __nv_bfloat16* kv, const int32_t* idx,
         part_lse = reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) +
                                             align_up((size_t)T * splits * kHeads * kDv * sizeof(float)));
     }
-    launch_pdl(sparse_mla_attn_tc_kernel, dim3(2 * T * splits), dim3(kThreads), kSmemBytes, st, tq128, tq64, q,
+    // persistent: one cluster per SM pair, each walking units cid, cid + clusters, ...
+    const int clusters = (int)std::min<long long>((long long)T * splits, std::max(1, num_sms() / 2));
+    launch_pdl(sparse_mla_attn_tc_kernel, dim3(2 * clusters), dim3(kThreads), kSmemBytes, st, tq128, tq64, q,
                kv, idx, pos, k_base, T, S, k, scale_log2, out, lse, pg, splits, part_o, part_lse);
     DSA_LAUNCH_CHECK("sparse_mla_attn_tc_kernel");
     if (splits > 1) {
