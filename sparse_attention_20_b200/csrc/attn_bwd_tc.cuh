@@ -1,0 +1,362 @@
+// Backward of the sparse MQA attention, dkv part, on the 5th-generation
+// tensor cores, for the MLA head shape (Hq = 128, d_qk = 576, d_v = 512).
+// Same results as attn_bwd_dkv_kernel (attn_bwd.cuh states the chain rule):
+// per query row t and chunk of 64 selected slots,
+//   z = Q_t C^T, dp = dO_t V^T                      (128 heads x 64 slots)
+//   p = exp(scale z - lse), g = scale p (dp - D)    (bf16, g also to g_ws)
+//   dC^T = Q_t^T g + dO_t^T p                        (576 columns x 64 slots)
+// and dC is scatter-added into dkv (fp32 atomics, one per element).
+//
+// One CTA of 256 threads per (row, 64 slots), two CTAs per SM (their phases
+// overlap):
+//  - warp 0 (one thread) streams Q_t and dO_t in 64-column tiles by TMA
+//    (128 rows x 128 B, 128B swizzle): 17 tiles for z and dp (a 2-stage
+//    ring), then 9 two-tile pairs for dC (two 32 KB buffers in the space of
+//    the gathered rows, free once z and dp are done);
+//  - warps 1-3 gather the 64 selected latent rows (cp.async, 128B-swizzled
+//    64-column slabs, K-major B operand of z and dp); warp 1's first thread
+//    then issues every MMA;
+//  - warps 4-7 (one head per thread, the TMEM lane) form D and lse first,
+//    then read z and dp from TMEM, write p and g as MN-major tiles
+//    [head][slot] in the ring's space (the B operands of dC^T, whose A
+//    operands are the Q / dO tiles read MN-major), and finally add each dC^T
+//    tile (M = 128 columns, N = 64 slots) into dkv.
+// TMEM (256 columns): z [0,64) and dp [64,128), then dC^T tiles 0..3 at
+// [64m, 64m+64); tile 4 reuses tile 0's columns once they are drained.
+#pragma once
+#include <cuda.h>
+
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace dsa {
+namespace bwd_tc {
+
+using namespace sm100;
+
+constexpr int kHeads = 128, kDqk = 576, kDv = 512, kSlots = 64;
+constexpr int kThreads = 256;
+constexpr int kTile = 128 * 128;          // one [128 rows x 64 columns] bf16 tile, 128B swizzle
+constexpr int kCSlab = kSlots * 128;      // 64 gathered rows x 64 columns
+constexpr int kQTiles = kDqk / 64;        // 9
+constexpr int kVTiles = kDv / 64;         // 8
+constexpr int kRing = 2;
+constexpr int kGatherThreads = 96;
+constexpr int kOffC = 0;                                   // 9 slabs (72 KB); then 2 pair buffers
+constexpr int kOffRing = kOffC + kQTiles * kCSlab;         // 3 x 16 KB
+constexpr int kPGTile = kHeads * kSlots * 2;               // p or g: [128 heads][64 slots] bf16, 16 KB
+constexpr int kOffP = kOffRing;                            // p and g take the ring's space after z, dp
+constexpr int kOffG = kOffP + kPGTile;
+constexpr int kOffRows = kOffRing + kRing * kTile;         // 64 x long long
+constexpr int kOffBar = kOffRows + kSlots * 8;
+constexpr int kSmemBytes = kOffBar + 256 + 1024;           // + alignment slack
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kColZ = 0, kColDp = 64, kColDc = 0;
+
+enum : int {
+    B_CFULL = 0, B_AFULL = 1, B_AEMPTY = B_AFULL + kRing, B_ZDONE = B_AEMPTY + kRing, B_PG = B_ZDONE + 1,
+    B_PFULL = B_PG + 1, B_PEMPTY = B_PFULL + 2, B_TILE = B_PEMPTY + 2, B_T0FREE = B_TILE + 5,
+    B_DRAIN = B_T0FREE + 1, B_COUNT = B_DRAIN + 1
+};
+
+static_assert(2 * 2 * kTile <= kQTiles * kCSlab, "pair buffers fit in the gathered rows' space");
+static_assert(kOffRing % 1024 == 0 && kOffP % 1024 == 0 && kOffG % 1024 == 0, "alignment");
+static_assert(8 * B_COUNT + 16 <= 256, "barrier area");
+static_assert(kPGTile == kHeads * 128 && kOffG + kPGTile <= kOffRows && kOffBar - kOffRows == kSlots * 8,
+              "p / g tiles of 128-byte rows inside the ring, then the slot rows, then the barriers");
+static_assert(2 * (kSmemBytes + 1024) <= 233472, "two CTAs per SM");
+static_assert(kSmemBytes <= 232448, "shared memory");
+
+// kind::f16 instruction descriptor with both operand majors given.
+__host__ __device__ constexpr uint32_t idesc_bf16_ab(int M, int N, bool a_mn_major, bool b_mn_major)
+{
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn_major ? 1u : 0u) << 15) |
+           ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// Bounded wait whose outcome is the same for the whole warp.
+__device__ __forceinline__ bool wait_all(uint32_t b_addr, uint32_t par, volatile int* abort_flag, int tag, int c)
+{
+    return __all_sync(0xffffffffu, mbar_wait(b_addr, par, abort_flag, tag, c));
+}
+
+__device__ __forceinline__ void red_add_f32(float* p, float v)
+{
+    asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
+}
+
+// grid: x = slot chunk (64 slots), y = query row within the pass [r0, r0 + gridDim.y).
+// g_ws: bf16 [rows][128][slots_pad(k)], as attn_bwd_dkv_kernel writes it.
+__global__ void __launch_bounds__(kThreads, 2)
+attn_bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                       const __nv_bfloat16* __restrict__ kv, const int* __restrict__ idx,
+                       const int* __restrict__ pos, const int* __restrict__ k_base,
+                       const __nv_bfloat16* __restrict__ out, const float* __restrict__ lse,
+                       const __nv_bfloat16* __restrict__ dout, int r0, int T, int S, int k, int kp,
+                       float scale, float* __restrict__ dkv, __nv_bfloat16* __restrict__ g_ws)
+{
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t sbase = (raw + 1023u) & ~1023u;
+    uint8_t* sgen = smem_raw + (sbase - raw);
+    const uint32_t bar0 = sbase + kOffBar;
+    auto bar = [&](int i) -> uint32_t { return bar0 + 8u * (uint32_t)i; };
+    uint32_t* taddr_slot = reinterpret_cast<uint32_t*>(sgen + kOffBar + 8 * B_COUNT);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sgen + kOffBar + 8 * B_COUNT + 8);
+    long long* rows = reinterpret_cast<long long*>(sgen + kOffRows);
+
+    const int tl = blockIdx.y, t = r0 + tl, i0 = blockIdx.x * kSlots;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    long long base;
+    const int n_cand = row_candidates(pos, k_base, t, T, S, &base);
+    if (i0 >= min(k, n_cand)) return;   // whole chunk past the row's entries (uniform per CTA)
+
+    if (threadIdx.x < kSlots) {
+        const int i = i0 + threadIdx.x;
+        const int s = i < k ? idx[(size_t)t * k + i] : -1;
+        rows[threadIdx.x] = (i < k && s >= 0 && s < n_cand) ? base + s : -1ll;
+    }
+    if (threadIdx.x == 0) {
+        mbar_init(bar(B_CFULL), kGatherThreads);
+        for (int s = 0; s < kRing; ++s) {
+            mbar_init(bar(B_AFULL + s), 1);
+            mbar_init(bar(B_AEMPTY + s), 1);
+        }
+        mbar_init(bar(B_ZDONE), 1);
+        mbar_init(bar(B_PG), 4);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(bar(B_PFULL + b), 1);
+            mbar_init(bar(B_PEMPTY + b), 1);
+        }
+        for (int m = 0; m < 5; ++m) mbar_init(bar(B_TILE + m), 1);
+        mbar_init(bar(B_T0FREE), 4);    // tile 0's columns read by the four epilogue warps
+        mbar_init(bar(B_DRAIN), 1);
+        *abort_flag = 0;
+        fence_mbar_init_cluster();
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_u32(taddr_slot), kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *taddr_slot;
+    const uint32_t cs = sbase + kOffC, ring = sbase + kOffRing, ps = sbase + kOffP, gs = sbase + kOffG;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------- TMA
+        if (lane == 0) {
+            prefetch_tmap(&tm_q);
+            prefetch_tmap(&tm_do);
+            bool ok = true;
+            // z and dp: Q tiles 0..8, then dO tiles 0..7
+            for (int s = 0; ok && s < kQTiles + kVTiles; ++s) {
+                const int st = s % kRing;
+                if (s >= kRing && !mbar_wait(bar(B_AEMPTY + st), ((s - kRing) / kRing) & 1, abort_flag, 100, s)) {
+                    ok = false;
+                    break;
+                }
+                mbar_arrive_expect_tx(bar(B_AFULL + st), kTile);
+                if (s < kQTiles)
+                    tma_load_2d(ring + st * kTile, &tm_q, 64 * s, t * kHeads, bar(B_AFULL + st));
+                else
+                    tma_load_2d(ring + st * kTile, &tm_do, 64 * (s - kQTiles), t * kHeads, bar(B_AFULL + st));
+            }
+            // dC^T: for column tile m, the pair of Q tiles (2m, 2m+1), then the
+            // pair of dO tiles (m < 4); tile 4 has one Q tile (columns 512..575).
+            // The pair buffers overwrite the gathered rows: z and dp first.
+            if (ok) ok = mbar_wait(bar(B_ZDONE), 0, abort_flag, 101, 0);
+            int p = 0;
+            for (int m = 0; ok && m < 5; ++m) {
+                for (int kind = 0; kind < (m < 4 ? 2 : 1); ++kind, ++p) {
+                    const int pb = p & 1;
+                    if (p >= 2 && !mbar_wait(bar(B_PEMPTY + pb), ((p - 2) >> 1) & 1, abort_flag, 102, p)) {
+                        ok = false;
+                        break;
+                    }
+                    const int n_tiles = m < 4 ? 2 : 1;
+                    mbar_arrive_expect_tx(bar(B_PFULL + pb), n_tiles * kTile);
+                    for (int h = 0; h < n_tiles; ++h)
+                        tma_load_2d(cs + pb * 2 * kTile + h * kTile, kind == 0 ? (const void*)&tm_q : (const void*)&tm_do,
+                                    128 * m + 64 * h, t * kHeads, bar(B_PFULL + pb));
+                }
+            }
+        }
+    } else if (warp <= 3) {
+        // ---------------------------------------------------------- gather
+        // 64 rows x 72 sixteen-byte pieces; piece j of row r goes to slab j/8
+        // (64 columns), 16-byte unit (j%8) ^ (r%8) of the row's 128 bytes
+        const int g = threadIdx.x - 32;
+        const char* kvb = reinterpret_cast<const char*>(kv);
+        for (int e = g; e < kSlots * 72; e += kGatherThreads) {
+            const int r = e / 72, j = e - r * 72;
+            const long long row = rows[r];
+            const uint32_t dst = cs + (j >> 3) * kCSlab + r * 128 + (((j & 7) ^ (r & 7)) << 4);
+            cp_async16(dst, row >= 0 ? kvb + row * (kDqk * 2) + j * 16 : kvb, row >= 0 ? 16u : 0u);
+        }
+        cp_async_arrive_noinc(bar(B_CFULL));
+        if (warp == 1 && lane == 0) {
+            // ----------------------------------------------------- MMAs
+            const uint32_t id_a = idesc_bf16_ab(128, kSlots, false, false);   // z, dp
+            const uint32_t id_c = idesc_bf16_ab(128, kSlots, true, true);     // dC^T
+            bool ok = mbar_wait(bar(B_CFULL), 0, abort_flag, 200, 0);
+            // the rows were written by cp.async (generic proxy); the MMA reads
+            // them through the async proxy
+            fence_proxy_async_smem();
+            for (int s = 0; ok && s < kQTiles + kVTiles; ++s) {
+                const int st = s % kRing;
+                ok = mbar_wait(bar(B_AFULL + st), (s / kRing) & 1, abort_flag, 201, s);
+                if (!ok) break;
+                tc_fence_after();
+                const bool is_z = s < kQTiles;
+                const int slab = is_z ? s : s - kQTiles;
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    const uint64_t ad = smem_desc(ring + st * kTile + kk * 32, 16, 1024, kSwizzle128B);
+                    const uint64_t bd = smem_desc(cs + slab * kCSlab + kk * 32, 16, 1024, kSwizzle128B);
+                    mma_f16_ss(tmem + (is_z ? kColZ : kColDp), ad, bd, id_a, (slab > 0 || kk > 0) ? 1u : 0u);
+                }
+                mma_commit(bar(B_AEMPTY + st));
+            }
+            if (ok) mma_commit(bar(B_ZDONE));
+            // dC^T tile m (columns 128m .. 128m+127) = Q^T g + dO^T p over the
+            // 128 heads (8 K-steps): A = a pair buffer read MN-major (two
+            // 64-column tiles, LBO = one tile), B = g or p [head][slot]
+            if (ok) ok = mbar_wait(bar(B_PG), 0, abort_flag, 202, 0);
+            if (ok) tc_fence_after();
+            int p = 0;
+            for (int m = 0; ok && m < 5; ++m) {
+                // tile 4 reuses tile 0's columns once the epilogue has read them
+                if (m == 4) {
+                    ok = mbar_wait(bar(B_T0FREE), 0, abort_flag, 204, 0);
+                    if (!ok) break;
+                    tc_fence_after();
+                }
+                const uint32_t dcol = kColDc + 64 * (m & 3);
+                for (int kind = 0; kind < (m < 4 ? 2 : 1); ++kind, ++p) {
+                    const int pb = p & 1;
+                    ok = mbar_wait(bar(B_PFULL + pb), (p >> 1) & 1, abort_flag, 203, p);
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint32_t a0 = cs + pb * 2 * kTile;
+                    const uint32_t b0 = kind == 0 ? gs : ps;
+#pragma unroll
+                    for (int ks = 0; ks < kHeads / 16; ++ks) {
+                        const uint64_t ad = smem_desc(a0 + ks * 2048, kTile, 1024, kSwizzle128B);
+                        const uint64_t bd = smem_desc(b0 + ks * 2048, kTile, 1024, kSwizzle128B);
+                        mma_f16_ss(tmem + dcol, ad, bd, id_c, (kind > 0 || ks > 0) ? 1u : 0u);
+                    }
+                    mma_commit(bar(B_PEMPTY + pb));
+                }
+                if (ok) mma_commit(bar(B_TILE + m));
+            }
+            // every MMA issued completes before TMEM is released
+            mma_commit(bar(B_DRAIN));
+            const uint64_t t0 = globaltimer_ns();
+            while (!mbar_try_wait(bar(B_DRAIN), 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
+            }
+        }
+        cp_async_wait_all();
+    } else {
+        // -------------------------------------------------------- epilogue
+        const int h = threadIdx.x - 128;                       // head = TMEM lane
+        const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
+        constexpr float kLog2e = 1.4426950408889634f;
+        // D_h = dout_h . o_h and lse in base 2
+        float D = 0.f;
+        {
+            const uint4* gr = reinterpret_cast<const uint4*>(dout + ((size_t)t * kHeads + h) * kDv);
+            const uint4* orow = reinterpret_cast<const uint4*>(out + ((size_t)t * kHeads + h) * kDv);
+#pragma unroll 4
+            for (int v = 0; v < kDv / 8; ++v) {
+                const uint4 a = __ldg(gr + v), b = __ldg(orow + v);
+                const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    D = fmaf(bf16_lo(aw[e]), bf16_lo(bw[e]), fmaf(bf16_hi(aw[e]), bf16_hi(bw[e]), D));
+            }
+        }
+        const float l2 = lse[(size_t)t * kHeads + h] * kLog2e;
+        bool ok = wait_all(bar(B_ZDONE), 0, abort_flag, 300, 0);
+        if (ok) {
+            tc_fence_after();
+            // p and g for the 64 slots, 32 at a time, as [head][slot] rows of
+            // 128 B (128B swizzle: unit u of row h at (u ^ (h % 8)) * 16), and
+            // g to g_ws
+            const float zs = scale * kLog2e;
+            uint4* gw = reinterpret_cast<uint4*>(g_ws + ((size_t)tl * kHeads + h) * kp + i0);
+#pragma unroll 1
+            for (int half = 0; half < 2; ++half) {
+                uint32_t z[32], dp[32];
+                tmem_ld32(tmem + lane_addr + kColZ + 32 * half, z);
+                tmem_ld32(tmem + lane_addr + kColDp + 32 * half, dp);
+                tmem_wait_ld();
+#pragma unroll
+                for (int uu = 0; uu < 4; ++uu) {
+                    const int u = 4 * half + uu;
+                    uint32_t pp[4], gg[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        float pv[2], gv[2];
+#pragma unroll
+                        for (int f = 0; f < 2; ++f) {
+                            const int jl = 8 * uu + 2 * e + f;
+                            const bool valid = rows[32 * half + jl] >= 0;
+                            const float p = valid ? exp2f(fmaf(__uint_as_float(z[jl]), zs, -l2)) : 0.f;
+                            pv[f] = p;
+                            gv[f] = valid ? scale * p * (__uint_as_float(dp[jl]) - D) : 0.f;
+                        }
+                        pp[e] = pack_bf16x2(pv[0], pv[1]);
+                        gg[e] = pack_bf16x2(gv[0], gv[1]);
+                    }
+                    const uint32_t off = (uint32_t)h * 128 + (((uint32_t)u ^ (h & 7)) << 4);
+                    st_shared_v4(ps + off, make_uint4(pp[0], pp[1], pp[2], pp[3]));
+                    st_shared_v4(gs + off, make_uint4(gg[0], gg[1], gg[2], gg[3]));
+                    gw[u] = make_uint4(gg[0], gg[1], gg[2], gg[3]);
+                }
+            }
+            // z and dp are read (the dC^T tiles overwrite them), and the MMA
+            // reads p and g through the async proxy
+            tc_fence_before();
+            // the MMA reads p and g through the async proxy
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(B_PG));
+        }
+        // dC^T tiles: this thread's column of tile m, 64 slots (32 at a time)
+        for (int m = 0; ok && m < 5; ++m) {
+            ok = wait_all(bar(B_TILE + m), 0, abort_flag, 301, m);
+            if (!ok) break;
+            tc_fence_after();
+            const int col = 128 * m + h;
+#pragma unroll 1
+            for (int half = 0; half < 2; ++half) {
+                uint32_t v[32];
+                tmem_ld32(tmem + lane_addr + kColDc + 64 * (m & 3) + 32 * half, v);
+                tmem_wait_ld();
+                if (m == 0 && half == 1) {
+                    // tile 0's columns are read: tile 4 may overwrite them
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar(B_T0FREE));
+                }
+                if (col < kDqk) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const long long r = rows[32 * half + j];
+                        if (r >= 0) red_add_f32(dkv + (size_t)r * kDqk + col, __uint_as_float(v[j]));
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+}
+
+}  // namespace bwd_tc
+}  // namespace dsa

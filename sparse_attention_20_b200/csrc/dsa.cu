@@ -15,6 +15,7 @@
 
 #include "dsa.h"
 #include "attn_bwd.cuh"
+#include "attn_bwd_tc.cuh"
 #include "attn_simple.cuh"
 #include "attn_tc.cuh"
 #include "common.cuh"
@@ -766,11 +767,29 @@ int attn_bwd(const __nv_bfloat16* q, const __nv_bfloat16* kv, const int32_t* idx
     e = cudaFuncSetAttribute(attn_bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s_dq);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(attn_bwd_dq_kernel)");
     __nv_bfloat16* g_ws = reinterpret_cast<__nv_bfloat16*>(workspace);
+    // the MLA head shape runs the dkv part on the tensor-core kernel
+    const bool tc = Hq == dsa::bwd_tc::kHeads && d_qk == dsa::bwd_tc::kDqk && d_v == dsa::bwd_tc::kDv;
+    CUtensorMap tq, tdo;
+    if (tc) {
+        e = cudaFuncSetAttribute(dsa::bwd_tc::attn_bwd_dkv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 dsa::bwd_tc::kSmemBytes);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(attn_bwd_dkv_tc_kernel)");
+        if (int rc = make_tmap_bf16(&tq, q, d_qk, (uint64_t)T * Hq, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return rc;
+        if (int rc = make_tmap_bf16(&tdo, dout, d_v, (uint64_t)T * Hq, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+            return rc;
+    }
     for (int r0 = 0; r0 < T; r0 += rows) {
         const int n = std::min(rows, T - r0);
-        attn_bwd_dkv_kernel<<<dim3(slots_pad(k) / kSlots, n), kThreads, s_dkv, st>>>(
-            q, kv, idx, pos, k_base, out, lse, dout, r0, T, S, Hq, d_qk, d_v, k, scale, dkv, g_ws);
-        DSA_LAUNCH_CHECK("attn_bwd_dkv_kernel");
+        if (tc) {
+            dsa::bwd_tc::attn_bwd_dkv_tc_kernel<<<dim3(slots_pad(k) / kSlots, n), dsa::bwd_tc::kThreads,
+                                                  dsa::bwd_tc::kSmemBytes, st>>>(
+                tq, tdo, kv, idx, pos, k_base, out, lse, dout, r0, T, S, k, slots_pad(k), scale, dkv, g_ws);
+            DSA_LAUNCH_CHECK("attn_bwd_dkv_tc_kernel");
+        } else {
+            attn_bwd_dkv_kernel<<<dim3(slots_pad(k) / kSlots, n), kThreads, s_dkv, st>>>(
+                q, kv, idx, pos, k_base, out, lse, dout, r0, T, S, Hq, d_qk, d_v, k, scale, dkv, g_ws);
+            DSA_LAUNCH_CHECK("attn_bwd_dkv_kernel");
+        }
         attn_bwd_dq_kernel<<<dim3(dsa::ceil_div(d_qk, kCols), n), kThreads, s_dq, st>>>(
             kv, idx, pos, k_base, g_ws, r0, T, S, Hq, d_qk, k, dq);
         DSA_LAUNCH_CHECK("attn_bwd_dq_kernel");
