@@ -358,5 +358,172 @@ attn_bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     if (warp == 0) tmem_dealloc(tmem, kTmemCols);
 }
 
+// ------------------------------------------------------------- dq kernel
+
+// dq_t = g_t C: per query row, (128 heads x slots) times (slots x 576), fp32
+// out. Three CTAs per row, each 192 output columns (a 128 x 192 fp32 TMEM
+// accumulator); per chunk of 64 slots, g by TMA ([128 heads x 64 slots],
+// 128B swizzle: the K-major A operand) and the slots' 192 columns of the
+// latent rows by cp.async (three 128B-swizzled 64-column slabs: the B
+// operand read MN-major, as the forward's PV reads them). Two stages, two
+// CTAs per SM.
+constexpr int kDqCols = 192;
+constexpr int kDqStages = 2;
+constexpr int kDqGTile = kHeads * kSlots * 2;                 // 16 KB
+constexpr int kDqCSlab = kSlots * 128;                        // 64 rows x 64 columns
+constexpr int kDqStage = kDqGTile + 3 * kDqCSlab;              // 40 KB
+constexpr int kDqOffBar = kDqStages * kDqStage;
+constexpr int kDqSmem = kDqOffBar + 256 + 1024;
+constexpr int kDqThreads = 256;
+constexpr int kDqGatherThreads = 64;
+
+enum : int { D_FULL = 0, D_EMPTY = D_FULL + kDqStages, D_DONE = D_EMPTY + kDqStages, D_COUNT = D_DONE + 1 };
+
+static_assert(kDqGTile % 1024 == 0 && kDqStage % 1024 == 0, "alignment");
+static_assert(2 * (kDqSmem + 1024) <= 233472, "two CTAs per SM");
+
+// grid: x = 192-column block (0..2), y = query row within the pass.
+// tm_g: g_ws as [rows * 128, kp] bf16, box 64 slots x 128 heads, 128B swizzle.
+__global__ void __launch_bounds__(kDqThreads, 2)
+attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_g, const __nv_bfloat16* __restrict__ kv,
+                      const int* __restrict__ idx, const int* __restrict__ pos, const int* __restrict__ k_base,
+                      int r0, int T, int S, int k, float* __restrict__ dq)
+{
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t sbase = (raw + 1023u) & ~1023u;
+    uint8_t* sgen = smem_raw + (sbase - raw);
+    const uint32_t bar0 = sbase + kDqOffBar;
+    auto bar = [&](int i) -> uint32_t { return bar0 + 8u * (uint32_t)i; };
+    uint32_t* taddr_slot = reinterpret_cast<uint32_t*>(sgen + kDqOffBar + 8 * D_COUNT);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sgen + kDqOffBar + 8 * D_COUNT + 8);
+
+    const int tl = blockIdx.y, t = r0 + tl, cb = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    long long base;
+    const int n_cand = row_candidates(pos, k_base, t, T, S, &base);
+    const int n_ent = min(k, n_cand);
+    const int n_chunks = (n_ent + kSlots - 1) / kSlots;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kDqStages; ++s) {
+            mbar_init(bar(D_FULL + s), kDqGatherThreads + 1);   // gather threads + the TMA arrival
+            mbar_init(bar(D_EMPTY + s), 1);
+        }
+        mbar_init(bar(D_DONE), 1);
+        *abort_flag = 0;
+        fence_mbar_init_cluster();
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_u32(taddr_slot), 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *taddr_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------- MMA
+        if (lane == 0 && n_chunks > 0) {
+            const uint32_t id = idesc_bf16_ab(128, kDqCols, false, true);
+            bool ok = true;
+            for (int c = 0; ok && c < n_chunks; ++c) {
+                const int st = c % kDqStages;
+                ok = mbar_wait(bar(D_FULL + st), (c / kDqStages) & 1, abort_flag, 400, c);
+                if (!ok) break;
+                // the rows were written by cp.async (generic proxy)
+                fence_proxy_async_smem();
+                tc_fence_after();
+                const uint32_t gt = sbase + st * kDqStage, ct = gt + kDqGTile;
+#pragma unroll
+                for (int kk = 0; kk < kSlots / 16; ++kk) {
+                    const uint64_t ad = smem_desc(gt + kk * 32, 16, 1024, kSwizzle128B);
+                    const uint64_t bd = smem_desc(ct + kk * 2048, kDqCSlab, 1024, kSwizzle128B);
+                    mma_f16_ss(tmem, ad, bd, id, (c > 0 || kk > 0) ? 1u : 0u);
+                }
+                mma_commit(bar(D_EMPTY + st));
+            }
+            mma_commit(bar(D_DONE));
+        }
+    } else if (warp == 1) {
+        // -------------------------------------------------------- TMA of g
+        if (lane == 0) {
+            prefetch_tmap(&tm_g);
+            for (int c = 0; c < n_chunks; ++c) {
+                const int st = c % kDqStages;
+                if (c >= kDqStages &&
+                    !mbar_wait(bar(D_EMPTY + st), ((c - kDqStages) / kDqStages) & 1, abort_flag, 401, c))
+                    break;
+                mbar_arrive_expect_tx(bar(D_FULL + st), kDqGTile);
+                tma_load_2d(sbase + st * kDqStage, &tm_g, kSlots * c, tl * kHeads, bar(D_FULL + st));
+            }
+        }
+    } else if (warp <= 3) {
+        // ---------------------------------------------------------- gather
+        // Thread r copies slot r's 24 sixteen-byte pieces (192 columns) of
+        // every chunk: piece p goes to slab p/8, unit (p%8) ^ (r%8) of the
+        // row's 128 bytes. The next chunk's index is loaded one chunk ahead.
+        const int r = threadIdx.x - 64;
+        const char* kvb = reinterpret_cast<const char*>(kv);
+        auto slot_of = [&](int c) -> int {
+            const int i = c * kSlots + r;
+            const int s = i < n_ent ? idx[(size_t)t * k + i] : -1;
+            return (s >= 0 && s < n_cand) ? s : -1;
+        };
+        int s_next = n_chunks > 0 ? slot_of(0) : -1;
+        for (int c = 0; c < n_chunks; ++c) {
+            const int st = c % kDqStages;
+            const int s = s_next;
+            if (c + 1 < n_chunks) s_next = slot_of(c + 1);
+            if (c >= kDqStages) {
+                const bool got = mbar_wait(bar(D_EMPTY + st), ((c - kDqStages) / kDqStages) & 1, abort_flag, 402, c);
+                if (!__all_sync(0xffffffffu, got)) break;
+            }
+            const uint32_t ct = sbase + st * kDqStage + kDqGTile + r * 128;
+            const char* src = s >= 0 ? kvb + (base + s) * (kDqk * 2) + kDqCols * cb * 2 : kvb;
+#pragma unroll
+            for (int pc = 0; pc < 24; ++pc)
+                cp_async16(ct + (pc >> 3) * kDqCSlab + (((pc & 7) ^ (r & 7)) << 4), s >= 0 ? src + pc * 16 : kvb,
+                           s >= 0 ? 16u : 0u);
+            cp_async_arrive_noinc(bar(D_FULL + st));
+        }
+        cp_async_wait_all();
+    } else {
+        // -------------------------------------------------------- epilogue
+        const int h = threadIdx.x - 128;                       // head = TMEM lane
+        const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
+        float* dst = dq + ((size_t)t * kHeads + h) * kDqk + kDqCols * cb;
+        bool ok = true;
+        if (n_chunks > 0) {
+            ok = wait_all(bar(D_DONE), 0, abort_flag, 403, 0);
+            if (ok) tc_fence_after();
+        }
+        if (ok) {
+#pragma unroll 1
+            for (int q = 0; q < kDqCols / 32; ++q) {
+                uint32_t v[32];
+                if (n_chunks > 0) {
+                    tmem_ld32(tmem + lane_addr + 32 * q, v);
+                    tmem_wait_ld();
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) v[e] = 0u;
+                }
+                float4* d4 = reinterpret_cast<float4*>(dst + 32 * q);
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    d4[e] = make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
+                                        __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, 256);
+}
+
 }  // namespace bwd_tc
 }  // namespace dsa

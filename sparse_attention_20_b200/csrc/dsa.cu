@@ -769,7 +769,7 @@ int attn_bwd(const __nv_bfloat16* q, const __nv_bfloat16* kv, const int32_t* idx
     __nv_bfloat16* g_ws = reinterpret_cast<__nv_bfloat16*>(workspace);
     // the MLA head shape runs the dkv part on the tensor-core kernel
     const bool tc = Hq == dsa::bwd_tc::kHeads && d_qk == dsa::bwd_tc::kDqk && d_v == dsa::bwd_tc::kDv;
-    CUtensorMap tq, tdo;
+    CUtensorMap tq, tdo, tg;
     if (tc) {
         e = cudaFuncSetAttribute(dsa::bwd_tc::attn_bwd_dkv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  dsa::bwd_tc::kSmemBytes);
@@ -777,6 +777,13 @@ int attn_bwd(const __nv_bfloat16* q, const __nv_bfloat16* kv, const int32_t* idx
         if (int rc = make_tmap_bf16(&tq, q, d_qk, (uint64_t)T * Hq, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return rc;
         if (int rc = make_tmap_bf16(&tdo, dout, d_v, (uint64_t)T * Hq, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
             return rc;
+        // g_ws as [rows * 128, kp]: boxes of 64 slots x 128 heads
+        if (int rc = make_tmap_bf16(&tg, g_ws, slots_pad(k), (uint64_t)rows * Hq, 64, 128,
+                                    CU_TENSOR_MAP_SWIZZLE_128B))
+            return rc;
+        e = cudaFuncSetAttribute(dsa::bwd_tc::attn_bwd_dq_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 dsa::bwd_tc::kDqSmem);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(attn_bwd_dq_tc_kernel)");
     }
     for (int r0 = 0; r0 < T; r0 += rows) {
         const int n = std::min(rows, T - r0);
@@ -790,9 +797,16 @@ int attn_bwd(const __nv_bfloat16* q, const __nv_bfloat16* kv, const int32_t* idx
                 q, kv, idx, pos, k_base, out, lse, dout, r0, T, S, Hq, d_qk, d_v, k, scale, dkv, g_ws);
             DSA_LAUNCH_CHECK("attn_bwd_dkv_kernel");
         }
-        attn_bwd_dq_kernel<<<dim3(dsa::ceil_div(d_qk, kCols), n), kThreads, s_dq, st>>>(
-            kv, idx, pos, k_base, g_ws, r0, T, S, Hq, d_qk, k, dq);
-        DSA_LAUNCH_CHECK("attn_bwd_dq_kernel");
+        if (tc) {
+            dsa::bwd_tc::attn_bwd_dq_tc_kernel<<<dim3(d_qk / dsa::bwd_tc::kDqCols, n), dsa::bwd_tc::kDqThreads,
+                                                 dsa::bwd_tc::kDqSmem, st>>>(tg, kv, idx, pos, k_base, r0, T, S, k,
+                                                                             dq);
+            DSA_LAUNCH_CHECK("attn_bwd_dq_tc_kernel");
+        } else {
+            attn_bwd_dq_kernel<<<dim3(dsa::ceil_div(d_qk, kCols), n), kThreads, s_dq, st>>>(
+                kv, idx, pos, k_base, g_ws, r0, T, S, Hq, d_qk, k, dq);
+            DSA_LAUNCH_CHECK("attn_bwd_dq_kernel");
+        }
     }
     return DSA_OK;
 }
