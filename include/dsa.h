@@ -211,7 +211,7 @@ int dsa_sparse_mla_attn_split(const void* q, const void* kv, const int32_t* idx,
  * with T = 1); more lets the call take more rows per pass (up to 8192 per
  * pass, DSA_ERR_WORKSPACE below one row). Rows are processed in passes of
  * that many rows on `stream`; the workspace holds the bf16 scale*dz of one
- * pass between its two kernels.
+ * pass between its kernels, and each row's per-head dO.O.
  * Supported: Hq <= 128, d_qk % 16 == 0, d_qk <= 576, d_v % 16 == 0,
  * d_v <= d_qk, 1 <= k <= 4096 (DSA_ERR_UNSUPPORTED otherwise).
  */

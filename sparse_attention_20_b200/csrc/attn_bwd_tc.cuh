@@ -16,8 +16,8 @@
 //  - warps 1-3 gather the 64 selected latent rows (cp.async, 128B-swizzled
 //    64-column slabs, K-major B operand of z and dp); warp 1's first thread
 //    then issues every MMA;
-//  - warps 4-7 (one head per thread, the TMEM lane) form D and lse first,
-//    then read z and dp from TMEM, write p and g as MN-major tiles
+//  - warps 4-7 (one head per thread, the TMEM lane) read D (formed once per
+//    row by attn_bwd_delta_kernel) and lse, then read z and dp from TMEM, write p and g as MN-major tiles
 //    [head][slot] in the ring's space (the B operands of dC^T, whose A
 //    operands are the Q / dO tiles read MN-major), and finally add each dC^T
 //    tile (M = 128 columns, N = 64 slots) into dkv.
@@ -85,15 +85,45 @@ __device__ __forceinline__ void red_add_f32(float* p, float v)
     asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
 }
 
+// D_h = dout_h . o_h of every head of the pass's rows: d_ws[row][128] (fp32).
+// One CTA of 256 threads per row; warp w takes heads 16w .. 16w+15, its lanes
+// eight columns at a time.
+__global__ void __launch_bounds__(256)
+attn_bwd_delta_kernel(const __nv_bfloat16* __restrict__ out, const __nv_bfloat16* __restrict__ dout, int r0,
+                      float* __restrict__ d_ws)
+{
+    const int tl = blockIdx.x, t = r0 + tl;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int hh = 0; hh < 16; ++hh) {
+        const int h = warp * 16 + hh;
+        const uint4* gr = reinterpret_cast<const uint4*>(dout + ((size_t)t * kHeads + h) * kDv);
+        const uint4* orow = reinterpret_cast<const uint4*>(out + ((size_t)t * kHeads + h) * kDv);
+        float acc = 0.f;
+#pragma unroll
+        for (int it = 0; it < kDv / 256; ++it) {
+            const uint4 a = __ldg(gr + it * 32 + lane), b = __ldg(orow + it * 32 + lane);
+            const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                acc = fmaf(bf16_lo(aw[e]), bf16_lo(bw[e]), fmaf(bf16_hi(aw[e]), bf16_hi(bw[e]), acc));
+        }
+#pragma unroll
+        for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (lane == 0) d_ws[(size_t)tl * kHeads + h] = acc;
+    }
+}
+
 // grid: x = slot chunk (64 slots), y = query row within the pass [r0, r0 + gridDim.y).
-// g_ws: bf16 [rows][128][slots_pad(k)], as attn_bwd_dkv_kernel writes it.
+// g_ws: bf16 [rows][128][slots_pad(k)], as attn_bwd_dkv_kernel writes it;
+// d_ws: fp32 [rows][128], from attn_bwd_delta_kernel.
 __global__ void __launch_bounds__(kThreads, 2)
 attn_bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                        const __nv_bfloat16* __restrict__ kv, const int* __restrict__ idx,
                        const int* __restrict__ pos, const int* __restrict__ k_base,
                        const __nv_bfloat16* __restrict__ out, const float* __restrict__ lse,
                        const __nv_bfloat16* __restrict__ dout, int r0, int T, int S, int k, int kp,
-                       float scale, float* __restrict__ dkv, __nv_bfloat16* __restrict__ g_ws)
+                       float scale, float* __restrict__ dkv, __nv_bfloat16* __restrict__ g_ws,
+                       const float* __restrict__ d_ws)
 {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -263,20 +293,8 @@ attn_bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
         const int h = threadIdx.x - 128;                       // head = TMEM lane
         const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
         constexpr float kLog2e = 1.4426950408889634f;
-        // D_h = dout_h . o_h and lse in base 2
-        float D = 0.f;
-        {
-            const uint4* gr = reinterpret_cast<const uint4*>(dout + ((size_t)t * kHeads + h) * kDv);
-            const uint4* orow = reinterpret_cast<const uint4*>(out + ((size_t)t * kHeads + h) * kDv);
-#pragma unroll 4
-            for (int v = 0; v < kDv / 8; ++v) {
-                const uint4 a = __ldg(gr + v), b = __ldg(orow + v);
-                const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    D = fmaf(bf16_lo(aw[e]), bf16_lo(bw[e]), fmaf(bf16_hi(aw[e]), bf16_hi(bw[e]), D));
-            }
-        }
+        // D_h = dout_h . o_h (formed per row) and lse in base 2
+        const float D = d_ws[(size_t)tl * kHeads + h];
         const float l2 = lse[(size_t)t * kHeads + h] * kLog2e;
         bool ok = wait_all(bar(B_ZDONE), 0, abort_flag, 300, 0);
         if (ok) {

@@ -727,9 +727,10 @@ int attn_dispatch(const void* q, const void* kv, const int32_t* idx, const int32
 
 constexpr int kBwdRowsMax = 8192;   // query rows per pass of the backward (workspace size)
 
+// Per row of a pass: g (bf16 [heads_pad][slots_pad]) and D (fp32 [heads_pad]).
 size_t attn_bwd_row_bytes(int Hq, int k)
 {
-    return (size_t)dsa::bwd::heads_pad(Hq) * dsa::bwd::slots_pad(k) * sizeof(__nv_bfloat16);
+    return (size_t)dsa::bwd::heads_pad(Hq) * (dsa::bwd::slots_pad(k) * sizeof(__nv_bfloat16) + sizeof(float));
 }
 
 int check_attn_bwd(const void* q, const void* kv, const int32_t* idx, const int32_t* pos,
@@ -767,6 +768,9 @@ int attn_bwd(const __nv_bfloat16* q, const __nv_bfloat16* kv, const int32_t* idx
     e = cudaFuncSetAttribute(attn_bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s_dq);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(attn_bwd_dq_kernel)");
     __nv_bfloat16* g_ws = reinterpret_cast<__nv_bfloat16*>(workspace);
+    // D per row after the pass's g rows (16-byte aligned: heads_pad * slots_pad * 2 is)
+    float* d_ws = reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) +
+                                           (size_t)rows * heads_pad(Hq) * slots_pad(k) * sizeof(__nv_bfloat16));
     // the MLA head shape runs the dkv part on the tensor-core kernel
     const bool tc = Hq == dsa::bwd_tc::kHeads && d_qk == dsa::bwd_tc::kDqk && d_v == dsa::bwd_tc::kDv;
     CUtensorMap tq, tdo, tg;
@@ -788,9 +792,11 @@ int attn_bwd(const __nv_bfloat16* q, const __nv_bfloat16* kv, const int32_t* idx
     for (int r0 = 0; r0 < T; r0 += rows) {
         const int n = std::min(rows, T - r0);
         if (tc) {
+            dsa::bwd_tc::attn_bwd_delta_kernel<<<n, 256, 0, st>>>(out, dout, r0, d_ws);
+            DSA_LAUNCH_CHECK("attn_bwd_delta_kernel");
             dsa::bwd_tc::attn_bwd_dkv_tc_kernel<<<dim3(slots_pad(k) / kSlots, n), dsa::bwd_tc::kThreads,
                                                   dsa::bwd_tc::kSmemBytes, st>>>(
-                tq, tdo, kv, idx, pos, k_base, out, lse, dout, r0, T, S, k, slots_pad(k), scale, dkv, g_ws);
+                tq, tdo, kv, idx, pos, k_base, out, lse, dout, r0, T, S, k, slots_pad(k), scale, dkv, g_ws, d_ws);
             DSA_LAUNCH_CHECK("attn_bwd_dkv_tc_kernel");
         } else {
             attn_bwd_dkv_kernel<<<dim3(slots_pad(k) / kSlots, n), kThreads, s_dkv, st>>>(

@@ -133,9 +133,9 @@ def test_attention_backward_rejects_bad_arguments(lib):
     assert call(d_qk=576, d_v=504) == -2  # d_v not a multiple of 16
     assert call(wsb=ctypes.c_size_t(100)) == -5
     assert call(wsp=None) == -5
-    # one row of scratch: heads padded to 16, slots to 64, bf16
-    assert lib.dsa_sparse_mla_attn_bwd_workspace_size(1, 4, 32) == 16 * 64 * 2
-    assert lib.dsa_sparse_mla_attn_bwd_workspace_size(100000, 128, 2048) == 8192 * 128 * 2048 * 2
+    # one row of scratch: g (bf16, heads padded to 16, slots to 64) and D (fp32 per head)
+    assert lib.dsa_sparse_mla_attn_bwd_workspace_size(1, 4, 32) == 16 * 64 * 2 + 16 * 4
+    assert lib.dsa_sparse_mla_attn_bwd_workspace_size(100000, 128, 2048) == 8192 * 128 * (2048 * 2 + 4)
     assert lib.dsa_sparse_mla_attn_bwd_workspace_size(0, 128, 2048) == 0
 
 

@@ -94,7 +94,7 @@ def test_bwd_multi_pass_and_empty_rows():
     """A workspace of 3 rows forces several passes; rows without entries give dq = 0."""
     x, idx, dout = _case("tiny", 2, L=150)
     idx[[0, 7, 149]] = -1
-    ws = torch.empty(3 * 16 * 64 * 2, dtype=torch.uint8, device="cuda")
+    ws = torch.empty(3 * 16 * (64 * 2 + 4), dtype=torch.uint8, device="cuda")
     dq, dkv = _gpu(x, idx.cuda(), dout, workspace=ws)
     dq1, dkv1 = _gpu(x, idx.cuda(), dout)
     assert np.array_equal(dq, dq1)
