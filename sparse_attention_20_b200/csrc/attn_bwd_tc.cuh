@@ -543,5 +543,164 @@ attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_g, const __nv_bfloa
     if (warp == 0) tmem_dealloc(tmem, 256);
 }
 
+// ------------------------------------------------ head-summed probabilities
+
+// The indexer KL loss's target for the MLA head shape: per query row and
+// chunk of 64 selected slots, psum_s = sum_h exp(scale q_h.c_s - lse_h) (0
+// for non-candidates), into psum [rows][kp] fp32. z = Q_t C^T as in
+// attn_bwd_dkv_tc_kernel (Q_t by TMA in nine 64-column tiles, 2-stage ring;
+// the gathered rows the K-major B operand; z in TMEM), then each epilogue
+// thread (one head) forms its 64 probabilities and every warp sums them over
+// its 32 heads with a halving exchange (lane L ends with slots 2L and
+// 2L + 1), the four warps' sums meeting in shared memory.
+constexpr int kPsOffRing = kQTiles * kCSlab;                 // after the gathered rows
+constexpr int kPsOffRows = kPsOffRing + 2 * kTile;
+constexpr int kPsOffRed = kPsOffRows + kSlots * 8;           // [4 warps][64] fp32
+constexpr int kPsOffBar = kPsOffRed + 4 * kSlots * 4;
+constexpr int kPsSmem = kPsOffBar + 256 + 1024;
+
+enum : int { H_CFULL = 0, H_AFULL = 1, H_AEMPTY = 3, H_ZDONE = 5, H_COUNT = 6 };
+
+static_assert(kPsOffRing % 1024 == 0, "alignment");
+static_assert(2 * (kPsSmem + 1024) <= 233472, "two CTAs per SM");
+
+__global__ void __launch_bounds__(kThreads, 2)
+head_prob_sum_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __nv_bfloat16* __restrict__ kv,
+                        const int* __restrict__ idx, const int* __restrict__ pos, const int* __restrict__ k_base,
+                        const float* __restrict__ lse, int r0, int T, int S, int k, int kp, float scale,
+                        float* __restrict__ psum)
+{
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t sbase = (raw + 1023u) & ~1023u;
+    uint8_t* sgen = smem_raw + (sbase - raw);
+    const uint32_t bar0 = sbase + kPsOffBar;
+    auto bar = [&](int i) -> uint32_t { return bar0 + 8u * (uint32_t)i; };
+    uint32_t* taddr_slot = reinterpret_cast<uint32_t*>(sgen + kPsOffBar + 8 * H_COUNT);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sgen + kPsOffBar + 8 * H_COUNT + 8);
+    long long* rows = reinterpret_cast<long long*>(sgen + kPsOffRows);
+    float* red = reinterpret_cast<float*>(sgen + kPsOffRed);
+
+    const int tl = blockIdx.y, t = r0 + tl, i0 = blockIdx.x * kSlots;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    long long base;
+    const int n_cand = row_candidates(pos, k_base, t, T, S, &base);
+    if (i0 >= min(k, n_cand)) return;   // whole chunk past the row's entries (uniform per CTA)
+
+    if (threadIdx.x < kSlots) {
+        const int i = i0 + threadIdx.x;
+        const int s = i < k ? idx[(size_t)t * k + i] : -1;
+        rows[threadIdx.x] = (i < k && s >= 0 && s < n_cand) ? base + s : -1ll;
+    }
+    if (threadIdx.x == 0) {
+        mbar_init(bar(H_CFULL), kGatherThreads);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(bar(H_AFULL + s), 1);
+            mbar_init(bar(H_AEMPTY + s), 1);
+        }
+        mbar_init(bar(H_ZDONE), 1);
+        *abort_flag = 0;
+        fence_mbar_init_cluster();
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_u32(taddr_slot), 64);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *taddr_slot;
+    const uint32_t cs = sbase, ring = sbase + kPsOffRing;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            prefetch_tmap(&tm_q);
+            for (int s = 0; s < kQTiles; ++s) {
+                const int st = s & 1;
+                if (s >= 2 && !mbar_wait(bar(H_AEMPTY + st), ((s - 2) >> 1) & 1, abort_flag, 500, s)) break;
+                mbar_arrive_expect_tx(bar(H_AFULL + st), kTile);
+                tma_load_2d(ring + st * kTile, &tm_q, 64 * s, t * kHeads, bar(H_AFULL + st));
+            }
+        }
+    } else if (warp <= 3) {
+        const int g = threadIdx.x - 32;
+        const char* kvb = reinterpret_cast<const char*>(kv);
+        for (int e = g; e < kSlots * 72; e += kGatherThreads) {
+            const int r = e / 72, j = e - r * 72;
+            const long long row = rows[r];
+            const uint32_t dst = cs + (j >> 3) * kCSlab + r * 128 + (((j & 7) ^ (r & 7)) << 4);
+            cp_async16(dst, row >= 0 ? kvb + row * (kDqk * 2) + j * 16 : kvb, row >= 0 ? 16u : 0u);
+        }
+        cp_async_arrive_noinc(bar(H_CFULL));
+        if (warp == 1 && lane == 0) {
+            const uint32_t id = idesc_bf16_ab(128, kSlots, false, false);
+            bool ok = mbar_wait(bar(H_CFULL), 0, abort_flag, 501, 0);
+            fence_proxy_async_smem();
+            for (int s = 0; ok && s < kQTiles; ++s) {
+                const int st = s & 1;
+                ok = mbar_wait(bar(H_AFULL + st), (s >> 1) & 1, abort_flag, 502, s);
+                if (!ok) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    const uint64_t ad = smem_desc(ring + st * kTile + kk * 32, 16, 1024, kSwizzle128B);
+                    const uint64_t bd = smem_desc(cs + s * kCSlab + kk * 32, 16, 1024, kSwizzle128B);
+                    mma_f16_ss(tmem, ad, bd, id, (s > 0 || kk > 0) ? 1u : 0u);
+                }
+                mma_commit(bar(H_AEMPTY + st));
+            }
+            mma_commit(bar(H_ZDONE));
+            const uint64_t t0 = globaltimer_ns();
+            while (!mbar_try_wait(bar(H_ZDONE), 0) && globaltimer_ns() - t0 < kWaitLimitNs) {
+            }
+        }
+        cp_async_wait_all();
+    } else {
+        const int h = threadIdx.x - 128;
+        const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
+        constexpr float kLog2e = 1.4426950408889634f;
+        const float l2 = lse[(size_t)t * kHeads + h] * kLog2e, zs = scale * kLog2e;
+        const bool ok = wait_all(bar(H_ZDONE), 0, abort_flag, 503, 0);
+        float v[64];
+        if (ok) {
+            tc_fence_after();
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                uint32_t z[32];
+                tmem_ld32(tmem + lane_addr + 32 * half, z);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    v[32 * half + j] = rows[32 * half + j] >= 0 ? exp2f(fmaf(__uint_as_float(z[j]), zs, -l2)) : 0.f;
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < 64; ++j) v[j] = 0.f;
+        }
+        // halving exchange: keep the lower or upper half of the current slot
+        // range (by lane bit o), add the partner's copy of it
+#pragma unroll
+        for (int o = 16, n = 64; o >= 1; o >>= 1, n >>= 1) {
+            const bool up = (lane & o) != 0;
+#pragma unroll
+            for (int i = 0; i < n / 2; ++i) {
+                const float send = up ? v[i] : v[i + n / 2];
+                const float keep = up ? v[i + n / 2] : v[i];
+                v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+            }
+        }
+        red[(warp & 3) * kSlots + 2 * lane] = v[0];
+        red[(warp & 3) * kSlots + 2 * lane + 1] = v[1];
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (ok && h < kSlots)
+            psum[(size_t)tl * kp + i0 + h] = red[h] + red[kSlots + h] + red[2 * kSlots + h] + red[3 * kSlots + h];
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, 64);
+}
+
 }  // namespace bwd_tc
 }  // namespace dsa

@@ -864,11 +864,27 @@ int indexer_kl(const __nv_bfloat16* q, const __nv_bfloat16* kv, const int32_t* i
     e = cudaFuncSetAttribute(indexer_kl_row_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s_row);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(indexer_kl_row_kernel)");
     float* psum = reinterpret_cast<float*>(workspace);
+    // the MLA head shape forms the head-summed probabilities on the tensor cores
+    const bool tc = Hq == dsa::bwd_tc::kHeads && d_qk == dsa::bwd_tc::kDqk;
+    CUtensorMap tq;
+    if (tc) {
+        e = cudaFuncSetAttribute(dsa::bwd_tc::head_prob_sum_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 dsa::bwd_tc::kPsSmem);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(head_prob_sum_tc_kernel)");
+        if (int rc = make_tmap_bf16(&tq, q, d_qk, (uint64_t)T * Hq, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)) return rc;
+    }
     for (int r0 = 0; r0 < T; r0 += rows) {
         const int n = std::min(rows, T - r0);
-        head_prob_sum_kernel<<<dim3(dsa::bwd::slots_pad(k) / dsa::bwd::kSlots, n), dsa::bwd::kThreads, s_prob,
-                               st>>>(q, kv, idx, pos, k_base, lse, r0, T, S, Hq, d_qk, k, scale, psum);
-        DSA_LAUNCH_CHECK("head_prob_sum_kernel");
+        if (tc) {
+            dsa::bwd_tc::head_prob_sum_tc_kernel<<<dim3(dsa::bwd::slots_pad(k) / dsa::bwd::kSlots, n),
+                                                   dsa::bwd_tc::kThreads, dsa::bwd_tc::kPsSmem, st>>>(
+                tq, kv, idx, pos, k_base, lse, r0, T, S, k, dsa::bwd::slots_pad(k), scale, psum);
+            DSA_LAUNCH_CHECK("head_prob_sum_tc_kernel");
+        } else {
+            head_prob_sum_kernel<<<dim3(dsa::bwd::slots_pad(k) / dsa::bwd::kSlots, n), dsa::bwd::kThreads, s_prob,
+                                   st>>>(q, kv, idx, pos, k_base, lse, r0, T, S, Hq, d_qk, k, scale, psum);
+            DSA_LAUNCH_CHECK("head_prob_sum_kernel");
+        }
         indexer_kl_row_kernel<<<n, kRowThreads, s_row, st>>>(q_idx, w, k_idx, idx, pos, k_base, psum, r0, T, S,
                                                              H_I, d_I, k, loss, dw, dqi, dki);
         DSA_LAUNCH_CHECK("indexer_kl_row_kernel");
