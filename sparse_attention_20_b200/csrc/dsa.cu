@@ -16,6 +16,7 @@
 #include "dsa.h"
 #include "attn_bwd.cuh"
 #include "attn_bwd_tc.cuh"
+#include "mha_tc.cuh"
 #include "attn_simple.cuh"
 #include "attn_tc.cuh"
 #include "common.cuh"
@@ -1140,6 +1141,27 @@ int dsa_indexer_kl(const void* q, const void* kv, const int32_t* idx, const int3
                       reinterpret_cast<cudaStream_t>(stream));
 }
 
+// MHA mode, (d_h, d_hv) = (192, 128), on the tensor cores: TMA maps over the
+// head-interleaved rows of q, k and v.
+int mha_tc_launch(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v, int T, int S, int Hq,
+                  float scale, __nv_bfloat16* out, float* lse, cudaStream_t st)
+{
+    using namespace dsa::mha_tc;
+    cudaError_t e = cudaFuncSetAttribute(mha_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(mha_tc_kernel)");
+    CUtensorMap tq, tk, tv;
+    if (int rc = make_tmap_bf16(&tq, q, (uint64_t)Hq * kDh, (uint64_t)T, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+        return rc;
+    if (int rc = make_tmap_bf16(&tk, k, (uint64_t)Hq * kDh, (uint64_t)S, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+        return rc;
+    if (int rc = make_tmap_bf16(&tv, v, (uint64_t)Hq * kDv, (uint64_t)S, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+        return rc;
+    mha_tc_kernel<<<dim3(dsa::ceil_div(T, kRows), Hq), kThreads, kSmemBytes, st>>>(
+        tq, tk, tv, T, S, Hq, scale * 1.4426950408889634f, out, lse);
+    DSA_LAUNCH_CHECK("mha_tc_kernel");
+    return DSA_OK;
+}
+
 int dsa_mla_mha_attn(const void* q, const void* k, const void* v, int T, int S, int Hq, int d_h, int d_hv,
                      float scale, void* out, float* lse, void* stream)
 {
@@ -1154,7 +1176,7 @@ int dsa_mla_mha_attn(const void* q, const void* k, const void* v, int T, int S, 
     const bf *qq = reinterpret_cast<const bf*>(q), *kk = reinterpret_cast<const bf*>(k),
              *vv = reinterpret_cast<const bf*>(v);
     bf* oo = reinterpret_cast<bf*>(out);
-    if (d_h == 192 && d_hv == 128) return mha_launch<192, 128>(qq, kk, vv, T, S, Hq, scale, oo, lse, st);
+    if (d_h == 192 && d_hv == 128) return mha_tc_launch(qq, kk, vv, T, S, Hq, scale, oo, lse, st);
     if (d_h == 64 && d_hv == 64) return mha_launch<64, 64>(qq, kk, vv, T, S, Hq, scale, oo, lse, st);
     return fail(DSA_ERR_UNSUPPORTED, "d_h=%d, d_hv=%d (supported: (192, 128), (64, 64))", d_h, d_hv);
 }

@@ -51,6 +51,13 @@ def test_mha_192_128_all_rows(L, Hq):
     _check(*synth.mha_inputs("mha_short", device="cuda", seed=1, L=L, Hq=Hq))
 
 
+@pytest.mark.parametrize("L,T,Hq", [(1000, 300, 4), (129, 1, 2), (256, 256, 1)])
+def test_mha_192_128_tail_rows(L, T, Hq):
+    """The last T query rows of L tokens (pos[t] = t + L - T): query tiles
+    start past key tiles, the single-row case, and exact 128-row tiles."""
+    _check(*synth.mha_inputs("mha_short", device="cuda", seed=3, L=L, T=T, Hq=Hq))
+
+
 def test_mha_short_prefill_sampled_rows():
     """The 2048-token, 128-head short prefill bench.py --mha times."""
     q, k, v, scale = synth.mha_inputs("mha_short", device="cuda", seed=2)
