@@ -324,7 +324,7 @@ def attn_traffic():
                             ("attn_tc.cuh", "sm100.cuh", "common.cuh", "dsa.cu"))
 
 
-MHA_SOURCES = ("mha_attn.cuh", "attn_bwd.cuh", "sm100.cuh", "common.cuh", "dsa.cu")
+MHA_SOURCES = ("mha_tc.cuh", "mha_attn.cuh", "attn_bwd.cuh", "sm100.cuh", "common.cuh", "dsa.cu")
 
 
 def fp8_gemm_tflops(n=8192, reps=10):
@@ -942,7 +942,8 @@ def bench_mha(args, world, rank, local):
         "config": {"workload": f"{args.mha}: L={S}, rows={T}, Hq={Hq}, d_h={d_h}, d_hv={d_hv}, dense causal; "
                                f"inputs larger than L2, no flush",
                    "global_batch": world, "seq_len": S, "parallelism": f"replicas{world}"},
-        "roofline": {"bound": "tensor", "kernel": "mha_causal_kernel", "achieved": tf,
+        "roofline": {"bound": "tensor", "kernel": "mha_tc_kernel" if (d_h, d_hv) == (192, 128) else "mha_causal_kernel",
+                     "achieved": tf,
                      "peak": peaks["bf16"], "unit": "TFLOP/s", "frac": tf / peaks["bf16"],
                      "frac_of_sustained": tf / peaks["bf16_sustained"],
                      "traffic": (profiled_traffic("mha_causal_short_prefill2k.md", "mha", MHA_SOURCES)
