@@ -946,7 +946,7 @@ def bench_mha(args, world, rank, local):
                      "achieved": tf,
                      "peak": peaks["bf16"], "unit": "TFLOP/s", "frac": tf / peaks["bf16"],
                      "frac_of_sustained": tf / peaks["bf16_sustained"],
-                     "traffic": (profiled_traffic("mha_causal_short_prefill2k.md", "mha", MHA_SOURCES)
+                     "traffic": (profiled_traffic("mha_tc_short_prefill2k.md", "mha", MHA_SOURCES)
                                  if args.mha == "mha_short" and args.seq_len is None else None),
                      "peak_source": f"{peaks['source']} bf16 burst"},
         "gpu_launches": launches, "clocks": clk,
