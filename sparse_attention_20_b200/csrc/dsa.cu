@@ -1156,7 +1156,9 @@ int mha_tc_launch(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfl
         return rc;
     if (int rc = make_tmap_bf16(&tv, v, (uint64_t)Hq * kDv, (uint64_t)S, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
         return rc;
-    mha_tc_kernel<<<dim3(dsa::ceil_div(T, kRows), Hq), kThreads, kSmemBytes, st>>>(
+    // persistent: one CTA per SM walking the (query tile, head) units
+    const int units = dsa::ceil_div(T, kRows) * Hq;
+    mha_tc_kernel<<<std::min(units, num_sms()), kThreads, kSmemBytes, st>>>(
         tq, tk, tv, T, S, Hq, scale * 1.4426950408889634f, out, lse);
     DSA_LAUNCH_CHECK("mha_tc_kernel");
     return DSA_OK;

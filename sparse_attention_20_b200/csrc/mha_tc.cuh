@@ -2,7 +2,10 @@
 // value rows; mha_attn.cuh states the operation) on the 5th-generation tensor
 // cores, for the (d_h, d_hv) = (192, 128) head shape.
 //
-// One CTA of 384 threads per (128 query rows, head), one per SM:
+// Persistent: one CTA of 384 threads per SM walks the work units (128 query
+// rows, head) in order of decreasing causal length; every per-tile barrier
+// counts tiles across units, so the K/V ring and the QK MMAs run on into the
+// next unit while the softmax warps finish the current one:
 //  - warp 1 (one thread) loads the Q tile and streams 128-key tiles of K and
 //    V by TMA from the head's column window of the row-major tensors
 //    ([rows, Hq * d] bf16; 64-column boxes of 128 rows, 128B swizzle; a
@@ -36,8 +39,8 @@ constexpr int kStages = 2;
 constexpr int kOffQ = 0;
 constexpr int kOffKV = kOffQ + kQBytes;
 constexpr int kOffRed = kOffKV + kStages * kStageBytes;   // [2 parities][2 halves][128] row maxima
-constexpr int kOffLsum = kOffRed + 2 * 2 * kRows * 4;     // [2 halves][128] row sums
-constexpr int kOffBar = kOffLsum + 2 * kRows * 4;
+constexpr int kOffLsum = kOffRed + 2 * 2 * kRows * 4;     // [2 unit parities][2 halves][128] row sums
+constexpr int kOffBar = kOffLsum + 2 * 2 * kRows * 4;
 constexpr int kSmemBytes = kOffBar + 256 + 1024;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 0, kColS = 128, kColP = 384;
@@ -62,7 +65,23 @@ __device__ __forceinline__ bool wait_w(uint32_t b_addr, uint32_t par, volatile i
     return __all_sync(0xffffffffu, mbar_wait(b_addr, par, abort_flag, tag, c));
 }
 
-// grid: x = query tile (the last tiles, which see the most keys, first), y = head.
+// A work unit: query tile qt (rows 128 qt ..) of head h; unit u takes the
+// tiles in order of decreasing causal length, all heads of a tile together.
+struct Unit {
+    int t0, h, NT;
+};
+
+__device__ __forceinline__ Unit unit_of(int u, int n_qt, int Hq, int T, int S)
+{
+    Unit w;
+    w.t0 = (n_qt - 1 - u / Hq) * kRows;
+    w.h = u % Hq;
+    const int kmax = min(S, w.t0 + kRows + (S - T));   // keys this tile needs
+    w.NT = (kmax + kKeys - 1) / kKeys;
+    return w;
+}
+
+// grid: one CTA per SM (at most one per unit).
 // tm_q: q as [T, Hq * 192]; tm_k: k as [S, Hq * 192]; tm_v: v as [S, Hq * 128].
 __global__ void __launch_bounds__(kThreads, 1)
 mha_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -79,10 +98,12 @@ mha_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sgen + kOffBar + 8 * M_COUNT + 8);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int t0 = (int)(gridDim.x - 1 - blockIdx.x) * kRows, h = blockIdx.y;
     const int shift = S - T;                       // pos[t] = t + shift
-    const int kmax = min(S, t0 + kRows + shift);   // keys this tile needs
-    const int NT = (kmax + kKeys - 1) / kKeys;
+    const int n_qt = (T + kRows - 1) / kRows;
+    const int n_all = n_qt * Hq;
+    const int cta = blockIdx.x, ncta = gridDim.x;
+    const int n_units = cta < n_all ? (n_all - cta + ncta - 1) / ncta : 0;
+    auto unit = [&](int j) -> Unit { return unit_of(cta + j * ncta, n_qt, Hq, T, S); };
 
     if (threadIdx.x == 0) {
         mbar_init(bar(M_Q), 1);
@@ -112,65 +133,93 @@ mha_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 
     if (warp == 1) {
         // ------------------------------------------------------------- TMA
+        // Q of a unit once every QK of the previous unit has completed (they
+        // read the Q tile), then its K / V tiles through the ring
         if (lane == 0) {
             prefetch_tmap(&tm_q);
             prefetch_tmap(&tm_k);
             prefetch_tmap(&tm_v);
-            mbar_arrive_expect_tx(bar(M_Q), kQBytes);
-            for (int i = 0; i < 3; ++i) tma_load_2d(qs + i * kSlab, &tm_q, h * kDh + 64 * i, t0, bar(M_Q));
-            for (int j = 0; j < NT; ++j) {
-                const int st = j % kStages;
-                if (j >= kStages &&
-                    !mbar_wait(bar(M_KEMPTY + st), ((j - kStages) / kStages) & 1, abort_flag, 100, j))
+            int g = 0, g_prev_last = -1;
+            bool ok = true;
+            for (int j = 0; ok && j < n_units; ++j) {
+                const Unit w = unit(j);
+                if (g_prev_last >= 0 &&
+                    !mbar_wait(bar(M_SFULL + (g_prev_last & 1)), (g_prev_last >> 1) & 1, abort_flag, 102, j)) {
+                    ok = false;
                     break;
-                const uint32_t kvs = sbase + kOffKV + st * kStageBytes;
-                mbar_arrive_expect_tx(bar(M_KFULL + st), kStageBytes);
-                for (int i = 0; i < 3; ++i)
-                    tma_load_2d(kvs + i * kSlab, &tm_k, h * kDh + 64 * i, kKeys * j, bar(M_KFULL + st));
-                for (int i = 0; i < 2; ++i)
-                    tma_load_2d(kvs + (3 + i) * kSlab, &tm_v, h * kDv + 64 * i, kKeys * j, bar(M_KFULL + st));
+                }
+                mbar_arrive_expect_tx(bar(M_Q), kQBytes);
+                for (int i = 0; i < 3; ++i) tma_load_2d(qs + i * kSlab, &tm_q, w.h * kDh + 64 * i, w.t0, bar(M_Q));
+                for (int jt = 0; jt < w.NT; ++jt, ++g) {
+                    const int st = g % kStages;
+                    if (g >= kStages &&
+                        !mbar_wait(bar(M_KEMPTY + st), ((g - kStages) / kStages) & 1, abort_flag, 100, g)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t kvs = sbase + kOffKV + st * kStageBytes;
+                    mbar_arrive_expect_tx(bar(M_KFULL + st), kStageBytes);
+                    for (int i = 0; i < 3; ++i)
+                        tma_load_2d(kvs + i * kSlab, &tm_k, w.h * kDh + 64 * i, kKeys * jt, bar(M_KFULL + st));
+                    for (int i = 0; i < 2; ++i)
+                        tma_load_2d(kvs + (3 + i) * kSlab, &tm_v, w.h * kDv + 64 * i, kKeys * jt, bar(M_KFULL + st));
+                }
+                g_prev_last = g - 1;
             }
         }
     } else if (warp == 0) {
         // ------------------------------------------------------------- MMA
-        if (lane == 0) {
+        if (lane == 0 && n_units > 0) {
             const uint32_t id_qk = idesc(128, kKeys, false);
             const uint32_t id_pv = idesc(128, kDv, true);
-            bool ok = mbar_wait(bar(M_Q), 0, abort_flag, 101, 0);
-            int cq = 0, cp = 0;
+            bool ok = true;
+            int qj = 0, qc = 0, qg = 0;   // QK cursor: unit, tile of the unit, global tile
+            int pj = 0, pc = 0, pg = 0;   // PV cursor
+            Unit qu = unit(0), pu = qu;
             uint64_t t_idle = globaltimer_ns();
-            while (ok && cp < NT) {
+            while (ok && pj < n_units) {
                 bool progressed = false;
-                if (cq < NT && mbar_test_wait(bar(M_KFULL + cq % kStages), (cq / kStages) & 1) &&
-                    (cq < 2 || mbar_test_wait(bar(M_SFREE + (cq & 1)), ((cq - 2) >> 1) & 1))) {
-                    const int j = cq++;
+                if (qj < n_units && mbar_test_wait(bar(M_KFULL + qg % kStages), (qg / kStages) & 1) &&
+                    (qg < 2 || mbar_test_wait(bar(M_SFREE + (qg & 1)), ((qg - 2) >> 1) & 1)) &&
+                    (qc > 0 || mbar_test_wait(bar(M_Q), qj & 1))) {
+                    const int g = qg;
                     tc_fence_after();
-                    const uint32_t kvs = sbase + kOffKV + (j % kStages) * kStageBytes;
+                    const uint32_t kvs = sbase + kOffKV + (g % kStages) * kStageBytes;
 #pragma unroll
                     for (int i = 0; i < 3; ++i)
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk) {
                             const uint64_t ad = smem_desc(qs + i * kSlab + kk * 32, 16, 1024, kSwizzle128B);
                             const uint64_t bd = smem_desc(kvs + i * kSlab + kk * 32, 16, 1024, kSwizzle128B);
-                            mma_f16_ss(tmem + kColS + (j & 1) * kKeys, ad, bd, id_qk, (i > 0 || kk > 0) ? 1u : 0u);
+                            mma_f16_ss(tmem + kColS + (g & 1) * kKeys, ad, bd, id_qk, (i > 0 || kk > 0) ? 1u : 0u);
                         }
-                    mma_commit(bar(M_SFULL + (j & 1)));
+                    mma_commit(bar(M_SFULL + (g & 1)));
+                    ++qg;
+                    if (++qc == qu.NT) {
+                        qc = 0;
+                        if (++qj < n_units) qu = unit(qj);
+                    }
                     progressed = true;
                 }
-                if (cp < cq && mbar_test_wait(bar(M_PFULL + (cp & 1)), (cp >> 1) & 1)) {
-                    const int j = cp++;
+                if (pg < qg && mbar_test_wait(bar(M_PFULL + (pg & 1)), (pg >> 1) & 1)) {
+                    const int g = pg;
                     tc_fence_after();
-                    const uint32_t vs = sbase + kOffKV + (j % kStages) * kStageBytes + 3 * kSlab;
+                    const uint32_t vs = sbase + kOffKV + (g % kStages) * kStageBytes + 3 * kSlab;
 #pragma unroll
                     for (int kk = 0; kk < kKeys / 16; ++kk) {
                         // B = the V tile read MN-major: 64 values per 128-byte row,
                         // LBO = next 64 columns (slab), SBO = next 8 keys
                         const uint64_t bd = smem_desc(vs + kk * 2048, kSlab, 1024, kSwizzle128B);
-                        mma_f16_ts(tmem + kColO, tmem + kColP + (j & 1) * 64 + kk * 8, bd, id_pv,
-                                   (j > 0 || kk > 0) ? 1u : 0u);
+                        mma_f16_ts(tmem + kColO, tmem + kColP + (g & 1) * 64 + kk * 8, bd, id_pv,
+                                   (pc > 0 || kk > 0) ? 1u : 0u);
                     }
-                    mma_commit(bar(M_PVDONE + (j & 1)));
-                    mma_commit(bar(M_KEMPTY + (j % kStages)));
+                    mma_commit(bar(M_PVDONE + (g & 1)));
+                    mma_commit(bar(M_KEMPTY + (g % kStages)));
+                    ++pg;
+                    if (++pc == pu.NT) {
+                        pc = 0;
+                        if (++pj < n_units) pu = unit(pj);
+                    }
                     progressed = true;
                 }
                 if (progressed) {
@@ -179,7 +228,7 @@ mha_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     ok = false;
                 } else if (globaltimer_ns() - t_idle > kWaitLimitNs) {
                     *abort_flag = 1;
-                    report_timeout(M_PFULL, cp, 0);
+                    report_timeout(M_PFULL, pg, 0);
                     ok = false;
                 }
             }
@@ -193,120 +242,131 @@ mha_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         // --------------------------------------------- softmax + epilogue
         const int hs = (warp - 4) >> 2;
         const int i = (warp & 3) * 32 + lane;                  // query row of the tile = TMEM lane
-        const int t = t0 + i;
         const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
         float* red = reinterpret_cast<float*>(sgen + kOffRed);
         float* lsum_s = reinterpret_cast<float*>(sgen + kOffLsum);
-        float m_use = -INFINITY, l = 0.f;
         bool ok = true;
-        // keys s <= t + shift (and s < S) of this row
-        const int s_lim = t < T ? min(S - 1, t + shift) : -1;
-        for (int j = 0; ok && j < NT; ++j) {
-            const int b = j & 1;
-            if (!wait_w(bar(M_SFULL + b), (j >> 1) & 1, abort_flag, 200, j)) { ok = false; break; }
-            tc_fence_after();
-            uint32_t sr[64];
-            tmem_ld32(tmem + lane_addr + kColS + b * kKeys + 64 * hs, *reinterpret_cast<uint32_t(*)[32]>(sr));
-            tmem_ld32(tmem + lane_addr + kColS + b * kKeys + 64 * hs + 32, *reinterpret_cast<uint32_t(*)[32]>(sr + 32));
-            tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(M_SFREE + b));
-            const int s0 = kKeys * j + 64 * hs;
-            float x[64];
+        int g0 = 0;
+        for (int u = 0; ok && u < n_units; ++u) {
+            const Unit w = unit(u);
+            const int t = w.t0 + i, h = w.h, NT = w.NT;
+            float m_use = -INFINITY, l = 0.f;
+            // keys s <= t + shift (and s < S) of this row
+            const int s_lim = t < T ? min(S - 1, t + shift) : -1;
+            for (int j = 0; ok && j < NT; ++j) {
+                const int g = g0 + j;
+                const int b = g & 1;
+                if (!wait_w(bar(M_SFULL + b), (g >> 1) & 1, abort_flag, 200, g)) { ok = false; break; }
+                tc_fence_after();
+                uint32_t sr[64];
+                tmem_ld32(tmem + lane_addr + kColS + b * kKeys + 64 * hs, *reinterpret_cast<uint32_t(*)[32]>(sr));
+                tmem_ld32(tmem + lane_addr + kColS + b * kKeys + 64 * hs + 32,
+                          *reinterpret_cast<uint32_t(*)[32]>(sr + 32));
+                tmem_wait_ld();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(M_SFREE + b));
+                const int s0 = kKeys * j + 64 * hs;
+                float x[64];
 #pragma unroll
-            for (int c = 0; c < 64; ++c)
-                x[c] = s0 + c <= s_lim ? __uint_as_float(sr[c]) * scale_log2 : -INFINITY;
-            float mx = x[0];
+                for (int c = 0; c < 64; ++c)
+                    x[c] = s0 + c <= s_lim ? __uint_as_float(sr[c]) * scale_log2 : -INFINITY;
+                float mx = x[0];
 #pragma unroll
-            for (int c = 1; c < 64; ++c) mx = fmaxf(mx, x[c]);
-            // row maximum over both key halves (the other half lives in warp +-4)
-            red[(b * 2 + hs) * kRows + i] = mx;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(M_RED + b));
-            if (!wait_w(bar(M_RED + b), (j >> 1) & 1, abort_flag, 201, j)) { ok = false; break; }
-            const float mc = fmaxf(mx, red[(b * 2 + (hs ^ 1)) * kRows + i]);
-            const float m_new = fmaxf(m_use, mc);
-            const bool raise = m_new > m_use + 8.f;
-            const bool rescale = raise && m_use != -INFINITY;
-            const float f = rescale ? ex2(m_use - m_new) : 1.f;
-            if (__any_sync(0xffffffffu, rescale)) {
-                // O holds earlier tiles: rescale this half's 64 columns once
-                // PV(j-1) has landed (warp-wide TMEM access; f = 1 where the
-                // maximum did not move)
-                if (!wait_w(bar(M_PVDONE + ((j - 1) & 1)), ((j - 1) >> 1) & 1, abort_flag, 202, j)) {
+                for (int c = 1; c < 64; ++c) mx = fmaxf(mx, x[c]);
+                // row maximum over both key halves (the other half lives in warp +-4)
+                red[(b * 2 + hs) * kRows + i] = mx;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(M_RED + b));
+                if (!wait_w(bar(M_RED + b), (g >> 1) & 1, abort_flag, 201, g)) { ok = false; break; }
+                const float mc = fmaxf(mx, red[(b * 2 + (hs ^ 1)) * kRows + i]);
+                const float m_new = fmaxf(m_use, mc);
+                const bool raise = m_new > m_use + 8.f;
+                const bool rescale = raise && m_use != -INFINITY;
+                const float f = rescale ? ex2(m_use - m_new) : 1.f;
+                if (__any_sync(0xffffffffu, rescale)) {
+                    // O holds earlier tiles of this unit: rescale this half's 64
+                    // columns once PV(g-1) has landed (warp-wide TMEM access; f = 1
+                    // where the maximum did not move)
+                    if (!wait_w(bar(M_PVDONE + ((g - 1) & 1)), ((g - 1) >> 1) & 1, abort_flag, 202, g)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+#pragma unroll 1
+                    for (int q2 = 0; q2 < 2; ++q2) {
+                        uint32_t o[32];
+                        const uint32_t ta = tmem + lane_addr + kColO + 64 * hs + 32 * q2;
+                        tmem_ld32(ta, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+                        tmem_st32(ta, o);
+                    }
+                    tmem_wait_st();
+                }
+                l *= f;
+                if (raise) m_use = m_new;
+                const float msub = m_use == -INFINITY ? 0.f : m_use;
+                uint32_t pk[32];
+                float ps = 0.f;
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                    const float p0 = ex2(x[2 * c] - msub), p1 = ex2(x[2 * c + 1] - msub);
+                    ps += p0 + p1;
+                    pk[c] = pack_bf16x2(p0, p1);
+                }
+                l += ps;
+                // P buffer b is free once PV(g-2) has read it
+                if (g >= 2 && !wait_w(bar(M_PVDONE + b), ((g - 2) >> 1) & 1, abort_flag, 203, g)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
+                tmem_st32(tmem + lane_addr + kColP + b * 64 + 32 * hs, pk);
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(M_PFULL + b));
+            }
+            // row sum over both key halves (buffer u & 1)
+            if (ok) {
+                lsum_s[((u & 1) * 2 + hs) * kRows + i] = l;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(M_LSUM));
+                ok = wait_w(bar(M_LSUM), u & 1, abort_flag, 204, u);
+                if (ok) l += lsum_s[((u & 1) * 2 + (hs ^ 1)) * kRows + i];
+            }
+            if (ok) {
+                const int gl = g0 + NT - 1;
+                ok = wait_w(bar(M_PVDONE + (gl & 1)), (gl >> 1) & 1, abort_flag, 205, gl);
+            }
+            if (ok) {
+                tc_fence_after();
+                const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll 1
                 for (int q2 = 0; q2 < 2; ++q2) {
                     uint32_t o[32];
-                    const uint32_t ta = tmem + lane_addr + kColO + 64 * hs + 32 * q2;
-                    tmem_ld32(ta, o);
+                    tmem_ld32(tmem + lane_addr + kColO + 64 * hs + 32 * q2, o);
                     tmem_wait_ld();
+                    if (t < T) {
+                        uint32_t wv[16];
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
-                    tmem_st32(ta, o);
+                        for (int e = 0; e < 16; ++e)
+                            wv[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
+                        uint4* dst = reinterpret_cast<uint4*>(out + ((size_t)t * Hq + h) * kDv + 64 * hs + 32 * q2);
+#pragma unroll
+                        for (int v = 0; v < 4; ++v)
+                            dst[v] = make_uint4(wv[4 * v], wv[4 * v + 1], wv[4 * v + 2], wv[4 * v + 3]);
+                    }
                 }
-                tmem_wait_st();
+                // O is read: the next unit's first PV may overwrite it (its P
+                // arrives only after this warp's next tile)
+                tc_fence_before();
+                if (hs == 0 && t < T)
+                    lse[(size_t)t * Hq + h] = l > 0.f ? (m_use + __log2f(l)) * 0.69314718055994531f : -INFINITY;
             }
-            l *= f;
-            if (raise) m_use = m_new;
-            const float msub = m_use == -INFINITY ? 0.f : m_use;
-            uint32_t pk[32];
-            float ps = 0.f;
-#pragma unroll
-            for (int c = 0; c < 32; ++c) {
-                const float p0 = ex2(x[2 * c] - msub), p1 = ex2(x[2 * c + 1] - msub);
-                ps += p0 + p1;
-                pk[c] = pack_bf16x2(p0, p1);
-            }
-            l += ps;
-            // P buffer b is free once PV(j-2) has read it
-            if (j >= 2 && !wait_w(bar(M_PVDONE + b), ((j - 2) >> 1) & 1, abort_flag, 203, j)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            tmem_st32(tmem + lane_addr + kColP + b * 64 + 32 * hs, pk);
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(M_PFULL + b));
-        }
-        // row sum over both key halves
-        if (ok) {
-            lsum_s[hs * kRows + i] = l;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(M_LSUM));
-            ok = wait_w(bar(M_LSUM), 0, abort_flag, 204, 0);
-            if (ok) l += lsum_s[(hs ^ 1) * kRows + i];
-        }
-        if (ok) {
-            const int jl = NT - 1;
-            ok = wait_w(bar(M_PVDONE + (jl & 1)), (jl >> 1) & 1, abort_flag, 205, jl);
-        }
-        if (ok) {
-            tc_fence_after();
-            const float inv = l > 0.f ? 1.f / l : 0.f;
-#pragma unroll 1
-            for (int q2 = 0; q2 < 2; ++q2) {
-                uint32_t o[32];
-                tmem_ld32(tmem + lane_addr + kColO + 64 * hs + 32 * q2, o);
-                tmem_wait_ld();
-                if (t < T) {
-                    uint32_t w[16];
-#pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        w[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
-                    uint4* dst = reinterpret_cast<uint4*>(out + ((size_t)t * Hq + h) * kDv + 64 * hs + 32 * q2);
-#pragma unroll
-                    for (int v = 0; v < 4; ++v) dst[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
-                }
-            }
-            if (hs == 0 && t < T)
-                lse[(size_t)t * Hq + h] = l > 0.f ? (m_use + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+            g0 += NT;
         }
     }
 
