@@ -219,6 +219,46 @@ ChunkPlan chunk_plan(int T, int S, int k)
     return p;
 }
 
+// Few rows over long key ranges (decode) with d_I = 128: every key scored into
+// a dense score row, a filter by a threshold from group maxima, then a per-row
+// select (indexer_chunked.cuh, rs). Rows per launch block and the buffers
+// they need: the score rows (ld floats each, at most rs::kMaxKeys keys), the
+// rows' 16-key and 4-key group maxima, and the pairs each segment keeps with
+// their counts.
+struct RowScorePlan {
+    int RB, max_segs;
+    long long ld, g16_ld, g4_ld, cand_ld;
+    size_t off_g16, off_g4, off_cand, off_cnt, off_tau, bytes;
+};
+
+bool use_row_scores(int T, int S, int d_I)
+{
+    using namespace dsa::idx_chunk;
+    return d_I == 128 && S > kChunkKeys && T <= rs::kMaxRows;
+}
+
+RowScorePlan row_score_plan(int T, int S)
+{
+    using namespace dsa::idx_chunk;
+    RowScorePlan p;
+    p.ld = (long long)dsa::ceil_div(std::min(S, rs::kMaxKeys), rs::kTileKeys) * rs::kTileKeys;
+    p.g16_ld = p.ld / rs::kTileKeys * rs::kGroupsPerTile;
+    p.g4_ld = p.ld / 4;
+    p.max_segs = (int)dsa::ceil_div(p.ld, (long long)rs::kSegKeys);
+    p.cand_ld = (long long)p.max_segs * rs::kSegCap;
+    const size_t per_row = (size_t)p.ld * sizeof(float) + (size_t)(p.g16_ld + p.g4_ld) * sizeof(uint32_t) +
+                           (size_t)p.cand_ld * sizeof(uint2) + (size_t)p.max_segs * sizeof(int) + sizeof(uint32_t);
+    p.RB = (int)std::min<size_t>({(size_t)T, (size_t)rs::kMaxRows,
+                                  std::max<size_t>(1, kScoreBlockBytes / per_row)});
+    p.off_g16 = align_up((size_t)p.RB * p.ld * sizeof(float));
+    p.off_g4 = p.off_g16 + align_up((size_t)p.RB * p.g16_ld * sizeof(uint32_t));
+    p.off_cand = p.off_g4 + align_up((size_t)p.RB * p.g4_ld * sizeof(uint32_t));
+    p.off_cnt = p.off_cand + align_up((size_t)p.RB * p.cand_ld * sizeof(uint2));
+    p.off_tau = p.off_cnt + align_up((size_t)p.RB * p.max_segs * sizeof(int));
+    p.bytes = p.off_tau + align_up((size_t)p.RB * sizeof(uint32_t));
+    return p;
+}
+
 // Streaming (tensor-core) indexer: query rows per launch block and the
 // per-row buffers it needs.
 constexpr int kFusedRowsPerBlock = 32768;
@@ -247,7 +287,8 @@ FusedPlan fused_plan(int T, int S, int k)
 // tensor-core path exists for H_I = 8, d_I = 128 only).
 size_t indexer_workspace(int T, int S, int k, int H_I, int d_I)
 {
-    const size_t chunked = chunk_plan(T, S, k).bytes;
+    size_t chunked = chunk_plan(T, S, k).bytes;
+    if (use_row_scores(T, S, d_I)) chunked = std::max(chunked, row_score_plan(T, S).bytes);
     if (H_I != dsa::idx_tc::kHI || d_I != dsa::idx_tc::kDI) return chunked;
     return std::max(chunked, fused_plan(T, S, k).bytes);
 }
@@ -420,7 +461,22 @@ void chunk_topk_tma(int grid, cudaStream_t st, const CUtensorMap& tm_k, const Ch
                max_chunks, idx, a.pg);
 }
 
+// d_I = 128, few rows: the dense score rows (tm_k as for chunk_topk_tma)
+template <int NT>
+void row_scores_tma(int grid, cudaStream_t st, const CUtensorMap& tm_k, const ChunkArgs& a, float* scores,
+                    long long ld, uint32_t* g16, long long g16_ld, uint32_t* g4, long long g4_ld)
+{
+    using namespace dsa::idx_chunk;
+    cudaFuncSetAttribute(row_scores_tma_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         rs::kSmemBytes);
+    launch_pdl(row_scores_tma_kernel<NT>, dim3(grid), dim3(rs::kThreads), rs::kSmemBytes, st, tm_k, a.q_idx,
+               a.w, a.pos, a.k_base, a.T, a.S, a.H_I, a.row0, a.rows, a.k, scores, ld, g16, g16_ld, g4, g4_ld,
+               a.pg);
+}
+
 struct ChunkFns {
+    void (*row_scores)(int, cudaStream_t, const CUtensorMap&, const ChunkArgs&, float*, long long, uint32_t*,
+                       long long, uint32_t*, long long);
     void (*sample_tau)(cudaStream_t, const ChunkArgs&, int*, float*, long long, uint32_t*);
     void (*topk)(int, cudaStream_t, const ChunkArgs&, const uint32_t*, uint2*, long long, int*, int,
                  int32_t*);
@@ -431,8 +487,8 @@ struct ChunkFns {
 template <int NT, int DI>
 ChunkFns chunk_fns()
 {
-    return {ChunkKernels<NT, DI>::sample_tau, ChunkKernels<NT, DI>::topk,
-            DI == 128 ? chunk_topk_tma<NT> : nullptr};
+    return {DI == 128 ? row_scores_tma<NT> : nullptr, ChunkKernels<NT, DI>::sample_tau,
+            ChunkKernels<NT, DI>::topk, DI == 128 ? chunk_topk_tma<NT> : nullptr};
 }
 
 ChunkFns pick_chunk(int H_I, int d_I)
@@ -475,6 +531,50 @@ int indexer_chunked(const uint8_t* q_idx, const float* w, const uint8_t* k_idx, 
         const uint64_t key_rows = paged ? (uint64_t)pg.num_pages * pg.page_size : (uint64_t)S;
         if (int rc = make_tmap_u8(&tm_k, k_idx, 128, key_rows, paged ? tma::kTileKeys / 2 : tma::kTileKeys))
             return rc;
+    }
+    if (fn.row_scores && use_row_scores(T, S, d_I)) {
+        // every key into a dense score row; per segment, the scores above a
+        // threshold from group maxima; then one select CTA per row
+        const RowScorePlan q = row_score_plan(T, S);
+        float* scores = reinterpret_cast<float*>(ws);
+        uint32_t* g16 = reinterpret_cast<uint32_t*>(ws + q.off_g16);
+        uint32_t* g4 = reinterpret_cast<uint32_t*>(ws + q.off_g4);
+        uint2* rcand = reinterpret_cast<uint2*>(ws + q.off_cand);
+        int* rcnt = reinterpret_cast<int*>(ws + q.off_cnt);
+        uint32_t* rtau = reinterpret_cast<uint32_t*>(ws + q.off_tau);
+        cudaError_t e = cudaFuncSetAttribute(row_filter_kernel<rs::kFiltThreads>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, rs::kFiltSmem);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(row_tau_kernel<rs::kTauThreads>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     rs::kTauSmem);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(row_merge_kernel<rs::kMergeThreads>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, rs::kMergeSmem);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(row select kernels)");
+        for (int row0 = 0; row0 < T; row0 += q.RB) {
+            const int rows = std::min(q.RB, T - row0);
+            const ChunkArgs a{q_idx, w, k_idx, pos, k_base, T, S, H_I, k, row0, rows, nullptr, pg};
+            PhaseMark ph = phase_begin(kPhaseScores, st);
+            fn.row_scores(rs::kCtasPerSm * num_sms(), st, tm_k, a, scores, q.ld, g16, q.g16_ld, g4, q.g4_ld);
+            DSA_LAUNCH_CHECK("row_scores_tma_kernel");
+            phase_end(ph);
+            ph = phase_begin(kPhaseThreshold, st);
+            launch_pdl(row_tau_kernel<rs::kTauThreads>, dim3(rows), dim3(rs::kTauThreads), rs::kTauSmem, st, g16,
+                       q.g16_ld, g4, q.g4_ld, pos, k_base, T, S, row0, k, rtau, pg);
+            DSA_LAUNCH_CHECK("row_tau_kernel");
+            launch_pdl(row_filter_kernel<rs::kFiltThreads>, dim3(2 * num_sms()), dim3(rs::kFiltThreads),
+                       rs::kFiltSmem, st, scores, q.ld, rtau, pos, k_base, T, S, row0, rows, k, rcand, q.cand_ld,
+                       rcnt, q.max_segs, pg);
+            DSA_LAUNCH_CHECK("row_filter_kernel");
+            phase_end(ph);
+            ph = phase_begin(kPhaseSelect, st);
+            launch_pdl(row_merge_kernel<rs::kMergeThreads>, dim3(rows), dim3(rs::kMergeThreads), rs::kMergeSmem, st,
+                       scores, q.ld, rcand, q.cand_ld, rcnt, q.max_segs, q_idx, w, k_idx, H_I, d_I, pos, k_base, T,
+                       S, row0, k, idx, pg);
+            DSA_LAUNCH_CHECK("row_merge_kernel");
+            phase_end(ph);
+        }
+        return DSA_OK;
     }
     const int resident = (fn.topk_tma ? tma::kCtasPerSm : kCtasPerSm) * num_sms();
     auto topk = [&](const ChunkArgs& a, int grid, const uint32_t* tk) {

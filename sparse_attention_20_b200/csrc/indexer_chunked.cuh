@@ -456,6 +456,205 @@ chunk_topk_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const uint8_t* _
     }
 }
 
+// Few rows with long key ranges (decode): the rows' key tiles are concatenated
+// and cut into equal contiguous ranges, one per CTA, so the key stream has no
+// item boundaries, no per-item selection and at most a handful of row changes
+// per CTA. Every key of a row is scored into a dense score row
+// (scores[r * ld + s]) together with the largest order key of each group of
+// 16 scores (gmax16[r * g16_ld + 8 * tile + warp]: one group per scoring warp
+// and tile) and of each group of 4 (gmax4[r * g4_ld + 32 * tile + 4 * warp +
+// q]). The row's Top-k is selected afterwards from these (row_filter_kernel,
+// row_merge_kernel). Rows with at most k keys, or more than kMaxKeys, get no
+// tiles here (the merge writes the former directly and recomputes the
+// latter's scores).
+namespace rs {
+constexpr int kTileKeys = 128;
+constexpr int kTileBytes = kTileKeys * 128;
+constexpr int kStages = 6;
+constexpr int kScoreWarps = 8;
+constexpr int kThreads = (kScoreWarps + 1) * 32;
+constexpr int kCtasPerSm = 2;
+constexpr int kMaxRows = 2048;        // rows per launch: the tile table lives in shared memory
+constexpr int kMaxKeys = 1 << 20;     // longest row scored into the workspace
+constexpr int kGroupsPerTile = kScoreWarps;   // 16-key groups per tile
+constexpr int kOffTable = kStages * kTileBytes;
+constexpr int kOffBar = kOffTable + (kMaxRows + 1 + 3) / 4 * 16;
+constexpr int kSmemBytes = kOffBar + 128 + 1024;   // + alignment slack
+enum : int { B_FULL = 0, B_EMPTY = kStages, B_COUNT = 2 * kStages };
+static_assert(kTileKeys == kScoreWarps * 16, "one 16-key MMA block per scoring warp and tile");
+static_assert(2 * (kSmemBytes + 1024) <= 228 * 1024, "two CTAs per SM");
+
+// Tiles of a row of n keys on this path.
+__device__ __forceinline__ int row_tiles(int n, int k)
+{
+    return n > k && n <= kMaxKeys ? ceil_div(n, kTileKeys) : 0;
+}
+}  // namespace rs
+
+template <int NT>
+__global__ void __launch_bounds__(rs::kThreads, rs::kCtasPerSm)
+row_scores_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const uint8_t* __restrict__ q_idx,
+                      const float* __restrict__ w, const int* __restrict__ pos,
+                      const int* __restrict__ k_base, int T, int S, int H_I, int row0, int rows, int k,
+                      float* __restrict__ scores, long long ld, uint32_t* __restrict__ gmax16,
+                      long long g16_ld, uint32_t* __restrict__ gmax4, long long g4_ld, const PagedRows pg)
+{
+    // tm_k boxes: 128 key rows (contiguous ranges) or 64 (paged cache: a tile
+    // is two half-tiles, each inside one page of a multiple of 64 keys)
+    using namespace sm100;
+    constexpr int DI = 128;
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ int wsum[rs::kThreads / 32];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t sbase = (raw + 1023u) & ~1023u;
+    uint8_t* sgen = smem_raw + (sbase - raw);
+    int* tbl = reinterpret_cast<int*>(sgen + rs::kOffTable);
+    const uint32_t bar0 = sbase + rs::kOffBar;
+    auto bar = [&](int i) -> uint32_t { return bar0 + 8u * (uint32_t)i; };
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sgen + rs::kOffBar + 8 * rs::B_COUNT);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int gid = lane >> 2, tid4 = lane & 3;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < rs::kStages; ++s) {
+            mbar_init(bar(rs::B_FULL + s), 1);
+            mbar_init(bar(rs::B_EMPTY + s), rs::kScoreWarps);
+        }
+        *abort_flag = 0;
+        fence_mbar_init_cluster();
+        prefetch_tmap(&tm_k);
+    }
+    griddep_wait();
+    // tbl[r] = tiles of rows 0 .. r-1 (exclusive prefix over the rows)
+    auto tiles_of = [&](int r) -> int {
+        long long b;
+        const int* bt;
+        return rs::row_tiles(row_keys(pg, pos, k_base, row0 + r, T, S, &b, &bt), k);
+    };
+    {
+        const int per = ceil_div(rows, rs::kThreads);
+        const int a0 = min(rows, (int)threadIdx.x * per), a1 = min(rows, a0 + per);
+        int sum = 0;
+        for (int r = a0; r < a1; ++r) sum += tiles_of(r);
+        int incl = sum;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += v;
+        }
+        if (lane == 31) wsum[warp] = incl;
+        __syncthreads();
+        int acc = incl - sum, total = 0;
+#pragma unroll
+        for (int q = 0; q < rs::kThreads / 32; ++q) {
+            if (q < warp) acc += wsum[q];
+            total += wsum[q];
+        }
+        for (int r = a0; r < a1; ++r) {
+            tbl[r] = acc;
+            acc += tiles_of(r);
+        }
+        if (threadIdx.x == 0) tbl[rows] = total;
+        __syncthreads();
+    }
+    const long long G = tbl[rows];
+    const int g0 = (int)(G * blockIdx.x / gridDim.x), g1 = (int)(G * (blockIdx.x + 1) / gridDim.x);
+    if (g0 >= g1) return;
+    // the row holding tile g: the last r with tbl[r] <= g (rows without tiles
+    // share their offset with the next row and are skipped)
+    auto row_of = [&](int g) -> int {
+        int lo = 0, hi = rows - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (tbl[mid] <= g) lo = mid; else hi = mid - 1;
+        }
+        return lo;
+    };
+    int r = row_of(g0);
+    long long base;
+    const int* bt;
+    int n = row_keys(pg, pos, k_base, row0 + r, T, S, &base, &bt);
+
+    if (warp == rs::kScoreWarps) {
+        if (lane != 0) return;
+        for (int g = g0; g < g1; ++g) {
+            if (g >= tbl[r + 1]) {
+                do ++r; while (g >= tbl[r + 1]);
+                n = row_keys(pg, pos, k_base, row0 + r, T, S, &base, &bt);
+            }
+            const int i = g - g0, st = i % rs::kStages;
+            if (i >= rs::kStages &&
+                !mbar_wait(bar(rs::B_EMPTY + st), ((i - rs::kStages) / rs::kStages) & 1, abort_flag,
+                           640 + rs::B_EMPTY, i))
+                return;
+            mbar_arrive_expect_tx(bar(rs::B_FULL + st), rs::kTileBytes);
+            const int s0 = (g - tbl[r]) * rs::kTileKeys;
+            const uint32_t dst = sbase + st * rs::kTileBytes;
+            if (bt) {
+                tma_load_2d(dst, &tm_k, 0, (int)key_row(pg, bt, 0, s0), bar(rs::B_FULL + st));
+                // a second half that starts past the row's keys reloads the
+                // first half (never scored) instead of naming a page the row
+                // does not have
+                const int s1 = s0 + rs::kTileKeys / 2 < n ? s0 + rs::kTileKeys / 2 : s0;
+                tma_load_2d(dst + rs::kTileBytes / 2, &tm_k, 0, (int)key_row(pg, bt, 0, s1),
+                            bar(rs::B_FULL + st));
+            } else {
+                tma_load_2d(dst, &tm_k, 0, (int)(base + s0), bar(rs::B_FULL + st));
+            }
+        }
+        return;
+    }
+    QueryFrag<NT, DI> qf;
+    qf.load(q_idx, w, row0 + r, H_I, lane);
+    const int ra = warp * 16 + gid, rb = ra + 8;   // tile rows; both are gid mod 8
+    for (int g = g0; g < g1; ++g) {
+        if (g >= tbl[r + 1]) {
+            do ++r; while (g >= tbl[r + 1]);
+            n = row_keys(pg, pos, k_base, row0 + r, T, S, &base, &bt);
+            qf.load(q_idx, w, row0 + r, H_I, lane);
+        }
+        const int i = g - g0, st = i % rs::kStages;
+        const bool got = mbar_wait(bar(rs::B_FULL + st), (i / rs::kStages) & 1, abort_flag, 640 + rs::B_FULL, i);
+        if (!__all_sync(0xffffffffu, got)) break;
+        const uint32_t ts = sbase + st * rs::kTileBytes;
+        KeyQuarter<DI> A, B;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            // 16-byte chunk 2*tid4+h of the row, 128B swizzle: chunk ^ (row & 7)
+            const uint32_t col = (uint32_t)(((2 * tid4 + h) ^ gid) << 4);
+            const uint4 va = ld_shared_v4(ts + ra * 128 + col);
+            const uint4 vb = ld_shared_v4(ts + rb * 128 + col);
+            A.v[4 * h] = va.x; A.v[4 * h + 1] = va.y; A.v[4 * h + 2] = va.z; A.v[4 * h + 3] = va.w;
+            B.v[4 * h] = vb.x; B.v[4 * h + 1] = vb.y; B.v[4 * h + 2] = vb.z; B.v[4 * h + 3] = vb.w;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(rs::B_EMPTY + st));
+        float ia, ib;
+        qf.score(A, B, ia, ib);
+        const int j = g - tbl[r];
+        const int a = j * rs::kTileKeys + ra, b = a + 8;
+        uint32_t hi = 0u;   // an empty group's maximum is the smallest key
+        if (tid4 == 0) {
+            float* out = scores + (size_t)r * ld;
+            if (a < n) {
+                out[a] = ia;
+                hi = max(hi, score_key(ia));
+            }
+            if (b < n) {
+                out[b] = ib;
+                hi = max(hi, score_key(ib));
+            }
+        }
+        // lanes 0, 4, ..., 28 hold the values; one step leaves the maxima of
+        // four keys (gid, gid + 1 and their rb rows) in lanes 0, 8, 16, 24
+        hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, 4));
+        if ((lane & 7) == 0) gmax4[(size_t)r * g4_ld + (size_t)j * 32 + warp * 4 + (lane >> 3)] = hi;
+        hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, 8));
+        hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, 16));
+        if (lane == 0) gmax16[(size_t)r * g16_ld + (size_t)j * rs::kGroupsPerTile + warp] = hi;
+    }
+}
+
 // Scores recomputed from the key rows (the merge's exact fallback): q^I of the
 // row as fp32 in shared memory, up to 16 heads.
 struct RecomputedRow {
@@ -574,6 +773,371 @@ merge_topk_kernel(const uint2* __restrict__ cand, long long cand_ld, const int* 
     } else {
         block_topk<THREADS>(pairs, n_pairs, k, idx + (size_t)t * k, sm);
     }
+}
+
+// Row Top-k from the dense score rows of row_scores_tma_kernel, in three
+// steps, for rows of k < n <= rs::kMaxKeys keys.
+//
+// row_tau_kernel (one CTA per row): the row's threshold tau, a lower bound of
+// its k-th largest score taken from group maxima. With at least k groups, the
+// k-th largest group maximum is reached by at least k groups, so by at least
+// k scores: the 16-key groups where the row has k of them, else the 4-key
+// groups, else tau = 0 (rows of fewer than 4k keys keep everything);
+// range_floor rounds it down to a histogram sub-bin edge.
+//
+// row_filter_kernel: persistent CTAs over the (row, segment of kSegKeys keys)
+// items, cut into equal contiguous ranges. An item's scores reach shared
+// memory by one 1-D bulk copy; the scores >= tau are kept as (order key, s)
+// pairs in ascending s (each warp counts its share, one scan over the warps,
+// then each warp writes its share in order), up to kSegCap of them, at
+// cand[r * cand_ld + seg * kSegCap ...], with their count at
+// ccnt[r * max_segs + seg].
+//
+// row_merge_kernel (one CTA per row): the row's Top-k is among its kept pairs
+// (they hold every score >= tau). The segments' pairs are bulk-copied in
+// order into a staging area (each run at an even offset, for the copies'
+// 16-byte alignment), then packed into one list in ascending s. Their exact
+// Top-k (range-histogram select, or the radix select where the keys'
+// spread defeats it) is marked in a bitmap over the pairs and written in
+// ascending s. A row whose pairs did not fit (a segment over kSegCap, or
+// more than kMergeList in all: scores far from independent) is selected over
+// its score row in global memory instead, marked in a bitmap over s. A row
+// of at most k keys lists them and pads with -1; a row longer than kMaxKeys
+// gets the exact Top-k of scores it recomputes.
+namespace rs {
+constexpr int kSegKeys = 16384;
+constexpr int kSegCap = 8192;
+constexpr int kTauThreads = 512;
+constexpr int kMaxStaged = 16384;                        // group maxima staged in shared memory
+constexpr int kTauSmem = kMaxStaged * 4 + 16;
+constexpr int kFiltThreads = 512;
+constexpr int kOffSegTbl = kSegKeys * 4;                 // the segment, then the item table
+constexpr int kOffFiltBar = kOffSegTbl + (kMaxRows + 1 + 3) / 4 * 16;
+constexpr int kFiltSmem = kOffFiltBar + 16;
+constexpr int kMergeThreads = 256;
+constexpr int kMergeList = 8192;                         // pairs of a row in shared memory
+constexpr int kOffStage = kMergeList * 8;                // the list, then the staging area,
+constexpr int kOffListBits = 2 * kMergeList * 8;         // then the bitmap over the list
+constexpr int kOffMergeBar = kOffListBits + kMergeList / 8;
+constexpr int kMergeSmem = kOffMergeBar + 16;            // (or a bitmap over s, from 0)
+constexpr int kMaxSegs = kMaxKeys / kSegKeys;
+static_assert(kOffMergeBar >= kMaxKeys / 8, "a bitmap over the longest row fits below the barrier");
+static_assert(kSegCap >= 2 * 4 * 1024, "a row below 4k keys (k <= 2048) keeps all of them in one item");
+static_assert(kSegKeys % (kFiltThreads / 32 * 128) == 0, "whole float4 rows per warp");
+
+__device__ __forceinline__ int row_segs(int n, int k)
+{
+    return n > k && n <= kMaxKeys ? ceil_div(n, kSegKeys) : 0;
+}
+}  // namespace rs
+
+template <int THREADS>
+__global__ void __launch_bounds__(THREADS)
+row_tau_kernel(const uint32_t* __restrict__ gmax16, long long g16_ld, const uint32_t* __restrict__ gmax4,
+               long long g4_ld, const int* __restrict__ pos, const int* __restrict__ k_base, int T, int S,
+               int row0, int k, uint32_t* __restrict__ tau, const PagedRows pg)
+{
+    using namespace sm100;
+    __shared__ SelectSmem<THREADS> sm;
+    __shared__ int abort_s;
+    extern __shared__ __align__(16) uint8_t dyn[];
+    const uint32_t dyn_s = smem_u32(dyn);
+    const uint32_t bar = dyn_s + rs::kMaxStaged * 4;
+    const int tid = threadIdx.x, r = blockIdx.x;
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        abort_s = 0;
+        fence_mbar_init_cluster();
+    }
+    __syncthreads();
+    griddep_wait();
+    long long base;
+    const int* bt;
+    const int n = row_keys(pg, pos, k_base, row0 + r, T, S, &base, &bt);
+    const int tiles = rs::row_tiles(n, k);
+    const int m16 = tiles * rs::kGroupsPerTile, m4 = tiles * 32;
+    const uint32_t* gm = m16 >= k ? gmax16 + (size_t)r * g16_ld : m4 >= k ? gmax4 + (size_t)r * g4_ld : nullptr;
+    const int m = m16 >= k ? m16 : m4 >= k ? m4 : 0;
+    if (!gm) {
+        if (tid == 0) tau[r] = 0u;
+        return;
+    }
+    const uint32_t* src = gm;
+    if (m <= rs::kMaxStaged) {
+        if (tid == 0) {
+            mbar_arrive_expect_tx(bar, (uint32_t)m * 4u);
+            bulk_g2s(dyn_s, gm, (uint32_t)m * 4u, bar);
+        }
+        const bool got = mbar_wait(bar, 0, (volatile int*)&abort_s, 671, r);
+        if (__syncthreads_or(!got)) return;
+        src = reinterpret_cast<const uint32_t*>(dyn);
+    }
+    const uint32_t t = range_floor<THREADS>(src, m, k, sm);
+    if (tid == 0) tau[r] = t;
+}
+
+template <int THREADS>
+__global__ void __launch_bounds__(THREADS, 2)
+row_filter_kernel(const float* __restrict__ scores, long long ld, const uint32_t* __restrict__ tau,
+                  const int* __restrict__ pos, const int* __restrict__ k_base, int T, int S, int row0, int rows,
+                  int k, uint2* __restrict__ cand, long long cand_ld, int* __restrict__ ccnt, int max_segs,
+                  const PagedRows pg)
+{
+    using namespace sm100;
+    constexpr int W = THREADS / 32;
+    constexpr int kPerWarp = rs::kSegKeys / W;
+    static_assert(THREADS == rs::kFiltThreads && W <= 32, "launch shape");
+    __shared__ int wsum[W];
+    __shared__ int abort_s;
+    extern __shared__ __align__(16) uint8_t dyn[];
+    const uint32_t dyn_s = smem_u32(dyn);
+    const float* seg = reinterpret_cast<const float*>(dyn);
+    int* tbl = reinterpret_cast<int*>(dyn + rs::kOffSegTbl);
+    const uint32_t bar = dyn_s + rs::kOffFiltBar;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        abort_s = 0;
+        fence_mbar_init_cluster();
+    }
+    griddep_wait();
+    // tbl[r] = items of rows 0 .. r-1
+    auto segs_of = [&](int r) -> int {
+        long long b;
+        const int* bt;
+        return rs::row_segs(row_keys(pg, pos, k_base, row0 + r, T, S, &b, &bt), k);
+    };
+    {
+        const int per = ceil_div(rows, THREADS);
+        const int a0 = min(rows, tid * per), a1 = min(rows, a0 + per);
+        int sum = 0;
+        for (int r = a0; r < a1; ++r) sum += segs_of(r);
+        int incl = sum;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += v;
+        }
+        if (lane == 31) wsum[warp] = incl;
+        __syncthreads();
+        int acc = incl - sum, total = 0;
+#pragma unroll
+        for (int q = 0; q < W; ++q) {
+            if (q < warp) acc += wsum[q];
+            total += wsum[q];
+        }
+        for (int r = a0; r < a1; ++r) {
+            tbl[r] = acc;
+            acc += segs_of(r);
+        }
+        if (tid == 0) tbl[rows] = total;
+        __syncthreads();
+    }
+    const long long G = tbl[rows];
+    const int i0 = (int)(G * blockIdx.x / gridDim.x), i1 = (int)(G * (blockIdx.x + 1) / gridDim.x);
+    for (int item = i0, phase = 0; item < i1; ++item, ++phase) {
+        int r;
+        {
+            int lo = 0, hi = rows - 1;
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (tbl[mid] <= item) lo = mid; else hi = mid - 1;
+            }
+            r = lo;
+        }
+        const int sg = item - tbl[r];
+        long long base;
+        const int* bt;
+        const int n = row_keys(pg, pos, k_base, row0 + r, T, S, &base, &bt);
+        const int s0 = sg * rs::kSegKeys, cnt = min(rs::kSegKeys, n - s0);
+        if (tid == 0) {
+            // the last copy of a row is rounded up to 16 bytes: it stays inside ld
+            const uint32_t bytes = (uint32_t)(cnt * 4 + 15) & ~15u;
+            mbar_arrive_expect_tx(bar, bytes);
+            bulk_g2s(dyn_s, scores + (size_t)r * ld + s0, bytes, bar);
+        }
+        // the float whose order key is tau: x >= tf keeps every score whose
+        // key is >= tau (and at most a zero of the other sign besides, which
+        // ranks below k kept scores and is never selected); tau = 0 keeps all
+        const uint32_t tk = tau[r];
+        const float tf = tk ? key_score(tk) : -INFINITY;
+        const bool got = mbar_wait(bar, (uint32_t)(phase & 1), (volatile int*)&abort_s, 670, item);
+        if (__syncthreads_or(!got)) return;
+        // pad the last run of 128 past cnt with NaN, which no compare keeps
+        // (the copy left it stale)
+        float* segw = reinterpret_cast<float*>(dyn);
+        const int cnt128 = (cnt + 127) & ~127;
+        for (int i = cnt + tid; i < cnt128; i += THREADS) segw[i] = __int_as_float(0x7FC00000);
+        __syncthreads();
+        // warp w owns entries [w * kPerWarp, (w + 1) * kPerWarp) below cnt128:
+        // lane l takes entries 4l .. 4l+3 of each run of 128
+        const int e0 = warp * kPerWarp;
+        const int iters = max(0, min(kPerWarp, cnt128 - e0)) / 128;
+        auto bits_at = [&](int it, float4& v) -> uint32_t {
+            v = *reinterpret_cast<const float4*>(seg + e0 + it * 128 + 4 * lane);
+            return (uint32_t)(v.x >= tf) | (uint32_t)(v.y >= tf) << 1 | (uint32_t)(v.z >= tf) << 2 |
+                   (uint32_t)(v.w >= tf) << 3;
+        };
+        int mine = 0;
+#pragma unroll 4
+        for (int it = 0; it < iters; ++it) {
+            float4 v;
+            mine += __popc(bits_at(it, v));
+        }
+#pragma unroll
+        for (int off = 16; off; off >>= 1) mine += __shfl_xor_sync(0xffffffffu, mine, off);
+        if (lane == 0) wsum[warp] = mine;
+        __syncthreads();
+        const int x = lane < W ? wsum[lane] : 0;
+        int xi = x;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, xi, off);
+            if (lane >= off) xi += y;
+        }
+        int at = __shfl_sync(0xffffffffu, xi - x, warp);
+        const int total = __shfl_sync(0xffffffffu, xi, W - 1);
+        uint2* dst = cand + (size_t)r * cand_ld + (size_t)sg * rs::kSegCap;
+#pragma unroll 2
+        for (int it = 0; it < iters && at < rs::kSegCap; ++it) {
+            float4 v;
+            const uint32_t b = bits_at(it, v);
+            const float e[4] = {v.x, v.y, v.z, v.w};
+            const int c = __popc(b);
+            int incl = c;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incl, off);
+                if (lane >= off) incl += y;
+            }
+            int o = at + incl - c;
+            const int s = s0 + e0 + it * 128 + 4 * lane;
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                if (b >> q & 1u) {
+                    if (o < rs::kSegCap) dst[o] = make_uint2(score_key(e[q]), (uint32_t)(s + q));
+                    ++o;
+                }
+            at += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (tid == 0) ccnt[(size_t)r * max_segs + sg] = total;
+        __syncthreads();   // the segment buffer and wsum take the next item
+    }
+}
+
+// Pairs staged in shared memory; entry i is marked as bit i.
+struct PairList {
+    const uint2* p;
+    __device__ __forceinline__ uint32_t key(int i) const { return p[i].x; }
+    __device__ __forceinline__ int s(int i) const { return i; }
+};
+
+template <int THREADS>
+__global__ void __launch_bounds__(THREADS)
+row_merge_kernel(const float* __restrict__ scores, long long ld, const uint2* __restrict__ cand,
+                 long long cand_ld, const int* __restrict__ ccnt, int max_segs, const uint8_t* __restrict__ q_idx,
+                 const float* __restrict__ w, const uint8_t* __restrict__ k_idx, int H_I, int d_I,
+                 const int* __restrict__ pos, const int* __restrict__ k_base, int T, int S, int row0, int k,
+                 int32_t* __restrict__ idx, const PagedRows pg)
+{
+    using namespace sm100;
+    __shared__ SelectSmem<THREADS> sm;
+    __shared__ int cnt_s[rs::kMaxSegs], off_s[rs::kMaxSegs + 1], pre_s[rs::kMaxSegs + 1];
+    __shared__ int over_s, abort_s;
+    extern __shared__ __align__(16) uint8_t dyn[];
+    const uint32_t dyn_s = smem_u32(dyn);
+    const uint32_t bar = dyn_s + rs::kOffMergeBar;
+    const int r = blockIdx.x, t = row0 + r, tid = threadIdx.x;
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        abort_s = 0;
+        over_s = 0;
+        fence_mbar_init_cluster();
+    }
+    __syncthreads();
+    griddep_wait();
+    long long base;
+    const int* bt;
+    const int n = row_keys(pg, pos, k_base, t, T, S, &base, &bt);
+    int32_t* out = idx + (size_t)t * k;
+    if (n <= k) {
+        for (int i = tid; i < k; i += THREADS) out[i] = i < n ? i : -1;
+        return;
+    }
+    if (n > rs::kMaxKeys) {
+        float* qf = reinterpret_cast<float*>(dyn);
+        float* wf = qf + H_I * d_I;
+        const uint8_t* qrow = q_idx + (size_t)t * H_I * d_I;
+        for (int e = tid; e < H_I * d_I; e += THREADS) qf[e] = e4m3x2_to_float2((uint16_t)qrow[e]).x;
+        for (int j = tid; j < H_I; j += THREADS) wf[j] = w[(size_t)t * H_I + j];
+        __syncthreads();
+        block_topk<THREADS>(RecomputedRow{qf, wf, k_idx, pg, bt, base, H_I, d_I}, n, k, out, sm);
+        return;
+    }
+    const int nseg = rs::row_segs(n, k);
+    for (int sg = tid; sg < nseg; sg += THREADS) {
+        const int c = ccnt[(size_t)r * max_segs + sg];
+        cnt_s[sg] = c;
+        if (c > rs::kSegCap) over_s = 1;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        // segment sg's run is staged at off_s[sg] (even) and packed at pre_s[sg]
+        off_s[0] = 0;
+        pre_s[0] = 0;
+        for (int sg = 0; sg < nseg; ++sg) {
+            const int c = min(cnt_s[sg], rs::kSegCap);
+            off_s[sg + 1] = off_s[sg] + ((c + 1) & ~1);
+            pre_s[sg + 1] = pre_s[sg] + c;
+        }
+        if (off_s[nseg] > rs::kMergeList) over_s = 1;
+    }
+    __syncthreads();
+    int* warp_sums = reinterpret_cast<int*>(sm.hist[0]);
+    if (!over_s) {
+        const int c = pre_s[nseg];   // >= k: every score >= tau
+        uint2* list = reinterpret_cast<uint2*>(dyn);
+        const uint2* stage = reinterpret_cast<const uint2*>(dyn + rs::kOffStage);
+        uint32_t* lbm = reinterpret_cast<uint32_t*>(dyn + rs::kOffListBits);
+        const uint2* src = cand + (size_t)r * cand_ld;
+        if (tid == 0) {
+            mbar_arrive_expect_tx(bar, (uint32_t)off_s[nseg] * 8u);
+            for (int sg = 0; sg < nseg; ++sg) {
+                const uint32_t bytes = (uint32_t)(off_s[sg + 1] - off_s[sg]) * 8u;
+                if (bytes)
+                    bulk_g2s(dyn_s + rs::kOffStage + (uint32_t)off_s[sg] * 8u, src + (size_t)sg * rs::kSegCap,
+                             bytes, bar);
+            }
+        }
+        for (int i = tid; i < (c + 31) / 32; i += THREADS) lbm[i] = 0u;
+        const bool got = mbar_wait(bar, 0, (volatile int*)&abort_s, 672, r);
+        if (__syncthreads_or(!got)) return;
+        // pack: pair i of the list is in the last run whose packed start is <= i
+        for (int i = tid; i < c; i += THREADS) {
+            int lo = 0, hi = nseg - 1;
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (pre_s[mid] <= i) lo = mid; else hi = mid - 1;
+            }
+            list[i] = stage[off_s[lo] + (i - pre_s[lo])];
+        }
+        __syncthreads();
+        const PairList row{list};
+        if (!range_select_bitmap<THREADS>(row, c, k, lbm, sm))
+            block_select<THREADS>(row, c, k, [&](int, int i) { atomicOr(&lbm[i >> 5], 1u << (i & 31)); }, sm);
+        __syncthreads();
+        block_emit_bitmap<THREADS>(lbm, c, out, warp_sums, [&](int i) { return (int)list[i].y; });
+        return;
+    }
+    // the pairs did not fit: select over the score row in global memory
+    uint32_t* bm = reinterpret_cast<uint32_t*>(dyn);
+    for (int i = tid; i < (n + 31) / 32; i += THREADS) bm[i] = 0u;
+    __syncthreads();
+    const DenseScores row{scores + (size_t)r * ld};
+    if (!range_select_bitmap<THREADS>(row, n, k, bm, sm))
+        block_select<THREADS>(row, n, k, [&](int, int i) { atomicOr(&bm[i >> 5], 1u << (i & 31)); }, sm);
+    __syncthreads();
+    block_emit_bitmap<THREADS>(bm, n, out, warp_sums);
 }
 
 }  // namespace idx_chunk

@@ -243,48 +243,19 @@ __device__ void block_select(const Row& row, int n, int k, const Emit& emit, Sel
 constexpr int kRangeBins = 2048;
 constexpr int kRangeListCap = 128;   // uint2 entries in SelectSmem::total
 
-template <int THREADS, class Row>
-__device__ bool range_select_bitmap(const Row& row, int n, int k, uint32_t* bm, SelectSmem<THREADS>& sm)
+// With the kRangeBins-bin histogram in sm.hist complete and visible: the bin
+// holding the k-th entry from the top goes to sm.misc[0], k minus the entries
+// of the bins above it to misc[1], the bin's count to misc[2] (visible to
+// every thread on return; k must not exceed the histogram's total).
+template <int THREADS>
+__device__ void range_kth_bin(int k, SelectSmem<THREADS>& sm)
 {
     constexpr int W = THREADS / 32;
     constexpr int PER = kRangeBins / THREADS;
-    static_assert(W * 256 >= kRangeBins && kRangeBins % THREADS == 0, "histogram space");
-    static_assert(2 * kRangeListCap <= 256 && 2 * W <= 256, "list space");
     __shared__ uint32_t wsum[W];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    uint32_t* h = &sm.hist[0][0];
-    // 1. key range
-    uint32_t lo = 0xFFFFFFFFu, hi = 0u;
-    for (int i = tid; i < n; i += THREADS) {
-        const uint32_t key = row.key(i);
-        lo = min(lo, key);
-        hi = max(hi, key);
-    }
-#pragma unroll
-    for (int off = 16; off; off >>= 1) {
-        lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, off));
-        hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, off));
-    }
-    if (lane == 0) {
-        sm.total[warp] = lo;
-        sm.total[W + warp] = hi;
-    }
-    for (int b = tid; b < kRangeBins; b += THREADS) h[b] = 0u;
-    __syncthreads();
-    lo = sm.total[0];
-    hi = sm.total[W];
-#pragma unroll
-    for (int w = 1; w < W; ++w) {
-        lo = min(lo, sm.total[w]);
-        hi = max(hi, sm.total[W + w]);
-    }
-    if (lo == hi) return false;
-    const int shift = max(0, 32 - __clz(hi - lo) - 11);   // (hi - lo) >> shift < 2048
-    // 2. histogram
-    for (int i = tid; i < n; i += THREADS) atomicAdd(&h[(row.key(i) - lo) >> shift], 1u);
-    __syncthreads();
-    // 3. the bin of the k-th entry from the top: thread j owns the PER bins
-    //    just below the top j * PER
+    const uint32_t* h = &sm.hist[0][0];
+    // thread j owns the PER bins just below the top j * PER
     uint32_t c[PER], local = 0u;
 #pragma unroll
     for (int j = 0; j < PER; ++j) {
@@ -316,21 +287,40 @@ __device__ bool range_select_bitmap(const Row& row, int n, int k, uint32_t* bm, 
         }
     }
     __syncthreads();
+}
+
+// Steps 2-5 with the block's key range [lo, hi] known and the histogram
+// (sm.hist) zeroed and visible to every thread.
+// each(f) calls f(key, s) for every entry of the row (every thread of the
+// CTA calls it, each thread for its own share of the entries).
+template <int THREADS, class Each>
+__device__ bool range_select_core(const Each& each, int k, uint32_t lo, uint32_t hi, uint32_t* bm,
+                                  SelectSmem<THREADS>& sm)
+{
+    constexpr int W = THREADS / 32;
+    static_assert(W * 256 >= kRangeBins && kRangeBins % THREADS == 0, "histogram space");
+    static_assert(2 * kRangeListCap <= 256 && 2 * W <= 256, "list space");
+    const int tid = threadIdx.x;
+    uint32_t* h = &sm.hist[0][0];
+    if (lo == hi) return false;
+    const int shift = max(0, 32 - __clz(hi - lo) - 11);   // (hi - lo) >> shift < 2048
+    // 2. histogram
+    each([&](uint32_t key, uint32_t) { atomicAdd(&h[(key - lo) >> shift], 1u); });
+    __syncthreads();
+    // 3. the bin of the k-th entry from the top
+    range_kth_bin<THREADS>(k, sm);
     const uint32_t kb = (uint32_t)sm.misc[0];
     const int need = sm.misc[1], inb = sm.misc[2];
     if (inb > kRangeListCap) return false;
     // 4. mark the entries above bin kb, collect bin kb
     uint2* list = reinterpret_cast<uint2*>(sm.total);
-    for (int i = tid; i < n; i += THREADS) {
-        const uint32_t key = row.key(i);
+    each([&](uint32_t key, uint32_t s) {
         const uint32_t b = (key - lo) >> shift;
-        if (b > kb) {
-            const uint32_t s = (uint32_t)row.s(i);
+        if (b > kb)
             atomicOr(&bm[s >> 5], 1u << (s & 31));
-        } else if (b == kb) {
-            list[atomicAdd(&sm.counter[0], 1)] = make_uint2(key, (uint32_t)row.s(i));
-        }
-    }
+        else if (b == kb)
+            list[atomicAdd(&sm.counter[0], 1)] = make_uint2(key, s);
+    });
     __syncthreads();
     // 5. the first `need` entries of the bin by (key descending, s ascending)
     for (int j = tid; j < inb; j += THREADS) {
@@ -343,6 +333,132 @@ __device__ bool range_select_bitmap(const Row& row, int n, int k, uint32_t* bm, 
         if (rank < need) atomicOr(&bm[e.y >> 5], 1u << (e.y & 31));
     }
     return true;
+}
+
+template <int THREADS, class Row>
+__device__ bool range_select_bitmap(const Row& row, int n, int k, uint32_t* bm, SelectSmem<THREADS>& sm)
+{
+    constexpr int W = THREADS / 32;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    uint32_t* h = &sm.hist[0][0];
+    // 1. key range
+    uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+    for (int i = tid; i < n; i += THREADS) {
+        const uint32_t key = row.key(i);
+        lo = min(lo, key);
+        hi = max(hi, key);
+    }
+#pragma unroll
+    for (int off = 16; off; off >>= 1) {
+        lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, off));
+        hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, off));
+    }
+    if (lane == 0) {
+        sm.total[warp] = lo;
+        sm.total[W + warp] = hi;
+    }
+    for (int b = tid; b < kRangeBins; b += THREADS) h[b] = 0u;
+    __syncthreads();
+    lo = sm.total[0];
+    hi = sm.total[W];
+#pragma unroll
+    for (int w = 1; w < W; ++w) {
+        lo = min(lo, sm.total[w]);
+        hi = max(hi, sm.total[W + w]);
+    }
+    const auto each = [&](const auto& f) {
+        for (int i = tid; i < n; i += THREADS) f(row.key(i), (uint32_t)row.s(i));
+    };
+    return range_select_core<THREADS>(each, k, lo, hi, bm, sm);
+}
+
+// The same with the row's key range [lo, hi] given by the caller (every
+// thread passes the same values) and its entries visited by each(f), which
+// calls f(key, s) for this thread's share of them.
+template <int THREADS, class Each>
+__device__ bool range_select_bitmap_in(const Each& each, int k, uint32_t lo, uint32_t hi, uint32_t* bm,
+                                       SelectSmem<THREADS>& sm)
+{
+    uint32_t* h = &sm.hist[0][0];
+    for (int b = threadIdx.x; b < kRangeBins; b += THREADS) h[b] = 0u;
+    __syncthreads();
+    return range_select_core<THREADS>(each, k, lo, hi, bm, sm);
+}
+
+// A lower bound of the k-th largest of the non-zero order keys among
+// v[0..m) (shared or global memory; key 0 marks an empty entry), or 0 when
+// fewer than k are non-zero. The k-th largest is located in a kRangeBins-bin
+// histogram over the keys' range, then in a kRangeBins-bin histogram over
+// that bin; the result is the lower edge of the sub-bin holding it, so at
+// least k of the keys are >= it. Every thread of the CTA takes part and
+// returns it.
+template <int THREADS>
+__device__ uint32_t range_floor(const uint32_t* v, int m, int k, SelectSmem<THREADS>& sm)
+{
+    constexpr int W = THREADS / 32;
+    static_assert(W * 256 >= kRangeBins && kRangeBins % THREADS == 0, "histogram space");
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    uint32_t* h = &sm.hist[0][0];
+    uint32_t lo = 0xFFFFFFFFu, hi = 0u, cnt = 0u;
+    for (int i = tid; i < m; i += THREADS) {
+        const uint32_t x = v[i];
+        if (x) {
+            lo = min(lo, x);
+            hi = max(hi, x);
+            ++cnt;
+        }
+    }
+#pragma unroll
+    for (int off = 16; off; off >>= 1) {
+        lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, off));
+        hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, off));
+        cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
+    }
+    if (lane == 0) {
+        sm.total[warp] = lo;
+        sm.total[W + warp] = hi;
+        sm.total[2 * W + warp] = cnt;
+    }
+    for (int b = tid; b < kRangeBins; b += THREADS) h[b] = 0u;
+    __syncthreads();
+    lo = sm.total[0];
+    hi = sm.total[W];
+    cnt = sm.total[2 * W];
+#pragma unroll
+    for (int w = 1; w < W; ++w) {
+        lo = min(lo, sm.total[w]);
+        hi = max(hi, sm.total[W + w]);
+        cnt += sm.total[2 * W + w];
+    }
+    __syncthreads();   // sm.total is free again
+    if (cnt < (uint32_t)k) return 0u;
+    if (lo == hi) return lo;
+    // level 1: bins of 2^shift keys over [lo, hi]
+    const int shift = max(0, 32 - __clz(hi - lo) - 11);   // (hi - lo) >> shift < 2048
+    for (int i = tid; i < m; i += THREADS) {
+        const uint32_t x = v[i];
+        if (x) atomicAdd(&h[(x - lo) >> shift], 1u);
+    }
+    __syncthreads();
+    range_kth_bin<THREADS>(k, sm);
+    const uint32_t kb = (uint32_t)sm.misc[0];
+    const int need = sm.misc[1];
+    __syncthreads();   // sm.misc is read; the histogram is cleared next
+    const uint32_t b0 = lo + (kb << shift);
+    if (shift == 0) return b0;
+    // level 2: sub-bins of 2^shift2 keys over bin kb
+    const int shift2 = max(0, shift - 11);
+    for (int b = tid; b < kRangeBins; b += THREADS) h[b] = 0u;
+    __syncthreads();
+    for (int i = tid; i < m; i += THREADS) {
+        const uint32_t x = v[i];
+        if (x && ((x - lo) >> shift) == kb) atomicAdd(&h[(x - b0) >> shift2], 1u);
+    }
+    __syncthreads();
+    range_kth_bin<THREADS>(need, sm);
+    const uint32_t kb2 = (uint32_t)sm.misc[0];
+    __syncthreads();   // sm.misc is free again
+    return b0 + (kb2 << shift2);
 }
 
 // Writes the Top-k of `row` (n entries) to out[0..k) in storage order; slots
@@ -382,13 +498,17 @@ __device__ __forceinline__ void block_sort_ascending(int* v, int n, int cap)
         }
 }
 
-// Writes the positions of the set bits of bm (words covering [0, n)) to
-// out[0..) in ascending order: every thread emits the set bits of its run of
+// Writes map(position) of the set bits of bm (words covering [0, n)) to
+// out[0..) in ascending order of position: every thread emits the set bits of its run of
 // words at an offset from a block-wide prefix of their counts. warp_sums
 // holds THREADS / 32 ints of shared memory. Every thread of the CTA takes
 // part.
-template <int THREADS>
-__device__ void block_emit_bitmap(const uint32_t* bm, int n, int* out, int* warp_sums)
+struct SamePosition {
+    __device__ __forceinline__ int operator()(int i) const { return i; }
+};
+
+template <int THREADS, class Map = SamePosition>
+__device__ void block_emit_bitmap(const uint32_t* bm, int n, int* out, int* warp_sums, const Map& map = {})
 {
     const int words = (n + 31) >> 5;
     const int per = (words + THREADS - 1) / THREADS;
@@ -407,7 +527,7 @@ __device__ void block_emit_bitmap(const uint32_t* bm, int n, int* out, int* warp
     int pos = incl - cnt;
     for (int q = 0; q < warp; ++q) pos += warp_sums[q];
     for (int i = w0; i < w1; ++i)
-        for (uint32_t b = bm[i]; b; b &= b - 1u) out[pos++] = (i << 5) + __ffs(b) - 1;
+        for (uint32_t b = bm[i]; b; b &= b - 1u) out[pos++] = map((i << 5) + __ffs(b) - 1);
 }
 
 __host__ __device__ __forceinline__ int pow2_ceil(int x)

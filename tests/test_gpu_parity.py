@@ -98,20 +98,49 @@ def test_decode_integer_inputs_bit_exact():
     check_indexer(x, idx.cpu(), list(range(x.T)), exact=True)
 
 
-def test_decode_multi_chunk_integer_bit_exact():
-    """Rows of one to five 8192-key chunks (chunk Top-k, sampled threshold and
-    merge); integer FP8-exact inputs make many scores tie across chunks."""
+# Up to 2048 query rows per call take the decode form (every key of a row
+# scored into a dense score row, then a per-row select); more rows take the
+# chunked form (chunk Top-k under a sampled threshold, then a merge). A test
+# reaches the chunked form by repeating each query row `reps` times.
+DECODE_FORM_ROWS = 2048
+
+
+def _repeat_queries(x, reps):
+    if reps == 1:
+        return x
+    r = lambda t: t.repeat_interleave(reps, dim=0)
+    return synth.DSAInputs(x.config, r(x.q_idx), r(x.w), x.k_idx, r(x.q), x.kv, r(x.pos), r(x.k_base),
+                           x.k, x.scale, x.d_v, meta=x.meta)
+
+
+def _check_repeated(x, reps, idx):
+    rows = list(range(0, x.T, reps))
+    assert reps == 1 or x.T > DECODE_FORM_ROWS
+    check_indexer(x, _take(idx, rows), rows, exact=True)
+    if reps > 1:   # every copy of a query row selects the same set
+        v = idx.view(-1, reps, x.k)
+        assert torch.equal(v, v[:, :1].expand_as(v))
+
+
+@pytest.mark.parametrize("reps", [1, 700])
+def test_decode_multi_chunk_integer_bit_exact(reps):
+    """Rows of one to five 8192-key chunks; integer FP8-exact inputs make many
+    scores tie across chunks."""
     x = synth.decode_inputs("decode", device="cuda", seed=9, B=5, ctx=[8193, 16384, 20000, 40000, 9000],
                             overrides=dict(indexer="int", k=2048))
+    x = _repeat_queries(x, reps)
     idx = dsa.indexer_topk(x.q_idx, x.w, x.k_idx, x.k, pos=x.pos, k_base=x.k_base)
     torch.cuda.synchronize()
-    check_indexer(x, idx.cpu(), list(range(x.T)), exact=True)
+    _check_repeated(x, reps, idx)
 
 
-def test_decode_threshold_overshoot_still_exact():
-    """Only keys on a regular grid (s mod 4096 < 128) are non-zero, so a
-    threshold sampled on that grid keeps far fewer than k keys; the rows must
-    still get their exact Top-k (ties at score 0 go to the lowest s)."""
+@pytest.mark.parametrize("reps", [1, 700])
+def test_decode_threshold_overshoot_still_exact(reps):
+    """Only keys on a regular grid (s mod 4096 < 128) are non-zero: a threshold
+    sampled on that grid keeps far fewer than k keys (chunked form), and most
+    16-key groups tie at score 0, so the group-maximum filter keeps more pairs
+    than fit in shared memory (decode form). The rows must still get their
+    exact Top-k (ties at score 0 go to the lowest s)."""
     x = synth.decode_inputs("decode", device="cuda", seed=10, B=3, ctx=[30000, 50000, 12000],
                             overrides=dict(indexer="int", k=2048))
     base = x.bases().cpu().long()
@@ -121,6 +150,30 @@ def test_decode_threshold_overshoot_still_exact():
         s = torch.arange(p + 1)
         keep[b + s[(s % 4096) < 128]] = True
     x.k_idx[~keep.to(x.k_idx.device)] = 0
+    x = _repeat_queries(x, reps)
+    idx = dsa.indexer_topk(x.q_idx, x.w, x.k_idx, x.k, pos=x.pos, k_base=x.k_base)
+    torch.cuda.synchronize()
+    _check_repeated(x, reps, idx)
+
+
+def test_decode_all_scores_equal_takes_the_lowest_positions():
+    """Every key row identical: all scores tie, so each row's Top-k is its k
+    lowest positions (both the staged and the global-memory selections)."""
+    x = synth.decode_inputs("decode", device="cuda", seed=17, B=4, ctx=[9000, 16000, 20000, 70000],
+                            overrides=dict(indexer="int", k=2048))
+    x.k_idx[:] = x.k_idx[0]
+    idx = dsa.indexer_topk(x.q_idx, x.w, x.k_idx, x.k, pos=x.pos, k_base=x.k_base)
+    torch.cuda.synchronize()
+    want = torch.arange(x.k, dtype=torch.int32, device="cuda").expand(x.T, x.k)
+    assert torch.equal(idx, want)
+    check_indexer(x, idx.cpu(), list(range(x.T)), exact=True)
+
+
+def test_decode_row_longer_than_a_score_row_is_exact():
+    """A row of more than 2^20 keys is not scored into the workspace; the
+    select recomputes its scores and takes the exact Top-k (integer inputs)."""
+    x = synth.decode_inputs("decode", device="cuda", seed=18, B=2, ctx=[1100000, 30000],
+                            overrides=dict(indexer="int", k=2048))
     idx = dsa.indexer_topk(x.q_idx, x.w, x.k_idx, x.k, pos=x.pos, k_base=x.k_base)
     torch.cuda.synchronize()
     check_indexer(x, idx.cpu(), list(range(x.T)), exact=True)
