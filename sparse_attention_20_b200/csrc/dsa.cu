@@ -220,15 +220,14 @@ ChunkPlan chunk_plan(int T, int S, int k)
 }
 
 // Few rows over long key ranges (decode) with d_I = 128: every key scored into
-// a dense score row, a filter by a threshold from group maxima, then a per-row
-// select (indexer_chunked.cuh, rs). Rows per launch block and the buffers
-// they need: the score rows (ld floats each, at most rs::kMaxKeys keys), the
-// rows' 16-key and 4-key group maxima, and the pairs each segment keeps with
-// their counts.
+// a dense score row, a per-row threshold from group maxima, then a cluster per
+// row filters and selects (indexer_chunked.cuh, rs). Rows per launch block and
+// the buffers they need: the score rows (ld floats each, at most rs::kMaxKeys
+// keys), the rows' 16-key and 4-key group maxima, and the thresholds.
 struct RowScorePlan {
-    int RB, max_segs;
-    long long ld, g16_ld, g4_ld, cand_ld;
-    size_t off_g16, off_g4, off_cand, off_cnt, off_tau, bytes;
+    int RB;
+    long long ld, g16_ld, g4_ld;
+    size_t off_g16, off_g4, off_tau, bytes;
 };
 
 bool use_row_scores(int T, int S, int d_I)
@@ -244,17 +243,13 @@ RowScorePlan row_score_plan(int T, int S)
     p.ld = (long long)dsa::ceil_div(std::min(S, rs::kMaxKeys), rs::kTileKeys) * rs::kTileKeys;
     p.g16_ld = p.ld / rs::kTileKeys * rs::kGroupsPerTile;
     p.g4_ld = p.ld / 4;
-    p.max_segs = (int)dsa::ceil_div(p.ld, (long long)rs::kSegKeys);
-    p.cand_ld = (long long)p.max_segs * rs::kSegCap;
     const size_t per_row = (size_t)p.ld * sizeof(float) + (size_t)(p.g16_ld + p.g4_ld) * sizeof(uint32_t) +
-                           (size_t)p.cand_ld * sizeof(uint2) + (size_t)p.max_segs * sizeof(int) + sizeof(uint32_t);
+                           sizeof(uint32_t);
     p.RB = (int)std::min<size_t>({(size_t)T, (size_t)rs::kMaxRows,
                                   std::max<size_t>(1, kScoreBlockBytes / per_row)});
     p.off_g16 = align_up((size_t)p.RB * p.ld * sizeof(float));
     p.off_g4 = p.off_g16 + align_up((size_t)p.RB * p.g16_ld * sizeof(uint32_t));
-    p.off_cand = p.off_g4 + align_up((size_t)p.RB * p.g4_ld * sizeof(uint32_t));
-    p.off_cnt = p.off_cand + align_up((size_t)p.RB * p.cand_ld * sizeof(uint2));
-    p.off_tau = p.off_cnt + align_up((size_t)p.RB * p.max_segs * sizeof(int));
+    p.off_tau = p.off_g4 + align_up((size_t)p.RB * p.g4_ld * sizeof(uint32_t));
     p.bytes = p.off_tau + align_up((size_t)p.RB * sizeof(uint32_t));
     return p;
 }
@@ -533,23 +528,18 @@ int indexer_chunked(const uint8_t* q_idx, const float* w, const uint8_t* k_idx, 
             return rc;
     }
     if (fn.row_scores && use_row_scores(T, S, d_I)) {
-        // every key into a dense score row; per segment, the scores above a
-        // threshold from group maxima; then one select CTA per row
+        // every key into a dense score row; a threshold per row from group
+        // maxima; then a cluster per row filters and selects
         const RowScorePlan q = row_score_plan(T, S);
         float* scores = reinterpret_cast<float*>(ws);
         uint32_t* g16 = reinterpret_cast<uint32_t*>(ws + q.off_g16);
         uint32_t* g4 = reinterpret_cast<uint32_t*>(ws + q.off_g4);
-        uint2* rcand = reinterpret_cast<uint2*>(ws + q.off_cand);
-        int* rcnt = reinterpret_cast<int*>(ws + q.off_cnt);
         uint32_t* rtau = reinterpret_cast<uint32_t*>(ws + q.off_tau);
-        cudaError_t e = cudaFuncSetAttribute(row_filter_kernel<rs::kFiltThreads>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, rs::kFiltSmem);
+        cudaError_t e = cudaFuncSetAttribute(row_tau_kernel<rs::kTauThreads>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, rs::kTauSmem);
         if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(row_tau_kernel<rs::kTauThreads>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     rs::kTauSmem);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(row_merge_kernel<rs::kMergeThreads>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, rs::kMergeSmem);
+            e = cudaFuncSetAttribute(row_select_cluster_kernel<rs::kCsThreads>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, rs::kCsSmem);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(row select kernels)");
         for (int row0 = 0; row0 < T; row0 += q.RB) {
             const int rows = std::min(q.RB, T - row0);
@@ -562,16 +552,12 @@ int indexer_chunked(const uint8_t* q_idx, const float* w, const uint8_t* k_idx, 
             launch_pdl(row_tau_kernel<rs::kTauThreads>, dim3(rows), dim3(rs::kTauThreads), rs::kTauSmem, st, g16,
                        q.g16_ld, g4, q.g4_ld, pos, k_base, T, S, row0, k, rtau, pg);
             DSA_LAUNCH_CHECK("row_tau_kernel");
-            launch_pdl(row_filter_kernel<rs::kFiltThreads>, dim3(2 * num_sms()), dim3(rs::kFiltThreads),
-                       rs::kFiltSmem, st, scores, q.ld, rtau, pos, k_base, T, S, row0, rows, k, rcand, q.cand_ld,
-                       rcnt, q.max_segs, pg);
-            DSA_LAUNCH_CHECK("row_filter_kernel");
             phase_end(ph);
             ph = phase_begin(kPhaseSelect, st);
-            launch_pdl(row_merge_kernel<rs::kMergeThreads>, dim3(rows), dim3(rs::kMergeThreads), rs::kMergeSmem, st,
-                       scores, q.ld, rcand, q.cand_ld, rcnt, q.max_segs, q_idx, w, k_idx, H_I, d_I, pos, k_base, T,
-                       S, row0, k, idx, pg);
-            DSA_LAUNCH_CHECK("row_merge_kernel");
+            launch_pdl(row_select_cluster_kernel<rs::kCsThreads>, dim3(rs::kClusterCtas * rows),
+                       dim3(rs::kCsThreads), rs::kCsSmem, st, scores, q.ld, rtau, q_idx, w, k_idx, H_I, d_I, pos,
+                       k_base, T, S, row0, k, idx, pg);
+            DSA_LAUNCH_CHECK("row_select_cluster_kernel");
             phase_end(ph);
         }
         return DSA_OK;

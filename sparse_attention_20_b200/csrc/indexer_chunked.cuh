@@ -775,7 +775,7 @@ merge_topk_kernel(const uint2* __restrict__ cand, long long cand_ld, const int* 
     }
 }
 
-// Row Top-k from the dense score rows of row_scores_tma_kernel, in three
+// Row Top-k from the dense score rows of row_scores_tma_kernel, in two
 // steps, for rows of k < n <= rs::kMaxKeys keys.
 //
 // row_tau_kernel (one CTA per row): the row's threshold tau, a lower bound of
@@ -785,50 +785,35 @@ merge_topk_kernel(const uint2* __restrict__ cand, long long cand_ld, const int* 
 // groups, else tau = 0 (rows of fewer than 4k keys keep everything);
 // range_floor rounds it down to a histogram sub-bin edge.
 //
-// row_filter_kernel: persistent CTAs over the (row, segment of kSegKeys keys)
-// items, cut into equal contiguous ranges. An item's scores reach shared
-// memory by one 1-D bulk copy; the scores >= tau are kept as (order key, s)
-// pairs in ascending s (each warp counts its share, one scan over the warps,
-// then each warp writes its share in order), up to kSegCap of them, at
-// cand[r * cand_ld + seg * kSegCap ...], with their count at
-// ccnt[r * max_segs + seg].
-//
-// row_merge_kernel (one CTA per row): the row's Top-k is among its kept pairs
-// (they hold every score >= tau). The segments' pairs are bulk-copied in
-// order into a staging area (each run at an even offset, for the copies'
-// 16-byte alignment), then packed into one list in ascending s. Their exact
-// Top-k (range-histogram select, or the radix select where the keys'
-// spread defeats it) is marked in a bitmap over the pairs and written in
-// ascending s. A row whose pairs did not fit (a segment over kSegCap, or
-// more than kMergeList in all: scores far from independent) is selected over
-// its score row in global memory instead, marked in a bitmap over s. A row
-// of at most k keys lists them and pads with -1; a row longer than kMaxKeys
-// gets the exact Top-k of scores it recomputes.
+// row_select_cluster_kernel (a cluster of kClusterCtas CTAs per row): CTA q
+// streams the q-th contiguous part of the score row through two shared-memory
+// buffers (1-D bulk copies) and keeps its scores >= tau as (order key, s)
+// pairs in ascending s (a scan over the CTA per chunk). The parts' counts are
+// exchanged over distributed shared memory, each part's pairs are stored into
+// CTA 0 after the pairs of the parts before it, so CTA 0 holds every score
+// >= tau in ascending s, and CTA 0 takes their exact Top-k (range-histogram
+// select, or the radix select where the keys' spread defeats it), marked in a
+// bitmap over the pairs and written in ascending s. Parts that keep more than
+// kCsLocal pairs, or more than kCsList in all (scores far from independent),
+// send the row to CTA 0's exact select over the score row in global memory.
+// A row of at most k keys lists them and pads with -1; a row longer than
+// kMaxKeys gets the exact Top-k of scores it recomputes. Every CTA of a
+// cluster takes the same path through the cluster barriers.
 namespace rs {
-constexpr int kSegKeys = 16384;
-constexpr int kSegCap = 8192;
 constexpr int kTauThreads = 512;
-constexpr int kMaxStaged = 16384;                        // group maxima staged in shared memory
+constexpr int kMaxStaged = 16384;                          // group maxima staged in shared memory
 constexpr int kTauSmem = kMaxStaged * 4 + 16;
-constexpr int kFiltThreads = 512;
-constexpr int kOffSegTbl = kSegKeys * 4;                 // the segment, then the item table
-constexpr int kOffFiltBar = kOffSegTbl + (kMaxRows + 1 + 3) / 4 * 16;
-constexpr int kFiltSmem = kOffFiltBar + 16;
-constexpr int kMergeThreads = 256;
-constexpr int kMergeList = 8192;                         // pairs of a row in shared memory
-constexpr int kOffStage = kMergeList * 8;                // the list, then the staging area,
-constexpr int kOffListBits = 2 * kMergeList * 8;         // then the bitmap over the list
-constexpr int kOffMergeBar = kOffListBits + kMergeList / 8;
-constexpr int kMergeSmem = kOffMergeBar + 16;            // (or a bitmap over s, from 0)
-constexpr int kMaxSegs = kMaxKeys / kSegKeys;
-static_assert(kOffMergeBar >= kMaxKeys / 8, "a bitmap over the longest row fits below the barrier");
-static_assert(kSegCap >= 2 * 4 * 1024, "a row below 4k keys (k <= 2048) keeps all of them in one item");
-static_assert(kSegKeys % (kFiltThreads / 32 * 128) == 0, "whole float4 rows per warp");
-
-__device__ __forceinline__ int row_segs(int n, int k)
-{
-    return n > k && n <= kMaxKeys ? ceil_div(n, kSegKeys) : 0;
-}
+constexpr int kClusterCtas = 4;
+constexpr int kCsThreads = 512;
+constexpr int kCsChunk = kCsThreads * 4;                   // scores per copy: one float4 per thread
+constexpr int kCsLocal = 4096;                             // pairs one part keeps
+constexpr int kCsList = 8192;                              // pairs of the row in CTA 0
+constexpr int kOffCsLocal = (kCsList - kCsLocal) * 8;      // a part's pairs: the top of the list space
+constexpr int kOffCsBuf = kCsList * 8;                     // two chunk buffers
+constexpr int kOffCsBits = kOffCsBuf + 2 * kCsChunk * 4;   // bitmap over CTA 0's list
+constexpr int kOffCsBars = kOffCsBits + kCsList / 8;
+constexpr int kCsSmem = kOffCsBars + 16;
+static_assert(kCsLocal * 8 <= kOffCsLocal, "CTA 0 moves its own pairs down without overlap");
 }  // namespace rs
 
 template <int THREADS>
@@ -876,155 +861,6 @@ row_tau_kernel(const uint32_t* __restrict__ gmax16, long long g16_ld, const uint
     if (tid == 0) tau[r] = t;
 }
 
-template <int THREADS>
-__global__ void __launch_bounds__(THREADS, 2)
-row_filter_kernel(const float* __restrict__ scores, long long ld, const uint32_t* __restrict__ tau,
-                  const int* __restrict__ pos, const int* __restrict__ k_base, int T, int S, int row0, int rows,
-                  int k, uint2* __restrict__ cand, long long cand_ld, int* __restrict__ ccnt, int max_segs,
-                  const PagedRows pg)
-{
-    using namespace sm100;
-    constexpr int W = THREADS / 32;
-    constexpr int kPerWarp = rs::kSegKeys / W;
-    static_assert(THREADS == rs::kFiltThreads && W <= 32, "launch shape");
-    __shared__ int wsum[W];
-    __shared__ int abort_s;
-    extern __shared__ __align__(16) uint8_t dyn[];
-    const uint32_t dyn_s = smem_u32(dyn);
-    const float* seg = reinterpret_cast<const float*>(dyn);
-    int* tbl = reinterpret_cast<int*>(dyn + rs::kOffSegTbl);
-    const uint32_t bar = dyn_s + rs::kOffFiltBar;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    if (tid == 0) {
-        mbar_init(bar, 1);
-        abort_s = 0;
-        fence_mbar_init_cluster();
-    }
-    griddep_wait();
-    // tbl[r] = items of rows 0 .. r-1
-    auto segs_of = [&](int r) -> int {
-        long long b;
-        const int* bt;
-        return rs::row_segs(row_keys(pg, pos, k_base, row0 + r, T, S, &b, &bt), k);
-    };
-    {
-        const int per = ceil_div(rows, THREADS);
-        const int a0 = min(rows, tid * per), a1 = min(rows, a0 + per);
-        int sum = 0;
-        for (int r = a0; r < a1; ++r) sum += segs_of(r);
-        int incl = sum;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const int v = __shfl_up_sync(0xffffffffu, incl, off);
-            if (lane >= off) incl += v;
-        }
-        if (lane == 31) wsum[warp] = incl;
-        __syncthreads();
-        int acc = incl - sum, total = 0;
-#pragma unroll
-        for (int q = 0; q < W; ++q) {
-            if (q < warp) acc += wsum[q];
-            total += wsum[q];
-        }
-        for (int r = a0; r < a1; ++r) {
-            tbl[r] = acc;
-            acc += segs_of(r);
-        }
-        if (tid == 0) tbl[rows] = total;
-        __syncthreads();
-    }
-    const long long G = tbl[rows];
-    const int i0 = (int)(G * blockIdx.x / gridDim.x), i1 = (int)(G * (blockIdx.x + 1) / gridDim.x);
-    for (int item = i0, phase = 0; item < i1; ++item, ++phase) {
-        int r;
-        {
-            int lo = 0, hi = rows - 1;
-            while (lo < hi) {
-                const int mid = (lo + hi + 1) >> 1;
-                if (tbl[mid] <= item) lo = mid; else hi = mid - 1;
-            }
-            r = lo;
-        }
-        const int sg = item - tbl[r];
-        long long base;
-        const int* bt;
-        const int n = row_keys(pg, pos, k_base, row0 + r, T, S, &base, &bt);
-        const int s0 = sg * rs::kSegKeys, cnt = min(rs::kSegKeys, n - s0);
-        if (tid == 0) {
-            // the last copy of a row is rounded up to 16 bytes: it stays inside ld
-            const uint32_t bytes = (uint32_t)(cnt * 4 + 15) & ~15u;
-            mbar_arrive_expect_tx(bar, bytes);
-            bulk_g2s(dyn_s, scores + (size_t)r * ld + s0, bytes, bar);
-        }
-        // the float whose order key is tau: x >= tf keeps every score whose
-        // key is >= tau (and at most a zero of the other sign besides, which
-        // ranks below k kept scores and is never selected); tau = 0 keeps all
-        const uint32_t tk = tau[r];
-        const float tf = tk ? key_score(tk) : -INFINITY;
-        const bool got = mbar_wait(bar, (uint32_t)(phase & 1), (volatile int*)&abort_s, 670, item);
-        if (__syncthreads_or(!got)) return;
-        // pad the last run of 128 past cnt with NaN, which no compare keeps
-        // (the copy left it stale)
-        float* segw = reinterpret_cast<float*>(dyn);
-        const int cnt128 = (cnt + 127) & ~127;
-        for (int i = cnt + tid; i < cnt128; i += THREADS) segw[i] = __int_as_float(0x7FC00000);
-        __syncthreads();
-        // warp w owns entries [w * kPerWarp, (w + 1) * kPerWarp) below cnt128:
-        // lane l takes entries 4l .. 4l+3 of each run of 128
-        const int e0 = warp * kPerWarp;
-        const int iters = max(0, min(kPerWarp, cnt128 - e0)) / 128;
-        auto bits_at = [&](int it, float4& v) -> uint32_t {
-            v = *reinterpret_cast<const float4*>(seg + e0 + it * 128 + 4 * lane);
-            return (uint32_t)(v.x >= tf) | (uint32_t)(v.y >= tf) << 1 | (uint32_t)(v.z >= tf) << 2 |
-                   (uint32_t)(v.w >= tf) << 3;
-        };
-        int mine = 0;
-#pragma unroll 4
-        for (int it = 0; it < iters; ++it) {
-            float4 v;
-            mine += __popc(bits_at(it, v));
-        }
-#pragma unroll
-        for (int off = 16; off; off >>= 1) mine += __shfl_xor_sync(0xffffffffu, mine, off);
-        if (lane == 0) wsum[warp] = mine;
-        __syncthreads();
-        const int x = lane < W ? wsum[lane] : 0;
-        int xi = x;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, xi, off);
-            if (lane >= off) xi += y;
-        }
-        int at = __shfl_sync(0xffffffffu, xi - x, warp);
-        const int total = __shfl_sync(0xffffffffu, xi, W - 1);
-        uint2* dst = cand + (size_t)r * cand_ld + (size_t)sg * rs::kSegCap;
-#pragma unroll 2
-        for (int it = 0; it < iters && at < rs::kSegCap; ++it) {
-            float4 v;
-            const uint32_t b = bits_at(it, v);
-            const float e[4] = {v.x, v.y, v.z, v.w};
-            const int c = __popc(b);
-            int incl = c;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const int y = __shfl_up_sync(0xffffffffu, incl, off);
-                if (lane >= off) incl += y;
-            }
-            int o = at + incl - c;
-            const int s = s0 + e0 + it * 128 + 4 * lane;
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-                if (b >> q & 1u) {
-                    if (o < rs::kSegCap) dst[o] = make_uint2(score_key(e[q]), (uint32_t)(s + q));
-                    ++o;
-                }
-            at += __shfl_sync(0xffffffffu, incl, 31);
-        }
-        if (tid == 0) ccnt[(size_t)r * max_segs + sg] = total;
-        __syncthreads();   // the segment buffer and wsum take the next item
-    }
-}
-
 // Pairs staged in shared memory; entry i is marked as bit i.
 struct PairList {
     const uint2* p;
@@ -1033,25 +869,28 @@ struct PairList {
 };
 
 template <int THREADS>
-__global__ void __launch_bounds__(THREADS)
-row_merge_kernel(const float* __restrict__ scores, long long ld, const uint2* __restrict__ cand,
-                 long long cand_ld, const int* __restrict__ ccnt, int max_segs, const uint8_t* __restrict__ q_idx,
-                 const float* __restrict__ w, const uint8_t* __restrict__ k_idx, int H_I, int d_I,
-                 const int* __restrict__ pos, const int* __restrict__ k_base, int T, int S, int row0, int k,
-                 int32_t* __restrict__ idx, const PagedRows pg)
+__global__ void __cluster_dims__(rs::kClusterCtas, 1, 1) __launch_bounds__(THREADS, 2)
+row_select_cluster_kernel(const float* __restrict__ scores, long long ld, const uint32_t* __restrict__ tau,
+                          const uint8_t* __restrict__ q_idx, const float* __restrict__ w,
+                          const uint8_t* __restrict__ k_idx, int H_I, int d_I, const int* __restrict__ pos,
+                          const int* __restrict__ k_base, int T, int S, int row0, int k, int32_t* __restrict__ idx,
+                          const PagedRows pg)
 {
     using namespace sm100;
+    constexpr int W = THREADS / 32;
+    static_assert(THREADS == rs::kCsThreads && W <= 32, "launch shape");
     __shared__ SelectSmem<THREADS> sm;
-    __shared__ int cnt_s[rs::kMaxSegs], off_s[rs::kMaxSegs + 1], pre_s[rs::kMaxSegs + 1];
-    __shared__ int over_s, abort_s;
+    __shared__ int wsum[2][W];
+    __shared__ int count_s, abort_s;
     extern __shared__ __align__(16) uint8_t dyn[];
     const uint32_t dyn_s = smem_u32(dyn);
-    const uint32_t bar = dyn_s + rs::kOffMergeBar;
-    const int r = blockIdx.x, t = row0 + r, tid = threadIdx.x;
+    auto full = [&](int b) -> uint32_t { return dyn_s + rs::kOffCsBars + 8u * (uint32_t)b; };
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int q = (int)cluster_ctarank(), r = blockIdx.x / rs::kClusterCtas, t = row0 + r;
     if (tid == 0) {
-        mbar_init(bar, 1);
+        mbar_init(full(0), 1);
+        mbar_init(full(1), 1);
         abort_s = 0;
-        over_s = 0;
         fence_mbar_init_cluster();
     }
     __syncthreads();
@@ -1061,10 +900,12 @@ row_merge_kernel(const float* __restrict__ scores, long long ld, const uint2* __
     const int n = row_keys(pg, pos, k_base, t, T, S, &base, &bt);
     int32_t* out = idx + (size_t)t * k;
     if (n <= k) {
-        for (int i = tid; i < k; i += THREADS) out[i] = i < n ? i : -1;
+        if (q == 0)
+            for (int i = tid; i < k; i += THREADS) out[i] = i < n ? i : -1;
         return;
     }
     if (n > rs::kMaxKeys) {
+        if (q != 0) return;
         float* qf = reinterpret_cast<float*>(dyn);
         float* wf = qf + H_I * d_I;
         const uint8_t* qrow = q_idx + (size_t)t * H_I * d_I;
@@ -1074,70 +915,108 @@ row_merge_kernel(const float* __restrict__ scores, long long ld, const uint2* __
         block_topk<THREADS>(RecomputedRow{qf, wf, k_idx, pg, bt, base, H_I, d_I}, n, k, out, sm);
         return;
     }
-    const int nseg = rs::row_segs(n, k);
-    for (int sg = tid; sg < nseg; sg += THREADS) {
-        const int c = ccnt[(size_t)r * max_segs + sg];
-        cnt_s[sg] = c;
-        if (c > rs::kSegCap) over_s = 1;
-    }
-    __syncthreads();
-    if (tid == 0) {
-        // segment sg's run is staged at off_s[sg] (even) and packed at pre_s[sg]
-        off_s[0] = 0;
-        pre_s[0] = 0;
-        for (int sg = 0; sg < nseg; ++sg) {
-            const int c = min(cnt_s[sg], rs::kSegCap);
-            off_s[sg + 1] = off_s[sg] + ((c + 1) & ~1);
-            pre_s[sg + 1] = pre_s[sg] + c;
+    const float* sc = scores + (size_t)r * ld;
+    // this CTA's part [a, b) of the row, in chunks of kCsChunk scores
+    const int span = ceil_div(ceil_div(n, rs::kClusterCtas), rs::kCsChunk) * rs::kCsChunk;
+    const int a = min(n, q * span), b = min(n, a + span);
+    const int nch = ceil_div(b - a, rs::kCsChunk);
+    // the float whose order key is tau: x >= tf keeps every score whose key
+    // is >= tau (and at most a zero of the other sign besides, which ranks
+    // below k kept scores and is never selected); tau = 0 keeps all
+    const uint32_t tk = tau[r];
+    const float tf = tk ? key_score(tk) : -INFINITY;
+    auto issue = [&](int j) {
+        const int s0 = a + j * rs::kCsChunk;
+        // the last copy of a row is rounded up to 16 bytes: it stays inside ld
+        const uint32_t bytes = (uint32_t)(min(rs::kCsChunk, b - s0) * 4 + 15) & ~15u;
+        mbar_arrive_expect_tx(full(j & 1), bytes);
+        bulk_g2s(dyn_s + rs::kOffCsBuf + (uint32_t)(j & 1) * rs::kCsChunk * 4u, sc + s0, bytes, full(j & 1));
+    };
+    if (tid == 0)
+        for (int j = 0; j < min(nch, 2); ++j) issue(j);
+    uint2* local = reinterpret_cast<uint2*>(dyn + rs::kOffCsLocal);
+    int running = 0;
+    bool bad = false;
+    for (int j = 0; j < nch; ++j) {
+        const bool got = mbar_wait(full(j & 1), (uint32_t)((j >> 1) & 1), (volatile int*)&abort_s, 673, j);
+        const int s = a + j * rs::kCsChunk + 4 * tid;
+        const float4 v = *reinterpret_cast<const float4*>(dyn + rs::kOffCsBuf + (j & 1) * rs::kCsChunk * 4 + 16 * tid);
+        const float e[4] = {v.x, v.y, v.z, v.w};
+        uint32_t bits = 0u;
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            if (s + u < b && e[u] >= tf) bits |= 1u << u;
+        const int cnt = __popc(bits);
+        int incl = cnt;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int x = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += x;
         }
-        if (off_s[nseg] > rs::kMergeList) over_s = 1;
+        if (lane == 31) wsum[j & 1][warp] = incl;
+        if (__syncthreads_or(!got)) {
+            bad = true;   // a copy timed out: the row takes the global-memory select
+            break;
+        }
+        // every thread has read buffer j & 1: refill it
+        if (tid == 0 && j + 2 < nch) issue(j + 2);
+        const int x = lane < W ? wsum[j & 1][lane] : 0;
+        int xi = x;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, xi, off);
+            if (lane >= off) xi += y;
+        }
+        int at = running + __shfl_sync(0xffffffffu, xi - x, warp) + incl - cnt;
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            if (bits >> u & 1u) {
+                if (at < rs::kCsLocal) local[at] = make_uint2(score_key(e[u]), (uint32_t)(s + u));
+                ++at;
+            }
+        running += __shfl_sync(0xffffffffu, xi, W - 1);
     }
-    __syncthreads();
+    if (tid == 0) count_s = bad ? rs::kCsLocal + 1 : running;
+    __syncthreads();   // every thread's pairs of the last chunk are written
+    uint2* list = reinterpret_cast<uint2*>(dyn);
+    if (q == 0) {
+        // CTA 0's pairs go first: move them down (the two ranges do not
+        // overlap), before any other part stores into the list
+        for (int i = tid; i < min(running, rs::kCsLocal); i += THREADS) list[i] = local[i];
+    }
+    cluster_sync();   // 1: every part's count is final (and every CTA of the cluster runs)
+    int before = 0, total = 0;
+    bool over = false;
+#pragma unroll
+    for (int p = 0; p < rs::kClusterCtas; ++p) {
+        const int c = (int)ld_cluster_u32(mapa(smem_u32(&count_s), (uint32_t)p));
+        over |= c > rs::kCsLocal;
+        if (p < q) before += c;
+        total += c;
+    }
+    over |= total > rs::kCsList;
+    cluster_sync();   // 2: every CTA has read the counts (none exits before that)
     int* warp_sums = reinterpret_cast<int*>(sm.hist[0]);
-    if (!over_s) {
-        const int c = pre_s[nseg];   // >= k: every score >= tau
-        uint2* list = reinterpret_cast<uint2*>(dyn);
-        const uint2* stage = reinterpret_cast<const uint2*>(dyn + rs::kOffStage);
-        uint32_t* lbm = reinterpret_cast<uint32_t*>(dyn + rs::kOffListBits);
-        const uint2* src = cand + (size_t)r * cand_ld;
-        if (tid == 0) {
-            mbar_arrive_expect_tx(bar, (uint32_t)off_s[nseg] * 8u);
-            for (int sg = 0; sg < nseg; ++sg) {
-                const uint32_t bytes = (uint32_t)(off_s[sg + 1] - off_s[sg]) * 8u;
-                if (bytes)
-                    bulk_g2s(dyn_s + rs::kOffStage + (uint32_t)off_s[sg] * 8u, src + (size_t)sg * rs::kSegCap,
-                             bytes, bar);
-            }
-        }
-        for (int i = tid; i < (c + 31) / 32; i += THREADS) lbm[i] = 0u;
-        const bool got = mbar_wait(bar, 0, (volatile int*)&abort_s, 672, r);
-        if (__syncthreads_or(!got)) return;
-        // pack: pair i of the list is in the last run whose packed start is <= i
-        for (int i = tid; i < c; i += THREADS) {
-            int lo = 0, hi = nseg - 1;
-            while (lo < hi) {
-                const int mid = (lo + hi + 1) >> 1;
-                if (pre_s[mid] <= i) lo = mid; else hi = mid - 1;
-            }
-            list[i] = stage[off_s[lo] + (i - pre_s[lo])];
-        }
-        __syncthreads();
-        const PairList row{list};
-        if (!range_select_bitmap<THREADS>(row, c, k, lbm, sm))
-            block_select<THREADS>(row, c, k, [&](int, int i) { atomicOr(&lbm[i >> 5], 1u << (i & 31)); }, sm);
-        __syncthreads();
-        block_emit_bitmap<THREADS>(lbm, c, out, warp_sums, [&](int i) { return (int)list[i].y; });
+    if (over) {
+        // (the same decision in every CTA: no further cluster barrier)
+        if (q != 0) return;
+        block_topk<THREADS>(DenseScores{sc}, n, k, out, sm);
         return;
     }
-    // the pairs did not fit: select over the score row in global memory
-    uint32_t* bm = reinterpret_cast<uint32_t*>(dyn);
-    for (int i = tid; i < (n + 31) / 32; i += THREADS) bm[i] = 0u;
+    if (q != 0) {
+        const uint32_t dst = mapa(dyn_s, 0u) + (uint32_t)before * 8u;
+        for (int i = tid; i < running; i += THREADS) st_cluster_v2(dst + 8u * (uint32_t)i, local[i]);
+    }
+    cluster_sync();   // 3: every part's pairs are in CTA 0 (release / acquire)
+    if (q != 0) return;
+    uint32_t* lbm = reinterpret_cast<uint32_t*>(dyn + rs::kOffCsBits);
+    for (int i = tid; i < (total + 31) / 32; i += THREADS) lbm[i] = 0u;
     __syncthreads();
-    const DenseScores row{scores + (size_t)r * ld};
-    if (!range_select_bitmap<THREADS>(row, n, k, bm, sm))
-        block_select<THREADS>(row, n, k, [&](int, int i) { atomicOr(&bm[i >> 5], 1u << (i & 31)); }, sm);
+    const PairList row{list};
+    if (!range_select_bitmap<THREADS>(row, total, k, lbm, sm))
+        block_select<THREADS>(row, total, k, [&](int, int i) { atomicOr(&lbm[i >> 5], 1u << (i & 31)); }, sm);
     __syncthreads();
-    block_emit_bitmap<THREADS>(bm, n, out, warp_sums);
+    block_emit_bitmap<THREADS>(lbm, total, out, warp_sums, [&](int i) { return (int)list[i].y; });
 }
 
 }  // namespace idx_chunk
