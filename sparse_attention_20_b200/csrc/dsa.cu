@@ -220,14 +220,14 @@ ChunkPlan chunk_plan(int T, int S, int k)
 }
 
 // Few rows over long key ranges (decode) with d_I = 128: every key scored into
-// a dense score row, a per-row threshold from group maxima, then a cluster per
-// row filters and selects (indexer_chunked.cuh, rs). Rows per launch block and
-// the buffers they need: the score rows (ld floats each, at most rs::kMaxKeys
-// keys), the rows' 16-key and 4-key group maxima, and the thresholds.
+// a dense score row, then a cluster per row thresholds, filters and selects
+// (indexer_chunked.cuh, rs). Rows per launch block and the buffers they need:
+// the score rows (ld floats each, at most rs::kMaxKeys keys) and the rows'
+// 16-key and 4-key group maxima.
 struct RowScorePlan {
     int RB;
     long long ld, g16_ld, g4_ld;
-    size_t off_g16, off_g4, off_tau, bytes;
+    size_t off_g16, off_g4, bytes;
 };
 
 bool use_row_scores(int T, int S, int d_I)
@@ -243,14 +243,12 @@ RowScorePlan row_score_plan(int T, int S)
     p.ld = (long long)dsa::ceil_div(std::min(S, rs::kMaxKeys), rs::kTileKeys) * rs::kTileKeys;
     p.g16_ld = p.ld / rs::kTileKeys * rs::kGroupsPerTile;
     p.g4_ld = p.ld / 4;
-    const size_t per_row = (size_t)p.ld * sizeof(float) + (size_t)(p.g16_ld + p.g4_ld) * sizeof(uint32_t) +
-                           sizeof(uint32_t);
+    const size_t per_row = (size_t)p.ld * sizeof(float) + (size_t)(p.g16_ld + p.g4_ld) * sizeof(uint32_t);
     p.RB = (int)std::min<size_t>({(size_t)T, (size_t)rs::kMaxRows,
                                   std::max<size_t>(1, kScoreBlockBytes / per_row)});
     p.off_g16 = align_up((size_t)p.RB * p.ld * sizeof(float));
     p.off_g4 = p.off_g16 + align_up((size_t)p.RB * p.g16_ld * sizeof(uint32_t));
-    p.off_tau = p.off_g4 + align_up((size_t)p.RB * p.g4_ld * sizeof(uint32_t));
-    p.bytes = p.off_tau + align_up((size_t)p.RB * sizeof(uint32_t));
+    p.bytes = p.off_g4 + align_up((size_t)p.RB * p.g4_ld * sizeof(uint32_t));
     return p;
 }
 
@@ -528,18 +526,14 @@ int indexer_chunked(const uint8_t* q_idx, const float* w, const uint8_t* k_idx, 
             return rc;
     }
     if (fn.row_scores && use_row_scores(T, S, d_I)) {
-        // every key into a dense score row; a threshold per row from group
-        // maxima; then a cluster per row filters and selects
+        // every key into a dense score row, then a cluster per row
+        // thresholds, filters and selects
         const RowScorePlan q = row_score_plan(T, S);
         float* scores = reinterpret_cast<float*>(ws);
         uint32_t* g16 = reinterpret_cast<uint32_t*>(ws + q.off_g16);
         uint32_t* g4 = reinterpret_cast<uint32_t*>(ws + q.off_g4);
-        uint32_t* rtau = reinterpret_cast<uint32_t*>(ws + q.off_tau);
-        cudaError_t e = cudaFuncSetAttribute(row_tau_kernel<rs::kTauThreads>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, rs::kTauSmem);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(row_select_cluster_kernel<rs::kCsThreads>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, rs::kCsSmem);
+        cudaError_t e = cudaFuncSetAttribute(row_select_cluster_kernel<rs::kCsThreads>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, rs::kCsSmem);
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(row select kernels)");
         for (int row0 = 0; row0 < T; row0 += q.RB) {
             const int rows = std::min(q.RB, T - row0);
@@ -548,15 +542,10 @@ int indexer_chunked(const uint8_t* q_idx, const float* w, const uint8_t* k_idx, 
             fn.row_scores(rs::kCtasPerSm * num_sms(), st, tm_k, a, scores, q.ld, g16, q.g16_ld, g4, q.g4_ld);
             DSA_LAUNCH_CHECK("row_scores_tma_kernel");
             phase_end(ph);
-            ph = phase_begin(kPhaseThreshold, st);
-            launch_pdl(row_tau_kernel<rs::kTauThreads>, dim3(rows), dim3(rs::kTauThreads), rs::kTauSmem, st, g16,
-                       q.g16_ld, g4, q.g4_ld, pos, k_base, T, S, row0, k, rtau, pg);
-            DSA_LAUNCH_CHECK("row_tau_kernel");
-            phase_end(ph);
             ph = phase_begin(kPhaseSelect, st);
             launch_pdl(row_select_cluster_kernel<rs::kCsThreads>, dim3(rs::kClusterCtas * rows),
-                       dim3(rs::kCsThreads), rs::kCsSmem, st, scores, q.ld, rtau, q_idx, w, k_idx, H_I, d_I, pos,
-                       k_base, T, S, row0, k, idx, pg);
+                       dim3(rs::kCsThreads), rs::kCsSmem, st, scores, q.ld, g16, q.g16_ld, g4, q.g4_ld, q_idx, w,
+                       k_idx, H_I, d_I, pos, k_base, T, S, row0, k, idx, pg);
             DSA_LAUNCH_CHECK("row_select_cluster_kernel");
             phase_end(ph);
         }

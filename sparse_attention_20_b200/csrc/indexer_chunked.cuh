@@ -775,20 +775,21 @@ merge_topk_kernel(const uint2* __restrict__ cand, long long cand_ld, const int* 
     }
 }
 
-// Row Top-k from the dense score rows of row_scores_tma_kernel, in two
-// steps, for rows of k < n <= rs::kMaxKeys keys.
+// Row Top-k from the dense score rows of row_scores_tma_kernel, for rows of
+// k < n <= rs::kMaxKeys keys: row_select_cluster_kernel, a cluster of
+// kClusterCtas CTAs per row.
 //
-// row_tau_kernel (one CTA per row): the row's threshold tau, a lower bound of
-// its k-th largest score taken from group maxima. With at least k groups, the
-// k-th largest group maximum is reached by at least k groups, so by at least
-// k scores: the 16-key groups where the row has k of them, else the 4-key
-// groups, else tau = 0 (rows of fewer than 4k keys keep everything);
-// range_floor rounds it down to a histogram sub-bin edge.
-//
-// row_select_cluster_kernel (a cluster of kClusterCtas CTAs per row): CTA q
-// streams the q-th contiguous part of the score row through two shared-memory
-// buffers (1-D bulk copies) and keeps its scores >= tau as (order key, s)
-// pairs in ascending s (a scan over the CTA per chunk). The parts' counts are
+// Every CTA first takes the row's threshold tau, a lower bound of its k-th
+// largest score, from group maxima. With at least k groups, the k-th largest
+// group maximum is reached by at least k groups, so by at least k scores: the
+// 16-key groups where the row has k of them, else the 4-key groups, else
+// tau = 0 (rows of fewer than 4k keys keep everything); range_floor rounds it
+// down to a histogram sub-bin edge. Then CTA q streams the q-th contiguous
+// part of the score row through a ring of kCsStages shared-memory buffers
+// (1-D bulk copies; four of them in the lower half of the pair space, which is
+// free until the pairs are gathered) and keeps its scores >= tau as
+// (order key, s) pairs in ascending s (a scan over the CTA per chunk). The
+// parts' counts are
 // exchanged over distributed shared memory, each part's pairs are stored into
 // CTA 0 after the pairs of the parts before it, so CTA 0 holds every score
 // >= tau in ascending s, and CTA 0 takes their exact Top-k (range-histogram
@@ -800,66 +801,24 @@ merge_topk_kernel(const uint2* __restrict__ cand, long long cand_ld, const int* 
 // kMaxKeys gets the exact Top-k of scores it recomputes. Every CTA of a
 // cluster takes the same path through the cluster barriers.
 namespace rs {
-constexpr int kTauThreads = 512;
-constexpr int kMaxStaged = 16384;                          // group maxima staged in shared memory
-constexpr int kTauSmem = kMaxStaged * 4 + 16;
+constexpr int kMaxStaged = 16384;                          // group maxima staged in the pair space
 constexpr int kClusterCtas = 4;
 constexpr int kCsThreads = 512;
 constexpr int kCsChunk = kCsThreads * 4;                   // scores per copy: one float4 per thread
 constexpr int kCsLocal = 4096;                             // pairs one part keeps
 constexpr int kCsList = 8192;                              // pairs of the row in CTA 0
 constexpr int kOffCsLocal = (kCsList - kCsLocal) * 8;      // a part's pairs: the top of the list space
-constexpr int kOffCsBuf = kCsList * 8;                     // two chunk buffers
+constexpr int kCsStages = 6;
+constexpr int kOffCsBuf = kCsList * 8;                     // chunk buffers 0, 1 (2..5: the pair space)
 constexpr int kOffCsBits = kOffCsBuf + 2 * kCsChunk * 4;   // bitmap over CTA 0's list
 constexpr int kOffCsBars = kOffCsBits + kCsList / 8;
-constexpr int kCsSmem = kOffCsBars + 16;
+constexpr int kCsSmem = kOffCsBars + 8 * (kCsStages + 1);
 static_assert(kCsLocal * 8 <= kOffCsLocal, "CTA 0 moves its own pairs down without overlap");
+static_assert(kMaxStaged * 4 <= kOffCsBuf, "the group maxima fit the pair space");
+static_assert((kCsStages - 2) * kCsChunk * 4 <= kOffCsLocal, "buffers 2.. stay below the part's pairs");
+// shared-memory offset of ring buffer st
+__host__ __device__ constexpr int cs_buf(int st) { return st < 2 ? kOffCsBuf + st * kCsChunk * 4 : (st - 2) * kCsChunk * 4; }
 }  // namespace rs
-
-template <int THREADS>
-__global__ void __launch_bounds__(THREADS)
-row_tau_kernel(const uint32_t* __restrict__ gmax16, long long g16_ld, const uint32_t* __restrict__ gmax4,
-               long long g4_ld, const int* __restrict__ pos, const int* __restrict__ k_base, int T, int S,
-               int row0, int k, uint32_t* __restrict__ tau, const PagedRows pg)
-{
-    using namespace sm100;
-    __shared__ SelectSmem<THREADS> sm;
-    __shared__ int abort_s;
-    extern __shared__ __align__(16) uint8_t dyn[];
-    const uint32_t dyn_s = smem_u32(dyn);
-    const uint32_t bar = dyn_s + rs::kMaxStaged * 4;
-    const int tid = threadIdx.x, r = blockIdx.x;
-    if (tid == 0) {
-        mbar_init(bar, 1);
-        abort_s = 0;
-        fence_mbar_init_cluster();
-    }
-    __syncthreads();
-    griddep_wait();
-    long long base;
-    const int* bt;
-    const int n = row_keys(pg, pos, k_base, row0 + r, T, S, &base, &bt);
-    const int tiles = rs::row_tiles(n, k);
-    const int m16 = tiles * rs::kGroupsPerTile, m4 = tiles * 32;
-    const uint32_t* gm = m16 >= k ? gmax16 + (size_t)r * g16_ld : m4 >= k ? gmax4 + (size_t)r * g4_ld : nullptr;
-    const int m = m16 >= k ? m16 : m4 >= k ? m4 : 0;
-    if (!gm) {
-        if (tid == 0) tau[r] = 0u;
-        return;
-    }
-    const uint32_t* src = gm;
-    if (m <= rs::kMaxStaged) {
-        if (tid == 0) {
-            mbar_arrive_expect_tx(bar, (uint32_t)m * 4u);
-            bulk_g2s(dyn_s, gm, (uint32_t)m * 4u, bar);
-        }
-        const bool got = mbar_wait(bar, 0, (volatile int*)&abort_s, 671, r);
-        if (__syncthreads_or(!got)) return;
-        src = reinterpret_cast<const uint32_t*>(dyn);
-    }
-    const uint32_t t = range_floor<THREADS>(src, m, k, sm);
-    if (tid == 0) tau[r] = t;
-}
 
 // Pairs staged in shared memory; entry i is marked as bit i.
 struct PairList {
@@ -870,7 +829,8 @@ struct PairList {
 
 template <int THREADS>
 __global__ void __cluster_dims__(rs::kClusterCtas, 1, 1) __launch_bounds__(THREADS, 2)
-row_select_cluster_kernel(const float* __restrict__ scores, long long ld, const uint32_t* __restrict__ tau,
+row_select_cluster_kernel(const float* __restrict__ scores, long long ld, const uint32_t* __restrict__ gmax16,
+                          long long g16_ld, const uint32_t* __restrict__ gmax4, long long g4_ld,
                           const uint8_t* __restrict__ q_idx, const float* __restrict__ w,
                           const uint8_t* __restrict__ k_idx, int H_I, int d_I, const int* __restrict__ pos,
                           const int* __restrict__ k_base, int T, int S, int row0, int k, int32_t* __restrict__ idx,
@@ -888,8 +848,7 @@ row_select_cluster_kernel(const float* __restrict__ scores, long long ld, const 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int q = (int)cluster_ctarank(), r = blockIdx.x / rs::kClusterCtas, t = row0 + r;
     if (tid == 0) {
-        mbar_init(full(0), 1);
-        mbar_init(full(1), 1);
+        for (int st = 0; st <= rs::kCsStages; ++st) mbar_init(full(st), 1);   // the last: the group maxima
         abort_s = 0;
         fence_mbar_init_cluster();
     }
@@ -920,27 +879,49 @@ row_select_cluster_kernel(const float* __restrict__ scores, long long ld, const 
     const int span = ceil_div(ceil_div(n, rs::kClusterCtas), rs::kCsChunk) * rs::kCsChunk;
     const int a = min(n, q * span), b = min(n, a + span);
     const int nch = ceil_div(b - a, rs::kCsChunk);
+    auto issue = [&](int j) {
+        const int s0 = a + j * rs::kCsChunk, st = j % rs::kCsStages;
+        // the last copy of a row is rounded up to 16 bytes: it stays inside ld
+        const uint32_t bytes = (uint32_t)(min(rs::kCsChunk, b - s0) * 4 + 15) & ~15u;
+        mbar_arrive_expect_tx(full(st), bytes);
+        bulk_g2s(dyn_s + (uint32_t)rs::cs_buf(st), sc + s0, bytes, full(st));
+    };
+    // the row's group maxima (16-key groups where there are k of them)
+    const int tiles = rs::row_tiles(n, k);
+    const int m16 = tiles * rs::kGroupsPerTile, m4 = tiles * 32;
+    const uint32_t* gm = m16 >= k ? gmax16 + (size_t)r * g16_ld : m4 >= k ? gmax4 + (size_t)r * g4_ld : nullptr;
+    const int m = m16 >= k ? m16 : m4 >= k ? m4 : 0;
+    const bool stage = gm && m <= rs::kMaxStaged;
+    // chunks 0 and 1 go to the buffers above the pair space at once; the
+    // maxima are staged in the pair space, and chunks 2.. follow once tau is
+    // taken from them
+    if (tid == 0) {
+        if (stage) {
+            mbar_arrive_expect_tx(full(rs::kCsStages), (uint32_t)m * 4u);
+            bulk_g2s(dyn_s, gm, (uint32_t)m * 4u, full(rs::kCsStages));
+        }
+        for (int j = 0; j < min(nch, 2); ++j) issue(j);
+    }
+    bool bad = false;
+    uint32_t tk = 0u;
+    if (gm) {
+        if (stage) bad = __syncthreads_or(!mbar_wait(full(rs::kCsStages), 0, (volatile int*)&abort_s, 674, 0));
+        if (!bad) tk = range_floor<THREADS>(stage ? reinterpret_cast<const uint32_t*>(dyn) : gm, m, k, sm);
+    }
+    // (range_floor ends with a barrier: the staged maxima are no longer read)
+    if (tid == 0 && !bad)
+        for (int j = 2; j < min(nch, rs::kCsStages); ++j) issue(j);
     // the float whose order key is tau: x >= tf keeps every score whose key
     // is >= tau (and at most a zero of the other sign besides, which ranks
     // below k kept scores and is never selected); tau = 0 keeps all
-    const uint32_t tk = tau[r];
     const float tf = tk ? key_score(tk) : -INFINITY;
-    auto issue = [&](int j) {
-        const int s0 = a + j * rs::kCsChunk;
-        // the last copy of a row is rounded up to 16 bytes: it stays inside ld
-        const uint32_t bytes = (uint32_t)(min(rs::kCsChunk, b - s0) * 4 + 15) & ~15u;
-        mbar_arrive_expect_tx(full(j & 1), bytes);
-        bulk_g2s(dyn_s + rs::kOffCsBuf + (uint32_t)(j & 1) * rs::kCsChunk * 4u, sc + s0, bytes, full(j & 1));
-    };
-    if (tid == 0)
-        for (int j = 0; j < min(nch, 2); ++j) issue(j);
     uint2* local = reinterpret_cast<uint2*>(dyn + rs::kOffCsLocal);
     int running = 0;
-    bool bad = false;
-    for (int j = 0; j < nch; ++j) {
-        const bool got = mbar_wait(full(j & 1), (uint32_t)((j >> 1) & 1), (volatile int*)&abort_s, 673, j);
+    for (int j = 0; j < nch && !bad; ++j) {
+        const int st = j % rs::kCsStages;
+        const bool got = mbar_wait(full(st), (uint32_t)((j / rs::kCsStages) & 1), (volatile int*)&abort_s, 673, j);
         const int s = a + j * rs::kCsChunk + 4 * tid;
-        const float4 v = *reinterpret_cast<const float4*>(dyn + rs::kOffCsBuf + (j & 1) * rs::kCsChunk * 4 + 16 * tid);
+        const float4 v = *reinterpret_cast<const float4*>(dyn + rs::cs_buf(st) + 16 * tid);
         const float e[4] = {v.x, v.y, v.z, v.w};
         uint32_t bits = 0u;
 #pragma unroll
@@ -958,8 +939,8 @@ row_select_cluster_kernel(const float* __restrict__ scores, long long ld, const 
             bad = true;   // a copy timed out: the row takes the global-memory select
             break;
         }
-        // every thread has read buffer j & 1: refill it
-        if (tid == 0 && j + 2 < nch) issue(j + 2);
+        // every thread has read buffer st: refill it
+        if (tid == 0 && j + rs::kCsStages < nch) issue(j + rs::kCsStages);
         const int x = lane < W ? wsum[j & 1][lane] : 0;
         int xi = x;
 #pragma unroll
