@@ -548,10 +548,17 @@ def bench_ours(args, world, rank, local):
 def topk_phases(dsa, bp, bd, stream):
     """The indexer's phases timed on their own (one extra step after the timed
     region, CUDA events around each phase inside the library): the Top-k
-    selection alone, reported as GB/s over its candidate traffic. Candidate
-    bytes per row that needs a selection (n > k): the threshold keeps about
-    2k (score, s) pairs of 8 bytes (all n when n <= 2k), read once, plus the
-    k int32 indices written."""
+    selection alone, reported as GB/s over the bytes it moves, per row that
+    needs a selection (n > k).
+
+    - Prefill (streaming indexer): the threshold keeps about 2k (score, s)
+      pairs of 8 bytes (all n when n <= 2k), read once, plus the k int32
+      indices written.
+    - Decode (up to 2048 rows over long key ranges): the select reads the
+      row's dense score row once (4 bytes per key), each of the row's four
+      CTAs stages the row's group maxima (4 bytes each: one per 16 keys, or
+      per 4 keys where there are fewer than k 16-key groups), and the k int32
+      indices are written."""
     out = {}
     for name, b in (("prefill", bp), ("decode", bd)):
         dsa.phase_timing(True)
@@ -562,10 +569,16 @@ def topk_phases(dsa, bp, bd, stream):
         n = b.x.positions().cpu().long() + 1
         k = b.x.k
         sel = n > k
-        cand_bytes = float((torch.clamp(n[sel], max=2 * k) * 8).sum().item() + int(sel.sum().item()) * k * 4)
+        if name == "prefill":
+            nbytes = float((torch.clamp(n[sel], max=2 * k) * 8).sum().item() + int(sel.sum().item()) * k * 4)
+        else:
+            ns = n[sel]
+            tiles = (ns + 127) // 128
+            m = torch.where(tiles * 8 >= k, tiles * 8, torch.where(tiles * 32 >= k, tiles * 32, 0))
+            nbytes = float((ns * 4 + 4 * m * 4 + k * 4).sum().item())
         out[name] = {"scores_ms": ph["scores"], "threshold_ms": ph["threshold"], "select_ms": ph["select"],
-                     "select_candidate_bytes": cand_bytes,
-                     "select_gbs": cand_bytes / (ph["select"] * 1e-3) / 1e9 if ph["select"] > 0 else None}
+                     "select_bytes": nbytes,
+                     "select_gbs": nbytes / (ph["select"] * 1e-3) / 1e9 if ph["select"] > 0 else None}
     return out
 
 

@@ -827,6 +827,36 @@ struct PairList {
     __device__ __forceinline__ int s(int i) const { return i; }
 };
 
+// The cluster kernel's rare paths, kept out of line so that its hot loop and
+// the common select stay small in the instruction cache.
+template <int THREADS>
+__device__ __noinline__ void recomputed_row_topk(const uint8_t* q_idx, const float* w, const uint8_t* k_idx,
+                                                 int H_I, int d_I, const PagedRows& pg, const int* bt,
+                                                 long long base, int t, int n, int k, int32_t* out, float* buf,
+                                                 SelectSmem<THREADS>& sm)
+{
+    float* wf = buf + H_I * d_I;
+    const uint8_t* qrow = q_idx + (size_t)t * H_I * d_I;
+    for (int e = threadIdx.x; e < H_I * d_I; e += THREADS) buf[e] = e4m3x2_to_float2((uint16_t)qrow[e]).x;
+    for (int j = threadIdx.x; j < H_I; j += THREADS) wf[j] = w[(size_t)t * H_I + j];
+    __syncthreads();
+    block_topk<THREADS>(RecomputedRow{buf, wf, k_idx, pg, bt, base, H_I, d_I}, n, k, out, sm);
+}
+
+template <int THREADS, class Row>
+__device__ __noinline__ void radix_topk_out_of_line(const Row& row, int n, int k, int32_t* out,
+                                                    SelectSmem<THREADS>& sm)
+{
+    block_topk<THREADS>(row, n, k, out, sm);
+}
+
+template <int THREADS>
+__device__ __noinline__ void radix_mark_out_of_line(const PairList& row, int n, int k, uint32_t* bm,
+                                                    SelectSmem<THREADS>& sm)
+{
+    block_select<THREADS>(row, n, k, [&](int, int i) { atomicOr(&bm[i >> 5], 1u << (i & 31)); }, sm);
+}
+
 template <int THREADS>
 __global__ void __cluster_dims__(rs::kClusterCtas, 1, 1) __launch_bounds__(THREADS, 2)
 row_select_cluster_kernel(const float* __restrict__ scores, long long ld, const uint32_t* __restrict__ gmax16,
@@ -840,7 +870,7 @@ row_select_cluster_kernel(const float* __restrict__ scores, long long ld, const 
     constexpr int W = THREADS / 32;
     static_assert(THREADS == rs::kCsThreads && W <= 32, "launch shape");
     __shared__ SelectSmem<THREADS> sm;
-    __shared__ int wsum[2][W];
+    __shared__ int wsum[2][2][W];
     __shared__ int count_s, abort_s;
     extern __shared__ __align__(16) uint8_t dyn[];
     const uint32_t dyn_s = smem_u32(dyn);
@@ -864,14 +894,9 @@ row_select_cluster_kernel(const float* __restrict__ scores, long long ld, const 
         return;
     }
     if (n > rs::kMaxKeys) {
-        if (q != 0) return;
-        float* qf = reinterpret_cast<float*>(dyn);
-        float* wf = qf + H_I * d_I;
-        const uint8_t* qrow = q_idx + (size_t)t * H_I * d_I;
-        for (int e = tid; e < H_I * d_I; e += THREADS) qf[e] = e4m3x2_to_float2((uint16_t)qrow[e]).x;
-        for (int j = tid; j < H_I; j += THREADS) wf[j] = w[(size_t)t * H_I + j];
-        __syncthreads();
-        block_topk<THREADS>(RecomputedRow{qf, wf, k_idx, pg, bt, base, H_I, d_I}, n, k, out, sm);
+        if (q == 0)
+            recomputed_row_topk<THREADS>(q_idx, w, k_idx, H_I, d_I, pg, bt, base, t, n, k, out,
+                                         reinterpret_cast<float*>(dyn), sm);
         return;
     }
     const float* sc = scores + (size_t)r * ld;
@@ -917,45 +942,73 @@ row_select_cluster_kernel(const float* __restrict__ scores, long long ld, const 
     const float tf = tk ? key_score(tk) : -INFINITY;
     uint2* local = reinterpret_cast<uint2*>(dyn + rs::kOffCsLocal);
     int running = 0;
-    for (int j = 0; j < nch && !bad; ++j) {
-        const int st = j % rs::kCsStages;
-        const bool got = mbar_wait(full(st), (uint32_t)((j / rs::kCsStages) & 1), (volatile int*)&abort_s, 673, j);
-        const int s = a + j * rs::kCsChunk + 4 * tid;
-        const float4 v = *reinterpret_cast<const float4*>(dyn + rs::cs_buf(st) + 16 * tid);
-        const float e[4] = {v.x, v.y, v.z, v.w};
-        uint32_t bits = 0u;
+    // two chunks per pass of the CTA (one barrier for both): chunk j's pairs,
+    // then chunk j + 1's
+    for (int j = 0; j < nch && !bad; j += 2) {
+        const bool two = j + 1 < nch;
+        bool got = mbar_wait(full(j % rs::kCsStages), (uint32_t)((j / rs::kCsStages) & 1),
+                             (volatile int*)&abort_s, 673, j);
+        if (two)
+            got = mbar_wait(full((j + 1) % rs::kCsStages), (uint32_t)(((j + 1) / rs::kCsStages) & 1),
+                            (volatile int*)&abort_s, 673, j + 1) && got;
+        float e[2][4];
+        uint32_t bits[2];
+        int cnt[2], incl[2];
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
-            if (s + u < b && e[u] >= tf) bits |= 1u << u;
-        const int cnt = __popc(bits);
-        int incl = cnt;
+        for (int h = 0; h < 2; ++h) {
+            const int s = a + (j + h) * rs::kCsChunk + 4 * tid;
+            const float4 v = *reinterpret_cast<const float4*>(dyn + rs::cs_buf((j + h) % rs::kCsStages) + 16 * tid);
+            e[h][0] = v.x;
+            e[h][1] = v.y;
+            e[h][2] = v.z;
+            e[h][3] = v.w;
+            bits[h] = 0u;
 #pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const int x = __shfl_up_sync(0xffffffffu, incl, off);
-            if (lane >= off) incl += x;
+            for (int u = 0; u < 4; ++u)
+                if ((h == 0 || two) && s + u < b && e[h][u] >= tf) bits[h] |= 1u << u;
+            cnt[h] = __popc(bits[h]);
+            incl[h] = cnt[h];
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int x = __shfl_up_sync(0xffffffffu, incl[h], off);
+                if (lane >= off) incl[h] += x;
+            }
         }
-        if (lane == 31) wsum[j & 1][warp] = incl;
+        const int par = (j >> 1) & 1;
+        if (lane == 31) {
+            wsum[par][0][warp] = incl[0];
+            wsum[par][1][warp] = incl[1];
+        }
         if (__syncthreads_or(!got)) {
             bad = true;   // a copy timed out: the row takes the global-memory select
             break;
         }
-        // every thread has read buffer st: refill it
-        if (tid == 0 && j + rs::kCsStages < nch) issue(j + rs::kCsStages);
-        const int x = lane < W ? wsum[j & 1][lane] : 0;
-        int xi = x;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, xi, off);
-            if (lane >= off) xi += y;
+        // every thread has read both buffers: refill them
+        if (tid == 0) {
+            if (j + rs::kCsStages < nch) issue(j + rs::kCsStages);
+            if (j + 1 + rs::kCsStages < nch) issue(j + 1 + rs::kCsStages);
         }
-        int at = running + __shfl_sync(0xffffffffu, xi - x, warp) + incl - cnt;
+        int base_h = running;
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
-            if (bits >> u & 1u) {
-                if (at < rs::kCsLocal) local[at] = make_uint2(score_key(e[u]), (uint32_t)(s + u));
-                ++at;
+        for (int h = 0; h < 2; ++h) {
+            const int x = lane < W ? wsum[par][h][lane] : 0;
+            int xi = x;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, xi, off);
+                if (lane >= off) xi += y;
             }
-        running += __shfl_sync(0xffffffffu, xi, W - 1);
+            int at = base_h + __shfl_sync(0xffffffffu, xi - x, warp) + incl[h] - cnt[h];
+            const int s = a + (j + h) * rs::kCsChunk + 4 * tid;
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (bits[h] >> u & 1u) {
+                    if (at < rs::kCsLocal) local[at] = make_uint2(score_key(e[h][u]), (uint32_t)(s + u));
+                    ++at;
+                }
+            base_h += __shfl_sync(0xffffffffu, xi, W - 1);
+        }
+        running = base_h;
     }
     if (tid == 0) count_s = bad ? rs::kCsLocal + 1 : running;
     __syncthreads();   // every thread's pairs of the last chunk are written
@@ -980,8 +1033,7 @@ row_select_cluster_kernel(const float* __restrict__ scores, long long ld, const 
     int* warp_sums = reinterpret_cast<int*>(sm.hist[0]);
     if (over) {
         // (the same decision in every CTA: no further cluster barrier)
-        if (q != 0) return;
-        block_topk<THREADS>(DenseScores{sc}, n, k, out, sm);
+        if (q == 0) radix_topk_out_of_line<THREADS>(DenseScores{sc}, n, k, out, sm);
         return;
     }
     if (q != 0) {
@@ -994,8 +1046,7 @@ row_select_cluster_kernel(const float* __restrict__ scores, long long ld, const 
     for (int i = tid; i < (total + 31) / 32; i += THREADS) lbm[i] = 0u;
     __syncthreads();
     const PairList row{list};
-    if (!range_select_bitmap<THREADS>(row, total, k, lbm, sm))
-        block_select<THREADS>(row, total, k, [&](int, int i) { atomicOr(&lbm[i >> 5], 1u << (i & 31)); }, sm);
+    if (!range_select_bitmap<THREADS>(row, total, k, lbm, sm)) radix_mark_out_of_line<THREADS>(row, total, k, lbm, sm);
     __syncthreads();
     block_emit_bitmap<THREADS>(lbm, total, out, warp_sums, [&](int i) { return (int)list[i].y; });
 }
