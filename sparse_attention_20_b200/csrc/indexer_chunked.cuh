@@ -1028,7 +1028,10 @@ row_select_cluster_kernel(const float* __restrict__ scores, long long ld, const 
         if (p < q) before += c;
         total += c;
     }
-    over |= total > rs::kCsList;
+    // (total >= k always holds: tau is at most the k-th largest score; a row
+    // short of k pairs would still take the exact global select, so the
+    // selects below never see fewer than k entries)
+    over |= total > rs::kCsList || total < k;
     cluster_sync();   // 2: every CTA has read the counts (none exits before that)
     int* warp_sums = reinterpret_cast<int*>(sm.hist[0]);
     if (over) {

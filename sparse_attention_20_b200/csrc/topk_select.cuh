@@ -246,7 +246,8 @@ constexpr int kRangeListCap = 128;   // uint2 entries in SelectSmem::total
 // With the kRangeBins-bin histogram in sm.hist complete and visible: the bin
 // holding the k-th entry from the top goes to sm.misc[0], k minus the entries
 // of the bins above it to misc[1], the bin's count to misc[2] (visible to
-// every thread on return; k must not exceed the histogram's total).
+// every thread on return). If the histogram holds fewer than k entries,
+// misc[2] is INT_MAX.
 template <int THREADS>
 __device__ void range_kth_bin(int k, SelectSmem<THREADS>& sm)
 {
@@ -269,7 +270,14 @@ __device__ void range_kth_bin(int k, SelectSmem<THREADS>& sm)
         if (lane >= off) incl += v;
     }
     if (lane == 31) wsum[warp] = incl;
-    if (tid == 0) sm.counter[0] = 0;
+    if (tid == 0) {
+        sm.counter[0] = 0;
+        // what a histogram of fewer than k entries leaves: no bin, and a
+        // boundary "count" above any list capacity (range_select_core declines)
+        sm.misc[0] = 0;
+        sm.misc[1] = k;
+        sm.misc[2] = 0x7FFFFFFF;
+    }
     __syncthreads();
     uint32_t before = incl - local;
     for (int w = 0; w < warp; ++w) before += wsum[w];
