@@ -67,7 +67,7 @@ def parse():
     ap.add_argument("--replicas", action="store_true",
                     help="with several ranks, run the whole workload on every rank (weak scaling) "
                          "instead of splitting its query rows and sequences between them")
-    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--seed", type=int, default=0)
@@ -584,7 +584,8 @@ def topk_phases(dsa, bp, bd, stream):
 
 def bench_e2e(args, world, dsa, bp, bd, stream, tokens):
     """Same step through the C ABI with inputs in pinned host memory: every step
-    copies its inputs host->device and reads idx/out/lse back."""
+    copies its inputs host->device and reads idx/out/lse back (consecutive
+    steps' copies overlap in the two directions)."""
     def host(t):
         try:
             h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
@@ -604,28 +605,55 @@ def bench_e2e(args, world, dsa, bp, bd, stream, tokens):
     h2d = sum(h.numel() * h.element_size() for h, _ in pairs_in)
     d2h = sum(h.numel() * h.element_size() for h, _ in pairs_out)
 
+    # Three streams: uploads, compute (the library's launches) and downloads.
+    # A step's compute waits for its own upload and for the previous step's
+    # download (the output buffers); its upload waits for the previous step's
+    # compute (the input buffers). So step i+1's inputs upload while step i's
+    # results download (PCIe runs both directions at once), and every step
+    # still moves all of its inputs in and all of its results out.
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    state = {"computed": None, "downloaded": None}
+
     def step():
-        for h, d in pairs_in:
-            d.copy_(h, non_blocking=True)
+        with torch.cuda.stream(s_in):
+            if state["computed"] is not None:
+                s_in.wait_event(state["computed"])
+            for h, d in pairs_in:
+                d.copy_(h, non_blocking=True)
+            uploaded = torch.cuda.Event()
+            uploaded.record(s_in)
+        stream.wait_event(uploaded)
+        if state["downloaded"] is not None:
+            stream.wait_event(state["downloaded"])
         for b in (bp, bd):
             run_indexer(dsa, b, stream)
             run_attn(dsa, b, stream)
-        for h, d in pairs_out:
-            h.copy_(d, non_blocking=True)
+        computed = torch.cuda.Event()
+        computed.record(stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(computed)
+            for h, d in pairs_out:
+                h.copy_(d, non_blocking=True)
+            downloaded = torch.cuda.Event()
+            downloaded.record(s_out)
+        state["computed"], state["downloaded"] = computed, downloaded
 
     step()
     torch.cuda.synchronize()
+    state["computed"] = state["downloaded"] = None
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
-    start.record(stream)
+    start.record(s_in)
     for _ in range(args.e2e_steps):
         step()
-    end.record(stream)
+    s_out.wait_event(state["computed"])
+    end.record(s_out)
     torch.cuda.synchronize()
     ms = max_over_ranks(world, start.elapsed_time(end)) / args.e2e_steps
     return {"value": tokens / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "copies": "step i+1's upload overlaps step i's download; compute waits for both",
             "pinned": all(h.is_pinned() for h, _ in pairs_in + pairs_out)}
 
 
