@@ -287,10 +287,11 @@ __device__ __forceinline__ int sampled_valid(int n)
     return m;
 }
 
-// tau_t: the r-th largest sampled score with r = ceil(alpha * k * m / n); rows
-// that can keep every candidate get -inf. The row's samples are staged in
-// shared memory (dynamic, samp_ld floats) so the radix passes read them once
-// from global memory.
+// tau_t: the r-th largest sampled score with r = ceil(alpha * k * m / n),
+// rounded down to its order key's top 16 bits (two radix passes; the
+// threshold only steers how many candidates the filter keeps, which it
+// raises by about a hundredth); rows that can keep every candidate get -inf.
+// The row's samples are staged in shared memory (dynamic, samp_ld floats).
 template <int THREADS>
 __global__ void __launch_bounds__(THREADS)
 indexer_tau_kernel(const float* __restrict__ samp, int samp_ld, int T, int S, int k, int row0,
@@ -312,7 +313,7 @@ indexer_tau_kernel(const float* __restrict__ samp, int samp_ld, int T, int S, in
             __syncthreads();
             int take_eq, count_eq;
             const uint32_t kth = radix_kth_key<THREADS>(SmemScores{samp_s, 0}, stored, (int)r, sm, &take_eq,
-                                                        &count_eq);
+                                                        &count_eq, 2);
             out = key_score(kth);
         }
     }

@@ -118,15 +118,18 @@ __device__ __forceinline__ void clear_hist(SelectSmem<THREADS>& sm)
 
 // Returns the key of the k-th largest entry; *take_eq = entries equal to it
 // that belong to the Top-k, *count_eq = entries equal to it. Requires n > k.
+// With digits < 4 only the top 8 * digits bits are resolved: the result is
+// the k-th largest key with its lower bits cleared, a lower bound of it (and
+// *take_eq, *count_eq refer to that bucket).
 template <int THREADS, class G = CtaGroup, class Row>
 __device__ uint32_t radix_kth_key(const Row& row, int n, int k, SelectSmem<THREADS>& sm,
-                                  int* take_eq, int* count_eq)
+                                  int* take_eq, int* count_eq, int digits = 4)
 {
     const int warp = G::tid() >> 5;
     uint32_t prefix = 0u, mask = 0u;
     int need = k, cnt = 0;
 #pragma unroll 1
-    for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int shift = 24; shift >= 32 - 8 * digits; shift -= 8) {
         clear_hist<THREADS, G>(sm);
         for (int i = G::tid(); i < n; i += THREADS) {
             const uint32_t key = row.key(i);
