@@ -62,6 +62,9 @@ def test_workspace_sizes(lib):
     # decode-like: 64 rows over a 4.5M-key packed cache stay within one block
     dec = dsa.workspace_size(64, 4_500_000, 8, 128, 2048, 128, 576, 512)
     assert 0 < dec <= 1 << 30
+    # the decode form of 64 rows over 128K keys: each row's dense score row
+    # (131072 x 4 B) and its 16-key and 4-key group maxima ((8192 + 32768) x 4 B)
+    assert dsa.workspace_size(64, 131072, 8, 128, 2048, 128, 576, 512) == 64 * (131072 + 8192 + 32768) * 4
 
 
 FAKE = ctypes.c_void_p(0x10000)          # aligned, never dereferenced: checks fail first
