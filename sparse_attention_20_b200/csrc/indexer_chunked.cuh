@@ -463,10 +463,11 @@ chunk_topk_tma_kernel(const __grid_constant__ CUtensorMap tm_k, const uint8_t* _
 // (scores[r * ld + s]) together with the largest order key of each group of
 // 16 scores (gmax16[r * g16_ld + 8 * tile + warp]: one group per scoring warp
 // and tile) and of each group of 4 (gmax4[r * g4_ld + 32 * tile + 4 * warp +
-// q]). The row's Top-k is selected afterwards from these (row_filter_kernel,
-// row_merge_kernel). Rows with at most k keys, or more than kMaxKeys, get no
-// tiles here (the merge writes the former directly and recomputes the
-// latter's scores).
+// q]: keys gid, gid + 1, gid + 8, gid + 9 of the warp's 16, q = gid / 2).
+// The row's Top-k is selected afterwards from these
+// (row_select_cluster_kernel). Rows with at most k keys, or more than
+// kMaxKeys, get no tiles here (the select writes the former directly and
+// recomputes the latter's scores).
 namespace rs {
 constexpr int kTileKeys = 128;
 constexpr int kTileBytes = kTileKeys * 128;
