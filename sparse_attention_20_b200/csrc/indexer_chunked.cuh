@@ -789,10 +789,10 @@ merge_topk_kernel(const uint2* __restrict__ cand, long long cand_ld, const int* 
 // part of the score row through a ring of kCsStages shared-memory buffers
 // (1-D bulk copies; four of them in the lower half of the pair space, which is
 // free until the pairs are gathered) and keeps its scores >= tau as
-// (order key, s) pairs in ascending s (a scan over the CTA per chunk). The
-// parts' counts are
-// exchanged over distributed shared memory, each part's pairs are stored into
-// CTA 0 after the pairs of the parts before it, so CTA 0 holds every score
+// (order key, s) pairs in ascending s (a scan over the CTA per two stages).
+// The parts' counts are exchanged over distributed shared memory, each part's
+// pairs are stored into CTA 0 after the pairs of the parts before it, so
+// CTA 0 holds every score
 // >= tau in ascending s, and CTA 0 takes their exact Top-k (range-histogram
 // select, or the radix select where the keys' spread defeats it), marked in a
 // bitmap over the pairs and written in ascending s. Parts that keep more than
